@@ -1,0 +1,107 @@
+"""fp64 CPU oracle for the EFLA forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library and its Python binding
+never import it, and it imports nothing from them.
+
+The arithmetic lives in ``efla_oracle.c`` (plain C, fp64, one token at a time,
+libm ``expm1``, built with ``-O2`` and no fast-math).  This module only
+compiles it with gcc and marshals numpy arrays through ctypes.
+
+Source of the recurrence: "Exact Flow Linear Attention: Exact Solution from
+Continuous-Time Dynamics", technical summary, Methodology 2 (lambda = ||k||^2)
+and Methodology 3 (alpha and the update rule); readout o_t = S_t^T q_t.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "efla_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile efla_oracle.c into liboracle.so with gcc (no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-fPIC", "-shared",
+             "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.efla_oracle_alpha.restype = ctypes.c_double
+        lib.efla_oracle_alpha.argtypes = [ctypes.c_double, ctypes.c_double]
+        lib.efla_oracle_step.restype = ctypes.c_double
+        lib.efla_oracle_step.argtypes = [ctypes.c_int, ctypes.c_int, dp, dp, dp, dp,
+                                         ctypes.c_double, dp]
+        lib.efla_oracle_fwd.restype = ctypes.c_int
+        lib.efla_oracle_fwd.argtypes = [ctypes.c_int] * 5 + [dp] * 7 + [ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    """Contiguous fp64 numpy copy of a numpy array or a (CPU) torch tensor."""
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu")
+        import torch  # local: only when given torch tensors
+
+        a = a.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def alpha(lam: float, beta: float) -> float:
+    """alpha = (1 - exp(-beta*lam))/lam, evaluated as -expm1(-beta*lam)/lam; beta at lam == 0."""
+    return float(_load().efla_oracle_alpha(float(lam), float(beta)))
+
+
+def step(S, q, k, v, beta: float):
+    """One recurrent token on one head.  Returns (S_t, o_t, alpha_t); S is not modified."""
+    S = _f64(S).copy()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    dk, dv = S.shape
+    o = np.zeros(dv)
+    a = _load().efla_oracle_step(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta), _ptr(o))
+    return S, o, float(a)
+
+
+def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True):
+    """Token-by-token forward over [B,H,L,d] inputs.  Returns (o, S_final) in fp64.
+
+    q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L]; S0: [B,H,dk,dv] or None (zeros).
+    """
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, H, L, dk) and v.shape == (B, H, L, dv) and beta.shape == (B, H, L)
+    s0 = None
+    if S0 is not None:
+        s0 = _f64(S0)
+        assert s0.shape == (B, H, dk, dv)
+    o = np.zeros((B, H, L, dv)) if want_o else None
+    S = np.zeros((B, H, dk, dv))
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().efla_oracle_fwd(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                 _ptr(s0) if s0 is not None else None,
+                                 _ptr(o) if o is not None else None, _ptr(S), int(nthreads))
+    if rc != 0:
+        raise MemoryError("oracle forward failed to allocate")
+    return o, S
