@@ -1,0 +1,386 @@
+"""Benchmark of the EFLA forward hot path on B200.
+
+One step = one pass of the whole hot path over one batch of the 1.3B-LM-shaped
+workload: the chunkwise forward (B=4, H=16, L=4096, dk=dv=128, chunk=64, bf16)
+followed by the recurrent decode step of its decode batch (B=64, H=16, one
+token each, fp32 carried state).  Throughput is token-heads per second
+(B*H*L + B_dec*H_dec per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 3|4|5] [--no-e2e] [--no-cpu-baseline]
+
+Under torchrun (WORLD_SIZE > 1) every rank runs its own replica of the workload
+on disjoint heads (seeded per rank): heads are independent, so there is no
+collective on the data path ("weak" scaling); the only collectives are the
+barriers around the timed region and the max-reduction of its time.
+
+Prints ONE JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from delta_rule_linear_efla_b200 import inputs  # noqa: E402
+
+METRIC = "EFLA fwd tokens/s per GPU (B*H*L/time) and % of binding roofline"
+UNIT = "token-heads/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def alg_bytes_chunk(w) -> int:
+    """Algorithmic HBM bytes of one chunk forward: read q, k, v, beta; write o (all in the
+    input dtype) per token-head, plus the fp32 final state per head (S0 is zero here and
+    not read)."""
+    es = 2 if w.dtype == "bf16" else 4
+    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * es
+    return w.token_heads * per_tok + w.B * w.H * w.dk * w.dv * 4
+
+
+def alg_bytes_decode(Bd, Hd, dk, dv, es=2) -> int:
+    """Read + write of the fp32 state per head, plus q, k, v, beta in and o out."""
+    return Bd * Hd * (2 * dk * dv * 4 + (2 * dk + 2 * dv + 1) * es)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
+    """The fp64 oracle (as it stands) on a bounded sample of the workload: a subset of its
+    heads at full sequence length, on all host cores."""
+    import oracle
+
+    oracle.build()
+    cores = os.cpu_count() or 1
+    x = inputs.make_inputs(inputs.workload(w.id, B=1, H=1))
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], nthreads=1)
+    t_head = max(time.perf_counter() - t0, 1e-3)
+    # about `seconds_target` of wall time with every core busy on whole heads
+    heads = max(1, min(w.B * w.H, cores * max(1, int(seconds_target / t_head))))
+    H = min(heads, w.H)
+    B = max(1, min(w.B, heads // H))
+    xs = inputs.make_inputs(inputs.workload(w.id, B=B, H=H))
+    threads = min(cores, B * H)
+    t0 = time.perf_counter()
+    oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    n = B * H * w.L
+    return {"value": n / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d heads (B=%d, H=%d) at full L=%d, fp64 token-by-token, %.1f s"
+                      % (B * H, w.B * w.H, B, H, w.L, dt)}
+
+
+def run_reference(args) -> None:
+    """The oracle timed on host cores: each step is a bounded sample of the workload."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    w = inputs.WORKLOADS[args.workload]
+    cores = os.cpu_count() or 1
+    H = min(w.H, cores)
+    xs = inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 1024)))
+    threads = min(cores, H)
+    for _ in range(args.warmup):
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    n = H * xs["q"].shape[2] * args.steps
+    val = n / dt
+    sample = "%d heads x L=%d of workload %s per step, fp64 token-by-token" % (
+        H, xs["q"].shape[2], w.name)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def _config(w) -> dict:
+    c = {"workload": "%s (B=%d H=%d L=%d dk=%d dv=%d chunk=%d %s)" % (
+        w.name, w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.dtype),
+        "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+        "l2": "inputs > L2 (126 MB): two rotating input sets per rank"}
+    if w.decode:
+        c["decode"] = "B=%d H=%d one token, fp32 carried state" % (w.decode["B"], w.decode["H"])
+    return c
+
+
+def run_ours(args) -> None:
+    from delta_rule_linear_efla_b200 import efla
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = inputs.WORKLOADS[args.workload]
+    peaks = _peaks()
+
+    # ---- inputs: two rotating sets so consecutive steps do not hit in L2 ----
+    sets = []
+    for r in range(2):
+        x = inputs.make_inputs(w, seed=1000 + w.id + 7919 * (2 * rank + r))
+        sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
+    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype(), device=dev) for _ in range(2)]
+    Sf_buf = [torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
+    ws_bytes = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype())
+    wsp = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    path = efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype())
+
+    dec = None
+    if w.decode:
+        d = inputs.make_decode_inputs(w, seed=w.decode["seed"] + 7919 * rank)
+        dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()
+              if k != "prefix"}
+        p = d["prefix"]
+        pd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in p.items()}
+        _, S_carry = efla.chunk_fwd(pd["q"], pd["k"], pd["v"], pd["beta"], None, chunk=w.chunk)
+        dd["S_init"] = S_carry
+        dd["S"] = [S_carry.clone(), S_carry.clone()]
+        dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=w.torch_dtype(), device=dev)
+        dec = dd
+    tok_dec = (w.decode["B"] * w.decode["H"]) if w.decode else 0
+    tok_step = w.token_heads + tok_dec
+
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev_pair=None):
+        x = sets[i % 2]
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        efla.chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], chunk=w.chunk,
+                       o=o_buf[i % 2], S_final=Sf_buf[i % 2], workspace=wsp)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+        if dec is not None:
+            efla.recurrent_step(dec["q"], dec["k"], dec["v"], dec["beta"], dec["S"][i % 2],
+                                o=dec["o"])
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(dev.index if dev.index is not None else 0)
+    clk.start()
+    l0 = efla.kernel_launches()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = efla.kernel_launches() - l0
+    clocks = clk.stop()
+    if ws > 1:
+        torch.distributed.barrier()
+    ms_local = t_start.elapsed_time(t_end)
+    ms = _max_over_ranks(ms_local, ws, dev)
+    chunk_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    chunk_ms = _max_over_ranks(chunk_ms, ws, dev)
+    err = efla.last_device_error()
+    if err != 0:
+        raise RuntimeError("device error word set: %s" % efla.status_str(err))
+
+    value = tok_step * args.steps * ws / (ms / 1e3)
+    alg = alg_bytes_chunk(w)
+    achieved = alg / (chunk_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm"], "traffic": None,
+                "kernel": "efla_chunk_fwd (%s path)" % path,
+                "alg_bytes_per_launch": alg, "avg_launch_ms": chunk_ms,
+                "peak_source": peaks["src"] + " (MEASURED_PEAKS.json hbm_gbs)"}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        xh = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v)
+              for k, v in inputs.make_inputs(w, seed=4242 + rank).items()}
+        o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype()).pin_memory()
+        S_host = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
+        h2d = sum(xh[k].numel() * xh[k].element_size() for k in ("q", "k", "v", "beta"))
+        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+        if dec is not None:
+            dh = {k: dec[k].cpu().pin_memory() for k in ("q", "k", "v", "beta")}
+            S_dec_host = dec["S_init"].cpu().pin_memory()
+            od_host = torch.empty_like(dec["o"], device="cpu").pin_memory()
+            h2d += sum(t.numel() * t.element_size() for t in dh.values()) + S_dec_host.numel() * 4
+            d2h += od_host.numel() * od_host.element_size() + S_dec_host.numel() * 4
+
+        def e2e_step():
+            g = {k: xh[k].to(dev, non_blocking=True) for k in ("q", "k", "v", "beta")}
+            o, S = efla.chunk_fwd(g["q"], g["k"], g["v"], g["beta"], None, chunk=w.chunk,
+                                  o=o_buf[0], S_final=Sf_buf[0], workspace=wsp)
+            o_host.copy_(o, non_blocking=True)
+            S_host.copy_(S, non_blocking=True)
+            if dec is not None:
+                gd = {k: dh[k].to(dev, non_blocking=True) for k in dh}
+                Sd = S_dec_host.to(dev, non_blocking=True)
+                od = efla.recurrent_step(gd["q"], gd["k"], gd["v"], gd["beta"], Sd, o=dec["o"])
+                od_host.copy_(od, non_blocking=True)
+                S_dec_host.copy_(Sd, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if ws > 1:
+            torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = _max_over_ranks(a.elapsed_time(b), ws, dev)
+        e2e = {"value": tok_step * n_e2e * ws / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic", "config": _config(w), "roofline": roofline, "cpu_baseline": cpu,
+        "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
+        "path": path, "token_heads_per_step": tok_step,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,130 @@
+// api.cu -- extern "C" entry points declared in include/efla.h.
+//
+// Each entry point validates its arguments on the host, selects kernels and
+// enqueues them on the caller's stream.  No device memory is allocated here.
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/efla.h"
+#include "launchers.h"
+
+namespace efla {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace efla
+
+namespace {
+
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+efla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA; }
+
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char *efla_status_str(int status) {
+    switch (status) {
+        case EFLA_OK: return "ok";
+        case EFLA_ERR_NULL: return "null pointer";
+        case EFLA_ERR_SHAPE: return "invalid size";
+        case EFLA_ERR_DTYPE: return "invalid dtype";
+        case EFLA_ERR_UNSUPPORTED: return "unsupported size or chunk";
+        case EFLA_ERR_CUDA: return "CUDA error";
+        case EFLA_ERR_TIMEOUT: return "device wait timed out";
+        case EFLA_ERR_WORKSPACE: return "workspace missing or too small";
+        case EFLA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int efla_version(void) { return 100; /* 0.1.0 */ }
+
+efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int H, int L, int dk,
+                       efla_dtype dt, void *stream) {
+    if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
+    if (B < 0 || H < 0 || L < 0 || dk < 1) return EFLA_ERR_SHAPE;
+    if (dk > 256) return EFLA_ERR_UNSUPPORTED;
+    const long long ntok = (long long)B * H * L;
+    if (ntok == 0) return EFLA_OK;
+    if (!k || !beta || !alpha) return EFLA_ERR_NULL;
+    if (!aligned16(k) || !aligned16(beta) || !aligned16(alpha)) return EFLA_ERR_ALIGN;
+    return from_cuda(efla::launch_alpha(k, beta, alpha, ntok, dk, dt == EFLA_BF16,
+                                        (cudaStream_t)stream));
+}
+
+int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt) {
+    return efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16) ? 1 : 0;
+}
+
+size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int chunk,
+                                     efla_dtype dt) {
+    if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1 || !chunk_ok(chunk)) return 0;
+    if (dt != EFLA_F32 && dt != EFLA_BF16) return 0;
+    if (efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16))
+        return efla::tc_workspace_bytes(B, H, L, dk, dv, chunk);
+    return 0;
+}
+
+efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
+                           const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
+                           int dv, int chunk, efla_dtype dt, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
+    if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
+    if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
+    if (dk > 128 || dv > 128 || !chunk_ok(chunk)) return EFLA_ERR_UNSUPPORTED;
+    if (L > 0 && (!q || !k || !v || !beta || !o)) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S0) ||
+        !aligned16(o) || !aligned16(S_final))
+        return EFLA_ERR_ALIGN;
+    const bool bf16 = dt == EFLA_BF16;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (L == 0) {
+        if (!S_final) return EFLA_OK;
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        if (S0 == S_final) return EFLA_OK;
+        return from_cuda(S0 ? cudaMemcpyAsync(S_final, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(S_final, 0, bytes, s));
+    }
+    if (efla::tc_supported(B, H, L, dk, dv, chunk, bf16)) {
+        const size_t need = efla::tc_workspace_bytes(B, H, L, dk, dv, chunk);
+        if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return EFLA_ERR_ALIGN;
+        return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
+                                               chunk, workspace, s));
+    }
+    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
+                                             chunk, bf16, s));
+}
+
+efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
+                                float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
+                                void *stream) {
+    if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
+    if ((long long)B * H > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (dk > 256 || dv > 256) return EFLA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S) ||
+        !aligned16(o))
+        return EFLA_ERR_ALIGN;
+    return from_cuda(efla::launch_decode(q, k, v, beta, S, o, B * H, dk, dv, dt == EFLA_BF16,
+                                         (cudaStream_t)stream));
+}
+
+unsigned long long efla_kernel_launches(void) {
+    return efla::g_launches.load(std::memory_order_relaxed);
+}
+
+efla_status efla_last_device_error(void *stream) {
+    unsigned int word = 0;
+    if (efla::tc_read_and_clear_error(&word, (cudaStream_t)stream) != cudaSuccess)
+        return EFLA_ERR_CUDA;
+    return word ? EFLA_ERR_TIMEOUT : EFLA_OK;
+}
+
+}  // extern "C"

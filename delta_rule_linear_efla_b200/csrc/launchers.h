@@ -1,0 +1,39 @@
+// launchers.h -- host-side launch functions of the EFLA kernels (internal to
+// the library; the public ABI is include/efla.h).  Each returns a
+// cudaError_t from cudaGetLastError() after its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace efla {
+
+// Host-side count of kernels enqueued by the library (efla_kernel_launches).
+void count_launches(unsigned n);
+
+// Per-token alpha (fused norm + closed-form coefficient).  is_bf16 selects the
+// element type of k and beta.
+cudaError_t launch_alpha(const void *k, const void *beta, float *alpha, long long ntok, int dk,
+                         bool is_bf16, cudaStream_t s);
+
+// SIMT fp32 chunkwise forward: WY/UT per chunk, state carried in fp32.
+// Any dk, dv <= 128 and chunk <= 64.
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
+                              const float *S0, void *o, float *S_final, int B, int H, int L,
+                              int dk, int dv, int chunk, bool is_bf16, cudaStream_t s);
+
+// Recurrent single-token step per head (decode), S updated in place.
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
+                          float *S, void *o, int BH, int dk, int dv, bool is_bf16,
+                          cudaStream_t s);
+
+// Tensor-core (tcgen05) chunkwise forward, bf16 only.
+bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
+size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
+                            const float *S0, void *o, float *S_final, int B, int H, int L,
+                            int dk, int dv, int chunk, void *ws, cudaStream_t s);
+// Device error word of the tensor-core kernels (bounded waits): read and clear.
+cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s);
+
+}  // namespace efla

@@ -1,0 +1,186 @@
+"""Python binding of the C-ABI library libefla.so (include/efla.h).
+
+Argument marshalling only: this module checks tensor dtypes, shapes and
+devices, allocates outputs and workspace with torch, and passes raw device
+pointers plus the current CUDA stream to the library.  Every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback: if
+the library is missing or no CUDA device is present, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libefla.so")
+
+EFLA_F32, EFLA_BF16 = 0, 1
+
+# Every extern "C" symbol declared in include/efla.h.
+ABI_SYMBOLS = (
+    "efla_status_str", "efla_version", "efla_alpha", "efla_chunk_fwd_workspace_size",
+    "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
+    "efla_kernel_launches",
+)
+
+_lib = None
+
+
+class EflaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (where, status_str(status), status))
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libefla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError("libefla.so is not built (%s); run `python -m "
+                           "delta_rule_linear_efla_b200.build` on a machine with nvcc" % p)
+    L = ctypes.CDLL(p)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.efla_status_str.restype = ctypes.c_char_p
+    L.efla_status_str.argtypes = [i]
+    L.efla_version.restype = i
+    L.efla_version.argtypes = []
+    L.efla_alpha.restype = i
+    L.efla_alpha.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    L.efla_chunk_fwd_workspace_size.restype = sz
+    L.efla_chunk_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.efla_chunk_fwd.restype = i
+    L.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    L.efla_recurrent_step.restype = i
+    L.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.efla_last_device_error.restype = i
+    L.efla_last_device_error.argtypes = [vp]
+    L.efla_chunk_fwd_path.restype = i
+    L.efla_chunk_fwd_path.argtypes = [i, i, i, i, i, i, i]
+    L.efla_kernel_launches.restype = ctypes.c_ulonglong
+    L.efla_kernel_launches.argtypes = []
+    if path is None:
+        _lib = L
+    return L
+
+
+def status_str(status: int) -> str:
+    return load_library().efla_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise EflaError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return EFLA_F32
+    if t.dtype == torch.bfloat16:
+        return EFLA_BF16
+    raise TypeError("EFLA tensors must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    return t.data_ptr()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def alpha(k: torch.Tensor, beta: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """alpha_t = -expm1(-beta_t ||k_t||^2)/||k_t||^2 (beta_t at ||k_t|| = 0); [B,H,L] fp32."""
+    B, H, L, dk = k.shape
+    if beta.shape != (B, H, L) or beta.dtype != k.dtype:
+        raise ValueError("beta must be [B,H,L] with k's dtype")
+    if out is None:
+        out = torch.empty((B, H, L), dtype=torch.float32, device=k.device)
+    _check(load_library().efla_alpha(_dev(k, "k"), _dev(beta, "beta"),
+                                      _dev(out, "alpha", torch.float32), B, H, L, dk,
+                                      _dtype_code(k), _stream_handle(stream)), "efla_alpha")
+    return out
+
+
+def workspace_size(B: int, H: int, L: int, dk: int, dv: int, chunk: int, dtype) -> int:
+    code = EFLA_BF16 if dtype == torch.bfloat16 else EFLA_F32
+    return int(load_library().efla_chunk_fwd_workspace_size(B, H, L, dk, dv, chunk, code))
+
+
+def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype) -> str:
+    code = EFLA_BF16 if dtype == torch.bfloat16 else EFLA_F32
+    return "tcgen05" if load_library().efla_chunk_fwd_path(B, H, L, dk, dv, chunk, code) else "simt"
+
+
+def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
+              want_state: bool = True, workspace=None, stream=None):
+    """EFLA forward in the WY/UT chunkwise form.  Returns (o, S_final or None).
+
+    q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L], all float32 or all bfloat16 on one
+    CUDA device; S0: [B,H,dk,dv] float32 or None.  o has the inputs' dtype; S_final is
+    float32.  S_final may be S0 (in-place carry)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L):
+        raise ValueError("shape mismatch: q,k [B,H,L,dk], v [B,H,L,dv], beta [B,H,L]")
+    code = _dtype_code(q)
+    for name, t in (("k", k), ("v", v), ("beta", beta)):
+        if t.dtype != q.dtype:
+            raise TypeError("%s must have q's dtype %s" % (name, q.dtype))
+    if o is None:
+        o = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = workspace_size(B, H, L, dk, dv, chunk, q.dtype)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
+    st = load_library().efla_chunk_fwd(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
+        _dev(S0, "S0", torch.float32) if S0 is not None else None,
+        _dev(o, "o", q.dtype),
+        _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
+        B, H, L, dk, dv, int(chunk), code, ws_ptr, ws_bytes, _stream_handle(stream))
+    _check(st, "efla_chunk_fwd")
+    return o, S_final
+
+
+def recurrent_step(q, k, v, beta, S, o=None, stream=None):
+    """One decode token per head; S ([B,H,dk,dv] float32) is updated in place.  Returns o."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:2] != (B, H) or beta.shape != (B, H) or \
+            S.shape != (B, H, dk, dv):
+        raise ValueError("shape mismatch: q,k [B,H,dk], v [B,H,dv], beta [B,H], S [B,H,dk,dv]")
+    code = _dtype_code(q)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = load_library().efla_recurrent_step(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
+        _dev(S, "S", torch.float32), _dev(o, "o", q.dtype), B, H, dk, dv, code,
+        _stream_handle(stream))
+    _check(st, "efla_recurrent_step")
+    return o
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded (host-side counter)."""
+    return int(load_library().efla_kernel_launches())
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise and return (and clear) the device error word's status code."""
+    return int(load_library().efla_last_device_error(_stream_handle(stream)))

@@ -1,0 +1,157 @@
+/*
+ * efla.h -- C ABI of the B200 (sm_100a) Exact Flow Linear Attention forward.
+ *
+ * Method: "Exact Flow Linear Attention: Exact Solution from Continuous-Time
+ * Dynamics" (technical summary).  Per head, for t = 1..L:
+ *
+ *   lambda_t = ||k_t||^2                                     (Methodology 2)
+ *   alpha_t  = (1 - exp(-beta_t lambda_t)) / lambda_t        (Methodology 3)
+ *   S_t      = (I - alpha_t k_t k_t^T) S_{t-1} + alpha_t k_t v_t^T
+ *                                                            (Methodology 3)
+ *   o_t      = S_t^T q_t          (delta-rule readout, after the update)
+ *
+ * The summary states that this update keeps the delta rule's rank-1 algebra
+ * and therefore its WY/UT chunkwise parallel form (Methodology 3, last
+ * paragraph); efla_chunk_fwd evaluates that form.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them past the call.  The library allocates no
+ *    device memory: scratch space comes from the caller's workspace.
+ *  - Layouts are dense row-major (C order):
+ *        q, k : [B, H, L, dk]      v, o : [B, H, L, dv]      beta : [B, H, L]
+ *        S0, S_final, S : [B, H, dk, dv]  (fp32; row i is key dimension i)
+ *        alpha : [B, H, L]  (fp32)
+ *    q, k, v, beta and o share the element type `dt`.
+ *  - Pointers must be aligned to 16 bytes.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call is asynchronous with respect to the host: it checks its arguments on
+ *    the host, enqueues kernels on `stream` and returns.  Nothing here
+ *    synchronises the device.
+ *  - Errors are returned as efla_status; no call aborts or throws.  Argument
+ *    errors are detected before anything is enqueued.  EFLA_ERR_CUDA reports a
+ *    failed launch (cudaGetLastError after the launch).  Faults that happen
+ *    later on the device surface through the CUDA runtime as usual.
+ *  - Input values are not inspected: NaN/Inf propagate, negative beta is
+ *    evaluated by the same formula.
+ *  - No scaling or normalisation is applied to q or k (lambda is the raw
+ *    squared norm).
+ */
+#ifndef EFLA_H_
+#define EFLA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EFLA_OK = 0,
+    EFLA_ERR_NULL = 1,        /* a required pointer is NULL */
+    EFLA_ERR_SHAPE = 2,       /* a size is negative, zero where not allowed, or too large */
+    EFLA_ERR_DTYPE = 3,       /* unknown efla_dtype */
+    EFLA_ERR_UNSUPPORTED = 4, /* valid but not implemented (e.g. dk > 256) */
+    EFLA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+    EFLA_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+    EFLA_ERR_WORKSPACE = 7,   /* workspace missing or smaller than the query said */
+    EFLA_ERR_ALIGN = 8        /* a pointer is not 16-byte aligned */
+} efla_status;
+
+typedef enum {
+    EFLA_F32 = 0,  /* float32 inputs/outputs; all arithmetic in fp32 */
+    EFLA_BF16 = 1  /* bfloat16 inputs/outputs; fp32 state and accumulation */
+} efla_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *efla_status_str(int status);
+
+/* ABI version: major*10000 + minor*100 + patch. */
+int efla_version(void);
+
+/*
+ * efla_alpha -- per-token effective coefficient (Methodology 2 and 3).
+ *
+ *   alpha[b,h,t] = -expm1(-beta*lambda)/lambda,  lambda = sum_i k[b,h,t,i]^2,
+ *   and alpha = beta when beta*lambda is 0 (the lambda -> 0 limit).
+ *
+ * k: [B,H,L,dk] of type dt; beta: [B,H,L] of type dt; alpha: [B,H,L] fp32.
+ * Sizes: B,H,L >= 0 (0 tokens is a no-op), 1 <= dk <= 256.
+ */
+efla_status efla_alpha(const void *k, const void *beta, float *alpha,
+                       int B, int H, int L, int dk, efla_dtype dt, void *stream);
+
+/*
+ * Bytes of device workspace efla_chunk_fwd needs for these sizes (0 when the
+ * selected kernels need none).  The same arguments must be passed to
+ * efla_chunk_fwd.  Returns 0 for invalid sizes as well (efla_chunk_fwd then
+ * reports the error).
+ */
+size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int chunk,
+                                     efla_dtype dt);
+
+/*
+ * efla_chunk_fwd -- the whole forward pass in the WY/UT chunkwise form
+ * (Methodology 3: rank-1 updates keep the delta rule's chunkwise
+ * parallelism).  For every head (b, h), chunks of `chunk` tokens are folded
+ * into the carried state; the last chunk may be partial (L need not be a
+ * multiple of chunk).
+ *
+ *   q, k  : [B,H,L,dk]  (dt)          v : [B,H,L,dv] (dt)     beta : [B,H,L] (dt)
+ *   S0    : [B,H,dk,dv] fp32 initial state, or NULL for zeros
+ *   o     : [B,H,L,dv]  (dt) output, o_t = S_t^T q_t
+ *   S_final : [B,H,dk,dv] fp32 state after token L, or NULL to skip
+ *   chunk : 16, 32 or 64 (tokens per WY/UT block)
+ *   workspace, workspace_bytes : caller-owned device scratch of at least
+ *       efla_chunk_fwd_workspace_size(...) bytes (may be NULL when that is 0);
+ *       its contents on entry are ignored and on exit unspecified.
+ * S0 and S_final may alias (in-place state carry).  o must not alias inputs.
+ * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  L == 0 copies S0 to S_final.
+ * Calls on the same workspace must be ordered on one stream.
+ */
+efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
+                           const float *S0, void *o, float *S_final,
+                           int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * efla_recurrent_step -- one decode token per head: the update rule of
+ * Methodology 3 applied once, S updated in place, then o = S^T q.
+ *
+ *   q, k : [B,H,dk] (dt)   v : [B,H,dv] (dt)   beta : [B,H] (dt)
+ *   S    : [B,H,dk,dv] fp32, read and overwritten with the new state
+ *   o    : [B,H,dv] (dt)
+ * Sizes: B,H >= 1, 1 <= dk <= 256, 1 <= dv <= 256.
+ */
+efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
+                                float *S, void *o, int B, int H, int dk, int dv,
+                                efla_dtype dt, void *stream);
+
+/*
+ * Reads and clears the library's device error word after synchronising
+ * `stream`.  Kernels that wait on barriers do so with bounded spins; when a
+ * wait gives up the kernel records it here and exits, leaving the context
+ * usable.  Returns EFLA_OK, EFLA_ERR_TIMEOUT, or EFLA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+efla_status efla_last_device_error(void *stream);
+
+/*
+ * Which chunk-forward kernels the library selects for these sizes:
+ * 0 = SIMT fp32 path, 1 = tensor-core (tcgen05) path.  For tests and tools.
+ */
+int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt);
+
+/*
+ * Number of kernels this library has enqueued since it was loaded (a
+ * host-side counter, incremented per launch; thread-safe).  Lets a caller
+ * count the library's launches inside a timed region.
+ */
+unsigned long long efla_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EFLA_H_ */

@@ -1,0 +1,113 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol that
+include/efla.h declares, and rejects bad arguments on the host before any CUDA
+call (fake pointer values are never dereferenced on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from delta_rule_linear_efla_b200 import efla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from delta_rule_linear_efla_b200 import build
+
+    build.build()
+    return efla.load_library()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "efla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(efla_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    decl = declared_symbols()
+    assert len(decl) >= 8
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert sorted(efla.ABI_SYMBOLS) == sorted(decl)
+
+
+def test_status_strings_and_version(lib):
+    assert efla.status_str(0) == "ok"
+    assert "aligned" in efla.status_str(8)
+    assert efla.status_str(99) == "unknown status"
+    assert lib.efla_version() >= 100
+
+
+BF16, F32 = efla.EFLA_BF16, efla.EFLA_F32
+P = 0x10000  # a fake, 16-byte aligned address (never dereferenced below)
+
+
+def _chunk(lib, **kw):
+    a = dict(q=P, k=P, v=P, beta=P, S0=None, o=P, Sf=P, B=1, H=1, L=64, dk=64, dv=64, chunk=64,
+             dt=BF16, ws=None, wsb=0, s=None)
+    a.update(kw)
+    return lib.efla_chunk_fwd(a["q"], a["k"], a["v"], a["beta"], a["S0"], a["o"], a["Sf"], a["B"],
+                              a["H"], a["L"], a["dk"], a["dv"], a["chunk"], a["dt"], a["ws"],
+                              a["wsb"], a["s"])
+
+
+def test_chunk_fwd_host_errors(lib):
+    assert _chunk(lib, dt=7) == 3                    # EFLA_ERR_DTYPE
+    assert _chunk(lib, B=0) == 2                     # EFLA_ERR_SHAPE
+    assert _chunk(lib, L=-1) == 2
+    assert _chunk(lib, dk=0) == 2
+    assert _chunk(lib, dk=129) == 4                  # EFLA_ERR_UNSUPPORTED
+    assert _chunk(lib, chunk=48) == 4
+    assert _chunk(lib, chunk=128) == 4
+    assert _chunk(lib, q=None) == 1                  # EFLA_ERR_NULL
+    assert _chunk(lib, o=None) == 1
+    assert _chunk(lib, k=P + 2) == 8                 # EFLA_ERR_ALIGN
+    assert _chunk(lib, S0=P + 4) == 8
+
+
+def test_recurrent_step_host_errors(lib):
+    f = lib.efla_recurrent_step
+    assert f(P, P, P, P, P, P, 1, 1, 64, 64, 9, None) == 3
+    assert f(P, P, P, P, P, P, 0, 1, 64, 64, BF16, None) == 2
+    assert f(P, P, P, P, P, P, 1, 1, 300, 64, BF16, None) == 4
+    assert f(P, None, P, P, P, P, 1, 1, 64, 64, BF16, None) == 1
+    assert f(P, P, P, P, P + 8, P, 1, 1, 64, 64, BF16, None) == 8
+
+
+def test_alpha_host_errors(lib):
+    f = lib.efla_alpha
+    assert f(P, P, P, 1, 1, 4, 16, 5, None) == 3
+    assert f(P, P, P, 1, 1, 4, 0, BF16, None) == 2
+    assert f(P, P, P, 1, 1, 4, 512, BF16, None) == 4
+    assert f(None, P, P, 1, 1, 4, 16, BF16, None) == 1
+    assert f(P, P, P, 1, 1, 0, 16, BF16, None) == 0  # zero tokens: nothing to do
+
+
+def test_workspace_query_is_host_only(lib):
+    for wid_sizes in ((8, 8, 2048, 128, 128, 64), (1, 1, 64, 16, 16, 16), (4, 16, 4096, 128, 128, 64)):
+        for dt in (BF16, F32):
+            n = lib.efla_chunk_fwd_workspace_size(*wid_sizes, dt)
+            assert n >= 0
+            path = lib.efla_chunk_fwd_path(*wid_sizes, dt)
+            assert path in (0, 1)
+            if path == 0:
+                assert n == 0
+    assert lib.efla_chunk_fwd_workspace_size(1, 1, 64, 16, 16, 48, BF16) == 0
+
+
+def test_binding_fails_loudly_without_cuda():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    q = torch.zeros(1, 1, 4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        efla.chunk_fwd(q, q, q, torch.zeros(1, 1, 4, dtype=torch.bfloat16))
+
+
+def test_binding_raises_when_library_missing(tmp_path):
+    with pytest.raises(RuntimeError):
+        efla.load_library(str(tmp_path / "missing.so"))

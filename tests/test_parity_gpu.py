@@ -1,0 +1,164 @@
+"""GPU parity: the CUDA chunkwise forward (through the C ABI) against the fp64
+oracle, element by element on the same seeded inputs.
+
+Bounds: max|x_gpu - x_oracle| / RMS(x_oracle) <= 1e-4 for fp32 inputs and
+<= 2e-2 for bf16 inputs with fp32 accumulation, for o and for S_final.  The
+oracle sees the exact dtype-rounded values the GPU sees.
+
+Sizes: every workload at its full size (workload 5 is checked on sampled
+heads the oracle computes one by one, all heads are checked for finiteness),
+plus smaller cases that span several chunks and end in a ragged tail, and the
+edge cases (L = 0, L = 1, L < chunk, dk != dv, S_final aliasing S0, zero keys,
+beta = 0).
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import rel_err
+from delta_rule_linear_efla_b200 import efla, inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+def _to_dev(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def _run_gpu(x, chunk=None):
+    d = _to_dev(x)
+    o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=chunk or x["chunk"])
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    return o.float().cpu(), S.cpu()
+
+
+def _oracle(oracle_mod, x, heads=None):
+    """Oracle on all heads, or on a list of (b, h) heads."""
+    if heads is None:
+        return oracle_mod.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"])
+    os_, Ss = [], []
+    for b, h in heads:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        o, S = oracle_mod.fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]),
+                              None if x["S0"] is None else sl(x["S0"]))
+        os_.append(o[0, 0])
+        Ss.append(S[0, 0])
+    return np.stack(os_), np.stack(Ss)
+
+
+def _check(x, o_gpu, S_gpu, o_ref, S_ref, heads=None):
+    tol = TOL[x["workload"].dtype]
+    if heads is not None:
+        o_gpu = torch.stack([o_gpu[b, h] for b, h in heads])
+        S_gpu = torch.stack([S_gpu[b, h] for b, h in heads])
+    eo, es = rel_err(o_gpu.numpy(), o_ref), rel_err(S_gpu.numpy(), S_ref)
+    assert eo <= tol and es <= tol, (eo, es, tol)
+    return eo, es
+
+
+@pytest.mark.parametrize("wid", [1, 2, 3, 4])
+def test_workload_full_size(oracle_mod, wid):
+    x = inputs.make_inputs(wid)
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+def test_workload5_full_size_sampled_heads(oracle_mod):
+    x = inputs.make_inputs(5)
+    o, S = _run_gpu(x)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    heads = [(0, 0), (0, 15)]
+    o_ref, S_ref = _oracle(oracle_mod, x, heads)
+    _check(x, o, S, o_ref, S_ref, heads)
+
+
+@pytest.mark.parametrize("wid,L,B,H", [(2, 333, 1, 3), (3, 200, 2, 2), (4, 130, 1, 4),
+                                       (5, 1000, 1, 3), (1, 37, 2, 2)])
+def test_ragged_tail(oracle_mod, wid, L, B, H):
+    x = inputs.make_inputs(inputs.workload(wid, L=L, B=B, H=H))
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_chunk_sizes(oracle_mod, chunk, dtype):
+    x = inputs.make_inputs(inputs.workload(3, L=150, B=1, H=2, dk=64, dv=64, dtype=dtype))
+    o, S = _run_gpu(x, chunk=chunk)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (32, 16), (96, 80), (128, 128)])
+def test_rectangular_and_odd_heads(oracle_mod, dk, dv):
+    x = inputs.make_inputs(inputs.workload(2, L=100, B=1, H=2, dk=dk, dv=dv))
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+@pytest.mark.parametrize("L", [1, 5, 63, 64, 65])
+def test_short_sequences(oracle_mod, L):
+    x = inputs.make_inputs(inputs.workload(2, L=L, B=1, H=2))
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+def test_empty_sequence_copies_state():
+    x = inputs.make_inputs(inputs.workload(2, L=0, B=1, H=2))
+    d = _to_dev(x)
+    o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64)
+    assert o.numel() == 0
+    assert torch.equal(S.cpu(), x["S0"])
+    o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], None, chunk=64)
+    assert torch.count_nonzero(S) == 0
+
+
+def test_zero_keys_and_zero_beta_are_noops(oracle_mod):
+    w = inputs.workload(3, L=192, B=1, H=2)
+    x = inputs.make_inputs(w)
+    x["k"][:, :, 10:20] = 0
+    x["beta"][:, :, 70:90] = 0
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+def test_state_aliasing_and_resume(oracle_mod):
+    """S_final may alias S0; running L in two calls with the state carried equals one
+    call (bit-exact when the split falls on a chunk boundary)."""
+    x = inputs.make_inputs(inputs.workload(2, L=256, B=1, H=2))
+    d = _to_dev(x)
+    o_full, S_full = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64)
+    S = d["S0"].clone()
+    sl = lambda t, a, b: t[:, :, a:b].contiguous()
+    o1, _ = efla.chunk_fwd(sl(d["q"], 0, 128), sl(d["k"], 0, 128), sl(d["v"], 0, 128),
+                           sl(d["beta"], 0, 128), S, chunk=64, S_final=S)
+    o2, _ = efla.chunk_fwd(sl(d["q"], 128, 256), sl(d["k"], 128, 256), sl(d["v"], 128, 256),
+                           sl(d["beta"], 128, 256), S, chunk=64, S_final=S)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([o1, o2], dim=2), o_full)
+    assert torch.equal(S, S_full)
+
+
+def test_linearity_in_values_and_state():
+    """o and S_final are linear in (V, S0) for fixed q, k, beta (fp32 inputs)."""
+    w = inputs.workload(1, L=80, B=1, H=2)
+    x = inputs.make_inputs(w)
+    d = _to_dev(x)
+    g = torch.Generator().manual_seed(3)
+    V2 = torch.randn(d["v"].shape, generator=g).cuda()
+    S1 = 0.1 * torch.randn((1, 2, 16, 16), generator=g).cuda()
+    S2 = 0.1 * torch.randn((1, 2, 16, 16), generator=g).cuda()
+    a, b = 0.75, -1.5
+    o1, F1 = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], S1, chunk=16)
+    o2, F2 = efla.chunk_fwd(d["q"], d["k"], V2, d["beta"], S2, chunk=16)
+    o3, F3 = efla.chunk_fwd(d["q"], d["k"], a * d["v"] + b * V2, d["beta"], a * S1 + b * S2, chunk=16)
+    assert rel_err(o3.cpu().numpy(), (a * o1 + b * o2).cpu().numpy()) < 1e-5
+    assert rel_err(F3.cpu().numpy(), (a * F1 + b * F2).cpu().numpy()) < 1e-5
