@@ -17,6 +17,10 @@ void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_rela
 namespace {
 
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_elem(const void *p, efla_dtype dt) {
+    const uintptr_t m = dt == EFLA_BF16 ? 1u : 3u;
+    return p == nullptr || (reinterpret_cast<uintptr_t>(p) & m) == 0;
+}
 
 efla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA; }
 
@@ -36,7 +40,7 @@ const char *efla_status_str(int status) {
         case EFLA_ERR_CUDA: return "CUDA error";
         case EFLA_ERR_TIMEOUT: return "device wait timed out";
         case EFLA_ERR_WORKSPACE: return "workspace missing or too small";
-        case EFLA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case EFLA_ERR_ALIGN: return "pointer not aligned as required";
         default: return "unknown status";
     }
 }
@@ -51,7 +55,8 @@ efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int
     const long long ntok = (long long)B * H * L;
     if (ntok == 0) return EFLA_OK;
     if (!k || !beta || !alpha) return EFLA_ERR_NULL;
-    if (!aligned16(k) || !aligned16(beta) || !aligned16(alpha)) return EFLA_ERR_ALIGN;
+    if (!aligned_elem(k, dt) || !aligned_elem(beta, dt) || !aligned_elem(alpha, EFLA_F32))
+        return EFLA_ERR_ALIGN;
     return from_cuda(efla::launch_alpha(k, beta, alpha, ntok, dk, dt == EFLA_BF16,
                                         (cudaStream_t)stream));
 }
@@ -78,8 +83,8 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
     if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
     if (dk > 128 || dv > 128 || !chunk_ok(chunk)) return EFLA_ERR_UNSUPPORTED;
     if (L > 0 && (!q || !k || !v || !beta || !o)) return EFLA_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S0) ||
-        !aligned16(o) || !aligned16(S_final))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_elem(beta, dt) ||
+        !aligned16(S0) || !aligned16(o) || !aligned16(S_final))
         return EFLA_ERR_ALIGN;
     const bool bf16 = dt == EFLA_BF16;
     cudaStream_t s = (cudaStream_t)stream;
@@ -109,8 +114,8 @@ efla_status efla_recurrent_step(const void *q, const void *k, const void *v, con
     if ((long long)B * H > 0x7fffffffLL) return EFLA_ERR_SHAPE;
     if (dk > 256 || dv > 256) return EFLA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S) ||
-        !aligned16(o))
+    if (!aligned_elem(q, dt) || !aligned_elem(k, dt) || !aligned_elem(v, dt) ||
+        !aligned_elem(beta, dt) || !aligned16(S) || !aligned_elem(o, dt))
         return EFLA_ERR_ALIGN;
     return from_cuda(efla::launch_decode(q, k, v, beta, S, o, B * H, dk, dv, dt == EFLA_BF16,
                                          (cudaStream_t)stream));

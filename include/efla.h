@@ -24,7 +24,10 @@
  *        S0, S_final, S : [B, H, dk, dv]  (fp32; row i is key dimension i)
  *        alpha : [B, H, L]  (fp32)
  *    q, k, v, beta and o share the element type `dt`.
- *  - Pointers must be aligned to 16 bytes.
+ *  - Alignment: fp32 state pointers (S, S0, S_final) and, for
+ *    efla_chunk_fwd, q, k, v and o must be 16-byte aligned (they are read
+ *    with 16-byte vector or bulk-tensor copies); every other pointer must be
+ *    aligned to its element size.  Violations return EFLA_ERR_ALIGN.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    call is asynchronous with respect to the host: it checks its arguments on
  *    the host, enqueues kernels on `stream` and returns.  Nothing here
@@ -56,7 +59,7 @@ typedef enum {
     EFLA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
     EFLA_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
     EFLA_ERR_WORKSPACE = 7,   /* workspace missing or smaller than the query said */
-    EFLA_ERR_ALIGN = 8        /* a pointer is not 16-byte aligned */
+    EFLA_ERR_ALIGN = 8        /* a pointer is not aligned as required */
 } efla_status;
 
 typedef enum {

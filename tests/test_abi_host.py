@@ -74,7 +74,8 @@ def test_recurrent_step_host_errors(lib):
     assert f(P, P, P, P, P, P, 0, 1, 64, 64, BF16, None) == 2
     assert f(P, P, P, P, P, P, 1, 1, 300, 64, BF16, None) == 4
     assert f(P, None, P, P, P, P, 1, 1, 64, 64, BF16, None) == 1
-    assert f(P, P, P, P, P + 8, P, 1, 1, 64, 64, BF16, None) == 8
+    assert f(P, P, P, P, P + 8, P, 1, 1, 64, 64, BF16, None) == 8   # S must be 16-byte aligned
+    assert f(P, P, P, P + 1, P, P, 1, 1, 64, 64, BF16, None) == 8   # bf16 needs 2-byte alignment
 
 
 def test_alpha_host_errors(lib):
