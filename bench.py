@@ -47,11 +47,11 @@ def _peaks():
 
 
 def alg_bytes_chunk(w) -> int:
-    """Algorithmic HBM bytes of one chunk forward: read q, k, v, beta; write o (all in the
-    input dtype) per token-head, plus the fp32 final state per head (S0 is zero here and
+    """Algorithmic HBM bytes of one chunk forward: read q, k, v, beta (input dtype) and
+    write o (fp32) per token-head, plus the fp32 final state per head (S0 is zero here and
     not read)."""
     es = 2 if w.dtype == "bf16" else 4
-    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * es
+    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * 4
     return w.token_heads * per_tok + w.B * w.H * w.dk * w.dv * 4
 
 
@@ -195,7 +195,8 @@ def _config(w) -> dict:
     c = {"workload": "%s (B=%d H=%d L=%d dk=%d dv=%d chunk=%d %s)" % (
         w.name, w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.dtype),
         "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
-        "l2": "inputs > L2 (126 MB): two rotating input sets per rank"}
+        "l2": "inputs > L2 (126 MB): two rotating input sets per rank",
+        "o_dtype": "fp32"}
     if w.decode:
         c["decode"] = "B=%d H=%d one token, fp32 carried state" % (w.decode["B"], w.decode["H"])
     return c
@@ -222,9 +223,10 @@ def run_ours(args) -> None:
     for r in range(2):
         x = inputs.make_inputs(w, seed=1000 + w.id + 7919 * (2 * rank + r))
         sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
-    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype(), device=dev) for _ in range(2)]
+    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
     Sf_buf = [torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
-    ws_bytes = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype())
+    ws_bytes = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(),
+                                   torch.float32)
     wsp = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     path = efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype())
 
@@ -238,7 +240,7 @@ def run_ours(args) -> None:
         _, S_carry = efla.chunk_fwd(pd["q"], pd["k"], pd["v"], pd["beta"], None, chunk=w.chunk)
         dd["S_init"] = S_carry
         dd["S"] = [S_carry.clone(), S_carry.clone()]
-        dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=w.torch_dtype(), device=dev)
+        dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=torch.float32, device=dev)
         dec = dd
     tok_dec = (w.decode["B"] * w.decode["H"]) if w.decode else 0
     tok_step = w.token_heads + tok_dec
@@ -301,7 +303,7 @@ def run_ours(args) -> None:
     if not args.no_e2e:
         xh = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v)
               for k, v in inputs.make_inputs(w, seed=4242 + rank).items()}
-        o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype()).pin_memory()
+        o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32).pin_memory()
         S_host = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
         h2d = sum(xh[k].numel() * xh[k].element_size() for k in ("q", "k", "v", "beta"))
         d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4

@@ -26,6 +26,8 @@ efla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? EFLA_OK : EFLA_
 
 bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
 
+bool dtype_ok(efla_dtype d) { return d == EFLA_F32 || d == EFLA_BF16; }
+
 }  // namespace
 
 extern "C" {
@@ -61,14 +63,16 @@ efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int
                                         (cudaStream_t)stream));
 }
 
-int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt) {
+int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                        efla_dtype o_dt) {
+    (void)o_dt;
     return efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16) ? 1 : 0;
 }
 
 size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int chunk,
-                                     efla_dtype dt) {
+                                     efla_dtype dt, efla_dtype o_dt) {
     if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1 || !chunk_ok(chunk)) return 0;
-    if (dt != EFLA_F32 && dt != EFLA_BF16) return 0;
+    if (!dtype_ok(dt) || !dtype_ok(o_dt)) return 0;
     if (efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16))
         return efla::tc_workspace_bytes(B, H, L, dk, dv, chunk);
     return 0;
@@ -76,9 +80,9 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
 
 efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
                            const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
-                           int dv, int chunk, efla_dtype dt, void *workspace,
+                           int dv, int chunk, efla_dtype dt, efla_dtype o_dt, void *workspace,
                            size_t workspace_bytes, void *stream) {
-    if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
+    if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
     if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
     if (dk > 128 || dv > 128 || !chunk_ok(chunk)) return EFLA_ERR_UNSUPPORTED;
@@ -86,7 +90,7 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_elem(beta, dt) ||
         !aligned16(S0) || !aligned16(o) || !aligned16(S_final))
         return EFLA_ERR_ALIGN;
-    const bool bf16 = dt == EFLA_BF16;
+    const bool bf16 = dt == EFLA_BF16, o_bf16 = o_dt == EFLA_BF16;
     cudaStream_t s = (cudaStream_t)stream;
     if (L == 0) {
         if (!S_final) return EFLA_OK;
@@ -100,25 +104,25 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
         if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
         if (!aligned16(workspace)) return EFLA_ERR_ALIGN;
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
-                                               chunk, workspace, s));
+                                               chunk, o_bf16, workspace, s));
     }
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
-                                             chunk, bf16, s));
+                                             chunk, bf16, o_bf16, s));
 }
 
 efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
                                 float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
-                                void *stream) {
-    if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
+                                efla_dtype o_dt, void *stream) {
+    if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
     if ((long long)B * H > 0x7fffffffLL) return EFLA_ERR_SHAPE;
     if (dk > 256 || dv > 256) return EFLA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_NULL;
     if (!aligned_elem(q, dt) || !aligned_elem(k, dt) || !aligned_elem(v, dt) ||
-        !aligned_elem(beta, dt) || !aligned16(S) || !aligned_elem(o, dt))
+        !aligned_elem(beta, dt) || !aligned16(S) || !aligned_elem(o, o_dt))
         return EFLA_ERR_ALIGN;
     return from_cuda(efla::launch_decode(q, k, v, beta, S, o, B * H, dk, dv, dt == EFLA_BF16,
-                                         (cudaStream_t)stream));
+                                         o_dt == EFLA_BF16, (cudaStream_t)stream));
 }
 
 unsigned long long efla_kernel_launches(void) {

@@ -47,10 +47,10 @@ struct SimtSmem {
     }
 };
 
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(SIMT_THREADS)
     chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const T *__restrict__ beta, const float *__restrict__ S0, T *__restrict__ o,
+                      const T *__restrict__ beta, const float *__restrict__ S0, TO *__restrict__ o,
                       float *__restrict__ S_final, int L, int dk, int dv, int C, int NV) {
     extern __shared__ float sm[];
     const SimtSmem lay(dk, C, NV);
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
             float s = 0.f;
             for (int d = 0; d < dk; ++d) s = fmaf(Qs[i * dkp + d], Ss[d * NVp + n], s);
             for (int j = 0; j <= i; ++j) s = fmaf(Ps[i * Cp + j], Vs[j * NVp + n], s);
-            o[(row0 + i) * dv + v0 + n] = from_f32<T>(s);
+            o[(row0 + i) * dv + v0 + n] = from_f32<TO>(s);
         }
         __syncthreads();
         // S <- S + K^T U'
@@ -178,30 +178,34 @@ __global__ void __launch_bounds__(SIMT_THREADS)
     }
 }
 
-cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
-                              const float *S0, void *o, float *S_final, int B, int H, int L,
-                              int dk, int dv, int chunk, bool is_bf16, cudaStream_t s) {
+template <typename T, typename TO>
+static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const void *beta,
+                                 const float *S0, void *o, float *S_final, int B, int H, int L,
+                                 int dk, int dv, int chunk, cudaStream_t s) {
     const int NV = dv < SIMT_NV ? dv : SIMT_NV;
     const SimtSmem lay(dk, chunk, NV);
     dim3 grid(B * H, (dv + NV - 1) / NV);
-    cudaError_t e;
-    if (is_bf16) {
-        e = cudaFuncSetAttribute(chunk_simt_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
-        if (e != cudaSuccess) return e;
-        chunk_simt_kernel<__nv_bfloat16><<<grid, SIMT_THREADS, lay.total, s>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            (const __nv_bfloat16 *)beta, S0, (__nv_bfloat16 *)o, S_final, L, dk, dv, chunk, NV);
-    } else {
-        e = cudaFuncSetAttribute(chunk_simt_kernel<float>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
-        if (e != cudaSuccess) return e;
-        chunk_simt_kernel<float><<<grid, SIMT_THREADS, lay.total, s>>>(
-            (const float *)q, (const float *)k, (const float *)v, (const float *)beta, S0,
-            (float *)o, S_final, L, dk, dv, chunk, NV);
-    }
+    cudaError_t e = cudaFuncSetAttribute(chunk_simt_kernel<T, TO>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)lay.total);
+    if (e != cudaSuccess) return e;
+    chunk_simt_kernel<T, TO><<<grid, SIMT_THREADS, lay.total, s>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S0, (TO *)o, S_final, L, dk,
+        dv, chunk, NV);
     count_launches(1);
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
+                              const float *S0, void *o, float *S_final, int B, int H, int L,
+                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16,
+                              cudaStream_t s) {
+    using bf = __nv_bfloat16;
+    if (is_bf16)
+        return o_bf16 ? launch_simt_t<bf, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s)
+                      : launch_simt_t<bf, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s);
+    return o_bf16 ? launch_simt_t<float, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s)
+                  : launch_simt_t<float, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s);
 }
 
 }  // namespace efla

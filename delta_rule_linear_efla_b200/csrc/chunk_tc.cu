@@ -9,7 +9,8 @@ static __device__ unsigned int g_tc_error = 0;
 bool tc_supported(int, int, int, int, int, int, bool) { return false; }
 size_t tc_workspace_bytes(int, int, int, int, int, int) { return 0; }
 cudaError_t launch_chunk_tc(const void *, const void *, const void *, const void *, const float *,
-                            void *, float *, int, int, int, int, int, int, void *, cudaStream_t) {
+                            void *, float *, int, int, int, int, int, int, bool, void *,
+                            cudaStream_t) {
     return cudaErrorNotSupported;
 }
 

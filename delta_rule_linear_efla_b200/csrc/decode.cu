@@ -24,10 +24,10 @@ struct DecodeCfg {
     static constexpr int PASSES = DK / RPP;
 };
 
-template <typename T, int DK, int DV>
+template <typename T, typename TO, int DK, int DV>
 __global__ void __launch_bounds__(DecodeCfg<T, DK, DV>::NT)
     decode_reg_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const T *__restrict__ beta, float *__restrict__ S, T *__restrict__ o) {
+                      const T *__restrict__ beta, float *__restrict__ S, TO *__restrict__ o) {
     using Cfg = DecodeCfg<T, DK, DV>;
     constexpr int TPR = Cfg::TPR, RPP = Cfg::RPP, PASSES = Cfg::PASSES, NT = Cfg::NT;
     __shared__ float ks[DK], qs[DK], vs[DV];
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, DK, DV>::NT)
         }
         const float u = sc[0] * (vs[c] - x);
         us[c] = u;
-        o[(size_t)bh * DV + c] = from_f32<T>(fmaf(sc[1], u, y));
+        o[(size_t)bh * DV + c] = from_f32<TO>(fmaf(sc[1], u, y));
     }
     __syncthreads();
     const float4 u4 = *reinterpret_cast<const float4 *>(&us[4 * cg]);
@@ -98,11 +98,11 @@ __global__ void __launch_bounds__(DecodeCfg<T, DK, DV>::NT)
 }
 
 // Any dk, dv <= 256: one thread per state column, two passes over the state.
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(256)
     decode_generic_kernel(const T *__restrict__ q, const T *__restrict__ k,
                           const T *__restrict__ v, const T *__restrict__ beta,
-                          float *__restrict__ S, T *__restrict__ o, int dk, int dv) {
+                          float *__restrict__ S, TO *__restrict__ o, int dk, int dv) {
     __shared__ float ks[256], qs[256];
     __shared__ float sc[2];
     const int bh = blockIdx.x, tid = threadIdx.x;
@@ -134,54 +134,58 @@ __global__ void __launch_bounds__(256)
             y = fmaf(s, qs[r], y);
         }
         const float u = sc[0] * (to_f32(v[(size_t)bh * dv + c]) - x);
-        o[(size_t)bh * dv + c] = from_f32<T>(fmaf(sc[1], u, y));
+        o[(size_t)bh * dv + c] = from_f32<TO>(fmaf(sc[1], u, y));
         for (int r = 0; r < dk; ++r) Sh[(size_t)r * dv + c] = fmaf(ks[r], u, Sh[(size_t)r * dv + c]);
     }
 }
 
-template <typename T, int DK, int DV>
+template <typename T, typename TO, int DK, int DV>
 static void launch_reg(const void *q, const void *k, const void *v, const void *beta, float *S,
                        void *o, int BH, cudaStream_t s) {
-    decode_reg_kernel<T, DK, DV><<<BH, DecodeCfg<T, DK, DV>::NT, 0, s>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S, (T *)o);
+    decode_reg_kernel<T, TO, DK, DV><<<BH, DecodeCfg<T, DK, DV>::NT, 0, s>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S, (TO *)o);
 }
 
-template <typename T, int DK>
+template <typename T, typename TO, int DK>
 static bool dispatch_dv(const void *q, const void *k, const void *v, const void *beta, float *S,
                         void *o, int BH, int dv, cudaStream_t s) {
     switch (dv) {
-        case 16: launch_reg<T, DK, 16>(q, k, v, beta, S, o, BH, s); return true;
-        case 32: launch_reg<T, DK, 32>(q, k, v, beta, S, o, BH, s); return true;
-        case 64: launch_reg<T, DK, 64>(q, k, v, beta, S, o, BH, s); return true;
-        case 128: launch_reg<T, DK, 128>(q, k, v, beta, S, o, BH, s); return true;
+        case 16: launch_reg<T, TO, DK, 16>(q, k, v, beta, S, o, BH, s); return true;
+        case 32: launch_reg<T, TO, DK, 32>(q, k, v, beta, S, o, BH, s); return true;
+        case 64: launch_reg<T, TO, DK, 64>(q, k, v, beta, S, o, BH, s); return true;
+        case 128: launch_reg<T, TO, DK, 128>(q, k, v, beta, S, o, BH, s); return true;
         default: return false;
     }
 }
 
-template <typename T>
+template <typename T, typename TO>
 static void dispatch(const void *q, const void *k, const void *v, const void *beta, float *S,
                      void *o, int BH, int dk, int dv, cudaStream_t s) {
     bool done = false;
     switch (dk) {
-        case 16: done = dispatch_dv<T, 16>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 32: done = dispatch_dv<T, 32>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 64: done = dispatch_dv<T, 64>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 128: done = dispatch_dv<T, 128>(q, k, v, beta, S, o, BH, dv, s); break;
+        case 16: done = dispatch_dv<T, TO, 16>(q, k, v, beta, S, o, BH, dv, s); break;
+        case 32: done = dispatch_dv<T, TO, 32>(q, k, v, beta, S, o, BH, dv, s); break;
+        case 64: done = dispatch_dv<T, TO, 64>(q, k, v, beta, S, o, BH, dv, s); break;
+        case 128: done = dispatch_dv<T, TO, 128>(q, k, v, beta, S, o, BH, dv, s); break;
         default: break;
     }
     if (!done)
-        decode_generic_kernel<T><<<BH, 256, 0, s>>>((const T *)q, (const T *)k, (const T *)v,
-                                                    (const T *)beta, S, (T *)o, dk, dv);
+        decode_generic_kernel<T, TO><<<BH, 256, 0, s>>>((const T *)q, (const T *)k, (const T *)v,
+                                                        (const T *)beta, S, (TO *)o, dk, dv);
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
-                          float *S, void *o, int BH, int dk, int dv, bool is_bf16,
+                          float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
                           cudaStream_t s) {
+    using bf = __nv_bfloat16;
     if (BH <= 0) return cudaSuccess;
-    if (is_bf16)
-        dispatch<__nv_bfloat16>(q, k, v, beta, S, o, BH, dk, dv, s);
-    else
-        dispatch<float>(q, k, v, beta, S, o, BH, dk, dv, s);
+    if (is_bf16) {
+        if (o_bf16) dispatch<bf, bf>(q, k, v, beta, S, o, BH, dk, dv, s);
+        else dispatch<bf, float>(q, k, v, beta, S, o, BH, dk, dv, s);
+    } else {
+        if (o_bf16) dispatch<float, bf>(q, k, v, beta, S, o, BH, dk, dv, s);
+        else dispatch<float, float>(q, k, v, beta, S, o, BH, dk, dv, s);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

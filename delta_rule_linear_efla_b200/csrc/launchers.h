@@ -18,13 +18,15 @@ cudaError_t launch_alpha(const void *k, const void *beta, float *alpha, long lon
 
 // SIMT fp32 chunkwise forward: WY/UT per chunk, state carried in fp32.
 // Any dk, dv <= 128 and chunk <= 64.
+// o_bf16 selects the output element type (fp32 or bf16).
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
                               const float *S0, void *o, float *S_final, int B, int H, int L,
-                              int dk, int dv, int chunk, bool is_bf16, cudaStream_t s);
+                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16,
+                              cudaStream_t s);
 
 // Recurrent single-token step per head (decode), S updated in place.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
-                          float *S, void *o, int BH, int dk, int dv, bool is_bf16,
+                          float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
                           cudaStream_t s);
 
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
@@ -32,7 +34,7 @@ bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
 size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
                             const float *S0, void *o, float *S_final, int B, int H, int L,
-                            int dk, int dv, int chunk, void *ws, cudaStream_t s);
+                            int dk, int dv, int chunk, bool o_bf16, void *ws, cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits): read and clear.
 cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s);
 

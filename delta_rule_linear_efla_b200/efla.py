@@ -52,15 +52,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_alpha.restype = i
     L.efla_alpha.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
     L.efla_chunk_fwd_workspace_size.restype = sz
-    L.efla_chunk_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.efla_chunk_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
     L.efla_chunk_fwd.restype = i
-    L.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    L.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
     L.efla_recurrent_step.restype = i
-    L.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     L.efla_last_device_error.restype = i
     L.efla_last_device_error.argtypes = [vp]
     L.efla_chunk_fwd_path.restype = i
-    L.efla_chunk_fwd_path.argtypes = [i, i, i, i, i, i, i]
+    L.efla_chunk_fwd_path.argtypes = [i, i, i, i, i, i, i, i]
     L.efla_kernel_launches.restype = ctypes.c_ulonglong
     L.efla_kernel_launches.argtypes = []
     if path is None:
@@ -77,12 +77,16 @@ def _check(status: int, where: str) -> None:
         raise EflaError(status, where)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.float32:
+def _code(dtype) -> int:
+    if dtype == torch.float32:
         return EFLA_F32
-    if t.dtype == torch.bfloat16:
+    if dtype == torch.bfloat16:
         return EFLA_BF16
-    raise TypeError("EFLA tensors must be float32 or bfloat16, got %s" % t.dtype)
+    raise TypeError("EFLA tensors must be float32 or bfloat16, got %s" % dtype)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return _code(t.dtype)
 
 
 def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
@@ -114,23 +118,25 @@ def alpha(k: torch.Tensor, beta: torch.Tensor, out: torch.Tensor | None = None, 
     return out
 
 
-def workspace_size(B: int, H: int, L: int, dk: int, dv: int, chunk: int, dtype) -> int:
-    code = EFLA_BF16 if dtype == torch.bfloat16 else EFLA_F32
-    return int(load_library().efla_chunk_fwd_workspace_size(B, H, L, dk, dv, chunk, code))
+def workspace_size(B: int, H: int, L: int, dk: int, dv: int, chunk: int, dtype,
+                   o_dtype=torch.float32) -> int:
+    return int(load_library().efla_chunk_fwd_workspace_size(B, H, L, dk, dv, chunk, _code(dtype),
+                                                            _code(o_dtype)))
 
 
-def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype) -> str:
-    code = EFLA_BF16 if dtype == torch.bfloat16 else EFLA_F32
-    return "tcgen05" if load_library().efla_chunk_fwd_path(B, H, L, dk, dv, chunk, code) else "simt"
+def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype, o_dtype=torch.float32) -> str:
+    p = load_library().efla_chunk_fwd_path(B, H, L, dk, dv, chunk, _code(dtype), _code(o_dtype))
+    return "tcgen05" if p else "simt"
 
 
 def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
-              want_state: bool = True, workspace=None, stream=None):
+              want_state: bool = True, workspace=None, o_dtype=torch.float32, stream=None):
     """EFLA forward in the WY/UT chunkwise form.  Returns (o, S_final or None).
 
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L], all float32 or all bfloat16 on one
-    CUDA device; S0: [B,H,dk,dv] float32 or None.  o has the inputs' dtype; S_final is
-    float32.  S_final may be S0 (in-place carry)."""
+    CUDA device; S0: [B,H,dk,dv] float32 or None.  o is float32 by default (the fp32
+    accumulator) or bfloat16 with o_dtype=torch.bfloat16; S_final is float32 and may be S0
+    (in-place carry)."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L):
@@ -139,11 +145,14 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
     for name, t in (("k", k), ("v", v), ("beta", beta)):
         if t.dtype != q.dtype:
             raise TypeError("%s must have q's dtype %s" % (name, q.dtype))
+    if o is not None:
+        o_dtype = o.dtype
+    o_code = _code(o_dtype)
     if o is None:
-        o = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((B, H, L, dv), dtype=o_dtype, device=q.device)
     if S_final is None and want_state:
         S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
-    need = workspace_size(B, H, L, dk, dv, chunk, q.dtype)
+    need = workspace_size(B, H, L, dk, dv, chunk, q.dtype, o_dtype)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
@@ -151,26 +160,29 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
     st = load_library().efla_chunk_fwd(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
         _dev(S0, "S0", torch.float32) if S0 is not None else None,
-        _dev(o, "o", q.dtype),
+        _dev(o, "o", o_dtype),
         _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
-        B, H, L, dk, dv, int(chunk), code, ws_ptr, ws_bytes, _stream_handle(stream))
+        B, H, L, dk, dv, int(chunk), code, o_code, ws_ptr, ws_bytes, _stream_handle(stream))
     _check(st, "efla_chunk_fwd")
     return o, S_final
 
 
-def recurrent_step(q, k, v, beta, S, o=None, stream=None):
-    """One decode token per head; S ([B,H,dk,dv] float32) is updated in place.  Returns o."""
+def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None):
+    """One decode token per head; S ([B,H,dk,dv] float32) is updated in place.  Returns o
+    (float32 by default, or bfloat16 with o_dtype=torch.bfloat16)."""
     B, H, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:2] != (B, H) or beta.shape != (B, H) or \
             S.shape != (B, H, dk, dv):
         raise ValueError("shape mismatch: q,k [B,H,dk], v [B,H,dv], beta [B,H], S [B,H,dk,dv]")
     code = _dtype_code(q)
+    if o is not None:
+        o_dtype = o.dtype
     if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((B, H, dv), dtype=o_dtype, device=q.device)
     st = load_library().efla_recurrent_step(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
-        _dev(S, "S", torch.float32), _dev(o, "o", q.dtype), B, H, dk, dv, code,
+        _dev(S, "S", torch.float32), _dev(o, "o", o_dtype), B, H, dk, dv, code, _code(o_dtype),
         _stream_handle(stream))
     _check(st, "efla_recurrent_step")
     return o

@@ -23,7 +23,8 @@
  *        q, k : [B, H, L, dk]      v, o : [B, H, L, dv]      beta : [B, H, L]
  *        S0, S_final, S : [B, H, dk, dv]  (fp32; row i is key dimension i)
  *        alpha : [B, H, L]  (fp32)
- *    q, k, v, beta and o share the element type `dt`.
+ *    q, k, v and beta share the element type `dt`; o has the element type
+ *    `o_dt` (fp32 keeps the fp32 accumulator; bf16 rounds it).
  *  - Alignment: fp32 state pointers (S, S0, S_final) and, for
  *    efla_chunk_fwd, q, k, v and o must be 16-byte aligned (they are read
  *    with 16-byte vector or bulk-tensor copies); every other pointer must be
@@ -92,7 +93,7 @@ efla_status efla_alpha(const void *k, const void *beta, float *alpha,
  * reports the error).
  */
 size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int chunk,
-                                     efla_dtype dt);
+                                     efla_dtype dt, efla_dtype o_dt);
 
 /*
  * efla_chunk_fwd -- the whole forward pass in the WY/UT chunkwise form
@@ -103,7 +104,7 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
  *
  *   q, k  : [B,H,L,dk]  (dt)          v : [B,H,L,dv] (dt)     beta : [B,H,L] (dt)
  *   S0    : [B,H,dk,dv] fp32 initial state, or NULL for zeros
- *   o     : [B,H,L,dv]  (dt) output, o_t = S_t^T q_t
+ *   o     : [B,H,L,dv]  (o_dt) output, o_t = S_t^T q_t
  *   S_final : [B,H,dk,dv] fp32 state after token L, or NULL to skip
  *   chunk : 16, 32 or 64 (tokens per WY/UT block)
  *   workspace, workspace_bytes : caller-owned device scratch of at least
@@ -116,7 +117,8 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
 efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
                            const float *S0, void *o, float *S_final,
                            int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
-                           void *workspace, size_t workspace_bytes, void *stream);
+                           efla_dtype o_dt, void *workspace, size_t workspace_bytes,
+                           void *stream);
 
 /*
  * efla_recurrent_step -- one decode token per head: the update rule of
@@ -124,12 +126,12 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
  *
  *   q, k : [B,H,dk] (dt)   v : [B,H,dv] (dt)   beta : [B,H] (dt)
  *   S    : [B,H,dk,dv] fp32, read and overwritten with the new state
- *   o    : [B,H,dv] (dt)
+ *   o    : [B,H,dv] (o_dt)
  * Sizes: B,H >= 1, 1 <= dk <= 256, 1 <= dv <= 256.
  */
 efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
                                 float *S, void *o, int B, int H, int dk, int dv,
-                                efla_dtype dt, void *stream);
+                                efla_dtype dt, efla_dtype o_dt, void *stream);
 
 /*
  * Reads and clears the library's device error word after synchronising
@@ -144,7 +146,8 @@ efla_status efla_last_device_error(void *stream);
  * Which chunk-forward kernels the library selects for these sizes:
  * 0 = SIMT fp32 path, 1 = tensor-core (tcgen05) path.  For tests and tools.
  */
-int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt);
+int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                        efla_dtype o_dt);
 
 /*
  * Number of kernels this library has enqueued since it was loaded (a

@@ -47,15 +47,16 @@ P = 0x10000  # a fake, 16-byte aligned address (never dereferenced below)
 
 def _chunk(lib, **kw):
     a = dict(q=P, k=P, v=P, beta=P, S0=None, o=P, Sf=P, B=1, H=1, L=64, dk=64, dv=64, chunk=64,
-             dt=BF16, ws=None, wsb=0, s=None)
+             dt=BF16, odt=F32, ws=None, wsb=0, s=None)
     a.update(kw)
     return lib.efla_chunk_fwd(a["q"], a["k"], a["v"], a["beta"], a["S0"], a["o"], a["Sf"], a["B"],
-                              a["H"], a["L"], a["dk"], a["dv"], a["chunk"], a["dt"], a["ws"],
-                              a["wsb"], a["s"])
+                              a["H"], a["L"], a["dk"], a["dv"], a["chunk"], a["dt"], a["odt"],
+                              a["ws"], a["wsb"], a["s"])
 
 
 def test_chunk_fwd_host_errors(lib):
     assert _chunk(lib, dt=7) == 3                    # EFLA_ERR_DTYPE
+    assert _chunk(lib, odt=2) == 3
     assert _chunk(lib, B=0) == 2                     # EFLA_ERR_SHAPE
     assert _chunk(lib, L=-1) == 2
     assert _chunk(lib, dk=0) == 2
@@ -70,12 +71,14 @@ def test_chunk_fwd_host_errors(lib):
 
 def test_recurrent_step_host_errors(lib):
     f = lib.efla_recurrent_step
-    assert f(P, P, P, P, P, P, 1, 1, 64, 64, 9, None) == 3
-    assert f(P, P, P, P, P, P, 0, 1, 64, 64, BF16, None) == 2
-    assert f(P, P, P, P, P, P, 1, 1, 300, 64, BF16, None) == 4
-    assert f(P, None, P, P, P, P, 1, 1, 64, 64, BF16, None) == 1
-    assert f(P, P, P, P, P + 8, P, 1, 1, 64, 64, BF16, None) == 8   # S must be 16-byte aligned
-    assert f(P, P, P, P + 1, P, P, 1, 1, 64, 64, BF16, None) == 8   # bf16 needs 2-byte alignment
+    assert f(P, P, P, P, P, P, 1, 1, 64, 64, 9, F32, None) == 3
+    assert f(P, P, P, P, P, P, 1, 1, 64, 64, BF16, 9, None) == 3
+    assert f(P, P, P, P, P, P, 0, 1, 64, 64, BF16, F32, None) == 2
+    assert f(P, P, P, P, P, P, 1, 1, 300, 64, BF16, F32, None) == 4
+    assert f(P, None, P, P, P, P, 1, 1, 64, 64, BF16, F32, None) == 1
+    assert f(P, P, P, P, P + 8, P, 1, 1, 64, 64, BF16, F32, None) == 8   # S: 16-byte aligned
+    assert f(P, P, P, P + 1, P, P, 1, 1, 64, 64, BF16, F32, None) == 8   # bf16: 2-byte aligned
+    assert f(P, P, P, P, P, P + 2, 1, 1, 64, 64, BF16, F32, None) == 8   # fp32 o: 4-byte aligned
 
 
 def test_alpha_host_errors(lib):
@@ -90,13 +93,13 @@ def test_alpha_host_errors(lib):
 def test_workspace_query_is_host_only(lib):
     for wid_sizes in ((8, 8, 2048, 128, 128, 64), (1, 1, 64, 16, 16, 16), (4, 16, 4096, 128, 128, 64)):
         for dt in (BF16, F32):
-            n = lib.efla_chunk_fwd_workspace_size(*wid_sizes, dt)
+            n = lib.efla_chunk_fwd_workspace_size(*wid_sizes, dt, F32)
             assert n >= 0
-            path = lib.efla_chunk_fwd_path(*wid_sizes, dt)
+            path = lib.efla_chunk_fwd_path(*wid_sizes, dt, F32)
             assert path in (0, 1)
             if path == 0:
                 assert n == 0
-    assert lib.efla_chunk_fwd_workspace_size(1, 1, 64, 16, 16, 48, BF16) == 0
+    assert lib.efla_chunk_fwd_workspace_size(1, 1, 64, 16, 16, 48, BF16, F32) == 0
 
 
 def test_binding_fails_loudly_without_cuda():

@@ -68,6 +68,22 @@ def test_decode_shapes(oracle_mod, dk, dv, dtype):
     assert rel_err(S.cpu().numpy(), S_ref) <= 1e-4
 
 
+def test_decode_bf16_output():
+    g = torch.Generator().manual_seed(5)
+    q = (torch.randn((4, 16, 128), generator=g) / 11.3).bfloat16()
+    k = (torch.randn((4, 16, 128), generator=g) / 11.3).bfloat16()
+    v = torch.randn((4, 16, 128), generator=g).bfloat16()
+    beta = torch.sigmoid(torch.randn((4, 16), generator=g)).bfloat16()
+    S0 = 0.3 * torch.randn((4, 16, 128, 128), generator=g)
+    S1, S2 = S0.cuda(), S0.cuda()
+    o32 = efla.recurrent_step(q.cuda(), k.cuda(), v.cuda(), beta.cuda(), S1)
+    o16 = efla.recurrent_step(q.cuda(), k.cuda(), v.cuda(), beta.cuda(), S2, o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16 and o32.dtype == torch.float32
+    assert torch.equal(o16, o32.bfloat16())
+    assert torch.equal(S1, S2)
+
+
 def test_decode_matches_one_token_chunk_forward():
     """A decode step equals a one-token chunk forward from the same state."""
     x = inputs.make_inputs(inputs.workload(2, L=1, B=2, H=3))
@@ -94,5 +110,5 @@ def test_alpha_kernel(oracle_mod, dtype):
     ref = np.vectorize(oracle_mod.alpha)(lam, bt)
     got = a.cpu().double().numpy()
     rel = np.abs(got - ref) / np.abs(ref)
-    assert rel.max() < 2e-6, rel.max()
+    assert rel.max() < 1e-5, rel.max()  # fp32 sum of dk squares + expm1f
     assert np.array_equal(got[0, 0, :5], bt[0, 0, :5].astype(np.float32).astype(np.float64))

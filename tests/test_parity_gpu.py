@@ -2,8 +2,11 @@
 oracle, element by element on the same seeded inputs.
 
 Bounds: max|x_gpu - x_oracle| / RMS(x_oracle) <= 1e-4 for fp32 inputs and
-<= 2e-2 for bf16 inputs with fp32 accumulation, for o and for S_final.  The
-oracle sees the exact dtype-rounded values the GPU sees.
+<= 2e-2 for bf16 inputs with fp32 accumulation, for o and for S_final; o is
+the fp32 accumulator (the library's default output type).  The oracle sees the
+exact dtype-rounded values the GPU sees.  The optional bf16 output adds its own
+rounding, at most half a bf16 ulp (2^-8 relative) per element, so it is checked
+against 2e-2 + 2^-8 max|o| / RMS(o).
 
 Sizes: every workload at its full size (workload 5 is checked on sampled
 heads the oracle computes one by one, all heads are checked for finiteness),
@@ -145,6 +148,21 @@ def test_state_aliasing_and_resume(oracle_mod):
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([o1, o2], dim=2), o_full)
     assert torch.equal(S, S_full)
+
+
+@pytest.mark.parametrize("wid", [3, 5])
+def test_bf16_output_option(oracle_mod, wid):
+    x = inputs.make_inputs(inputs.workload(wid, L=300, B=1, H=2))
+    d = _to_dev(x)
+    o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64,
+                          o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    rms = float(np.sqrt(np.mean(o_ref ** 2)))
+    bound = 2e-2 + 2.0 ** -8 * float(np.abs(o_ref).max()) / rms
+    assert rel_err(o.float().cpu().numpy(), o_ref) <= bound
+    assert rel_err(S.cpu().numpy(), S_ref) <= 2e-2
 
 
 def test_linearity_in_values_and_state():
