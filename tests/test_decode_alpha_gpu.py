@@ -93,8 +93,12 @@ def test_decode_matches_one_token_chunk_forward():
     o2 = efla.recurrent_step(d["q"][:, :, 0].contiguous(), d["k"][:, :, 0].contiguous(),
                              d["v"][:, :, 0].contiguous(), d["beta"][:, :, 0].contiguous(), S)
     torch.cuda.synchronize()
+    # the chunk forward of bf16 inputs runs on the tensor cores with fp16 operands
+    # (relative rounding 2^-11 per operand); the decode step is fp32 throughout
+    tc = efla.chunk_fwd_path(2, 3, 1, 64, 64, 64, torch.bfloat16) == "tcgen05"
+    tol = 1e-2 if tc else 1e-5
     assert rel_err(o2.float().cpu().numpy(), o1[:, :, 0].float().cpu().numpy()) < 2e-2
-    assert rel_err(S.cpu().numpy(), S1.cpu().numpy()) < 1e-5
+    assert rel_err(S.cpu().numpy(), S1.cpu().numpy()) < tol
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])

@@ -165,6 +165,33 @@ def test_bf16_output_option(oracle_mod, wid):
     assert rel_err(S.cpu().numpy(), S_ref) <= 2e-2
 
 
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
+def test_tensor_core_path_selected(dk, dv):
+    """bf16 inputs with chunk 64 and head sizes 64/128 take the tcgen05 kernels."""
+    assert efla.chunk_fwd_path(2, 4, 1000, dk, dv, 64, torch.bfloat16) == "tcgen05"
+    assert efla.chunk_fwd_path(2, 4, 1000, dk, dv, 64, torch.float32) == "simt"
+    assert efla.chunk_fwd_path(2, 4, 1000, dk, dv, 32, torch.bfloat16) == "simt"
+
+
+def test_tensor_core_state_carry_across_calls(oracle_mod):
+    """Chunk boundaries aligned to calls: two tcgen05 calls with the state carried equal
+    one call up to the fp16 rounding of the carried state's operand copy."""
+    x = inputs.make_inputs(inputs.workload(4, L=512, B=1, H=2))
+    d = _to_dev(x)
+    o_full, S_full = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], None, chunk=64)
+    sl = lambda t, a, b: t[:, :, a:b].contiguous()
+    o1, S1 = efla.chunk_fwd(sl(d["q"], 0, 256), sl(d["k"], 0, 256), sl(d["v"], 0, 256),
+                            sl(d["beta"], 0, 256), None, chunk=64)
+    o2, S2 = efla.chunk_fwd(sl(d["q"], 256, 512), sl(d["k"], 256, 512), sl(d["v"], 256, 512),
+                            sl(d["beta"], 256, 512), S1, chunk=64)
+    torch.cuda.synchronize()
+    # loading S0 into the tensor-memory state is exact, so the split run is bit-identical
+    assert torch.equal(torch.cat([o1, o2], dim=2), o_full)
+    assert torch.equal(S2, S_full)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    assert rel_err(S2.cpu().numpy(), S_ref) < 2e-2
+
+
 def test_linearity_in_values_and_state():
     """o and S_final are linear in (V, S0) for fixed q, k, beta (fp32 inputs)."""
     w = inputs.workload(1, L=80, B=1, H=2)
