@@ -43,6 +43,7 @@ const char *efla_status_str(int status) {
         case EFLA_ERR_TIMEOUT: return "device wait timed out";
         case EFLA_ERR_WORKSPACE: return "workspace missing or too small";
         case EFLA_ERR_ALIGN: return "pointer not aligned as required";
+        case EFLA_ERR_TOO_LARGE: return "sizes exceed the fixed scratch of efla_chunk_fwd_noalloc";
         default: return "unknown status";
     }
 }

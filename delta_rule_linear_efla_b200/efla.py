@@ -22,7 +22,7 @@ EFLA_F32, EFLA_BF16 = 0, 1
 ABI_SYMBOLS = (
     "efla_status_str", "efla_version", "efla_alpha", "efla_chunk_fwd_workspace_size",
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
-    "efla_kernel_launches",
+    "efla_kernel_launches", "efla_chunk_fwd_noalloc",
 )
 
 _lib = None
@@ -63,6 +63,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_chunk_fwd_path.argtypes = [i, i, i, i, i, i, i, i]
     L.efla_kernel_launches.restype = ctypes.c_ulonglong
     L.efla_kernel_launches.argtypes = []
+    L.efla_chunk_fwd_noalloc.restype = i
+    L.efla_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
     if path is None:
         _lib = L
     return L
@@ -164,6 +166,20 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
         _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
         B, H, L, dk, dv, int(chunk), code, o_code, ws_ptr, ws_bytes, _stream_handle(stream))
     _check(st, "efla_chunk_fwd")
+    return o, S_final
+
+
+def chunk_fwd_noalloc(q, k, v, beta, o, S_final=None, S0=None, chunk: int = 64, stream=None):
+    """chunk_fwd for callers that cannot allocate device memory: the caller passes every
+    output buffer and the library uses its own fixed scratch (efla_chunk_fwd_noalloc)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    st = load_library().efla_chunk_fwd_noalloc(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
+        _dev(S0, "S0", torch.float32) if S0 is not None else None, _dev(o, "o"),
+        _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
+        B, H, L, dk, dv, int(chunk), _dtype_code(q), _dtype_code(o), _stream_handle(stream))
+    _check(st, "efla_chunk_fwd_noalloc")
     return o, S_final
 
 

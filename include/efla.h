@@ -60,7 +60,8 @@ typedef enum {
     EFLA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
     EFLA_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
     EFLA_ERR_WORKSPACE = 7,   /* workspace missing or smaller than the query said */
-    EFLA_ERR_ALIGN = 8        /* a pointer is not aligned as required */
+    EFLA_ERR_ALIGN = 8,       /* a pointer is not aligned as required */
+    EFLA_ERR_TOO_LARGE = 9    /* sizes need more than the fixed scratch of efla_chunk_fwd_noalloc */
 } efla_status;
 
 typedef enum {
@@ -119,6 +120,46 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
                            int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
                            efla_dtype o_dt, void *workspace, size_t workspace_bytes,
                            void *stream);
+
+/*
+ * efla_chunk_fwd_noalloc -- the same forward pass as efla_chunk_fwd for callers
+ * that cannot allocate device memory.  The paper has no counterpart: this is
+ * an interface for embedding, not part of the method.
+ *
+ * Who cannot allocate: code that is handed only its input and output buffers,
+ * with no allocator and no workspace (for example an operator plugin inside a
+ * runtime whose memory pool owns all device memory), and latency-critical
+ * loops that must not call cudaMalloc, which can synchronise the device and
+ * can fail at run time when memory is short.  Such callers cannot provide the
+ * workspace efla_chunk_fwd asks for.
+ *
+ * Scratch: instead of a caller workspace, the tensor-core path keeps its
+ * per-chunk T*diag(alpha) tiles (8 KiB per 64-token chunk of each head) in one
+ * fixed array of EFLA_NOALLOC_SCRATCH_BYTES inside the library's device code.
+ * Every GPU on which the library's kernels are loaded holds that memory until
+ * the process exits.  Sizes that need more -- B*H*ceil(L/64) > 4096 chunks on
+ * the tensor-core path -- return EFLA_ERR_TOO_LARGE before anything is
+ * enqueued.  Sizes served by the SIMT path need no scratch at all.
+ *
+ * Set-up: the first call on a device looks up the array's device address once
+ * for that device (it must be the current device); make that first call before
+ * any stream capture.
+ *
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents.  Nothing in it has to start at zero: each call writes every byte it
+ * later reads.  Calls whose GPU work overlaps (different streams with no
+ * ordering between them, on the same device) race on the array and give wrong
+ * results; order them.
+ *
+ * Arguments, layouts, sizes and the remaining errors are those of
+ * efla_chunk_fwd.  Allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library call.
+ */
+#define EFLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+efla_status efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *beta,
+                                   const float *S0, void *o, float *S_final,
+                                   int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                                   efla_dtype o_dt, void *stream);
 
 /*
  * efla_recurrent_step -- one decode token per head: the update rule of
