@@ -280,9 +280,9 @@ struct StateLayout {
     static constexpr int OFF_WT = 2 * STAGE;         // W^T, MN-major B operand [DK x C]
     static constexpr int OFF_P = OFF_WT + DK * 128;  // P, K-major B operand [C x C]
     static constexpr int OFF_UP = OFF_P + TB;        // U'^T, K-major A operand [DV x C]
-    static constexpr int OFF_S = OFF_UP + DV * 128;  // S^T, K-major A operand [DV x DK]
+    static constexpr int OFF_S = OFF_UP + DV * 128;  // S^T, K-major A operand [DV x DK], 2 slots
     static constexpr int S_SLAB = DV * 128;          // bytes per 64-column slab of S^T
-    static constexpr int BYTES = OFF_S + DV * DK * 2;
+    static constexpr int BYTES = OFF_S + 2 * DV * DK * 2;
     static constexpr int SMEM = BYTES + 1024;        // alignment slack
 };
 
@@ -307,8 +307,28 @@ __device__ __forceinline__ void store_row_f16(uint8_t *tile, int row, int ch0, c
     *reinterpret_cast<uint4 *>(tile + tc::sw128_off(row, ch0 + 1)) = u1;
 }
 
+// Warp roles of the state kernel.  Three warpgroups (one warp per TMEM lane
+// quarter each) plus two single-thread roles:
+//   warps 0-3   converter: bf16 -> fp16 in place for the Q, K, V tiles of a stage
+//   warps 4-7   side:      W^T and P from TMEM to fp16 operand tiles; O^T to global
+//   warps 8-11  chain:     U'^T = U^T - X^T and the fp16 copy of the new state
+//   warp 12     MMA issuer (one thread)
+//   warp 13     TMA producer (one thread)
+// Hand-offs are mbarriers (arrive count 1; a warpgroup arrives through one thread
+// after a named barrier).  Every wait is bounded and also ends when any role has
+// flagged an abort.
+constexpr int ST_WARPS = 14;
+constexpr int ST_THREADS = ST_WARPS * 32;
+constexpr int W_ISSUE = 12, W_PROD = 13;
+
+struct StateBars {
+    uint64_t full[2], conv[2], freeb[2];
+    uint64_t wdone, pdone, xdone, sdone, odone, drain;
+    uint64_t wt_ready, p_ready, o_free, up_ready, s_ready;
+};
+
 template <int DK, int DV, typename TO>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
@@ -318,16 +338,18 @@ __global__ void __launch_bounds__(THREADS)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    __shared__ uint64_t full[2], mma_bar;
+    __shared__ StateBars bars;
     __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = warp >> 2, gtid = tid & 127;  // warpgroup and thread within it
     const int bh = blockIdx.x;
     if (tid == 0) {
-        tc::mbar_init(&full[0], 1);
-        tc::mbar_init(&full[1], 1);
-        tc::mbar_init(&mma_bar, 1);
+        uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
+        for (int i = 0; i < (int)(sizeof(StateBars) / sizeof(uint64_t)); ++i) tc::mbar_init(b + i, 1);
         tc::fence_mbar_init();
+        abort_flag = 0;
         tc::tma_prefetch_desc(&tmap_q);
         tc::tma_prefetch_desc(&tmap_k);
         tc::tma_prefetch_desc(&tmap_v);
@@ -340,19 +362,15 @@ __global__ void __launch_bounds__(THREADS)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t sb = tc::smem_u32(base);
-    auto st_q = [&](int s) { return sb + s * Lay::STAGE; };
-    auto st_k = [&](int s) { return sb + s * Lay::STAGE + Lay::QB; };
-    auto st_v = [&](int s) { return sb + s * Lay::STAGE + 2 * Lay::QB; };
-    auto st_t = [&](int s) { return sb + s * Lay::STAGE + 2 * Lay::QB + Lay::VB; };
-    const uint32_t wt_s = sb + Lay::OFF_WT, p_s = sb + Lay::OFF_P, up_s = sb + Lay::OFF_UP,
-                   s_s = sb + Lay::OFF_S;
-    const int vrow = acc_row<DV>(warp, lane);  // state column v owned by this thread
+    const uint32_t wt_s = sb + Lay::OFF_WT, p_s = sb + Lay::OFF_P, up_s = sb + Lay::OFF_UP;
+    auto s16 = [&](int slot) { return sb + Lay::OFF_S + slot * (DV * DK * 2); };
+    uint8_t *s16p[2] = {base + Lay::OFF_S, base + Lay::OFF_S + DV * DK * 2};
+    const int vrow = acc_row<DV>(warp & 3, lane);  // state column v of this thread's TMEM lane
 
-    // ---- initial state: S^T into TMEM (fp32) and its fp16 operand copy
-    {
-        uint8_t *stile = base + Lay::OFF_S;
+    // ---- initial state (chain warpgroup): S^T into TMEM and its fp16 copy (slot 0)
+    if (wg == 2) {
 #pragma unroll
         for (int cb = 0; cb < DK / 16; ++cb) {
             float v[16];
@@ -360,95 +378,162 @@ __global__ void __launch_bounds__(THREADS)
             for (int j = 0; j < 16; ++j)
                 v[j] = (S0 && vrow >= 0) ? S0[((size_t)bh * DK + cb * 16 + j) * DV + vrow] : 0.f;
             if (S0) tc::tmem_st16(tmem + lane_base + TM_S + cb * 16, v);
-            if (vrow >= 0) store_row_f16(stile + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
+            if (vrow >= 0) store_row_f16(s16p[0] + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
         }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
     }
-    tc::fence_async_smem();
-    tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
 
-    bool issued[2] = {false, false};
-    auto issue = [&](int stage, int n) {
-        uint64_t *bar = &full[stage];
-        tc::mbar_expect_tx(bar, Lay::STAGE);
-        uint8_t *q = base + stage * Lay::STAGE;
+    const long long budget = WAIT_BUDGET;
+    if (warp == W_PROD) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int last[2] = {-1, -1};
+            for (int n = 0; n < NC; ++n) {
+                const int st = n & 1;
+                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeb[st], ((n - 2) >> 1) & 1, &abort_flag, budget))
+                    break;
+                uint64_t *bar = &bars.full[st];
+                tc::mbar_expect_tx(bar, Lay::STAGE);
+                uint8_t *q = base + st * Lay::STAGE;
 #pragma unroll
-        for (int s = 0; s < DK / 64; ++s) {
-            tc::tma_load_3d(q + s * 8192, &tmap_q, bar, s * 64, n * C, bh);
-            tc::tma_load_3d(q + Lay::QB + s * 8192, &tmap_k, bar, s * 64, n * C, bh);
-        }
+                for (int s = 0; s < DK / 64; ++s) {
+                    tc::tma_load_3d(q + s * 8192, &tmap_q, bar, s * 64, n * C, bh);
+                    tc::tma_load_3d(q + Lay::QB + s * 8192, &tmap_k, bar, s * 64, n * C, bh);
+                }
 #pragma unroll
-        for (int s = 0; s < DV / 64; ++s)
-            tc::tma_load_3d(q + 2 * Lay::QB + s * 8192, &tmap_v, bar, s * 64, n * C, bh);
-        tc::tma_load_2d(q + 2 * Lay::QB + Lay::VB, &tmap_t, bar, 0, (bh * NC + n) * C);
-    };
-    if (tid == 0) {
-        for (int st = 0; st < 2 && st < NC; ++st) {
-            issue(st, st);
-            issued[st] = true;
+                for (int s = 0; s < DV / 64; ++s)
+                    tc::tma_load_3d(q + 2 * Lay::QB + s * 8192, &tmap_v, bar, s * 64, n * C, bh);
+                tc::tma_load_2d(q + 2 * Lay::QB + Lay::VB, &tmap_t, bar, 0, (bh * NC + n) * C);
+                last[st] = n;
+            }
+            if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
+                for (int st = 0; st < 2; ++st)
+                    if (last[st] >= 0) tc::mbar_wait(&bars.full[st], (last[st] >> 1) & 1, budget / 4);
+            }
         }
-    }
-
-    uint32_t mma_phase = 0;
-    bool aborted = false, mma_pending = false;
-    int n = 0;
-    for (; n < NC; ++n) {
-        const int st = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const int c0 = n * C;
-        bool ok = tc::mbar_wait(&full[st], ph, WAIT_BUDGET);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        // ---- bf16 -> fp16 in place for the Q, K, V tiles of this stage
-        {
+    } else if (warp == W_ISSUE) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_w = tc::idesc_f16(DK, 64, true, false);
+            constexpr uint32_t id_u = tc::idesc_f16(DV, 64, true, false);
+            constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);
+            constexpr uint32_t id_x = tc::idesc_f16(DV, 64, false, true);
+            constexpr uint32_t id_s = tc::idesc_f16(DV, DK, false, true);
+            constexpr uint32_t id_o = tc::idesc_f16(DV, 64, false, false);
+            bool issued_any = false;
+            for (int n = 0; n < NC; ++n) {
+                const int st = n & 1;
+                const uint32_t sq = sb + st * Lay::STAGE, sk = sq + Lay::QB, sv = sq + 2 * Lay::QB,
+                               stt = sv + Lay::VB;
+                const uint32_t cur = s16(n & 1);
+                if (!tc::mbar_wait_or_abort(&bars.conv[st], (n >> 1) & 1, &abort_flag, budget)) break;
+                tc::tc_fence_after();
+                issued_any = true;
+                // W^T = K^T Ta^T ; U^T = V^T Ta^T ; P = Q K^T
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_W, tc::sdesc(sk + kk * 2048, 8192, 1024),
+                                 tc::sdesc(stt + kk * 32, 16, 1024), id_w, kk > 0);
+                tc::mma_commit(&bars.wdone);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_U, tc::sdesc(sv + kk * 2048, 8192, 1024),
+                                 tc::sdesc(stt + kk * 32, 16, 1024), id_u, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    tc::mma_bf16(tmem + TM_P, tc::sdesc(sq + off, 16, 1024),
+                                 tc::sdesc(sk + off, 16, 1024), id_p, kk > 0);
+                }
+                tc::mma_commit(&bars.pdone);
+                // X^T = S^T W^T  (needs W^T(n) in smem and S_n in smem)
+                if (!tc::mbar_wait_or_abort(&bars.wt_ready, n & 1, &abort_flag, budget)) break;
+                if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    tc::mma_bf16(tmem + TM_X,
+                                 tc::sdesc(cur + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(wt_s + kk * 2048, 8192, 1024), id_x, kk > 0);
+                tc::mma_commit(&bars.xdone);
+                // O^T = S^T Q^T (first part; TMEM O must have been read out)
+                if (n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    tc::mma_bf16(tmem + TM_O,
+                                 tc::sdesc(cur + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(sq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
+                                 kk > 0);
+                // S^T += U'^T K
+                if (!tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget)) break;
+                tc::tc_fence_after();
+                const uint32_t acc0 = (n > 0 || S0) ? 1u : 0u;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_S, tc::sdesc(up_s + kk * 32, 16, 1024),
+                                 tc::sdesc(sk + kk * 2048, 8192, 1024), id_s, kk > 0 ? 1u : acc0);
+                tc::mma_commit(&bars.sdone);
+                // O^T += U'^T P^T
+                if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_O, tc::sdesc(up_s + kk * 32, 16, 1024),
+                                 tc::sdesc(p_s + kk * 32, 16, 1024), id_o, 1u);
+                tc::mma_commit(&bars.odone);
+                tc::mma_commit(&bars.freeb[st]);
+            }
+            if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
+                tc::mma_commit(&bars.drain);
+                tc::mbar_wait(&bars.drain, 0, budget / 4);
+            }
+        }
+    } else if (wg == 0) {
+        // ---------------------------------------------------------- converter
+        for (int n = 0; n < NC; ++n) {
+            const int st = n & 1;
+            const bool ok = tc::mbar_wait_or_abort(&bars.full[st], (n >> 1) & 1, &abort_flag, budget);
+            if (tc::named_bar_or(1, 128, !ok)) break;
             uint4 *t = reinterpret_cast<uint4 *>(base + st * Lay::STAGE);
             constexpr int N16 = (2 * Lay::QB + Lay::VB) / 16;
-            for (int i = tid; i < N16; i += THREADS) {
+#pragma unroll 4
+            for (int i = gtid; i < N16; i += 128) {
                 uint4 u = t[i];
                 u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
                 u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
                 t[i] = u;
             }
+            tc::fence_async_smem();
+            tc::named_bar_sync(1, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.conv[st]);
         }
-        tc::fence_async_smem();
-        __syncthreads();
-        // ---- group 1: W^T, U^T, P
-        if (tid == 0) {
-            issued[st] = false;
+    } else if (wg == 1) {
+        // ---------------------------------------------------------- side epilogue
+        const int drow = acc_row<DK>(warp & 3, lane);
+        const int prow = acc_row<64>(warp & 3, lane);
+        for (int n = 0; n < NC; ++n) {
+            const int c0 = n * C;
+            bool ok = tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(2, 128, !ok)) break;
             tc::tc_fence_after();
-            constexpr uint32_t id_w = tc::idesc_f16(DK, 64, true, false);
-            constexpr uint32_t id_u = tc::idesc_f16(DV, 64, true, false);
-            constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t b = tc::sdesc(st_t(st) + kk * 32, 16, 1024);
-                tc::mma_bf16(tmem + TM_W, tc::sdesc(st_k(st) + kk * 2048, 8192, 1024), b, id_w, kk > 0);
-                tc::mma_bf16(tmem + TM_U, tc::sdesc(st_v(st) + kk * 2048, 8192, 1024), b, id_u, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                tc::mma_bf16(tmem + TM_P, tc::sdesc(st_q(st) + off, 16, 1024),
-                             tc::sdesc(st_k(st) + off, 16, 1024), id_p, kk > 0);
-            }
-            tc::mma_commit(&mma_bar);
-        }
-        mma_pending = true;
-        ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc::tc_fence_after();
-        // ---- epilogue A: W^T -> fp16 MN-major tile; P -> masked fp16 K-major tile
-        {
-            const int drow = acc_row<DK>(warp, lane);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 float v[16];
                 tc::tmem_ld16(tmem + lane_base + TM_W + cb * 16, v);
                 if (drow >= 0) store_row_f16(base + Lay::OFF_WT, drow, 2 * cb, v);
             }
-            const int prow = acc_row<64>(warp, lane);
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::named_bar_sync(2, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.wt_ready);
+
+            ok = tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(2, 128, !ok)) break;
+            tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 float v[16];
@@ -460,76 +545,14 @@ __global__ void __launch_bounds__(THREADS)
                     store_row_f16(base + Lay::OFF_P, prow, 2 * cb, v);
                 }
             }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        // ---- group 2: X^T = S^T W^T
-        if (tid == 0) {
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::named_bar_sync(2, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.p_ready);
+
+            ok = tc::mbar_wait_or_abort(&bars.odone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(2, 128, !ok)) break;
             tc::tc_fence_after();
-            constexpr uint32_t id_x = tc::idesc_f16(DV, 64, false, true);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                tc::mma_bf16(tmem + TM_X,
-                             tc::sdesc(s_s + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
-                             tc::sdesc(wt_s + kk * 2048, 8192, 1024), id_x, kk > 0);
-            tc::mma_commit(&mma_bar);
-        }
-        mma_pending = true;
-        ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc::tc_fence_after();
-        // ---- epilogue B: U'^T = U^T - X^T -> fp16 K-major tile
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float u[16], x[16];
-            tc::tmem_ld16(tmem + lane_base + TM_U + cb * 16, u);
-            tc::tmem_ld16(tmem + lane_base + TM_X + cb * 16, x);
-            if (vrow >= 0) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) u[j] -= x[j];
-                store_row_f16(base + Lay::OFF_UP, vrow, 2 * cb, u);
-            }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        // ---- group 3: S^T += U'^T K ; O^T = S^T Q^T + U'^T P^T
-        if (tid == 0) {
-            tc::tc_fence_after();
-            constexpr uint32_t id_s = tc::idesc_f16(DV, DK, false, true);
-            constexpr uint32_t id_o = tc::idesc_f16(DV, 64, false, false);
-            const uint32_t acc0 = (n > 0 || S0) ? 1u : 0u;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::sdesc(up_s + kk * 32, 16, 1024),
-                             tc::sdesc(st_k(st) + kk * 2048, 8192, 1024), id_s, kk > 0 ? 1u : acc0);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                tc::mma_bf16(tmem + TM_O,
-                             tc::sdesc(s_s + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
-                             tc::sdesc(st_q(st) + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
-                             kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_O, tc::sdesc(up_s + kk * 32, 16, 1024),
-                             tc::sdesc(p_s + kk * 32, 16, 1024), id_o, 1u);
-            tc::mma_commit(&mma_bar);
-        }
-        mma_pending = true;
-        ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc::tc_fence_after();
-        if (tid == 0 && n + 2 < NC) {  // every read of this stage has completed
-            issue(st, n + 2);
-            issued[st] = true;
-        }
-        // ---- epilogue C: O^T -> global (coalesced along v), S^T -> fp16 operand copy
-        {
             const int cl = min(C, L - c0);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
@@ -542,43 +565,66 @@ __global__ void __launch_bounds__(THREADS)
                         if (cb * 16 + j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
                 }
             }
-            uint8_t *stile = base + Lay::OFF_S;
+            tc::tc_fence_before();
+            tc::named_bar_sync(2, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.o_free);
+        }
+    } else if (wg == 2) {
+        // ---------------------------------------------------------- chain epilogue
+        bool done_all = true;
+        for (int n = 0; n < NC; ++n) {
+            bool ok = tc::mbar_wait_or_abort(&bars.xdone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
+            tc::tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                float u[16], x[16];
+                tc::tmem_ld16(tmem + lane_base + TM_U + cb * 16, u);
+                tc::tmem_ld16(tmem + lane_base + TM_X + cb * 16, x);
+                if (vrow >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) u[j] -= x[j];
+                    store_row_f16(base + Lay::OFF_UP, vrow, 2 * cb, u);
+                }
+            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::named_bar_sync(3, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.up_ready);
+
+            ok = tc::mbar_wait_or_abort(&bars.sdone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
+            tc::tc_fence_after();
+            if (n + 1 < NC) {
+                uint8_t *stile = s16p[(n + 1) & 1];
+#pragma unroll
+                for (int cb = 0; cb < DK / 16; ++cb) {
+                    float v[16];
+                    tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
+                    if (vrow >= 0) store_row_f16(stile + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
+                }
+                tc::fence_async_smem();
+            }
+            tc::tc_fence_before();
+            tc::named_bar_sync(3, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.s_ready);
+        }
+        if (done_all && S_final) {
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {
                 float v[16];
                 tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
-                if (vrow >= 0) store_row_f16(stile + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
-            }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-    }
-    if (aborted) {
-        if (tid == 0) {
-            record_error(2u);
-            for (int st = 0; st < 2; ++st) {
-                if (!issued[st]) continue;
-                const int m = (n % 2 == st) ? n : n + 1;  // the outstanding chunk of stage st
-                tc::mbar_wait(&full[st], (m >> 1) & 1, WAIT_BUDGET / 4);
-            }
-            if (mma_pending) tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET / 4);
-        }
-        __syncthreads();
-    } else if (S_final) {
-        tc::tc_fence_after();
+                if (vrow >= 0) {
 #pragma unroll
-        for (int cb = 0; cb < DK / 16; ++cb) {
-            float v[16];
-            tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
-            if (vrow >= 0) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) S_final[((size_t)bh * DK + cb * 16 + j) * DV + vrow] = v[j];
+                    for (int j = 0; j < 16; ++j)
+                        S_final[((size_t)bh * DK + cb * 16 + j) * DV + vrow] = v[j];
+                }
             }
         }
     }
     tc::tc_fence_before();
     __syncthreads();
+    if (tid == 0 && abort_flag) record_error(2u);
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
@@ -652,7 +698,7 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
     e = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ssm);
     if (e != cudaSuccess) return e;
-    tc_state_kernel<DK, DV, TO><<<BH, THREADS, ssm, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC);
+    tc_state_kernel<DK, DV, TO><<<BH, ST_THREADS, ssm, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC);
     count_launches(2);
     return cudaGetLastError();
 }
