@@ -259,35 +259,39 @@ __global__ void __launch_bounds__(THREADS)
 }
 
 // ------------------------------------------------------------------ state
-// Transposed products so that the state and value dimensions are the MMA M
-// dimension (M = 128 runs the tensor core at its full rate):
-//   W^T  = K^T Ta^T              [DK x C]
-//   U^T  = V^T Ta^T              [DV x C]
-//   P    = Q K^T                 [C x C]   (masked to the lower triangle incl. diagonal)
-//   X^T  = S^T W^T               [DV x C]
-//   U'^T = U^T - X^T
-//   S^T += U'^T K                [DV x DK] (fp32 accumulator resident in TMEM)
-//   O^T  = S^T Q^T + U'^T P^T    [DV x C]
+// Products are arranged so that the state and value dimensions are the MMA M
+// dimension and so that every MMA is as wide (N) as the algebra allows; a
+// tcgen05.mma instruction costs about the same for every N up to 128, so
+// products that share an operand are fused into one wide instruction stream:
+//
+//   U'^T  = V^T Ta^T                   [DV x C]   prefill of the U' accumulator
+//   W     = Ta K                       [C x DK]
+//   P^T   = K Q^T                      [C x C]    masked to c_in <= c_out
+//   D1:  [O^T | U'^T] += S^T [Q | -W]^T           O^T from zero, U'^T = U^T - X^T
+//   D2:  [S^T | O^T]  += U'^T [K | P^T]           state update and intra-chunk output
+//
+// TMEM columns (fp32): S^T [0, DK), O^T [DK, DK+64), U'^T [DK+64, DK+128),
+// W [256, 256+DK), P^T [384, 448); [O^T | U'^T] and [S^T | O^T] are contiguous.
+// The A operands of D1 and D2 -- the fp16 copy of S^T and fp16 U'^T -- also live
+// in tensor memory (packed two per column: S^T at [448, 448+DK/2), U'^T over the
+// first 32 columns of its own fp32 accumulator), which keeps them out of shared
+// memory: with small N an MMA is bound by shared-memory bandwidth.
 // MMA operands are fp16 (the bf16 Q, K, V tiles are converted in place; fp16
 // holds every bf16 value of magnitude >= 2^-14 exactly and rounds the
 // intermediates 8x finer than bf16); accumulation is fp32.
 template <int DK, int DV>
 struct StateLayout {
-    static constexpr int QB = DK * C * 2;            // Q or K tile, DK/64 slabs of 8 KB
-    static constexpr int VB = DV * C * 2;            // V tile, DV/64 slabs
-    static constexpr int TB = C * C * 2;             // Ta tile
-    static constexpr int STAGE = 2 * QB + VB + TB;
-    static constexpr int OFF_WT = 2 * STAGE;         // W^T, MN-major B operand [DK x C]
-    static constexpr int OFF_P = OFF_WT + DK * 128;  // P, K-major B operand [C x C]
-    static constexpr int OFF_UP = OFF_P + TB;        // U'^T, K-major A operand [DV x C]
-    static constexpr int OFF_S = OFF_UP + DV * 128;  // S^T, K-major A operand [DV x DK], 2 slots
-    static constexpr int S_SLAB = DV * 128;          // bytes per 64-column slab of S^T
-    static constexpr int BYTES = OFF_S + 2 * DV * DK * 2;
-    static constexpr int SMEM = BYTES + 1024;        // alignment slack
+    static constexpr int QW_SLAB = 16384;                // per 64-column K slab: 64 Q rows, 64 -W rows
+    static constexpr int QW = (DK / 64) * QW_SLAB;
+    static constexpr int KP = (DK / 64 + 1) * 8192;       // K slabs then the P^T block (MN-major)
+    static constexpr int VB = (DV / 64) * 8192;
+    static constexpr int TB = C * C * 2;
+    static constexpr int OFF_QW = 0, OFF_KP = QW, OFF_V = QW + KP, OFF_T = QW + KP + VB;
+    static constexpr int STAGE = OFF_T + TB;
+    static constexpr int TX = DK * 128 * 2 + VB + TB;     // bytes the TMA delivers per stage
+    static constexpr int BYTES = 2 * STAGE;
+    static constexpr int SMEM = BYTES + 1024;             // alignment slack
 };
-
-// TMEM columns (fp32): S^T [0, DK), W^T, U^T, X^T, P, O^T 64 each.
-constexpr uint32_t TM_S = 0, TM_W = 128, TM_U = 192, TM_X = 256, TM_P = 320, TM_O = 384;
 
 // Row of an M-row accumulator held by this thread, or -1: M = 128 puts row r in
 // lane r; M = 64 puts row r in lane (r % 16) + 32 (r / 16).
@@ -297,34 +301,41 @@ __device__ __forceinline__ int acc_row(int warp, int lane) {
     else return lane < 16 ? 16 * warp + lane : -1;
 }
 
-__device__ __forceinline__ void store_row_f16(uint8_t *tile, int row, int ch0, const float (&v)[16]) {
-    uint4 u0, u1;
-    u0.x = tc::pack_f16(v[0], v[1]);   u0.y = tc::pack_f16(v[2], v[3]);
-    u0.z = tc::pack_f16(v[4], v[5]);   u0.w = tc::pack_f16(v[6], v[7]);
-    u1.x = tc::pack_f16(v[8], v[9]);   u1.y = tc::pack_f16(v[10], v[11]);
-    u1.z = tc::pack_f16(v[12], v[13]); u1.w = tc::pack_f16(v[14], v[15]);
-    *reinterpret_cast<uint4 *>(tile + tc::sw128_off(row, ch0)) = u0;
-    *reinterpret_cast<uint4 *>(tile + tc::sw128_off(row, ch0 + 1)) = u1;
+__device__ __forceinline__ void store_row_f16x32(uint8_t *tile, int row, int ch0, const float (&v)[32]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = tc::pack_f16(v[8 * c + 0], v[8 * c + 1]); u.y = tc::pack_f16(v[8 * c + 2], v[8 * c + 3]);
+        u.z = tc::pack_f16(v[8 * c + 4], v[8 * c + 5]); u.w = tc::pack_f16(v[8 * c + 6], v[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + tc::sw128_off(row, ch0 + c)) = u;
+    }
 }
 
-// Warp roles of the state kernel.  Three warpgroups (one warp per TMEM lane
-// quarter each) plus two single-thread roles:
+// Warp roles.  Four warpgroups (one warp per TMEM lane quarter each) plus two
+// single-thread roles; hand-offs are mbarriers (arrive count 1; a warpgroup
+// arrives through one thread after a named barrier).  Every wait is bounded and
+// also ends as soon as any role has flagged an abort.
 //   warps 0-3   converter: bf16 -> fp16 in place for the Q, K, V tiles of a stage
-//   warps 4-7   side:      W^T and P from TMEM to fp16 operand tiles; O^T to global
-//   warps 8-11  chain:     U'^T = U^T - X^T and the fp16 copy of the new state
-//   warp 12     MMA issuer (one thread)
-//   warp 13     TMA producer (one thread)
-// Hand-offs are mbarriers (arrive count 1; a warpgroup arrives through one thread
-// after a named barrier).  Every wait is bounded and also ends when any role has
-// flagged an abort.
-constexpr int ST_WARPS = 14;
+//   warps 4-7   side:      -W and the masked P^T from TMEM into the B operand tiles
+//   warps 8-11  chain:     U'^T and the new state from TMEM into the A operand tiles
+//   warps 12-15 output:    O^T from TMEM to global memory, then zero it for the next chunk
+//   warp 16     MMA issuer (one thread)
+//   warp 17     TMA producer (one thread)
+constexpr int ST_WARPS = 18;
 constexpr int ST_THREADS = ST_WARPS * 32;
-constexpr int W_ISSUE = 12, W_PROD = 13;
+constexpr int W_ISSUE = 16, W_PROD = 17;
+constexpr uint32_t TM_W = 256, TM_P = 384, TM_S16 = 448;
+
+// Pack 32 fp32 values into 16 words of fp16 pairs (element 2j in the low half).
+__device__ __forceinline__ void pack32_f16(const float (&v)[32], uint32_t (&w)[16]) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+}
 
 struct StateBars {
     uint64_t full[2], conv[2], freeb[2];
-    uint64_t wdone, pdone, xdone, sdone, odone, drain;
-    uint64_t wt_ready, p_ready, o_free, up_ready, s_ready;
+    uint64_t wpdone, d1done, d2done, drain;
+    uint64_t side_ready, up_ready, s_ready, o_free;
 };
 
 template <int DK, int DV, typename TO>
@@ -335,6 +346,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC) {
     using Lay = StateLayout<DK, DV>;
+    constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     __shared__ volatile int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = warp >> 2, gtid = tid & 127;  // warpgroup and thread within it
+    const int wg = warp >> 2, gtid = tid & 127;
     const int bh = blockIdx.x;
     if (tid == 0) {
         uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
@@ -364,23 +376,30 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     const uint32_t tmem = tmem_base;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t sb = tc::smem_u32(base);
-    const uint32_t wt_s = sb + Lay::OFF_WT, p_s = sb + Lay::OFF_P, up_s = sb + Lay::OFF_UP;
-    auto s16 = [&](int slot) { return sb + Lay::OFF_S + slot * (DV * DK * 2); };
-    uint8_t *s16p[2] = {base + Lay::OFF_S, base + Lay::OFF_S + DV * DK * 2};
     const int vrow = acc_row<DV>(warp & 3, lane);  // state column v of this thread's TMEM lane
 
-    // ---- initial state (chain warpgroup): S^T into TMEM and its fp16 copy (slot 0)
+    // ---- initial state (chain warpgroup): S^T, its fp16 copy and a zero O^T in TMEM
     if (wg == 2) {
 #pragma unroll
-        for (int cb = 0; cb < DK / 16; ++cb) {
-            float v[16];
+        for (int cb = 0; cb < DK / 32; ++cb) {
+            float v[32];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                v[j] = (S0 && vrow >= 0) ? S0[((size_t)bh * DK + cb * 16 + j) * DV + vrow] : 0.f;
-            if (S0) tc::tmem_st16(tmem + lane_base + TM_S + cb * 16, v);
-            if (vrow >= 0) store_row_f16(s16p[0] + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
+            for (int j = 0; j < 32; ++j)
+                v[j] = (S0 && vrow >= 0) ? S0[((size_t)bh * DK + cb * 32 + j) * DV + vrow] : 0.f;
+            float lo[16], hi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { lo[j] = v[j]; hi[j] = v[16 + j]; }
+            tc::tmem_st16(tmem + lane_base + TM_S + cb * 32, lo);
+            tc::tmem_st16(tmem + lane_base + TM_S + cb * 32 + 16, hi);
+            uint32_t w[16];
+            pack32_f16(v, w);
+            tc::tmem_st16u(tmem + lane_base + TM_S16 + cb * 16, w);
         }
-        tc::fence_async_smem();
+        float z[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) z[j] = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
         tc::tc_fence_before();
     }
     __syncthreads();
@@ -396,17 +415,17 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeb[st], ((n - 2) >> 1) & 1, &abort_flag, budget))
                     break;
                 uint64_t *bar = &bars.full[st];
-                tc::mbar_expect_tx(bar, Lay::STAGE);
-                uint8_t *q = base + st * Lay::STAGE;
+                tc::mbar_expect_tx(bar, Lay::TX);
+                uint8_t *stg = base + st * Lay::STAGE;
 #pragma unroll
-                for (int s = 0; s < DK / 64; ++s) {
-                    tc::tma_load_3d(q + s * 8192, &tmap_q, bar, s * 64, n * C, bh);
-                    tc::tma_load_3d(q + Lay::QB + s * 8192, &tmap_k, bar, s * 64, n * C, bh);
+                for (int j = 0; j < DK / 64; ++j) {
+                    tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, bar, j * 64, n * C, bh);
+                    tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, bar, j * 64, n * C, bh);
                 }
 #pragma unroll
-                for (int s = 0; s < DV / 64; ++s)
-                    tc::tma_load_3d(q + 2 * Lay::QB + s * 8192, &tmap_v, bar, s * 64, n * C, bh);
-                tc::tma_load_2d(q + 2 * Lay::QB + Lay::VB, &tmap_t, bar, 0, (bh * NC + n) * C);
+                for (int j = 0; j < DV / 64; ++j)
+                    tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, bar, j * 64, n * C, bh);
+                tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, bar, 0, (bh * NC + n) * C);
                 last[st] = n;
             }
             if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
@@ -417,75 +436,74 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     } else if (warp == W_ISSUE) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t id_w = tc::idesc_f16(DK, 64, true, false);
             constexpr uint32_t id_u = tc::idesc_f16(DV, 64, true, false);
+            constexpr uint32_t id_w = tc::idesc_f16(64, DK, false, true);
             constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);
-            constexpr uint32_t id_x = tc::idesc_f16(DV, 64, false, true);
-            constexpr uint32_t id_s = tc::idesc_f16(DV, DK, false, true);
-            constexpr uint32_t id_o = tc::idesc_f16(DV, 64, false, false);
-            bool issued_any = false;
-            for (int n = 0; n < NC; ++n) {
-                const int st = n & 1;
-                const uint32_t sq = sb + st * Lay::STAGE, sk = sq + Lay::QB, sv = sq + 2 * Lay::QB,
-                               stt = sv + Lay::VB;
-                const uint32_t cur = s16(n & 1);
-                if (!tc::mbar_wait_or_abort(&bars.conv[st], (n >> 1) & 1, &abort_flag, budget)) break;
-                tc::tc_fence_after();
-                issued_any = true;
-                // W^T = K^T Ta^T ; U^T = V^T Ta^T ; P = Q K^T
+            constexpr uint32_t id_d1 = tc::idesc_f16(DV, 128, false, false);
+            constexpr uint32_t id_d2 = tc::idesc_f16(DV, DK + 64, false, true);
+            auto stage_addr = [&](int n) { return sb + (n & 1) * Lay::STAGE; };
+            // U'^T := V^T Ta^T (prefill of the U' accumulator)
+            auto issue_u = [&](int n) {
+                const uint32_t stg = stage_addr(n);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + TM_W, tc::sdesc(sk + kk * 2048, 8192, 1024),
-                                 tc::sdesc(stt + kk * 32, 16, 1024), id_w, kk > 0);
-                tc::mma_commit(&bars.wdone);
+                    tc::mma_bf16(tmem + TM_U, tc::sdesc(stg + Lay::OFF_V + kk * 2048, 8192, 1024),
+                                 tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024), id_u, kk > 0);
+            };
+            // W = Ta K ; P^T = K Q^T  (into their own TMEM columns, read out by the side group)
+            auto issue_wp = [&](int n) {
+                const uint32_t stg = stage_addr(n);
+                const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + TM_U, tc::sdesc(sv + kk * 2048, 8192, 1024),
-                                 tc::sdesc(stt + kk * 32, 16, 1024), id_u, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    tc::mma_bf16(tmem + TM_P, tc::sdesc(sq + off, 16, 1024),
-                                 tc::sdesc(sk + off, 16, 1024), id_p, kk > 0);
-                }
-                tc::mma_commit(&bars.pdone);
-                // X^T = S^T W^T  (needs W^T(n) in smem and S_n in smem)
-                if (!tc::mbar_wait_or_abort(&bars.wt_ready, n & 1, &abort_flag, budget)) break;
-                if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget)) break;
-                tc::tc_fence_after();
+                    tc::mma_bf16(tmem + TM_W, tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024),
+                                 tc::sdesc(kp + kk * 2048, 8192, 1024), id_w, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    tc::mma_bf16(tmem + TM_X,
-                                 tc::sdesc(cur + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc(wt_s + kk * 2048, 8192, 1024), id_x, kk > 0);
-                tc::mma_commit(&bars.xdone);
-                // O^T = S^T Q^T (first part; TMEM O must have been read out)
+                    tc::mma_bf16(tmem + TM_P, tc::sdesc(kp + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
+                                 id_p, kk > 0);
+                tc::mma_commit(&bars.wpdone);
+            };
+            bool issued_any = false;
+            bool ok = tc::mbar_wait_or_abort(&bars.conv[0], 0, &abort_flag, budget);
+            if (ok) {
+                tc::tc_fence_after();
+                issued_any = true;
+                issue_u(0);
+                issue_wp(0);
+            }
+            for (int n = 0; ok && n < NC; ++n) {
+                const int st = n & 1;
+                const uint32_t stg = stage_addr(n);
+                const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
+                // D1: [O^T | U'^T] += S^T [Q | -W]^T   (A = fp16 S^T in TMEM)
+                if (!tc::mbar_wait_or_abort(&bars.side_ready, n & 1, &abort_flag, budget)) break;
+                if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget)) break;
                 if (n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    tc::mma_bf16(tmem + TM_O,
-                                 tc::sdesc(cur + (kk >> 2) * Lay::S_SLAB + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc(sq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
-                                 kk > 0);
-                // S^T += U'^T K
+                    tc::mma_tmem_a(tmem + TM_O, tmem + TM_S16 + kk * 8,
+                                   tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
+                                   id_d1, 1u);
+                tc::mma_commit(&bars.d1done);
+                // D2: [S^T | O^T] += U'^T [K | P^T]   (A = fp16 U'^T in TMEM)
                 if (!tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
-                const uint32_t acc0 = (n > 0 || S0) ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + TM_S, tc::sdesc(up_s + kk * 32, 16, 1024),
-                                 tc::sdesc(sk + kk * 2048, 8192, 1024), id_s, kk > 0 ? 1u : acc0);
-                tc::mma_commit(&bars.sdone);
-                // O^T += U'^T P^T
-                if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
-                tc::tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + TM_O, tc::sdesc(up_s + kk * 32, 16, 1024),
-                                 tc::sdesc(p_s + kk * 32, 16, 1024), id_o, 1u);
-                tc::mma_commit(&bars.odone);
+                    tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
+                                   tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
+                tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeb[st]);
+                // next chunk's products while this chunk's epilogues run
+                if (n + 1 < NC) {
+                    if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) break;
+                    tc::tc_fence_after();
+                    issue_wp(n + 1);
+                    issue_u(n + 1);
+                }
             }
             if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
                 tc::mma_commit(&bars.drain);
@@ -498,14 +516,27 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             const int st = n & 1;
             const bool ok = tc::mbar_wait_or_abort(&bars.full[st], (n >> 1) & 1, &abort_flag, budget);
             if (tc::named_bar_or(1, 128, !ok)) break;
-            uint4 *t = reinterpret_cast<uint4 *>(base + st * Lay::STAGE);
-            constexpr int N16 = (2 * Lay::QB + Lay::VB) / 16;
-#pragma unroll 4
-            for (int i = gtid; i < N16; i += 128) {
-                uint4 u = t[i];
+            uint8_t *stg = base + st * Lay::STAGE;
+            auto cvt = [](uint4 *t) {
+                uint4 u = *t;
                 u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
                 u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-                t[i] = u;
+                *t = u;
+            };
+            // Q: first 8 KB of each QW slab; K: the DK/64 K slabs; V: all V slabs
+#pragma unroll
+            for (int j = 0; j < DK / 64; ++j) {
+                uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
+#pragma unroll
+                for (int i = gtid; i < 512; i += 128) cvt(tq + i);
+            }
+            {
+                uint4 *tk = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
+#pragma unroll
+                for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
+                uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
+#pragma unroll
+                for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
             }
             tc::fence_async_smem();
             tc::named_bar_sync(1, 128);
@@ -513,97 +544,72 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         }
     } else if (wg == 1) {
         // ---------------------------------------------------------- side epilogue
-        const int drow = acc_row<DK>(warp & 3, lane);
-        const int prow = acc_row<64>(warp & 3, lane);
+        const int crow = acc_row<64>(warp & 3, lane);  // token row of the M = 64 accumulators
         for (int n = 0; n < NC; ++n) {
-            const int c0 = n * C;
-            bool ok = tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget);
+            const int st = n & 1;
+            uint8_t *stg = base + st * Lay::STAGE;
+            const bool ok = tc::mbar_wait_or_abort(&bars.wpdone, n & 1, &abort_flag, budget);
             if (tc::named_bar_or(2, 128, !ok)) break;
             tc::tc_fence_after();
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float v[16];
-                tc::tmem_ld16(tmem + lane_base + TM_W + cb * 16, v);
-                if (drow >= 0) store_row_f16(base + Lay::OFF_WT, drow, 2 * cb, v);
+            for (int cb = 0; cb < DK / 32; ++cb) {  // -W rows into rows 64.. of the QW slabs
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + TM_W + cb * 32, v);
+                if (crow >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = -v[j];
+                    store_row_f16x32(stg + Lay::OFF_QW + (cb >> 1) * Lay::QW_SLAB, 64 + crow, (cb & 1) * 4, v);
+                }
             }
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.wt_ready);
-
-            ok = tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(2, 128, !ok)) break;
-            tc::tc_fence_after();
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float v[16];
-                tc::tmem_ld16(tmem + lane_base + TM_P + cb * 16, v);
-                if (prow >= 0) {
+            for (int cb = 0; cb < 2; ++cb) {  // masked P^T (row c_in, column c_out >= c_in)
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + TM_P + cb * 32, v);
+                if (crow >= 0) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (cb * 16 + j > prow) v[j] = 0.f;
-                    store_row_f16(base + Lay::OFF_P, prow, 2 * cb, v);
+                    for (int j = 0; j < 32; ++j)
+                        if (cb * 32 + j < crow) v[j] = 0.f;
+                    store_row_f16x32(stg + Lay::OFF_KP + (DK / 64) * 8192, crow, cb * 4, v);
                 }
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
             tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.p_ready);
-
-            ok = tc::mbar_wait_or_abort(&bars.odone, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(2, 128, !ok)) break;
-            tc::tc_fence_after();
-            const int cl = min(C, L - c0);
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float v[16];
-                tc::tmem_ld16(tmem + lane_base + TM_O + cb * 16, v);
-                if (vrow >= 0) {
-                    TO *dst = o + ((size_t)bh * L + c0 + cb * 16) * DV + vrow;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (cb * 16 + j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
-                }
-            }
-            tc::tc_fence_before();
-            tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.o_free);
+            if (gtid == 0) tc::mbar_arrive(&bars.side_ready);
         }
     } else if (wg == 2) {
         // ---------------------------------------------------------- chain epilogue
         bool done_all = true;
         for (int n = 0; n < NC; ++n) {
-            bool ok = tc::mbar_wait_or_abort(&bars.xdone, n & 1, &abort_flag, budget);
+            bool ok = tc::mbar_wait_or_abort(&bars.d1done, n & 1, &abort_flag, budget);
             if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
             tc::tc_fence_after();
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float u[16], x[16];
-                tc::tmem_ld16(tmem + lane_base + TM_U + cb * 16, u);
-                tc::tmem_ld16(tmem + lane_base + TM_X + cb * 16, x);
-                if (vrow >= 0) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) u[j] -= x[j];
-                    store_row_f16(base + Lay::OFF_UP, vrow, 2 * cb, u);
-                }
+            {
+                float u0[32], u1[32];
+                tc::tmem_ld32(tmem + lane_base + TM_U, u0);
+                tc::tmem_ld32(tmem + lane_base + TM_U + 32, u1);
+                uint32_t w0[16], w1[16];
+                pack32_f16(u0, w0);
+                pack32_f16(u1, w1);
+                tc::tmem_st16u(tmem + lane_base + TM_U, w0);       // packed over its own fp32 columns
+                tc::tmem_st16u(tmem + lane_base + TM_U + 16, w1);
             }
-            tc::fence_async_smem();
             tc::tc_fence_before();
             tc::named_bar_sync(3, 128);
             if (gtid == 0) tc::mbar_arrive(&bars.up_ready);
 
-            ok = tc::mbar_wait_or_abort(&bars.sdone, n & 1, &abort_flag, budget);
+            ok = tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget);
             if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
             tc::tc_fence_after();
             if (n + 1 < NC) {
-                uint8_t *stile = s16p[(n + 1) & 1];
 #pragma unroll
-                for (int cb = 0; cb < DK / 16; ++cb) {
-                    float v[16];
-                    tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
-                    if (vrow >= 0) store_row_f16(stile + (cb >> 2) * Lay::S_SLAB, vrow, (cb & 3) * 2, v);
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    float v[32];
+                    tc::tmem_ld32(tmem + lane_base + TM_S + cb * 32, v);
+                    uint32_t w[16];
+                    pack32_f16(v, w);
+                    tc::tmem_st16u(tmem + lane_base + TM_S16 + cb * 16, w);
                 }
-                tc::fence_async_smem();
             }
             tc::tc_fence_before();
             tc::named_bar_sync(3, 128);
@@ -620,6 +626,34 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                         S_final[((size_t)bh * DK + cb * 16 + j) * DV + vrow] = v[j];
                 }
             }
+        }
+    } else if (wg == 3) {
+        // ---------------------------------------------------------- output
+        float z[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) z[j] = 0.f;
+        for (int n = 0; n < NC; ++n) {
+            const int c0 = n * C;
+            const bool ok = tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(4, 128, !ok)) break;
+            tc::tc_fence_after();
+            const int cl = min(C, L - c0);
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + TM_O + cb * 32, v);
+                if (vrow >= 0) {
+                    TO *dst = o + ((size_t)bh * L + c0 + cb * 32) * DV + vrow;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (cb * 32 + j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
+                }
+            }
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
+            tc::tc_fence_before();
+            tc::named_bar_sync(4, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.o_free);
         }
     }
     tc::tc_fence_before();
