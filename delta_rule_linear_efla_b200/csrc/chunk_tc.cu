@@ -46,78 +46,73 @@ constexpr long long WAIT_BUDGET = 2000000000LL;  // ~1 s of SM cycles
 __device__ __forceinline__ void record_error(unsigned code) { atomicOr(&g_tc_error, code); }
 
 // ------------------------------------------------------------------ prep
-struct PrepSmem {
-    static constexpr int A_STRIDE = C + 1;
+// One chunk at a time (all chunks in parallel across the grid):
+//   1. K arrives by TMA; a per row from the squared norm (fp32).
+//   2. Gram G = K K^T on the tensor cores (tcgen05, TMEM accumulator).
+//   3. A = strictly-lower(diag(a) G); T = (I + A)^{-1} by blocked forward
+//      substitution on 16x16 blocks: the diagonal blocks by fp32 substitution
+//      on CUDA cores, the off-diagonal blocks level by level as
+//        T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ
+//      with warp-level mma.sync (fp16 operands, fp32 accumulation).
+//   4. Ta = T diag(a), rounded to fp16, written to the workspace (64x64 per chunk).
+namespace prep {
+constexpr int LD16 = 72;   // fp16 row stride (halves) of the 64x64 operand tiles
+
+struct Smem {
     template <int DK>
     static constexpr int k_bytes() { return DK * C * 2; }
+    static constexpr int A16 = C * LD16 * 2;      // A, fp16, row-major
+    static constexpr int TD16 = 4 * 16 * 24 * 2;  // T's diagonal blocks, fp16, row-major (A operands)
+    static constexpr int T16T = C * LD16 * 2;     // T, fp16, transposed (B operands)
+    static constexpr int TA16 = C * LD16 * 2;     // T diag(a), fp16, row-major (the output tile)
+    static constexpr int ADIAG = C * 16 * 4;      // diagonal 16x16 blocks of A, fp32
+    static constexpr int RT = 4 * 16 * 24 * 2;    // per-warp 16x16 scratch (transposed R), fp16
+    template <int DK>
+    static constexpr int bytes() { return 2 * k_bytes<DK>() + A16 + TD16 + T16T + TA16 + ADIAG + RT + C * 4; }
 };
 
-// T = (I + A)^{-1} for the 64x64 strictly lower A (row stride 65), result in Ts.
-// Diagonal 16x16 blocks by forward substitution (one column per thread, in
-// registers), then the off-diagonal blocks level by level:
-//   T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ.
-__device__ __forceinline__ void unit_lower_inverse(const float *As, float *Ts, float *Rs, int tid) {
-    constexpr int S = PrepSmem::A_STRIDE;
-    for (int idx = tid; idx < C * C; idx += THREADS) Ts[(idx >> 6) * S + (idx & 63)] = 0.f;
-    __syncthreads();
-    if (tid < 64) {
-        const int b = tid >> 4, c = tid & 15;
-        const float *Ab = As + (16 * b) * S + 16 * b;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s = (i == c) ? 1.f : 0.f;
-#pragma unroll
-            for (int m = 0; m < i; ++m) s = fmaf(-Ab[i * S + m], x[m], s);
-            x[i] = s;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Ts[(16 * b + i) * S + 16 * b + c] = x[i];
-    }
-    __syncthreads();
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nblk = 4 - lvl;
-        for (int e = tid; e < nblk * 256; e += THREADS) {
-            const int J = e >> 8, I = J + lvl, r = (e >> 4) & 15, cc = e & 15;
-            float s = 0.f;
-            for (int K = J; K < I; ++K) {
-                const float *Ar = As + (16 * I + r) * S + 16 * K;
-                const float *Tc = Ts + (16 * K) * S + 16 * J + cc;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) s = fmaf(Ar[m], Tc[m * S], s);
-            }
-            Rs[J * 256 + r * 16 + cc] = s;
-        }
-        __syncthreads();
-        for (int e = tid; e < nblk * 256; e += THREADS) {
-            const int J = e >> 8, I = J + lvl, r = (e >> 4) & 15, cc = e & 15;
-            const float *Tr = Ts + (16 * I + r) * S + 16 * I;
-            float s = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) s = fmaf(Tr[m], Rs[J * 256 + m * 16 + cc], s);
-            Ts[(16 * I + r) * S + 16 * J + cc] = -s;
-        }
-        __syncthreads();
-    }
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// A fragment (16x16, row-major source with row stride ld halves) at (r0, k0).
+__device__ __forceinline__ void load_a(uint32_t (&a)[4], const __half *M, int ld, int r0, int k0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    a[0] = *reinterpret_cast<const uint32_t *>(M + (r0 + g) * ld + k0 + 2 * t);
+    a[1] = *reinterpret_cast<const uint32_t *>(M + (r0 + g + 8) * ld + k0 + 2 * t);
+    a[2] = *reinterpret_cast<const uint32_t *>(M + (r0 + g) * ld + k0 + 2 * t + 8);
+    a[3] = *reinterpret_cast<const uint32_t *>(M + (r0 + g + 8) * ld + k0 + 2 * t + 8);
+}
+// B fragment (16 x 8) of B[k][n], read from its transpose Bt[n][k] (row stride ld).
+__device__ __forceinline__ void load_b(uint32_t &b0, uint32_t &b1, const __half *Bt, int ld, int k0, int n0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    b0 = *reinterpret_cast<const uint32_t *>(Bt + (n0 + g) * ld + k0 + 2 * t);
+    b1 = *reinterpret_cast<const uint32_t *>(Bt + (n0 + g) * ld + k0 + 2 * t + 8);
+}
+}  // namespace prep
 
 template <int DK>
 __global__ void __launch_bounds__(THREADS)
     tc_prep_kernel(const __grid_constant__ CUtensorMap tmap_k, const __nv_bfloat16 *__restrict__ beta,
                    __half *__restrict__ ta_out, int L, int NC, int total) {
-    constexpr int KB = PrepSmem::k_bytes<DK>();
-    constexpr int S = PrepSmem::A_STRIDE;
+    using namespace prep;
+    constexpr int KB = Smem::k_bytes<DK>();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
     uint8_t *Kt[2] = {base, base + KB};
-    float *As = reinterpret_cast<float *>(base + 2 * KB);
-    float *Ts = As + C * S;
-    float *Rs = Ts + C * S;
-    float *al = Rs + 3 * 256;
+    __half *A16 = reinterpret_cast<__half *>(base + 2 * KB);
+    __half *TD16 = A16 + C * LD16;                   // [4][16][24]
+    __half *T16t = TD16 + 4 * 16 * 24;
+    __half *Ta16 = T16t + C * LD16;
+    float *Ad = reinterpret_cast<float *>(Ta16 + C * LD16);  // [64 rows][16]: A's diagonal blocks
+    __half *Rt = reinterpret_cast<__half *>(Ad + C * 16);
+    float *al = reinterpret_cast<float *>(Rt + 4 * 16 * 24);
     __shared__ uint64_t full[2], mma_bar;
     __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -125,7 +120,6 @@ __global__ void __launch_bounds__(THREADS)
         tc::mbar_init(&full[1], 1);
         tc::mbar_init(&mma_bar, 1);
         tc::fence_mbar_init();
-        abort_flag = 0;
         tc::tma_prefetch_desc(&tmap_k);
     }
     if (warp == 0) {
@@ -179,7 +173,7 @@ __global__ void __launch_bounds__(THREADS)
         // a per row: squared norm from the swizzled K tile, beta with a bounds check
         if (tid < C) {
             const int r = tid;
-            float s = 0.f;
+            float sq = 0.f;
 #pragma unroll
             for (int sl = 0; sl < DK / 64; ++sl) {
 #pragma unroll
@@ -189,20 +183,21 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = __bfloat1622float2(h[e]);
-                        s = fmaf(f.x, f.x, fmaf(f.y, f.y, s));
+                        sq = fmaf(f.x, f.x, fmaf(f.y, f.y, sq));
                     }
                 }
             }
             const float b = (c0 + r < L) ? __bfloat162float(beta[(size_t)bh * L + c0 + r]) : 0.f;
-            al[r] = alpha_from(s, b);
+            al[r] = alpha_from(sq, b);
         }
         ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = false;
         tc::tc_fence_after();
+        // ---- A = strictly-lower(diag(a) G): fp16 copy (all blocks), fp32 diagonal blocks
         {
-            const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 layout)
+            const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 accumulator layout)
             const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
@@ -211,36 +206,116 @@ __global__ void __launch_bounds__(THREADS)
                 if (lane < 16) {
                     const float ar = al[r];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int col = cb * 16 + j;
-                        As[r * S + col] = (col < r) ? ar * v[j] : 0.f;
+                    for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * v[j] : 0.f;
+                    uint4 *dst = reinterpret_cast<uint4 *>(A16 + r * LD16 + cb * 16);
+                    dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
+                                        tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
+                    dst[1] = make_uint4(tc::pack_f16(v[8], v[9]), tc::pack_f16(v[10], v[11]),
+                                        tc::pack_f16(v[12], v[13]), tc::pack_f16(v[14], v[15]));
+                    if (cb == (r >> 4)) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) Ad[r * 16 + j] = v[j];
                     }
                 }
             }
         }
         tc::tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0) {  // the K tile of this stage is free: prefetch two chunks ahead
             const int g2 = g + 2 * gridDim.x;
             if (g2 < total) {
                 issue(st, g2);
                 issued[st] = true;
             }
         }
-        unit_lower_inverse(As, Ts, Rs, tid);
+        // ---- diagonal blocks: column c of (I + A_bb)^{-1}, one column per thread
+        if (tid < 64) {
+            const int b = tid >> 4, c = tid & 15;
+            const float ac = al[16 * b + c];
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float *arow = Ad + (16 * b + i) * 16;
+                float s0 = (i == c) ? 1.f : 0.f, s1 = 0.f;  // two chains: half the dependent latency
+#pragma unroll
+                for (int m = 0; m + 1 < i; m += 2) {
+                    s0 = fmaf(-arow[m], x[m], s0);
+                    s1 = fmaf(-arow[m + 1], x[m + 1], s1);
+                }
+                if (i & 1) s0 = fmaf(-arow[i - 1], x[i - 1], s0);
+                x[i] = s0 + s1;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int row = 16 * b + i, col = 16 * b + c;
+                TD16[(b * 16 + i) * 24 + c] = __float2half_rn(x[i]);
+                T16t[col * LD16 + row] = __float2half_rn(x[i]);
+                Ta16[row * LD16 + col] = __float2half_rn(x[i] * ac);
+            }
+        } else {
+            // zero the strictly-upper 16x16 blocks of the output tile
+            for (int e = tid - 64; e < 6 * 128; e += 64) {
+                const int blk = e >> 7, w = e & 127;
+                const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int J = blk < 3 ? 1 + blk : (blk < 5 ? blk - 1 : 3);
+                *reinterpret_cast<uint32_t *>(Ta16 + (16 * I + (w >> 3)) * LD16 + 16 * J + 2 * (w & 7)) = 0u;
+            }
+        }
+        __syncthreads();
+        // ---- off-diagonal blocks, one 16x16 block per warp, level by level
+        for (int lvl = 1; lvl < 4; ++lvl) {
+            const int J = warp, I = J + lvl;
+            if (I < 4) {
+                float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int K = J; K < I; ++K) {
+                    uint32_t a[4];
+                    load_a(a, A16, LD16, 16 * I, 16 * K, lane);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        uint32_t b0, b1;
+                        load_b(b0, b1, T16t, LD16, 16 * K, 16 * J + 8 * nt, lane);
+                        mma16816(r[nt], a, b0, b1);
+                    }
+                }
+                // R -> fp16, transposed, into this warp's scratch
+                __half *rt = Rt + warp * 16 * 24;
+                const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int n0 = 8 * nt + 2 * tq;
+                    rt[(n0) * 24 + gq] = __float2half_rn(r[nt][0]);
+                    rt[(n0 + 1) * 24 + gq] = __float2half_rn(r[nt][1]);
+                    rt[(n0) * 24 + gq + 8] = __float2half_rn(r[nt][2]);
+                    rt[(n0 + 1) * 24 + gq + 8] = __float2half_rn(r[nt][3]);
+                }
+                __syncwarp();
+                uint32_t a[4];
+                load_a(a, TD16 + I * 16 * 24, 24, 0, 0, lane);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    uint32_t b0, b1;
+                    load_b(b0, b1, rt, 24, 0, 8 * nt, lane);
+                    mma16816(d, a, b0, b1);
+                    const int row = 16 * I + gq, col = 16 * J + 8 * nt + 2 * tq;
+                    const float a0 = al[col], a1 = al[col + 1];
+                    *reinterpret_cast<uint32_t *>(Ta16 + row * LD16 + col) = tc::pack_f16(-d[0] * a0, -d[1] * a1);
+                    *reinterpret_cast<uint32_t *>(Ta16 + (row + 8) * LD16 + col) = tc::pack_f16(-d[2] * a0, -d[3] * a1);
+                    T16t[col * LD16 + row] = __float2half_rn(-d[0]);
+                    T16t[(col + 1) * LD16 + row] = __float2half_rn(-d[1]);
+                    T16t[col * LD16 + row + 8] = __float2half_rn(-d[2]);
+                    T16t[(col + 1) * LD16 + row + 8] = __float2half_rn(-d[3]);
+                }
+            }
+            __syncthreads();
+        }
+        // ---- the assembled fp16 Ta tile -> workspace (row-major 64x64), 16-byte stores
         {
             const int i = tid >> 1, h = tid & 1;
             uint4 *dst = reinterpret_cast<uint4 *>(ta_out + ((size_t)g * C + i) * C + h * 32);
+            const uint4 *src = reinterpret_cast<const uint4 *>(Ta16 + i * LD16 + h * 32);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 u;
-                const int j0 = h * 32 + q4 * 8;
-                u.x = tc::pack_f16(Ts[i * S + j0 + 0] * al[j0 + 0], Ts[i * S + j0 + 1] * al[j0 + 1]);
-                u.y = tc::pack_f16(Ts[i * S + j0 + 2] * al[j0 + 2], Ts[i * S + j0 + 3] * al[j0 + 3]);
-                u.z = tc::pack_f16(Ts[i * S + j0 + 4] * al[j0 + 4], Ts[i * S + j0 + 5] * al[j0 + 5]);
-                u.w = tc::pack_f16(Ts[i * S + j0 + 6] * al[j0 + 6], Ts[i * S + j0 + 7] * al[j0 + 7]);
-                dst[q4] = u;
-            }
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = src[q4];
         }
         __syncthreads();
     }
@@ -706,7 +781,7 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint
 
 template <int DK>
 int prep_smem_bytes() {
-    return 2 * PrepSmem::k_bytes<DK>() + (2 * C * PrepSmem::A_STRIDE + 3 * 256 + C) * 4 + 1024;
+    return prep::Smem::bytes<DK>() + 1024;
 }
 
 template <int DK, int DV, typename TO>
@@ -723,7 +798,15 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
     cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<DK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
     if (e != cudaSuccess) return e;
-    const int pgrid = total < 148 * 3 ? total : 148 * 3;
+    cudaFuncSetAttribute(tc_prep_kernel<DK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int dev = 0, nsm = 148, smem_sm = 228 * 1024;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    }
+    int per_sm = smem_sm / (psm + 1024);  // 1 KiB per CTA is reserved by the system
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    const int pgrid = total < nsm * per_sm ? total : nsm * per_sm;
     tc_prep_kernel<DK><<<pgrid, THREADS, psm, s>>>(mk, (const __nv_bfloat16 *)beta, (__half *)ws,
                                                     L, NC, total);
     e = cudaGetLastError();
