@@ -363,7 +363,6 @@ struct StateLayout {
     static constexpr int TB = C * C * 2;
     static constexpr int OFF_QW = 0, OFF_KP = QW, OFF_V = QW + KP, OFF_T = QW + KP + VB;
     static constexpr int STAGE = OFF_T + TB;
-    static constexpr int TX = DK * 128 * 2 + VB + TB;     // bytes the TMA delivers per stage
     static constexpr int BYTES = 2 * STAGE;
     static constexpr int SMEM = BYTES + 1024;             // alignment slack
 };
@@ -407,10 +406,16 @@ __device__ __forceinline__ void pack32_f16(const float (&v)[32], uint32_t (&w)[1
     for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
 }
 
+// Each stage is three buffer groups with their own load and release barriers, so
+// every group is refilled as soon as its last reader is done:
+//   V and Ta  -- read by U'^T(n) and W(n)            released after U'^T(n)
+//   Q (+ -W)  -- read by P^T(n) and D1(n)            released after D1(n)
+//   K (+ P^T) -- read by W(n), P^T(n) and D2(n)      released after D2(n)
 struct StateBars {
-    uint64_t full[2], conv[2], freeb[2];
-    uint64_t wpdone, d1done, d2done, drain;
-    uint64_t side_ready, up_ready, s_ready, o_free;
+    uint64_t fullV[2], fullQ[2], fullK[2], conv[2];
+    uint64_t freeV[2], freeQ[2], freeK[2];
+    uint64_t wdone, pdone, d1done, d2done, drain;
+    uint64_t w_ready, p_ready, up_ready, s_ready, o_free;
 };
 
 template <int DK, int DV, typename TO>
@@ -487,25 +492,34 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             int last[2] = {-1, -1};
             for (int n = 0; n < NC; ++n) {
                 const int st = n & 1;
-                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeb[st], ((n - 2) >> 1) & 1, &abort_flag, budget))
-                    break;
-                uint64_t *bar = &bars.full[st];
-                tc::mbar_expect_tx(bar, Lay::TX);
+                const uint32_t par = ((n - 2) >> 1) & 1;
                 uint8_t *stg = base + st * Lay::STAGE;
-#pragma unroll
-                for (int j = 0; j < DK / 64; ++j) {
-                    tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, bar, j * 64, n * C, bh);
-                    tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, bar, j * 64, n * C, bh);
-                }
+                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeV[st], par, &abort_flag, budget)) break;
+                tc::mbar_expect_tx(&bars.fullV[st], Lay::VB + Lay::TB);
 #pragma unroll
                 for (int j = 0; j < DV / 64; ++j)
-                    tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, bar, j * 64, n * C, bh);
-                tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, bar, 0, (bh * NC + n) * C);
+                    tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
+                tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C);
+                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeQ[st], par, &abort_flag, budget)) break;
+                tc::mbar_expect_tx(&bars.fullQ[st], DK * 128);
+#pragma unroll
+                for (int j = 0; j < DK / 64; ++j)
+                    tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
+                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeK[st], par, &abort_flag, budget)) break;
+                tc::mbar_expect_tx(&bars.fullK[st], DK * 128);
+#pragma unroll
+                for (int j = 0; j < DK / 64; ++j)
+                    tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, &bars.fullK[st], j * 64, n * C, bh);
                 last[st] = n;
             }
             if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
-                for (int st = 0; st < 2; ++st)
-                    if (last[st] >= 0) tc::mbar_wait(&bars.full[st], (last[st] >> 1) & 1, budget / 4);
+                for (int st = 0; st < 2; ++st) {
+                    if (last[st] < 0) continue;
+                    const uint32_t par = (last[st] >> 1) & 1;
+                    tc::mbar_wait(&bars.fullV[st], par, budget / 8);
+                    tc::mbar_wait(&bars.fullQ[st], par, budget / 8);
+                    tc::mbar_wait(&bars.fullK[st], par, budget / 8);
+                }
             }
         }
     } else if (warp == W_ISSUE) {
@@ -524,36 +538,45 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_U, tc::sdesc(stg + Lay::OFF_V + kk * 2048, 8192, 1024),
                                  tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024), id_u, kk > 0);
+                tc::mma_commit(&bars.freeV[n & 1]);  // V and Ta of this stage are no longer read
             };
-            // W = Ta K ; P^T = K Q^T  (into their own TMEM columns, read out by the side group)
-            auto issue_wp = [&](int n) {
+            // W = Ta K (its own TMEM columns; the side group stores -W as a B operand)
+            auto issue_w = [&](int n) {
                 const uint32_t stg = stage_addr(n);
-                const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_W, tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024),
-                                 tc::sdesc(kp + kk * 2048, 8192, 1024), id_w, kk > 0);
+                                 tc::sdesc(stg + Lay::OFF_KP + kk * 2048, 8192, 1024), id_w, kk > 0);
+                tc::mma_commit(&bars.wdone);
+            };
+            // P^T = K Q^T (its own TMEM columns; the side group stores the masked P^T)
+            auto issue_p = [&](int n) {
+                const uint32_t stg = stage_addr(n);
+                const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
                     tc::mma_bf16(tmem + TM_P, tc::sdesc(kp + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
                                  tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
                                  id_p, kk > 0);
-                tc::mma_commit(&bars.wpdone);
+                tc::mma_commit(&bars.pdone);
             };
+            // Tensor-pipe order per chunk: D1(n), W(n+1), D2(n), P^T(n+1), U'^T(n+1), so the
+            // next chunk's products run while this chunk's epilogues do.
             bool issued_any = false;
             bool ok = tc::mbar_wait_or_abort(&bars.conv[0], 0, &abort_flag, budget);
             if (ok) {
                 tc::tc_fence_after();
                 issued_any = true;
+                issue_w(0);
+                issue_p(0);
                 issue_u(0);
-                issue_wp(0);
             }
             for (int n = 0; ok && n < NC; ++n) {
                 const int st = n & 1;
                 const uint32_t stg = stage_addr(n);
                 const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
                 // D1: [O^T | U'^T] += S^T [Q | -W]^T   (A = fp16 S^T in TMEM)
-                if (!tc::mbar_wait_or_abort(&bars.side_ready, n & 1, &abort_flag, budget)) break;
+                if (!tc::mbar_wait_or_abort(&bars.w_ready, n & 1, &abort_flag, budget)) break;
                 if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget)) break;
                 if (n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
@@ -563,20 +586,24 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                                    tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
                                    id_d1, 1u);
                 tc::mma_commit(&bars.d1done);
+                tc::mma_commit(&bars.freeQ[st]);
+                if (n + 1 < NC) {  // W of the next chunk (its TMEM was read out before D1(n))
+                    if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) break;
+                    tc::tc_fence_after();
+                    issue_w(n + 1);
+                }
                 // D2: [S^T | O^T] += U'^T [K | P^T]   (A = fp16 U'^T in TMEM)
                 if (!tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget)) break;
+                if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
                                    tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
                 tc::mma_commit(&bars.d2done);
-                tc::mma_commit(&bars.freeb[st]);
-                // next chunk's products while this chunk's epilogues run
-                if (n + 1 < NC) {
-                    if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) break;
-                    tc::tc_fence_after();
-                    issue_wp(n + 1);
+                tc::mma_commit(&bars.freeK[st]);
+                if (n + 1 < NC) {  // P^T and the U' prefill of the next chunk
+                    issue_p(n + 1);
                     issue_u(n + 1);
                 }
             }
@@ -587,31 +614,37 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         }
     } else if (wg == 0) {
         // ---------------------------------------------------------- converter
+        auto cvt = [](uint4 *t) {
+            uint4 u = *t;
+            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+            *t = u;
+        };
         for (int n = 0; n < NC; ++n) {
             const int st = n & 1;
-            const bool ok = tc::mbar_wait_or_abort(&bars.full[st], (n >> 1) & 1, &abort_flag, budget);
-            if (tc::named_bar_or(1, 128, !ok)) break;
+            const uint32_t par = (n >> 1) & 1;
             uint8_t *stg = base + st * Lay::STAGE;
-            auto cvt = [](uint4 *t) {
-                uint4 u = *t;
-                u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
-                u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-                *t = u;
-            };
-            // Q: first 8 KB of each QW slab; K: the DK/64 K slabs; V: all V slabs
+            bool ok = tc::mbar_wait_or_abort(&bars.fullV[st], par, &abort_flag, budget);
+            if (tc::named_bar_or(1, 128, !ok)) break;
+            {
+                uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
 #pragma unroll
-            for (int j = 0; j < DK / 64; ++j) {
+                for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
+            }
+            ok = tc::mbar_wait_or_abort(&bars.fullQ[st], par, &abort_flag, budget);
+            if (tc::named_bar_or(1, 128, !ok)) break;
+#pragma unroll
+            for (int j = 0; j < DK / 64; ++j) {  // Q: the first 8 KB of each QW slab
                 uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
 #pragma unroll
                 for (int i = gtid; i < 512; i += 128) cvt(tq + i);
             }
+            ok = tc::mbar_wait_or_abort(&bars.fullK[st], par, &abort_flag, budget);
+            if (tc::named_bar_or(1, 128, !ok)) break;
             {
                 uint4 *tk = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
 #pragma unroll
                 for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
-                uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
-#pragma unroll
-                for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
             }
             tc::fence_async_smem();
             tc::named_bar_sync(1, 128);
@@ -623,7 +656,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         for (int n = 0; n < NC; ++n) {
             const int st = n & 1;
             uint8_t *stg = base + st * Lay::STAGE;
-            const bool ok = tc::mbar_wait_or_abort(&bars.wpdone, n & 1, &abort_flag, budget);
+            bool ok = tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget);
             if (tc::named_bar_or(2, 128, !ok)) break;
             tc::tc_fence_after();
 #pragma unroll
@@ -636,6 +669,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     store_row_f16x32(stg + Lay::OFF_QW + (cb >> 1) * Lay::QW_SLAB, 64 + crow, (cb & 1) * 4, v);
                 }
             }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::named_bar_sync(2, 128);
+            if (gtid == 0) tc::mbar_arrive(&bars.w_ready);
+
+            ok = tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget);
+            if (tc::named_bar_or(2, 128, !ok)) break;
+            tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {  // masked P^T (row c_in, column c_out >= c_in)
                 float v[32];
@@ -650,7 +691,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             tc::fence_async_smem();
             tc::tc_fence_before();
             tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.side_ready);
+            if (gtid == 0) tc::mbar_arrive(&bars.p_ready);
         }
     } else if (wg == 2) {
         // ---------------------------------------------------------- chain epilogue
@@ -660,14 +701,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
             tc::tc_fence_after();
             {
-                float u0[32], u1[32];
-                tc::tmem_ld32(tmem + lane_base + TM_U, u0);
-                tc::tmem_ld32(tmem + lane_base + TM_U + 32, u1);
-                uint32_t w0[16], w1[16];
-                pack32_f16(u0, w0);
-                pack32_f16(u1, w1);
-                tc::tmem_st16u(tmem + lane_base + TM_U, w0);       // packed over its own fp32 columns
-                tc::tmem_st16u(tmem + lane_base + TM_U + 16, w1);
+                float u[64];
+                tc::tmem_ld64(tmem + lane_base + TM_U, u);
+                uint32_t w[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
+                tc::tmem_st32u(tmem + lane_base + TM_U, w);  // packed over its own fp32 columns
             }
             tc::tc_fence_before();
             tc::named_bar_sync(3, 128);
@@ -678,12 +717,13 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             tc::tc_fence_after();
             if (n + 1 < NC) {
 #pragma unroll
-                for (int cb = 0; cb < DK / 32; ++cb) {
-                    float v[32];
-                    tc::tmem_ld32(tmem + lane_base + TM_S + cb * 32, v);
-                    uint32_t w[16];
-                    pack32_f16(v, w);
-                    tc::tmem_st16u(tmem + lane_base + TM_S16 + cb * 16, w);
+                for (int cb = 0; cb < DK / 64; ++cb) {
+                    float v[64];
+                    tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
+                    uint32_t w[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+                    tc::tmem_st32u(tmem + lane_base + TM_S16 + cb * 32, w);
                 }
             }
             tc::tc_fence_before();
@@ -713,22 +753,19 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             if (tc::named_bar_or(4, 128, !ok)) break;
             tc::tc_fence_after();
             const int cl = min(C, L - c0);
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                float v[32];
-                tc::tmem_ld32(tmem + lane_base + TM_O + cb * 32, v);
-                if (vrow >= 0) {
-                    TO *dst = o + ((size_t)bh * L + c0 + cb * 32) * DV + vrow;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (cb * 32 + j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
-                }
-            }
+            float v[64];
+            tc::tmem_ld64(tmem + lane_base + TM_O, v);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
             tc::tc_fence_before();
             tc::named_bar_sync(4, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.o_free);
+            if (gtid == 0) tc::mbar_arrive(&bars.o_free);  // TMEM O is zero again: D1(n+1) may run
+            if (vrow >= 0) {
+                TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
+            }
         }
     }
     tc::tc_fence_before();
