@@ -68,7 +68,7 @@ struct Smem {
     static constexpr int ADIAG = C * 16 * 4;      // diagonal 16x16 blocks of A, fp32
     static constexpr int RT = 4 * 16 * 24 * 2;    // per-warp 16x16 scratch (transposed R), fp16
     template <int DK>
-    static constexpr int bytes() { return 2 * k_bytes<DK>() + A16 + TD16 + T16T + TA16 + ADIAG + RT + C * 4; }
+    static constexpr int bytes() { return k_bytes<DK>() + A16 + TD16 + T16T + TA16 + ADIAG + RT + C * 4; }
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -103,21 +103,20 @@ __global__ void __launch_bounds__(THREADS)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    uint8_t *Kt[2] = {base, base + KB};
-    __half *A16 = reinterpret_cast<__half *>(base + 2 * KB);
+    uint8_t *Kt = base;  // one K tile: refilled as soon as the Gram MMA and the norms have read it
+    __half *A16 = reinterpret_cast<__half *>(base + KB);
     __half *TD16 = A16 + C * LD16;                   // [4][16][24]
     __half *T16t = TD16 + 4 * 16 * 24;
     __half *Ta16 = T16t + C * LD16;
     float *Ad = reinterpret_cast<float *>(Ta16 + C * LD16);  // [64 rows][16]: A's diagonal blocks
     __half *Rt = reinterpret_cast<__half *>(Ad + C * 16);
     float *al = reinterpret_cast<float *>(Rt + 4 * 16 * 24);
-    __shared__ uint64_t full[2], mma_bar;
+    __shared__ uint64_t full, mma_bar;
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        tc::mbar_init(&full[0], 1);
-        tc::mbar_init(&full[1], 1);
+        tc::mbar_init(&full, 1);
         tc::mbar_init(&mma_bar, 1);
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_k);
@@ -129,38 +128,32 @@ __global__ void __launch_bounds__(THREADS)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_base;
-    bool issued[2] = {false, false};
+    bool issued = false;
 
-    auto issue = [&](int stage, int g) {
+    auto issue = [&](int g) {
         const int bh = g / NC, n = g - bh * NC;
-        tc::mbar_expect_tx(&full[stage], KB);
+        tc::mbar_expect_tx(&full, KB);
 #pragma unroll
         for (int s = 0; s < DK / 64; ++s)
-            tc::tma_load_3d(Kt[stage] + s * 8192, &tmap_k, &full[stage], s * 64, n * C, bh);
+            tc::tma_load_3d(Kt + s * 8192, &tmap_k, &full, s * 64, n * C, bh);
     };
-    if (tid == 0) {
-        for (int st = 0; st < 2; ++st) {
-            const int g = blockIdx.x + st * gridDim.x;
-            if (g < total) {
-                issue(st, g);
-                issued[st] = true;
-            }
-        }
+    if (tid == 0 && blockIdx.x < total) {
+        issue(blockIdx.x);
+        issued = true;
     }
     uint32_t mma_phase = 0;
     int it = 0;
     bool aborted = false;
     bool mma_pending = false;
     for (int g = blockIdx.x; g < total; g += gridDim.x, ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
+        const uint32_t ph = it & 1;
         const int bh = g / NC, n = g - bh * NC, c0 = n * C;
-        bool ok = tc::mbar_wait(&full[st], ph, WAIT_BUDGET);
+        bool ok = tc::mbar_wait(&full, ph, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         if (tid == 0) {
-            issued[st] = false;
+            issued = false;
             tc::tc_fence_after();
-            const uint32_t kb = tc::smem_u32(Kt[st]);
+            const uint32_t kb = tc::smem_u32(Kt);
             constexpr uint32_t id = tc::idesc_bf16(64, 64, false, false);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
@@ -178,7 +171,7 @@ __global__ void __launch_bounds__(THREADS)
             for (int sl = 0; sl < DK / 64; ++sl) {
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(Kt[st] + sl * 8192 + tc::sw128_off(r, ch));
+                    const uint4 u = *reinterpret_cast<const uint4 *>(Kt + sl * 8192 + tc::sw128_off(r, ch));
                     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -191,10 +184,14 @@ __global__ void __launch_bounds__(THREADS)
             al[r] = alpha_from(sq, b);
         }
         ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        if (__syncthreads_or(!ok)) { aborted = true; break; }  // also: every norm has been read
         mma_phase ^= 1;
         mma_pending = false;
         tc::tc_fence_after();
+        if (tid == 0 && g + (int)gridDim.x < total) {  // the K tile is free: fetch the next chunk
+            issue(g + gridDim.x);
+            issued = true;
+        }
         // ---- A = strictly-lower(diag(a) G): fp16 copy (all blocks), fp32 diagonal blocks
         {
             const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 accumulator layout)
@@ -221,13 +218,6 @@ __global__ void __launch_bounds__(THREADS)
         }
         tc::tc_fence_before();
         __syncthreads();
-        if (tid == 0) {  // the K tile of this stage is free: prefetch two chunks ahead
-            const int g2 = g + 2 * gridDim.x;
-            if (g2 < total) {
-                issue(st, g2);
-                issued[st] = true;
-            }
-        }
         // ---- diagonal blocks: column c of (I + A_bb)^{-1}, one column per thread
         if (tid < 64) {
             const int b = tid >> 4, c = tid & 15;
@@ -322,8 +312,7 @@ __global__ void __launch_bounds__(THREADS)
     if (aborted) {
         if (tid == 0) {
             record_error(1u);
-            for (int st = 0; st < 2; ++st)  // drain copies still in flight (bounded)
-                if (issued[st]) tc::mbar_wait(&full[st], ((it + (st != (it & 1))) >> 1) & 1, WAIT_BUDGET / 4);
+            if (issued) tc::mbar_wait(&full, it & 1, WAIT_BUDGET / 4);  // drain the copy in flight
             if (mma_pending) tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET / 4);
         }
         __syncthreads();
