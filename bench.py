@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
+from delta_rule_linear_efla_b200 import dist as edist  # noqa: E402
 from delta_rule_linear_efla_b200 import inputs  # noqa: E402
 
 METRIC = "EFLA fwd tokens/s per GPU (B*H*L/time) and % of binding roofline"
@@ -114,21 +115,36 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def _dist():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources the library is built from (ties profiled counters to a build)."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "delta_rule_linear_efla_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(os.path.basename(f).encode())
+            h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
 
 
-def _max_over_ranks(x: float, ws: int, device) -> float:
-    if ws == 1:
-        return x
-    import torch.distributed as dist
-
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+def profiled_traffic(w) -> int | None:
+    """DRAM bytes of one efla_chunk_fwd call from the committed ncu capture, if it was taken on
+    this workload and on the current kernel sources; None otherwise."""
+    if w.id != 4:
+        return None
+    p = os.path.join(ROOT, "profiles", "dram_traffic_lm1p3b.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        line = line.split("#")[0].strip()
+        if "=" in line:
+            k, v = (x.strip() for x in line.split("=", 1))
+            kv[k] = v
+    if kv.get("source_hash") != kernel_source_hash():
+        return None
+    return int(kv["chunk_fwd_bytes"])
 
 
 def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
@@ -159,7 +175,7 @@ def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
 
 def run_reference(args) -> None:
     """The oracle timed on host cores: each step is a bounded sample of the workload."""
-    ws, rank, _ = _dist()
+    ws, rank, _ = edist.world()
     if rank != 0:
         return
     import oracle
@@ -205,14 +221,10 @@ def _config(w) -> dict:
 def run_ours(args) -> None:
     from delta_rule_linear_efla_b200 import efla
 
-    ws, rank, local = _dist()
+    ws, rank, local = edist.world()
     if ws > 1:
-        import datetime
-
-        import torch.distributed as dist
-
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        edist.init("nccl", timeout_s=120)
     dev = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(dev)
     w = inputs.WORKLOADS[args.workload]
@@ -221,7 +233,7 @@ def run_ours(args) -> None:
     # ---- inputs: two rotating sets so consecutive steps do not hit in L2 ----
     sets = []
     for r in range(2):
-        x = inputs.make_inputs(w, seed=1000 + w.id + 7919 * (2 * rank + r))
+        x = inputs.make_inputs(w, seed=edist.replica_seed(1000 + w.id, rank, r))
         sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
     o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
     Sf_buf = [torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
@@ -232,7 +244,7 @@ def run_ours(args) -> None:
 
     dec = None
     if w.decode:
-        d = inputs.make_decode_inputs(w, seed=w.decode["seed"] + 7919 * rank)
+        d = inputs.make_decode_inputs(w, seed=edist.replica_seed(w.decode["seed"], rank))
         dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()
               if k != "prefix"}
         p = d["prefix"]
@@ -262,8 +274,7 @@ def run_ours(args) -> None:
     for i in range(max(3, args.warmup)):
         step(i)
     torch.cuda.synchronize(dev)
-    if ws > 1:
-        torch.distributed.barrier()
+    edist.barrier()
     torch.cuda.synchronize(dev)
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -279,24 +290,24 @@ def run_ours(args) -> None:
     torch.cuda.synchronize(dev)
     launches = efla.kernel_launches() - l0
     clocks = clk.stop()
-    if ws > 1:
-        torch.distributed.barrier()
+    edist.barrier()
     ms_local = t_start.elapsed_time(t_end)
-    ms = _max_over_ranks(ms_local, ws, dev)
+    ms = edist.max_over_ranks(ms_local, dev)
     chunk_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    chunk_ms = _max_over_ranks(chunk_ms, ws, dev)
+    chunk_ms = edist.max_over_ranks(chunk_ms, dev)
     err = efla.last_device_error()
     if err != 0:
         raise RuntimeError("device error word set: %s" % efla.status_str(err))
 
-    value = tok_step * args.steps * ws / (ms / 1e3)
+    value = edist.aggregate_rate(tok_step, args.steps, ws, ms)
     alg = alg_bytes_chunk(w)
     achieved = alg / (chunk_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm"], "traffic": None,
-                "kernel": "efla_chunk_fwd (%s path)" % path,
+                "frac": achieved / peaks["hbm"], "traffic": profiled_traffic(w),
+                "kernel": "efla_chunk_fwd (%s path: prep + state kernels)" % path,
                 "alg_bytes_per_launch": alg, "avg_launch_ms": chunk_ms,
-                "peak_source": peaks["src"] + " (MEASURED_PEAKS.json hbm_gbs)"}
+                "peak_source": peaks["src"] + " (MEASURED_PEAKS.json hbm_gbs, copy burst)",
+                "source_hash": kernel_source_hash()}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -330,8 +341,7 @@ def run_ours(args) -> None:
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)
-        if ws > 1:
-            torch.distributed.barrier()
+        edist.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, min(args.steps, 10))
         a.record(stream)
@@ -339,8 +349,8 @@ def run_ours(args) -> None:
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = _max_over_ranks(a.elapsed_time(b), ws, dev)
-        e2e = {"value": tok_step * n_e2e * ws / (e_ms / 1e3), "unit": UNIT,
+        e_ms = edist.max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": edist.aggregate_rate(tok_step, n_e2e, ws, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
 
