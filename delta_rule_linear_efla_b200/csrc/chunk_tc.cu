@@ -400,12 +400,24 @@ __device__ __forceinline__ void pack32_f16(const float (&v)[32], uint32_t (&w)[1
 //   V and Ta  -- read by U'^T(n) and W(n)            released after U'^T(n)
 //   Q (+ -W)  -- read by P^T(n) and D1(n)            released after D1(n)
 //   K (+ P^T) -- read by W(n), P^T(n) and D2(n)      released after D2(n)
+// The barriers an epilogue warpgroup signals take one arrival per warp, so no warp
+// waits for the other three before the issuer can go on.
 struct StateBars {
-    uint64_t fullV[2], fullQ[2], fullK[2], conv[2];
+    uint64_t fullV[2], fullQ[2], fullK[2];
     uint64_t freeV[2], freeQ[2], freeK[2];
     uint64_t wdone, pdone, d1done, d2done, drain;
-    uint64_t w_ready, p_ready, up_ready, s_ready, o_free;
+    // per-warp arrivals (4 each) from here on
+    uint64_t conv[2], w_ready, p_ready, up_ready_a, up_ready, s_ready_a, s_ready, o_free;
 };
+constexpr int BARS_ONE = 17;  // barriers before `conv` take a single arrival
+
+// Signal `bar` once this warp's TMEM and shared-memory writes are done (a shared-memory
+// writer issues fence.proxy.async first, so the tensor core sees its stores).
+__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
+    tc::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(bar);
+}
 
 template <int DK, int DV, typename TO>
 __global__ void __launch_bounds__(ST_THREADS, 1)
@@ -428,7 +440,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     const int bh = blockIdx.x;
     if (tid == 0) {
         uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
-        for (int i = 0; i < (int)(sizeof(StateBars) / sizeof(uint64_t)); ++i) tc::mbar_init(b + i, 1);
+        for (int i = 0; i < (int)(sizeof(StateBars) / sizeof(uint64_t)); ++i)
+            tc::mbar_init(b + i, i < BARS_ONE ? 1 : 4);
         tc::fence_mbar_init();
         abort_flag = 0;
         tc::tma_prefetch_desc(&tmap_q);
@@ -565,30 +578,48 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 const uint32_t stg = stage_addr(n);
                 const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
                 // D1: [O^T | U'^T] += S^T [Q | -W]^T   (A = fp16 S^T in TMEM)
+                // the first 64 rows of S^T are packed before the rest: start on them
                 if (!tc::mbar_wait_or_abort(&bars.w_ready, n & 1, &abort_flag, budget)) break;
-                if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget)) break;
                 if (n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
+                if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready_a, (n - 1) & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
+                bool ok2 = true;
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    if (kk == 4 && n > 0) {
+                        ok2 = tc::mbar_wait_or_abort(&bars.s_ready, (n - 1) & 1, &abort_flag, budget);
+                        if (!ok2) break;
+                        tc::tc_fence_after();
+                    }
                     tc::mma_tmem_a(tmem + TM_O, tmem + TM_S16 + kk * 8,
                                    tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
                                    id_d1, 1u);
+                }
+                if (!ok2) break;
                 tc::mma_commit(&bars.d1done);
                 tc::mma_commit(&bars.freeQ[st]);
                 if (n + 1 < NC) {  // W of the next chunk (its TMEM was read out before D1(n))
+                    // shared-memory handshake only: the fence before D1(n) already orders
+                    // this MMA after the side group's TMEM reads of W(n)
                     if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) break;
-                    tc::tc_fence_after();
                     issue_w(n + 1);
                 }
                 // D2: [S^T | O^T] += U'^T [K | P^T]   (A = fp16 U'^T in TMEM)
-                if (!tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget)) break;
+                // U' is packed in two halves of 32 tokens: start on the first
                 if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
+                if (!tc::mbar_wait_or_abort(&bars.up_ready_a, n & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
+                for (int kk = 0; kk < 4; ++kk) {
+                    if (kk == 2) {
+                        ok2 = tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget);
+                        if (!ok2) break;
+                        tc::tc_fence_after();
+                    }
                     tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
                                    tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
+                }
+                if (!ok2) break;
                 tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeK[st]);
                 if (n + 1 < NC) {  // P^T and the U' prefill of the next chunk
@@ -613,31 +644,27 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             const int st = n & 1;
             const uint32_t par = (n >> 1) & 1;
             uint8_t *stg = base + st * Lay::STAGE;
-            bool ok = tc::mbar_wait_or_abort(&bars.fullV[st], par, &abort_flag, budget);
-            if (tc::named_bar_or(1, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.fullV[st], par, &abort_flag, budget)) break;
             {
                 uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
 #pragma unroll
                 for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
             }
-            ok = tc::mbar_wait_or_abort(&bars.fullQ[st], par, &abort_flag, budget);
-            if (tc::named_bar_or(1, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.fullQ[st], par, &abort_flag, budget)) break;
 #pragma unroll
             for (int j = 0; j < DK / 64; ++j) {  // Q: the first 8 KB of each QW slab
                 uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
 #pragma unroll
                 for (int i = gtid; i < 512; i += 128) cvt(tq + i);
             }
-            ok = tc::mbar_wait_or_abort(&bars.fullK[st], par, &abort_flag, budget);
-            if (tc::named_bar_or(1, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.fullK[st], par, &abort_flag, budget)) break;
             {
                 uint4 *tk = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
 #pragma unroll
                 for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
             }
             tc::fence_async_smem();
-            tc::named_bar_sync(1, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.conv[st]);
+            warp_arrive(&bars.conv[st], lane);
         }
     } else if (wg == 1) {
         // ---------------------------------------------------------- side epilogue
@@ -645,8 +672,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         for (int n = 0; n < NC; ++n) {
             const int st = n & 1;
             uint8_t *stg = base + st * Lay::STAGE;
-            bool ok = tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(2, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {  // -W rows into rows 64.. of the QW slabs
@@ -659,12 +685,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
             tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.w_ready);
+            warp_arrive(&bars.w_ready, lane);
 
-            ok = tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(2, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {  // masked P^T (row c_in, column c_out >= c_in)
@@ -678,35 +701,30 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
             tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_bar_sync(2, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.p_ready);
+            warp_arrive(&bars.p_ready, lane);
         }
     } else if (wg == 2) {
         // ---------------------------------------------------------- chain epilogue
         bool done_all = true;
         for (int n = 0; n < NC; ++n) {
-            bool ok = tc::mbar_wait_or_abort(&bars.d1done, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
+            if (!tc::mbar_wait_or_abort(&bars.d1done, n & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
-            {
-                float u[64];
-                tc::tmem_ld64(tmem + lane_base + TM_U, u);
-                uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
-                tc::tmem_st32u(tmem + lane_base + TM_U, w);  // packed over its own fp32 columns
+            for (int h = 0; h < 2; ++h) {  // U'^T to fp16 in place, 32 tokens at a time
+                float u[32];
+                tc::tmem_ld32(tmem + lane_base + TM_U + h * 32, u);
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
+                tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, w);  // over fp32 columns already read
+                warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
             }
-            tc::tc_fence_before();
-            tc::named_bar_sync(3, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.up_ready);
 
-            ok = tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(3, 128, !ok)) { done_all = false; break; }
+            if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
-            if (n + 1 < NC) {
 #pragma unroll
-                for (int cb = 0; cb < DK / 64; ++cb) {
+            for (int cb = 0; cb < DK / 64; ++cb) {  // S^T to fp16, 64 rows of S at a time
+                if (n + 1 < NC) {
                     float v[64];
                     tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
                     uint32_t w[32];
@@ -714,10 +732,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
                     tc::tmem_st32u(tmem + lane_base + TM_S16 + cb * 32, w);
                 }
+                if (cb == 0) warp_arrive(&bars.s_ready_a, lane);
             }
-            tc::tc_fence_before();
-            tc::named_bar_sync(3, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.s_ready);
+            warp_arrive(&bars.s_ready, lane);
         }
         if (done_all && S_final) {
 #pragma unroll
@@ -738,17 +755,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         for (int j = 0; j < 16; ++j) z[j] = 0.f;
         for (int n = 0; n < NC; ++n) {
             const int c0 = n * C;
-            const bool ok = tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget);
-            if (tc::named_bar_or(4, 128, !ok)) break;
+            if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
             const int cl = min(C, L - c0);
             float v[64];
             tc::tmem_ld64(tmem + lane_base + TM_O, v);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
-            tc::tc_fence_before();
-            tc::named_bar_sync(4, 128);
-            if (gtid == 0) tc::mbar_arrive(&bars.o_free);  // TMEM O is zero again: D1(n+1) may run
+            warp_arrive(&bars.o_free, lane);  // TMEM O is zero again: D1(n+1) may run
             if (vrow >= 0) {
                 TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
 #pragma unroll
