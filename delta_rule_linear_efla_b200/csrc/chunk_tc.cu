@@ -144,6 +144,14 @@ __global__ void __launch_bounds__(THREADS)
         issue(blockIdx.x);
         issued = true;
     }
+    // beta of row `tid` of chunk g (0 past the sequence end), loaded one chunk ahead so
+    // the global-load latency is not on the chunk's critical path
+    auto load_beta = [&](int gg) {
+        if (tid >= C || gg >= total) return 0.f;
+        const int bh = gg / NC, n = gg - bh * NC;
+        return n * C + tid < L ? __bfloat162float(beta[(size_t)bh * L + n * C + tid]) : 0.f;
+    };
+    float beta_next = load_beta(blockIdx.x);
     uint32_t mma_phase = 0;
     int it = 0;
     bool aborted = false;
@@ -151,10 +159,14 @@ __global__ void __launch_bounds__(THREADS)
     for (int g = blockIdx.x; g < total; g += gridDim.x, ++it) {
         const uint32_t ph = it & 1;
         const int bh = g / NC, n = g - bh * NC, c0 = n * C;
+        const float beta_row = beta_next;
+        beta_next = load_beta(g + gridDim.x);
+        (void)bh;
+        (void)c0;
         bool ok = tc::mbar_wait(&full, ph, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
-        if (tid == 0) {
-            issued = false;
+        if (tid == 0) issued = false;
+        if (tid == 96) {  // warp 3 issues: warps 0-1 compute the norms meanwhile
             tc::tc_fence_after();
             const uint32_t kb = tc::smem_u32(Kt);
             constexpr uint32_t id = tc::idesc_bf16(64, 64, false, false);
@@ -166,7 +178,7 @@ __global__ void __launch_bounds__(THREADS)
             tc::mma_commit(&mma_bar);
         }
         mma_pending = true;
-        // a per row: squared norm from the swizzled K tile, beta with a bounds check
+        // a per row: squared norm from the swizzled K tile
         if (tid < C) {
             const int r = tid;
             float sq = 0.f;
@@ -183,8 +195,7 @@ __global__ void __launch_bounds__(THREADS)
                     }
                 }
             }
-            const float b = (c0 + r < L) ? __bfloat162float(beta[(size_t)bh * L + c0 + r]) : 0.f;
-            al[r] = alpha_from(sq, b);
+            al[r] = alpha_from(sq, beta_row);
         }
         ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }  // also: every norm has been read
@@ -199,14 +210,15 @@ __global__ void __launch_bounds__(THREADS)
         {
             const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 accumulator layout)
             const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+            float g64[64];
+            tc::tmem_ld64(ta, g64);  // the whole row at once: one wait
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
-                float v[16];
-                tc::tmem_ld16(ta + cb * 16, v);
                 if (lane < 16) {
                     const float ar = al[r];
+                    float v[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * v[j] : 0.f;
+                    for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * g64[cb * 16 + j] : 0.f;
                     uint4 *dst = reinterpret_cast<uint4 *>(A16 + r * LD16 + cb * 16);
                     dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
                                         tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
