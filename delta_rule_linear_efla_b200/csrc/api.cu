@@ -67,7 +67,8 @@ efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int
 int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
                         efla_dtype o_dt) {
     (void)o_dt;
-    return efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16) ? 1 : 0;
+    if (!efla::tc_supported(B, H, L, dk, dv, chunk, dt == EFLA_BF16)) return 0;
+    return efla::tc_segments(B, H, L, dk, dv) >= 3 ? 2 : 1;
 }
 
 size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int chunk,

@@ -440,7 +440,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
-                    TO *__restrict__ o, float *__restrict__ S_final, int L, int NC) {
+                    TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
+                    float *__restrict__ segbuf, int G, int seg_chunks, int pass) {
     using Lay = StateLayout<DK, DV>;
     constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
     extern __shared__ uint8_t smem_raw[];
@@ -452,7 +453,39 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = warp >> 2, gtid = tid & 127;
-    const int bh = blockIdx.x;
+    // ---- the run this CTA makes: head bh, chunks [n0, n1), and what it starts from and keeps.
+    // pass 0: the whole sequence.  With the sequence cut into G segments of seg_chunks chunks
+    // (each segment maps the state affinely, S_out = P S_in + H), pass 1 runs segment 0 from
+    // S0 and, for every middle segment g, H_g (from zero) and P_g (the transition: from the
+    // identity with v = 0), with no output; pass 2 runs segments 1..G-1 from their true
+    // starting states, which the combine kernel chains together in between.
+    int bh = blockIdx.x, n0 = 0, n1 = NC, mode = 0;  // mode 0: outputs, 1: H run, 2: P run
+    const size_t DD = (size_t)DK * DV;
+    const float *s0p = S0 ? S0 + (size_t)bh * DD : nullptr;
+    float *sfp = S_final ? S_final + (size_t)bh * DD : nullptr;
+    if (pass == 1) {
+        const int R = 2 * G - 3, r = blockIdx.x % R, g = (r + 1) / 2;
+        bh = blockIdx.x / R;
+        n0 = g * seg_chunks;
+        n1 = min(NC, n0 + seg_chunks);
+        float *seg = segbuf + ((size_t)bh * G + g) * 3 * DD;  // [S_in | H | P] of segment g
+        if (r == 0) {
+            s0p = S0 ? S0 + (size_t)bh * DD : nullptr;
+            sfp = segbuf + ((size_t)bh * G + 1) * 3 * DD;  // S_in of segment 1
+        } else {
+            mode = (r & 1) ? 1 : 2;
+            s0p = nullptr;
+            sfp = seg + (size_t)mode * DD;
+        }
+    } else if (pass == 2) {
+        const int R = G - 1, g = 1 + (int)blockIdx.x % R;
+        bh = blockIdx.x / R;
+        n0 = g * seg_chunks;
+        n1 = min(NC, n0 + seg_chunks);
+        s0p = segbuf + ((size_t)bh * G + g) * 3 * DD;
+        sfp = (g == G - 1 && S_final) ? S_final + (size_t)bh * DD : nullptr;
+    }
+    const int cnt = n1 - n0;  // chunks of this run; stage and barrier phases follow the local index
     if (tid == 0) {
         uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(StateBars) / sizeof(uint64_t)); ++i)
@@ -475,6 +508,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     const uint32_t sb = tc::smem_u32(base);
     const int vrow = acc_row<DV>(warp & 3, lane);  // state column v of this thread's TMEM lane
 
+    // ---- a P run reads no values: its V tiles stay zero
+    if (mode == 2) {
+        for (int i = tid; i < 2 * Lay::VB / 16; i += ST_THREADS) {
+            const int stg = i / (Lay::VB / 16), w = i - stg * (Lay::VB / 16);
+            reinterpret_cast<uint4 *>(base + stg * Lay::STAGE + Lay::OFF_V)[w] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        tc::fence_async_smem();
+    }
     // ---- initial state (chain warpgroup): S^T, its fp16 copy and a zero O^T in TMEM
     if (wg == 2) {
 #pragma unroll
@@ -482,7 +523,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                v[j] = (S0 && vrow >= 0) ? S0[((size_t)bh * DK + cb * 32 + j) * DV + vrow] : 0.f;
+                v[j] = mode == 2 ? (cb * 32 + j == vrow ? 1.f : 0.f)
+                                 : ((s0p && vrow >= 0) ? s0p[(size_t)(cb * 32 + j) * DV + vrow] : 0.f);
             float lo[16], hi[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) { lo[j] = v[j]; hi[j] = v[16 + j]; }
@@ -507,27 +549,29 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
             int last[2] = {-1, -1};
-            for (int n = 0; n < NC; ++n) {
-                const int st = n & 1;
-                const uint32_t par = ((n - 2) >> 1) & 1;
+            for (int i = 0; i < cnt; ++i) {
+                const int n = n0 + i, st = i & 1;
+                const uint32_t par = ((i - 2) >> 1) & 1;
                 uint8_t *stg = base + st * Lay::STAGE;
-                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeV[st], par, &abort_flag, budget)) break;
-                tc::mbar_expect_tx(&bars.fullV[st], Lay::VB + Lay::TB);
+                if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeV[st], par, &abort_flag, budget)) break;
+                tc::mbar_expect_tx(&bars.fullV[st], (mode == 2 ? 0 : Lay::VB) + Lay::TB);
+                if (mode != 2) {
 #pragma unroll
-                for (int j = 0; j < DV / 64; ++j)
-                    tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
+                    for (int j = 0; j < DV / 64; ++j)
+                        tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
+                }
                 tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C);
-                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeQ[st], par, &abort_flag, budget)) break;
+                if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeQ[st], par, &abort_flag, budget)) break;
                 tc::mbar_expect_tx(&bars.fullQ[st], DK * 128);
 #pragma unroll
                 for (int j = 0; j < DK / 64; ++j)
                     tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
-                if (n >= 2 && !tc::mbar_wait_or_abort(&bars.freeK[st], par, &abort_flag, budget)) break;
+                if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeK[st], par, &abort_flag, budget)) break;
                 tc::mbar_expect_tx(&bars.fullK[st], DK * 128);
 #pragma unroll
                 for (int j = 0; j < DK / 64; ++j)
                     tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, &bars.fullK[st], j * 64, n * C, bh);
-                last[st] = n;
+                last[st] = i;
             }
             if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
                 for (int st = 0; st < 2; ++st) {
@@ -588,7 +632,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 issue_p(0);
                 issue_u(0);
             }
-            for (int n = 0; ok && n < NC; ++n) {
+            for (int n = 0; ok && n < cnt; ++n) {  // n: local chunk index
                 const int st = n & 1;
                 const uint32_t stg = stage_addr(n);
                 const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
@@ -613,7 +657,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (!ok2) break;
                 tc::mma_commit(&bars.d1done);
                 tc::mma_commit(&bars.freeQ[st]);
-                if (n + 1 < NC) {  // W of the next chunk (its TMEM was read out before D1(n))
+                if (n + 1 < cnt) {  // W of the next chunk (its TMEM was read out before D1(n))
                     // shared-memory handshake only: the fence before D1(n) already orders
                     // this MMA after the side group's TMEM reads of W(n)
                     if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) break;
@@ -637,7 +681,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (!ok2) break;
                 tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeK[st]);
-                if (n + 1 < NC) {  // P^T and the U' prefill of the next chunk
+                if (n + 1 < cnt) {  // P^T and the U' prefill of the next chunk
                     issue_p(n + 1);
                     issue_u(n + 1);
                 }
@@ -655,12 +699,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
             *t = u;
         };
-        for (int n = 0; n < NC; ++n) {
+        for (int n = 0; n < cnt; ++n) {  // n: local chunk index
             const int st = n & 1;
             const uint32_t par = (n >> 1) & 1;
             uint8_t *stg = base + st * Lay::STAGE;
             if (!tc::mbar_wait_or_abort(&bars.fullV[st], par, &abort_flag, budget)) break;
-            {
+            if (mode != 2) {
                 uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
 #pragma unroll
                 for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
@@ -684,7 +728,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     } else if (wg == 1) {
         // ---------------------------------------------------------- side epilogue
         const int crow = acc_row<64>(warp & 3, lane);  // token row of the M = 64 accumulators
-        for (int n = 0; n < NC; ++n) {
+        for (int n = 0; n < cnt; ++n) {  // n: local chunk index
             const int st = n & 1;
             uint8_t *stg = base + st * Lay::STAGE;
             if (!tc::mbar_wait_or_abort(&bars.wdone, n & 1, &abort_flag, budget)) break;
@@ -721,7 +765,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     } else if (wg == 2) {
         // ---------------------------------------------------------- chain epilogue
         bool done_all = true;
-        for (int n = 0; n < NC; ++n) {
+        for (int n = 0; n < cnt; ++n) {  // n: local chunk index
             if (!tc::mbar_wait_or_abort(&bars.d1done, n & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
 #pragma unroll
@@ -739,7 +783,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < DK / 64; ++cb) {  // S^T to fp16, 64 rows of S at a time
-                if (n + 1 < NC) {
+                if (n + 1 < cnt) {
                     float v[64];
                     tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
                     uint32_t w[32];
@@ -751,7 +795,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             }
             warp_arrive(&bars.s_ready, lane);
         }
-        if (done_all && S_final) {
+        if (done_all && sfp) {
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {
                 float v[16];
@@ -759,7 +803,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (vrow >= 0) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        S_final[((size_t)bh * DK + cb * 16 + j) * DV + vrow] = v[j];
+                        sfp[(size_t)(cb * 16 + j) * DV + vrow] = v[j];
                 }
             }
         }
@@ -768,8 +812,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         float z[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) z[j] = 0.f;
-        for (int n = 0; n < NC; ++n) {
-            const int c0 = n * C;
+        for (int n = 0; n < cnt; ++n) {  // n: local chunk index
+            const int c0 = (n0 + n) * C;
             if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
             const int cl = min(C, L - c0);
@@ -778,7 +822,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
             warp_arrive(&bars.o_free, lane);  // TMEM O is zero again: D1(n+1) may run
-            if (vrow >= 0) {
+            if (mode == 0 && vrow >= 0) {
                 TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
@@ -791,6 +835,48 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     if (tid == 0 && abort_flag) record_error(2u);
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
+
+// ------------------------------------------------------------------ segment chaining
+// Each sequence segment maps the state affinely, S_out = P S_in + H (P is the product of
+// the segment's transitions I - K^T W, H the segment's state from zero).  This chains
+// S_in(g+1) = P_g S_in(g) + H_g for g = 1..G-2 in fp32, one 16-column block of the state
+// per CTA (the state's columns evolve independently), one state row per thread.
+template <int D>
+__global__ void __launch_bounds__(D) seg_combine_kernel(float *__restrict__ segbuf, int G) {
+    extern __shared__ float csm[];
+    float *Ps = csm;                 // P_g, [D][D + 1] (padded: row-per-thread reads)
+    float *X = csm + D * (D + 1);    // the running S_in block, [D][16]
+    constexpr int NB = D / 16;
+    const int cbk = blockIdx.x % NB, bh = blockIdx.x / NB, t = threadIdx.x;
+    const size_t DD = (size_t)D * D;
+    float *seg = segbuf + (size_t)bh * G * 3 * DD;  // per segment: [S_in | H | P]
+#pragma unroll
+    for (int c = 0; c < 16; ++c) X[t * 16 + c] = seg[3 * DD + (size_t)t * D + cbk * 16 + c];
+    for (int g = 1; g + 1 < G; ++g) {
+        const float *P = seg + ((size_t)g * 3 + 2) * DD, *Hm = seg + ((size_t)g * 3 + 1) * DD;
+        __syncthreads();  // X written, Ps no longer read
+        for (int i = t; i < D * D; i += D) Ps[(i / D) * (D + 1) + i % D] = P[i];
+        __syncthreads();
+        float y[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) y[c] = Hm[(size_t)t * D + cbk * 16 + c];
+        for (int m = 0; m < D; ++m) {
+            const float pm = Ps[t * (D + 1) + m];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) y[c] = fmaf(pm, X[m * 16 + c], y[c]);
+        }
+        __syncthreads();  // every row has read X
+        float *Sn = seg + (size_t)(g + 1) * 3 * DD;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            X[t * 16 + c] = y[c];
+            Sn[(size_t)t * D + cbk * 16 + c] = y[c];
+        }
+    }
+}
+
+template <int D>
+constexpr int combine_smem_bytes() { return (D * (D + 1) + D * 16) * (int)sizeof(float); }
 
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -839,10 +925,28 @@ int prep_smem_bytes() {
     return prep::Smem::bytes<DK>() + 1024;
 }
 
+// Sequence segments: with few heads and a long sequence, the sequence is cut into G
+// segments that run in parallel (pass 1: segment 0 plus each middle segment's H and P;
+// pass 2: segments 1..G-1 from their chained starting states).  Pass 1 takes BH (2G - 3)
+// CTAs, so G grows while that fits the SMs, up to SEG_MAX, and every segment keeps at
+// least 16 chunks.  The workspace reserves SEG_MAX segments' state whenever the sizes
+// allow segments (dk == dv, at least 48 chunks, at most 48 heads).
+constexpr int SEG_MAX = 8;
+bool seg_sizes_ok(long long BH, int NC, int dk, int dv) { return dk == dv && NC >= 48 && BH <= 48; }
+int seg_count(long long BH, int NC, int dk, int dv, int nsm) {
+    if (!seg_sizes_ok(BH, NC, dk, dv)) return 1;
+    long long G = ((long long)nsm + 3 * BH) / (2 * BH);
+    G = G < SEG_MAX ? G : SEG_MAX;
+    G = G < NC / 16 ? G : NC / 16;
+    return G >= 3 ? (int)G : 1;
+}
+size_t ta_bytes(size_t total) { return (total * C * C * sizeof(__half) + 255) / 256 * 256; }
+
 // What a launch needs to know about the current device, worked out once per device
 // and kernel instantiation (the kernels' shared-memory attributes are set then too),
 // so that a call costs the tensor-map encodings and the two launches and nothing more.
 struct TcDevInfo {
+    int nsm = 0;
     int prep_grid = 0;  // CTAs of the prep kernel: every SM, as many as fit by shared memory
     cudaError_t err = cudaSuccess;
 };
@@ -874,7 +978,11 @@ TcDevInfo tc_dev_info() {
     if (d.err == cudaSuccess)
         d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      StateLayout<DK, DV>::SMEM);
+    if (d.err == cudaSuccess && DK == DV)
+        d.err = cudaFuncSetAttribute(seg_combine_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     combine_smem_bytes<DK>());
     if (d.err != cudaSuccess) return d;
+    d.nsm = nsm;
     int per_sm = smem_sm / (psm + 1024);  // 1 KiB per CTA is reserved by the system
     per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
     d.prep_grid = nsm * per_sm;
@@ -900,12 +1008,27 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
                                                                       (__half *)ws, L, NC, total);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC; two
-    // heads' chunk loops on the two SMs of one TPC each run 15-25% slower (measured), so
-    // nothing else is scheduled beside this kernel.
-    tc_state_kernel<DK, DV, TO><<<BH, ST_THREADS, StateLayout<DK, DV>::SMEM, s>>>(mq, mk, mv, mt, S0, (TO *)o,
-                                                                                 S_final, L, NC);
-    count_launches(2);
+    constexpr int SSM = StateLayout<DK, DV>::SMEM;
+    const int G = seg_count(BH, NC, DK, DV, di.nsm);
+    if (G < 3) {
+        // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
+        // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
+        // (measured), so nothing else is scheduled beside this kernel.
+        tc_state_kernel<DK, DV, TO><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC,
+                                                               nullptr, 1, NC, 0);
+        count_launches(2);
+        return cudaGetLastError();
+    }
+    if constexpr (DK == DV) {
+        const int seg_chunks = (NC + G - 1) / G;
+        float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
+        tc_state_kernel<DK, DV, TO><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1);
+        seg_combine_kernel<DK><<<BH * (DV / 16), DK, combine_smem_bytes<DK>(), s>>>(segbuf, G);
+        tc_state_kernel<DK, DV, TO><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2);
+        count_launches(4);
+    }
     return cudaGetLastError();
 }
 
@@ -929,9 +1052,22 @@ bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16) 
 }
 
 size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk) {
-    (void)dk; (void)dv; (void)chunk;
-    const size_t total = (size_t)B * H * ((L + C - 1) / C);
-    return total * C * C * sizeof(__half);
+    (void)chunk;
+    const long long BH = (long long)B * H;
+    const int NC = (L + C - 1) / C;
+    const size_t total = (size_t)BH * NC;
+    if (!seg_sizes_ok(BH, NC, dk, dv)) return total * C * C * sizeof(__half);
+    return ta_bytes(total) + (size_t)BH * SEG_MAX * 3 * dk * dv * sizeof(float);
+}
+
+int tc_segments(int B, int H, int L, int dk, int dv) {
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 1;
+    }
+    return seg_count((long long)B * H, (L + C - 1) / C, dk, dv, nsm);
 }
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,

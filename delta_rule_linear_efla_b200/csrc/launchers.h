@@ -32,6 +32,7 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
 size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
+int tc_segments(int B, int H, int L, int dk, int dv);  // sequence segments the launch uses (1: none)
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
                             const float *S0, void *o, float *S_final, int B, int H, int L,
                             int dk, int dv, int chunk, bool o_bf16, void *ws, cudaStream_t s);

@@ -128,7 +128,7 @@ def workspace_size(B: int, H: int, L: int, dk: int, dv: int, chunk: int, dtype,
 
 def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype, o_dtype=torch.float32) -> str:
     p = load_library().efla_chunk_fwd_path(B, H, L, dk, dv, chunk, _code(dtype), _code(o_dtype))
-    return "tcgen05" if p else "simt"
+    return {0: "simt", 1: "tcgen05", 2: "tcgen05-segments"}[p]
 
 
 def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,

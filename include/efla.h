@@ -184,8 +184,13 @@ efla_status efla_recurrent_step(const void *q, const void *k, const void *v, con
 efla_status efla_last_device_error(void *stream);
 
 /*
- * Which chunk-forward kernels the library selects for these sizes:
- * 0 = SIMT fp32 path, 1 = tensor-core (tcgen05) path.  For tests and tools.
+ * Which chunk-forward kernels the library selects for these sizes on the current
+ * device: 0 = SIMT fp32 path, 1 = tensor-core (tcgen05) path, 2 = tensor-core path
+ * with the sequence cut into segments that run in parallel (few heads, long
+ * sequences: each segment maps the state affinely, S_out = P S_in + H, so the
+ * segments' maps are computed side by side, chained, and the segments rerun from
+ * their true starting states).  Without a usable device, 2 is never reported.
+ * For tests and tools.
  */
 int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
                         efla_dtype o_dt);

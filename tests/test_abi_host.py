@@ -96,7 +96,7 @@ def test_workspace_query_is_host_only(lib):
             n = lib.efla_chunk_fwd_workspace_size(*wid_sizes, dt, F32)
             assert n >= 0
             path = lib.efla_chunk_fwd_path(*wid_sizes, dt, F32)
-            assert path in (0, 1)
+            assert path in (0, 1, 2)
             if path == 0:
                 assert n == 0
     assert lib.efla_chunk_fwd_workspace_size(1, 1, 64, 16, 16, 48, BF16, F32) == 0
@@ -115,3 +115,13 @@ def test_binding_fails_loudly_without_cuda():
 def test_binding_raises_when_library_missing(tmp_path):
     with pytest.raises(RuntimeError):
         efla.load_library(str(tmp_path / "missing.so"))
+
+
+def test_workspace_reserves_segment_state(lib):
+    """Sizes that may run as sequence segments reserve eight segments' [S_in | H | P] fp32
+    states per head after the Ta tiles; other sizes need only the Ta tiles (8 KiB per chunk)."""
+    ta = 16 * 1024 * 64 * 64 * 2
+    assert lib.efla_chunk_fwd_workspace_size(1, 16, 65536, 128, 128, 64, BF16, F32) == \
+        ta + 16 * 8 * 3 * 128 * 128 * 4
+    assert lib.efla_chunk_fwd_workspace_size(4, 16, 4096, 128, 128, 64, BF16, F32) == 4 * 16 * 64 * 8192
+    assert lib.efla_chunk_fwd_workspace_size(1, 2, 4096, 128, 64, 64, BF16, F32) == 2 * 64 * 8192

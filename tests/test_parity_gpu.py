@@ -207,3 +207,50 @@ def test_linearity_in_values_and_state():
     o3, F3 = efla.chunk_fwd(d["q"], d["k"], a * d["v"] + b * V2, d["beta"], a * S1 + b * S2, chunk=16)
     assert rel_err(o3.cpu().numpy(), (a * o1 + b * o2).cpu().numpy()) < 1e-5
     assert rel_err(F3.cpu().numpy(), (a * F1 + b * F2).cpu().numpy()) < 1e-5
+
+
+# ---- sequence segments: few heads and a long sequence run as parallel segments whose affine
+# state maps (S_out = P S_in + H) are chained and then rerun from their true starting states
+
+
+def test_segment_path_selection():
+    bf = torch.bfloat16
+    assert efla.chunk_fwd_path(1, 16, 65536, 128, 128, 64, bf) == "tcgen05-segments"
+    assert efla.chunk_fwd_path(1, 48, 4096, 128, 128, 64, bf) == "tcgen05-segments"
+    assert efla.chunk_fwd_path(1, 49, 4096, 128, 128, 64, bf) == "tcgen05"   # too many heads
+    assert efla.chunk_fwd_path(1, 2, 47 * 64, 128, 128, 64, bf) == "tcgen05"  # too few chunks
+    assert efla.chunk_fwd_path(1, 2, 4096, 128, 64, 64, bf) == "tcgen05"      # dk != dv
+
+
+@pytest.mark.parametrize("L", [48 * 64 - 10, 48 * 64])
+def test_segments_stiff_parity(oracle_mod, L):
+    """Workload-5 distributions (key norms over six decades, 5% of values x10) on two heads,
+    cut into three segments; the first length ends in a ragged chunk."""
+    x = inputs.make_inputs(inputs.workload(5, B=1, H=2, L=L))
+    assert efla.chunk_fwd_path(1, 2, L, 128, 128, 64, torch.bfloat16) == "tcgen05-segments"
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+def test_segments_from_nonzero_state(oracle_mod):
+    """A nonzero initial state enters through segment 0 and every later segment's start."""
+    x = inputs.make_inputs(inputs.workload(2, B=1, H=3, L=64 * 64, dk=128, dv=128))
+    assert x["S0"] is not None and float(x["S0"].abs().max()) > 0
+    assert efla.chunk_fwd_path(1, 3, 64 * 64, 128, 128, 64, torch.bfloat16) == "tcgen05-segments"
+    o, S = _run_gpu(x)
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
+
+
+def test_segments_in_place_state_carry(oracle_mod):
+    """S_final may alias S0 with segments too: the segments read S0 before the last writes it."""
+    x = inputs.make_inputs(inputs.workload(2, B=1, H=2, L=64 * 64, dk=128, dv=128))
+    d = _to_dev(x)
+    S = d["S0"].clone()
+    o, S_out = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], S, chunk=64, S_final=S)
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    assert S_out.data_ptr() == S.data_ptr()
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o.float().cpu(), S.cpu(), o_ref, S_ref)
