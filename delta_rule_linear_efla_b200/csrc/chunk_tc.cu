@@ -434,7 +434,8 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
     if (lane == 0) tc::mbar_arrive(bar);
 }
 
-template <int DK, int DV, typename TO>
+// SEG = false compiles the one-pass form only (pass 0); SEG = true also takes the segment runs.
+template <int DK, int DV, typename TO, bool SEG>
 __global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -463,6 +464,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     const size_t DD = (size_t)DK * DV;
     const float *s0p = S0 ? S0 + (size_t)bh * DD : nullptr;
     float *sfp = S_final ? S_final + (size_t)bh * DD : nullptr;
+    if (!SEG) pass = 0;
     if (pass == 1) {
         const int R = 2 * G - 3, r = blockIdx.x % R, g = (r + 1) / 2;
         bh = blockIdx.x / R;
@@ -485,6 +487,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         s0p = segbuf + ((size_t)bh * G + g) * 3 * DD;
         sfp = (g == G - 1 && S_final) ? S_final + (size_t)bh * DD : nullptr;
     }
+    if (!SEG) mode = 0;
     const int cnt = n1 - n0;  // chunks of this run; stage and barrier phases follow the local index
     if (tid == 0) {
         uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
@@ -840,43 +843,59 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 // Each sequence segment maps the state affinely, S_out = P S_in + H (P is the product of
 // the segment's transitions I - K^T W, H the segment's state from zero).  This chains
 // S_in(g+1) = P_g S_in(g) + H_g for g = 1..G-2 in fp32, one 16-column block of the state
-// per CTA (the state's columns evolve independently), one state row per thread.
+// per CTA (the state's columns evolve independently), one state row per thread: the
+// thread's row of P_g comes straight from global memory with all its loads in flight.
 template <int D>
 __global__ void __launch_bounds__(D) seg_combine_kernel(float *__restrict__ segbuf, int G) {
-    extern __shared__ float csm[];
-    float *Ps = csm;                 // P_g, [D][D + 1] (padded: row-per-thread reads)
-    float *X = csm + D * (D + 1);    // the running S_in block, [D][16]
+    __shared__ __align__(16) float X[D][16];  // the running S_in block
     constexpr int NB = D / 16;
     const int cbk = blockIdx.x % NB, bh = blockIdx.x / NB, t = threadIdx.x;
     const size_t DD = (size_t)D * D;
     float *seg = segbuf + (size_t)bh * G * 3 * DD;  // per segment: [S_in | H | P]
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(seg + 3 * DD + (size_t)t * D + cbk * 16);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) X[t * 16 + c] = seg[3 * DD + (size_t)t * D + cbk * 16 + c];
+        for (int c = 0; c < 4; ++c) reinterpret_cast<float4 *>(X[t])[c] = src[c];
+    }
     for (int g = 1; g + 1 < G; ++g) {
-        const float *P = seg + ((size_t)g * 3 + 2) * DD, *Hm = seg + ((size_t)g * 3 + 1) * DD;
-        __syncthreads();  // X written, Ps no longer read
-        for (int i = t; i < D * D; i += D) Ps[(i / D) * (D + 1) + i % D] = P[i];
-        __syncthreads();
+        const float4 *prow = reinterpret_cast<const float4 *>(seg + ((size_t)g * 3 + 2) * DD + (size_t)t * D);
+        const float4 *hrow = reinterpret_cast<const float4 *>(seg + ((size_t)g * 3 + 1) * DD + (size_t)t * D + cbk * 16);
+        float4 p[D / 4];
+#pragma unroll
+        for (int m = 0; m < D / 4; ++m) p[m] = prow[m];
         float y[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) y[c] = Hm[(size_t)t * D + cbk * 16 + c];
-        for (int m = 0; m < D; ++m) {
-            const float pm = Ps[t * (D + 1) + m];
+        for (int c = 0; c < 4; ++c) {
+            const float4 h = hrow[c];
+            y[4 * c] = h.x; y[4 * c + 1] = h.y; y[4 * c + 2] = h.z; y[4 * c + 3] = h.w;
+        }
+        __syncthreads();  // X holds S_in(g)
 #pragma unroll
-            for (int c = 0; c < 16; ++c) y[c] = fmaf(pm, X[m * 16 + c], y[c]);
+        for (int m4 = 0; m4 < D / 4; ++m4) {
+            const float pm[4] = {p[m4].x, p[m4].y, p[m4].z, p[m4].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 *xr = reinterpret_cast<const float4 *>(X[4 * m4 + e]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 xv = xr[c];
+                    y[4 * c] = fmaf(pm[e], xv.x, y[4 * c]);
+                    y[4 * c + 1] = fmaf(pm[e], xv.y, y[4 * c + 1]);
+                    y[4 * c + 2] = fmaf(pm[e], xv.z, y[4 * c + 2]);
+                    y[4 * c + 3] = fmaf(pm[e], xv.w, y[4 * c + 3]);
+                }
+            }
         }
         __syncthreads();  // every row has read X
-        float *Sn = seg + (size_t)(g + 1) * 3 * DD;
+        float4 *dst = reinterpret_cast<float4 *>(seg + (size_t)(g + 1) * 3 * DD + (size_t)t * D + cbk * 16);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            X[t * 16 + c] = y[c];
-            Sn[(size_t)t * D + cbk * 16 + c] = y[c];
+        for (int c = 0; c < 4; ++c) {
+            const float4 v = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+            reinterpret_cast<float4 *>(X[t])[c] = v;
+            dst[c] = v;
         }
     }
 }
-
-template <int D>
-constexpr int combine_smem_bytes() { return (D * (D + 1) + D * 16) * (int)sizeof(float); }
 
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -976,11 +995,11 @@ TcDevInfo tc_dev_info() {
     if (d.err == cudaSuccess)
         d.err = cudaFuncSetAttribute(tc_prep_kernel<DK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (d.err == cudaSuccess)
-        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     StateLayout<DK, DV>::SMEM);
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
     if (d.err == cudaSuccess && DK == DV)
-        d.err = cudaFuncSetAttribute(seg_combine_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     combine_smem_bytes<DK>());
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
     if (d.err != cudaSuccess) return d;
     d.nsm = nsm;
     int per_sm = smem_sm / (psm + 1024);  // 1 KiB per CTA is reserved by the system
@@ -1014,18 +1033,18 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
-        tc_state_kernel<DK, DV, TO><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC,
-                                                               nullptr, 1, NC, 0);
+        tc_state_kernel<DK, DV, TO, false><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final,
+                                                                      L, NC, nullptr, 1, NC, 0);
         count_launches(2);
         return cudaGetLastError();
     }
     if constexpr (DK == DV) {
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
-        tc_state_kernel<DK, DV, TO><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
+        tc_state_kernel<DK, DV, TO, true><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
             mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1);
-        seg_combine_kernel<DK><<<BH * (DV / 16), DK, combine_smem_bytes<DK>(), s>>>(segbuf, G);
-        tc_state_kernel<DK, DV, TO><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
+        seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
+        tc_state_kernel<DK, DV, TO, true><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
             mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2);
         count_launches(4);
     }
