@@ -49,6 +49,13 @@ def _load():
                                          ctypes.c_double, dp]
         lib.efla_oracle_fwd.restype = ctypes.c_int
         lib.efla_oracle_fwd.argtypes = [ctypes.c_int] * 5 + [dp] * 7 + [ctypes.c_int]
+        lib.efla_oracle_coeff.restype = ctypes.c_double
+        lib.efla_oracle_coeff.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.efla_oracle_step_rule.restype = ctypes.c_double
+        lib.efla_oracle_step_rule.argtypes = [ctypes.c_int, ctypes.c_int, dp, dp, dp, dp,
+                                              ctypes.c_double, dp, ctypes.c_int]
+        lib.efla_oracle_fwd_rule.restype = ctypes.c_int
+        lib.efla_oracle_fwd_rule.argtypes = [ctypes.c_int] * 5 + [dp] * 7 + [ctypes.c_int] * 2
         _lib = lib
     return _lib
 
@@ -67,25 +74,34 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def alpha(lam: float, beta: float) -> float:
-    """alpha = (1 - exp(-beta*lam))/lam, evaluated as -expm1(-beta*lam)/lam; beta at lam == 0."""
-    return float(_load().efla_oracle_alpha(float(lam), float(beta)))
+RULES = {"exact": 0, "euler": 1}
 
 
-def step(S, q, k, v, beta: float):
+def alpha(lam: float, beta: float, rule: str = "exact") -> float:
+    """alpha = (1 - exp(-beta*lam))/lam, evaluated as -expm1(-beta*lam)/lam; beta at lam == 0.
+    rule="euler": the delta rule's coefficient, beta."""
+    if rule == "exact":
+        return float(_load().efla_oracle_alpha(float(lam), float(beta)))
+    return float(_load().efla_oracle_coeff(float(lam), float(beta), RULES[rule]))
+
+
+def step(S, q, k, v, beta: float, rule: str = "exact"):
     """One recurrent token on one head.  Returns (S_t, o_t, alpha_t); S is not modified."""
     S = _f64(S).copy()
     q, k, v = _f64(q), _f64(k), _f64(v)
     dk, dv = S.shape
     o = np.zeros(dv)
-    a = _load().efla_oracle_step(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta), _ptr(o))
+    a = _load().efla_oracle_step_rule(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta),
+                                      _ptr(o), RULES[rule])
     return S, o, float(a)
 
 
-def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True):
+def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True,
+        rule: str = "exact"):
     """Token-by-token forward over [B,H,L,d] inputs.  Returns (o, S_final) in fp64.
 
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L]; S0: [B,H,dk,dv] or None (zeros).
+    rule="euler" takes the delta rule's explicit Euler step (alpha = beta) instead.
     """
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
     B, H, L, dk = q.shape
@@ -99,9 +115,10 @@ def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True
     S = np.zeros((B, H, dk, dv))
     if nthreads is None:
         nthreads = os.cpu_count() or 1
-    rc = _load().efla_oracle_fwd(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
-                                 _ptr(s0) if s0 is not None else None,
-                                 _ptr(o) if o is not None else None, _ptr(S), int(nthreads))
+    rc = _load().efla_oracle_fwd_rule(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                      _ptr(s0) if s0 is not None else None,
+                                      _ptr(o) if o is not None else None, _ptr(S), int(nthreads),
+                                      RULES[rule])
     if rc != 0:
         raise MemoryError("oracle forward failed to allocate")
     return o, S

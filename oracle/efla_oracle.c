@@ -17,6 +17,11 @@
  *   o_t      = S_t^T q_t      (the standard delta-rule readout, taken after
  *                              the update; the summary prints no readout)
  *
+ * and, for comparison, the delta rule that the summary identifies as the
+ * explicit Euler step of the same ODE, dS/dtau = -k k^T S + k v^T over an
+ * interval beta_t (Methodology 1; Key Contributions): S + beta_t (k v^T -
+ * k k^T S), i.e. the same update with alpha_t = beta_t ("rule" 1 below).
+ *
  * Readings where the pages are silent:
  *   - alpha is evaluated as -expm1(-beta*lambda)/lambda, which is the same
  *     number without the cancellation of 1 - exp(x) for small x; at
@@ -48,6 +53,12 @@ double efla_oracle_alpha(double lambda, double beta)
     return -expm1(-beta * lambda) / lambda;
 }
 
+/* The coefficient of the rank-1 update under a rule: 0 = exact flow, 1 = Euler step. */
+double efla_oracle_coeff(double lambda, double beta, int rule)
+{
+    return rule == 1 ? beta : efla_oracle_alpha(lambda, beta);
+}
+
 /*
  * One token of the recurrence on one head, in place.
  *   S  : dk x dv, row-major (S[i*dv + j]), updated to S_t
@@ -55,12 +66,12 @@ double efla_oracle_alpha(double lambda, double beta)
  *   x  : scratch of length dv supplied by the caller
  */
 static void step_one(int dk, int dv, double *S, const double *q, const double *k,
-                     const double *v, double beta, double *o, double *x)
+                     const double *v, double beta, double *o, double *x, int rule)
 {
     double lambda = 0.0;
     for (int i = 0; i < dk; ++i)
         lambda += k[i] * k[i];
-    const double alpha = efla_oracle_alpha(lambda, beta);
+    const double alpha = efla_oracle_coeff(lambda, beta, rule);
 
     /* x = S^T k  (so that (I - alpha k k^T) S = S - alpha k x^T) */
     for (int j = 0; j < dv; ++j)
@@ -87,11 +98,11 @@ static void step_one(int dk, int dv, double *S, const double *q, const double *k
 }
 
 /*
- * Single token on a single head (the decode form).  S is updated in place.
- * Returns alpha_t.
+ * Single token on a single head (the decode form) under a rule.  S is updated
+ * in place.  Returns the coefficient used.
  */
-double efla_oracle_step(int dk, int dv, double *S, const double *q, const double *k,
-                        const double *v, double beta, double *o)
+double efla_oracle_step_rule(int dk, int dv, double *S, const double *q, const double *k,
+                             const double *v, double beta, double *o, int rule)
 {
     double *x = (double *)malloc(sizeof(double) * (size_t)(dv > 0 ? dv : 1));
     if (!x)
@@ -99,9 +110,16 @@ double efla_oracle_step(int dk, int dv, double *S, const double *q, const double
     double lambda = 0.0;
     for (int i = 0; i < dk; ++i)
         lambda += k[i] * k[i];
-    step_one(dk, dv, S, q, k, v, beta, o, x);
+    step_one(dk, dv, S, q, k, v, beta, o, x, rule);
     free(x);
-    return efla_oracle_alpha(lambda, beta);
+    return efla_oracle_coeff(lambda, beta, rule);
+}
+
+/* The exact-flow step (rule 0).  Returns alpha_t. */
+double efla_oracle_step(int dk, int dv, double *S, const double *q, const double *k,
+                        const double *v, double beta, double *o)
+{
+    return efla_oracle_step_rule(dk, dv, S, q, k, v, beta, o, 0);
 }
 
 /* ---- whole forward pass over [B, H, L, d] tensors ---------------------- */
@@ -110,6 +128,7 @@ typedef struct {
     int B, H, L, dk, dv;
     const double *q, *k, *v, *beta, *S0;
     double *o, *S_final;
+    int rule;
     int next_head; /* shared work counter */
     pthread_mutex_t lock;
     int failed;
@@ -132,7 +151,7 @@ static void run_head(fwd_job *J, int bh)
     for (int t = 0; t < L; ++t) {
         const size_t tok = (size_t)bh * L + t;
         step_one(dk, dv, S, J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
-                 J->beta[tok], J->o ? J->o + tok * dv : NULL, x);
+                 J->beta[tok], J->o ? J->o + tok * dv : NULL, x, J->rule);
     }
     free(x);
 }
@@ -158,12 +177,13 @@ static void *worker(void *arg)
  *   o may be NULL (state only).  nthreads <= 0 means one thread.
  * Returns 0 on success, -1 on allocation failure.
  */
-int efla_oracle_fwd(int B, int H, int L, int dk, int dv, const double *q, const double *k,
-                    const double *v, const double *beta, const double *S0, double *o,
-                    double *S_final, int nthreads)
+int efla_oracle_fwd_rule(int B, int H, int L, int dk, int dv, const double *q, const double *k,
+                         const double *v, const double *beta, const double *S0, double *o,
+                         double *S_final, int nthreads, int rule)
 {
     fwd_job J;
     J.B = B; J.H = H; J.L = L; J.dk = dk; J.dv = dv;
+    J.rule = rule;
     J.q = q; J.k = k; J.v = v; J.beta = beta; J.S0 = S0;
     J.o = o; J.S_final = S_final;
     J.next_head = 0;
@@ -187,4 +207,12 @@ int efla_oracle_fwd(int B, int H, int L, int dk, int dv, const double *q, const 
     free(th);
     pthread_mutex_destroy(&J.lock);
     return J.failed ? -1 : 0;
+}
+
+/* The exact-flow forward pass (rule 0). */
+int efla_oracle_fwd(int B, int H, int L, int dk, int dv, const double *q, const double *k,
+                    const double *v, const double *beta, const double *S0, double *o,
+                    double *S_final, int nthreads)
+{
+    return efla_oracle_fwd_rule(B, H, L, dk, dv, q, k, v, beta, S0, o, S_final, nthreads, 0);
 }
