@@ -156,7 +156,7 @@ def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
     cores = os.cpu_count() or 1
     x = inputs.make_inputs(inputs.workload(w.id, B=1, H=1))
     t0 = time.perf_counter()
-    oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], nthreads=1)
+    oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], nthreads=1, rule=RULE)
     t_head = max(time.perf_counter() - t0, 1e-3)
     # about `seconds_target` of wall time with every core busy on whole heads
     heads = max(1, min(w.B * w.H, cores * max(1, int(seconds_target / t_head))))
@@ -164,13 +164,17 @@ def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
     B = max(1, min(w.B, heads // H))
     xs = inputs.make_inputs(inputs.workload(w.id, B=B, H=H))
     threads = min(cores, B * H)
+    # repeat the sample until it amounts to ~seconds_target of CPU work (core-seconds)
+    reps, dt = 0, 0.0
     t0 = time.perf_counter()
-    oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
-    dt = time.perf_counter() - t0
-    n = B * H * w.L
+    while reps < 50 and (reps == 0 or dt * threads < seconds_target):
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
+        reps += 1
+        dt = time.perf_counter() - t0
+    n = B * H * w.L * reps
     return {"value": n / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": "%d of %d heads (B=%d, H=%d) at full L=%d, fp64 token-by-token, %.1f s"
-                      % (B * H, w.B * w.H, B, H, w.L, dt)}
+            "sample": "%d of %d heads (B=%d, H=%d) at full L=%d, %d pass(es), fp64 token-by-token, "
+                      "%.1f s on %d threads" % (B * H, w.B * w.H, B, H, w.L, reps, dt, threads)}
 
 
 def run_reference(args) -> None:
@@ -187,10 +191,10 @@ def run_reference(args) -> None:
     xs = inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 1024)))
     threads = min(cores, H)
     for _ in range(args.warmup):
-        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads)
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
     dt = time.perf_counter() - t0
     n = H * xs["q"].shape[2] * args.steps
     val = n / dt
@@ -207,12 +211,15 @@ def run_reference(args) -> None:
     }), flush=True)
 
 
+RULE = "exact"  # set from --rule: "exact" (the method) or "euler" (the delta rule, for comparison)
+
+
 def _config(w) -> dict:
     c = {"workload": "%s (B=%d H=%d L=%d dk=%d dv=%d chunk=%d %s)" % (
         w.name, w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.dtype),
         "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
         "l2": "inputs > L2 (126 MB): two rotating input sets per rank",
-        "o_dtype": "fp32"}
+        "o_dtype": "fp32", "rule": RULE}
     if w.decode:
         c["decode"] = "B=%d H=%d one token, fp32 carried state" % (w.decode["B"], w.decode["H"])
     return c
@@ -249,7 +256,8 @@ def run_ours(args) -> None:
               if k != "prefix"}
         p = d["prefix"]
         pd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in p.items()}
-        _, S_carry = efla.chunk_fwd(pd["q"], pd["k"], pd["v"], pd["beta"], None, chunk=w.chunk)
+        _, S_carry = efla.chunk_fwd(pd["q"], pd["k"], pd["v"], pd["beta"], None, chunk=w.chunk,
+                                    rule=RULE)
         dd["S_init"] = S_carry
         dd["S"] = [S_carry.clone(), S_carry.clone()]
         dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=torch.float32, device=dev)
@@ -264,12 +272,12 @@ def run_ours(args) -> None:
         if ev_pair is not None:
             ev_pair[0].record(stream)
         efla.chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], chunk=w.chunk,
-                       o=o_buf[i % 2], S_final=Sf_buf[i % 2], workspace=wsp)
+                       o=o_buf[i % 2], S_final=Sf_buf[i % 2], workspace=wsp, rule=RULE)
         if ev_pair is not None:
             ev_pair[1].record(stream)
         if dec is not None:
             efla.recurrent_step(dec["q"], dec["k"], dec["v"], dec["beta"], dec["S"][i % 2],
-                                o=dec["o"])
+                                o=dec["o"], rule=RULE)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -328,13 +336,14 @@ def run_ours(args) -> None:
         def e2e_step():
             g = {k: xh[k].to(dev, non_blocking=True) for k in ("q", "k", "v", "beta")}
             o, S = efla.chunk_fwd(g["q"], g["k"], g["v"], g["beta"], None, chunk=w.chunk,
-                                  o=o_buf[0], S_final=Sf_buf[0], workspace=wsp)
+                                  o=o_buf[0], S_final=Sf_buf[0], workspace=wsp, rule=RULE)
             o_host.copy_(o, non_blocking=True)
             S_host.copy_(S, non_blocking=True)
             if dec is not None:
                 gd = {k: dh[k].to(dev, non_blocking=True) for k in dh}
                 Sd = S_dec_host.to(dev, non_blocking=True)
-                od = efla.recurrent_step(gd["q"], gd["k"], gd["v"], gd["beta"], Sd, o=dec["o"])
+                od = efla.recurrent_step(gd["q"], gd["k"], gd["v"], gd["beta"], Sd, o=dec["o"],
+                                         rule=RULE)
                 od_host.copy_(od, non_blocking=True)
                 S_dec_host.copy_(Sd, non_blocking=True)
 
@@ -385,7 +394,13 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rule", choices=["exact", "euler"], default="exact",
+                    help="update rule: the exact flow (default) or the delta rule's Euler step, "
+                         "for the throughput comparison (the workload's keys are not normalised, "
+                         "so under euler only the time is meaningful)")
     args = ap.parse_args()
+    global RULE
+    RULE = args.rule
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -15,7 +15,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) alpha_kernel(const T *__restrict__ k,
                                                     const T *__restrict__ beta,
                                                     float *__restrict__ alpha, long long ntok,
-                                                    int dk) {
+                                                    int dk, bool euler) {
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntok;
@@ -27,21 +27,22 @@ __global__ void __launch_bounds__(256) alpha_kernel(const T *__restrict__ k,
             s = fmaf(x, x, s);
         }
         s = warp_sum(s);
-        if (lane == 0) alpha[t] = alpha_from(s, to_f32(beta[t]));
+        if (lane == 0) alpha[t] = alpha_rule(s, to_f32(beta[t]), euler);
     }
 }
 
 cudaError_t launch_alpha(const void *k, const void *beta, float *alpha, long long ntok, int dk,
-                         bool is_bf16, cudaStream_t s) {
+                         bool is_bf16, bool euler, cudaStream_t s) {
     if (ntok <= 0) return cudaSuccess;
     long long blocks = (ntok + 7) / 8;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
     if (is_bf16)
         alpha_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, alpha, ntok, dk);
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, alpha, ntok, dk, euler);
     else
         alpha_kernel<float><<<(unsigned)blocks, 256, 0, s>>>((const float *)k,
-                                                             (const float *)beta, alpha, ntok, dk);
+                                                             (const float *)beta, alpha, ntok, dk,
+                                                             euler);
     count_launches(1);
     return cudaGetLastError();
 }

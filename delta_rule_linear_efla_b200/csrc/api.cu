@@ -28,6 +28,8 @@ bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
 
 bool dtype_ok(efla_dtype d) { return d == EFLA_F32 || d == EFLA_BF16; }
 
+bool rule_ok(efla_rule r) { return r == EFLA_RULE_EXACT || r == EFLA_RULE_EULER; }
+
 }  // namespace
 
 extern "C" {
@@ -44,14 +46,16 @@ const char *efla_status_str(int status) {
         case EFLA_ERR_WORKSPACE: return "workspace missing or too small";
         case EFLA_ERR_ALIGN: return "pointer not aligned as required";
         case EFLA_ERR_TOO_LARGE: return "sizes exceed the fixed scratch of efla_chunk_fwd_noalloc";
+        case EFLA_ERR_RULE: return "unknown update rule";
         default: return "unknown status";
     }
 }
 
 int efla_version(void) { return 100; /* 0.1.0 */ }
 
-efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int H, int L, int dk,
-                       efla_dtype dt, void *stream) {
+efla_status efla_alpha_rule(const void *k, const void *beta, float *alpha, int B, int H, int L,
+                            int dk, efla_dtype dt, efla_rule rule, void *stream) {
+    if (!rule_ok(rule)) return EFLA_ERR_RULE;
     if (dt != EFLA_F32 && dt != EFLA_BF16) return EFLA_ERR_DTYPE;
     if (B < 0 || H < 0 || L < 0 || dk < 1) return EFLA_ERR_SHAPE;
     if (dk > 256) return EFLA_ERR_UNSUPPORTED;
@@ -61,7 +65,12 @@ efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int
     if (!aligned_elem(k, dt) || !aligned_elem(beta, dt) || !aligned_elem(alpha, EFLA_F32))
         return EFLA_ERR_ALIGN;
     return from_cuda(efla::launch_alpha(k, beta, alpha, ntok, dk, dt == EFLA_BF16,
-                                        (cudaStream_t)stream));
+                                        rule == EFLA_RULE_EULER, (cudaStream_t)stream));
+}
+
+efla_status efla_alpha(const void *k, const void *beta, float *alpha, int B, int H, int L, int dk,
+                       efla_dtype dt, void *stream) {
+    return efla_alpha_rule(k, beta, alpha, B, H, L, dk, dt, EFLA_RULE_EXACT, stream);
 }
 
 int efla_chunk_fwd_path(int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
@@ -80,10 +89,13 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
     return 0;
 }
 
-efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
-                           const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
-                           int dv, int chunk, efla_dtype dt, efla_dtype o_dt, void *workspace,
-                           size_t workspace_bytes, void *stream) {
+efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, const void *beta,
+                                const float *S0, void *o, float *S_final, int B, int H, int L,
+                                int dk, int dv, int chunk, efla_dtype dt, efla_dtype o_dt,
+                                efla_rule rule, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    if (!rule_ok(rule)) return EFLA_ERR_RULE;
+    const bool euler = rule == EFLA_RULE_EULER;
     if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
     if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
@@ -106,15 +118,24 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
         if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
         if (!aligned16(workspace)) return EFLA_ERR_ALIGN;
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
-                                               chunk, o_bf16, workspace, s));
+                                               chunk, o_bf16, euler, workspace, s));
     }
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
-                                             chunk, bf16, o_bf16, s));
+                                             chunk, bf16, o_bf16, euler, s));
 }
 
-efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
-                                float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
-                                efla_dtype o_dt, void *stream) {
+efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
+                           const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
+                           int dv, int chunk, efla_dtype dt, efla_dtype o_dt, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    return efla_chunk_fwd_rule(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, dt, o_dt,
+                               EFLA_RULE_EXACT, workspace, workspace_bytes, stream);
+}
+
+efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v, const void *beta,
+                                     float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
+                                     efla_dtype o_dt, efla_rule rule, void *stream) {
+    if (!rule_ok(rule)) return EFLA_ERR_RULE;
     if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
     if ((long long)B * H > 0x7fffffffLL) return EFLA_ERR_SHAPE;
@@ -124,7 +145,15 @@ efla_status efla_recurrent_step(const void *q, const void *k, const void *v, con
         !aligned_elem(beta, dt) || !aligned16(S) || !aligned_elem(o, o_dt))
         return EFLA_ERR_ALIGN;
     return from_cuda(efla::launch_decode(q, k, v, beta, S, o, B * H, dk, dv, dt == EFLA_BF16,
-                                         o_dt == EFLA_BF16, (cudaStream_t)stream));
+                                         o_dt == EFLA_BF16, rule == EFLA_RULE_EULER,
+                                         (cudaStream_t)stream));
+}
+
+efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
+                                float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
+                                efla_dtype o_dt, void *stream) {
+    return efla_recurrent_step_rule(q, k, v, beta, S, o, B, H, dk, dv, dt, o_dt, EFLA_RULE_EXACT,
+                                    stream);
 }
 
 unsigned long long efla_kernel_launches(void) {

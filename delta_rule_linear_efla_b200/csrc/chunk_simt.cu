@@ -51,7 +51,8 @@ template <typename T, typename TO>
 __global__ void __launch_bounds__(SIMT_THREADS)
     chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const T *__restrict__ beta, const float *__restrict__ S0, TO *__restrict__ o,
-                      float *__restrict__ S_final, int L, int dk, int dv, int C, int NV) {
+                      float *__restrict__ S_final, int L, int dk, int dv, int C, int NV,
+                      bool euler) {
     extern __shared__ float sm[];
     const SimtSmem lay(dk, C, NV);
     float *Ks = sm + lay.off_K, *Qs = sm + lay.off_Q, *Ws = sm + lay.off_W;
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
             float s = 0.f;
             for (int d = lane; d < dk; d += 32) s = fmaf(Ks[i * dkp + d], Ks[i * dkp + d], s);
             s = warp_sum(s);
-            if (lane == 0) al[i] = alpha_from(s, to_f32(beta[row0 + i]));
+            if (lane == 0) al[i] = alpha_rule(s, to_f32(beta[row0 + i]), euler);
         }
         __syncthreads();
         // A = strictly-lower(diag(alpha) K K^T) and P = lower-incl-diag(Q K^T)
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
 template <typename T, typename TO>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const void *beta,
                                  const float *S0, void *o, float *S_final, int B, int H, int L,
-                                 int dk, int dv, int chunk, cudaStream_t s) {
+                                 int dk, int dv, int chunk, bool euler, cudaStream_t s) {
     const int NV = dv < SIMT_NV ? dv : SIMT_NV;
     const SimtSmem lay(dk, chunk, NV);
     dim3 grid(B * H, (dv + NV - 1) / NV);
@@ -191,21 +192,21 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
     if (e != cudaSuccess) return e;
     chunk_simt_kernel<T, TO><<<grid, SIMT_THREADS, lay.total, s>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S0, (TO *)o, S_final, L, dk,
-        dv, chunk, NV);
+        dv, chunk, NV, euler);
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
                               const float *S0, void *o, float *S_final, int B, int H, int L,
-                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16,
+                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16, bool euler,
                               cudaStream_t s) {
     using bf = __nv_bfloat16;
     if (is_bf16)
-        return o_bf16 ? launch_simt_t<bf, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s)
-                      : launch_simt_t<bf, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s);
-    return o_bf16 ? launch_simt_t<float, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s)
-                  : launch_simt_t<float, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, s);
+        return o_bf16 ? launch_simt_t<bf, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, euler, s)
+                      : launch_simt_t<bf, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, euler, s);
+    return o_bf16 ? launch_simt_t<float, bf>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, euler, s)
+                  : launch_simt_t<float, float>(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, euler, s);
 }
 
 }  // namespace efla

@@ -100,7 +100,7 @@ __device__ __forceinline__ void load_b(uint32_t &b0, uint32_t &b1, const __half 
 template <int DK>
 __global__ void __launch_bounds__(THREADS)
     tc_prep_kernel(const __grid_constant__ CUtensorMap tmap_k, const __nv_bfloat16 *__restrict__ beta,
-                   __half *__restrict__ ta_out, int L, int NC, int total) {
+                   __half *__restrict__ ta_out, int L, int NC, int total, bool euler) {
     using namespace prep;
     constexpr int KB = Smem::k_bytes<DK>();
     extern __shared__ uint8_t smem_raw[];
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(THREADS)
                     }
                 }
             }
-            al[r] = alpha_from(sq, beta_row);
+            al[r] = alpha_rule(sq, beta_row, euler);
         }
         ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }  // also: every norm has been read
@@ -1012,8 +1012,8 @@ TcDevInfo tc_dev_info() {
 
 template <int DK, int DV, typename TO>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void *beta,
-                        const float *S0, void *o, float *S_final, int B, int H, int L, void *ws,
-                        cudaStream_t s) {
+                        const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
+                        void *ws, cudaStream_t s) {
     const int BH = B * H, NC = (L + C - 1) / C, total = BH * NC;
     const TcDevInfo di = tc_dev_info<DK, DV, TO>();
     if (di.err != cudaSuccess) return di.err;
@@ -1024,7 +1024,7 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         return cudaErrorInvalidValue;
     const int pgrid = total < di.prep_grid ? total : di.prep_grid;
     tc_prep_kernel<DK><<<pgrid, THREADS, prep_smem_bytes<DK>(), s>>>(mk, (const __nv_bfloat16 *)beta,
-                                                                      (__half *)ws, L, NC, total);
+                                                                      (__half *)ws, L, NC, total, euler);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     constexpr int SSM = StateLayout<DK, DV>::SMEM;
@@ -1054,9 +1054,9 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
 template <int DK, int DV>
 cudaError_t launch_tc_o(const void *q, const void *k, const void *v, const void *beta,
                         const float *S0, void *o, float *S_final, int B, int H, int L, bool o_bf16,
-                        void *ws, cudaStream_t s) {
-    return o_bf16 ? launch_tc_t<DK, DV, __nv_bfloat16>(q, k, v, beta, S0, o, S_final, B, H, L, ws, s)
-                  : launch_tc_t<DK, DV, float>(q, k, v, beta, S0, o, S_final, B, H, L, ws, s);
+                        bool euler, void *ws, cudaStream_t s) {
+    return o_bf16 ? launch_tc_t<DK, DV, __nv_bfloat16>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s)
+                  : launch_tc_t<DK, DV, float>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s);
 }
 
 }  // namespace
@@ -1091,15 +1091,16 @@ int tc_segments(int B, int H, int L, int dk, int dv) {
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
                             const float *S0, void *o, float *S_final, int B, int H, int L,
-                            int dk, int dv, int chunk, bool o_bf16, void *ws, cudaStream_t s) {
+                            int dk, int dv, int chunk, bool o_bf16, bool euler, void *ws,
+                            cudaStream_t s) {
     (void)chunk;
     if (dk == 128 && dv == 128)
-        return launch_tc_o<128, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, ws, s);
+        return launch_tc_o<128, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
     if (dk == 128 && dv == 64)
-        return launch_tc_o<128, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, ws, s);
+        return launch_tc_o<128, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
     if (dk == 64 && dv == 128)
-        return launch_tc_o<64, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, ws, s);
-    return launch_tc_o<64, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, ws, s);
+        return launch_tc_o<64, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
+    return launch_tc_o<64, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
 }
 
 cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s) {

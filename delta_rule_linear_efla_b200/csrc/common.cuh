@@ -30,6 +30,13 @@ __device__ __forceinline__ float alpha_from(float lambda, float beta) {
     return -expm1f(-x) / lambda;
 }
 
+// The coefficient under the selected rule: the exact flow above, or the explicit Euler
+// step of the same ODE ("Exact Flow Linear Attention", technical summary, Key
+// Contributions: the delta rule is that Euler step), whose coefficient is beta itself.
+__device__ __forceinline__ float alpha_rule(float lambda, float beta, bool euler) {
+    return euler ? beta : alpha_from(lambda, beta);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -27,7 +27,8 @@ struct DecodeCfg {
 template <typename T, typename TO, int DK, int DV>
 __global__ void __launch_bounds__(DecodeCfg<T, DK, DV>::NT)
     decode_reg_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const T *__restrict__ beta, float *__restrict__ S, TO *__restrict__ o) {
+                      const T *__restrict__ beta, float *__restrict__ S, TO *__restrict__ o,
+                      bool euler) {
     using Cfg = DecodeCfg<T, DK, DV>;
     constexpr int TPR = Cfg::TPR, RPP = Cfg::RPP, PASSES = Cfg::PASSES, NT = Cfg::NT;
     __shared__ float ks[DK], qs[DK], vs[DV];
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, DK, DV>::NT)
         l = warp_sum(l);
         kq = warp_sum(kq);
         if (tid == 0) {
-            sc[0] = alpha_from(l, to_f32(beta[bh]));
+            sc[0] = alpha_rule(l, to_f32(beta[bh]), euler);
             sc[1] = kq;
         }
     }
@@ -102,7 +103,7 @@ template <typename T, typename TO>
 __global__ void __launch_bounds__(256)
     decode_generic_kernel(const T *__restrict__ q, const T *__restrict__ k,
                           const T *__restrict__ v, const T *__restrict__ beta,
-                          float *__restrict__ S, TO *__restrict__ o, int dk, int dv) {
+                          float *__restrict__ S, TO *__restrict__ o, int dk, int dv, bool euler) {
     __shared__ float ks[256], qs[256];
     __shared__ float sc[2];
     const int bh = blockIdx.x, tid = threadIdx.x;
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(256)
         l = warp_sum(l);
         kq = warp_sum(kq);
         if (tid == 0) {
-            sc[0] = alpha_from(l, to_f32(beta[bh]));
+            sc[0] = alpha_rule(l, to_f32(beta[bh]), euler);
             sc[1] = kq;
         }
     }
@@ -141,50 +142,50 @@ __global__ void __launch_bounds__(256)
 
 template <typename T, typename TO, int DK, int DV>
 static void launch_reg(const void *q, const void *k, const void *v, const void *beta, float *S,
-                       void *o, int BH, cudaStream_t s) {
+                       void *o, int BH, bool euler, cudaStream_t s) {
     decode_reg_kernel<T, TO, DK, DV><<<BH, DecodeCfg<T, DK, DV>::NT, 0, s>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S, (TO *)o);
+        (const T *)q, (const T *)k, (const T *)v, (const T *)beta, S, (TO *)o, euler);
 }
 
 template <typename T, typename TO, int DK>
 static bool dispatch_dv(const void *q, const void *k, const void *v, const void *beta, float *S,
-                        void *o, int BH, int dv, cudaStream_t s) {
+                        void *o, int BH, int dv, bool euler, cudaStream_t s) {
     switch (dv) {
-        case 16: launch_reg<T, TO, DK, 16>(q, k, v, beta, S, o, BH, s); return true;
-        case 32: launch_reg<T, TO, DK, 32>(q, k, v, beta, S, o, BH, s); return true;
-        case 64: launch_reg<T, TO, DK, 64>(q, k, v, beta, S, o, BH, s); return true;
-        case 128: launch_reg<T, TO, DK, 128>(q, k, v, beta, S, o, BH, s); return true;
+        case 16: launch_reg<T, TO, DK, 16>(q, k, v, beta, S, o, BH, euler, s); return true;
+        case 32: launch_reg<T, TO, DK, 32>(q, k, v, beta, S, o, BH, euler, s); return true;
+        case 64: launch_reg<T, TO, DK, 64>(q, k, v, beta, S, o, BH, euler, s); return true;
+        case 128: launch_reg<T, TO, DK, 128>(q, k, v, beta, S, o, BH, euler, s); return true;
         default: return false;
     }
 }
 
 template <typename T, typename TO>
 static void dispatch(const void *q, const void *k, const void *v, const void *beta, float *S,
-                     void *o, int BH, int dk, int dv, cudaStream_t s) {
+                     void *o, int BH, int dk, int dv, bool euler, cudaStream_t s) {
     bool done = false;
     switch (dk) {
-        case 16: done = dispatch_dv<T, TO, 16>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 32: done = dispatch_dv<T, TO, 32>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 64: done = dispatch_dv<T, TO, 64>(q, k, v, beta, S, o, BH, dv, s); break;
-        case 128: done = dispatch_dv<T, TO, 128>(q, k, v, beta, S, o, BH, dv, s); break;
+        case 16: done = dispatch_dv<T, TO, 16>(q, k, v, beta, S, o, BH, dv, euler, s); break;
+        case 32: done = dispatch_dv<T, TO, 32>(q, k, v, beta, S, o, BH, dv, euler, s); break;
+        case 64: done = dispatch_dv<T, TO, 64>(q, k, v, beta, S, o, BH, dv, euler, s); break;
+        case 128: done = dispatch_dv<T, TO, 128>(q, k, v, beta, S, o, BH, dv, euler, s); break;
         default: break;
     }
     if (!done)
         decode_generic_kernel<T, TO><<<BH, 256, 0, s>>>((const T *)q, (const T *)k, (const T *)v,
-                                                        (const T *)beta, S, (TO *)o, dk, dv);
+                                                        (const T *)beta, S, (TO *)o, dk, dv, euler);
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
                           float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
-                          cudaStream_t s) {
+                          bool euler, cudaStream_t s) {
     using bf = __nv_bfloat16;
     if (BH <= 0) return cudaSuccess;
     if (is_bf16) {
-        if (o_bf16) dispatch<bf, bf>(q, k, v, beta, S, o, BH, dk, dv, s);
-        else dispatch<bf, float>(q, k, v, beta, S, o, BH, dk, dv, s);
+        if (o_bf16) dispatch<bf, bf>(q, k, v, beta, S, o, BH, dk, dv, euler, s);
+        else dispatch<bf, float>(q, k, v, beta, S, o, BH, dk, dv, euler, s);
     } else {
-        if (o_bf16) dispatch<float, bf>(q, k, v, beta, S, o, BH, dk, dv, s);
-        else dispatch<float, float>(q, k, v, beta, S, o, BH, dk, dv, s);
+        if (o_bf16) dispatch<float, bf>(q, k, v, beta, S, o, BH, dk, dv, euler, s);
+        else dispatch<float, float>(q, k, v, beta, S, o, BH, dk, dv, euler, s);
     }
     count_launches(1);
     return cudaGetLastError();

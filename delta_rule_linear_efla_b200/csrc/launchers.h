@@ -13,21 +13,22 @@ void count_launches(unsigned n);
 
 // Per-token alpha (fused norm + closed-form coefficient).  is_bf16 selects the
 // element type of k and beta.
+// euler: the coefficient is beta (the delta rule's explicit Euler step) instead of the exact flow's.
 cudaError_t launch_alpha(const void *k, const void *beta, float *alpha, long long ntok, int dk,
-                         bool is_bf16, cudaStream_t s);
+                         bool is_bf16, bool euler, cudaStream_t s);
 
 // SIMT fp32 chunkwise forward: WY/UT per chunk, state carried in fp32.
 // Any dk, dv <= 128 and chunk <= 64.
 // o_bf16 selects the output element type (fp32 or bf16).
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
                               const float *S0, void *o, float *S_final, int B, int H, int L,
-                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16,
+                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16, bool euler,
                               cudaStream_t s);
 
 // Recurrent single-token step per head (decode), S updated in place.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
                           float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
-                          cudaStream_t s);
+                          bool euler, cudaStream_t s);
 
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
@@ -35,7 +36,8 @@ size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
 int tc_segments(int B, int H, int L, int dk, int dv);  // sequence segments the launch uses (1: none)
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
                             const float *S0, void *o, float *S_final, int B, int H, int L,
-                            int dk, int dv, int chunk, bool o_bf16, void *ws, cudaStream_t s);
+                            int dk, int dv, int chunk, bool o_bf16, bool euler, void *ws,
+                            cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits): read and clear.
 cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s);
 

@@ -17,12 +17,15 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libefla.so")
 
 EFLA_F32, EFLA_BF16 = 0, 1
+# Update rules: the exact flow (the method) and the delta rule's explicit Euler step.
+RULES = {"exact": 0, "euler": 1}
 
 # Every extern "C" symbol declared in include/efla.h.
 ABI_SYMBOLS = (
     "efla_status_str", "efla_version", "efla_alpha", "efla_chunk_fwd_workspace_size",
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
-    "efla_kernel_launches", "efla_chunk_fwd_noalloc",
+    "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
+    "efla_recurrent_step_rule",
 )
 
 _lib = None
@@ -65,6 +68,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_kernel_launches.argtypes = []
     L.efla_chunk_fwd_noalloc.restype = i
     L.efla_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+    L.efla_alpha_rule.restype = i
+    L.efla_alpha_rule.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp]
+    L.efla_chunk_fwd_rule.restype = i
+    L.efla_chunk_fwd_rule.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz, vp]
+    L.efla_recurrent_step_rule.restype = i
+    L.efla_recurrent_step_rule.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     if path is None:
         _lib = L
     return L
@@ -91,6 +100,12 @@ def _dtype_code(t: torch.Tensor) -> int:
     return _code(t.dtype)
 
 
+def _rule(rule: str) -> int:
+    if rule not in RULES:
+        raise ValueError("rule must be one of %s, got %r" % (sorted(RULES), rule))
+    return RULES[rule]
+
+
 def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
@@ -107,16 +122,19 @@ def _stream_handle(stream) -> int:
     return stream.cuda_stream
 
 
-def alpha(k: torch.Tensor, beta: torch.Tensor, out: torch.Tensor | None = None, stream=None):
-    """alpha_t = -expm1(-beta_t ||k_t||^2)/||k_t||^2 (beta_t at ||k_t|| = 0); [B,H,L] fp32."""
+def alpha(k: torch.Tensor, beta: torch.Tensor, out: torch.Tensor | None = None, stream=None,
+          rule: str = "exact"):
+    """alpha_t = -expm1(-beta_t ||k_t||^2)/||k_t||^2 (beta_t at ||k_t|| = 0); [B,H,L] fp32.
+    rule="euler" gives the delta rule's coefficient, alpha_t = beta_t."""
     B, H, L, dk = k.shape
     if beta.shape != (B, H, L) or beta.dtype != k.dtype:
         raise ValueError("beta must be [B,H,L] with k's dtype")
     if out is None:
         out = torch.empty((B, H, L), dtype=torch.float32, device=k.device)
-    _check(load_library().efla_alpha(_dev(k, "k"), _dev(beta, "beta"),
-                                      _dev(out, "alpha", torch.float32), B, H, L, dk,
-                                      _dtype_code(k), _stream_handle(stream)), "efla_alpha")
+    _check(load_library().efla_alpha_rule(_dev(k, "k"), _dev(beta, "beta"),
+                                           _dev(out, "alpha", torch.float32), B, H, L, dk,
+                                           _dtype_code(k), _rule(rule), _stream_handle(stream)),
+           "efla_alpha_rule")
     return out
 
 
@@ -132,8 +150,10 @@ def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype, o_dtype=torch.float32) -> str:
 
 
 def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
-              want_state: bool = True, workspace=None, o_dtype=torch.float32, stream=None):
+              want_state: bool = True, workspace=None, o_dtype=torch.float32, stream=None,
+              rule: str = "exact"):
     """EFLA forward in the WY/UT chunkwise form.  Returns (o, S_final or None).
+    rule="euler" runs the same kernels with the delta rule's coefficient alpha = beta.
 
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L], all float32 or all bfloat16 on one
     CUDA device; S0: [B,H,dk,dv] float32 or None.  o is float32 by default (the fp32
@@ -159,13 +179,14 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
     ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
-    st = load_library().efla_chunk_fwd(
+    st = load_library().efla_chunk_fwd_rule(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
         _dev(S0, "S0", torch.float32) if S0 is not None else None,
         _dev(o, "o", o_dtype),
         _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
-        B, H, L, dk, dv, int(chunk), code, o_code, ws_ptr, ws_bytes, _stream_handle(stream))
-    _check(st, "efla_chunk_fwd")
+        B, H, L, dk, dv, int(chunk), code, o_code, _rule(rule), ws_ptr, ws_bytes,
+        _stream_handle(stream))
+    _check(st, "efla_chunk_fwd_rule")
     return o, S_final
 
 
@@ -183,9 +204,11 @@ def chunk_fwd_noalloc(q, k, v, beta, o, S_final=None, S0=None, chunk: int = 64, 
     return o, S_final
 
 
-def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None):
+def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None,
+                   rule: str = "exact"):
     """One decode token per head; S ([B,H,dk,dv] float32) is updated in place.  Returns o
-    (float32 by default, or bfloat16 with o_dtype=torch.bfloat16)."""
+    (float32 by default, or bfloat16 with o_dtype=torch.bfloat16).  rule="euler" takes the
+    delta rule's step (alpha = beta)."""
     B, H, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:2] != (B, H) or beta.shape != (B, H) or \
@@ -196,11 +219,11 @@ def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None)
         o_dtype = o.dtype
     if o is None:
         o = torch.empty((B, H, dv), dtype=o_dtype, device=q.device)
-    st = load_library().efla_recurrent_step(
+    st = load_library().efla_recurrent_step_rule(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
         _dev(S, "S", torch.float32), _dev(o, "o", o_dtype), B, H, dk, dv, code, _code(o_dtype),
-        _stream_handle(stream))
-    _check(st, "efla_recurrent_step")
+        _rule(rule), _stream_handle(stream))
+    _check(st, "efla_recurrent_step_rule")
     return o
 
 

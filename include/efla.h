@@ -61,13 +61,31 @@ typedef enum {
     EFLA_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
     EFLA_ERR_WORKSPACE = 7,   /* workspace missing or smaller than the query said */
     EFLA_ERR_ALIGN = 8,       /* a pointer is not aligned as required */
-    EFLA_ERR_TOO_LARGE = 9    /* sizes need more than the fixed scratch of efla_chunk_fwd_noalloc */
+    EFLA_ERR_TOO_LARGE = 9,   /* sizes need more than the fixed scratch of efla_chunk_fwd_noalloc */
+    EFLA_ERR_RULE = 10        /* unknown efla_rule */
 } efla_status;
 
 typedef enum {
     EFLA_F32 = 0,  /* float32 inputs/outputs; all arithmetic in fp32 */
     EFLA_BF16 = 1  /* bfloat16 inputs/outputs; fp32 state and accumulation */
 } efla_dtype;
+
+/*
+ * Update rule.  Both integrate the same per-token ODE, dS/dtau = -k k^T S + k v^T
+ * over an interval of length beta_t (Methodology 1), and share every kernel,
+ * layout and error; they differ in the coefficient alpha_t of the rank-1 update
+ * S_t = (I - alpha_t k_t k_t^T) S_{t-1} + alpha_t k_t v_t^T:
+ *   EFLA_RULE_EXACT -- the exact flow, alpha_t = (1 - e^{-beta_t lambda_t}) /
+ *                      lambda_t (Methodology 3).  The method; the default of
+ *                      every entry point without a rule argument.
+ *   EFLA_RULE_EULER -- one explicit Euler step of the ODE, alpha_t = beta_t: the
+ *                      delta rule (DeltaNet), which the summary identifies as
+ *                      that Euler step (Key Contributions) and compares against.
+ */
+typedef enum {
+    EFLA_RULE_EXACT = 0,
+    EFLA_RULE_EULER = 1
+} efla_rule;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *efla_status_str(int status);
@@ -86,6 +104,12 @@ int efla_version(void);
  */
 efla_status efla_alpha(const void *k, const void *beta, float *alpha,
                        int B, int H, int L, int dk, efla_dtype dt, void *stream);
+
+/* efla_alpha under a chosen update rule (alpha = beta for EFLA_RULE_EULER).
+ * EFLA_ERR_RULE for an unknown rule; otherwise as efla_alpha. */
+efla_status efla_alpha_rule(const void *k, const void *beta, float *alpha,
+                            int B, int H, int L, int dk, efla_dtype dt, efla_rule rule,
+                            void *stream);
 
 /*
  * Bytes of device workspace efla_chunk_fwd needs for these sizes (0 when the
@@ -120,6 +144,15 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
                            int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
                            efla_dtype o_dt, void *workspace, size_t workspace_bytes,
                            void *stream);
+
+/* efla_chunk_fwd under a chosen update rule: the same kernels, workspace and
+ * paths, with alpha = beta for EFLA_RULE_EULER.  EFLA_ERR_RULE for an unknown
+ * rule; otherwise as efla_chunk_fwd. */
+efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, const void *beta,
+                                const float *S0, void *o, float *S_final,
+                                int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                                efla_dtype o_dt, efla_rule rule, void *workspace,
+                                size_t workspace_bytes, void *stream);
 
 /*
  * efla_chunk_fwd_noalloc -- the same forward pass as efla_chunk_fwd for callers
@@ -173,6 +206,14 @@ efla_status efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v, 
 efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
                                 float *S, void *o, int B, int H, int dk, int dv,
                                 efla_dtype dt, efla_dtype o_dt, void *stream);
+
+/* efla_recurrent_step under a chosen update rule (alpha = beta for
+ * EFLA_RULE_EULER).  EFLA_ERR_RULE for an unknown rule; otherwise as
+ * efla_recurrent_step. */
+efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v,
+                                     const void *beta, float *S, void *o, int B, int H, int dk,
+                                     int dv, efla_dtype dt, efla_dtype o_dt, efla_rule rule,
+                                     void *stream);
 
 /*
  * Reads and clears the library's device error word after synchronising

@@ -125,3 +125,14 @@ def test_workspace_reserves_segment_state(lib):
         ta + 16 * 8 * 3 * 128 * 128 * 4
     assert lib.efla_chunk_fwd_workspace_size(4, 16, 4096, 128, 128, 64, BF16, F32) == 4 * 16 * 64 * 8192
     assert lib.efla_chunk_fwd_workspace_size(1, 2, 4096, 128, 64, 64, BF16, F32) == 2 * 64 * 8192
+
+
+def test_unknown_rule_is_refused_on_the_host(lib):
+    P = ctypes.c_void_p(16)
+    EFLA_ERR_RULE = 10
+    assert lib.efla_alpha_rule(P, P, P, 1, 1, 4, 16, BF16, 2, None) == EFLA_ERR_RULE
+    assert lib.efla_chunk_fwd_rule(P, P, P, P, None, P, None, 1, 1, 64, 16, 16, 64, BF16, F32, 7,
+                                   None, 0, None) == EFLA_ERR_RULE
+    assert lib.efla_recurrent_step_rule(P, P, P, P, P, P, 1, 1, 16, 16, BF16, F32, -1,
+                                        None) == EFLA_ERR_RULE
+    assert "rule" in lib.efla_status_str(EFLA_ERR_RULE).decode()
