@@ -156,6 +156,19 @@ efla_status efla_recurrent_step(const void *q, const void *k, const void *v, con
                                     stream);
 }
 
+efla_status efla_state_affine(const float *P, const float *S_in, const float *Hm, float *S_out,
+                              int B, int H, int dk, int dv, void *stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
+    if ((long long)B * H * ((dv + 15) / 16) > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (dk > 256 || dv > 256) return EFLA_ERR_UNSUPPORTED;
+    if (!P || !S_out) return EFLA_ERR_NULL;
+    if (!aligned_elem(P, EFLA_F32) || !aligned_elem(S_in, EFLA_F32) || !aligned_elem(Hm, EFLA_F32) ||
+        !aligned_elem(S_out, EFLA_F32))
+        return EFLA_ERR_ALIGN;
+    return from_cuda(efla::launch_state_affine(P, S_in, Hm, S_out, B * H, dk, dv,
+                                               (cudaStream_t)stream));
+}
+
 unsigned long long efla_kernel_launches(void) {
     return efla::g_launches.load(std::memory_order_relaxed);
 }

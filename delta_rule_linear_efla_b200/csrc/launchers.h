@@ -30,6 +30,10 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
                           float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
                           bool euler, cudaStream_t s);
 
+// S_out = P S_in + H per head (fp32); S_in and H may be NULL (zero); S_out may alias S_in.
+cudaError_t launch_state_affine(const float *P, const float *S_in, const float *H, float *S_out,
+                                int BH, int dk, int dv, cudaStream_t s);
+
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
 size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);

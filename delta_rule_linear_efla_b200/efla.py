@@ -25,7 +25,7 @@ ABI_SYMBOLS = (
     "efla_status_str", "efla_version", "efla_alpha", "efla_chunk_fwd_workspace_size",
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
     "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
-    "efla_recurrent_step_rule",
+    "efla_recurrent_step_rule", "efla_state_affine",
 )
 
 _lib = None
@@ -72,6 +72,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_alpha_rule.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp]
     L.efla_chunk_fwd_rule.restype = i
     L.efla_chunk_fwd_rule.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz, vp]
+    L.efla_state_affine.restype = i
+    L.efla_state_affine.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
     L.efla_recurrent_step_rule.restype = i
     L.efla_recurrent_step_rule.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     if path is None:
@@ -225,6 +227,29 @@ def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None,
         _rule(rule), _stream_handle(stream))
     _check(st, "efla_recurrent_step_rule")
     return o
+
+
+def state_affine(P, S_in=None, H=None, out=None, stream=None):
+    """S_out = P S_in + H per head in fp32 (P [B,H,dk,dk]; S_in, H, out [B,H,dk,dv]; S_in or H
+    None means zero; out may be S_in).  Chains the affine state maps of sequence stretches."""
+    B, Hh, dk, dk2 = P.shape
+    if dk2 != dk:
+        raise ValueError("P must be [B,H,dk,dk]")
+    ref = S_in if S_in is not None else (H if H is not None else out)
+    if ref is None:
+        raise ValueError("one of S_in, H or out must give the value dimension")
+    dv = ref.shape[-1]
+    for name, t in (("S_in", S_in), ("H", H), ("out", out)):
+        if t is not None and t.shape != (B, Hh, dk, dv):
+            raise ValueError("%s must be [B,H,dk,dv]" % name)
+    if out is None:
+        out = torch.empty((B, Hh, dk, dv), dtype=torch.float32, device=P.device)
+    st = load_library().efla_state_affine(
+        _dev(P, "P", torch.float32), _dev(S_in, "S_in", torch.float32) if S_in is not None else None,
+        _dev(H, "H", torch.float32) if H is not None else None, _dev(out, "out", torch.float32),
+        B, Hh, dk, dv, _stream_handle(stream))
+    _check(st, "efla_state_affine")
+    return out
 
 
 def kernel_launches() -> int:

@@ -216,6 +216,23 @@ efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v
                                      void *stream);
 
 /*
+ * efla_state_affine -- S_out = P S_in + H for every head, in fp32.  No counterpart
+ * on the pages as a call: it chains the affine state maps of sequence stretches
+ * (a stretch of tokens maps the state as S_out = P S_in + H, where P is the
+ * product of the stretch's transitions I - alpha k k^T and H its state from zero,
+ * by the update rule of Methodology 3), so that stretches held by different GPUs
+ * can be run side by side and then given their true starting states.
+ *
+ *   P     : [B,H,dk,dk] fp32     S_in, H, S_out : [B,H,dk,dv] fp32
+ * S_in or H may be NULL (zero).  S_out may alias S_in (not P or H).
+ * Sizes: B,H >= 1, 1 <= dk,dv <= 256.  Pointers aligned to 4 bytes.
+ * P for a stretch is the S_final of efla_chunk_fwd run over it from S0 = I with
+ * v = 0 (dv = dk); H is its S_final from S0 = NULL.
+ */
+efla_status efla_state_affine(const float *P, const float *S_in, const float *H, float *S_out,
+                              int B, int Hh, int dk, int dv, void *stream);
+
+/*
  * Reads and clears the library's device error word after synchronising
  * `stream`.  Kernels that wait on barriers do so with bounded spins; when a
  * wait gives up the kernel records it here and exits, leaving the context
