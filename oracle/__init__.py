@@ -54,6 +54,8 @@ def _load():
         lib.efla_oracle_step_rule.restype = ctypes.c_double
         lib.efla_oracle_step_rule.argtypes = [ctypes.c_int, ctypes.c_int, dp, dp, dp, dp,
                                               ctypes.c_double, dp, ctypes.c_int]
+        lib.efla_oracle_bwd.restype = None
+        lib.efla_oracle_bwd.argtypes = [ctypes.c_int] * 5 + [dp] * 12 + [ctypes.c_int]
         lib.efla_oracle_fwd_rule.restype = ctypes.c_int
         lib.efla_oracle_fwd_rule.argtypes = [ctypes.c_int] * 5 + [dp] * 7 + [ctypes.c_int] * 2
         _lib = lib
@@ -122,3 +124,21 @@ def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True
     if rc != 0:
         raise MemoryError("oracle forward failed to allocate")
     return o, S
+
+
+def bwd(q, k, v, beta, dO, S0=None, dS_final=None, rule: str = "exact"):
+    """Gradients (dq, dk, dv, dbeta, dS0) of a loss through fwd(), given dO = dL/do and
+    dS_final = dL/dS_final (None = 0).  fp64, token by token, heads in sequence."""
+    q, k, v, beta, dO = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(dO)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    assert dO.shape == (B, H, L, dv)
+    s0 = _f64(S0) if S0 is not None else None
+    dsf = _f64(dS_final) if dS_final is not None else None
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    db, dS0 = np.zeros_like(beta), np.zeros((B, H, dk, dv))
+    _load().efla_oracle_bwd(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                            _ptr(s0) if s0 is not None else None, _ptr(dO),
+                            _ptr(dsf) if dsf is not None else None, _ptr(dq), _ptr(dkk), _ptr(dvv),
+                            _ptr(db), _ptr(dS0), RULES[rule])
+    return dq, dkk, dvv, db, dS0

@@ -216,3 +216,123 @@ int efla_oracle_fwd(int B, int H, int L, int dk, int dv, const double *q, const 
 {
     return efla_oracle_fwd_rule(B, H, L, dk, dv, q, k, v, beta, S0, o, S_final, nthreads, 0);
 }
+
+/* ---- backward pass (reverse mode through the token recurrence) --------------------------
+ *
+ * Gradients of a loss through the forward above, given do (dL/do_t) and dS_final (dL/dS_L,
+ * may be NULL = 0): dq, dk, dv, dbeta and dS0 (dL/dS0).  Per token the forward is
+ *   lambda = k.k, a = f(lambda, beta), x = S^T k, r = v - x, u = a r, S' = S + k u^T,
+ *   o = S'^T q,
+ * and the reverse step, with G = dL/dS' gathered from the later tokens, is
+ *   G += q do^T;  dq = S' do;  du = G^T k;  dk = G u;  da = du.r;  dv = a du;  dx = -a du;
+ *   dS = G + k dx^T;  dk += S dx;  dbeta = da df/dbeta;  dk += 2 da df/dlambda k;  G = dS.
+ * For the exact rule df/dbeta = e^{-beta lambda} and df/dlambda = (beta e^{-beta lambda} - a) /
+ * lambda (its series in x = beta lambda near 0); for the Euler rule df/dbeta = 1 and
+ * df/dlambda = 0.  The states S_t come from a forward sweep kept in full (the oracle has memory
+ * to spare).  Pinned in the tests by central finite differences of the forward.
+ */
+static void coeff_grads(double lambda, double beta, int rule, double *dfdb, double *dfdl)
+{
+    if (rule == 1) {
+        *dfdb = 1.0;
+        *dfdl = 0.0;
+        return;
+    }
+    const double x = beta * lambda;
+    *dfdb = exp(-x);
+    if (fabs(x) < 1e-4) {  /* beta^2 (-1/2 + x/3 - x^2/8 + x^3/30) */
+        *dfdl = beta * beta * (-0.5 + x / 3.0 - x * x / 8.0 + x * x * x / 30.0);
+    } else {
+        const double a = efla_oracle_alpha(lambda, beta);
+        *dfdl = (beta * exp(-x) - a) / lambda;
+    }
+}
+
+static void bwd_head(int L, int dk, int dv, const double *q, const double *k, const double *v,
+                     const double *beta, const double *S0, const double *dO, const double *dSL,
+                     double *dq, double *dkk, double *dvv, double *db, double *dS0, int rule)
+{
+    const size_t sz = (size_t)dk * dv;
+    double *Ss = (double *)malloc(sizeof(double) * sz * (size_t)(L + 1)); /* S_0 .. S_L */
+    double *G = (double *)malloc(sizeof(double) * sz);
+    double *x = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+    if (!Ss || !G || !x || !du || !u) {
+        free(Ss); free(G); free(x); free(du); free(u);
+        return;
+    }
+    if (S0) memcpy(Ss, S0, sizeof(double) * sz);
+    else memset(Ss, 0, sizeof(double) * sz);
+    for (int t = 0; t < L; ++t) {
+        memcpy(Ss + sz * (size_t)(t + 1), Ss + sz * (size_t)t, sizeof(double) * sz);
+        step_one(dk, dv, Ss + sz * (size_t)(t + 1), q + (size_t)t * dk, k + (size_t)t * dk,
+                 v + (size_t)t * dv, beta[t], NULL, x, rule);
+    }
+    if (dSL) memcpy(G, dSL, sizeof(double) * sz);
+    else memset(G, 0, sizeof(double) * sz);
+    for (int t = L - 1; t >= 0; --t) {
+        const double *S = Ss + sz * (size_t)t, *Sp = Ss + sz * (size_t)(t + 1);
+        const double *qt = q + (size_t)t * dk, *kt = k + (size_t)t * dk, *vt = v + (size_t)t * dv;
+        const double *dot = dO + (size_t)t * dv;
+        double lambda = 0.0;
+        for (int i = 0; i < dk; ++i) lambda += kt[i] * kt[i];
+        const double a = efla_oracle_coeff(lambda, beta[t], rule);
+        for (int j = 0; j < dv; ++j) {  /* x = S^T k, u = a (v - x) */
+            double s = 0.0;
+            for (int i = 0; i < dk; ++i) s += S[(size_t)i * dv + j] * kt[i];
+            x[j] = s;
+            u[j] = a * (vt[j] - s);
+        }
+        for (int i = 0; i < dk; ++i)  /* G += q do^T */
+            for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] += qt[i] * dot[j];
+        for (int i = 0; i < dk; ++i) {  /* dq = S' do */
+            double s = 0.0;
+            for (int j = 0; j < dv; ++j) s += Sp[(size_t)i * dv + j] * dot[j];
+            dq[(size_t)t * dk + i] = s;
+        }
+        double da = 0.0;
+        for (int j = 0; j < dv; ++j) {  /* du = G^T k, da = du.r, dv = a du */
+            double s = 0.0;
+            for (int i = 0; i < dk; ++i) s += G[(size_t)i * dv + j] * kt[i];
+            du[j] = s;
+            da += s * (vt[j] - x[j]);
+            dvv[(size_t)t * dv + j] = a * s;
+        }
+        for (int i = 0; i < dk; ++i) {  /* dk = G u + S dx with dx = -a du */
+            double s1 = 0.0, s2 = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                s1 += G[(size_t)i * dv + j] * u[j];
+                s2 += S[(size_t)i * dv + j] * (-a * du[j]);
+            }
+            dkk[(size_t)t * dk + i] = s1 + s2;
+        }
+        double dfdb, dfdl;
+        coeff_grads(lambda, beta[t], rule, &dfdb, &dfdl);
+        db[t] = da * dfdb;
+        for (int i = 0; i < dk; ++i) dkk[(size_t)t * dk + i] += 2.0 * da * dfdl * kt[i];
+        for (int i = 0; i < dk; ++i)  /* G = G + k dx^T */
+            for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] += kt[i] * (-a * du[j]);
+    }
+    if (dS0) memcpy(dS0, G, sizeof(double) * sz);
+    free(Ss); free(G); free(x); free(du); free(u);
+}
+
+/*
+ * Backward pass over [B,H,L,d] tensors (heads in sequence):
+ *   dO : [B,H,L,dv]   dS_final : [B,H,dk,dv] or NULL
+ *   dq, dk : [B,H,L,dk]   dv : [B,H,L,dv]   dbeta : [B,H,L]   dS0 : [B,H,dk,dv] or NULL
+ */
+void efla_oracle_bwd(int B, int H, int L, int dk, int dv, const double *q, const double *k,
+                     const double *v, const double *beta, const double *S0, const double *dO,
+                     const double *dS_final, double *dq, double *dkk, double *dvv, double *dbeta,
+                     double *dS0, int rule)
+{
+    const size_t sz = (size_t)dk * dv;
+    for (int bh = 0; bh < B * H; ++bh) {
+        const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
+        bwd_head(L, dk, dv, q + tk, k + tk, v + tv, beta + tb, S0 ? S0 + sz * bh : NULL, dO + tv,
+                 dS_final ? dS_final + sz * bh : NULL, dq + tk, dkk + tk, dvv + tv, dbeta + tb,
+                 dS0 ? dS0 + sz * bh : NULL, rule);
+    }
+}
