@@ -169,6 +169,36 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *Hm
                                                (cudaStream_t)stream));
 }
 
+size_t efla_bwd_workspace_size(int B, int H, int L, int dk, int dv) {
+    if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1 || dk > 128 || dv > 128) return 0;
+    return efla::bwd_workspace_bytes(B, H, L, dk, dv);
+}
+
+efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,
+                     const float *S0, const float *dO, const float *dS_final, float *dq,
+                     float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                     int dk, int dv, efla_dtype dt, efla_rule rule, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+    if (!rule_ok(rule)) return EFLA_ERR_RULE;
+    if (!dtype_ok(dt)) return EFLA_ERR_DTYPE;
+    if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
+    if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
+    if (dk > 128 || dv > 128) return EFLA_ERR_UNSUPPORTED;
+    if (L > 0 && (!q || !k || !v || !beta || !dO || !dq || !dkey || !dval || !dbeta))
+        return EFLA_ERR_NULL;
+    if (!aligned_elem(q, dt) || !aligned_elem(k, dt) || !aligned_elem(v, dt) ||
+        !aligned_elem(beta, dt))
+        return EFLA_ERR_ALIGN;
+    const void *fp[] = {S0, dO, dS_final, dq, dkey, dval, dbeta, dS0, workspace};
+    for (const void *p : fp)
+        if (!aligned_elem(p, EFLA_F32)) return EFLA_ERR_ALIGN;
+    const size_t need = efla::bwd_workspace_bytes(B, H, L, dk, dv);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
+    return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_final, dq, dkey, dval, dbeta, dS0,
+                                      B, H, L, dk, dv, dt == EFLA_BF16, rule == EFLA_RULE_EULER,
+                                      workspace, (cudaStream_t)stream));
+}
+
 unsigned long long efla_kernel_launches(void) {
     return efla::g_launches.load(std::memory_order_relaxed);
 }

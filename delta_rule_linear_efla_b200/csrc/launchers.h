@@ -34,6 +34,13 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
 cudaError_t launch_state_affine(const float *P, const float *S_in, const float *H, float *S_out,
                                 int BH, int dk, int dv, cudaStream_t s);
 
+// Backward pass (SIMT, one CTA per head): gradients of the forward given dO and dS_final.
+size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv);
+cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
+                       const float *S0, const float *dO, const float *dSL, float *dq, float *dkey,
+                       float *dval, float *dbeta, float *dS0, int B, int H, int L, int dk, int dv,
+                       bool is_bf16, bool euler, void *ws, cudaStream_t s);
+
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
 size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);

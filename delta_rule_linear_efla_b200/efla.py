@@ -25,7 +25,7 @@ ABI_SYMBOLS = (
     "efla_status_str", "efla_version", "efla_alpha", "efla_chunk_fwd_workspace_size",
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
     "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
-    "efla_recurrent_step_rule", "efla_state_affine",
+    "efla_recurrent_step_rule", "efla_state_affine", "efla_bwd_workspace_size", "efla_bwd",
 )
 
 _lib = None
@@ -72,6 +72,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_alpha_rule.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp]
     L.efla_chunk_fwd_rule.restype = i
     L.efla_chunk_fwd_rule.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz, vp]
+    L.efla_bwd_workspace_size.restype = sz
+    L.efla_bwd_workspace_size.argtypes = [i, i, i, i, i]
+    L.efla_bwd.restype = i
+    L.efla_bwd.argtypes = [vp] * 12 + [i] * 7 + [vp, sz, vp]
     L.efla_state_affine.restype = i
     L.efla_state_affine.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
     L.efla_recurrent_step_rule.restype = i
@@ -250,6 +254,67 @@ def state_affine(P, S_in=None, H=None, out=None, stream=None):
         B, Hh, dk, dv, _stream_handle(stream))
     _check(st, "efla_state_affine")
     return out
+
+
+def bwd(q, k, v, beta, dO, S0=None, dS_final=None, want_dS0: bool = True, rule: str = "exact",
+        workspace=None, stream=None):
+    """Gradients of chunk_fwd: returns (dq, dk, dv, dbeta, dS0 or None), all float32, given
+    dO = dL/do (float32 [B,H,L,dv]) and dS_final = dL/dS_final (float32 or None = 0)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L) or \
+            dO.shape != (B, H, L, dv):
+        raise ValueError("shape mismatch: q,k [B,H,L,dk], v,dO [B,H,L,dv], beta [B,H,L]")
+    code = _dtype_code(q)
+    for name, t in (("k", k), ("v", v), ("beta", beta)):
+        if t.dtype != q.dtype:
+            raise TypeError("%s must have q's dtype %s" % (name, q.dtype))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dkey, dval = torch.empty((B, H, L, dk), **f32), torch.empty((B, H, L, dk), **f32), \
+        torch.empty((B, H, L, dv), **f32)
+    dbeta = torch.empty((B, H, L), **f32)
+    dS0 = torch.empty((B, H, dk, dv), **f32) if want_dS0 else None
+    need = int(load_library().efla_bwd_workspace_size(B, H, L, dk, dv))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if need else None
+    st = load_library().efla_bwd(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
+        _dev(S0, "S0", torch.float32) if S0 is not None else None, _dev(dO, "dO", torch.float32),
+        _dev(dS_final, "dS_final", torch.float32) if dS_final is not None else None,
+        _dev(dq, "dq"), _dev(dkey, "dk"), _dev(dval, "dv"), _dev(dbeta, "dbeta"),
+        _dev(dS0, "dS0") if dS0 is not None else None, B, H, L, dk, dv, code, _rule(rule),
+        ws_ptr, need if ws_ptr else 0, _stream_handle(stream))
+    _check(st, "efla_bwd")
+    return dq, dkey, dval, dbeta, dS0
+
+
+class EflaFunction(torch.autograd.Function):
+    """(o, S_final) = EFLA forward with autograd: the forward is chunk_fwd and the backward is
+    efla_bwd.  Gradients flow to q, k, v, beta (in their dtype) and to S0 when given."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, beta, S0, rule="exact", chunk=64):
+        o, S = chunk_fwd(q, k, v, beta, S0, chunk=chunk, rule=rule)
+        ctx.save_for_backward(q, k, v, beta, S0 if S0 is not None else torch.empty(0))
+        ctx.has_S0, ctx.rule = S0 is not None, rule
+        return o, S
+
+    @staticmethod
+    def backward(ctx, dO, dS):
+        q, k, v, beta, S0 = ctx.saved_tensors
+        dO = dO.float().contiguous() if dO is not None else torch.zeros(
+            q.shape[:3] + v.shape[-1:], dtype=torch.float32, device=q.device)
+        dS = dS.float().contiguous() if dS is not None else None
+        dq, dk, dv, db, dS0 = bwd(q, k, v, beta, dO, S0 if ctx.has_S0 else None, dS,
+                                  want_dS0=ctx.has_S0, rule=ctx.rule)
+        return (dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), db.to(beta.dtype),
+                dS0 if ctx.has_S0 else None, None, None)
+
+
+def efla_attention(q, k, v, beta, S0=None, rule: str = "exact", chunk: int = 64):
+    """Differentiable EFLA forward: (o, S_final) with gradients through efla_bwd."""
+    return EflaFunction.apply(q, k, v, beta, S0, rule, chunk)
 
 
 def kernel_launches() -> int:

@@ -233,6 +233,31 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *H,
                               int B, int Hh, int dk, int dv, void *stream);
 
 /*
+ * efla_bwd -- gradients of efla_chunk_fwd_rule (the same function of the inputs:
+ * the chunkwise form equals the token recurrence): given dO = dL/do and dS_final
+ * = dL/dS_final (NULL = 0), writes dq, dkey, dval (the gradients with respect to
+ * q, k, v), dbeta and dS0 (NULL to skip).  Reverse mode through the update of
+ * Methodology 3 (or the Euler step under EFLA_RULE_EULER), including the
+ * dependence of alpha on ||k||^2 and beta.  The pages give no backward pass; its
+ * arithmetic is derived from the forward.
+ *
+ *   q, k : [B,H,L,dk] (dt)   v : [B,H,L,dv] (dt)   beta : [B,H,L] (dt)
+ *   S0 : [B,H,dk,dv] fp32 or NULL        dO : [B,H,L,dv] fp32
+ *   dq, dkey : [B,H,L,dk] fp32   dval : [B,H,L,dv] fp32   dbeta : [B,H,L] fp32
+ *   dS0 : [B,H,dk,dv] fp32 or NULL
+ *   workspace : efla_bwd_workspace_size(B,H,L,dk,dv) bytes, caller-owned scratch
+ * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  Pointers aligned to their element.
+ * One CTA per head walks the sequence twice (forward, then reverse): a first,
+ * correct path whose time grows with L per head, not a tuned kernel.
+ */
+size_t efla_bwd_workspace_size(int B, int H, int L, int dk, int dv);
+efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,
+                     const float *S0, const float *dO, const float *dS_final, float *dq,
+                     float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                     int dk, int dv, efla_dtype dt, efla_rule rule, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
  * Reads and clears the library's device error word after synchronising
  * `stream`.  Kernels that wait on barriers do so with bounded spins; when a
  * wait gives up the kernel records it here and exits, leaving the context
