@@ -56,6 +56,55 @@ def alg_bytes_chunk(w) -> int:
     return w.token_heads * per_tok + w.B * w.H * w.dk * w.dv * 4
 
 
+def alg_bytes_bwd(w) -> int:
+    """Algorithmic HBM bytes of one backward call: read q, k, v, beta (input dtype) and dO
+    (fp32), write dq, dk, dv (fp32) and dbeta (fp32) per token-head; S0 is zero here and
+    dS_final is not given."""
+    es = 2 if w.dtype == "bf16" else 4
+    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * 4 + (2 * w.dk + w.dv) * 4 + 4
+    return w.token_heads * per_tok
+
+
+def run_bwd(args) -> None:
+    """--pass bwd: the backward pass (efla_bwd) timed on the workload, one GPU."""
+    from delta_rule_linear_efla_b200 import efla
+
+    dev = torch.device("cuda", 0)
+    w = inputs.WORKLOADS[args.workload]
+    x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inputs.make_inputs(w).items()}
+    g = torch.Generator().manual_seed(77)
+    dO = torch.randn(w.B, w.H, w.L, w.dv, generator=g).to(dev)
+    ws = torch.empty(max(1, efla.load_library().efla_bwd_workspace_size(w.B, w.H, w.L, w.dk, w.dv)),
+                     dtype=torch.uint8, device=dev)
+    call = lambda: efla.bwd(x["q"], x["k"], x["v"], x["beta"], dO, x["S0"], None, want_dS0=False,
+                            rule=RULE, workspace=ws)
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(0)
+    clk.start()
+    a.record()
+    for _ in range(args.steps):
+        call()
+    b.record()
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    ms = a.elapsed_time(b) / args.steps
+    alg = alg_bytes_bwd(w)
+    peaks = _peaks()
+    achieved = alg / (ms / 1e3) / 1e9
+    print(json.dumps({
+        "metric": "EFLA bwd tokens/s per GPU (B*H*L/time) and % of binding roofline", "value":
+        w.token_heads / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic", "config": _config(w),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": None, "kernel": "efla_bwd (SIMT)",
+                     "alg_bytes_per_launch": alg, "avg_launch_ms": ms},
+        "gpu_launches": args.steps, "clocks": clocks}))
+
+
 def alg_bytes_decode(Bd, Hd, dk, dv, es=2) -> int:
     """Read + write of the fp32 state per head, plus q, k, v, beta in and o out."""
     return Bd * Hd * (2 * dk * dv * 4 + (2 * dk + 2 * dv + 1) * es)
@@ -394,6 +443,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd (default): the forward step; bwd: the backward pass alone")
     ap.add_argument("--rule", choices=["exact", "euler"], default="exact",
                     help="update rule: the exact flow (default) or the delta rule's Euler step, "
                          "for the throughput comparison (the workload's keys are not normalised, "
@@ -405,6 +456,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.pass_ == "bwd":
+        run_bwd(args)
     else:
         run_ours(args)
 
