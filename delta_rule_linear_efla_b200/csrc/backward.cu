@@ -50,6 +50,25 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
     return s;
 }
 
+// sum_j M[row][j] w[j] over this thread's half of the columns (two threads per row).  With an
+// even dv the walk starts at column 2*row + half and wraps, so the 16 rows of a warp read 32
+// different banks instead of two.
+__device__ __forceinline__ float row_dot_half(const float *M, const float *w, int row, int half,
+                                              int dv) {
+    float s = 0.f;
+    if (dv % 2 == 0) {
+        int j = (2 * row + half) % dv;
+        for (int m = 0; m < dv / 2; ++m) {
+            s = fmaf(M[row * dv + j], w[j], s);
+            j += 2;
+            if (j >= dv) j -= dv;
+        }
+    } else {
+        for (int j = half; j < dv; j += 2) s = fmaf(M[row * dv + j], w[j], s);
+    }
+    return s;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(BWD_THREADS)
     bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
@@ -89,7 +108,13 @@ __global__ void __launch_bounds__(BWD_THREADS)
             R[(size_t)t * dv + tid] = r;
         }
         __syncthreads();
-        for (int e = tid; e < DD; e += BWD_THREADS) S[e] = fmaf(a * ks[e / dv], rs[e % dv], S[e]);
+        if (BWD_THREADS % dv == 0) {  // fixed column per thread: no division per element
+            const int j = tid % dv;
+            for (int i = tid / dv; i < dk; i += BWD_THREADS / dv)
+                S[i * dv + j] = fmaf(a * ks[i], rs[j], S[i * dv + j]);
+        } else {
+            for (int e = tid; e < DD; e += BWD_THREADS) S[e] = fmaf(a * ks[e / dv], rs[e % dv], S[e]);
+        }
         __syncthreads();
     }
     for (int e = tid; e < DD; e += BWD_THREADS) CK[(size_t)NB * DD + e] = S[e];
@@ -117,11 +142,15 @@ __global__ void __launch_bounds__(BWD_THREADS)
             const float bt = to_f32(beta[tb + t]);
             const float a = alpha_rule(lambda, bt, euler);
             // G += q do^T; dq = S' do (S holds S' = the state after token t)
-            for (int e = tid; e < DD; e += BWD_THREADS) G[e] = fmaf(qs[e / dv], dos[e % dv], G[e]);
+            if (BWD_THREADS % dv == 0) {
+                const int j = tid % dv;
+                for (int i = tid / dv; i < dk; i += BWD_THREADS / dv)
+                    G[i * dv + j] = fmaf(qs[i], dos[j], G[i * dv + j]);
+            } else {
+                for (int e = tid; e < DD; e += BWD_THREADS) G[e] = fmaf(qs[e / dv], dos[e % dv], G[e]);
+            }
             {
-                float s = 0.f;
-                if (row < dk)
-                    for (int j = half; j < dv; j += 2) s = fmaf(S[row * dv + j], dos[j], s);
+                float s = row < dk ? row_dot_half(S, dos, row, half, dv) : 0.f;
                 s += __shfl_xor_sync(0xffffffffu, s, 1);
                 if (row < dk && half == 0) dq[tk + (size_t)t * dk + row] = s;
             }
@@ -138,22 +167,26 @@ __global__ void __launch_bounds__(BWD_THREADS)
             }
             const float da = block_sum(dap, red);  // syncs: dus, dxs visible
             // dk = G u + (added below) S dx + 2 da df/dlambda k, with u = a r
-            float dka = 0.f;
-            if (row < dk)
-                for (int j = half; j < dv; j += 2) dka = fmaf(G[row * dv + j], a * rs[j], dka);
+            float dka = row < dk ? a * row_dot_half(G, rs, row, half, dv) : 0.f;  // G u, u = a r
             dka += __shfl_xor_sync(0xffffffffu, dka, 1);
             const float krow = row < dk ? ks[row] : 0.f;  // ks is rewritten by the next token
             __syncthreads();  // every read of G and S' for this token is done
             // S = S' - a k r^T (the state before token t); G += k dx^T (dL/dS)
-            for (int e = tid; e < DD; e += BWD_THREADS) {
-                const int i = e / dv, j = e % dv;
-                S[e] = fmaf(-a * ks[i], rs[j], S[e]);
-                G[e] = fmaf(ks[i], dxs[j], G[e]);
+            if (BWD_THREADS % dv == 0) {
+                const int j = tid % dv;
+                for (int i = tid / dv; i < dk; i += BWD_THREADS / dv) {
+                    S[i * dv + j] = fmaf(-a * ks[i], rs[j], S[i * dv + j]);
+                    G[i * dv + j] = fmaf(ks[i], dxs[j], G[i * dv + j]);
+                }
+            } else {
+                for (int e = tid; e < DD; e += BWD_THREADS) {
+                    const int i = e / dv, j = e % dv;
+                    S[e] = fmaf(-a * ks[i], rs[j], S[e]);
+                    G[e] = fmaf(ks[i], dxs[j], G[e]);
+                }
             }
             __syncthreads();
-            float dkb = 0.f;
-            if (row < dk)
-                for (int j = half; j < dv; j += 2) dkb = fmaf(S[row * dv + j], dxs[j], dkb);
+            float dkb = row < dk ? row_dot_half(S, dxs, row, half, dv) : 0.f;
             dkb += __shfl_xor_sync(0xffffffffu, dkb, 1);
             float dfdb, dfdl;
             coeff_grads(lambda, bt, euler, a, dfdb, dfdl);
