@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(BWD_THREADS)
     extern __shared__ float sm[];
     const int DD = dk * dv, NB = (L + BWD_BLOCK - 1) / BWD_BLOCK;
     float *S = sm, *G = sm + DD;
-    float *qs = G + DD, *ks = qs + 128, *dos = ks + 128, *rs = dos + 128, *dus = rs + 128;
-    float *dxs = dus + 128, *red = dxs + 128;
+    float *qs = G + DD, *ks = qs + 128, *dos = ks + 128, *rs = dos + 128, *dxs = rs + 128;
+    float *red = dxs + 128;
     const int tid = threadIdx.x, bh = blockIdx.x;
     const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
     float *R = ws + (size_t)bh * ((size_t)L * dv + (size_t)(NB + 1) * DD);  // r of every token
@@ -160,12 +160,11 @@ __global__ void __launch_bounds__(BWD_THREADS)
             if (tid < dv) {
                 float s = 0.f;
                 for (int i = 0; i < dk; ++i) s = fmaf(G[i * dv + tid], ks[i], s);
-                dus[tid] = s;
                 dxs[tid] = -a * s;
                 dval[tv + (size_t)t * dv + tid] = a * s;
                 dap = s * rs[tid];
             }
-            const float da = block_sum(dap, red);  // syncs: dus, dxs visible
+            const float da = block_sum(dap, red);  // syncs: dxs visible
             // dk = G u + (added below) S dx + 2 da df/dlambda k, with u = a r
             float dka = row < dk ? a * row_dot_half(G, rs, row, half, dv) : 0.f;  // G u, u = a r
             dka += __shfl_xor_sync(0xffffffffu, dka, 1);
@@ -210,7 +209,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
                        float *dval, float *dbeta, float *dS0, int B, int H, int L, int dk, int dv,
                        bool is_bf16, bool euler, void *ws, cudaStream_t s) {
     const int BH = B * H;
-    const size_t smem = (size_t)(2 * dk * dv + 6 * 128 + 32) * sizeof(float);
+    const size_t smem = (size_t)(2 * dk * dv + 5 * 128 + 32) * sizeof(float);
     cudaError_t e;
     if (is_bf16) {
         e = cudaFuncSetAttribute(bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -11,18 +11,19 @@
 //   O  = Q S + lower-incl-diagonal(Q K^T) U'   (o_t = S_t^T q_t)
 //   S <- S + K^T U'
 //
-// Two kernels:
-//  prep  -- one chunk at a time, all chunks in parallel: the fused squared norm
-//           and a, the Gram matrix K K^T on the tensor cores (TMEM accumulator),
-//           the unit-lower-triangular inverse T by blocked forward substitution
-//           on CUDA cores in fp32, and Ta = T diag(a) written as bf16 to the
-//           workspace (64x64 per chunk).
-//  state -- one CTA per (head, 64-column slice of the state), chunks in order.
-//           W = Ta K, U = Ta V, P = Q K^T, X = W S, dS = K^T U' and
-//           O = Q S + mask(P) U' are tcgen05 MMAs with fp32 accumulators in
-//           TMEM; the carried state S is fp32 in registers (one row per
-//           thread) with a bf16 copy in shared memory as the MMA operand.
-//           Q, K, V and Ta arrive by TMA (128-byte swizzle), double buffered.
+// Kernels:
+//  prep  -- one chunk per 128-thread pipeline, every chunk in parallel: the squared
+//           norms and a, the Gram matrix K K^T on the tensor cores (TMEM accumulator),
+//           the unit-lower-triangular inverse T (16x16 diagonal blocks by fp32
+//           substitution, the off-diagonal blocks by mma.sync block merges), and
+//           Ta = T diag(a) written as fp16 to the workspace (64x64 per chunk).
+//  state -- one CTA per head (or per segment run of a head), chunks in order, warp-
+//           specialised: TMA loads q, k, v, Ta (128-byte swizzle, double buffered), an
+//           in-place bf16 -> fp16 conversion, one thread issuing every tcgen05.mma
+//           (W, P^T, the U' prefill and the fused D1/D2 products), and epilogue
+//           warpgroups that move results between TMEM and the operand tiles; the
+//           fp32 state S^T stays in TMEM across chunks, with an fp16 copy as D1's A.
+//  seg_combine -- for sequence segments: chains the segments' affine state maps.
 //
 // Every mbarrier wait is bounded; a wait that gives up sets the device error
 // word, drains the copies this CTA has in flight (again bounded), releases
