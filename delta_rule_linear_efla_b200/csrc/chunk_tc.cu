@@ -68,11 +68,13 @@ struct Smem {
     static constexpr int A16 = C * LD16 * 2;      // A, fp16, row-major
     static constexpr int TD16 = 4 * 16 * 24 * 2;  // T's diagonal blocks, fp16, row-major (A operands)
     static constexpr int T16T = C * LD16 * 2;     // T, fp16, transposed (B operands)
-    static constexpr int TA16 = C * LD16 * 2;     // T diag(a), fp16, row-major (the output tile)
+    // A's fp32 diagonal blocks (read by the diagonal solve) share their space with the
+    // per-warp transposed-R scratch of the block merges, which run after the solve.
     static constexpr int ADIAG = C * 16 * 4;      // diagonal 16x16 blocks of A, fp32
     static constexpr int RT = 4 * 16 * 24 * 2;    // per-warp 16x16 scratch (transposed R), fp16
+    static constexpr int AD_RT = ADIAG > RT ? ADIAG : RT;
     template <int DK>
-    static constexpr int bytes() { return k_bytes<DK>() + A16 + TD16 + T16T + TA16 + ADIAG + RT + C * 4; }
+    static constexpr int bytes() { return k_bytes<DK>() + A16 + TD16 + T16T + AD_RT + C * 4; }
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -111,10 +113,9 @@ __global__ void __launch_bounds__(THREADS)
     __half *A16 = reinterpret_cast<__half *>(base + KB);
     __half *TD16 = A16 + C * LD16;                   // [4][16][24]
     __half *T16t = TD16 + 4 * 16 * 24;
-    __half *Ta16 = T16t + C * LD16;
-    float *Ad = reinterpret_cast<float *>(Ta16 + C * LD16);  // [64 rows][16]: A's diagonal blocks
-    __half *Rt = reinterpret_cast<__half *>(Ad + C * 16);
-    float *al = reinterpret_cast<float *>(Rt + 4 * 16 * 24);
+    float *Ad = reinterpret_cast<float *>(T16t + C * LD16);  // [64 rows][16]: A's diagonal blocks
+    __half *Rt = reinterpret_cast<__half *>(Ad);             // after the solve: merge scratch
+    float *al = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Ad) + Smem::AD_RT);
     __shared__ uint64_t full, mma_bar;
     __shared__ uint32_t tmem_base;
 
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(THREADS)
     for (int g = blockIdx.x; g < total; g += gridDim.x, ++it) {
         const uint32_t ph = it & 1;
         const int bh = g / NC, n = g - bh * NC, c0 = n * C;
+        __half *gta = ta_out + (size_t)g * C * C;  // this chunk's Ta tile (row-major 64x64)
         const float beta_row = beta_next;
         beta_next = load_beta(g + gridDim.x);
         (void)bh;
@@ -211,15 +213,14 @@ __global__ void __launch_bounds__(THREADS)
         {
             const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 accumulator layout)
             const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
-            float g64[64];
-            tc::tmem_ld64(ta, g64);  // the whole row at once: one wait
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
+                float v[16];
+                tc::tmem_ld16(ta + cb * 16, v);
                 if (lane < 16) {
                     const float ar = al[r];
-                    float v[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * g64[cb * 16 + j] : 0.f;
+                    for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * v[j] : 0.f;
                     uint4 *dst = reinterpret_cast<uint4 *>(A16 + r * LD16 + cb * 16);
                     dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
                                         tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(THREADS)
                 const int row = 16 * b + i, col = 16 * b + c;
                 TD16[(b * 16 + i) * 24 + c] = __float2half_rn(x[i]);
                 T16t[col * LD16 + row] = __float2half_rn(x[i]);
-                Ta16[row * LD16 + col] = __float2half_rn(x[i] * ac);
+                gta[row * C + col] = __float2half_rn(x[i] * ac);
             }
         } else {
             // zero the strictly-upper 16x16 blocks of the output tile
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(THREADS)
                 const int blk = e >> 7, w = e & 127;
                 const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
                 const int J = blk < 3 ? 1 + blk : (blk < 5 ? blk - 1 : 3);
-                *reinterpret_cast<uint32_t *>(Ta16 + (16 * I + (w >> 3)) * LD16 + 16 * J + 2 * (w & 7)) = 0u;
+                *reinterpret_cast<uint32_t *>(gta + (16 * I + (w >> 3)) * C + 16 * J + 2 * (w & 7)) = 0u;
             }
         }
         __syncthreads();
@@ -305,8 +306,8 @@ __global__ void __launch_bounds__(THREADS)
                     mma16816(d, a, b0, b1);
                     const int row = 16 * I + gq, col = 16 * J + 8 * nt + 2 * tq;
                     const float a0 = al[col], a1 = al[col + 1];
-                    *reinterpret_cast<uint32_t *>(Ta16 + row * LD16 + col) = tc::pack_f16(-d[0] * a0, -d[1] * a1);
-                    *reinterpret_cast<uint32_t *>(Ta16 + (row + 8) * LD16 + col) = tc::pack_f16(-d[2] * a0, -d[3] * a1);
+                    *reinterpret_cast<uint32_t *>(gta + row * C + col) = tc::pack_f16(-d[0] * a0, -d[1] * a1);
+                    *reinterpret_cast<uint32_t *>(gta + (row + 8) * C + col) = tc::pack_f16(-d[2] * a0, -d[3] * a1);
                     T16t[col * LD16 + row] = __float2half_rn(-d[0]);
                     T16t[(col + 1) * LD16 + row] = __float2half_rn(-d[1]);
                     T16t[col * LD16 + row + 8] = __float2half_rn(-d[2]);
@@ -315,15 +316,6 @@ __global__ void __launch_bounds__(THREADS)
             }
             __syncthreads();
         }
-        // ---- the assembled fp16 Ta tile -> workspace (row-major 64x64), 16-byte stores
-        {
-            const int i = tid >> 1, h = tid & 1;
-            uint4 *dst = reinterpret_cast<uint4 *>(ta_out + ((size_t)g * C + i) * C + h * 32);
-            const uint4 *src = reinterpret_cast<const uint4 *>(Ta16 + i * LD16 + h * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = src[q4];
-        }
-        __syncthreads();
     }
     if (aborted) {
         if (tid == 0) {
