@@ -74,7 +74,12 @@ struct Smem {
     static constexpr int RT = 4 * 16 * 24 * 2;    // per-warp 16x16 scratch (transposed R), fp16
     static constexpr int AD_RT = ADIAG > RT ? ADIAG : RT;
     template <int DK>
-    static constexpr int bytes() { return k_bytes<DK>() + A16 + TD16 + T16T + AD_RT + C * 4; }
+    static constexpr int bytes() { return region0<DK>() + T16T + C * 4; }
+    // The K tile is dead once the Gram MMA and the norms have read it; the solve's A, T
+    // diagonal blocks and scratch then take its place (the next K is loaded after the solve).
+    static constexpr int SCRATCH = A16 + TD16 + AD_RT;
+    template <int DK>
+    static constexpr int region0() { return k_bytes<DK>() > SCRATCH ? k_bytes<DK>() : SCRATCH; }
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -109,13 +114,13 @@ __global__ void __launch_bounds__(THREADS)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    uint8_t *Kt = base;  // one K tile: refilled as soon as the Gram MMA and the norms have read it
-    __half *A16 = reinterpret_cast<__half *>(base + KB);
+    uint8_t *Kt = base;  // the K tile; after the Gram and the norms, the solve's scratch below
+    __half *A16 = reinterpret_cast<__half *>(base);
     __half *TD16 = A16 + C * LD16;                   // [4][16][24]
-    __half *T16t = TD16 + 4 * 16 * 24;
-    float *Ad = reinterpret_cast<float *>(T16t + C * LD16);  // [64 rows][16]: A's diagonal blocks
-    __half *Rt = reinterpret_cast<__half *>(Ad);             // after the solve: merge scratch
-    float *al = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Ad) + Smem::AD_RT);
+    float *Ad = reinterpret_cast<float *>(TD16 + 4 * 16 * 24);  // [64 rows][16]: A's diagonal blocks
+    __half *Rt = reinterpret_cast<__half *>(Ad);                // after the solve: merge scratch
+    __half *T16t = reinterpret_cast<__half *>(base + Smem::region0<DK>());
+    float *al = reinterpret_cast<float *>(T16t + C * LD16);
     __shared__ uint64_t full, mma_bar;
     __shared__ uint32_t tmem_base;
 
@@ -205,10 +210,6 @@ __global__ void __launch_bounds__(THREADS)
         mma_phase ^= 1;
         mma_pending = false;
         tc::tc_fence_after();
-        if (tid == 0 && g + (int)gridDim.x < total) {  // the K tile is free: fetch the next chunk
-            issue(g + gridDim.x);
-            issued = true;
-        }
         // ---- A = strictly-lower(diag(a) G): fp16 copy (all blocks), fp32 diagonal blocks
         {
             const int r = 16 * warp + lane;  // valid for lane < 16 (M = 64 accumulator layout)
@@ -315,6 +316,11 @@ __global__ void __launch_bounds__(THREADS)
                 }
             }
             __syncthreads();
+        }
+        if (tid == 0 && g + (int)gridDim.x < total) {  // the solve's scratch is dead: next K tile
+            tc::fence_async_smem();
+            issue(g + gridDim.x);
+            issued = true;
         }
     }
     if (aborted) {
