@@ -199,6 +199,11 @@ efla_status efla_bwd(const void *q, const void *k, const void *v, const void *be
                                       workspace, (cudaStream_t)stream));
 }
 
+efla_status efla_selftest_bounded_wait(long long budget_cycles, void *stream) {
+    if (budget_cycles < 1 || budget_cycles > 2000000000LL) return EFLA_ERR_SHAPE;
+    return from_cuda(efla::launch_selftest_wait(budget_cycles, (cudaStream_t)stream));
+}
+
 unsigned long long efla_kernel_launches(void) {
     return efla::g_launches.load(std::memory_order_relaxed);
 }

@@ -838,6 +838,19 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------------------------ bounded-wait self-test
+// One thread waits on an mbarrier that nothing arrives on, for at most `budget` cycles, then
+// records a timeout in the device error word the way the kernels above do and returns: the
+// test of that path, without a fault or a hang (nothing else is in flight in this CTA).
+__global__ void selftest_wait_kernel(long long budget) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+        if (!tc::mbar_wait(&bar, 0, budget)) record_error(4u);
+    }
+}
+
 // ------------------------------------------------------------------ segment chaining
 // Each sequence segment maps the state affinely, S_out = P S_in + H (P is the product of
 // the segment's transitions I - K^T W, H the segment's state from zero).  This chains
@@ -1100,6 +1113,12 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
     if (dk == 64 && dv == 128)
         return launch_tc_o<64, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
     return launch_tc_o<64, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
+}
+
+cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s) {
+    selftest_wait_kernel<<<1, 32, 0, s>>>(budget_cycles);
+    count_launches(1);
+    return cudaGetLastError();
 }
 
 cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s) {

@@ -49,6 +49,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
                             const float *S0, void *o, float *S_final, int B, int H, int L,
                             int dk, int dv, int chunk, bool o_bf16, bool euler, void *ws,
                             cudaStream_t s);
+// A kernel whose one bounded wait runs out (nothing arrives): records a timeout, then returns.
+cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits): read and clear.
 cudaError_t tc_read_and_clear_error(unsigned int *out, cudaStream_t s);
 

@@ -26,6 +26,7 @@ ABI_SYMBOLS = (
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
     "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
     "efla_recurrent_step_rule", "efla_state_affine", "efla_bwd_workspace_size", "efla_bwd",
+    "efla_selftest_bounded_wait",
 )
 
 _lib = None
@@ -76,6 +77,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_bwd_workspace_size.argtypes = [i, i, i, i, i]
     L.efla_bwd.restype = i
     L.efla_bwd.argtypes = [vp] * 12 + [i] * 7 + [vp, sz, vp]
+    L.efla_selftest_bounded_wait.restype = i
+    L.efla_selftest_bounded_wait.argtypes = [ctypes.c_longlong, vp]
     L.efla_state_affine.restype = i
     L.efla_state_affine.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
     L.efla_recurrent_step_rule.restype = i
@@ -315,6 +318,13 @@ class EflaFunction(torch.autograd.Function):
 def efla_attention(q, k, v, beta, S0=None, rule: str = "exact", chunk: int = 64):
     """Differentiable EFLA forward: (o, S_final) with gradients through efla_bwd."""
     return EflaFunction.apply(q, k, v, beta, S0, rule, chunk)
+
+
+def selftest_bounded_wait(budget_cycles: int = 1_000_000, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (its wait runs out by design); read the
+    outcome with last_device_error()."""
+    _check(load_library().efla_selftest_bounded_wait(int(budget_cycles), _stream_handle(stream)),
+           "efla_selftest_bounded_wait")
 
 
 def kernel_launches() -> int:

@@ -267,6 +267,18 @@ efla_status efla_bwd(const void *q, const void *k, const void *v, const void *be
 efla_status efla_last_device_error(void *stream);
 
 /*
+ * efla_selftest_bounded_wait -- a test hook for the failure path (no counterpart
+ * on the pages): launches one small kernel whose single wait is on an mbarrier
+ * that nothing arrives on, bounded by budget_cycles (1 .. 2e9 SM cycles, about
+ * a second at most).  When the bound runs out the kernel records a timeout in
+ * the device error word, exactly as the forward kernels do when a wait gives up,
+ * and returns; nothing faults or hangs and the context stays usable.  A later
+ * efla_last_device_error then reports EFLA_ERR_TIMEOUT (and clears the word).
+ * EFLA_ERR_SHAPE for a budget outside its range.
+ */
+efla_status efla_selftest_bounded_wait(long long budget_cycles, void *stream);
+
+/*
  * Which chunk-forward kernels the library selects for these sizes on the current
  * device: 0 = SIMT fp32 path, 1 = tensor-core (tcgen05) path, 2 = tensor-core path
  * with the sequence cut into segments that run in parallel (few heads, long

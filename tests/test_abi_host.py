@@ -136,3 +136,9 @@ def test_unknown_rule_is_refused_on_the_host(lib):
     assert lib.efla_recurrent_step_rule(P, P, P, P, P, P, 1, 1, 16, 16, BF16, F32, -1,
                                         None) == EFLA_ERR_RULE
     assert "rule" in lib.efla_status_str(EFLA_ERR_RULE).decode()
+
+
+def test_selftest_budget_is_checked_on_the_host(lib):
+    EFLA_ERR_SHAPE = 2
+    assert lib.efla_selftest_bounded_wait(0, None) == EFLA_ERR_SHAPE
+    assert lib.efla_selftest_bounded_wait(3_000_000_000, None) == EFLA_ERR_SHAPE

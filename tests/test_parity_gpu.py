@@ -254,3 +254,16 @@ def test_segments_in_place_state_carry(oracle_mod):
     assert S_out.data_ptr() == S.data_ptr()
     o_ref, S_ref = _oracle(oracle_mod, x)
     _check(x, o.float().cpu(), S.cpu(), o_ref, S_ref)
+
+
+def test_bounded_wait_reports_timeout_and_leaves_the_context_usable(oracle_mod):
+    """A wait that nothing completes gives up after its bound, sets the device error word
+    (read as EFLA_ERR_TIMEOUT, then cleared) and returns; the next forward runs normally."""
+    EFLA_ERR_TIMEOUT = 6
+    efla.selftest_bounded_wait(1_000_000)
+    assert efla.last_device_error() == EFLA_ERR_TIMEOUT
+    assert efla.last_device_error() == 0  # read-and-clear
+    x = inputs.make_inputs(inputs.workload(4, B=1, H=2, L=200))
+    o, S = _run_gpu(x)  # asserts the error word is clear again
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    _check(x, o, S, o_ref, S_ref)
