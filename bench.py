@@ -236,21 +236,30 @@ def run_reference(args) -> None:
     oracle.build()
     w = inputs.WORKLOADS[args.workload]
     cores = os.cpu_count() or 1
-    H = min(w.H, cores)
-    xs = inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 1024)))
-    threads = min(cores, H)
+    bwd = args.pass_ == "bwd"
+    # the backward oracle runs heads one after another (it keeps every state): a smaller sample
+    H = min(w.H, 2 if bwd else cores)
+    xs = inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 512 if bwd else 1024)))
+    threads = 1 if bwd else min(cores, H)
+    if bwd:
+        dO = torch.randn(xs["v"].shape, generator=torch.Generator().manual_seed(77), dtype=torch.float64)
+        run = lambda: oracle.bwd(xs["q"], xs["k"], xs["v"], xs["beta"], dO, xs["S0"], None, rule=RULE)
+    else:
+        run = lambda: oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads,
+                                 rule=RULE)
     for _ in range(args.warmup):
-        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
+        run()
     dt = time.perf_counter() - t0
     n = H * xs["q"].shape[2] * args.steps
     val = n / dt
-    sample = "%d heads x L=%d of workload %s per step, fp64 token-by-token" % (
-        H, xs["q"].shape[2], w.name)
+    sample = "%d heads x L=%d of workload %s per step, fp64 token-by-token%s" % (
+        H, xs["q"].shape[2], w.name, " (backward)" if bwd else "")
+    metric = "EFLA bwd tokens/s per GPU (B*H*L/time) and % of binding roofline" if bwd else METRIC
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": val, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(w),
