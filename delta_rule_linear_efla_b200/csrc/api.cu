@@ -192,6 +192,7 @@ efla_status efla_bwd(const void *q, const void *k, const void *v, const void *be
     const void *fp[] = {S0, dO, dS_final, dq, dkey, dval, dbeta, dS0, workspace};
     for (const void *p : fp)
         if (!aligned_elem(p, EFLA_F32)) return EFLA_ERR_ALIGN;
+    if (!aligned16(workspace)) return EFLA_ERR_ALIGN;  // float4 rows of the saved states
     const size_t need = efla::bwd_workspace_bytes(B, H, L, dk, dv);
     if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
     return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_final, dq, dkey, dval, dbeta, dS0,

@@ -7,18 +7,30 @@
 //   G += q do^T;  dq = S' do;  du = G^T k;  dk = G u;  da = du.r;  dv = a du;  dx = -a du;
 //   dk += S dx;  dbeta = da df/dbeta;  dk += 2 da df/dlambda k;  G += k dx^T  (-> dL/dS).
 //
-// One CTA per head, 256 threads, S and G in shared memory (d <= 128).  A forward sweep stores
-// every token's r and the state at every 64-token boundary in the workspace; the reverse sweep
-// starts each 64-token block from the stored state at its end and steps back exactly with
-// S = S' - a k r^T, so rounding never accumulates over more than 64 tokens.  This is the first
-// correct path for the backward: it is bound by the per-token barrier chain, not by HBM.
+// The state's columns evolve independently (column j: s <- (I - a k k^T) s + a k v_j), so the
+// work is split by columns: one CTA per (head, block of 16 state columns), one state row per
+// thread (128 threads, dk <= 128), that row of S and of G in registers.  What couples the column
+// blocks is linear -- dq, dk and dbeta are sums over the columns (dk and dbeta through da, itself
+// a sum over the columns) -- so each CTA writes its share of them to the workspace and a second
+// kernel adds the shares up in a fixed order: the result does not depend on scheduling.
+//
+// A forward sweep stores each column block's r and its state every 64 tokens; the reverse sweep
+// starts each 64-token block from the stored state at its end and steps back with
+// S = S' - a k r^T, so rounding never accumulates over more than 64 tokens.  Each token takes
+// one CTA-wide sum (the 16 column dot products over the rows, and lambda = |k|^2): a
+// reduce-scatter across each warp's lanes, then one barrier to add the four warps' shares
+// through shared memory, double-buffered by token parity so that one barrier per token suffices.
+#include <algorithm>
+#include <cstdint>
+
 #include "common.cuh"
 #include "launchers.h"
 
 namespace efla {
 
-constexpr int BWD_THREADS = 256;
-constexpr int BWD_BLOCK = 64;  // tokens between stored states
+constexpr int BW_THREADS = 128;  // one state row per thread (dk <= 128)
+constexpr int BW_CB = 16;        // state columns per CTA
+constexpr int BWD_BLOCK = 64;    // tokens between stored states
 
 // df/dbeta and df/dlambda of the coefficient under the rule.
 __device__ __forceinline__ void coeff_grads(float lambda, float beta, bool euler, float a,
@@ -37,195 +49,318 @@ __device__ __forceinline__ void coeff_grads(float lambda, float beta, bool euler
     }
 }
 
-// Sum over the CTA of one value per thread (all threads call it; the result is returned to all).
-__device__ __forceinline__ float block_sum(float v, float *red) {
-    v = warp_sum(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    float s = 0.f;
+struct BwdRed {  // the four warps' shares of one CTA-wide sum, double-buffered by token parity
+    float col[2][BW_THREADS / 32][BW_CB];
+    float lam[2][BW_THREADS / 32];
+};
+
+// Sum over the warp of 16 values per lane, scattered: every lane returns the sum of value
+// (lane >> 1).  Each step halves the values a lane keeps and trades the other half with the
+// lane whose index differs in one bit: 8 + 4 + 2 + 1 + 1 shuffles in place of 16 x 5.
+__device__ __forceinline__ float warp_reduce_scatter16(float (&p)[BW_CB], int lane) {
 #pragma unroll
-    for (int i = 0; i < BWD_THREADS / 32; ++i) s += red[i];
-    return s;
-}
-
-// sum_j M[row][j] w[j] over this thread's half of the columns (two threads per row).  With an
-// even dv the walk starts at column 2*row + half and wraps, so the 16 rows of a warp read 32
-// different banks instead of two.
-__device__ __forceinline__ float row_dot_half(const float *M, const float *w, int row, int half,
-                                              int dv) {
-    float s = 0.f;
-    if (dv % 2 == 0) {
-        int j = (2 * row + half) % dv;
-        for (int m = 0; m < dv / 2; ++m) {
-            s = fmaf(M[row * dv + j], w[j], s);
-            j += 2;
-            if (j >= dv) j -= dv;
-        }
-    } else {
-        for (int j = half; j < dv; j += 2) s = fmaf(M[row * dv + j], w[j], s);
+    for (int m = 0; m < 8; ++m) {
+        const bool up = lane & 16;
+        const float send = up ? p[m] : p[m + 8], keep = up ? p[m + 8] : p[m];
+        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
     }
-    return s;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const bool up = lane & 8;
+        const float send = up ? p[m] : p[m + 4], keep = up ? p[m + 4] : p[m];
+        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const bool up = lane & 4;
+        const float send = up ? p[m] : p[m + 2], keep = up ? p[m + 2] : p[m];
+        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? p[0] : p[1], keep = up ? p[1] : p[0];
+        p[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(BWD_THREADS)
-    bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-               const T *__restrict__ beta, const float *__restrict__ S0, const float *__restrict__ dO,
-               const float *__restrict__ dSL, float *__restrict__ dq, float *__restrict__ dkey,
-               float *__restrict__ dval, float *__restrict__ dbeta, float *__restrict__ dS0, int L,
-               int dk, int dv, bool euler, float *__restrict__ ws) {
-    extern __shared__ float sm[];
-    const int DD = dk * dv, NB = (L + BWD_BLOCK - 1) / BWD_BLOCK;
-    float *S = sm, *G = sm + DD;
-    float *qs = G + DD, *ks = qs + 128, *dos = ks + 128, *rs = dos + 128, *dxs = rs + 128;
-    float *red = dxs + 128;
-    const int tid = threadIdx.x, bh = blockIdx.x;
-    const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
-    float *R = ws + (size_t)bh * ((size_t)L * dv + (size_t)(NB + 1) * DD);  // r of every token
-    float *CK = R + (size_t)L * dv;                                         // states S_{64 b}, S_L
-
-    // ---- forward sweep: r_t and the block-boundary states
-    for (int e = tid; e < DD; e += BWD_THREADS) S[e] = S0 ? S0[(size_t)bh * DD + e] : 0.f;
+// CTA-wide sums of p[0..16) (into out) and of lp (returned).  Every thread calls it; one barrier.
+__device__ __forceinline__ float cta_sum16(float (&p)[BW_CB], float lp, BwdRed &red, int par,
+                                           float (&out)[BW_CB]) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const float c = warp_reduce_scatter16(p, lane);
+    const float l = warp_sum(lp);
+    if ((lane & 1) == 0) red.col[par][w][lane >> 1] = c;
+    if (lane == 0) red.lam[par][w] = l;
     __syncthreads();
-    for (int t = 0; t < L; ++t) {
-        if (t % BWD_BLOCK == 0)
-            for (int e = tid; e < DD; e += BWD_THREADS) CK[(size_t)(t / BWD_BLOCK) * DD + e] = S[e];
-        float kk = 0.f;
-        if (tid < dk) {
-            const float kv = to_f32(k[tk + (size_t)t * dk + tid]);
-            ks[tid] = kv;
-            kk = kv * kv;
+#pragma unroll
+    for (int j4 = 0; j4 < BW_CB / 4; ++j4) {
+        float4 a = reinterpret_cast<const float4 *>(red.col[par][0])[j4];
+#pragma unroll
+        for (int ww = 1; ww < BW_THREADS / 32; ++ww) {
+            const float4 b = reinterpret_cast<const float4 *>(red.col[par][ww])[j4];
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
         }
-        const float lambda = block_sum(kk, red);  // (syncs: ks is visible)
-        const float a = alpha_rule(lambda, to_f32(beta[tb + t]), euler);
-        if (tid < dv) {  // r = v - S^T k
-            float x = 0.f;
-            for (int i = 0; i < dk; ++i) x = fmaf(S[i * dv + tid], ks[i], x);
-            const float r = to_f32(v[tv + (size_t)t * dv + tid]) - x;
-            rs[tid] = r;
-            R[(size_t)t * dv + tid] = r;
-        }
-        __syncthreads();
-        if (BWD_THREADS % dv == 0) {  // fixed column per thread: no division per element
-            const int j = tid % dv;
-            for (int i = tid / dv; i < dk; i += BWD_THREADS / dv)
-                S[i * dv + j] = fmaf(a * ks[i], rs[j], S[i * dv + j]);
-        } else {
-            for (int e = tid; e < DD; e += BWD_THREADS) S[e] = fmaf(a * ks[e / dv], rs[e % dv], S[e]);
-        }
-        __syncthreads();
+        out[4 * j4 + 0] = a.x; out[4 * j4 + 1] = a.y; out[4 * j4 + 2] = a.z; out[4 * j4 + 3] = a.w;
     }
-    for (int e = tid; e < DD; e += BWD_THREADS) CK[(size_t)NB * DD + e] = S[e];
+    const float4 lv = *reinterpret_cast<const float4 *>(red.lam[par]);
+    return ((lv.x + lv.y) + lv.z) + lv.w;
+}
+
+// Value j == i of a register array without dynamic indexing (which would go through local memory).
+__device__ __forceinline__ float pick(const float (&x)[BW_CB], int i) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < BW_CB; ++j) m = (i == j) ? x[j] : m;
+    return m;
+}
+
+__device__ __forceinline__ void load_row16(const float *p, float (&x)[BW_CB]) {
+#pragma unroll
+    for (int j4 = 0; j4 < BW_CB / 4; ++j4) {
+        const float4 a = reinterpret_cast<const float4 *>(p)[j4];
+        x[4 * j4] = a.x; x[4 * j4 + 1] = a.y; x[4 * j4 + 2] = a.z; x[4 * j4 + 3] = a.w;
+    }
+}
+
+__device__ __forceinline__ void store_row16(float *p, const float (&x)[BW_CB]) {
+#pragma unroll
+    for (int j4 = 0; j4 < BW_CB / 4; ++j4)
+        reinterpret_cast<float4 *>(p)[j4] = make_float4(x[4 * j4], x[4 * j4 + 1], x[4 * j4 + 2], x[4 * j4 + 3]);
+}
+
+// Workspace, per (head, column block): r of every token [L][16], then the block's state at every
+// 64-token boundary and at the end [NB + 1][dk][16]; after all of those the column blocks' shares
+// of dq and dk ([NS][B*H][L][dk] each) and of dbeta ([NS][B*H][L]).
+template <typename T>
+__global__ void __launch_bounds__(BW_THREADS, 4)
+    bwd_cols_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                    const T *__restrict__ beta, const float *__restrict__ S0,
+                    const float *__restrict__ dO, const float *__restrict__ dSL,
+                    float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
+                    bool euler, float *__restrict__ ws, float *__restrict__ part) {
+    __shared__ __align__(16) BwdRed red;
+    __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
+    __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
+    __shared__ float bb[BWD_BLOCK];                         // beta
+    const int tid = threadIdx.x, row = tid;
+    const int bh = blockIdx.x / NS, s = blockIdx.x % NS, c0 = s * BW_CB;
+    const int BH = gridDim.x / NS, nc = min(BW_CB, dv - c0);
+    const int NB = (L + BWD_BLOCK - 1) / BWD_BLOCK;
+    const bool act = row < dk;
+    const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
+    const size_t DD = (size_t)dk * dv;
+    float *R = ws + ((size_t)bh * NS + s) * ((size_t)L * BW_CB + (size_t)(NB + 1) * dk * BW_CB);
+    float *CK = R + (size_t)L * BW_CB;
+    const size_t nq = (size_t)BH * L * dk;
+    float *pdq = part + (size_t)s * nq + tk;
+    float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
+    float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
+
+    float S[BW_CB], G[BW_CB];
+#pragma unroll
+    for (int j = 0; j < BW_CB; ++j)
+        S[j] = (S0 && act && j < nc) ? S0[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
+
+    // ---- forward sweep: r of every token and the block-boundary states
+    int par = 0;
+    float kr1 = (act && L > 0) ? to_f32(k[tk + row]) : 0.f;
+    float kr2 = (act && L > 1) ? to_f32(k[tk + dk + row]) : 0.f;
+    for (int b = 0; b < NB; ++b) {
+        const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
+        __syncthreads();  // the previous block's reads of xb and bb are done
+        for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
+            const int tt = e / BW_CB, j = e % BW_CB;
+            xb[tt][j] = j < nc ? to_f32(v[tv + (size_t)(t0 + tt) * dv + c0 + j]) : 0.f;
+        }
+        for (int e = tid; e < cnt; e += BW_THREADS) bb[e] = to_f32(beta[tb + t0 + e]);
+        if (act) store_row16(CK + ((size_t)b * dk + row) * BW_CB, S);
+        __syncthreads();
+        for (int tt = 0; tt < cnt; ++tt) {
+            const int t = t0 + tt;
+            const float ki = kr1;
+            kr1 = kr2;
+            kr2 = (act && t + 2 < L) ? to_f32(k[tk + (size_t)(t + 2) * dk + row]) : 0.f;
+            float p[BW_CB], x[BW_CB], r[BW_CB];
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) p[j] = S[j] * ki;
+            const float lambda = cta_sum16(p, ki * ki, red, par, x);  // x = S^T k
+            const float a = alpha_rule(lambda, bb[tt], euler);
+            load_row16(xb[tt], r);
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) r[j] -= x[j];  // r = v - S^T k
+            if (tid < BW_CB) R[(size_t)t * BW_CB + tid] = pick(r, tid);
+            const float ak = a * ki;
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) S[j] = fmaf(ak, r[j], S[j]);
+            par ^= 1;
+        }
+    }
+    if (act) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
 
     // ---- reverse sweep
-    for (int e = tid; e < DD; e += BWD_THREADS) G[e] = dSL ? dSL[(size_t)bh * DD + e] : 0.f;
-    const int row = tid >> 1, half = tid & 1;  // two threads per state row for row reductions
+#pragma unroll
+    for (int j = 0; j < BW_CB; ++j)
+        G[j] = (dSL && act && j < nc) ? dSL[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
+    kr1 = (act && L > 0) ? to_f32(k[tk + (size_t)(L - 1) * dk + row]) : 0.f;
+    kr2 = (act && L > 1) ? to_f32(k[tk + (size_t)(L - 2) * dk + row]) : 0.f;
+    float qr1 = (act && L > 0) ? to_f32(q[tk + (size_t)(L - 1) * dk + row]) : 0.f;
+    float qr2 = (act && L > 1) ? to_f32(q[tk + (size_t)(L - 2) * dk + row]) : 0.f;
     for (int b = NB - 1; b >= 0; --b) {
+        const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
+        __syncthreads();  // the previous block's reads of xb, rb and bb are done
+        for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
+            const int tt = e / BW_CB, j = e % BW_CB;
+            xb[tt][j] = j < nc ? dO[tv + (size_t)(t0 + tt) * dv + c0 + j] : 0.f;
+            rb[tt][j] = R[(size_t)(t0 + tt) * BW_CB + j];
+        }
+        for (int e = tid; e < cnt; e += BW_THREADS) bb[e] = to_f32(beta[tb + t0 + e]);
+        if (act) load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);  // S' after the block
         __syncthreads();
-        for (int e = tid; e < DD; e += BWD_THREADS) S[e] = CK[(size_t)(b + 1) * DD + e];
-        const int t_end = min(L, (b + 1) * BWD_BLOCK);
-        for (int t = t_end - 1; t >= b * BWD_BLOCK; --t) {
-            float kk = 0.f;
-            if (tid < dk) {
-                const float kv = to_f32(k[tk + (size_t)t * dk + tid]);
-                ks[tid] = kv;
-                kk = kv * kv;
-                qs[tid] = to_f32(q[tk + (size_t)t * dk + tid]);
+        for (int tt = cnt - 1; tt >= 0; --tt) {
+            const int t = t0 + tt;
+            const float ki = kr1, qi = qr1;
+            kr1 = kr2;
+            qr1 = qr2;
+            kr2 = (act && t >= 2) ? to_f32(k[tk + (size_t)(t - 2) * dk + row]) : 0.f;
+            qr2 = (act && t >= 2) ? to_f32(q[tk + (size_t)(t - 2) * dk + row]) : 0.f;
+            float d[BW_CB], r[BW_CB], p[BW_CB], du[BW_CB];
+            load_row16(xb[tt], d);
+            load_row16(rb[tt], r);
+            // G += q do^T;  dq = S' do
+            float dqp = 0.f;
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) {
+                G[j] = fmaf(qi, d[j], G[j]);
+                dqp = fmaf(S[j], d[j], dqp);
             }
-            if (tid < dv) {
-                dos[tid] = dO[tv + (size_t)t * dv + tid];
-                rs[tid] = R[(size_t)t * dv + tid];
-            }
-            const float lambda = block_sum(kk, red);  // syncs: the vectors and S are visible
-            const float bt = to_f32(beta[tb + t]);
+            // du = G^T k
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) p[j] = G[j] * ki;
+            const float lambda = cta_sum16(p, ki * ki, red, par, du);
+            const float bt = bb[tt];
             const float a = alpha_rule(lambda, bt, euler);
-            // G += q do^T; dq = S' do (S holds S' = the state after token t)
-            if (BWD_THREADS % dv == 0) {
-                const int j = tid % dv;
-                for (int i = tid / dv; i < dk; i += BWD_THREADS / dv)
-                    G[i * dv + j] = fmaf(qs[i], dos[j], G[i * dv + j]);
-            } else {
-                for (int e = tid; e < DD; e += BWD_THREADS) G[e] = fmaf(qs[e / dv], dos[e % dv], G[e]);
+            float da = 0.f;  // this column block's share of da = du . r
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) da = fmaf(du[j], r[j], da);
+            // S = S' - a k r^T;  dk = a G r - a S du + 2 da df/dlambda k;  G -= a k du^T
+            const float ak = a * ki;
+            float gr = 0.f, sdu = 0.f;
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j) {
+                S[j] = fmaf(-ak, r[j], S[j]);
+                gr = fmaf(G[j], r[j], gr);
+                sdu = fmaf(S[j], du[j], sdu);
+                G[j] = fmaf(-ak, du[j], G[j]);
             }
-            {
-                float s = row < dk ? row_dot_half(S, dos, row, half, dv) : 0.f;
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                if (row < dk && half == 0) dq[tk + (size_t)t * dk + row] = s;
-            }
-            __syncthreads();
-            // du = G^T k, dv = a du, da = du . r
-            float dap = 0.f;
-            if (tid < dv) {
-                float s = 0.f;
-                for (int i = 0; i < dk; ++i) s = fmaf(G[i * dv + tid], ks[i], s);
-                dxs[tid] = -a * s;
-                dval[tv + (size_t)t * dv + tid] = a * s;
-                dap = s * rs[tid];
-            }
-            const float da = block_sum(dap, red);  // syncs: dxs visible
-            // dk = G u + (added below) S dx + 2 da df/dlambda k, with u = a r
-            float dka = row < dk ? a * row_dot_half(G, rs, row, half, dv) : 0.f;  // G u, u = a r
-            dka += __shfl_xor_sync(0xffffffffu, dka, 1);
-            const float krow = row < dk ? ks[row] : 0.f;  // ks is rewritten by the next token
-            __syncthreads();  // every read of G and S' for this token is done
-            // S = S' - a k r^T (the state before token t); G += k dx^T (dL/dS)
-            if (BWD_THREADS % dv == 0) {
-                const int j = tid % dv;
-                for (int i = tid / dv; i < dk; i += BWD_THREADS / dv) {
-                    S[i * dv + j] = fmaf(-a * ks[i], rs[j], S[i * dv + j]);
-                    G[i * dv + j] = fmaf(ks[i], dxs[j], G[i * dv + j]);
-                }
-            } else {
-                for (int e = tid; e < DD; e += BWD_THREADS) {
-                    const int i = e / dv, j = e % dv;
-                    S[e] = fmaf(-a * ks[i], rs[j], S[e]);
-                    G[e] = fmaf(ks[i], dxs[j], G[e]);
-                }
-            }
-            __syncthreads();
-            float dkb = row < dk ? row_dot_half(S, dxs, row, half, dv) : 0.f;
-            dkb += __shfl_xor_sync(0xffffffffu, dkb, 1);
             float dfdb, dfdl;
             coeff_grads(lambda, bt, euler, a, dfdb, dfdl);
-            if (row < dk && half == 0)
-                dkey[tk + (size_t)t * dk + row] = dka + dkb + 2.f * da * dfdl * krow;
-            if (tid == 0) dbeta[tb + t] = da * dfdb;
+            if (act) {
+                pdq[(size_t)t * dk + row] = dqp;
+                pdk[(size_t)t * dk + row] = a * (gr - sdu) + 2.f * da * dfdl * ki;
+            }
+            if (tid < nc) dval[tv + (size_t)t * dv + c0 + tid] = a * pick(du, tid);
+            if (tid == 0) pdb[t] = da * dfdb;
+            par ^= 1;
         }
     }
-    __syncthreads();
-    if (dS0)
-        for (int e = tid; e < DD; e += BWD_THREADS) dS0[(size_t)bh * DD + e] = G[e];
+    if (dS0 && act) {
+#pragma unroll
+        for (int j = 0; j < BW_CB; ++j)
+            if (j < nc) dS0[(size_t)bh * DD + (size_t)row * dv + c0 + j] = G[j];
+    }
+}
+
+// out[e] = sum over s = 0..NS-1 of part[s n + e], in that order (blockIdx.y picks dq, dk, dbeta).
+struct SumSeg {
+    const float *part;
+    float *out;
+    size_t n;
+    int vec;  // 1: n % 4 == 0 and both arrays 16-byte aligned
+};
+struct SumSegs {
+    SumSeg seg[3];
+};
+
+__global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS) {
+    const SumSeg g = blockIdx.y == 0 ? segs.seg[0] : (blockIdx.y == 1 ? segs.seg[1] : segs.seg[2]);
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g.vec) {
+        const size_t n4 = g.n / 4;
+        const float4 *p4 = reinterpret_cast<const float4 *>(g.part);
+        float4 *o4 = reinterpret_cast<float4 *>(g.out);
+        for (size_t e = i0; e < n4; e += stride) {
+            float4 a = p4[e];
+            for (int s = 1; s < NS; ++s) {
+                const float4 b = p4[(size_t)s * n4 + e];
+                a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+            }
+            o4[e] = a;
+        }
+    } else {
+        for (size_t e = i0; e < g.n; e += stride) {
+            float a = g.part[e];
+            for (int s = 1; s < NS; ++s) a += g.part[(size_t)s * g.n + e];
+            g.out[e] = a;
+        }
+    }
+}
+
+static size_t bwd_state_floats(size_t BH, int L, int dk, int dv) {
+    const size_t NB = (size_t)(L + BWD_BLOCK - 1) / BWD_BLOCK;
+    const size_t NS = (size_t)(dv + BW_CB - 1) / BW_CB;
+    return BH * NS * ((size_t)L * BW_CB + (NB + 1) * (size_t)dk * BW_CB);
 }
 
 size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv) {
-    const size_t NB = (size_t)(L + BWD_BLOCK - 1) / BWD_BLOCK;
-    return (size_t)B * H * ((size_t)L * dv + (NB + 1) * (size_t)dk * dv) * sizeof(float);
+    const size_t BH = (size_t)B * H, NS = (size_t)(dv + BW_CB - 1) / BW_CB;
+    const size_t shares = NS * BH * (size_t)L * (2 * (size_t)dk + 1);
+    return (bwd_state_floats(BH, L, dk, dv) + shares) * sizeof(float);
 }
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
                        const float *S0, const float *dO, const float *dSL, float *dq, float *dkey,
                        float *dval, float *dbeta, float *dS0, int B, int H, int L, int dk, int dv,
                        bool is_bf16, bool euler, void *ws, cudaStream_t s) {
-    const int BH = B * H;
-    const size_t smem = (size_t)(2 * dk * dv + 5 * 128 + 32) * sizeof(float);
-    cudaError_t e;
-    if (is_bf16) {
-        e = cudaFuncSetAttribute(bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        bwd_kernel<__nv_bfloat16><<<BH, BWD_THREADS, smem, s>>>(
+    const long long BH = (long long)B * H;
+    const int NS = (dv + BW_CB - 1) / BW_CB;
+    if (BH * NS > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    float *state = (float *)ws;
+    float *part = state + bwd_state_floats((size_t)BH, L, dk, dv);
+    const int grid = (int)(BH * NS);
+    if (is_bf16)
+        bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            (const __nv_bfloat16 *)beta, S0, dO, dSL, dq, dkey, dval, dbeta, dS0, L, dk, dv, euler,
-            (float *)ws);
-    } else {
-        e = cudaFuncSetAttribute(bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        bwd_kernel<float><<<BH, BWD_THREADS, smem, s>>>((const float *)q, (const float *)k, (const float *)v,
-                                                       (const float *)beta, S0, dO, dSL, dq, dkey, dval,
-                                                       dbeta, dS0, L, dk, dv, euler, (float *)ws);
-    }
+            (const __nv_bfloat16 *)beta, S0, dO, dSL, dval, dS0, L, dk, dv, NS, euler, state, part);
+    else
+        bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
+                                                          (const float *)v, (const float *)beta, S0,
+                                                          dO, dSL, dval, dS0, L, dk, dv, NS, euler,
+                                                          state, part);
+    count_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || L == 0) return e;
+    // add the column blocks' shares of dq, dk and dbeta
+    const size_t nq = (size_t)BH * L * dk, nb = (size_t)BH * L;
+    auto seg = [&](const float *pp, float *out, size_t n) {
+        SumSeg g;
+        g.part = pp;
+        g.out = out;
+        g.n = n;
+        g.vec = (n % 4 == 0 && ((uintptr_t)pp % 16) == 0 && ((uintptr_t)out % 16) == 0) ? 1 : 0;
+        return g;
+    };
+    SumSegs segs;
+    segs.seg[0] = seg(part, dq, nq);
+    segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq);
+    segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb);
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const size_t want = (nq / 4 + 255) / 256;
+    const int gx = (int)std::min<size_t>(std::max<size_t>(want, 1), (size_t)nsm * 8);
+    bwd_sum_kernel<<<dim3(gx, 3), 256, 0, s>>>(segs, NS);
     count_launches(1);
     return cudaGetLastError();
 }

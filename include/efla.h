@@ -245,10 +245,15 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *H,
  *   S0 : [B,H,dk,dv] fp32 or NULL        dO : [B,H,L,dv] fp32
  *   dq, dkey : [B,H,L,dk] fp32   dval : [B,H,L,dv] fp32   dbeta : [B,H,L] fp32
  *   dS0 : [B,H,dk,dv] fp32 or NULL
- *   workspace : efla_bwd_workspace_size(B,H,L,dk,dv) bytes, caller-owned scratch
- * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  Pointers aligned to their element.
- * One CTA per head walks the sequence twice (forward, then reverse): a first,
- * correct path whose time grows with L per head, not a tuned kernel.
+ *   workspace : efla_bwd_workspace_size(B,H,L,dk,dv) bytes, caller-owned scratch,
+ *               16-byte aligned
+ * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  Other pointers aligned to their
+ * element.  The state's columns evolve independently, so one CTA takes one head
+ * and 16 of its state columns and walks the sequence twice (forward, then
+ * reverse); dq, dkey and dbeta are sums over the columns, and a second kernel adds
+ * the column blocks' shares in a fixed order (the result does not depend on
+ * scheduling).  EFLA_ERR_ALIGN: a misaligned pointer.  EFLA_ERR_WORKSPACE: the
+ * workspace is missing or too small.
  */
 size_t efla_bwd_workspace_size(int B, int H, int L, int dk, int dv);
 efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,

@@ -142,3 +142,23 @@ def test_selftest_budget_is_checked_on_the_host(lib):
     EFLA_ERR_SHAPE = 2
     assert lib.efla_selftest_bounded_wait(0, None) == EFLA_ERR_SHAPE
     assert lib.efla_selftest_bounded_wait(3_000_000_000, None) == EFLA_ERR_SHAPE
+
+
+def test_bwd_workspace_size_and_alignment(lib):
+    """The backward's workspace: per (head, 16-column block) r of every token and the block's
+    state every 64 tokens and at the end, then the column blocks' shares of dq, dk and dbeta.
+    A workspace that is not 16-byte aligned is refused before any CUDA call."""
+    B, H, L, dk, dv = 4, 16, 4096, 128, 128
+    NS, NB = 8, 64
+    state = B * H * NS * (L * 16 + (NB + 1) * dk * 16)
+    shares = NS * B * H * L * (2 * dk + 1)
+    assert lib.efla_bwd_workspace_size(B, H, L, dk, dv) == 4 * (state + shares)
+    # ragged: dv = 20 takes two column blocks, L = 65 two token blocks
+    assert lib.efla_bwd_workspace_size(1, 1, 65, 8, 20) == 4 * (2 * (65 * 16 + 3 * 8 * 16) + 2 * 65 * 17)
+    assert lib.efla_bwd_workspace_size(1, 1, 16, 129, 16) == 0
+    P = ctypes.c_void_p(64)
+    EFLA_ERR_ALIGN, EFLA_ERR_WORKSPACE = 8, 7
+    args = [P, P, P, P, None, P, None, P, P, P, P, None, 1, 1, 16, 16, 16, F32, 0]
+    need = lib.efla_bwd_workspace_size(1, 1, 16, 16, 16)
+    assert lib.efla_bwd(*args, ctypes.c_void_p(64 + 4), need, None) == EFLA_ERR_ALIGN
+    assert lib.efla_bwd(*args, P, need - 4, None) == EFLA_ERR_WORKSPACE

@@ -33,7 +33,10 @@ def _case(wid, rule, seed=5, **kw):
 
 @pytest.mark.parametrize("rule", ["exact", "euler"])
 @pytest.mark.parametrize("wid,kw", [(1, {}), (2, dict(B=1, H=2, L=130, dk=32, dv=16)),
-                                    (4, dict(B=1, H=2, L=200)), (3, dict(B=1, H=1, L=77, dk=128, dv=64))])
+                                    (4, dict(B=1, H=2, L=200)), (3, dict(B=1, H=1, L=77, dk=128, dv=64)),
+                                    (2, dict(B=2, H=1, L=65, dk=40, dv=20)),
+                                    (3, dict(B=1, H=1, L=64, dk=7, dv=5)),
+                                    (4, dict(B=1, H=1, L=129, dk=128, dv=100))])
 def test_backward_matches_oracle(oracle_mod, rule, wid, kw):
     x = _case(wid, rule, **kw)
     d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
@@ -64,3 +67,14 @@ def test_backward_empty_sequence_passes_the_state_gradient_through():
     dq, dk, dv, db, dS0 = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
     torch.cuda.synchronize()
     assert dq.numel() == 0 and torch.equal(dS0.cpu(), x["dS"])
+
+
+def test_backward_is_deterministic():
+    """The column blocks' shares are added in a fixed order: two runs agree bit for bit."""
+    x = _case(4, "exact", B=1, H=3, L=300)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    a = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
+    b = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
+    torch.cuda.synchronize()
+    for u, w in zip(a, b):
+        assert torch.equal(u, w)
