@@ -84,11 +84,13 @@ def run_bwd(args) -> None:
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = ClockSampler(0)
     clk.start()
+    l0 = efla.kernel_launches()
     a.record()
     for _ in range(args.steps):
         call()
     b.record()
     torch.cuda.synchronize(dev)
+    launches = efla.kernel_launches() - l0
     clocks = clk.stop()
     ms = a.elapsed_time(b) / args.steps
     alg = alg_bytes_bwd(w)
@@ -100,9 +102,9 @@ def run_bwd(args) -> None:
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic", "config": _config(w),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm"], "traffic": None, "kernel": "efla_bwd (SIMT)",
+                     "frac": achieved / peaks["hbm"], "traffic": None, "kernel": "efla_bwd (SIMT: coefficients, column-block sweeps, share sum)",
                      "alg_bytes_per_launch": alg, "avg_launch_ms": ms},
-        "gpu_launches": args.steps, "clocks": clocks}))
+        "gpu_launches": int(launches), "clocks": clocks}))
 
 
 def alg_bytes_decode(Bd, Hd, dk, dv, es=2) -> int:
@@ -164,16 +166,18 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+FWD_SOURCES = ("chunk_tc.cu", "common.cuh", "tc_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources the library is built from (ties profiled counters to a build)."""
-    import glob
+    """Hash of the CUDA sources the chunk forward's kernels are built from (the tcgen05 prep,
+    state and segment kernels and the helpers they include): ties profiled counters to them."""
     import hashlib
 
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "delta_rule_linear_efla_b200", "csrc", "*"))):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(os.path.basename(f).encode())
-            h.update(open(f, "rb").read())
+    for f in FWD_SOURCES:
+        h.update(f.encode())
+        h.update(open(os.path.join(ROOT, "delta_rule_linear_efla_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 

@@ -28,8 +28,13 @@
 
 namespace efla {
 
-constexpr int BW_THREADS = 128;  // one state row per thread (dk <= 128)
-constexpr int BW_CB = 16;        // state columns per CTA
+#ifndef EFLA_BWD_ROWS_PER_THREAD
+#define EFLA_BWD_ROWS_PER_THREAD 1
+#endif
+constexpr int BW_RPT = EFLA_BWD_ROWS_PER_THREAD;  // state rows per thread
+constexpr int BW_THREADS = 128 / BW_RPT;           // 128 rows per CTA (dk <= 128)
+constexpr int BW_MINB = BW_RPT == 1 ? 4 : 6;       // CTAs per SM the register budget allows
+constexpr int BW_CB = 16;                          // state columns per CTA
 constexpr int BWD_BLOCK = 64;    // tokens between stored states
 
 // df/dbeta and df/dlambda of the coefficient under the rule.
@@ -51,8 +56,27 @@ __device__ __forceinline__ void coeff_grads(float lambda, float beta, bool euler
 
 struct BwdRed {  // the four warps' shares of one CTA-wide sum, double-buffered by token parity
     float col[2][BW_THREADS / 32][BW_CB];
-    float lam[2][BW_THREADS / 32];
 };
+
+// Two fp32 lanes at once (packed f32x2 arithmetic of sm_100; each lane rounds as the scalar op).
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rd, {%0, %1};\n\tfma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1) {
+    asm("{\n\t.reg .b64 ra, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+        "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
 
 // Sum over the warp of 16 values per lane, scattered: every lane returns the sum of value
 // (lane >> 1).  Each step halves the values a lane keeps and trades the other half with the
@@ -84,35 +108,26 @@ __device__ __forceinline__ float warp_reduce_scatter16(float (&p)[BW_CB], int la
     return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
 }
 
-// CTA-wide sums of p[0..16) (into out) and of lp (returned).  Every thread calls it; one barrier.
-__device__ __forceinline__ float cta_sum16(float (&p)[BW_CB], float lp, BwdRed &red, int par,
-                                           float (&out)[BW_CB]) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const float c = warp_reduce_scatter16(p, lane);
-    const float l = warp_sum(lp);
-    if ((lane & 1) == 0) red.col[par][w][lane >> 1] = c;
-    if (lane == 0) red.lam[par][w] = l;
-    __syncthreads();
+// Column c of a CTA-wide sum: the four warps' shares added in the order 0, 1, 2, 3.
+__device__ __forceinline__ float col_sum(const BwdRed &red, int par, int c) {
+    float a = red.col[par][0][c];
 #pragma unroll
-    for (int j4 = 0; j4 < BW_CB / 4; ++j4) {
-        float4 a = reinterpret_cast<const float4 *>(red.col[par][0])[j4];
-#pragma unroll
-        for (int ww = 1; ww < BW_THREADS / 32; ++ww) {
-            const float4 b = reinterpret_cast<const float4 *>(red.col[par][ww])[j4];
-            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-        }
-        out[4 * j4 + 0] = a.x; out[4 * j4 + 1] = a.y; out[4 * j4 + 2] = a.z; out[4 * j4 + 3] = a.w;
-    }
-    const float4 lv = *reinterpret_cast<const float4 *>(red.lam[par]);
-    return ((lv.x + lv.y) + lv.z) + lv.w;
+    for (int ww = 1; ww < BW_THREADS / 32; ++ww) a += red.col[par][ww][c];
+    return a;
 }
 
-// Value j == i of a register array without dynamic indexing (which would go through local memory).
-__device__ __forceinline__ float pick(const float (&x)[BW_CB], int i) {
-    float m = 0.f;
+// CTA-wide sums of p[0..16) into out (every thread calls it; one barrier).  Each lane adds up
+// one column's four warp shares (lanes 2c and 2c + 1 take column c) and the totals reach every
+// lane by shuffles: shared memory sees one conflict-free load per warp share, not a broadcast
+// read of all 64 shares by every thread.
+__device__ __forceinline__ void cta_sum16(float (&p)[BW_CB], BwdRed &red, int par, float (&out)[BW_CB]) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const float c = warp_reduce_scatter16(p, lane);
+    if ((lane & 1) == 0) red.col[par][w][lane >> 1] = c;
+    __syncthreads();
+    const float t = col_sum(red, par, lane >> 1);
 #pragma unroll
-    for (int j = 0; j < BW_CB; ++j) m = (i == j) ? x[j] : m;
-    return m;
+    for (int j = 0; j < BW_CB; ++j) out[j] = __shfl_sync(0xffffffffu, t, 2 * j);
 }
 
 __device__ __forceinline__ void load_row16(const float *p, float (&x)[BW_CB]) {
@@ -129,25 +144,56 @@ __device__ __forceinline__ void store_row16(float *p, const float (&x)[BW_CB]) {
         reinterpret_cast<float4 *>(p)[j4] = make_float4(x[4 * j4], x[4 * j4 + 1], x[4 * j4 + 2], x[4 * j4 + 3]);
 }
 
-// Workspace, per (head, column block): r of every token [L][16], then the block's state at every
-// 64-token boundary and at the end [NB + 1][dk][16]; after all of those the column blocks' shares
-// of dq and dk ([NS][B*H][L][dk] each) and of dbeta ([NS][B*H][L]).
+// Per token: (lambda = |k|^2, a = f(lambda, beta), df/dbeta, df/dlambda), one warp per token.
+// Every column block of a head reads them, so they are computed once, ahead of the sweeps.
 template <typename T>
-__global__ void __launch_bounds__(BW_THREADS, 4)
+__global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ k, const T *__restrict__ beta,
+                                                       size_t ntok, int dk, bool euler,
+                                                       float4 *__restrict__ coef) {
+    const int lane = threadIdx.x & 31;
+    for (size_t tok = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); tok < ntok; tok += (size_t)gridDim.x * 8) {
+        float s = 0.f;
+        for (int i = lane; i < dk; i += 32) {
+            const float x = to_f32(k[tok * dk + i]);
+            s = fmaf(x, x, s);
+        }
+        s = warp_sum(s);
+        if (lane == 0) {
+            const float bt = to_f32(beta[tok]);
+            const float a = alpha_rule(s, bt, euler);
+            float dfdb, dfdl;
+            coeff_grads(s, bt, euler, a, dfdb, dfdl);
+            coef[tok] = make_float4(s, a, dfdb, dfdl);
+        }
+    }
+}
+
+// Workspace: the per-token coefficients [B*H][L] (float4); per (head, column block) r of every
+// token [L][16], then the block's state at every 64-token boundary and at the end
+// [NB + 1][dk][16]; after all of those the column blocks' shares of dq and dk
+// ([NS][B*H][L][dk] each) and of dbeta ([NS][B*H][L]).
+template <typename T>
+__global__ void __launch_bounds__(BW_THREADS, BW_MINB)
     bwd_cols_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                    const T *__restrict__ beta, const float *__restrict__ S0,
+                    const float4 *__restrict__ coef, const float *__restrict__ S0,
                     const float *__restrict__ dO, const float *__restrict__ dSL,
                     float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
-                    bool euler, float *__restrict__ ws, float *__restrict__ part) {
+                    float *__restrict__ ws, float *__restrict__ part) {
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
-    __shared__ float bb[BWD_BLOCK];                         // beta
-    const int tid = threadIdx.x, row = tid;
+    __shared__ __align__(16) float4 cb[BWD_BLOCK];        // the block's token coefficients
+    const int tid = threadIdx.x;
     const int bh = blockIdx.x / NS, s = blockIdx.x % NS, c0 = s * BW_CB;
     const int BH = gridDim.x / NS, nc = min(BW_CB, dv - c0);
     const int NB = (L + BWD_BLOCK - 1) / BWD_BLOCK;
-    const bool act = row < dk;
+    int row[BW_RPT];  // this thread's state rows: tid, tid + BW_THREADS, ...
+    bool act[BW_RPT];
+#pragma unroll
+    for (int u = 0; u < BW_RPT; ++u) {
+        row[u] = tid + u * BW_THREADS;
+        act[u] = row[u] < dk;
+    }
     const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
     const size_t DD = (size_t)dk * dv;
     float *R = ws + ((size_t)bh * NS + s) * ((size_t)L * BW_CB + (size_t)(NB + 1) * dk * BW_CB);
@@ -156,118 +202,165 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     float *pdq = part + (size_t)s * nq + tk;
     float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
     float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
+    auto ld = [&](const T *x, int t, int u) {  // element row[u] of token t's q or k (0 off the edge)
+        return (act[u] && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row[u]]) : 0.f;
+    };
 
-    float S[BW_CB], G[BW_CB];
+    float S[BW_RPT][BW_CB], G[BW_RPT][BW_CB];
 #pragma unroll
-    for (int j = 0; j < BW_CB; ++j)
-        S[j] = (S0 && act && j < nc) ? S0[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
+    for (int u = 0; u < BW_RPT; ++u)
+#pragma unroll
+        for (int j = 0; j < BW_CB; ++j)
+            S[u][j] = (S0 && act[u] && j < nc) ? S0[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] : 0.f;
 
     // ---- forward sweep: r of every token and the block-boundary states
     int par = 0;
-    float kr1 = (act && L > 0) ? to_f32(k[tk + row]) : 0.f;
-    float kr2 = (act && L > 1) ? to_f32(k[tk + dk + row]) : 0.f;
+    float kr1[BW_RPT], kr2[BW_RPT], qr1[BW_RPT], qr2[BW_RPT];
+#pragma unroll
+    for (int u = 0; u < BW_RPT; ++u) {
+        kr1[u] = ld(k, 0, u);
+        kr2[u] = ld(k, 1, u);
+    }
     for (int b = 0; b < NB; ++b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
-        __syncthreads();  // the previous block's reads of xb and bb are done
+        __syncthreads();  // the previous block's reads of xb and cb are done
         for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
             const int tt = e / BW_CB, j = e % BW_CB;
             xb[tt][j] = j < nc ? to_f32(v[tv + (size_t)(t0 + tt) * dv + c0 + j]) : 0.f;
         }
-        for (int e = tid; e < cnt; e += BW_THREADS) bb[e] = to_f32(beta[tb + t0 + e]);
-        if (act) store_row16(CK + ((size_t)b * dk + row) * BW_CB, S);
+        for (int e = tid; e < cnt; e += BW_THREADS) cb[e] = coef[tb + t0 + e];
+#pragma unroll
+        for (int u = 0; u < BW_RPT; ++u)
+            if (act[u]) store_row16(CK + ((size_t)b * dk + row[u]) * BW_CB, S[u]);
         __syncthreads();
         for (int tt = 0; tt < cnt; ++tt) {
             const int t = t0 + tt;
-            const float ki = kr1;
-            kr1 = kr2;
-            kr2 = (act && t + 2 < L) ? to_f32(k[tk + (size_t)(t + 2) * dk + row]) : 0.f;
+            float ki[BW_RPT];
+#pragma unroll
+            for (int u = 0; u < BW_RPT; ++u) {
+                ki[u] = kr1[u];
+                kr1[u] = kr2[u];
+                kr2[u] = ld(k, t + 2, u);
+            }
             float p[BW_CB], x[BW_CB], r[BW_CB];
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) p[j] = S[j] * ki;
-            const float lambda = cta_sum16(p, ki * ki, red, par, x);  // x = S^T k
-            const float a = alpha_rule(lambda, bb[tt], euler);
+            for (int j = 0; j < BW_CB; j += 2) {
+                mul2(p[j], p[j + 1], S[0][j], S[0][j + 1], ki[0], ki[0]);
+#pragma unroll
+                for (int u = 1; u < BW_RPT; ++u) fma2(p[j], p[j + 1], S[u][j], S[u][j + 1], ki[u], ki[u]);
+            }
+            cta_sum16(p, red, par, x);  // x = S^T k
+            const float a = cb[tt].y;
             load_row16(xb[tt], r);
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) r[j] -= x[j];  // r = v - S^T k
-            if (tid < BW_CB) R[(size_t)t * BW_CB + tid] = pick(r, tid);
-            const float ak = a * ki;
+            for (int j = 0; j < BW_CB; j += 2) add2(r[j], r[j + 1], -x[j], -x[j + 1]);  // r = v - S^T k
+            if (tid < BW_CB) R[(size_t)t * BW_CB + tid] = xb[tt][tid] + -col_sum(red, par, tid);
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) S[j] = fmaf(ak, r[j], S[j]);
+            for (int u = 0; u < BW_RPT; ++u) {
+                const float ak = a * ki[u];
+#pragma unroll
+                for (int j = 0; j < BW_CB; j += 2) fma2(S[u][j], S[u][j + 1], ak, ak, r[j], r[j + 1]);
+            }
             par ^= 1;
         }
     }
-    if (act) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
+#pragma unroll
+    for (int u = 0; u < BW_RPT; ++u)
+        if (act[u]) store_row16(CK + ((size_t)NB * dk + row[u]) * BW_CB, S[u]);
 
     // ---- reverse sweep
 #pragma unroll
-    for (int j = 0; j < BW_CB; ++j)
-        G[j] = (dSL && act && j < nc) ? dSL[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
-    kr1 = (act && L > 0) ? to_f32(k[tk + (size_t)(L - 1) * dk + row]) : 0.f;
-    kr2 = (act && L > 1) ? to_f32(k[tk + (size_t)(L - 2) * dk + row]) : 0.f;
-    float qr1 = (act && L > 0) ? to_f32(q[tk + (size_t)(L - 1) * dk + row]) : 0.f;
-    float qr2 = (act && L > 1) ? to_f32(q[tk + (size_t)(L - 2) * dk + row]) : 0.f;
+    for (int u = 0; u < BW_RPT; ++u) {
+#pragma unroll
+        for (int j = 0; j < BW_CB; ++j)
+            G[u][j] = (dSL && act[u] && j < nc) ? dSL[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] : 0.f;
+        kr1[u] = ld(k, L - 1, u);
+        kr2[u] = ld(k, L - 2, u);
+        qr1[u] = ld(q, L - 1, u);
+        qr2[u] = ld(q, L - 2, u);
+    }
     for (int b = NB - 1; b >= 0; --b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
-        __syncthreads();  // the previous block's reads of xb, rb and bb are done
+        __syncthreads();  // the previous block's reads of xb, rb and cb are done
         for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
             const int tt = e / BW_CB, j = e % BW_CB;
             xb[tt][j] = j < nc ? dO[tv + (size_t)(t0 + tt) * dv + c0 + j] : 0.f;
             rb[tt][j] = R[(size_t)(t0 + tt) * BW_CB + j];
         }
-        for (int e = tid; e < cnt; e += BW_THREADS) bb[e] = to_f32(beta[tb + t0 + e]);
-        if (act) load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);  // S' after the block
+        for (int e = tid; e < cnt; e += BW_THREADS) cb[e] = coef[tb + t0 + e];
+#pragma unroll
+        for (int u = 0; u < BW_RPT; ++u)  // S' after the block
+            if (act[u]) load_row16(CK + ((size_t)(b + 1) * dk + row[u]) * BW_CB, S[u]);
         __syncthreads();
         for (int tt = cnt - 1; tt >= 0; --tt) {
             const int t = t0 + tt;
-            const float ki = kr1, qi = qr1;
-            kr1 = kr2;
-            qr1 = qr2;
-            kr2 = (act && t >= 2) ? to_f32(k[tk + (size_t)(t - 2) * dk + row]) : 0.f;
-            qr2 = (act && t >= 2) ? to_f32(q[tk + (size_t)(t - 2) * dk + row]) : 0.f;
+            float ki[BW_RPT], qi[BW_RPT];
+#pragma unroll
+            for (int u = 0; u < BW_RPT; ++u) {
+                ki[u] = kr1[u];
+                qi[u] = qr1[u];
+                kr1[u] = kr2[u];
+                qr1[u] = qr2[u];
+                kr2[u] = ld(k, t - 2, u);
+                qr2[u] = ld(q, t - 2, u);
+            }
             float d[BW_CB], r[BW_CB], p[BW_CB], du[BW_CB];
             load_row16(xb[tt], d);
             load_row16(rb[tt], r);
             // G += q do^T;  dq = S' do
-            float dqp = 0.f;
+            float dq0[BW_RPT], dq1[BW_RPT];
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) {
-                G[j] = fmaf(qi, d[j], G[j]);
-                dqp = fmaf(S[j], d[j], dqp);
+            for (int u = 0; u < BW_RPT; ++u) {
+                dq0[u] = 0.f;
+                dq1[u] = 0.f;
+#pragma unroll
+                for (int j = 0; j < BW_CB; j += 2) {
+                    fma2(G[u][j], G[u][j + 1], qi[u], qi[u], d[j], d[j + 1]);
+                    fma2(dq0[u], dq1[u], S[u][j], S[u][j + 1], d[j], d[j + 1]);
+                }
             }
             // du = G^T k
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) p[j] = G[j] * ki;
-            const float lambda = cta_sum16(p, ki * ki, red, par, du);
-            const float bt = bb[tt];
-            const float a = alpha_rule(lambda, bt, euler);
-            float da = 0.f;  // this column block's share of da = du . r
+            for (int j = 0; j < BW_CB; j += 2) {
+                mul2(p[j], p[j + 1], G[0][j], G[0][j + 1], ki[0], ki[0]);
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) da = fmaf(du[j], r[j], da);
+                for (int u = 1; u < BW_RPT; ++u) fma2(p[j], p[j + 1], G[u][j], G[u][j + 1], ki[u], ki[u]);
+            }
+            cta_sum16(p, red, par, du);
+            const float4 cf = cb[tt];  // (lambda, a, df/dbeta, df/dlambda)
+            const float a = cf.y;
+            float da0 = 0.f, da1 = 0.f;  // this column block's share of da = du . r
+#pragma unroll
+            for (int j = 0; j < BW_CB; j += 2) fma2(da0, da1, du[j], du[j + 1], r[j], r[j + 1]);
+            const float da = da0 + da1;
             // S = S' - a k r^T;  dk = a G r - a S du + 2 da df/dlambda k;  G -= a k du^T
-            const float ak = a * ki;
-            float gr = 0.f, sdu = 0.f;
 #pragma unroll
-            for (int j = 0; j < BW_CB; ++j) {
-                S[j] = fmaf(-ak, r[j], S[j]);
-                gr = fmaf(G[j], r[j], gr);
-                sdu = fmaf(S[j], du[j], sdu);
-                G[j] = fmaf(-ak, du[j], G[j]);
+            for (int u = 0; u < BW_RPT; ++u) {
+                const float nak = -a * ki[u];
+                float gr0 = 0.f, gr1 = 0.f, sd0 = 0.f, sd1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < BW_CB; j += 2) {
+                    fma2(S[u][j], S[u][j + 1], nak, nak, r[j], r[j + 1]);
+                    fma2(gr0, gr1, G[u][j], G[u][j + 1], r[j], r[j + 1]);
+                    fma2(sd0, sd1, S[u][j], S[u][j + 1], du[j], du[j + 1]);
+                    fma2(G[u][j], G[u][j + 1], nak, nak, du[j], du[j + 1]);
+                }
+                if (act[u]) {
+                    pdq[(size_t)t * dk + row[u]] = dq0[u] + dq1[u];
+                    pdk[(size_t)t * dk + row[u]] = a * ((gr0 + gr1) - (sd0 + sd1)) + 2.f * da * cf.w * ki[u];
+                }
             }
-            float dfdb, dfdl;
-            coeff_grads(lambda, bt, euler, a, dfdb, dfdl);
-            if (act) {
-                pdq[(size_t)t * dk + row] = dqp;
-                pdk[(size_t)t * dk + row] = a * (gr - sdu) + 2.f * da * dfdl * ki;
-            }
-            if (tid < nc) dval[tv + (size_t)t * dv + c0 + tid] = a * pick(du, tid);
-            if (tid == 0) pdb[t] = da * dfdb;
+            if (tid < nc) dval[tv + (size_t)t * dv + c0 + tid] = a * col_sum(red, par, tid);
+            if (tid == 0) pdb[t] = da * cf.z;
             par ^= 1;
         }
     }
-    if (dS0 && act) {
+    if (dS0) {
 #pragma unroll
-        for (int j = 0; j < BW_CB; ++j)
-            if (j < nc) dS0[(size_t)bh * DD + (size_t)row * dv + c0 + j] = G[j];
+        for (int u = 0; u < BW_RPT; ++u)
+#pragma unroll
+            for (int j = 0; j < BW_CB; ++j)
+                if (act[u] && j < nc) dS0[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] = G[u][j];
     }
 }
 
@@ -315,8 +408,9 @@ static size_t bwd_state_floats(size_t BH, int L, int dk, int dv) {
 
 size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv) {
     const size_t BH = (size_t)B * H, NS = (size_t)(dv + BW_CB - 1) / BW_CB;
+    const size_t coef = 4 * BH * (size_t)L;
     const size_t shares = NS * BH * (size_t)L * (2 * (size_t)dk + 1);
-    return (bwd_state_floats(BH, L, dk, dv) + shares) * sizeof(float);
+    return (coef + bwd_state_floats(BH, L, dk, dv) + shares) * sizeof(float);
 }
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
@@ -326,18 +420,33 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     const long long BH = (long long)B * H;
     const int NS = (dv + BW_CB - 1) / BW_CB;
     if (BH * NS > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    float *state = (float *)ws;
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const size_t ntok = (size_t)BH * L;
+    float4 *coef = (float4 *)ws;
+    float *state = (float *)ws + 4 * ntok;
     float *part = state + bwd_state_floats((size_t)BH, L, dk, dv);
+    if (ntok > 0) {
+        const int gc = (int)std::min<size_t>((ntok + 7) / 8, (size_t)nsm * 64);
+        if (is_bf16)
+            bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)k,
+                                                               (const __nv_bfloat16 *)beta, ntok, dk,
+                                                               euler, coef);
+        else
+            bwd_coeff_kernel<float><<<gc, 256, 0, s>>>((const float *)k, (const float *)beta, ntok, dk,
+                                                       euler, coef);
+        count_launches(1);
+    }
     const int grid = (int)(BH * NS);
     if (is_bf16)
         bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            (const __nv_bfloat16 *)beta, S0, dO, dSL, dval, dS0, L, dk, dv, NS, euler, state, part);
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, dO,
+            dSL, dval, dS0, L, dk, dv, NS, state, part);
     else
         bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
-                                                          (const float *)v, (const float *)beta, S0,
-                                                          dO, dSL, dval, dS0, L, dk, dv, NS, euler,
-                                                          state, part);
+                                                          (const float *)v, coef, S0, dO, dSL, dval,
+                                                          dS0, L, dk, dv, NS, state, part);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || L == 0) return e;
@@ -355,9 +464,6 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     segs.seg[0] = seg(part, dq, nq);
     segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq);
     segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb);
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const size_t want = (nq / 4 + 255) / 256;
     const int gx = (int)std::min<size_t>(std::max<size_t>(want, 1), (size_t)nsm * 8);
     bwd_sum_kernel<<<dim3(gx, 3), 256, 0, s>>>(segs, NS);
