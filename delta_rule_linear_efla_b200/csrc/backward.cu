@@ -16,10 +16,12 @@
 //
 // A forward sweep stores each column block's r and its state every 64 tokens; the reverse sweep
 // starts each 64-token block from the stored state at its end and steps back with
-// S = S' - a k r^T, so rounding never accumulates over more than 64 tokens.  Each token takes
-// one CTA-wide sum (the 16 column dot products over the rows, and lambda = |k|^2): a
+// S = S' - a k r^T, so rounding never accumulates over more than 64 tokens.  Tokens go in
+// pairs, with one CTA-wide sum per pair (32 column dot products over the rows): a
 // reduce-scatter across each warp's lanes, then one barrier to add the four warps' shares
-// through shared memory, double-buffered by token parity so that one barrier per token suffices.
+// through shared memory, double-buffered by parity so that one barrier per pair suffices.
+// The per-token coefficients and the two dot products that link a pair's tokens come from a
+// prologue kernel.
 #include <algorithm>
 #include <cstdint>
 
@@ -28,14 +30,9 @@
 
 namespace efla {
 
-#ifndef EFLA_BWD_ROWS_PER_THREAD
-#define EFLA_BWD_ROWS_PER_THREAD 1
-#endif
-constexpr int BW_RPT = EFLA_BWD_ROWS_PER_THREAD;  // state rows per thread
-constexpr int BW_THREADS = 128 / BW_RPT;           // 128 rows per CTA (dk <= 128)
-constexpr int BW_MINB = BW_RPT == 1 ? 4 : 6;       // CTAs per SM the register budget allows
-constexpr int BW_CB = 16;                          // state columns per CTA
-constexpr int BWD_BLOCK = 64;    // tokens between stored states
+constexpr int BW_THREADS = 128;  // one state row per thread (dk <= 128)
+constexpr int BW_CB = 16;        // state columns per CTA
+constexpr int BWD_BLOCK = 64;    // tokens between stored states (even: tokens go in pairs)
 
 // df/dbeta and df/dlambda of the coefficient under the rule.
 __device__ __forceinline__ void coeff_grads(float lambda, float beta, bool euler, float a,
@@ -54,8 +51,8 @@ __device__ __forceinline__ void coeff_grads(float lambda, float beta, bool euler
     }
 }
 
-struct BwdRed {  // the four warps' shares of one CTA-wide sum, double-buffered by token parity
-    float col[2][BW_THREADS / 32][BW_CB];
+struct BwdRed {  // the four warps' shares of one CTA-wide sum, double-buffered by parity
+    float col[2][BW_THREADS / 32][2 * BW_CB];
 };
 
 // Two fp32 lanes at once (packed f32x2 arithmetic of sm_100; each lane rounds as the scalar op).
@@ -78,59 +75,46 @@ __device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1) {
         : "f"(a0), "f"(a1));
 }
 
-// Sum over the warp of 16 values per lane, scattered: every lane returns the sum of value
-// (lane >> 1).  Each step halves the values a lane keeps and trades the other half with the
-// lane whose index differs in one bit: 8 + 4 + 2 + 1 + 1 shuffles in place of 16 x 5.
-__device__ __forceinline__ float warp_reduce_scatter16(float (&p)[BW_CB], int lane) {
+// Sum over the warp of 32 values per lane, scattered: lane l returns the sum of value l.  Each
+// step halves the values a lane keeps and trades the other half with the lane whose index
+// differs in one bit: 16 + 8 + 4 + 2 + 1 shuffles in place of 32 x 5.
+__device__ __forceinline__ float warp_reduce_scatter32(float (&p)[2 * BW_CB], int lane) {
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const bool up = lane & 16;
-        const float send = up ? p[m] : p[m + 8], keep = up ? p[m + 8] : p[m];
-        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
+    for (int h = 16; h >= 1; h >>= 1) {
+        const bool up = lane & h;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const bool up = lane & 8;
-        const float send = up ? p[m] : p[m + 4], keep = up ? p[m + 4] : p[m];
-        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        for (int m = 0; m < h; ++m) {
+            const float send = up ? p[m] : p[m + h], keep = up ? p[m + h] : p[m];
+            p[m] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+        }
     }
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        const bool up = lane & 4;
-        const float send = up ? p[m] : p[m + 2], keep = up ? p[m + 2] : p[m];
-        p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    {
-        const bool up = lane & 2;
-        const float send = up ? p[0] : p[1], keep = up ? p[1] : p[0];
-        p[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-    return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
+    return p[0];
 }
 
-// Column c of a CTA-wide sum: the four warps' shares added in the order 0, 1, 2, 3.
-__device__ __forceinline__ float col_sum(const BwdRed &red, int par, int c) {
-    float a = red.col[par][0][c];
-#pragma unroll
-    for (int ww = 1; ww < BW_THREADS / 32; ++ww) a += red.col[par][ww][c];
-    return a;
-}
-
-// CTA-wide sums of p[0..16) into out (every thread calls it; one barrier).  Each lane adds up
-// one column's four warp shares (lanes 2c and 2c + 1 take column c) and the totals reach every
-// lane by shuffles: shared memory sees one conflict-free load per warp share, not a broadcast
-// read of all 64 shares by every thread.
-__device__ __forceinline__ void cta_sum16(float (&p)[BW_CB], BwdRed &red, int par, float (&out)[BW_CB]) {
+// CTA-wide sums of p[0..32) into out (every thread calls it; one barrier).  Lane l adds up the
+// four warps' shares of value l and the totals reach every lane by shuffles: shared memory sees
+// one conflict-free load per warp share, not a broadcast read of all of them by every thread.
+__device__ __forceinline__ void cta_sum32(float (&p)[2 * BW_CB], BwdRed &red, int par,
+                                          float (&out)[2 * BW_CB]) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const float c = warp_reduce_scatter16(p, lane);
-    if ((lane & 1) == 0) red.col[par][w][lane >> 1] = c;
+    red.col[par][w][lane] = warp_reduce_scatter32(p, lane);
     __syncthreads();
-    const float t = col_sum(red, par, lane >> 1);
+    float t = red.col[par][0][lane];
 #pragma unroll
-    for (int j = 0; j < BW_CB; ++j) out[j] = __shfl_sync(0xffffffffu, t, 2 * j);
+    for (int ww = 1; ww < BW_THREADS / 32; ++ww) t += red.col[par][ww][lane];
+#pragma unroll
+    for (int j = 0; j < 2 * BW_CB; ++j) out[j] = __shfl_sync(0xffffffffu, t, j);
 }
 
-__device__ __forceinline__ void load_row16(const float *p, float (&x)[BW_CB]) {
+// Value i of a register array without dynamic indexing (which would go through local memory).
+__device__ __forceinline__ float pick(const float *x, int i) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < BW_CB; ++j) m = (i == j) ? x[j] : m;
+    return m;
+}
+
+__device__ __forceinline__ void load_row16(const float *p, float *x) {
 #pragma unroll
     for (int j4 = 0; j4 < BW_CB / 4; ++j4) {
         const float4 a = reinterpret_cast<const float4 *>(p)[j4];
@@ -138,42 +122,62 @@ __device__ __forceinline__ void load_row16(const float *p, float (&x)[BW_CB]) {
     }
 }
 
-__device__ __forceinline__ void store_row16(float *p, const float (&x)[BW_CB]) {
+__device__ __forceinline__ void store_row16(float *p, const float *x) {
 #pragma unroll
     for (int j4 = 0; j4 < BW_CB / 4; ++j4)
         reinterpret_cast<float4 *>(p)[j4] = make_float4(x[4 * j4], x[4 * j4 + 1], x[4 * j4 + 2], x[4 * j4 + 3]);
 }
 
-// Per token: (lambda = |k|^2, a = f(lambda, beta), df/dbeta, df/dlambda), one warp per token.
-// Every column block of a head reads them, so they are computed once, ahead of the sweeps.
+// Per token t, two float4: (lambda = |k_t|^2, a_t, df/dbeta, df/dlambda) and
+// (q_t . k_t, k_t . k_{t-1}, 0, 0) (k_{-1} = 0); one warp per token.  Every column block of a
+// head reads them, so they are computed once, ahead of the sweeps.
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ k, const T *__restrict__ beta,
-                                                       size_t ntok, int dk, bool euler,
-                                                       float4 *__restrict__ coef) {
+__global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                                                       const T *__restrict__ beta, size_t ntok, int L,
+                                                       int dk, bool euler, float4 *__restrict__ coef) {
     const int lane = threadIdx.x & 31;
     for (size_t tok = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); tok < ntok; tok += (size_t)gridDim.x * 8) {
-        float s = 0.f;
+        const bool first = tok % (size_t)L == 0;
+        float lam = 0.f, qk = 0.f, kk = 0.f;
         for (int i = lane; i < dk; i += 32) {
             const float x = to_f32(k[tok * dk + i]);
-            s = fmaf(x, x, s);
+            lam = fmaf(x, x, lam);
+            qk = fmaf(to_f32(q[tok * dk + i]), x, qk);
+            if (!first) kk = fmaf(to_f32(k[(tok - 1) * dk + i]), x, kk);
         }
-        s = warp_sum(s);
+        lam = warp_sum(lam);
+        qk = warp_sum(qk);
+        kk = warp_sum(kk);
         if (lane == 0) {
             const float bt = to_f32(beta[tok]);
-            const float a = alpha_rule(s, bt, euler);
+            const float a = alpha_rule(lam, bt, euler);
             float dfdb, dfdl;
-            coeff_grads(s, bt, euler, a, dfdb, dfdl);
-            coef[tok] = make_float4(s, a, dfdb, dfdl);
+            coeff_grads(lam, bt, euler, a, dfdb, dfdl);
+            coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
+            coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
         }
     }
 }
 
-// Workspace: the per-token coefficients [B*H][L] (float4); per (head, column block) r of every
-// token [L][16], then the block's state at every 64-token boundary and at the end
-// [NB + 1][dk][16]; after all of those the column blocks' shares of dq and dk
-// ([NS][B*H][L][dk] each) and of dbeta ([NS][B*H][L]).
+// Tokens go through both sweeps in pairs, with one CTA-wide sum per pair.  Forward, for the
+// pair (t, t+1) from S = S_{t-1}: the sum gives y0 = S^T k_t and y1 = S^T k_{t+1}; then
+//   r_t = v_t - y0,  r_{t+1} = v_{t+1} - (y1 + a_t (k_t . k_{t+1}) r_t),
+//   S += a_t k_t r_t^T + a_{t+1} k_{t+1} r_{t+1}^T.
+// Reverse, for the pair (t, t-1) from S = S_t and G = dL/dS_t without token t's own q do^T:
+// G1 = G + q_t do_t^T; the sum gives du_t = G1^T k_t and z = G1^T k_{t-1}; token t's step
+// (above) makes G2 = G1 - a_t k_t du_t^T, and then
+//   du_{t-1} = (G2 + q_{t-1} do_{t-1}^T)^T k_{t-1}
+//            = z - a_t (k_t . k_{t-1}) du_t + (q_{t-1} . k_{t-1}) do_{t-1}.
+// Pairs are aligned to even token offsets in each 64-token block; a block with an odd count
+// (the last one) pairs its last token with an absent one, whose k, q, v, dO, r and
+// coefficients are all zero, so that it changes nothing.
+//
+// Workspace: the coefficients [B*H][L][2] (float4); per (head, column block) r of every token
+// [L][16], then the block's state at every 64-token boundary and at the end [NB + 1][dk][16];
+// after all of those the column blocks' shares of dq and dk ([NS][B*H][L][dk] each) and of
+// dbeta ([NS][B*H][L]).
 template <typename T>
-__global__ void __launch_bounds__(BW_THREADS, BW_MINB)
+__global__ void __launch_bounds__(BW_THREADS, 4)
     bwd_cols_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float4 *__restrict__ coef, const float *__restrict__ S0,
                     const float *__restrict__ dO, const float *__restrict__ dSL,
@@ -182,18 +186,12 @@ __global__ void __launch_bounds__(BW_THREADS, BW_MINB)
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
-    __shared__ __align__(16) float4 cb[BWD_BLOCK];        // the block's token coefficients
-    const int tid = threadIdx.x;
+    __shared__ __align__(16) float4 cb[BWD_BLOCK][2];     // the block's token coefficients
+    const int tid = threadIdx.x, row = tid;
     const int bh = blockIdx.x / NS, s = blockIdx.x % NS, c0 = s * BW_CB;
     const int BH = gridDim.x / NS, nc = min(BW_CB, dv - c0);
     const int NB = (L + BWD_BLOCK - 1) / BWD_BLOCK;
-    int row[BW_RPT];  // this thread's state rows: tid, tid + BW_THREADS, ...
-    bool act[BW_RPT];
-#pragma unroll
-    for (int u = 0; u < BW_RPT; ++u) {
-        row[u] = tid + u * BW_THREADS;
-        act[u] = row[u] < dk;
-    }
+    const bool act = row < dk;
     const size_t tk = (size_t)bh * L * dk, tv = (size_t)bh * L * dv, tb = (size_t)bh * L;
     const size_t DD = (size_t)dk * dv;
     float *R = ws + ((size_t)bh * NS + s) * ((size_t)L * BW_CB + (size_t)(NB + 1) * dk * BW_CB);
@@ -202,165 +200,195 @@ __global__ void __launch_bounds__(BW_THREADS, BW_MINB)
     float *pdq = part + (size_t)s * nq + tk;
     float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
     float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
-    auto ld = [&](const T *x, int t, int u) {  // element row[u] of token t's q or k (0 off the edge)
-        return (act[u] && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row[u]]) : 0.f;
+    auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
+        return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
+    };
+    // the block's per-token rows and coefficients, zero at the absent partner of an odd count
+    auto stage = [&](int t0, int cnt, bool reverse) {
+        const int n = cnt + (cnt & 1);
+        for (int e = tid; e < n * BW_CB; e += BW_THREADS) {
+            const int tt = e / BW_CB, j = e % BW_CB;
+            const bool in = tt < cnt && j < nc;
+            const size_t g = tv + (size_t)(t0 + tt) * dv + c0 + j;
+            if (reverse) {
+                xb[tt][j] = in ? dO[g] : 0.f;
+                rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
+            } else {
+                xb[tt][j] = in ? to_f32(v[g]) : 0.f;
+            }
+        }
+        for (int e = tid; e < 2 * n; e += BW_THREADS)
+            cb[e >> 1][e & 1] = (e >> 1) < cnt ? coef[2 * (tb + t0) + e] : make_float4(0.f, 0.f, 0.f, 0.f);
     };
 
-    float S[BW_RPT][BW_CB], G[BW_RPT][BW_CB];
+    float S[BW_CB], G[BW_CB];
 #pragma unroll
-    for (int u = 0; u < BW_RPT; ++u)
-#pragma unroll
-        for (int j = 0; j < BW_CB; ++j)
-            S[u][j] = (S0 && act[u] && j < nc) ? S0[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] : 0.f;
+    for (int j = 0; j < BW_CB; ++j)
+        S[j] = (S0 && act && j < nc) ? S0[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
 
     // ---- forward sweep: r of every token and the block-boundary states
     int par = 0;
-    float kr1[BW_RPT], kr2[BW_RPT], qr1[BW_RPT], qr2[BW_RPT];
-#pragma unroll
-    for (int u = 0; u < BW_RPT; ++u) {
-        kr1[u] = ld(k, 0, u);
-        kr2[u] = ld(k, 1, u);
-    }
+    float kn0 = ld(k, 0), kn1 = ld(k, 1);  // k rows of the next pair
     for (int b = 0; b < NB; ++b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb and cb are done
-        for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
-            const int tt = e / BW_CB, j = e % BW_CB;
-            xb[tt][j] = j < nc ? to_f32(v[tv + (size_t)(t0 + tt) * dv + c0 + j]) : 0.f;
-        }
-        for (int e = tid; e < cnt; e += BW_THREADS) cb[e] = coef[tb + t0 + e];
-#pragma unroll
-        for (int u = 0; u < BW_RPT; ++u)
-            if (act[u]) store_row16(CK + ((size_t)b * dk + row[u]) * BW_CB, S[u]);
+        stage(t0, cnt, false);
+        if (act) store_row16(CK + ((size_t)b * dk + row) * BW_CB, S);
         __syncthreads();
-        for (int tt = 0; tt < cnt; ++tt) {
+        for (int tt = 0; tt < cnt; tt += 2) {
             const int t = t0 + tt;
-            float ki[BW_RPT];
-#pragma unroll
-            for (int u = 0; u < BW_RPT; ++u) {
-                ki[u] = kr1[u];
-                kr1[u] = kr2[u];
-                kr2[u] = ld(k, t + 2, u);
-            }
-            float p[BW_CB], x[BW_CB], r[BW_CB];
+            const float k0 = kn0, k1 = kn1;
+            kn0 = ld(k, t + 2);
+            kn1 = ld(k, t + 3);
+            float p[2 * BW_CB], y[2 * BW_CB];
 #pragma unroll
             for (int j = 0; j < BW_CB; j += 2) {
-                mul2(p[j], p[j + 1], S[0][j], S[0][j + 1], ki[0], ki[0]);
-#pragma unroll
-                for (int u = 1; u < BW_RPT; ++u) fma2(p[j], p[j + 1], S[u][j], S[u][j + 1], ki[u], ki[u]);
+                mul2(p[j], p[j + 1], S[j], S[j + 1], k0, k0);
+                mul2(p[BW_CB + j], p[BW_CB + j + 1], S[j], S[j + 1], k1, k1);
             }
-            cta_sum16(p, red, par, x);  // x = S^T k
-            const float a = cb[tt].y;
-            load_row16(xb[tt], r);
+            cta_sum32(p, red, par, y);  // y = [S^T k_t | S^T k_{t+1}]
+            const float a0 = cb[tt][0].y, a1 = cb[tt + 1][0].y, kap = cb[tt + 1][1].y;
+            float r0[BW_CB], r1[BW_CB];
+            load_row16(xb[tt], r0);
+            load_row16(xb[tt + 1], r1);
+            const float c = a0 * kap;
 #pragma unroll
-            for (int j = 0; j < BW_CB; j += 2) add2(r[j], r[j + 1], -x[j], -x[j + 1]);  // r = v - S^T k
-            if (tid < BW_CB) R[(size_t)t * BW_CB + tid] = xb[tt][tid] + -col_sum(red, par, tid);
+            for (int j = 0; j < BW_CB; j += 2) {
+                add2(r0[j], r0[j + 1], -y[j], -y[j + 1]);  // r_t = v_t - S^T k_t
+                float x0 = y[BW_CB + j], x1 = y[BW_CB + j + 1];
+                fma2(x0, x1, c, c, r0[j], r0[j + 1]);      // S_t^T k_{t+1}
+                add2(r1[j], r1[j + 1], -x0, -x1);
+            }
+            if (tid < BW_CB) {
+                R[(size_t)t * BW_CB + tid] = pick(r0, tid);
+                if (tt + 1 < cnt) R[(size_t)(t + 1) * BW_CB + tid] = pick(r1, tid);
+            }
+            const float ak0 = a0 * k0, ak1 = a1 * k1;
 #pragma unroll
-            for (int u = 0; u < BW_RPT; ++u) {
-                const float ak = a * ki[u];
-#pragma unroll
-                for (int j = 0; j < BW_CB; j += 2) fma2(S[u][j], S[u][j + 1], ak, ak, r[j], r[j + 1]);
+            for (int j = 0; j < BW_CB; j += 2) {
+                fma2(S[j], S[j + 1], ak0, ak0, r0[j], r0[j + 1]);
+                fma2(S[j], S[j + 1], ak1, ak1, r1[j], r1[j + 1]);
             }
             par ^= 1;
         }
     }
-#pragma unroll
-    for (int u = 0; u < BW_RPT; ++u)
-        if (act[u]) store_row16(CK + ((size_t)NB * dk + row[u]) * BW_CB, S[u]);
+    if (act) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
 
     // ---- reverse sweep
 #pragma unroll
-    for (int u = 0; u < BW_RPT; ++u) {
-#pragma unroll
-        for (int j = 0; j < BW_CB; ++j)
-            G[u][j] = (dSL && act[u] && j < nc) ? dSL[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] : 0.f;
-        kr1[u] = ld(k, L - 1, u);
-        kr2[u] = ld(k, L - 2, u);
-        qr1[u] = ld(q, L - 1, u);
-        qr2[u] = ld(q, L - 2, u);
-    }
+    for (int j = 0; j < BW_CB; ++j)
+        G[j] = (dSL && act && j < nc) ? dSL[(size_t)bh * DD + (size_t)row * dv + c0 + j] : 0.f;
+    // the top pair of the last block: (L, L-1) when L is odd (token L absent), else (L-1, L-2)
+    const int top = L - 1 + (L & 1);
+    kn0 = ld(k, top);
+    kn1 = ld(k, top - 1);
+    float qn0 = ld(q, top), qn1 = ld(q, top - 1);
     for (int b = NB - 1; b >= 0; --b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb, rb and cb are done
-        for (int e = tid; e < cnt * BW_CB; e += BW_THREADS) {
-            const int tt = e / BW_CB, j = e % BW_CB;
-            xb[tt][j] = j < nc ? dO[tv + (size_t)(t0 + tt) * dv + c0 + j] : 0.f;
-            rb[tt][j] = R[(size_t)(t0 + tt) * BW_CB + j];
-        }
-        for (int e = tid; e < cnt; e += BW_THREADS) cb[e] = coef[tb + t0 + e];
-#pragma unroll
-        for (int u = 0; u < BW_RPT; ++u)  // S' after the block
-            if (act[u]) load_row16(CK + ((size_t)(b + 1) * dk + row[u]) * BW_CB, S[u]);
+        stage(t0, cnt, true);
+        if (act) load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);  // S' after the block
         __syncthreads();
-        for (int tt = cnt - 1; tt >= 0; --tt) {
+        for (int tt = cnt - 1 + (cnt & 1); tt > 0; tt -= 2) {  // pair (t, t-1), t = t0 + tt
             const int t = t0 + tt;
-            float ki[BW_RPT], qi[BW_RPT];
-#pragma unroll
-            for (int u = 0; u < BW_RPT; ++u) {
-                ki[u] = kr1[u];
-                qi[u] = qr1[u];
-                kr1[u] = kr2[u];
-                qr1[u] = qr2[u];
-                kr2[u] = ld(k, t - 2, u);
-                qr2[u] = ld(q, t - 2, u);
-            }
-            float d[BW_CB], r[BW_CB], p[BW_CB], du[BW_CB];
-            load_row16(xb[tt], d);
-            load_row16(rb[tt], r);
-            // G += q do^T;  dq = S' do
-            float dq0[BW_RPT], dq1[BW_RPT];
-#pragma unroll
-            for (int u = 0; u < BW_RPT; ++u) {
-                dq0[u] = 0.f;
-                dq1[u] = 0.f;
-#pragma unroll
-                for (int j = 0; j < BW_CB; j += 2) {
-                    fma2(G[u][j], G[u][j + 1], qi[u], qi[u], d[j], d[j + 1]);
-                    fma2(dq0[u], dq1[u], S[u][j], S[u][j + 1], d[j], d[j + 1]);
-                }
-            }
-            // du = G^T k
+            const float k0 = kn0, k1 = kn1, q0 = qn0, q1 = qn1;
+            kn0 = ld(k, t - 2);
+            kn1 = ld(k, t - 3);
+            qn0 = ld(q, t - 2);
+            qn1 = ld(q, t - 3);
+            float d0[BW_CB], r0[BW_CB];
+            load_row16(xb[tt], d0);
+            load_row16(rb[tt], r0);
+            // token t: G1 = G + q_t do_t^T;  dq_t = S_t do_t
+            float dqa = 0.f, dqb = 0.f;
 #pragma unroll
             for (int j = 0; j < BW_CB; j += 2) {
-                mul2(p[j], p[j + 1], G[0][j], G[0][j + 1], ki[0], ki[0]);
-#pragma unroll
-                for (int u = 1; u < BW_RPT; ++u) fma2(p[j], p[j + 1], G[u][j], G[u][j + 1], ki[u], ki[u]);
+                fma2(G[j], G[j + 1], q0, q0, d0[j], d0[j + 1]);
+                fma2(dqa, dqb, S[j], S[j + 1], d0[j], d0[j + 1]);
             }
-            cta_sum16(p, red, par, du);
-            const float4 cf = cb[tt];  // (lambda, a, df/dbeta, df/dlambda)
-            const float a = cf.y;
-            float da0 = 0.f, da1 = 0.f;  // this column block's share of da = du . r
+            float p[2 * BW_CB], du[2 * BW_CB];  // du = [G1^T k_t | G1^T k_{t-1}]
 #pragma unroll
-            for (int j = 0; j < BW_CB; j += 2) fma2(da0, da1, du[j], du[j + 1], r[j], r[j + 1]);
-            const float da = da0 + da1;
-            // S = S' - a k r^T;  dk = a G r - a S du + 2 da df/dlambda k;  G -= a k du^T
+            for (int j = 0; j < BW_CB; j += 2) {
+                mul2(p[j], p[j + 1], G[j], G[j + 1], k0, k0);
+                mul2(p[BW_CB + j], p[BW_CB + j + 1], G[j], G[j + 1], k1, k1);
+            }
+            cta_sum32(p, red, par, du);
+            const float4 cA0 = cb[tt][0], cB0 = cb[tt][1], cA1 = cb[tt - 1][0], cB1 = cb[tt - 1][1];
+            const float a0 = cA0.y, a1 = cA1.y;
+            // token t: da, S_{t-1} = S_t - a k r^T, dk, G2 = G1 - a k du^T
+            float daa = 0.f, dab = 0.f;
 #pragma unroll
-            for (int u = 0; u < BW_RPT; ++u) {
-                const float nak = -a * ki[u];
+            for (int j = 0; j < BW_CB; j += 2) fma2(daa, dab, du[j], du[j + 1], r0[j], r0[j + 1]);
+            const float da0 = daa + dab;
+            {
+                const float nak = -a0 * k0;
                 float gr0 = 0.f, gr1 = 0.f, sd0 = 0.f, sd1 = 0.f;
 #pragma unroll
                 for (int j = 0; j < BW_CB; j += 2) {
-                    fma2(S[u][j], S[u][j + 1], nak, nak, r[j], r[j + 1]);
-                    fma2(gr0, gr1, G[u][j], G[u][j + 1], r[j], r[j + 1]);
-                    fma2(sd0, sd1, S[u][j], S[u][j + 1], du[j], du[j + 1]);
-                    fma2(G[u][j], G[u][j + 1], nak, nak, du[j], du[j + 1]);
+                    fma2(S[j], S[j + 1], nak, nak, r0[j], r0[j + 1]);
+                    fma2(gr0, gr1, G[j], G[j + 1], r0[j], r0[j + 1]);
+                    fma2(sd0, sd1, S[j], S[j + 1], du[j], du[j + 1]);
+                    fma2(G[j], G[j + 1], nak, nak, du[j], du[j + 1]);
                 }
-                if (act[u]) {
-                    pdq[(size_t)t * dk + row[u]] = dq0[u] + dq1[u];
-                    pdk[(size_t)t * dk + row[u]] = a * ((gr0 + gr1) - (sd0 + sd1)) + 2.f * da * cf.w * ki[u];
+                if (tt < cnt) {
+                    if (act) {
+                        pdq[(size_t)t * dk + row] = dqa + dqb;
+                        pdk[(size_t)t * dk + row] = a0 * ((gr0 + gr1) - (sd0 + sd1)) + 2.f * da0 * cA0.w * k0;
+                    }
+                    if (tid < nc) dval[tv + (size_t)t * dv + c0 + tid] = a0 * pick(du, tid);
+                    if (tid == 0) pdb[t] = da0 * cA0.z;
                 }
             }
-            if (tid < nc) dval[tv + (size_t)t * dv + c0 + tid] = a * col_sum(red, par, tid);
-            if (tid == 0) pdb[t] = da * cf.z;
+            // token t-1: du_{t-1} = z - a_t (k_t . k_{t-1}) du_t + (q_{t-1} . k_{t-1}) do_{t-1}
+            float d1[BW_CB], r1[BW_CB];
+            load_row16(xb[tt - 1], d1);
+            load_row16(rb[tt - 1], r1);
+            {
+                const float c = -a0 * cB0.y, e = cB1.x;
+#pragma unroll
+                for (int j = 0; j < BW_CB; j += 2) {
+                    fma2(du[BW_CB + j], du[BW_CB + j + 1], c, c, du[j], du[j + 1]);
+                    fma2(du[BW_CB + j], du[BW_CB + j + 1], e, e, d1[j], d1[j + 1]);
+                }
+            }
+            float *du1 = du + BW_CB;
+            // G3 = G2 + q_{t-1} do_{t-1}^T;  dq_{t-1} = S_{t-1} do_{t-1}
+            dqa = 0.f;
+            dqb = 0.f;
+#pragma unroll
+            for (int j = 0; j < BW_CB; j += 2) {
+                fma2(G[j], G[j + 1], q1, q1, d1[j], d1[j + 1]);
+                fma2(dqa, dqb, S[j], S[j + 1], d1[j], d1[j + 1]);
+            }
+            daa = 0.f;
+            dab = 0.f;
+#pragma unroll
+            for (int j = 0; j < BW_CB; j += 2) fma2(daa, dab, du1[j], du1[j + 1], r1[j], r1[j + 1]);
+            const float da1 = daa + dab;
+            {
+                const float nak = -a1 * k1;
+                float gr0 = 0.f, gr1 = 0.f, sd0 = 0.f, sd1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < BW_CB; j += 2) {
+                    fma2(S[j], S[j + 1], nak, nak, r1[j], r1[j + 1]);
+                    fma2(gr0, gr1, G[j], G[j + 1], r1[j], r1[j + 1]);
+                    fma2(sd0, sd1, S[j], S[j + 1], du1[j], du1[j + 1]);
+                    fma2(G[j], G[j + 1], nak, nak, du1[j], du1[j + 1]);
+                }
+                if (act) {
+                    pdq[(size_t)(t - 1) * dk + row] = dqa + dqb;
+                    pdk[(size_t)(t - 1) * dk + row] = a1 * ((gr0 + gr1) - (sd0 + sd1)) + 2.f * da1 * cA1.w * k1;
+                }
+                if (tid < nc) dval[tv + (size_t)(t - 1) * dv + c0 + tid] = a1 * pick(du1, tid);
+                if (tid == 0) pdb[t - 1] = da1 * cA1.z;
+            }
             par ^= 1;
         }
     }
-    if (dS0) {
+    if (dS0 && act) {
 #pragma unroll
-        for (int u = 0; u < BW_RPT; ++u)
-#pragma unroll
-            for (int j = 0; j < BW_CB; ++j)
-                if (act[u] && j < nc) dS0[(size_t)bh * DD + (size_t)row[u] * dv + c0 + j] = G[u][j];
+        for (int j = 0; j < BW_CB; ++j)
+            if (j < nc) dS0[(size_t)bh * DD + (size_t)row * dv + c0 + j] = G[j];
     }
 }
 
@@ -408,7 +436,7 @@ static size_t bwd_state_floats(size_t BH, int L, int dk, int dv) {
 
 size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv) {
     const size_t BH = (size_t)B * H, NS = (size_t)(dv + BW_CB - 1) / BW_CB;
-    const size_t coef = 4 * BH * (size_t)L;
+    const size_t coef = 8 * BH * (size_t)L;
     const size_t shares = NS * BH * (size_t)L * (2 * (size_t)dk + 1);
     return (coef + bwd_state_floats(BH, L, dk, dv) + shares) * sizeof(float);
 }
@@ -425,17 +453,17 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const size_t ntok = (size_t)BH * L;
     float4 *coef = (float4 *)ws;
-    float *state = (float *)ws + 4 * ntok;
+    float *state = (float *)ws + 8 * ntok;
     float *part = state + bwd_state_floats((size_t)BH, L, dk, dv);
     if (ntok > 0) {
         const int gc = (int)std::min<size_t>((ntok + 7) / 8, (size_t)nsm * 64);
         if (is_bf16)
-            bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)k,
-                                                               (const __nv_bfloat16 *)beta, ntok, dk,
-                                                               euler, coef);
+            bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>(
+                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, ntok, L,
+                dk, euler, coef);
         else
-            bwd_coeff_kernel<float><<<gc, 256, 0, s>>>((const float *)k, (const float *)beta, ntok, dk,
-                                                       euler, coef);
+            bwd_coeff_kernel<float><<<gc, 256, 0, s>>>((const float *)q, (const float *)k,
+                                                       (const float *)beta, ntok, L, dk, euler, coef);
         count_launches(1);
     }
     const int grid = (int)(BH * NS);

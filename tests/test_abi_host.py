@@ -145,19 +145,19 @@ def test_selftest_budget_is_checked_on_the_host(lib):
 
 
 def test_bwd_workspace_size_and_alignment(lib):
-    """The backward's workspace: four fp32 coefficients per token; per (head, 16-column block)
+    """The backward's workspace: eight fp32 coefficients per token; per (head, 16-column block)
     r of every token and the block's state every 64 tokens and at the end; then the column
     blocks' shares of dq, dk and dbeta.  A workspace that is not 16-byte aligned is refused
     before any CUDA call."""
     B, H, L, dk, dv = 4, 16, 4096, 128, 128
     NS, NB = 8, 64
-    coef = 4 * B * H * L
+    coef = 8 * B * H * L
     state = B * H * NS * (L * 16 + (NB + 1) * dk * 16)
     shares = NS * B * H * L * (2 * dk + 1)
     assert lib.efla_bwd_workspace_size(B, H, L, dk, dv) == 4 * (coef + state + shares)
     # ragged: dv = 20 takes two column blocks, L = 65 two token blocks
     assert lib.efla_bwd_workspace_size(1, 1, 65, 8, 20) == \
-        4 * (4 * 65 + 2 * (65 * 16 + 3 * 8 * 16) + 2 * 65 * 17)
+        4 * (8 * 65 + 2 * (65 * 16 + 3 * 8 * 16) + 2 * 65 * 17)
     assert lib.efla_bwd_workspace_size(1, 1, 16, 129, 16) == 0
     P = ctypes.c_void_p(64)
     EFLA_ERR_ALIGN, EFLA_ERR_WORKSPACE = 8, 7

@@ -36,7 +36,10 @@ def _case(wid, rule, seed=5, **kw):
                                     (4, dict(B=1, H=2, L=200)), (3, dict(B=1, H=1, L=77, dk=128, dv=64)),
                                     (2, dict(B=2, H=1, L=65, dk=40, dv=20)),
                                     (3, dict(B=1, H=1, L=64, dk=7, dv=5)),
-                                    (4, dict(B=1, H=1, L=129, dk=128, dv=100))])
+                                    (4, dict(B=1, H=1, L=129, dk=128, dv=100)),
+                                    (2, dict(B=1, H=2, L=1, dk=16, dv=16)),
+                                    (2, dict(B=1, H=1, L=2, dk=16, dv=32)),
+                                    (2, dict(B=1, H=1, L=63, dk=64, dv=16))])
 def test_backward_matches_oracle(oracle_mod, rule, wid, kw):
     x = _case(wid, rule, **kw)
     d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
