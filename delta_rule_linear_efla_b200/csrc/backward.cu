@@ -130,11 +130,13 @@ __device__ __forceinline__ void store_row16(float *p, const float *x) {
 
 // Per token t, two float4: (lambda = |k_t|^2, a_t, df/dbeta, df/dlambda) and
 // (q_t . k_t, k_t . k_{t-1}, 0, 0) (k_{-1} = 0); one warp per token.  Every column block of a
-// head reads them, so they are computed once, ahead of the sweeps.
+// head reads them, so they are computed once, ahead of the sweeps.  zero_alpha[head] is set when a
+// token of the head has a = 0 (zero beta).
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                        const T *__restrict__ beta, size_t ntok, int L,
-                                                       int dk, bool euler, float4 *__restrict__ coef) {
+                                                       int dk, bool euler, float4 *__restrict__ coef,
+                                                       int *__restrict__ zero_alpha) {
     const int lane = threadIdx.x & 31;
     for (size_t tok = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); tok < ntok; tok += (size_t)gridDim.x * 8) {
         const bool first = tok % (size_t)L == 0;
@@ -155,6 +157,7 @@ __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q,
             coeff_grads(lam, bt, euler, a, dfdb, dfdl);
             coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
             coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
+            if (a == 0.f) atomicOr(zero_alpha + tok / (size_t)L, 1);  // u / a cannot give this head's r
         }
     }
 }
@@ -182,7 +185,8 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
                     const float4 *__restrict__ coef, const float *__restrict__ S0,
                     const float *__restrict__ dO, const float *__restrict__ dSL,
                     float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
-                    float *__restrict__ ws, float *__restrict__ part) {
+                    float *__restrict__ ws, float *__restrict__ part, const float *__restrict__ u_saved,
+                    const float *__restrict__ ck_saved, const int *__restrict__ zero_alpha) {
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
@@ -200,6 +204,10 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     float *pdq = part + (size_t)s * nq + tk;
     float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
     float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
+    // The tensor-core forward may have saved every token's u = a r and the state after every
+    // 64-token block: then this sweep's forward half is not needed (unless a token of the head
+    // has a = 0, where r cannot be had from u).
+    const bool saved = u_saved != nullptr && zero_alpha[bh] == 0;
     auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
         return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
     };
@@ -212,7 +220,10 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             const size_t g = tv + (size_t)(t0 + tt) * dv + c0 + j;
             if (reverse) {
                 xb[tt][j] = in ? dO[g] : 0.f;
-                rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
+                if (saved)
+                    rb[tt][j] = in ? u_saved[g] / coef[2 * (tb + t0 + tt)].y : 0.f;
+                else
+                    rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
             } else {
                 xb[tt][j] = in ? to_f32(v[g]) : 0.f;
             }
@@ -229,7 +240,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // ---- forward sweep: r of every token and the block-boundary states
     int par = 0;
     float kn0 = ld(k, 0), kn1 = ld(k, 1);  // k rows of the next pair
-    for (int b = 0; b < NB; ++b) {
+    for (int b = 0; b < (saved ? 0 : NB); ++b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb and cb are done
         stage(t0, cnt, false);
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             par ^= 1;
         }
     }
-    if (act) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
+    if (act && !saved) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
 
     // ---- reverse sweep
 #pragma unroll
@@ -287,7 +298,12 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb, rb and cb are done
         stage(t0, cnt, true);
-        if (act) load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);  // S' after the block
+        if (act) {  // S' after the block
+            if (saved)
+                load_row16(ck_saved + (((size_t)bh * NB + b) * dk + row) * dv + c0, S);
+            else
+                load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);
+        }
         __syncthreads();
         for (int tt = cnt - 1 + (cnt & 1); tt > 0; tt -= 2) {  // pair (t, t-1), t = t0 + tt
             const int t = t0 + tt;
@@ -434,11 +450,38 @@ static size_t bwd_state_floats(size_t BH, int L, int dk, int dv) {
     return BH * NS * ((size_t)L * BW_CB + (NB + 1) * (size_t)dk * BW_CB);
 }
 
+// Sizes for which the tensor-core forward (bf16 inputs) saves u and the block states for the
+// reverse sweep.  The workspace is sized for it whenever the sizes allow it (the input dtype is
+// not an argument of the size query).
+static bool bwd_tc_saves(int B, int H, int L, int dk, int dv) {
+    return L > 0 && tc_supported(B, H, L, dk, dv, BWD_BLOCK, true);
+}
+
+struct BwdLayout {  // float offsets into the workspace
+    size_t coef, zero, state, part, tc, u, ck, total;
+};
+
+static BwdLayout bwd_layout(int B, int H, int L, int dk, int dv) {
+    const size_t BH = (size_t)B * H, NS = (size_t)(dv + BW_CB - 1) / BW_CB, ntok = BH * (size_t)L;
+    const size_t NB = (size_t)(L + BWD_BLOCK - 1) / BWD_BLOCK;
+    auto up = [](size_t f) { return (f + 63) / 64 * 64; };  // every region 256-byte aligned
+    BwdLayout a;
+    a.coef = 0;
+    a.zero = up(8 * ntok);
+    a.state = a.zero + up(BH);
+    a.part = a.state + up(bwd_state_floats(BH, L, dk, dv));
+    a.tc = a.part + up(NS * ntok * (2 * (size_t)dk + 1));
+    a.u = a.ck = a.total = a.tc;
+    if (bwd_tc_saves(B, H, L, dk, dv)) {
+        a.u = a.tc + up((tc_workspace_bytes(B, H, L, dk, dv, BWD_BLOCK) + 3) / 4);
+        a.ck = a.u + up(ntok * (size_t)dv);
+        a.total = a.ck + BH * NB * (size_t)dk * dv;
+    }
+    return a;
+}
+
 size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv) {
-    const size_t BH = (size_t)B * H, NS = (size_t)(dv + BW_CB - 1) / BW_CB;
-    const size_t coef = 8 * BH * (size_t)L;
-    const size_t shares = NS * BH * (size_t)L * (2 * (size_t)dk + 1);
-    return (coef + bwd_state_floats(BH, L, dk, dv) + shares) * sizeof(float);
+    return bwd_layout(B, H, L, dk, dv).total * sizeof(float);
 }
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
@@ -452,31 +495,47 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const size_t ntok = (size_t)BH * L;
-    float4 *coef = (float4 *)ws;
-    float *state = (float *)ws + 8 * ntok;
-    float *part = state + bwd_state_floats((size_t)BH, L, dk, dv);
+    const BwdLayout lay = bwd_layout(B, H, L, dk, dv);
+    float *wsf = (float *)ws;
+    float4 *coef = (float4 *)(wsf + lay.coef);
+    int *zero_alpha = (int *)(wsf + lay.zero);
+    float *state = wsf + lay.state;
+    float *part = wsf + lay.part;
+    float *u_saved = nullptr, *ck_saved = nullptr;
+    cudaError_t e;
+    if (is_bf16 && bwd_tc_saves(B, H, L, dk, dv)) {
+        // the tensor-core forward, saving u and the block states instead of writing outputs
+        u_saved = wsf + lay.u;
+        ck_saved = wsf + lay.ck;
+        e = launch_chunk_tc_save(q, k, v, beta, S0, B, H, L, dk, dv, euler, wsf + lay.tc, u_saved, ck_saved, s);
+        if (e != cudaSuccess) return e;
+    }
     if (ntok > 0) {
+        e = cudaMemsetAsync(zero_alpha, 0, (size_t)BH * sizeof(int), s);
+        if (e != cudaSuccess) return e;
         const int gc = (int)std::min<size_t>((ntok + 7) / 8, (size_t)nsm * 64);
         if (is_bf16)
             bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>(
                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, ntok, L,
-                dk, euler, coef);
+                dk, euler, coef, zero_alpha);
         else
             bwd_coeff_kernel<float><<<gc, 256, 0, s>>>((const float *)q, (const float *)k,
-                                                       (const float *)beta, ntok, L, dk, euler, coef);
+                                                       (const float *)beta, ntok, L, dk, euler, coef,
+                                                       zero_alpha);
         count_launches(1);
     }
     const int grid = (int)(BH * NS);
     if (is_bf16)
         bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, dO,
-            dSL, dval, dS0, L, dk, dv, NS, state, part);
+            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, zero_alpha);
     else
         bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
                                                           (const float *)v, coef, S0, dO, dSL, dval,
-                                                          dS0, L, dk, dv, NS, state, part);
+                                                          dS0, L, dk, dv, NS, state, part, nullptr,
+                                                          nullptr, zero_alpha);
     count_launches(1);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess || L == 0) return e;
     // add the column blocks' shares of dq, dk and dbeta
     const size_t nq = (size_t)BH * L * dk, nb = (size_t)BH * L;

@@ -33,6 +33,8 @@
 #include <atomic>
 #include <mutex>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "launchers.h"
 #include "tc_ptx.cuh"
@@ -434,14 +436,15 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
 }
 
 // SEG = false compiles the one-pass form only (pass 0); SEG = true also takes the segment runs.
-template <int DK, int DV, typename TO, bool SEG>
+template <int DK, int DV, typename TO, bool SEG, bool SAVE = false>
 __global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
-                    float *__restrict__ segbuf, int G, int seg_chunks, int pass) {
+                    float *__restrict__ segbuf, int G, int seg_chunks, int pass,
+                    float *__restrict__ u_out, float *__restrict__ ck_out) {
     using Lay = StateLayout<DK, DV>;
     constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
     extern __shared__ uint8_t smem_raw[];
@@ -779,6 +782,13 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
                 tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, w);  // over fp32 columns already read
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
+                if (SAVE && u_out && mode == 0 && vrow >= 0) {  // u_t = a_t r_t of every token, for the backward
+                    const int t0 = (n0 + n) * C + h * 32;
+                    float *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (t0 + j < L) dst[(size_t)j * DV] = u[j];
+                }
             }
 
             if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) { done_all = false; break; }
@@ -796,6 +806,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (cb == 0) warp_arrive(&bars.s_ready_a, lane);
             }
             warp_arrive(&bars.s_ready, lane);
+            if (SAVE && ck_out && mode == 0) {
+                // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
+                // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
+                // warp-collective: every lane takes it, the lanes that hold a state column store.
+                float *dst = ck_out + ((size_t)bh * NC + n0 + n) * DD + (vrow >= 0 ? vrow : 0);
+#pragma unroll 1
+                for (int cb = 0; cb < DK / 16; ++cb) {
+                    float v[16];
+                    tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
+                    if (vrow >= 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) dst[(size_t)(cb * 16 + j) * DV] = v[j];
+                    }
+                }
+            }
         }
         if (done_all && sfp) {
 #pragma unroll
@@ -824,7 +849,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
             warp_arrive(&bars.o_free, lane);  // TMEM O is zero again: D1(n+1) may run
-            if (mode == 0 && vrow >= 0) {
+            if (mode == 0 && vrow >= 0 && o) {
                 TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
@@ -1012,6 +1037,14 @@ TcDevInfo tc_dev_info() {
     if (d.err == cudaSuccess && DK == DV)
         d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+    if constexpr (std::is_same<TO, float>::value) {  // the saving forward of the backward
+        if (d.err == cudaSuccess)
+            d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+        if (d.err == cudaSuccess && DK == DV)
+            d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+    }
     if (d.err != cudaSuccess) return d;
     d.nsm = nsm;
     int per_sm = smem_sm / (psm + 1024);  // 1 KiB per CTA is reserved by the system
@@ -1022,10 +1055,10 @@ TcDevInfo tc_dev_info() {
     return d;
 }
 
-template <int DK, int DV, typename TO>
+template <int DK, int DV, typename TO, bool SAVE = false>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void *beta,
                         const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
-                        void *ws, cudaStream_t s) {
+                        void *ws, cudaStream_t s, float *u_out = nullptr, float *ck_out = nullptr) {
     const int BH = B * H, NC = (L + C - 1) / C, total = BH * NC;
     const TcDevInfo di = tc_dev_info<DK, DV, TO>();
     if (di.err != cudaSuccess) return di.err;
@@ -1045,19 +1078,19 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
-        tc_state_kernel<DK, DV, TO, false><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final,
-                                                                      L, NC, nullptr, 1, NC, 0);
+        tc_state_kernel<DK, DV, TO, false, SAVE><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final,
+                                                                      L, NC, nullptr, 1, NC, 0, u_out, ck_out);
         count_launches(2);
         return cudaGetLastError();
     }
     if constexpr (DK == DV) {
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
-        tc_state_kernel<DK, DV, TO, true><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1);
+        tc_state_kernel<DK, DV, TO, true, SAVE><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out);
         seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
-        tc_state_kernel<DK, DV, TO, true><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2);
+        tc_state_kernel<DK, DV, TO, true, SAVE><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out);
         count_launches(4);
     }
     return cudaGetLastError();
@@ -1113,6 +1146,22 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
     if (dk == 64 && dv == 128)
         return launch_tc_o<64, 128>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
     return launch_tc_o<64, 64>(q, k, v, beta, S0, o, S_final, B, H, L, o_bf16, euler, ws, s);
+}
+
+cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
+                                 const float *S0, int B, int H, int L, int dk, int dv, bool euler,
+                                 void *ws, float *u_out, float *ck_out, cudaStream_t s) {
+    if (dk == 128 && dv == 128)
+        return launch_tc_t<128, 128, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
+                                                  u_out, ck_out);
+    if (dk == 128 && dv == 64)
+        return launch_tc_t<128, 64, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
+                                                 u_out, ck_out);
+    if (dk == 64 && dv == 128)
+        return launch_tc_t<64, 128, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
+                                                 u_out, ck_out);
+    return launch_tc_t<64, 64, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s, u_out,
+                                            ck_out);
 }
 
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s) {

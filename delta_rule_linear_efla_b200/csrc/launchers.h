@@ -49,6 +49,13 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
                             const float *S0, void *o, float *S_final, int B, int H, int L,
                             int dk, int dv, int chunk, bool o_bf16, bool euler, void *ws,
                             cudaStream_t s);
+// The tensor-core forward without outputs, saving what the backward needs instead: every
+// token's u_t = a_t (v_t - S_{t-1}^T k_t) into u_out [B*H][L][dv] and the state after every
+// 64-token chunk into ck_out [B*H][ceil(L/64)][dk][dv] (fp32).  Same sizes as launch_chunk_tc,
+// chunk 64, and the same workspace.
+cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
+                                 const float *S0, int B, int H, int L, int dk, int dv, bool euler,
+                                 void *ws, float *u_out, float *ck_out, cudaStream_t s);
 // A kernel whose one bounded wait runs out (nothing arrives): records a timeout, then returns.
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits): read and clear.

@@ -102,3 +102,22 @@ def test_backward_full_size_sampled_heads(oracle_mod):
         for name, g, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
             e = rel_err(sl(g).numpy(), r)
             assert e <= TOL["bf16"], (b, h, name, e)
+
+
+@pytest.mark.parametrize("rule", ["exact", "euler"])
+def test_backward_with_a_zero_beta_token(oracle_mod, rule):
+    """bf16 heads of 128 take the reverse sweep from the tensor-core forward's saved u = a r and
+    block states; a head with a zero beta (a = 0, where u / a cannot give r) walks the forward
+    itself.  Head 0 has one, head 1 none: both must match the oracle."""
+    x = _case(4, rule, B=1, H=2, L=200)
+    beta = x["beta"].clone()
+    beta[0, 0, 17] = 0
+    x["beta"] = beta
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    got = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"], rule=rule)
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], x["dO"], x["S0"], x["dS"], rule=rule)
+    for name, g, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+        e = rel_err(g.cpu().numpy(), r)
+        assert e <= TOL["bf16"], (name, e)
