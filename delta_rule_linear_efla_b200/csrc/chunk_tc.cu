@@ -849,7 +849,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
             warp_arrive(&bars.o_free, lane);  // TMEM O is zero again: D1(n+1) may run
-            if (mode == 0 && vrow >= 0 && o) {
+            if (mode == 0 && vrow >= 0 && (!SAVE || o)) {  // the saving forward writes no o
                 TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
