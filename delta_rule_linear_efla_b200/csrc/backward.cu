@@ -130,13 +130,16 @@ __device__ __forceinline__ void store_row16(float *p, const float *x) {
 
 // Per token t, two float4: (lambda = |k_t|^2, a_t, df/dbeta, df/dlambda) and
 // (q_t . k_t, k_t . k_{t-1}, 0, 0) (k_{-1} = 0); one warp per token.  Every column block of a
-// head reads them, so they are computed once, ahead of the sweeps.  zero_alpha[head] is set when a
-// token of the head has a = 0 (zero beta).
+// head reads them, so they are computed once, ahead of the sweeps.  It also gathers, per head,
+// what decides whether the reverse sweep may take r = u / a from the tensor-core forward's u (see
+// saved_ok below): hs[head] = {a token has a = 0; max lambda (float bits); INT_MAX - min a
+// (float bits); max a (float bits)}, every field zero-initialised (a >= 0, lambda >= 0, so the
+// bit patterns order as the values do).
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                        const T *__restrict__ beta, size_t ntok, int L,
                                                        int dk, bool euler, float4 *__restrict__ coef,
-                                                       int *__restrict__ zero_alpha) {
+                                                       int *__restrict__ hs) {
     const int lane = threadIdx.x & 31;
     for (size_t tok = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); tok < ntok; tok += (size_t)gridDim.x * 8) {
         const bool first = tok % (size_t)L == 0;
@@ -157,7 +160,11 @@ __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q,
             coeff_grads(lam, bt, euler, a, dfdb, dfdl);
             coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
             coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
-            if (a == 0.f) atomicOr(zero_alpha + tok / (size_t)L, 1);  // u / a cannot give this head's r
+            int *h = hs + 4 * (tok / (size_t)L);
+            if (a == 0.f) atomicOr(h, 1);  // u / a cannot give this head's r
+            atomicMax(h + 1, __float_as_int(lam));
+            atomicMax(h + 2, 0x7fffffff - __float_as_int(a));
+            atomicMax(h + 3, __float_as_int(a));
         }
     }
 }
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
                     const float *__restrict__ dO, const float *__restrict__ dSL,
                     float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
                     float *__restrict__ ws, float *__restrict__ part, const float *__restrict__ u_saved,
-                    const float *__restrict__ ck_saved, const int *__restrict__ zero_alpha) {
+                    const float *__restrict__ ck_saved, const int *__restrict__ hs) {
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
@@ -205,9 +212,22 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
     float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
     // The tensor-core forward may have saved every token's u = a r and the state after every
-    // 64-token block: then this sweep's forward half is not needed (unless a token of the head
-    // has a = 0, where r cannot be had from u).
-    const bool saved = u_saved != nullptr && zero_alpha[bh] == 0;
+    // 64-token block: then this sweep's forward half is not needed.  u carries the fp16 operand
+    // rounding of the chunk products, an absolute error at the scale of the chunk's largest u;
+    // r = u / a divides it by a, so a token whose a is small next to its neighbours' gets a
+    // large relative error in r (and in dbeta).  Emulating those roundings, the error grows with
+    // the keys' squared norm (dbeta's max error over its RMS: 0.007 with ||k||^2 up to 16,
+    // 0.013 up to 32, 0.032 for the stiff inputs with ||k||^2 up to 100) far more than with the
+    // spread of a from small betas (0.006 at a max/min ratio of 800).  So the saved values are
+    // used only for heads whose largest ||k||^2 is at most 16, whose a spans at most a factor of
+    // 1024, and that have no a = 0; other heads walk the forward in fp32 themselves.
+    bool saved = false;
+    if (u_saved != nullptr) {
+        const int *h = hs + 4 * bh;
+        const float lam_max = __int_as_float(h[1]), a_min = __int_as_float(0x7fffffff - h[2]);
+        const float a_max = __int_as_float(h[3]);
+        saved = h[0] == 0 && lam_max <= 16.f && a_max <= 1024.f * a_min;
+    }
     auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
         return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
     };
@@ -468,7 +488,7 @@ static BwdLayout bwd_layout(int B, int H, int L, int dk, int dv) {
     BwdLayout a;
     a.coef = 0;
     a.zero = up(8 * ntok);
-    a.state = a.zero + up(BH);
+    a.state = a.zero + up(4 * BH);
     a.part = a.state + up(bwd_state_floats(BH, L, dk, dv));
     a.tc = a.part + up(NS * ntok * (2 * (size_t)dk + 1));
     a.u = a.ck = a.total = a.tc;
@@ -498,7 +518,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     const BwdLayout lay = bwd_layout(B, H, L, dk, dv);
     float *wsf = (float *)ws;
     float4 *coef = (float4 *)(wsf + lay.coef);
-    int *zero_alpha = (int *)(wsf + lay.zero);
+    int *hs = (int *)(wsf + lay.zero);  // per-head statistics for the saved-forward gate
     float *state = wsf + lay.state;
     float *part = wsf + lay.part;
     float *u_saved = nullptr, *ck_saved = nullptr;
@@ -511,29 +531,29 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
         if (e != cudaSuccess) return e;
     }
     if (ntok > 0) {
-        e = cudaMemsetAsync(zero_alpha, 0, (size_t)BH * sizeof(int), s);
+        e = cudaMemsetAsync(hs, 0, 4 * (size_t)BH * sizeof(int), s);
         if (e != cudaSuccess) return e;
         const int gc = (int)std::min<size_t>((ntok + 7) / 8, (size_t)nsm * 64);
         if (is_bf16)
             bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>(
                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, ntok, L,
-                dk, euler, coef, zero_alpha);
+                dk, euler, coef, hs);
         else
             bwd_coeff_kernel<float><<<gc, 256, 0, s>>>((const float *)q, (const float *)k,
                                                        (const float *)beta, ntok, L, dk, euler, coef,
-                                                       zero_alpha);
+                                                       hs);
         count_launches(1);
     }
     const int grid = (int)(BH * NS);
     if (is_bf16)
         bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, dO,
-            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, zero_alpha);
+            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, hs);
     else
         bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
                                                           (const float *)v, coef, S0, dO, dSL, dval,
                                                           dS0, L, dk, dv, NS, state, part, nullptr,
-                                                          nullptr, zero_alpha);
+                                                          nullptr, hs);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess || L == 0) return e;

@@ -146,7 +146,7 @@ def test_selftest_budget_is_checked_on_the_host(lib):
 
 def test_bwd_workspace_size_and_alignment(lib):
     """The backward's workspace, every region rounded up to 256 bytes: eight fp32 coefficients per
-    token; a zero-alpha flag per head; per (head, 16-column block) r of every token and the
+    token; four ints of statistics per head; per (head, 16-column block) r of every token and the
     block's state every 64 tokens and at the end; the column blocks' shares of dq, dk and dbeta;
     and, where the tensor-core forward can run (bf16 inputs), its workspace, every token's u and
     the state after every 64-token block.  A workspace that is not 16-byte aligned is refused
@@ -154,14 +154,14 @@ def test_bwd_workspace_size_and_alignment(lib):
     up = lambda f: (f + 63) // 64 * 64
     B, H, L, dk, dv = 4, 16, 4096, 128, 128
     NS, NB, BH = 8, 64, B * H
-    base = up(8 * BH * L) + up(BH) + up(BH * NS * (L * 16 + (NB + 1) * dk * 16)) + \
+    base = up(8 * BH * L) + up(4 * BH) + up(BH * NS * (L * 16 + (NB + 1) * dk * 16)) + \
         up(NS * BH * L * (2 * dk + 1))
     tc = lib.efla_chunk_fwd_workspace_size(B, H, L, dk, dv, 64, BF16, F32)
     saved = up(tc // 4) + up(BH * L * dv) + BH * NB * dk * dv
     assert lib.efla_bwd_workspace_size(B, H, L, dk, dv) == 4 * (base + saved)
     # ragged, no tensor-core forward (d_k = 8): dv = 20 takes two column blocks, L = 65 two blocks
     assert lib.efla_bwd_workspace_size(1, 1, 65, 8, 20) == \
-        4 * (up(8 * 65) + up(1) + up(2 * (65 * 16 + 3 * 8 * 16)) + up(2 * 65 * 17))
+        4 * (up(8 * 65) + up(4) + up(2 * (65 * 16 + 3 * 8 * 16)) + up(2 * 65 * 17))
     assert lib.efla_bwd_workspace_size(1, 1, 16, 129, 16) == 0
     P = ctypes.c_void_p(64)
     EFLA_ERR_ALIGN, EFLA_ERR_WORKSPACE = 8, 7
