@@ -22,6 +22,11 @@
 // through shared memory, double-buffered by parity so that one barrier per pair suffices.
 // The per-token coefficients and the two dot products that link a pair's tokens come from a
 // prologue kernel.
+//
+// With bf16 inputs at the tensor-core sizes, the tensor-core forward runs first and saves every
+// token's u = a r and the state after every 64-token chunk; heads that pass an accuracy gate
+// (moderate key norms, see saved_ok in bwd_cols_kernel) then skip the forward sweep and take
+// r = u / a and the block states from it.
 #include <algorithm>
 #include <cstdint>
 
@@ -220,13 +225,13 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // 0.013 up to 32, 0.032 for the stiff inputs with ||k||^2 up to 100) far more than with the
     // spread of a from small betas (0.006 at a max/min ratio of 800).  So the saved values are
     // used only for heads whose largest ||k||^2 is at most 16, whose a spans at most a factor of
-    // 1024, and that have no a = 0; other heads walk the forward in fp32 themselves.
-    bool saved = false;
+    // 1024, and that have no a = 0; other heads walk the forward in fp32 themselves (saved_ok).
+    bool saved_ok = false;
     if (u_saved != nullptr) {
         const int *h = hs + 4 * bh;
         const float lam_max = __int_as_float(h[1]), a_min = __int_as_float(0x7fffffff - h[2]);
         const float a_max = __int_as_float(h[3]);
-        saved = h[0] == 0 && lam_max <= 16.f && a_max <= 1024.f * a_min;
+        saved_ok = h[0] == 0 && lam_max <= 16.f && a_max <= 1024.f * a_min;
     }
     auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
         return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             const size_t g = tv + (size_t)(t0 + tt) * dv + c0 + j;
             if (reverse) {
                 xb[tt][j] = in ? dO[g] : 0.f;
-                if (saved)
+                if (saved_ok)
                     rb[tt][j] = in ? u_saved[g] / coef[2 * (tb + t0 + tt)].y : 0.f;
                 else
                     rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // ---- forward sweep: r of every token and the block-boundary states
     int par = 0;
     float kn0 = ld(k, 0), kn1 = ld(k, 1);  // k rows of the next pair
-    for (int b = 0; b < (saved ? 0 : NB); ++b) {
+    for (int b = 0; b < (saved_ok ? 0 : NB); ++b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb and cb are done
         stage(t0, cnt, false);
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             par ^= 1;
         }
     }
-    if (act && !saved) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
+    if (act && !saved_ok) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
 
     // ---- reverse sweep
 #pragma unroll
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
         __syncthreads();  // the previous block's reads of xb, rb and cb are done
         stage(t0, cnt, true);
         if (act) {  // S' after the block
-            if (saved)
+            if (saved_ok)
                 load_row16(ck_saved + (((size_t)bh * NB + b) * dk + row) * dv + c0, S);
             else
                 load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);
