@@ -252,8 +252,14 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *H,
  * and 16 of its state columns and walks the sequence twice (forward, then
  * reverse); dq, dkey and dbeta are sums over the columns, and a second kernel adds
  * the column blocks' shares in a fixed order (the result does not depend on
- * scheduling).  EFLA_ERR_ALIGN: a misaligned pointer.  EFLA_ERR_WORKSPACE: the
- * workspace is missing or too small.
+ * scheduling).  With bf16 inputs at the sizes efla_chunk_fwd runs on tensor cores
+ * (chunk 64), that forward runs first and saves every token's alpha r and the
+ * state after every 64 tokens; heads whose largest ||k||^2 is at most 16 and
+ * whose alpha spans at most a factor of 1024 (none zero) take their reverse
+ * sweep from it and skip the forward walk, the others walk it in fp32.  The
+ * workspace size covers that forward whenever the sizes allow it.
+ * EFLA_ERR_ALIGN: a misaligned pointer.  EFLA_ERR_WORKSPACE: the workspace is
+ * missing or too small.
  */
 size_t efla_bwd_workspace_size(int B, int H, int L, int dk, int dv);
 efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,
