@@ -58,6 +58,11 @@ def _load():
         lib.efla_oracle_bwd.argtypes = [ctypes.c_int] * 5 + [dp] * 12 + [ctypes.c_int]
         lib.efla_oracle_fwd_rule.restype = ctypes.c_int
         lib.efla_oracle_fwd_rule.argtypes = [ctypes.c_int] * 5 + [dp] * 7 + [ctypes.c_int] * 2
+        lib.efla_oracle_fwd_gated.restype = ctypes.c_int
+        lib.efla_oracle_fwd_gated.argtypes = [ctypes.c_int] * 5 + [dp] * 8 + [ctypes.c_int] * 2
+        lib.efla_oracle_step_gated.restype = ctypes.c_double
+        lib.efla_oracle_step_gated.argtypes = [ctypes.c_int, ctypes.c_int, dp, dp, dp, dp,
+                                               ctypes.c_double, ctypes.c_double, dp, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -87,25 +92,33 @@ def alpha(lam: float, beta: float, rule: str = "exact") -> float:
     return float(_load().efla_oracle_coeff(float(lam), float(beta), RULES[rule]))
 
 
-def step(S, q, k, v, beta: float, rule: str = "exact"):
-    """One recurrent token on one head.  Returns (S_t, o_t, alpha_t); S is not modified."""
+def step(S, q, k, v, beta: float, rule: str = "exact", g: float | None = None):
+    """One recurrent token on one head.  Returns (S_t, o_t, alpha_t); S is not modified.
+    g: the gated form's decay of this token (None: no decay)."""
     S = _f64(S).copy()
     q, k, v = _f64(q), _f64(k), _f64(v)
     dk, dv = S.shape
     o = np.zeros(dv)
-    a = _load().efla_oracle_step_rule(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta),
-                                      _ptr(o), RULES[rule])
+    if g is None:
+        a = _load().efla_oracle_step_rule(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta),
+                                          _ptr(o), RULES[rule])
+    else:
+        a = _load().efla_oracle_step_gated(dk, dv, _ptr(S), _ptr(q), _ptr(k), _ptr(v), float(beta),
+                                           float(g), _ptr(o), RULES[rule])
     return S, o, float(a)
 
 
 def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True,
-        rule: str = "exact"):
+        rule: str = "exact", g=None):
     """Token-by-token forward over [B,H,L,d] inputs.  Returns (o, S_final) in fp64.
 
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L]; S0: [B,H,dk,dv] or None (zeros).
     rule="euler" takes the delta rule's explicit Euler step (alpha = beta) instead.
+    g: [B,H,L] per-token decay of the gated form S_t = g_t (I - alpha_t k_t k_t^T) S_{t-1}
+    + alpha_t k_t v_t^T, or None (no decay).
     """
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    gg = None if g is None else _f64(g)
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     assert k.shape == (B, H, L, dk) and v.shape == (B, H, L, dv) and beta.shape == (B, H, L)
@@ -117,10 +130,13 @@ def fwd(q, k, v, beta, S0=None, nthreads: int | None = None, want_o: bool = True
     S = np.zeros((B, H, dk, dv))
     if nthreads is None:
         nthreads = os.cpu_count() or 1
-    rc = _load().efla_oracle_fwd_rule(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
-                                      _ptr(s0) if s0 is not None else None,
-                                      _ptr(o) if o is not None else None, _ptr(S), int(nthreads),
-                                      RULES[rule])
+    if gg is not None:
+        assert gg.shape == (B, H, L)
+    rc = _load().efla_oracle_fwd_gated(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                       _ptr(gg) if gg is not None else None,
+                                       _ptr(s0) if s0 is not None else None,
+                                       _ptr(o) if o is not None else None, _ptr(S), int(nthreads),
+                                       RULES[rule])
     if rc != 0:
         raise MemoryError("oracle forward failed to allocate")
     return o, S

@@ -22,6 +22,15 @@
  * interval beta_t (Methodology 1; Key Contributions): S + beta_t (k v^T -
  * k k^T S), i.e. the same update with alpha_t = beta_t ("rule" 1 below).
  *
+ * Gated form (a per-token decay g_t in (0, 1] on the carried state): the summary
+ * names Gated DeltaNet among its baselines (Experimental Results) but prints no
+ * equations for it.  The reading taken here is Gated DeltaNet's placement of the
+ * gate, on the previous state's transition, with EFLA's coefficient:
+ *
+ *   S_t = g_t (I - alpha_t k_t k_t^T) S_{t-1} + alpha_t k_t v_t^T
+ *
+ * so that g_t = 1 is EFLA itself and k_t = 0 is a pure decay S_t = g_t S_{t-1}.
+ *
  * Readings where the pages are silent:
  *   - alpha is evaluated as -expm1(-beta*lambda)/lambda, which is the same
  *     number without the cancellation of 1 - exp(x) for small x; at
@@ -66,7 +75,7 @@ double efla_oracle_coeff(double lambda, double beta, int rule)
  *   x  : scratch of length dv supplied by the caller
  */
 static void step_one(int dk, int dv, double *S, const double *q, const double *k,
-                     const double *v, double beta, double *o, double *x, int rule)
+                     const double *v, double beta, double *o, double *x, int rule, double g)
 {
     double lambda = 0.0;
     for (int i = 0; i < dk; ++i)
@@ -80,11 +89,20 @@ static void step_one(int dk, int dv, double *S, const double *q, const double *k
         for (int j = 0; j < dv; ++j)
             x[j] += S[(size_t)i * dv + j] * k[i];
 
-    /* S_t = S - alpha k x^T + alpha k v^T */
-    for (int i = 0; i < dk; ++i) {
-        const double ak = alpha * k[i];
-        for (int j = 0; j < dv; ++j)
-            S[(size_t)i * dv + j] += ak * (v[j] - x[j]);
+    /* S_t = g (S - alpha k x^T) + alpha k v^T; without a gate (g = 1) this is
+       S + alpha k (v - x)^T, evaluated exactly so */
+    if (g == 1.0) {
+        for (int i = 0; i < dk; ++i) {
+            const double ak = alpha * k[i];
+            for (int j = 0; j < dv; ++j)
+                S[(size_t)i * dv + j] += ak * (v[j] - x[j]);
+        }
+    } else {
+        for (int i = 0; i < dk; ++i) {
+            const double ak = alpha * k[i];
+            for (int j = 0; j < dv; ++j)
+                S[(size_t)i * dv + j] = g * (S[(size_t)i * dv + j] - ak * x[j]) + ak * v[j];
+        }
     }
 
     /* o_t = S_t^T q */
@@ -110,7 +128,22 @@ double efla_oracle_step_rule(int dk, int dv, double *S, const double *q, const d
     double lambda = 0.0;
     for (int i = 0; i < dk; ++i)
         lambda += k[i] * k[i];
-    step_one(dk, dv, S, q, k, v, beta, o, x, rule);
+    step_one(dk, dv, S, q, k, v, beta, o, x, rule, 1.0);
+    free(x);
+    return efla_oracle_coeff(lambda, beta, rule);
+}
+
+/* One token of the gated form (decay g on the previous state's transition). */
+double efla_oracle_step_gated(int dk, int dv, double *S, const double *q, const double *k,
+                              const double *v, double beta, double g, double *o, int rule)
+{
+    double *x = (double *)malloc(sizeof(double) * (size_t)(dv > 0 ? dv : 1));
+    if (!x)
+        return NAN;
+    double lambda = 0.0;
+    for (int i = 0; i < dk; ++i)
+        lambda += k[i] * k[i];
+    step_one(dk, dv, S, q, k, v, beta, o, x, rule, g);
     free(x);
     return efla_oracle_coeff(lambda, beta, rule);
 }
@@ -126,7 +159,7 @@ double efla_oracle_step(int dk, int dv, double *S, const double *q, const double
 
 typedef struct {
     int B, H, L, dk, dv;
-    const double *q, *k, *v, *beta, *S0;
+    const double *q, *k, *v, *beta, *gate, *S0;  /* gate: NULL = no decay */
     double *o, *S_final;
     int rule;
     int next_head; /* shared work counter */
@@ -151,7 +184,8 @@ static void run_head(fwd_job *J, int bh)
     for (int t = 0; t < L; ++t) {
         const size_t tok = (size_t)bh * L + t;
         step_one(dk, dv, S, J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
-                 J->beta[tok], J->o ? J->o + tok * dv : NULL, x, J->rule);
+                 J->beta[tok], J->o ? J->o + tok * dv : NULL, x, J->rule,
+                 J->gate ? J->gate[tok] : 1.0);
     }
     free(x);
 }
@@ -172,19 +206,19 @@ static void *worker(void *arg)
 
 /*
  * Full forward pass.
- *   q,k    : [B,H,L,dk]   v, o : [B,H,L,dv]   beta : [B,H,L]
+ *   q,k    : [B,H,L,dk]   v, o : [B,H,L,dv]   beta, gate : [B,H,L] (gate NULL: none)
  *   S0     : [B,H,dk,dv] or NULL (zeros)      S_final : [B,H,dk,dv]
  *   o may be NULL (state only).  nthreads <= 0 means one thread.
  * Returns 0 on success, -1 on allocation failure.
  */
-int efla_oracle_fwd_rule(int B, int H, int L, int dk, int dv, const double *q, const double *k,
-                         const double *v, const double *beta, const double *S0, double *o,
-                         double *S_final, int nthreads, int rule)
+int efla_oracle_fwd_gated(int B, int H, int L, int dk, int dv, const double *q, const double *k,
+                          const double *v, const double *beta, const double *gate,
+                          const double *S0, double *o, double *S_final, int nthreads, int rule)
 {
     fwd_job J;
     J.B = B; J.H = H; J.L = L; J.dk = dk; J.dv = dv;
     J.rule = rule;
-    J.q = q; J.k = k; J.v = v; J.beta = beta; J.S0 = S0;
+    J.q = q; J.k = k; J.v = v; J.beta = beta; J.gate = gate; J.S0 = S0;
     J.o = o; J.S_final = S_final;
     J.next_head = 0;
     J.failed = 0;
@@ -207,6 +241,15 @@ int efla_oracle_fwd_rule(int B, int H, int L, int dk, int dv, const double *q, c
     free(th);
     pthread_mutex_destroy(&J.lock);
     return J.failed ? -1 : 0;
+}
+
+/* Forward pass without a gate under a rule. */
+int efla_oracle_fwd_rule(int B, int H, int L, int dk, int dv, const double *q, const double *k,
+                         const double *v, const double *beta, const double *S0, double *o,
+                         double *S_final, int nthreads, int rule)
+{
+    return efla_oracle_fwd_gated(B, H, L, dk, dv, q, k, v, beta, NULL, S0, o, S_final, nthreads,
+                                 rule);
 }
 
 /* The exact-flow forward pass (rule 0). */
@@ -267,7 +310,7 @@ static void bwd_head(int L, int dk, int dv, const double *q, const double *k, co
     for (int t = 0; t < L; ++t) {
         memcpy(Ss + sz * (size_t)(t + 1), Ss + sz * (size_t)t, sizeof(double) * sz);
         step_one(dk, dv, Ss + sz * (size_t)(t + 1), q + (size_t)t * dk, k + (size_t)t * dk,
-                 v + (size_t)t * dv, beta[t], NULL, x, rule);
+                 v + (size_t)t * dv, beta[t], NULL, x, rule, 1.0);
     }
     if (dSL) memcpy(G, dSL, sizeof(double) * sz);
     else memset(G, 0, sizeof(double) * sz);
