@@ -137,7 +137,7 @@ __device__ __forceinline__ void store_row16(float *p, const float *x) {
 // (q_t . k_t, k_t . k_{t-1}, 0, 0) (k_{-1} = 0); one warp per token.  Every column block of a
 // head reads them, so they are computed once, ahead of the sweeps.  It also gathers, per head,
 // what decides whether the reverse sweep may take r = u / a from the tensor-core forward's u (see
-// saved_ok below): hs[head] = {a token has a = 0; max lambda (float bits); INT_MAX - min a
+// saved_ok below): hs[head] = {a token has a <= 0 (or NaN); max lambda (float bits); INT_MAX - min a
 // (float bits); max a (float bits)}, every field zero-initialised (a >= 0, lambda >= 0, so the
 // bit patterns order as the values do).
 template <typename T>
@@ -166,7 +166,10 @@ __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q,
             coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
             coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
             int *h = hs + 4 * (tok / (size_t)L);
-            if (a == 0.f) atomicOr(h, 1);  // u / a cannot give this head's r
+            // u / a cannot give this head's r when a is zero; a negative a (from a negative beta)
+            // or NaN would also escape the min/max statistics below, whose integer order holds for
+            // positive floats only: all of them send the head to the fp32 walk
+            if (!(a > 0.f)) atomicOr(h, 1);
             atomicMax(h + 1, __float_as_int(lam));
             atomicMax(h + 2, 0x7fffffff - __float_as_int(a));
             atomicMax(h + 3, __float_as_int(a));
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // 0.013 up to 32, 0.032 for the stiff inputs with ||k||^2 up to 100) far more than with the
     // spread of a from small betas (0.006 at a max/min ratio of 800).  So the saved values are
     // used only for heads whose largest ||k||^2 is at most 16, whose a spans at most a factor of
-    // 1024, and that have no a = 0; other heads walk the forward in fp32 themselves (saved_ok).
+    // 1024, and whose a are all positive; other heads walk the forward in fp32 themselves (saved_ok).
     bool saved_ok = false;
     if (u_saved != nullptr) {
         const int *h = hs + 4 * bh;

@@ -255,7 +255,7 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *H,
  * scheduling).  With bf16 inputs at the sizes efla_chunk_fwd runs on tensor cores
  * (chunk 64), that forward runs first and saves every token's alpha r and the
  * state after every 64 tokens; heads whose largest ||k||^2 is at most 16 and
- * whose alpha spans at most a factor of 1024 (none zero) take their reverse
+ * whose alpha spans at most a factor of 1024 (all positive) take their reverse
  * sweep from it and skip the forward walk, the others walk it in fp32.  The
  * workspace size covers that forward whenever the sizes allow it.
  * EFLA_ERR_ALIGN: a misaligned pointer.  EFLA_ERR_WORKSPACE: the workspace is

@@ -138,3 +138,39 @@ def test_backward_stiff_keys_take_the_fp32_walk(oracle_mod):
     for name, gg, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
         e = rel_err(gg.cpu().numpy(), r)
         assert e <= TOL["bf16"], (name, e)
+
+
+def test_backward_at_the_edge_of_the_saved_forward_gate(oracle_mod):
+    """A bf16 head of 128 that the gate lets through to the saved tensor-core forward at the edge
+    of both of its limits: the largest ||k||^2 just under 16 and alpha spanning close to a factor
+    of 1024 (betas log-uniform over three decades).  The gate's statistics are recomputed here from
+    the rounded inputs to make sure the head does take the saved path; every gradient, dbeta
+    included, must meet the bf16 bound."""
+    w = inputs.workload(4, B=1, H=2, L=512)
+    x = inputs.make_inputs(w, seed=41)
+    g = torch.Generator().manual_seed(42)
+    k = x["k"].double()
+    k = k / k.norm(dim=-1, keepdim=True)
+    n2 = torch.exp(np.log(0.25) + torch.rand(k.shape[:-1] + (1,), generator=g, dtype=torch.float64)
+                   * (np.log(15.5) - np.log(0.25)))
+    n2[..., 7, :] = 15.5  # one token of each head at the top of the range
+    x["k"] = (k * n2.sqrt()).to(torch.bfloat16)
+    beta = torch.exp(np.log(1.1e-3) + torch.rand(x["beta"].shape, generator=g, dtype=torch.float64)
+                     * (np.log(1.0) - np.log(1.1e-3)))
+    x["beta"] = beta.to(torch.bfloat16)
+    lam = x["k"].double().pow(2).sum(-1)
+    b = x["beta"].double()
+    a = -torch.expm1(-b * lam) / lam
+    for h in range(w.H):
+        assert 14.0 < float(lam[0, h].max()) <= 16.0
+        ratio = float(a[0, h].max() / a[0, h].min())
+        assert 500.0 < ratio <= 1024.0, ratio
+    dO = torch.randn(x["v"].shape, generator=g)
+    d = {kk: (v.cuda() if isinstance(v, torch.Tensor) else v) for kk, v in x.items()}
+    got = efla.bwd(d["q"], d["k"], d["v"], d["beta"], dO.cuda(), d["S0"], None)
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], dO, x["S0"], None)
+    for name, gg, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+        e = rel_err(gg.cpu().numpy(), r)
+        assert e <= TOL["bf16"], (name, e)
