@@ -89,11 +89,15 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
     return 0;
 }
 
-efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, const void *beta,
-                                const float *S0, void *o, float *S_final, int B, int H, int L,
-                                int dk, int dv, int chunk, efla_dtype dt, efla_dtype o_dt,
-                                efla_rule rule, void *workspace, size_t workspace_bytes,
-                                void *stream) {
+}  // extern "C"
+
+namespace efla {
+int chunk_fwd_entry(const void *q, const void *k, const void *v, const void *beta, const float *S0,
+                    void *o, float *S_final, int B, int H, int L, int dk, int dv, int chunk, int dt_i,
+                    int o_dt_i, int rule_i, void *workspace, size_t workspace_bytes, void *stream,
+                    bool allow_segments, const void *g) {
+    const efla_dtype dt = (efla_dtype)dt_i, o_dt = (efla_dtype)o_dt_i;
+    const efla_rule rule = (efla_rule)rule_i;
     if (!rule_ok(rule)) return EFLA_ERR_RULE;
     const bool euler = rule == EFLA_RULE_EULER;
     if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
@@ -101,6 +105,7 @@ efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, con
     if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
     if (dk > 128 || dv > 128 || !chunk_ok(chunk)) return EFLA_ERR_UNSUPPORTED;
     if (L > 0 && (!q || !k || !v || !beta || !o)) return EFLA_ERR_NULL;
+    if (!aligned_elem(g, dt)) return EFLA_ERR_ALIGN;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_elem(beta, dt) ||
         !aligned16(S0) || !aligned16(o) || !aligned16(S_final))
         return EFLA_ERR_ALIGN;
@@ -114,14 +119,37 @@ efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, con
                             : cudaMemsetAsync(S_final, 0, bytes, s));
     }
     if (efla::tc_supported(B, H, L, dk, dv, chunk, bf16)) {
-        const size_t need = efla::tc_workspace_bytes(B, H, L, dk, dv, chunk);
+        const size_t need = efla::tc_workspace_bytes(B, H, L, dk, dv, chunk, allow_segments);
         if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
         if (!aligned16(workspace)) return EFLA_ERR_ALIGN;
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
-                                               chunk, o_bf16, euler, workspace, s));
+                                               chunk, o_bf16, euler, workspace, s, allow_segments, g));
     }
-    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv,
+    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, g, S0, o, S_final, B, H, L, dk, dv,
                                              chunk, bf16, o_bf16, euler, s));
+}
+}  // namespace efla
+
+extern "C" {
+
+efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, const void *beta,
+                                const float *S0, void *o, float *S_final, int B, int H, int L,
+                                int dk, int dv, int chunk, efla_dtype dt, efla_dtype o_dt,
+                                efla_rule rule, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    return (efla_status)efla::chunk_fwd_entry(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, dt,
+                                              o_dt, rule, workspace, workspace_bytes, stream, true,
+                                              nullptr);
+}
+
+efla_status efla_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *beta,
+                                 const void *g, const float *S0, void *o, float *S_final, int B,
+                                 int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                                 efla_dtype o_dt, efla_rule rule, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    if (L > 0 && !g) return EFLA_ERR_NULL;
+    return (efla_status)efla::chunk_fwd_entry(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, dt,
+                                              o_dt, rule, workspace, workspace_bytes, stream, true, g);
 }
 
 efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
@@ -132,9 +160,9 @@ efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const vo
                                EFLA_RULE_EXACT, workspace, workspace_bytes, stream);
 }
 
-efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v, const void *beta,
-                                     float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
-                                     efla_dtype o_dt, efla_rule rule, void *stream) {
+static efla_status recurrent_step_entry(const void *q, const void *k, const void *v, const void *beta,
+                                       const void *g, float *S, void *o, int B, int H, int dk, int dv,
+                                       efla_dtype dt, efla_dtype o_dt, efla_rule rule, void *stream) {
     if (!rule_ok(rule)) return EFLA_ERR_RULE;
     if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
@@ -142,11 +170,24 @@ efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v
     if (dk > 256 || dv > 256) return EFLA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_NULL;
     if (!aligned_elem(q, dt) || !aligned_elem(k, dt) || !aligned_elem(v, dt) ||
-        !aligned_elem(beta, dt) || !aligned16(S) || !aligned_elem(o, o_dt))
+        !aligned_elem(beta, dt) || !aligned_elem(g, dt) || !aligned16(S) || !aligned_elem(o, o_dt))
         return EFLA_ERR_ALIGN;
-    return from_cuda(efla::launch_decode(q, k, v, beta, S, o, B * H, dk, dv, dt == EFLA_BF16,
+    return from_cuda(efla::launch_decode(q, k, v, beta, g, S, o, B * H, dk, dv, dt == EFLA_BF16,
                                          o_dt == EFLA_BF16, rule == EFLA_RULE_EULER,
                                          (cudaStream_t)stream));
+}
+
+efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v, const void *beta,
+                                     float *S, void *o, int B, int H, int dk, int dv, efla_dtype dt,
+                                     efla_dtype o_dt, efla_rule rule, void *stream) {
+    return recurrent_step_entry(q, k, v, beta, nullptr, S, o, B, H, dk, dv, dt, o_dt, rule, stream);
+}
+
+efla_status efla_recurrent_step_gated(const void *q, const void *k, const void *v, const void *beta,
+                                      const void *g, float *S, void *o, int B, int H, int dk, int dv,
+                                      efla_dtype dt, efla_dtype o_dt, efla_rule rule, void *stream) {
+    if (!g) return EFLA_ERR_NULL;
+    return recurrent_step_entry(q, k, v, beta, g, S, o, B, H, dk, dv, dt, o_dt, rule, stream);
 }
 
 efla_status efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,

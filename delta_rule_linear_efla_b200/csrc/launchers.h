@@ -19,16 +19,18 @@ cudaError_t launch_alpha(const void *k, const void *beta, float *alpha, long lon
 
 // SIMT fp32 chunkwise forward: WY/UT per chunk, state carried in fp32.
 // Any dk, dv <= 128 and chunk <= 64.
-// o_bf16 selects the output element type (fp32 or bf16).
+// o_bf16 selects the output element type (fp32 or bf16).  g: the gated form's per-token decay
+// ([B,H,L], the input type) or NULL for none.
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const void *beta,
-                              const float *S0, void *o, float *S_final, int B, int H, int L,
-                              int dk, int dv, int chunk, bool is_bf16, bool o_bf16, bool euler,
-                              cudaStream_t s);
+                              const void *g, const float *S0, void *o, float *S_final, int B,
+                              int H, int L, int dk, int dv, int chunk, bool is_bf16, bool o_bf16,
+                              bool euler, cudaStream_t s);
 
-// Recurrent single-token step per head (decode), S updated in place.
+// Recurrent single-token step per head (decode), S updated in place.  g: the gated form's
+// per-head decay of this token ([BH], the input type), or NULL for none.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *beta,
-                          float *S, void *o, int BH, int dk, int dv, bool is_bf16, bool o_bf16,
-                          bool euler, cudaStream_t s);
+                          const void *g, float *S, void *o, int BH, int dk, int dv, bool is_bf16,
+                          bool o_bf16, bool euler, cudaStream_t s);
 
 // S_out = P S_in + H per head (fp32); S_in and H may be NULL (zero); S_out may alias S_in.
 cudaError_t launch_state_affine(const float *P, const float *S_in, const float *H, float *S_out,
@@ -43,12 +45,23 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
 
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
-size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
+// allow_segments = false keeps the one-pass form (no sequence segments, whose state buffers
+// the workspace would otherwise have to hold).
+size_t tc_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk, bool allow_segments = true);
 int tc_segments(int B, int H, int L, int dk, int dv);  // sequence segments the launch uses (1: none)
+// g: the gated form's per-token decay ([B,H,L], bf16) or NULL.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *beta,
                             const float *S0, void *o, float *S_final, int B, int H, int L,
                             int dk, int dv, int chunk, bool o_bf16, bool euler, void *ws,
-                            cudaStream_t s);
+                            cudaStream_t s, bool allow_segments = true, const void *g = nullptr);
+
+// efla_chunk_fwd_rule with the choice of allowing sequence segments (the public entry points
+// allow them); returns an efla_status.
+// g: the gated form's per-token decay ([B,H,L], input type) or NULL.
+int chunk_fwd_entry(const void *q, const void *k, const void *v, const void *beta, const float *S0,
+                    void *o, float *S_final, int B, int H, int L, int dk, int dv, int chunk, int dt,
+                    int o_dt, int rule, void *workspace, size_t workspace_bytes, void *stream,
+                    bool allow_segments, const void *g);
 // The tensor-core forward without outputs, saving what the backward needs instead: every
 // token's u_t = a_t (v_t - S_{t-1}^T k_t) into u_out [B*H][L][dv] and the state after every
 // 64-token chunk into ck_out [B*H][ceil(L/64)][dk][dv] (fp32).  Same sizes as launch_chunk_tc,

@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "efla_chunk_fwd", "efla_recurrent_step", "efla_last_device_error", "efla_chunk_fwd_path",
     "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
     "efla_recurrent_step_rule", "efla_state_affine", "efla_bwd_workspace_size", "efla_bwd",
-    "efla_selftest_bounded_wait",
+    "efla_selftest_bounded_wait", "efla_chunk_fwd_gated", "efla_recurrent_step_gated",
 )
 
 _lib = None
@@ -83,6 +83,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_state_affine.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
     L.efla_recurrent_step_rule.restype = i
     L.efla_recurrent_step_rule.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    L.efla_chunk_fwd_gated.restype = i
+    L.efla_chunk_fwd_gated.argtypes = [vp] * 8 + [i] * 9 + [vp, sz, vp]
+    L.efla_recurrent_step_gated.restype = i
+    L.efla_recurrent_step_gated.argtypes = [vp] * 7 + [i] * 7 + [vp]
     if path is None:
         _lib = L
     return L
@@ -160,9 +164,11 @@ def chunk_fwd_path(B, H, L, dk, dv, chunk, dtype, o_dtype=torch.float32) -> str:
 
 def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
               want_state: bool = True, workspace=None, o_dtype=torch.float32, stream=None,
-              rule: str = "exact"):
+              rule: str = "exact", g=None):
     """EFLA forward in the WY/UT chunkwise form.  Returns (o, S_final or None).
     rule="euler" runs the same kernels with the delta rule's coefficient alpha = beta.
+    g: [B,H,L] per-token decay of the gated form S_t = g_t (I - alpha_t k_t k_t^T) S_{t-1}
+    + alpha_t k_t v_t^T (efla_chunk_fwd_gated), or None.
 
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; beta: [B,H,L], all float32 or all bfloat16 on one
     CUDA device; S0: [B,H,dk,dv] float32 or None.  o is float32 by default (the fp32
@@ -172,9 +178,11 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L):
         raise ValueError("shape mismatch: q,k [B,H,L,dk], v [B,H,L,dv], beta [B,H,L]")
+    if g is not None and g.shape != (B, H, L):
+        raise ValueError("g must be [B,H,L]")
     code = _dtype_code(q)
-    for name, t in (("k", k), ("v", v), ("beta", beta)):
-        if t.dtype != q.dtype:
+    for name, t in (("k", k), ("v", v), ("beta", beta), ("g", g)):
+        if t is not None and t.dtype != q.dtype:
             raise TypeError("%s must have q's dtype %s" % (name, q.dtype))
     if o is not None:
         o_dtype = o.dtype
@@ -188,14 +196,20 @@ def chunk_fwd(q, k, v, beta, S0=None, chunk: int = 64, o=None, S_final=None,
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
     ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
-    st = load_library().efla_chunk_fwd_rule(
-        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
-        _dev(S0, "S0", torch.float32) if S0 is not None else None,
-        _dev(o, "o", o_dtype),
-        _dev(S_final, "S_final", torch.float32) if S_final is not None else None,
-        B, H, L, dk, dv, int(chunk), code, o_code, _rule(rule), ws_ptr, ws_bytes,
-        _stream_handle(stream))
-    _check(st, "efla_chunk_fwd_rule")
+    S0p = _dev(S0, "S0", torch.float32) if S0 is not None else None
+    Sfp = _dev(S_final, "S_final", torch.float32) if S_final is not None else None
+    if g is None:
+        st = load_library().efla_chunk_fwd_rule(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"), S0p, _dev(o, "o", o_dtype),
+            Sfp, B, H, L, dk, dv, int(chunk), code, o_code, _rule(rule), ws_ptr, ws_bytes,
+            _stream_handle(stream))
+        _check(st, "efla_chunk_fwd_rule")
+    else:
+        st = load_library().efla_chunk_fwd_gated(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"), _dev(g, "g"), S0p,
+            _dev(o, "o", o_dtype), Sfp, B, H, L, dk, dv, int(chunk), code, o_code, _rule(rule),
+            ws_ptr, ws_bytes, _stream_handle(stream))
+        _check(st, "efla_chunk_fwd_gated")
     return o, S_final
 
 
@@ -214,10 +228,10 @@ def chunk_fwd_noalloc(q, k, v, beta, o, S_final=None, S0=None, chunk: int = 64, 
 
 
 def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None,
-                   rule: str = "exact"):
+                   rule: str = "exact", g=None):
     """One decode token per head; S ([B,H,dk,dv] float32) is updated in place.  Returns o
     (float32 by default, or bfloat16 with o_dtype=torch.bfloat16).  rule="euler" takes the
-    delta rule's step (alpha = beta)."""
+    delta rule's step (alpha = beta).  g: [B,H] decay of the gated form, or None."""
     B, H, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:2] != (B, H) or beta.shape != (B, H) or \
@@ -228,11 +242,20 @@ def recurrent_step(q, k, v, beta, S, o=None, o_dtype=torch.float32, stream=None,
         o_dtype = o.dtype
     if o is None:
         o = torch.empty((B, H, dv), dtype=o_dtype, device=q.device)
-    st = load_library().efla_recurrent_step_rule(
-        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
-        _dev(S, "S", torch.float32), _dev(o, "o", o_dtype), B, H, dk, dv, code, _code(o_dtype),
-        _rule(rule), _stream_handle(stream))
-    _check(st, "efla_recurrent_step_rule")
+    if g is None:
+        st = load_library().efla_recurrent_step_rule(
+            _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
+            _dev(S, "S", torch.float32), _dev(o, "o", o_dtype), B, H, dk, dv, code, _code(o_dtype),
+            _rule(rule), _stream_handle(stream))
+        _check(st, "efla_recurrent_step_rule")
+    else:
+        if g.shape != (B, H):
+            raise ValueError("g must be [B,H]")
+        st = load_library().efla_recurrent_step_gated(
+            _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dev(beta, "beta", q.dtype),
+            _dev(g, "g", q.dtype), _dev(S, "S", torch.float32), _dev(o, "o", o_dtype), B, H, dk, dv,
+            code, _code(o_dtype), _rule(rule), _stream_handle(stream))
+        _check(st, "efla_recurrent_step_gated")
     return o
 
 

@@ -127,6 +127,13 @@ def make_inputs(w: Workload | int, seed: int | None = None) -> dict:
     return dict(q=q, k=k, v=v, beta=beta, S0=S0, chunk=w.chunk, workload=w)
 
 
+def make_gate(shape, dtype, seed: int) -> torch.Tensor:
+    """Per-token decays for the gated form, sigmoid(N(2, 1)) (mean about 0.86, a few tokens near
+    0.5), drawn with their own seeded generator and rounded to `dtype`."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.sigmoid(2.0 + torch.randn(shape, generator=g, dtype=torch.float32)).to(dtype)
+
+
 def make_decode_inputs(w: Workload | int = 4, seed: int | None = None) -> dict:
     """Decode batch of a workload that carries one (workload 4).
 

@@ -138,6 +138,14 @@ size_t efla_chunk_fwd_workspace_size(int B, int H, int L, int dk, int dv, int ch
  * S0 and S_final may alias (in-place state carry).  o must not alias inputs.
  * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  L == 0 copies S0 to S_final.
  * Calls on the same workspace must be ordered on one stream.
+ * Range: with bf16 inputs, dk and dv in {64, 128} and chunk 64, the products
+ * run on the tensor cores with fp16 operands and fp32 accumulation: q, k and v
+ * are converted to fp16 (exact for bf16 values of magnitude 2^-14 .. 65504),
+ * and so are the intermediates u_t = alpha_t (v_t - S_{t-1}^T k_t) and the
+ * state's operand copy.  A value beyond fp16's largest finite magnitude,
+ * 65504, in the inputs or in those intermediates becomes inf and the outputs
+ * inf or NaN, with status EFLA_OK (input values are not inspected).  fp32
+ * inputs take the SIMT path, which has no such limit.
  */
 efla_status efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
                            const float *S0, void *o, float *S_final,
@@ -153,6 +161,32 @@ efla_status efla_chunk_fwd_rule(const void *q, const void *k, const void *v, con
                                 int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
                                 efla_dtype o_dt, efla_rule rule, void *workspace,
                                 size_t workspace_bytes, void *stream);
+
+/*
+ * efla_chunk_fwd_gated -- the gated form: a per-token decay g_t on the carried
+ * state,
+ *
+ *   S_t = g_t (I - alpha_t k_t k_t^T) S_{t-1} + alpha_t k_t v_t^T,  o_t = S_t^T q_t.
+ *
+ * The summary names Gated DeltaNet among its baselines (Experimental Results)
+ * without printing its equations; this is Gated DeltaNet's placement of the
+ * gate, on the previous state's transition, with EFLA's coefficient (or beta
+ * under EFLA_RULE_EULER, which is then Gated DeltaNet's own update).  g_t = 1
+ * is efla_chunk_fwd_rule; k_t = 0 is a pure decay S_t = g_t S_{t-1}.
+ *
+ *   g : [B,H,L] (dt), the decay of each token, expected in (0, 1] (not
+ *       checked: the chunkwise form takes its logarithm, so g <= 0 gives NaN).
+ * The chunkwise form carries the decays as cumulative logarithms within each
+ * chunk, so every factor it applies is a decay of at most 1.  Everything else
+ * (arguments, layouts, workspace, sizes, errors) is as efla_chunk_fwd_rule;
+ * the workspace query is efla_chunk_fwd_workspace_size.  EFLA_ERR_NULL when g
+ * is NULL and L > 0.
+ */
+efla_status efla_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *beta,
+                                 const void *g, const float *S0, void *o, float *S_final,
+                                 int B, int H, int L, int dk, int dv, int chunk, efla_dtype dt,
+                                 efla_dtype o_dt, efla_rule rule, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /*
  * efla_chunk_fwd_noalloc -- the same forward pass as efla_chunk_fwd for callers
@@ -214,6 +248,17 @@ efla_status efla_recurrent_step_rule(const void *q, const void *k, const void *v
                                      const void *beta, float *S, void *o, int B, int H, int dk,
                                      int dv, efla_dtype dt, efla_dtype o_dt, efla_rule rule,
                                      void *stream);
+
+/*
+ * efla_recurrent_step_gated -- one decode token of the gated form (see
+ * efla_chunk_fwd_gated): S <- g (I - alpha k k^T) S + alpha k v^T in place,
+ * then o = S^T q.  g : [B,H] (dt).  EFLA_ERR_NULL when g is NULL; otherwise as
+ * efla_recurrent_step_rule.
+ */
+efla_status efla_recurrent_step_gated(const void *q, const void *k, const void *v,
+                                      const void *beta, const void *g, float *S, void *o, int B,
+                                      int H, int dk, int dv, efla_dtype dt, efla_dtype o_dt,
+                                      efla_rule rule, void *stream);
 
 /*
  * efla_state_affine -- S_out = P S_in + H for every head, in fp32.  No counterpart
