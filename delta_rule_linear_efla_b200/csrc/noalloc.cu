@@ -41,14 +41,24 @@ extern "C" efla_status efla_chunk_fwd_noalloc(const void *q, const void *k, cons
                                               float *S_final, int B, int H, int L, int dk, int dv,
                                               int chunk, efla_dtype dt, efla_dtype o_dt,
                                               void *stream) {
-    // Sizes beyond the fixed scratch are refused before anything else happens.
-    const size_t need = efla_chunk_fwd_workspace_size(B, H, L, dk, dv, chunk, dt, o_dt);
+    // Scratch the call needs: with sequence segments where the sizes would take them, else in
+    // the one-pass form, which needs less (no segment states).  Sizes that fit neither way are
+    // refused before anything else happens.
+    size_t need = efla_chunk_fwd_workspace_size(B, H, L, dk, dv, chunk, dt, o_dt);
+    bool allow_segments = true;
+    if (need > EFLA_NOALLOC_SCRATCH_BYTES && dt == EFLA_BF16 &&
+        efla::tc_supported(B, H, L, dk, dv, chunk, true)) {
+        need = efla::tc_workspace_bytes(B, H, L, dk, dv, chunk, false);
+        allow_segments = false;
+    }
     if (need > EFLA_NOALLOC_SCRATCH_BYTES) return EFLA_ERR_TOO_LARGE;
     void *scratch = nullptr;
     if (need > 0) {
         const efla_status st = scratch_address(&scratch);
         if (st != EFLA_OK) return st;
     }
-    return efla_chunk_fwd(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, dt, o_dt, scratch,
-                          need > 0 ? (size_t)EFLA_NOALLOC_SCRATCH_BYTES : 0, stream);
+    return (efla_status)efla::chunk_fwd_entry(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, chunk, dt,
+                                              o_dt, EFLA_RULE_EXACT, scratch,
+                                              need > 0 ? (size_t)EFLA_NOALLOC_SCRATCH_BYTES : 0, stream,
+                                              allow_segments, nullptr);
 }

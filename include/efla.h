@@ -204,9 +204,13 @@ efla_status efla_chunk_fwd_gated(const void *q, const void *k, const void *v, co
  * per-chunk T*diag(alpha) tiles (8 KiB per 64-token chunk of each head) in one
  * fixed array of EFLA_NOALLOC_SCRATCH_BYTES inside the library's device code.
  * Every GPU on which the library's kernels are loaded holds that memory until
- * the process exits.  Sizes that need more -- B*H*ceil(L/64) > 4096 chunks on
- * the tensor-core path -- return EFLA_ERR_TOO_LARGE before anything is
- * enqueued.  Sizes served by the SIMT path need no scratch at all.
+ * the process exits.  Where efla_chunk_fwd would cut the sequence into
+ * segments (few heads, long sequences) it also keeps their states there; when
+ * those do not fit beside the tiles, this call runs the one-pass form instead
+ * (same results, fewer SMs busy).  Sizes whose tiles alone need more --
+ * B*H*ceil(L/64) > 4096 chunks on the tensor-core path -- return
+ * EFLA_ERR_TOO_LARGE before anything is enqueued.  Sizes served by the SIMT
+ * path need no scratch at all.
  *
  * Set-up: the first call on a device looks up the array's device address once
  * for that device (it must be the current device); make that first call before
