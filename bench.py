@@ -47,12 +47,15 @@ def _peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def alg_bytes_chunk(w) -> int:
-    """Algorithmic HBM bytes of one chunk forward: read q, k, v, beta (input dtype) and
-    write o (fp32) per token-head, plus the fp32 final state per head (S0 is zero here and
-    not read)."""
+def alg_bytes_chunk(w, o_bytes: int | None = None) -> int:
+    """Algorithmic HBM bytes of one chunk forward: read q, k, v, beta and write o per
+    token-head, plus the fp32 final state per head (S0 is zero here and not read).  By default
+    o is counted at the input dtype, the count of the hot-path scope table (1026 B per
+    token-head at dk = dv = 128 in bf16); o_bytes = 4 counts the fp32 output the library
+    writes by default."""
     es = 2 if w.dtype == "bf16" else 4
-    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * 4
+    ob = es if o_bytes is None else o_bytes
+    per_tok = (2 * w.dk + w.dv) * es + es + w.dv * ob + (es if GATED else 0)  # + the decay g
     return w.token_heads * per_tok + w.B * w.H * w.dk * w.dv * 4
 
 
@@ -174,8 +177,8 @@ FWD_SOURCES = ("chunk_tc.cu", "common.cuh", "tc_ptx.cuh")
 
 
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources the chunk forward's kernels are built from (the tcgen05 prep,
-    state and segment kernels and the helpers they include): ties profiled counters to them."""
+    """Hash of the CUDA sources the chunk forward's kernels are built from (the tcgen05 pair and
+    segment kernels and the helpers they include): ties profiled counters to them."""
     import hashlib
 
     h = hashlib.sha256()
@@ -211,21 +214,22 @@ def cpu_baseline(w, seconds_target: float = 12.0) -> dict:
 
     oracle.build()
     cores = os.cpu_count() or 1
-    x = inputs.make_inputs(inputs.workload(w.id, B=1, H=1))
+    x = _with_gate(inputs.make_inputs(inputs.workload(w.id, B=1, H=1)), 7)
     t0 = time.perf_counter()
-    oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], nthreads=1, rule=RULE)
+    oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], nthreads=1, rule=RULE, g=x.get("g"))
     t_head = max(time.perf_counter() - t0, 1e-3)
     # about `seconds_target` of wall time with every core busy on whole heads
     heads = max(1, min(w.B * w.H, cores * max(1, int(seconds_target / t_head))))
     H = min(heads, w.H)
     B = max(1, min(w.B, heads // H))
-    xs = inputs.make_inputs(inputs.workload(w.id, B=B, H=H))
+    xs = _with_gate(inputs.make_inputs(inputs.workload(w.id, B=B, H=H)), 8)
     threads = min(cores, B * H)
     # repeat the sample until it amounts to ~seconds_target of CPU work (core-seconds)
     reps, dt = 0, 0.0
     t0 = time.perf_counter()
     while reps < 50 and (reps == 0 or dt * threads < seconds_target):
-        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE)
+        oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads, rule=RULE,
+                   g=xs.get("g"))
         reps += 1
         dt = time.perf_counter() - t0
     n = B * H * w.L * reps
@@ -247,14 +251,14 @@ def run_reference(args) -> None:
     bwd = args.pass_ == "bwd"
     # the backward oracle runs heads one after another (it keeps every state): a smaller sample
     H = min(w.H, 2 if bwd else cores)
-    xs = inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 512 if bwd else 1024)))
+    xs = _with_gate(inputs.make_inputs(inputs.workload(w.id, B=1, H=H, L=min(w.L, 512 if bwd else 1024))), 9)
     threads = 1 if bwd else min(cores, H)
     if bwd:
         dO = torch.randn(xs["v"].shape, generator=torch.Generator().manual_seed(77), dtype=torch.float64)
         run = lambda: oracle.bwd(xs["q"], xs["k"], xs["v"], xs["beta"], dO, xs["S0"], None, rule=RULE)
     else:
         run = lambda: oracle.fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["S0"], nthreads=threads,
-                                 rule=RULE)
+                                 rule=RULE, g=xs.get("g"))
     for _ in range(args.warmup):
         run()
     t0 = time.perf_counter()
@@ -278,6 +282,14 @@ def run_reference(args) -> None:
 
 
 RULE = "exact"  # set from --rule: "exact" (the method) or "euler" (the delta rule, for comparison)
+GATED = False  # set from --gated: the gated form, a per-token decay g_t ~ sigmoid(N(2, 1))
+
+
+def _with_gate(x: dict, seed: int) -> dict:
+    """The inputs with the gated form's per-token decay added (when --gated)."""
+    if GATED:
+        x["g"] = inputs.make_gate(x["beta"].shape, x["beta"].dtype, seed)
+    return x
 
 
 def _config(w) -> dict:
@@ -286,9 +298,72 @@ def _config(w) -> dict:
         "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
         "l2": "inputs > L2 (126 MB): two rotating input sets per rank",
         "o_dtype": "fp32", "rule": RULE}
+    if GATED:
+        c["gate"] = "g_t ~ sigmoid(N(2, 1)) per token: S_t = g_t (I - a k k^T) S + a k v^T"
     if w.decode:
         c["decode"] = "B=%d H=%d one token, fp32 carried state" % (w.decode["B"], w.decode["H"])
     return c
+
+
+def _roofline(w, chunk_ms: float, peaks: dict, path: str, o_dtype=torch.float32) -> dict:
+    """HBM roofline of one efla_chunk_fwd call from its CUDA-event time.  `frac` counts the
+    algorithmic bytes with o at the input dtype (the hot-path scope table's count); the
+    `fp32_output` entry counts o at 4 bytes, what the call writes with an fp32 output."""
+    alg = alg_bytes_chunk(w)
+    achieved = alg / (chunk_ms / 1e3) / 1e9
+    r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+         "frac": achieved / peaks["hbm"], "alg_bytes_per_launch": alg, "avg_launch_ms": chunk_ms,
+         "kernel": "efla_chunk_fwd (%s path), o written as %s" % (
+             path, "fp32" if o_dtype == torch.float32 else "bf16"),
+         "peak_source": peaks["src"] + " (MEASURED_PEAKS.json hbm_gbs, copy burst)"}
+    if o_dtype == torch.float32:
+        alg32 = alg_bytes_chunk(w, o_bytes=4)
+        a32 = alg32 / (chunk_ms / 1e3) / 1e9
+        r["fp32_output"] = {"alg_bytes_per_launch": alg32, "achieved": a32, "frac": a32 / peaks["hbm"]}
+    return r
+
+
+def time_chunk_fwd(w, dev, peaks: dict, steps: int, o_dtype=torch.float32) -> dict:
+    """efla_chunk_fwd alone on a workload: two rotating input sets (larger than L2 together),
+    3 warm-up calls, then `steps` calls each timed with CUDA events on the launching stream."""
+    from delta_rule_linear_efla_b200 import efla
+
+    sets = []
+    for r in range(2):
+        x = _with_gate(inputs.make_inputs(w, seed=1000 + w.id + 17 * r), 500 + r)
+        sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
+    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=o_dtype, device=dev) for _ in range(2)]
+    Sf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    wsb = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(), o_dtype)
+    wsp = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    path = efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(), o_dtype)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(i):
+        x = sets[i % 2]
+        efla.chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], chunk=w.chunk, o=o_buf[i % 2],
+                       S_final=Sf, workspace=wsp, o_dtype=o_dtype, rule=RULE, g=x.get("g"))
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        call(i)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if efla.last_device_error() != 0:
+        raise RuntimeError("device error word set")
+    ms = [a.elapsed_time(b) for a, b in evs]
+    mean = sum(ms) / len(ms)
+    r = _roofline(w, mean, peaks, path, o_dtype)
+    r.update({"workload": _config(w)["workload"], "ms": mean, "ms_min": min(ms),
+              "token_heads_per_s": w.token_heads / (mean / 1e3), "steps": steps})
+    del sets, o_buf, wsp
+    torch.cuda.empty_cache()
+    return r
 
 
 def run_ours(args) -> None:
@@ -306,7 +381,8 @@ def run_ours(args) -> None:
     # ---- inputs: two rotating sets so consecutive steps do not hit in L2 ----
     sets = []
     for r in range(2):
-        x = inputs.make_inputs(w, seed=edist.replica_seed(1000 + w.id, rank, r))
+        x = _with_gate(inputs.make_inputs(w, seed=edist.replica_seed(1000 + w.id, rank, r)),
+                       edist.replica_seed(600, rank, r))
         sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
     o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
     Sf_buf = [torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
@@ -324,6 +400,8 @@ def run_ours(args) -> None:
         pd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in p.items()}
         _, S_carry = efla.chunk_fwd(pd["q"], pd["k"], pd["v"], pd["beta"], None, chunk=w.chunk,
                                     rule=RULE)
+        if GATED:
+            dd["g"] = inputs.make_gate((w.decode["B"], w.decode["H"]), w.torch_dtype(), 700 + rank).to(dev)
         dd["S_init"] = S_carry
         dd["S"] = [S_carry.clone(), S_carry.clone()]
         dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=torch.float32, device=dev)
@@ -338,12 +416,12 @@ def run_ours(args) -> None:
         if ev_pair is not None:
             ev_pair[0].record(stream)
         efla.chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], chunk=w.chunk,
-                       o=o_buf[i % 2], S_final=Sf_buf[i % 2], workspace=wsp, rule=RULE)
+                       o=o_buf[i % 2], S_final=Sf_buf[i % 2], workspace=wsp, rule=RULE, g=x.get("g"))
         if ev_pair is not None:
             ev_pair[1].record(stream)
         if dec is not None:
             efla.recurrent_step(dec["q"], dec["k"], dec["v"], dec["beta"], dec["S"][i % 2],
-                                o=dec["o"], rule=RULE)
+                                o=dec["o"], rule=RULE, g=dec.get("g"))
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -374,26 +452,22 @@ def run_ours(args) -> None:
         raise RuntimeError("device error word set: %s" % efla.status_str(err))
 
     value = edist.aggregate_rate(tok_step, args.steps, ws, ms)
-    alg = alg_bytes_chunk(w)
-    achieved = alg / (chunk_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm"], "traffic": profiled_traffic(w),
-                "kernel": "efla_chunk_fwd (%s path: prep + state kernels)" % path,
-                "alg_bytes_per_launch": alg, "avg_launch_ms": chunk_ms,
-                "peak_source": peaks["src"] + " (MEASURED_PEAKS.json hbm_gbs, copy burst)",
-                "source_hash": kernel_source_hash()}
+    roofline = _roofline(w, chunk_ms, peaks, path)
+    roofline["traffic"] = profiled_traffic(w)
+    roofline["source_hash"] = kernel_source_hash()
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
         xh = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v)
-              for k, v in inputs.make_inputs(w, seed=4242 + rank).items()}
+              for k, v in _with_gate(inputs.make_inputs(w, seed=4242 + rank), 4343 + rank).items()}
         o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32).pin_memory()
         S_host = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
-        h2d = sum(xh[k].numel() * xh[k].element_size() for k in ("q", "k", "v", "beta"))
+        names = ("q", "k", "v", "beta") + (("g",) if GATED else ())
+        h2d = sum(xh[k].numel() * xh[k].element_size() for k in names)
         d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
         if dec is not None:
-            dh = {k: dec[k].cpu().pin_memory() for k in ("q", "k", "v", "beta")}
+            dh = {k: dec[k].cpu().pin_memory() for k in ("q", "k", "v", "beta") + (("g",) if GATED else ())}
             S_dec_host = dec["S_init"].cpu().pin_memory()
             od_host = torch.empty_like(dec["o"], device="cpu").pin_memory()
             h2d += sum(t.numel() * t.element_size() for t in dh.values()) + S_dec_host.numel() * 4
@@ -403,7 +477,6 @@ def run_ours(args) -> None:
         # one copy stream and downloads on another, so step i+1's upload and step i's download
         # overlap step i's kernels.  Every step still moves its own inputs in and results out.
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        names = ("q", "k", "v", "beta")
         din = [{k: torch.empty_like(xh[k], device=dev) for k in names} for _ in range(2)]
         o_host2 = [o_host, torch.empty_like(o_host).pin_memory()]
         S_host2 = [S_host, torch.empty_like(S_host).pin_memory()]
@@ -430,10 +503,11 @@ def run_ours(args) -> None:
             stream.wait_event(ev["out_free"][j])  # step i-2's downloads are done with the outputs
             g = din[j]
             efla.chunk_fwd(g["q"], g["k"], g["v"], g["beta"], None, chunk=w.chunk, o=o_buf[j],
-                           S_final=Sf_buf[j], workspace=wsp, rule=RULE)
+                           S_final=Sf_buf[j], workspace=wsp, rule=RULE, g=g.get("g"))
             if dec is not None:
                 gd = ddin[j]
-                efla.recurrent_step(gd["q"], gd["k"], gd["v"], gd["beta"], Sd2[j], o=od2[j], rule=RULE)
+                efla.recurrent_step(gd["q"], gd["k"], gd["v"], gd["beta"], Sd2[j], o=od2[j], rule=RULE,
+                                    g=gd.get("g"))
             ev["in_free"][j].record(stream)
             ev["done"][j].record(stream)
             with torch.cuda.stream(s_out):
@@ -462,6 +536,17 @@ def run_ours(args) -> None:
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
 
+    per_workload = None
+    if ws == 1 and not args.no_per_workload:
+        per_workload = {}
+        for wid in (3, 4, 5):
+            if wid != w.id:
+                per_workload[str(wid)] = time_chunk_fwd(inputs.WORKLOADS[wid], dev, peaks, args.steps)
+        # the headline workload with o rounded to the input dtype (bf16), the output the
+        # algorithmic byte count assumes
+        per_workload["%d_o_bf16" % w.id] = time_chunk_fwd(w, dev, peaks, args.steps,
+                                                         o_dtype=torch.bfloat16)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -479,7 +564,7 @@ def run_ours(args) -> None:
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic", "config": _config(w), "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
-        "path": path, "token_heads_per_step": tok_step,
+        "path": path, "token_heads_per_step": tok_step, "per_workload": per_workload,
     }
     print(json.dumps(line), flush=True)
 
@@ -493,6 +578,10 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gated", action="store_true",
+                    help="the gated form: a per-token decay g_t ~ sigmoid(N(2, 1)) on the carried state")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip timing the other workloads' chunk forward after the timed region")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd (default): the forward step; bwd: the backward pass alone")
     ap.add_argument("--rule", choices=["exact", "euler"], default="exact",
@@ -500,10 +589,13 @@ def main():
                          "for the throughput comparison (the workload's keys are not normalised, "
                          "so under euler only the time is meaningful)")
     args = ap.parse_args()
-    global RULE
+    global RULE, GATED
     RULE = args.rule
+    GATED = args.gated
     if args.warmup < 3:
         args.warmup = 3
+    if args.gated and args.pass_ == "bwd":
+        raise SystemExit("--pass bwd: the backward pass is for the ungated form")
     if args.impl == "reference":
         run_reference(args)
     elif args.pass_ == "bwd":
