@@ -24,10 +24,23 @@
 //           warpgroups that move results between TMEM and the operand tiles; the
 //           fp32 state S^T stays in TMEM across chunks, with an fp16 copy as D1's A.
 //  seg_combine -- for sequence segments: chains the segments' affine state maps.
-//  pair::tc_pair_kernel -- the gated form (a per-token decay on the carried state): each run
-//           is a cluster of two CTAs, a state CTA with the chain's products and a producer
-//           CTA that computes the Gram, the triangular solve and W per chunk and hands Ta and
-//           -W over by bulk copies within the cluster (no prep kernel, no Ta in HBM).
+//
+// The gated form (a per-token decay g_t on the carried state, S_t = g_t (I - a_t k_t
+// k_t^T) S_{t-1} + a_t k_t v_t^T) runs on the same two kernels.  With l_t the cumulative
+// log-decay from the chunk start to token t (l_C at the chunk's last token) and
+// Gam_ts = e^{l_t - l_s}, the chunk algebra becomes
+//
+//   A  = strictly-lower(diag(a) (Gam o K K^T))    Ta = T diag(a) as before
+//   W  = Ta diag(e^{l}) K,  U = Ta V,  U' = U - W S
+//   O  = diag(e^{l}) Q S + (lower-incl(Gam) o Q K^T) U'
+//   S <- e^{l_C} S + K^T diag(e^{l_C - l}) U'
+//
+// and every factor it applies is a decay of at most 1 (a split of Gam into e^{l_t - l_C}
+// e^{l_C - l_s} would over- and underflow): the prep kernel weights the Gram by Gam; the
+// state kernel's converter writes q and k both as they are and with their rows scaled by
+// e^{l_t} (the scaled q for D1, the scaled k for W), the side group weights P^T by Gam, the chain group hands D2 U' twice
+// (as it is for the output, with its rows scaled by e^{l_C - l_t} for the state update),
+// and scales the fp32 state by the next chunk's e^{l_C} when it copies it for D1.
 //
 // Every mbarrier wait is bounded; a wait that gives up sets the device error
 // word, drains the copies this CTA has in flight (again bounded), releases
@@ -42,6 +55,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "tc_ptx.cuh"
+#include "tmap.h"
 
 namespace efla {
 
@@ -55,6 +69,29 @@ constexpr long long WAIT_BUDGET = 2000000000LL;  // ~1 s of SM cycles
 
 __device__ __forceinline__ void record_error(unsigned code) { atomicOr(&g_tc_error, code); }
 
+// ------------------------------------------------------------------ gated form: per-token log-decays
+// l_t of a chunk's tokens 2 lane and 2 lane + 1, for every lane of a warp (0 past the sequence
+// end, where the decay is taken as 1): a warp-wide inclusive scan of the pairs' logarithms.
+__device__ __forceinline__ float2 chunk_logdecay(const __nv_bfloat16 *gate_row, int t0, int L, int lane) {
+    const int t = t0 + 2 * lane;
+    const float x0 = t < L ? logf(__bfloat162float(gate_row[t])) : 0.f;
+    const float x1 = t + 1 < L ? logf(__bfloat162float(gate_row[t + 1])) : 0.f;
+    float s = x0 + x1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+    }
+    return make_float2(s - x1, s);
+}
+// Element t of a per-token quantity held as pairs (lane t / 2 holds tokens 2 lane, 2 lane + 1),
+// e.g. l_t itself or a factor made from it (every lane of the warp takes part; t need not be
+// uniform).
+__device__ __forceinline__ float logdecay_at(float2 p, int t) {
+    const float a = __shfl_sync(0xffffffffu, p.x, t >> 1), b = __shfl_sync(0xffffffffu, p.y, t >> 1);
+    return (t & 1) ? b : a;
+}
+
 // ------------------------------------------------------------------ prep
 // One chunk at a time (all chunks in parallel across the grid):
 //   1. K arrives by TMA; a per row from the squared norm (fp32).
@@ -65,6 +102,8 @@ __device__ __forceinline__ void record_error(unsigned code) { atomicOr(&g_tc_err
 //        T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ
 //      with warp-level mma.sync (fp16 operands, fp32 accumulation).
 //   4. Ta = T diag(a), rounded to fp16, written to the workspace (64x64 per chunk).
+// Gated form: the Gram's entry (t, s) is weighted by e^{l_t - l_s} (at most 1 below the
+// diagonal), with l the chunk's cumulative log-decays.
 namespace prep {
 constexpr int LD16 = 72;   // fp16 row stride (halves) of the 64x64 operand tiles
 
@@ -80,7 +119,7 @@ struct Smem {
     static constexpr int RT = 4 * 16 * 24 * 2;    // per-warp 16x16 scratch (transposed R), fp16
     static constexpr int AD_RT = ADIAG > RT ? ADIAG : RT;
     template <int DK>
-    static constexpr int bytes() { return region0<DK>() + T16T + C * 4; }
+    static constexpr int bytes() { return region0<DK>() + T16T + 2 * C * 4; }  // + a, l per row
     // The K tile is dead once the Gram MMA and the norms have read it; the solve's A, T
     // diagonal blocks and scratch then take its place (the next K is loaded after the solve).
     static constexpr int SCRATCH = A16 + TD16 + AD_RT;
@@ -111,10 +150,11 @@ __device__ __forceinline__ void load_b(uint32_t &b0, uint32_t &b1, const __half 
 }
 }  // namespace prep
 
-template <int DK>
+template <int DK, bool GATED = false>
 __global__ void __launch_bounds__(THREADS)
     tc_prep_kernel(const __grid_constant__ CUtensorMap tmap_k, const __nv_bfloat16 *__restrict__ beta,
-                   __half *__restrict__ ta_out, int L, int NC, int total, bool euler) {
+                   const __nv_bfloat16 *__restrict__ gate, __half *__restrict__ ta_out, int L, int NC,
+                   int total, bool euler) {
     using namespace prep;
     constexpr int KB = Smem::k_bytes<DK>();
     extern __shared__ uint8_t smem_raw[];
@@ -127,6 +167,7 @@ __global__ void __launch_bounds__(THREADS)
     __half *Rt = reinterpret_cast<__half *>(Ad);                // after the solve: merge scratch
     __half *T16t = reinterpret_cast<__half *>(base + Smem::region0<DK>());
     float *al = reinterpret_cast<float *>(T16t + C * LD16);
+    float *lg = al + C;  // gated: l_t of the chunk's rows
     __shared__ uint64_t full, mma_bar;
     __shared__ uint32_t tmem_base;
 
@@ -165,6 +206,18 @@ __global__ void __launch_bounds__(THREADS)
         return n * C + tid < L ? __bfloat162float(beta[(size_t)bh * L + n * C + tid]) : 0.f;
     };
     float beta_next = load_beta(blockIdx.x);
+    // gated: warp 0's lane holds log g of rows 2 lane and 2 lane + 1 of chunk gg (0 past the
+    // sequence end), also loaded a chunk ahead
+    auto load_gate = [&](int gg) {
+        float2 x = make_float2(0.f, 0.f);
+        if (!GATED || warp != 0 || gg >= total) return x;
+        const int bh = gg / NC, t = (gg - bh * NC) * C + 2 * lane;
+        const __nv_bfloat16 *row = gate + (size_t)bh * L;
+        if (t < L) x.x = logf(__bfloat162float(row[t]));
+        if (t + 1 < L) x.y = logf(__bfloat162float(row[t + 1]));
+        return x;
+    };
+    float2 gate_next = load_gate(blockIdx.x);
     uint32_t mma_phase = 0;
     int it = 0;
     bool aborted = false;
@@ -175,6 +228,8 @@ __global__ void __launch_bounds__(THREADS)
         __half *gta = ta_out + (size_t)g * C * C;  // this chunk's Ta tile (row-major 64x64)
         const float beta_row = beta_next;
         beta_next = load_beta(g + gridDim.x);
+        const float2 gate_pair = gate_next;
+        gate_next = load_gate(g + gridDim.x);
         (void)bh;
         (void)c0;
         bool ok = tc::mbar_wait(&full, ph, WAIT_BUDGET);
@@ -211,6 +266,16 @@ __global__ void __launch_bounds__(THREADS)
             }
             al[r] = alpha_rule(sq, beta_row, euler);
         }
+        if (GATED && warp == 0) {  // l_t: inclusive scan of the row pairs' log-decays
+            float sc = gate_pair.x + gate_pair.y;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += y;
+            }
+            lg[2 * lane] = sc - gate_pair.y;
+            lg[2 * lane + 1] = sc;
+        }
         ok = tc::mbar_wait(&mma_bar, mma_phase, WAIT_BUDGET);
         if (__syncthreads_or(!ok)) { aborted = true; break; }  // also: every norm has been read
         mma_phase ^= 1;
@@ -228,6 +293,12 @@ __global__ void __launch_bounds__(THREADS)
                     const float ar = al[r];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * v[j] : 0.f;
+                    if constexpr (GATED) {  // Gam o G below the diagonal: e^{l_r - l_c} <= 1
+                        const float lr = lg[r];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (cb * 16 + j < r) v[j] *= expf(fminf(lr - lg[cb * 16 + j], 0.f));
+                    }
                     uint4 *dst = reinterpret_cast<uint4 *>(A16 + r * LD16 + cb * 16);
                     dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
                                         tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
@@ -363,16 +434,25 @@ __global__ void __launch_bounds__(THREADS)
 // MMA operands are fp16 (the bf16 Q, K, V tiles are converted in place; fp16
 // holds every bf16 value of magnitude >= 2^-14 exactly and rounds the
 // intermediates 8x finer than bf16); accumulation is fp32.
-template <int DK, int DV>
+//
+// Gated form: two more fp16 tiles per stage -- q as it is (P^T's B; the QW slabs then hold q
+// with its rows scaled by e^{l_t}) and k with its rows scaled by e^{l_t} (W's B) -- and the
+// masked P^T leaves the stage for two single tiles, its fp16 value and the fp16 remainder
+// (P^T = hi + lo to 22 bits; the side group writes a chunk's only after the previous D2 has
+// run, which the P^T product of the chunk waits for in the tensor pipe).
+template <int DK, int DV, bool GATED = false>
 struct StateLayout {
     static constexpr int QW_SLAB = 16384;                // per 64-column K slab: 64 Q rows, 64 -W rows
     static constexpr int QW = (DK / 64) * QW_SLAB;
-    static constexpr int KP = (DK / 64 + 1) * 8192;       // K slabs then the P^T block (MN-major)
+    static constexpr int KP = (DK / 64 + (GATED ? 0 : 1)) * 8192;  // K slabs then the P^T block (MN-major)
     static constexpr int VB = (DV / 64) * 8192;
     static constexpr int TB = C * C * 2;
+    static constexpr int XB = GATED ? (DK / 64) * 8192 : 0;  // gated: q, and k scaled by e^{l}
     static constexpr int OFF_QW = 0, OFF_KP = QW, OFF_V = QW + KP, OFF_T = QW + KP + VB;
-    static constexpr int STAGE = OFF_T + TB;
-    static constexpr int BYTES = 2 * STAGE;
+    static constexpr int OFF_QP = OFF_T + TB, OFF_KH = OFF_QP + XB;
+    static constexpr int STAGE = OFF_KH + XB;
+    static constexpr int OFF_PH = 2 * STAGE, OFF_PL = OFF_PH + 8192;  // gated: P^T hi and lo
+    static constexpr int BYTES = 2 * STAGE + (GATED ? 2 * 8192 : 0);
     static constexpr int SMEM = BYTES + 1024;             // alignment slack
 };
 
@@ -440,7 +520,9 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
 }
 
 // SEG = false compiles the one-pass form only (pass 0); SEG = true also takes the segment runs.
-template <int DK, int DV, typename TO, bool SEG, bool SAVE = false>
+// SAVE: the forward of the backward pass (every token's u and the state after every chunk
+// instead of o).  GATED: the gated form, with the decays in `gate` ([B,H,L]).
+template <int DK, int DV, typename TO, bool SEG, bool SAVE = false, bool GATED = false>
 __global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -448,8 +530,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
                     float *__restrict__ segbuf, int G, int seg_chunks, int pass,
-                    float *__restrict__ u_out, float *__restrict__ ck_out) {
-    using Lay = StateLayout<DK, DV>;
+                    float *__restrict__ u_out, float *__restrict__ ck_out,
+                    const __nv_bfloat16 *__restrict__ gate) {
+    static_assert(!(SAVE && GATED), "the saving forward is for the ungated form");
+    using Lay = StateLayout<DK, DV, GATED>;
     constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
@@ -457,6 +541,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     __shared__ StateBars bars;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
+    // gated: per stage, l_t and e^{l_C - l_t} of the chunk's tokens and e^{l_C} (written by the
+    // converter with the stage's tiles; readers wait for the stage's conversion first)
+    __shared__ float gfac[GATED ? 2 * 3 * C : 1];
+    auto gf = [&](int st, int which) { return gfac + (st * 3 + which) * C; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = warp >> 2, gtid = tid & 127;
@@ -525,8 +613,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         }
         tc::fence_async_smem();
     }
-    // ---- initial state (chain warpgroup): S^T, its fp16 copy and a zero O^T in TMEM
+    // ---- initial state (chain warpgroup): S^T, its fp16 copy and a zero O^T in TMEM (gated:
+    // the fp32 S^T already scaled by the first chunk's e^{l_C}, which D2 adds to)
+    const __nv_bfloat16 *grow = GATED ? gate + (size_t)bh * L : nullptr;  // this head's decays
     if (wg == 2) {
+        float gC0 = 1.f;
+        if constexpr (GATED) gC0 = expf(__shfl_sync(0xffffffffu, chunk_logdecay(grow, n0 * C, L, lane).y, 31));
 #pragma unroll
         for (int cb = 0; cb < DK / 32; ++cb) {
             float v[32];
@@ -536,7 +628,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                                  : ((s0p && vrow >= 0) ? s0p[(size_t)(cb * 32 + j) * DV + vrow] : 0.f);
             float lo[16], hi[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) { lo[j] = v[j]; hi[j] = v[16 + j]; }
+            for (int j = 0; j < 16; ++j) { lo[j] = v[j] * gC0; hi[j] = v[16 + j] * gC0; }
             tc::tmem_st16(tmem + lane_base + TM_S + cb * 32, lo);
             tc::tmem_st16(tmem + lane_base + TM_S + cb * 32 + 16, hi);
             uint32_t w[16];
@@ -600,6 +692,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);
             constexpr uint32_t id_d1 = tc::idesc_f16(DV, 128, false, false);
             constexpr uint32_t id_d2 = tc::idesc_f16(DV, DK + 64, false, true);
+            constexpr uint32_t id_d2s = tc::idesc_f16(DV, DK, false, true);  // gated: S^T += U''^T K
+            constexpr uint32_t id_d2o = tc::idesc_f16(DV, 64, false, true);  // gated: O^T += U'^T P^T
             auto stage_addr = [&](int n) { return sb + (n & 1) * Lay::STAGE; };
             // U'^T := V^T Ta^T (prefill of the U' accumulator)
             auto issue_u = [&](int n) {
@@ -610,23 +704,27 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                                  tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024), id_u, kk > 0);
                 tc::mma_commit(&bars.freeV[n & 1]);  // V and Ta of this stage are no longer read
             };
-            // W = Ta K (its own TMEM columns; the side group stores -W as a B operand)
+            // W = Ta K (its own TMEM columns; the side group stores -W as a B operand); gated:
+            // W = Ta diag(e^{l}) K, from the converter's scaled copy of K
             auto issue_w = [&](int n) {
                 const uint32_t stg = stage_addr(n);
+                const uint32_t kw = stg + (GATED ? Lay::OFF_KH : Lay::OFF_KP);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_W, tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024),
-                                 tc::sdesc(stg + Lay::OFF_KP + kk * 2048, 8192, 1024), id_w, kk > 0);
+                                 tc::sdesc(kw + kk * 2048, 8192, 1024), id_w, kk > 0);
                 tc::mma_commit(&bars.wdone);
             };
-            // P^T = K Q^T (its own TMEM columns; the side group stores the masked P^T)
+            // P^T = K Q^T (its own TMEM columns; the side group stores the masked P^T); gated:
+            // Q from the converter's unscaled copy (the QW slabs hold the scaled one)
             auto issue_p = [&](int n) {
                 const uint32_t stg = stage_addr(n);
-                const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
+                const uint32_t qb = stg + (GATED ? Lay::OFF_QP : Lay::OFF_QW), kp = stg + Lay::OFF_KP;
+                constexpr int QSTRIDE = GATED ? 8192 : Lay::QW_SLAB;
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
                     tc::mma_bf16(tmem + TM_P, tc::sdesc(kp + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(qb + (kk >> 2) * QSTRIDE + (kk & 3) * 32, 16, 1024),
                                  id_p, kk > 0);
                 tc::mma_commit(&bars.pdone);
             };
@@ -677,15 +775,46 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
                 if (!tc::mbar_wait_or_abort(&bars.up_ready_a, n & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
+                if constexpr (!GATED) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    if (kk == 2) {
-                        ok2 = tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget);
-                        if (!ok2) break;
-                        tc::tc_fence_after();
+                    for (int kk = 0; kk < 4; ++kk) {
+                        if (kk == 2) {
+                            ok2 = tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget);
+                            if (!ok2) break;
+                            tc::tc_fence_after();
+                        }
+                        tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
+                                       tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
                     }
-                    tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
-                                   tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
+                } else {
+                    // gated: O^T += U'^T P^T with both factors as fp16 hi + lo (the lo x lo term
+                    // dropped): U' hi over TM_U's first 32 columns, U' lo where P^T's accumulator
+                    // was; then S^T += U''^T K with U'' = diag(e^{l_C - l}) U' (TM_U's next 32)
+                    const uint32_t ph = sb + Lay::OFF_PH, pl = sb + Lay::OFF_PL;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        if (kk == 2) {
+                            ok2 = tc::mbar_wait_or_abort(&bars.up_ready, n & 1, &abort_flag, budget);
+                            if (!ok2) break;
+                            tc::tc_fence_after();
+                        }
+                        tc::mma_tmem_a(tmem + TM_O, tmem + TM_U + kk * 8, tc::sdesc(ph + kk * 2048, 8192, 1024),
+                                       id_d2o, 1u);
+                    }
+                    if (ok2) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_tmem_a(tmem + TM_O, tmem + TM_U + kk * 8, tc::sdesc(pl + kk * 2048, 8192, 1024),
+                                           id_d2o, 1u);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_tmem_a(tmem + TM_O, tmem + TM_P + kk * 8, tc::sdesc(ph + kk * 2048, 8192, 1024),
+                                           id_d2o, 1u);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + 32 + kk * 8,
+                                           tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2s, 1u);
+                    }
                 }
                 if (!ok2) break;
                 tc::mma_commit(&bars.d2done);
@@ -708,10 +837,22 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
             *t = u;
         };
+        // gated: also the unscaled fp16 q (P^T's B) and k scaled by e^{l_t} (W's B); the QW
+        // slabs get q scaled by e^{l_t} (D1's B), K's tile stays unscaled.  Row r of a tile's
+        // 64-column slab is its 16-byte pieces 8 r .. 8 r + 7 (the swizzle stays within a row).
+        auto cvt2 = [](const uint4 *src, uint4 *plain, uint4 *scaled, float f) {
+            const uint4 u = *src;
+            *plain = make_uint4(tc::bf16x2_to_f16x2(u.x), tc::bf16x2_to_f16x2(u.y),
+                                tc::bf16x2_to_f16x2(u.z), tc::bf16x2_to_f16x2(u.w));
+            *scaled = make_uint4(tc::bf16x2_to_f16x2_scaled(u.x, f), tc::bf16x2_to_f16x2_scaled(u.y, f),
+                                 tc::bf16x2_to_f16x2_scaled(u.z, f), tc::bf16x2_to_f16x2_scaled(u.w, f));
+        };
         for (int n = 0; n < cnt; ++n) {  // n: local chunk index
             const int st = n & 1;
             const uint32_t par = (n >> 1) & 1;
             uint8_t *stg = base + st * Lay::STAGE;
+            float2 lp = make_float2(0.f, 0.f);  // gated: l_t of this chunk's token pairs
+            if constexpr (GATED) lp = chunk_logdecay(grow, (n0 + n) * C, L, lane);
             if (!tc::mbar_wait_or_abort(&bars.fullV[st], par, &abort_flag, budget)) break;
             if (mode != 2) {
                 uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
@@ -722,14 +863,38 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < DK / 64; ++j) {  // Q: the first 8 KB of each QW slab
                 uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
+                if constexpr (GATED) {
+                    uint4 *tqp = reinterpret_cast<uint4 *>(stg + Lay::OFF_QP + j * 8192);
 #pragma unroll
-                for (int i = gtid; i < 512; i += 128) cvt(tq + i);
+                    for (int i = gtid; i < 512; i += 128)
+                        cvt2(tq + i, tqp + i, tq + i, expf(logdecay_at(lp, i >> 3)));
+                } else {
+#pragma unroll
+                    for (int i = gtid; i < 512; i += 128) cvt(tq + i);
+                }
             }
             if (!tc::mbar_wait_or_abort(&bars.fullK[st], par, &abort_flag, budget)) break;
             {
                 uint4 *tk = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
+                if constexpr (GATED) {
+                    uint4 *tkh = reinterpret_cast<uint4 *>(stg + Lay::OFF_KH);
 #pragma unroll
-                for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
+                    for (int i = gtid; i < (DK / 64) * 512; i += 128)
+                        cvt2(tk + i, tk + i, tkh + i, expf(logdecay_at(lp, (i >> 3) & 63)));
+                    // the stage's decay factors: its previous chunk's readers finished before
+                    // D2 of that chunk, which the K tile's reload waited for
+                    if (gtid < 32) {
+                        const float lC = __shfl_sync(0xffffffffu, lp.y, 31);
+                        gf(st, 0)[2 * lane] = lp.x;
+                        gf(st, 0)[2 * lane + 1] = lp.y;
+                        gf(st, 1)[2 * lane] = expf(lC - lp.x);
+                        gf(st, 1)[2 * lane + 1] = expf(lC - lp.y);
+                        if (lane == 0) gf(st, 2)[0] = expf(lC);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
+                }
             }
             tc::fence_async_smem();
             warp_arrive(&bars.conv[st], lane);
@@ -756,6 +921,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             warp_arrive(&bars.w_ready, lane);
 
             if (!tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget)) break;
+            // gated: the chunk's l_t (the converter wrote them with the stage's tiles)
+            if (GATED && !tc::mbar_wait_or_abort(&bars.conv[st], (n >> 1) & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {  // masked P^T (row c_in, column c_out >= c_in)
@@ -765,7 +932,18 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (cb * 32 + j < crow) v[j] = 0.f;
-                    store_row_f16x32(stg + Lay::OFF_KP + (DK / 64) * 8192, crow, cb * 4, v);
+                    if constexpr (GATED) {  // entry (c_in, c_out) weighted by e^{l_out - l_in} <= 1
+                        const float *lt = gf(st, 0);
+                        const float lin = lt[crow];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= expf(fminf(lt[cb * 32 + j] - lin, 0.f));
+                        store_row_f16x32(base + Lay::OFF_PH, crow, cb * 4, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] -= __half2float(__float2half_rn(v[j]));
+                        store_row_f16x32(base + Lay::OFF_PL, crow, cb * 4, v);
+                    } else {
+                        store_row_f16x32(stg + Lay::OFF_KP + (DK / 64) * 8192, crow, cb * 4, v);
+                    }
                 }
             }
             tc::fence_async_smem();
@@ -775,8 +953,20 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         // ---------------------------------------------------------- chain epilogue
         bool done_all = true;
         for (int n = 0; n < cnt; ++n) {  // n: local chunk index
+            // gated: the chunk's e^{l_C - l_t} (the converter wrote them with the stage's tiles)
+            if (GATED && !tc::mbar_wait_or_abort(&bars.conv[n & 1], (n >> 1) & 1, &abort_flag, budget)) {
+                done_all = false;
+                break;
+            }
             if (!tc::mbar_wait_or_abort(&bars.d1done, n & 1, &abort_flag, budget)) { done_all = false; break; }
+            // gated: U'^T's fp16 remainder goes where P^T's accumulator was, once the side group
+            // has read it out
+            if (GATED && !tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) {
+                done_all = false;
+                break;
+            }
             tc::tc_fence_after();
+            uint32_t wsc[16];  // gated: the first half's U'' = e^{l_C - l_t} U', until its columns are read
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // U'^T to fp16 in place, 32 tokens at a time
                 float u[32];
@@ -785,6 +975,25 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
                 tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, w);  // over fp32 columns already read
+                if constexpr (GATED) {
+                    // the output's U' as hi + lo (the remainder after fp16 rounding, to 22 bits)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        w[j] = tc::pack_f16(u[2 * j] - __half2float(__float2half_rn(u[2 * j])),
+                                            u[2 * j + 1] - __half2float(__float2half_rn(u[2 * j + 1])));
+                    tc::tmem_st16u(tmem + lane_base + TM_P + h * 16, w);
+                    // U''^T after both halves' fp32 columns [32, 64) are read
+                    const float *e = gf(n & 1, 1) + h * 32;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(u[2 * j] * e[2 * j], u[2 * j + 1] * e[2 * j + 1]);
+                    if (h == 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) wsc[j] = w[j];
+                    } else {
+                        tc::tmem_st16u(tmem + lane_base + TM_U + 32, wsc);
+                        tc::tmem_st16u(tmem + lane_base + TM_U + 48, w);
+                    }
+                }
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
                 if (SAVE && u_out && mode == 0 && vrow >= 0) {  // u_t = a_t r_t of every token, for the backward
                     const int t0 = (n0 + n) * C + h * 32;
@@ -797,17 +1006,49 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 
             if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
-#pragma unroll
-            for (int cb = 0; cb < DK / 64; ++cb) {  // S^T to fp16, 64 rows of S at a time
-                if (n + 1 < cnt) {
-                    float v[64];
-                    tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
-                    uint32_t w[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
-                    tc::tmem_st32u(tmem + lane_base + TM_S16 + cb * 32, w);
+            float gCn = 1.f;  // gated: the next chunk's e^{l_C}, applied to the fp32 state for its D2
+            if (GATED && n + 1 < cnt) {
+                if (!tc::mbar_wait_or_abort(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, budget)) {
+                    done_all = false;
+                    break;
                 }
-                if (cb == 0) warp_arrive(&bars.s_ready_a, lane);
+                gCn = gf((n + 1) & 1, 2)[0];
+            }
+            if constexpr (!GATED) {
+#pragma unroll
+                for (int cb = 0; cb < DK / 64; ++cb) {  // S^T to fp16, 64 rows of S at a time
+                    if (n + 1 < cnt) {
+                        float v[64];
+                        tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
+                        uint32_t w[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+                        tc::tmem_st32u(tmem + lane_base + TM_S16 + cb * 32, w);
+                    }
+                    if (cb == 0) warp_arrive(&bars.s_ready_a, lane);
+                }
+            } else {
+                // 32 rows of S at a time: the fp16 copy of S for D1, then the fp32 S scaled by
+                // the next chunk's decay for its D2
+#pragma unroll
+                for (int p = 0; p < DK / 32; ++p) {
+                    if (n + 1 < cnt) {
+                        float v[32];
+                        tc::tmem_ld32(tmem + lane_base + TM_S + p * 32, v);
+                        uint32_t w[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+                        tc::tmem_st16u(tmem + lane_base + TM_S16 + p * 16, w);
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float x[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) x[j] = v[16 * h2 + j] * gCn;
+                            tc::tmem_st16(tmem + lane_base + TM_S + p * 32 + 16 * h2, x);
+                        }
+                    }
+                    if (p == 1) warp_arrive(&bars.s_ready_a, lane);
+                }
             }
             warp_arrive(&bars.s_ready, lane);
             if (SAVE && ck_out && mode == 0) {
@@ -867,957 +1108,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-// ------------------------------------------------------------------ gated form: cluster kernel
-namespace pair {
-// Each run -- a head, or a segment run of a head -- is a cluster of two CTAs:
-//   rank 0, the state CTA: the serial chunk chain.  Its tensor pipe carries the chain's
-//       products (the U' prefill, D1 and D2) and P^T = K Q^T; the fp32 state S^T stays in
-//       its tensor memory; its epilogue warps turn U'^T and S^T into the fp16 A operands
-//       of the next products, mask P^T into an operand tile and write the outputs.
-//   rank 1, the producer CTA: per chunk, the Gram K K^T on its own tensor core, the
-//       triangular solve for Ta = T diag(a) (three solve warpgroups take chunks in turn,
-//       so three solves are in flight), then W = Ta K; Ta and -W go to the state CTA's
-//       stage buffers by bulk copies within the cluster.  Nothing in it depends on the
-//       previous chunk, so it runs up to four chunks ahead of the chain.
-// Hand-offs are mbarriers: within a CTA as usual; across the cluster, the producer
-// announces each chunk's copies on the state CTA's barrier (remote arrive with the
-// expected bytes, then the copies' completion), and the state CTA's D1 commit arrives
-// on the producer's barrier when a stage's Ta and -W slots may be overwritten.
-// Warps of the state CTA:
-//   warps 0-3   converter: bf16 -> fp16 in place for the Q, K, V tiles of a stage
-//   warps 4-7   chain:     U'^T and the new state from TMEM into the A operands (TMEM)
-//   warps 8-11  output:    O^T from TMEM to global memory, then zero it for the next chunk
-//   warps 12-15 side:      P^T from TMEM, masked, into its operand tile
-//   warp 16     MMA issuer (one thread), warp 17 TMA producer (one thread)
-// Warps of the producer CTA:
-//   warps 0-3, 8-11, 12-15  solve groups 0, 1, 2 (chunk i goes to group i % 3)
-//   warps 4-7   epilogue:  -W from TMEM into a staging tile; one thread copies Ta and -W
-//   warp 16     MMA issuer (one thread), warp 17 TMA producer (one thread)
-constexpr int PR_WARPS = 18;
-constexpr int PR_THREADS = PR_WARPS * 32;
-constexpr int W_ISSUE = 16, W_PROD = 17;
-constexpr int NSLOT = 4;  // producer: K and Ta slots, chunk i in slot i % NSLOT
-constexpr int NGRP = 3;   // producer: solve groups, chunk i in group i % NGRP
-constexpr int WLAG = 2;   // producer issuer: W of chunk i is issued after the Gram of chunk i + WLAG
-
-template <int DK, int DV>
-struct PairLayout {
-    using S = StateLayout<DK, DV>;
-    // producer: NSLOT K tiles (DK/64 slabs of 64 rows x 128 bytes), NSLOT Ta tiles, two
-    // staged -W tiles, then one triangular-solve scratch region per solve group: A (fp16),
-    // T's diagonal blocks (fp16), A's fp32 diagonal blocks (later the merges' transposed R),
-    // T transposed (fp16) and a
-    static constexpr int KT = DK * 128;
-    static constexpr int P_K = 0, P_T = P_K + NSLOT * KT, P_W = P_T + NSLOT * C * C * 2,
-                         P_SOLVE = P_W + 2 * DK * 128;
-    static constexpr int S_A16 = 0, S_TD16 = C * prep::LD16 * 2, S_AD = S_TD16 + 4 * 16 * 24 * 2,
-                         S_T16T = S_AD + C * 16 * 4, S_AL = S_T16T + C * prep::LD16 * 2,
-                         SOLVE_BYTES = S_AL + C * 4, SOLVE_STRIDE = (SOLVE_BYTES + 1023) / 1024 * 1024;
-    static constexpr int P_BYTES = P_SOLVE + NGRP * SOLVE_STRIDE, S_BYTES = 2 * S::STAGE;
-    static constexpr int SMEM = (S_BYTES > P_BYTES ? S_BYTES : P_BYTES) + 1024;  // + alignment slack
-};
-
-// Barriers of both roles (each CTA initialises all of them and uses its own subset; the
-// cross-CTA ones sit at the same offset in both CTAs).
-struct PairBars {
-    // state CTA: its own loads and their release
-    uint64_t fullV[2], fullQ[2], fullK[2], freeV[2], freeQ[2], freeK[2];
-    // state CTA: the producer's Ta and -W of a stage have landed
-    uint64_t recvW[2];
-    uint64_t d1done, d2done, pdone, drain;
-    // producer CTA: K slots loaded / free, Gram done per solve group, W done per TMEM buffer
-    uint64_t kfull[NSLOT], kfree[NSLOT], gdone[NGRP], wdone[2];
-    // producer CTA: the state CTA has finished chunk i (its D1 read that chunk's Ta and -W),
-    // counted per slot i % NSLOT: one remote arrival per chunk
-    uint64_t sfree[NSLOT];
-    uint64_t pdrain;
-    // four arrivals (one per warp) from here on
-    uint64_t conv[2], up_ready_a, up_ready, s_ready_a, s_ready, o_free, p_ready;  // state CTA
-    uint64_t gread[NGRP], tready[NSLOT], wst[2];                                 // producer CTA
-};
-constexpr int PBARS_ONE = 21 + 3 * NSLOT + NGRP;  // barriers before `conv` take a single arrival
-static_assert(sizeof(PairBars) / sizeof(uint64_t) == PBARS_ONE + 8 + NGRP + NSLOT + 2, "barrier count");
-
-// Gated form (a per-token decay g_t on the carried state; Gated DeltaNet's gate placement):
-// within a chunk entered with state S, with l_t the cumulative log-decay from the chunk
-// start to token t (l_C at its last token) and Gam_ts = e^{l_t - l_s}, the chunk algebra is
-//   A  = strictly-lower(diag(a) (Gam o K K^T)),  W = T diag(a) diag(e^{l}) K,  U' = U - W S,
-//   O  = diag(e^{l}) Q S + (lower-incl(Gam) o Q K^T) U',
-//   S <- e^{l_C} S + K^T diag(e^{l_C - l}) U'.
-// On the tensor cores every factor applied is at most 1 (only the products e^{l_t - l_s},
-// s <= t, are bounded; a split into e^{l_t - l_C} e^{l_C - l_s} would over- and underflow
-// fp16): the producer scales K's rows by e^{l_t} when it converts K for W and weights the
-// Gram by Gam; the state CTA keeps Q S and the intra-chunk output in separate accumulators
-// and scales the first by e^{l_t} on output, weights P^T by Gam, then scales K's rows by
-// e^{l_C - l_t} for D2's state update once P^T has read K, and scales the fp32 state by
-// e^{l_C} before D2 adds to it.
-//
-// l_t of a chunk's tokens 2 lane and 2 lane + 1, for every lane of a warp (0 past the sequence
-// end, where the decay is taken as 1): a warp-wide inclusive scan of the pairs' logarithms.
-__device__ __forceinline__ float2 chunk_logdecay(const __nv_bfloat16 *gate_row, int t0, int L, int lane) {
-    const int t = t0 + 2 * lane;
-    const float x0 = t < L ? logf(__bfloat162float(gate_row[t])) : 0.f;
-    const float x1 = t + 1 < L ? logf(__bfloat162float(gate_row[t + 1])) : 0.f;
-    float s = x0 + x1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, s, o);
-        if (lane >= o) s += y;
-    }
-    return make_float2(s - x1, s);
-}
-// Element t of a per-token quantity held as pairs (lane t / 2 holds tokens 2 lane, 2 lane + 1),
-// e.g. l_t itself or a factor made from it (every lane of the warp takes part; t need not be
-// uniform).
-__device__ __forceinline__ float logdecay_at(float2 p, int t) {
-    const float a = __shfl_sync(0xffffffffu, p.x, t >> 1), b = __shfl_sync(0xffffffffu, p.y, t >> 1);
-    return (t & 1) ? b : a;
-}
-
-// SEG = false compiles the one-pass form only (pass 0); SEG = true also takes the segment runs.
-// SAVE: the forward of the backward pass (every token's u and the state after every chunk
-// instead of o).  GATED: the gated form, with the decays in `gate` ([B,H,L]).
-template <int DK, int DV, typename TO, bool SEG, bool SAVE = false, bool GATED = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
-    tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                   const __grid_constant__ CUtensorMap tmap_k,
-                   const __grid_constant__ CUtensorMap tmap_v,
-                   const __nv_bfloat16 *__restrict__ beta, bool euler, const float *__restrict__ S0,
-                   TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
-                   float *__restrict__ segbuf, int G, int seg_chunks, int pass,
-                   float *__restrict__ u_out, float *__restrict__ ck_out,
-                   const __nv_bfloat16 *__restrict__ gate) {
-    static_assert(!(SAVE && GATED), "the saving forward is for the ungated form");
-    using Lay = StateLayout<DK, DV>;
-    using PL = PairLayout<DK, DV>;
-    // state CTA (fp32 columns): S^T, then O^T that D2 adds to, then O^T that D1 adds to (the
-    // same accumulator without a gate, a separate one with it), then U'^T; D2 writes
-    // [S^T | O^T] and D1 [O^T | U'^T], each contiguous; P^T after them
-    constexpr uint32_t TM_S = 0, TM_O = DK, TM_OI = GATED ? DK + 64 : DK, TM_U = TM_OI + 64;
-    constexpr uint32_t TM_P = GATED ? 320 : 256;
-    static_assert(TM_U + 64 <= TM_P && TM_P + 64 <= TM_S16, "state CTA tensor memory layout");
-    // producer CTA: the Gram of each solve group (64 columns each), W in two buffers
-    constexpr uint32_t TP_G = 0, TP_W = 256;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_u32 = tc::smem_u32(smem_raw);
-    uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    __shared__ PairBars bars;
-    __shared__ uint32_t tmem_base;
-    __shared__ volatile int abort_flag;
-
-    const uint32_t rank = tc::cluster_rank();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = warp >> 2, gtid = tid & 127;
-    // ---- the run this cluster makes: head bh, chunks [n0, n1), and what it starts from and keeps.
-    // pass 0: the whole sequence.  With the sequence cut into G segments of seg_chunks chunks
-    // (each segment maps the state affinely, S_out = P S_in + H), pass 1 runs segment 0 from
-    // S0 and, for every middle segment g, H_g (from zero) and P_g (the transition: from the
-    // identity with v = 0), with no output; pass 2 runs segments 1..G-1 from their true
-    // starting states, which the combine kernel chains together in between.
-    const int run = blockIdx.x >> 1;
-    int bh = run, n0 = 0, n1 = NC, mode = 0;  // mode 0: outputs, 1: H run, 2: P run
-    const size_t DD = (size_t)DK * DV;
-    const float *s0p = S0 ? S0 + (size_t)bh * DD : nullptr;
-    float *sfp = S_final ? S_final + (size_t)bh * DD : nullptr;
-    if (!SEG) pass = 0;
-    if (pass == 1) {
-        const int R = 2 * G - 3, r = run % R, g = (r + 1) / 2;
-        bh = run / R;
-        n0 = g * seg_chunks;
-        n1 = min(NC, n0 + seg_chunks);
-        float *seg = segbuf + ((size_t)bh * G + g) * 3 * DD;  // [S_in | H | P] of segment g
-        if (r == 0) {
-            s0p = S0 ? S0 + (size_t)bh * DD : nullptr;
-            sfp = segbuf + ((size_t)bh * G + 1) * 3 * DD;  // S_in of segment 1
-        } else {
-            mode = (r & 1) ? 1 : 2;
-            s0p = nullptr;
-            sfp = seg + (size_t)mode * DD;
-        }
-    } else if (pass == 2) {
-        const int R = G - 1, g = 1 + run % R;
-        bh = run / R;
-        n0 = g * seg_chunks;
-        n1 = min(NC, n0 + seg_chunks);
-        s0p = segbuf + ((size_t)bh * G + g) * 3 * DD;
-        sfp = (g == G - 1 && S_final) ? S_final + (size_t)bh * DD : nullptr;
-    }
-    if (!SEG) mode = 0;
-    const int cnt = n1 - n0;  // chunks of this run; stage and barrier phases follow the local index
-    const __nv_bfloat16 *grow = GATED ? gate + (size_t)bh * L : nullptr;  // this head's decays
-    if (tid == 0) {
-        uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
-        for (int i = 0; i < (int)(sizeof(PairBars) / sizeof(uint64_t)); ++i)
-            tc::mbar_init(b + i, i < PBARS_ONE ? 1 : 4);
-        tc::fence_mbar_init();
-        abort_flag = 0;
-        tc::tma_prefetch_desc(&tmap_q);
-        tc::tma_prefetch_desc(&tmap_k);
-        if (rank == 0) tc::tma_prefetch_desc(&tmap_v);
-    }
-    if (warp == 0) {
-        tc::tmem_alloc(&tmem_base, 512);
-        tc::tmem_relinquish();
-    }
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t sb = tc::smem_u32(base);
-    const long long budget = WAIT_BUDGET;
-    // A wait that fails (bound run out, or an abort flagged) also flags the other CTA of the
-    // cluster, whose waits then end too.
-    const uint32_t peer_abort = tc::mapa(tc::smem_u32((const void *)&abort_flag), rank ^ 1u);
-    auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
-        if (tc::mbar_wait_or_abort(bar, parity, &abort_flag, budget)) return true;
-        tc::st_cluster_u32(peer_abort, 1u);
-        return false;
-    };
-    // The same for a whole warp: every lane waits and the warp takes one decision, so a
-    // warp never splits before a warp-collective TMEM access or a warp barrier.
-    auto wait_warp = [&](uint64_t *bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, wait(bar, parity)) != 0;
-    };
-
-    if (rank == 0) {
-        const int vrow = acc_row<DV>(warp & 3, lane);  // state column v of this thread's TMEM lane
-        // ---- a P run reads no values: its V tiles stay zero
-        if (mode == 2) {
-            for (int i = tid; i < 2 * Lay::VB / 16; i += PR_THREADS) {
-                const int stg = i / (Lay::VB / 16), w = i - stg * (Lay::VB / 16);
-                reinterpret_cast<uint4 *>(base + stg * Lay::STAGE + Lay::OFF_V)[w] = make_uint4(0u, 0u, 0u, 0u);
-            }
-            tc::fence_async_smem();
-        }
-        // ---- initial state (chain warpgroup): S^T, its fp16 copy and a zero O^T in TMEM (gated:
-        // the fp32 state scaled by the first chunk's total decay, which D2 adds to)
-        if (wg == 1) {
-            float gC0 = 1.f;
-            if constexpr (GATED) gC0 = expf(__shfl_sync(0xffffffffu, chunk_logdecay(grow, n0 * C, L, lane).y, 31));
-#pragma unroll
-            for (int cb = 0; cb < DK / 32; ++cb) {
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    v[j] = mode == 2 ? (cb * 32 + j == vrow ? 1.f : 0.f)
-                                     : ((s0p && vrow >= 0) ? s0p[(size_t)(cb * 32 + j) * DV + vrow] : 0.f);
-                float lo[16], hi[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) { lo[j] = gC0 * v[j]; hi[j] = gC0 * v[16 + j]; }
-                tc::tmem_st16(tmem + lane_base + TM_S + cb * 32, lo);
-                tc::tmem_st16(tmem + lane_base + TM_S + cb * 32 + 16, hi);
-                uint32_t w[16];
-                pack32_f16(v, w);
-                tc::tmem_st16u(tmem + lane_base + TM_S16 + cb * 16, w);
-            }
-            float z[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) z[j] = 0.f;
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
-            if constexpr (GATED) {
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_OI + cb * 16, z);
-            }
-            tc::tc_fence_before();
-        }
-    }
-    __syncthreads();
-    tc::tc_fence_after();
-    tc::cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
-
-    if (rank == 0) {
-        const int vrow = acc_row<DV>(warp & 3, lane);
-        if (warp == W_PROD) {
-            // ------------------------------------------------------ TMA producer (state)
-            if (lane == 0) {
-                int last[2] = {-1, -1};
-                for (int i = 0; i < cnt; ++i) {
-                    const int n = n0 + i, st = i & 1;
-                    const uint32_t par = ((i - 2) >> 1) & 1;
-                    uint8_t *stg = base + st * Lay::STAGE;
-                    if (i >= 2 && !wait(&bars.freeV[st], par)) break;
-                    tc::mbar_expect_tx(&bars.fullV[st], mode == 2 ? 0 : Lay::VB);
-                    if (mode != 2) {
-#pragma unroll
-                        for (int j = 0; j < DV / 64; ++j)
-                            tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
-                    }
-                    if (i >= 2 && !wait(&bars.freeQ[st], par)) break;
-                    tc::mbar_expect_tx(&bars.fullQ[st], DK * 128);
-#pragma unroll
-                    for (int j = 0; j < DK / 64; ++j)
-                        tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
-                    if (i >= 2 && !wait(&bars.freeK[st], par)) break;
-                    tc::mbar_expect_tx(&bars.fullK[st], DK * 128);
-#pragma unroll
-                    for (int j = 0; j < DK / 64; ++j)
-                        tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, &bars.fullK[st], j * 64, n * C, bh);
-                    last[st] = i;
-                }
-                if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
-                    for (int st = 0; st < 2; ++st) {
-                        if (last[st] < 0) continue;
-                        const uint32_t par = (last[st] >> 1) & 1;
-                        tc::mbar_wait(&bars.fullV[st], par, budget / 8);
-                        tc::mbar_wait(&bars.fullQ[st], par, budget / 8);
-                        tc::mbar_wait(&bars.fullK[st], par, budget / 8);
-                    }
-                }
-            }
-        } else if (warp == W_ISSUE) {
-            // ------------------------------------------------------ MMA issuer (state)
-            if (lane == 0) {
-                constexpr uint32_t id_u = tc::idesc_f16(DV, 64, true, false);
-                constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);
-                constexpr uint32_t id_d1 = tc::idesc_f16(DV, 128, false, false);
-                constexpr uint32_t id_d2 = tc::idesc_f16(DV, DK + 64, false, true);
-                auto stage_addr = [&](int n) { return sb + (n & 1) * Lay::STAGE; };
-                // U'^T := V^T Ta^T (prefill of the U' accumulator)
-                auto issue_u = [&](int n) {
-                    const uint32_t stg = stage_addr(n);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(tmem + TM_U, tc::sdesc(stg + Lay::OFF_V + kk * 2048, 8192, 1024),
-                                     tc::sdesc(stg + Lay::OFF_T + kk * 32, 16, 1024), id_u, kk > 0);
-                    tc::mma_commit(&bars.freeV[n & 1]);  // V and Ta of this stage are no longer read
-                };
-                // P^T = K Q^T (its own TMEM columns; the side group stores the masked P^T)
-                auto issue_p = [&](int n) {
-                    const uint32_t stg = stage_addr(n);
-                    const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        tc::mma_bf16(tmem + TM_P, tc::sdesc(kp + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                                     tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
-                                     id_p, kk > 0);
-                    tc::mma_commit(&bars.pdone);
-                };
-                // Tensor-pipe order per chunk: D1(n), P^T(n+1), D2(n), U'^T prefill(n+1): P^T runs
-                // while the chain epilogue packs U', the prefill while it packs the new state.
-                // A prefill waits for the stage's converted V and for the producer's Ta and -W.
-                bool issued_any = false;
-                bool ok = wait(&bars.conv[0], 0) && wait(&bars.recvW[0], 0);
-                if (ok) {
-                    tc::tc_fence_after();
-                    issued_any = true;
-                    issue_u(0);
-                    issue_p(0);
-                }
-                for (int n = 0; ok && n < cnt; ++n) {  // n: local chunk index
-                    const int st = n & 1;
-                    const uint32_t stg = stage_addr(n);
-                    const uint32_t qw = stg + Lay::OFF_QW, kp = stg + Lay::OFF_KP;
-                    // D1: [O^T | U'^T] += S^T [Q | -W]^T   (A = fp16 S^T in TMEM; -W from the producer)
-                    // the first 64 rows of S^T are packed before the rest: start on them
-                    if (n > 0 && !wait(&bars.o_free, (n - 1) & 1)) break;
-                    if (n > 0 && !wait(&bars.s_ready_a, (n - 1) & 1)) break;
-                    tc::tc_fence_after();
-                    bool ok2 = true;
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        if (kk == 4 && n > 0) {
-                            ok2 = wait(&bars.s_ready, (n - 1) & 1);
-                            if (!ok2) break;
-                            tc::tc_fence_after();
-                        }
-                        tc::mma_tmem_a(tmem + TM_OI, tmem + TM_S16 + kk * 8,
-                                       tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
-                                       id_d1, 1u);
-                    }
-                    if (!ok2) break;
-                    tc::mma_commit(&bars.d1done);
-                    tc::mma_commit(&bars.freeQ[st]);
-                    // P^T(n) has been read out of TMEM and stored (D2(n) reads it); P^T of the next
-                    // chunk goes here if that chunk's tiles are converted already, else after D2(n)
-                    if (!wait(&bars.p_ready, n & 1)) break;
-                    bool p_next = false;
-                    if (n + 1 < cnt && tc::mbar_try_wait(&bars.conv[(n + 1) & 1], ((n + 1) >> 1) & 1)) {
-                        tc::tc_fence_after();
-                        issue_p(n + 1);
-                        p_next = true;
-                    }
-                    // D2: [S^T | O^T] += U'^T [K | P^T]   (A = fp16 U'^T in TMEM)
-                    // U' is packed in two halves of 32 tokens: start on the first
-                    if (!wait(&bars.up_ready_a, n & 1)) break;
-                    tc::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        if (kk == 2) {
-                            ok2 = wait(&bars.up_ready, n & 1);
-                            if (!ok2) break;
-                            tc::tc_fence_after();
-                        }
-                        tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
-                                       tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
-                    }
-                    if (!ok2) break;
-                    tc::mma_commit(&bars.d2done);
-                    tc::mma_commit(&bars.freeK[st]);
-                    if (n + 1 < cnt) {  // P^T (unless issued above) and the U' prefill of the next chunk
-                        const uint32_t pn = ((n + 1) >> 1) & 1;
-                        if (!wait(&bars.conv[(n + 1) & 1], pn)) break;
-                        if (!wait(&bars.recvW[(n + 1) & 1], pn)) break;
-                        tc::tc_fence_after();
-                        if (!p_next) issue_p(n + 1);
-                        issue_u(n + 1);
-                    }
-                }
-                if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
-                    tc::mma_commit(&bars.drain);
-                    tc::mbar_wait(&bars.drain, 0, budget / 4);
-                }
-            }
-        } else if (wg == 0) {
-            // ------------------------------------------------------ converter (state)
-            auto cvt = [](uint4 *t) {
-                uint4 u = *t;
-                u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
-                u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-                *t = u;
-            };
-            for (int n = 0; n < cnt; ++n) {  // n: local chunk index
-                const int st = n & 1;
-                const uint32_t par = (n >> 1) & 1;
-                uint8_t *stg = base + st * Lay::STAGE;
-                if (!wait_warp(&bars.fullV[st], par)) break;
-                if (mode != 2) {
-                    uint4 *tv = reinterpret_cast<uint4 *>(stg + Lay::OFF_V);
-#pragma unroll
-                    for (int i = gtid; i < Lay::VB / 16; i += 128) cvt(tv + i);
-                }
-                if (!wait_warp(&bars.fullQ[st], par)) break;
-#pragma unroll
-                for (int j = 0; j < DK / 64; ++j) {  // Q: the first 8 KB of each QW slab
-                    uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
-#pragma unroll
-                    for (int i = gtid; i < 512; i += 128) cvt(tq + i);
-                }
-                if (!wait_warp(&bars.fullK[st], par)) break;
-                {
-                    uint4 *tk = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
-#pragma unroll
-                    for (int i = gtid; i < (DK / 64) * 512; i += 128) cvt(tk + i);
-                }
-                tc::fence_async_smem();
-                warp_arrive(&bars.conv[st], lane);
-            }
-        } else if (wg == 1) {
-            // ------------------------------------------------------ chain epilogue
-            bool done_all = true;
-            float2 lp = make_float2(0.f, 0.f);  // gated: l_t of this chunk's token pairs
-            if constexpr (GATED) lp = chunk_logdecay(grow, n0 * C, L, lane);
-            for (int n = 0; n < cnt; ++n) {  // n: local chunk index
-                if (!wait_warp(&bars.d1done, n & 1)) { done_all = false; break; }
-                tc::tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {  // U'^T to fp16 in place, 32 tokens at a time
-                    float u[32];
-                    tc::tmem_ld32(tmem + lane_base + TM_U + h * 32, u);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
-                    tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, w);  // over fp32 columns already read
-                    warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
-                    if (SAVE && u_out && mode == 0 && vrow >= 0) {  // u_t = a_t r_t of every token, for the backward
-                        const int t0 = (n0 + n) * C + h * 32;
-                        float *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (t0 + j < L) dst[(size_t)j * DV] = u[j];
-                    }
-                }
-
-                float gCn = 1.f;  // gated: the next chunk's total decay, applied to the fp32 state
-                if constexpr (GATED) {
-                    if (n + 1 < cnt) {
-                        lp = chunk_logdecay(grow, (n0 + n + 1) * C, L, lane);
-                        gCn = expf(__shfl_sync(0xffffffffu, lp.y, 31));
-                    }
-                }
-                if (!wait_warp(&bars.d2done, n & 1)) { done_all = false; break; }
-                tc::tc_fence_after();
-#pragma unroll
-                for (int cb = 0; cb < DK / 64; ++cb) {  // S^T to fp16, 64 rows of S at a time
-                    if (n + 1 < cnt) {
-                        if constexpr (GATED) {  // 32 rows at a time; D2 of the next chunk adds to e^{l_C} S
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                float v[32];
-                                tc::tmem_ld32(tmem + lane_base + TM_S + cb * 64 + hh * 32, v);
-                                uint32_t w[16];
-                                pack32_f16(v, w);
-                                tc::tmem_st16u(tmem + lane_base + TM_S16 + cb * 32 + hh * 16, w);
-#pragma unroll
-                                for (int q = 0; q < 2; ++q) {
-                                    float x[16];
-#pragma unroll
-                                    for (int j = 0; j < 16; ++j) x[j] = gCn * v[16 * q + j];
-                                    tc::tmem_st16(tmem + lane_base + TM_S + cb * 64 + hh * 32 + 16 * q, x);
-                                }
-                            }
-                        } else {
-                            float v[64];
-                            tc::tmem_ld64(tmem + lane_base + TM_S + cb * 64, v);
-                            uint32_t w[32];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
-                            tc::tmem_st32u(tmem + lane_base + TM_S16 + cb * 32, w);
-                        }
-                    }
-                    if (cb == 0) warp_arrive(&bars.s_ready_a, lane);
-                }
-                warp_arrive(&bars.s_ready, lane);
-                if (SAVE && ck_out && mode == 0) {
-                    // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
-                    // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
-                    // warp-collective: every lane takes it, the lanes that hold a state column store.
-                    float *dst = ck_out + ((size_t)bh * NC + n0 + n) * DD + (vrow >= 0 ? vrow : 0);
-#pragma unroll 1
-                    for (int cb = 0; cb < DK / 16; ++cb) {
-                        float v[16];
-                        tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
-                        if (vrow >= 0) {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) dst[(size_t)(cb * 16 + j) * DV] = v[j];
-                        }
-                    }
-                }
-            }
-            if (done_all && sfp) {
-#pragma unroll
-                for (int cb = 0; cb < DK / 16; ++cb) {
-                    float v[16];
-                    tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
-                    if (vrow >= 0) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            sfp[(size_t)(cb * 16 + j) * DV + vrow] = v[j];
-                    }
-                }
-            }
-        } else if (wg == 2) {
-            // ------------------------------------------------------ output
-            float z[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) z[j] = 0.f;
-            for (int n = 0; n < cnt; ++n) {  // n: local chunk index
-                const int c0 = (n0 + n) * C;
-                if (!wait_warp(&bars.d2done, n & 1)) break;
-                tc::tc_fence_after();
-                const int cl = min(C, L - c0);
-                if constexpr (GATED) {  // o_t = e^{l_t} (S^T q_t) + intra-chunk part, 32 tokens at a time
-                    const float2 lp = chunk_logdecay(grow, c0, L, lane);
-                    const float2 fp = make_float2(expf(lp.x), expf(lp.y));
-                    TO *dst = o + ((size_t)bh * L + c0) * DV + (vrow >= 0 ? vrow : 0);
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float v[32], vi[32];
-                        tc::tmem_ld32(tmem + lane_base + TM_O + hh * 32, v);
-                        tc::tmem_ld32(tmem + lane_base + TM_OI + hh * 32, vi);
-#pragma unroll
-                        for (int cb = 0; cb < 2; ++cb) {
-                            tc::tmem_st16(tmem + lane_base + TM_O + hh * 32 + cb * 16, z);
-                            tc::tmem_st16(tmem + lane_base + TM_OI + hh * 32 + cb * 16, z);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = fmaf(logdecay_at(fp, hh * 32 + j), vi[j], v[j]);
-                        if (hh == 1) warp_arrive(&bars.o_free, lane);  // both O accumulators are zero again
-                        if (mode == 0 && vrow >= 0) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (hh * 32 + j < cl) dst[(size_t)(hh * 32 + j) * DV] = from_f32<TO>(v[j]);
-                        }
-                    }
-                } else {
-                    float v[64];
-                    tc::tmem_ld64(tmem + lane_base + TM_O, v);
-#pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(tmem + lane_base + TM_O + cb * 16, z);
-                    warp_arrive(&bars.o_free, lane);  // TMEM O is zero again: D1(n+1) may run
-                    if (mode == 0 && vrow >= 0 && (!SAVE || o)) {  // the saving forward writes no o
-                        TO *dst = o + ((size_t)bh * L + c0) * DV + vrow;
-#pragma unroll
-                        for (int j = 0; j < 64; ++j)
-                            if (j < cl) dst[(size_t)j * DV] = from_f32<TO>(v[j]);
-                    }
-                }
-                // chunk n is done here: tell the producer, which reuses its slots (a remote
-                // arrive takes a while, so it is made here, off the chain)
-                if (gtid == 0) tc::mbar_arrive_remote(tc::mapa(tc::smem_u32(&bars.sfree[n % NSLOT]), 1));
-            }
-        } else if (wg == 3) {
-            // ------------------------------------------------------ side epilogue (state)
-            const int crow = acc_row<64>(warp & 3, lane);  // token row of the M = 64 accumulator
-            for (int n = 0; n < cnt; ++n) {  // n: local chunk index
-                uint8_t *stg = base + (n & 1) * Lay::STAGE;
-                float2 lp = make_float2(0.f, 0.f);
-                if constexpr (GATED) lp = chunk_logdecay(grow, (n0 + n) * C, L, lane);
-                if (!wait_warp(&bars.pdone, n & 1)) break;
-                tc::tc_fence_after();
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {  // masked P^T (row c_in, column c_out >= c_in)
-                    float v[32];
-                    tc::tmem_ld32(tmem + lane_base + TM_P + cb * 32, v);
-                    if constexpr (GATED) {  // gated: entry (c_in, c_out) scaled by e^{l_out - l_in} (<= 1 where kept)
-                        const float lin = logdecay_at(lp, crow < 0 ? 0 : crow);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] *= expf(fminf(logdecay_at(lp, cb * 32 + j) - lin, 0.f));
-                    }
-                    if (crow >= 0) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (cb * 32 + j < crow) v[j] = 0.f;
-                        store_row_f16x32(stg + Lay::OFF_KP + (DK / 64) * 8192, crow, cb * 4, v);
-                    }
-                }
-                if constexpr (GATED) {
-                    // P^T has read K: scale its rows by e^{l_C - l_t} <= 1 for D2's state update,
-                    // S += K^T diag(e^{l_C - l}) U' (this thread's elements e = gtid + 128 m are rows
-                    // (gtid >> 3) + 16 m of a slab)
-                    const float lC = __shfl_sync(0xffffffffu, lp.y, 31);
-                    float f[4];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) f[m] = expf(lC - logdecay_at(lp, (gtid >> 3) + 16 * m));
-                    uint4 *t = reinterpret_cast<uint4 *>(stg + Lay::OFF_KP);
-#pragma unroll
-                    for (int e = gtid, m = 0; e < (DK / 64) * 512; e += 128, m = (m + 1) & 3) {
-                        uint4 u = t[e];
-                        u.x = tc::f16x2_scale(u.x, f[m]); u.y = tc::f16x2_scale(u.y, f[m]);
-                        u.z = tc::f16x2_scale(u.z, f[m]); u.w = tc::f16x2_scale(u.w, f[m]);
-                        t[e] = u;
-                    }
-                }
-                tc::fence_async_smem();
-                warp_arrive(&bars.p_ready, lane);
-            }
-        }
-    } else {
-        if (warp == W_PROD) {
-            // ------------------------------------------------------ TMA producer (producer CTA)
-            if (lane == 0) {
-                int last[NSLOT];
-                for (int s = 0; s < NSLOT; ++s) last[s] = -1;
-                for (int i = 0; i < cnt; ++i) {
-                    const int n = n0 + i, s = i % NSLOT;
-                    if (i >= NSLOT && !wait(&bars.kfree[s], ((i / NSLOT) - 1) & 1)) break;
-                    tc::mbar_expect_tx(&bars.kfull[s], PL::KT);
-#pragma unroll
-                    for (int j = 0; j < DK / 64; ++j)
-                        tc::tma_load_3d(base + PL::P_K + s * PL::KT + j * 8192, &tmap_k, &bars.kfull[s], j * 64,
-                                        n * C, bh);
-                    last[s] = i;
-                }
-                if (abort_flag) {
-                    for (int s = 0; s < NSLOT; ++s)
-                        if (last[s] >= 0) tc::mbar_wait(&bars.kfull[s], (last[s] / NSLOT) & 1, budget / 8);
-                }
-            }
-        } else if (warp == W_ISSUE) {
-            // ------------------------------------------------------ MMA issuer (producer CTA)
-            // The Gram of chunk i is issued ahead of W of chunk i - WLAG, so that the solves of
-            // several chunks are in flight while W waits for the oldest.
-            if (lane == 0) {
-                constexpr uint32_t id_g = tc::idesc_bf16(64, 64, false, false);
-                constexpr uint32_t id_w = tc::idesc_f16(64, DK, false, true);
-                bool issued_any = false;
-                for (int it = 0; it < cnt + WLAG; ++it) {
-                    if (it < cnt) {  // Gram K K^T of chunk it (bf16), once its group has read its last one
-                        const int i = it, s = i % NSLOT, g = i % NGRP;
-                        if (!wait(&bars.kfull[s], (i / NSLOT) & 1)) break;
-                        if (i >= NGRP && !wait(&bars.gread[g], ((i / NGRP) - 1) & 1)) break;
-                        tc::tc_fence_after();
-                        issued_any = true;
-                        const uint32_t kb = sb + PL::P_K + s * PL::KT;
-#pragma unroll
-                        for (int kk = 0; kk < DK / 16; ++kk) {
-                            const uint64_t d = tc::sdesc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                            tc::mma_bf16(tmem + TP_G + g * 64, d, d, id_g, kk > 0);
-                        }
-                        tc::mma_commit(&bars.gdone[g]);
-                    }
-                    const int j = it - WLAG;
-                    if (j >= 0) {  // W = Ta K of chunk j (fp16: Ta from the solve, K converted by it)
-                        const int s = j % NSLOT, b = j & 1;
-                        if (!wait(&bars.tready[s], (j / NSLOT) & 1)) break;
-                        if (j >= 2 && !wait(&bars.wst[b], ((j - 2) >> 1) & 1)) break;
-                        tc::tc_fence_after();
-                        const uint32_t kb = sb + PL::P_K + s * PL::KT, tb = sb + PL::P_T + s * (C * C * 2);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_bf16(tmem + TP_W + b * DK, tc::sdesc(tb + kk * 32, 16, 1024),
-                                         tc::sdesc(kb + kk * 2048, 8192, 1024), id_w, kk > 0);
-                        tc::mma_commit(&bars.wdone[b]);
-                        tc::mma_commit(&bars.kfree[s]);  // the K slot is no longer read
-                    }
-                }
-                if (abort_flag && issued_any) {
-                    tc::mma_commit(&bars.pdrain);
-                    tc::mbar_wait(&bars.pdrain, 0, budget / 4);
-                }
-            }
-        } else if (wg != 1) {
-            // ------------------------------------------------------ triangular solve (producer CTA)
-            // Solve group g (warps 0-3, 8-11 or 12-15) takes chunks g, g + 3, ...: alpha per row
-            // from the Gram diagonal (the squared norm) and beta, A = strictly-lower(diag(a) G),
-            // T = (I + A)^{-1} by blocked forward substitution on 16x16 blocks (the diagonal
-            // blocks by fp32 substitution, one column per thread; the off-diagonal blocks level
-            // by level, T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, on warp-level mma.sync), Ta =
-            // T diag(a) as fp16 into the chunk's swizzled Ta slot, and the chunk's K to fp16.
-            using namespace prep;
-            const int g = wg == 0 ? 0 : wg - 1;
-            const int bar_id = 1 + g;
-            uint8_t *sol = base + PL::P_SOLVE + g * PL::SOLVE_STRIDE;
-            __half *A16 = reinterpret_cast<__half *>(sol + PL::S_A16);
-            __half *TD16 = reinterpret_cast<__half *>(sol + PL::S_TD16);
-            float *Ad = reinterpret_cast<float *>(sol + PL::S_AD);  // A's fp32 diagonal blocks
-            __half *Rt = reinterpret_cast<__half *>(sol + PL::S_AD);  // after the solve: merge scratch
-            __half *T16t = reinterpret_cast<__half *>(sol + PL::S_T16T);
-            float *al = reinterpret_cast<float *>(sol + PL::S_AL);
-            const int q4 = warp & 3;
-            const int crow = acc_row<64>(q4, lane);  // this thread's row of the M = 64 Gram
-            auto load_beta = [&](int i) {  // beta of row crow of local chunk i (0 past the end)
-                if (crow < 0 || i >= cnt) return 0.f;
-                const int t = (n0 + i) * C + crow;
-                return t < L ? __bfloat162float(beta[(size_t)bh * L + t]) : 0.f;
-            };
-            // element (r, c) of a swizzled Ta tile (128-byte rows of 64 fp16)
-            auto ta_at = [](uint8_t *T, int r, int c) { return T + tc::sw128_off(r, c >> 3) + (c & 7) * 2; };
-            float beta_next = load_beta(g);
-            for (int i = g; i < cnt; i += NGRP) {
-                const int s = i % NSLOT;
-                uint8_t *Tb = base + PL::P_T + s * (C * C * 2);
-                const float beta_row = beta_next;
-                beta_next = load_beta(i + NGRP);
-                // the Gram is in TMEM; the Ta slot's previous chunk (i - NSLOT) has been read by
-                // its W and copied out (the state CTA's D1 of that chunk has finished)
-                bool ok = wait_warp(&bars.gdone[g], (i / NGRP) & 1);
-                if (ok && i >= NSLOT) ok = wait_warp(&bars.sfree[s], ((i / NSLOT) - 1) & 1);
-                ok = !tc::named_bar_or(bar_id, 128, !ok);  // all four warps take the same decision
-                if (!ok) break;
-                tc::tc_fence_after();
-                float2 lp = make_float2(0.f, 0.f);  // gated: l_t of this chunk's token pairs
-                if constexpr (GATED) lp = chunk_logdecay(grow, (n0 + i) * C, L, lane);
-                {
-                    float g0[32], g1[32];  // this row of the Gram, columns 0..31 and 32..63
-                    tc::tmem_ld32(tmem + lane_base + TP_G + g * 64, g0);
-                    tc::tmem_ld32(tmem + lane_base + TP_G + g * 64 + 32, g1);
-                    warp_arrive(&bars.gread[g], lane);
-                    if constexpr (GATED) {  // Gam o G: entry (r, c) scaled by e^{l_r - l_c} (c < r: <= 1)
-                        const float lr = logdecay_at(lp, crow < 0 ? 0 : crow);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float e0 = fminf(lr - logdecay_at(lp, j), 0.f);
-                            const float e1 = fminf(lr - logdecay_at(lp, j + 32), 0.f);
-                            if (j != crow) g0[j] *= expf(e0);
-                            if (j + 32 != crow) g1[j] *= expf(e1);
-                        }
-                    }
-                    if (crow >= 0) {
-                        float lam = 0.f;  // the diagonal entry: this row's squared norm
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            lam = (j == crow) ? g0[j] : lam;
-                            lam = (j + 32 == crow) ? g1[j] : lam;
-                        }
-                        const float ar = alpha_rule(lam, beta_row, euler);
-                        al[crow] = ar;
-#pragma unroll
-                        for (int cb = 0; cb < 4; ++cb) {
-                            float v[16];
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int c = cb * 16 + j;
-                                v[j] = (c < crow) ? ar * (c < 32 ? g0[c] : g1[c - 32]) : 0.f;
-                            }
-                            uint4 *dst = reinterpret_cast<uint4 *>(A16 + crow * LD16 + cb * 16);
-                            dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
-                                                tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
-                            dst[1] = make_uint4(tc::pack_f16(v[8], v[9]), tc::pack_f16(v[10], v[11]),
-                                                tc::pack_f16(v[12], v[13]), tc::pack_f16(v[14], v[15]));
-                            if (cb == (crow >> 4)) {
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) Ad[crow * 16 + j] = v[j];
-                            }
-                        }
-                    }
-                }
-                tc::named_bar_sync(bar_id, 128);
-                // ---- diagonal blocks: column c of (I + A_bb)^{-1}, one column per thread
-                if (gtid < 64) {
-                    const int bb = gtid >> 4, c = gtid & 15;
-                    const float ac = al[16 * bb + c];
-                    float x[16];
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const float *arow = Ad + (16 * bb + r) * 16;
-                        float s0 = (r == c) ? 1.f : 0.f, s1 = 0.f;  // two chains: half the dependent latency
-#pragma unroll
-                        for (int m = 0; m + 1 < r; m += 2) {
-                            s0 = fmaf(-arow[m], x[m], s0);
-                            s1 = fmaf(-arow[m + 1], x[m + 1], s1);
-                        }
-                        if (r & 1) s0 = fmaf(-arow[r - 1], x[r - 1], s0);
-                        x[r] = s0 + s1;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const int row = 16 * bb + r, col = 16 * bb + c;
-                        TD16[(bb * 16 + r) * 24 + c] = __float2half_rn(x[r]);
-                        T16t[col * LD16 + row] = __float2half_rn(x[r]);
-                        *reinterpret_cast<__half *>(ta_at(Tb, row, col)) = __float2half_rn(x[r] * ac);
-                    }
-                } else {
-                    // zero the strictly-upper 16x16 blocks of the Ta tile
-                    for (int e = gtid - 64; e < 6 * 128; e += 64) {
-                        const int blk = e >> 7, w = e & 127;
-                        const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                        const int J = blk < 3 ? 1 + blk : (blk < 5 ? blk - 1 : 3);
-                        *reinterpret_cast<uint32_t *>(ta_at(Tb, 16 * I + (w >> 3), 16 * J + 2 * (w & 7))) = 0u;
-                    }
-                }
-                tc::named_bar_sync(bar_id, 128);
-                // ---- off-diagonal blocks, one 16x16 block per warp, level by level
-                for (int lvl = 1; lvl < 4; ++lvl) {
-                    const int J = q4, I = J + lvl;
-                    if (I < 4) {
-                        float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                        for (int K = J; K < I; ++K) {
-                            uint32_t a[4];
-                            load_a(a, A16, LD16, 16 * I, 16 * K, lane);
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt) {
-                                uint32_t b0, b1;
-                                load_b(b0, b1, T16t, LD16, 16 * K, 16 * J + 8 * nt, lane);
-                                mma16816(r[nt], a, b0, b1);
-                            }
-                        }
-                        // R -> fp16, transposed, into this warp's scratch
-                        __half *rt = Rt + q4 * 16 * 24;
-                        const int gq = lane >> 2, tq = lane & 3;
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const int c0 = 8 * nt + 2 * tq;
-                            rt[(c0) * 24 + gq] = __float2half_rn(r[nt][0]);
-                            rt[(c0 + 1) * 24 + gq] = __float2half_rn(r[nt][1]);
-                            rt[(c0) * 24 + gq + 8] = __float2half_rn(r[nt][2]);
-                            rt[(c0 + 1) * 24 + gq + 8] = __float2half_rn(r[nt][3]);
-                        }
-                        __syncwarp();
-                        uint32_t a[4];
-                        load_a(a, TD16 + I * 16 * 24, 24, 0, 0, lane);
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            float d[4] = {0.f, 0.f, 0.f, 0.f};
-                            uint32_t b0, b1;
-                            load_b(b0, b1, rt, 24, 0, 8 * nt, lane);
-                            mma16816(d, a, b0, b1);
-                            const int row = 16 * I + gq, col = 16 * J + 8 * nt + 2 * tq;
-                            const float a0 = al[col], a1 = al[col + 1];
-                            *reinterpret_cast<uint32_t *>(ta_at(Tb, row, col)) = tc::pack_f16(-d[0] * a0, -d[1] * a1);
-                            *reinterpret_cast<uint32_t *>(ta_at(Tb, row + 8, col)) = tc::pack_f16(-d[2] * a0, -d[3] * a1);
-                            T16t[col * LD16 + row] = __float2half_rn(-d[0]);
-                            T16t[(col + 1) * LD16 + row] = __float2half_rn(-d[1]);
-                            T16t[col * LD16 + row + 8] = __float2half_rn(-d[2]);
-                            T16t[(col + 1) * LD16 + row + 8] = __float2half_rn(-d[3]);
-                        }
-                    }
-                    tc::named_bar_sync(bar_id, 128);
-                }
-                // ---- the chunk's K to fp16 in place (W's operand; the Gram has read the bf16 tile);
-                // gated: row t scaled by e^{l_t} <= 1, so that W = Ta diag(e^{l}) K
-                {
-                    uint4 *t = reinterpret_cast<uint4 *>(base + PL::P_K + s * PL::KT);
-                    if constexpr (GATED) {
-                        // this thread's elements e = gtid + 128 m are rows (gtid >> 3) + 16 m of a slab
-                        float f[4];
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) f[m] = expf(logdecay_at(lp, (gtid >> 3) + 16 * m));
-#pragma unroll
-                        for (int e = gtid, m = 0; e < (DK / 64) * 512; e += 128, m = (m + 1) & 3) {
-                            uint4 u = t[e];
-                            u.x = tc::bf16x2_to_f16x2_scaled(u.x, f[m]); u.y = tc::bf16x2_to_f16x2_scaled(u.y, f[m]);
-                            u.z = tc::bf16x2_to_f16x2_scaled(u.z, f[m]); u.w = tc::bf16x2_to_f16x2_scaled(u.w, f[m]);
-                            t[e] = u;
-                        }
-                    } else {
-#pragma unroll 4
-                        for (int e = gtid; e < (DK / 64) * 512; e += 128) {
-                            uint4 u = t[e];
-                            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
-                            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-                            t[e] = u;
-                        }
-                    }
-                }
-                tc::fence_async_smem();  // Ta and K are read by the tensor core, Ta by a bulk copy
-                warp_arrive(&bars.tready[s], lane);
-            }
-        } else {
-            // ------------------------------------------------------ epilogue (producer CTA)
-            const int crow = acc_row<64>(warp & 3, lane);  // token row of the M = 64 accumulator
-            bool done_all = true;
-            for (int i = 0; i < cnt && done_all; ++i) {
-                const int b = i & 1;  // W's TMEM buffer, its staging tile and the state CTA's stage
-                const uint32_t par = (i >> 1) & 1;
-                // -W: its staging tile and the state CTA's slots are free once that CTA's D1 of the
-                // chunk two back has finished
-                if (!wait_warp(&bars.wdone[b], par)) { done_all = false; break; }
-                if (i >= 2 && !wait_warp(&bars.sfree[(i - 2) % NSLOT], ((i - 2) / NSLOT) & 1)) {
-                    done_all = false;
-                    break;
-                }
-                tc::tc_fence_after();
-#pragma unroll
-                for (int cb = 0; cb < DK / 32; ++cb) {
-                    float v[32];
-                    tc::tmem_ld32(tmem + lane_base + TP_W + b * DK + cb * 32, v);
-                    if (crow >= 0) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = -v[j];
-                        store_row_f16x32(base + PL::P_W + b * (DK * 128) + (cb >> 1) * 8192, crow, (cb & 1) * 4, v);
-                    }
-                }
-                tc::fence_async_smem();
-                warp_arrive(&bars.wst[b], lane);
-                if (warp == 4) {  // the copying warp: once all four warps have staged -W
-                    if (!wait_warp(&bars.wst[b], par)) { done_all = false; break; }
-                    if (lane == 0) {  // Ta and -W of this chunk into the state CTA's stage b
-                        const uint32_t rb = tc::mapa(tc::smem_u32(&bars.recvW[b]), 0);
-                        tc::mbar_arrive_expect_tx_remote(rb, DK * 128 + Lay::TB);
-                        tc::bulk_copy_to_peer(tc::mapa(sb + b * Lay::STAGE + Lay::OFF_T, 0),
-                                              sb + PL::P_T + (i % NSLOT) * (C * C * 2), Lay::TB, rb);
-#pragma unroll
-                        for (int j = 0; j < DK / 64; ++j)  // rows 64..127 of the state CTA's QW slab j
-                            tc::bulk_copy_to_peer(
-                                tc::mapa(sb + b * Lay::STAGE + Lay::OFF_QW + j * Lay::QW_SLAB + 8192, 0),
-                                sb + PL::P_W + b * (DK * 128) + j * 8192, 8192, rb);
-                    }
-                    __syncwarp();
-                }
-            }
-            // the state CTA's last releases arrive here: take them before this CTA may exit
-            if (done_all) {
-                for (int i = cnt > NSLOT ? cnt - NSLOT : 0; i < cnt; ++i)
-                    if (!wait_warp(&bars.sfree[i % NSLOT], (i / NSLOT) & 1)) break;
-            }
-        }
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && abort_flag) {
-        record_error(2u);
-        // copies and signals already in flight between the CTAs land well within this delay
-        if (rank == 1) {
-            const long long t0 = clock64();
-            while (clock64() - t0 < budget / 64) {
-            }
-        }
-    }
-    tc::cluster_sync();  // neither CTA exits while the other may still reach its shared memory
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
-}
-}  // namespace pair
 
 // ------------------------------------------------------------------ bounded-wait self-test
 // One thread waits on an mbarrier that nothing arrives on, for at most `budget` cycles, then
@@ -1891,45 +1181,13 @@ __global__ void __launch_bounds__(D) seg_combine_kernel(float *__restrict__ segb
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// bf16 tensor [d2][d1][d0] (d0 innermost) with a (b0, b1, 1) box, 128-byte swizzle;
-// out-of-range elements read as zero.
 bool make_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                  uint32_t b0, uint32_t b1) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-    const cuuint32_t box[3] = {b0, b1, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tmap::make_3d(m, ptr, d0, d1, d2, b0, b1);
 }
-
 bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint32_t b0,
                  uint32_t b1, CUtensorMapDataType dt) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {d0, d1};
-    const cuuint64_t strides[1] = {d0 * 2};
-    const cuuint32_t box[2] = {b0, b1};
-    const cuuint32_t es[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tmap::make_2d(m, ptr, d0, d1, b0, b1, dt);
 }
 
 template <int DK>
@@ -1953,16 +1211,6 @@ int seg_count(long long BH, int NC, int dk, int dv, int nsm) {
     return G >= 3 ? (int)G : 1;
 }
 size_t ta_bytes(size_t total) { return (total * C * C * sizeof(__half) + 255) / 256 * 256; }
-// The gated form's cluster kernel takes two SMs per run: pass 1's BH (2G - 3) runs fit the SMs
-// up to half as many segments.
-int seg_count_pair(long long BH, int NC, int dk, int dv, int nsm) {
-    if (!seg_sizes_ok(BH, NC, dk, dv)) return 1;
-    long long G = ((long long)nsm + 6 * BH) / (4 * BH);
-    G = G < SEG_MAX ? G : SEG_MAX;
-    G = G < NC / 16 ? G : NC / 16;
-    return G >= 3 ? (int)G : 1;
-}
-
 // What a launch needs to know about the current device, worked out once per device
 // and kernel instantiation (the kernels' shared-memory attributes are set then too),
 // so that a call costs the tensor-map encodings and the two launches and nothing more.
@@ -1993,9 +1241,9 @@ TcDevInfo tc_dev_info() {
     if (d.err == cudaSuccess)
         d.err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     if (d.err == cudaSuccess)
-        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
     if (d.err == cudaSuccess)
-        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK, false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (d.err == cudaSuccess)
         d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
@@ -2010,13 +1258,17 @@ TcDevInfo tc_dev_info() {
             d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true, true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
     }
-    constexpr int PSMEM = pair::PairLayout<DK, DV>::SMEM;  // the gated form's cluster kernel
+    constexpr int GSMEM = StateLayout<DK, DV, true>::SMEM;  // the gated form
     if (d.err == cudaSuccess)
-        d.err = cudaFuncSetAttribute(pair::tc_pair_kernel<DK, DV, TO, false, false, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM);
+        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+    if (d.err == cudaSuccess)
+        d.err = cudaFuncSetAttribute(tc_prep_kernel<DK, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (d.err == cudaSuccess)
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, GSMEM);
     if (d.err == cudaSuccess && DK == DV)
-        d.err = cudaFuncSetAttribute(pair::tc_pair_kernel<DK, DV, TO, true, false, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM);
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, GSMEM);
     if (d.err != cudaSuccess) return d;
     d.nsm = nsm;
     int per_sm = smem_sm / (psm + 1024);  // 1 KiB per CTA is reserved by the system
@@ -2027,47 +1279,13 @@ TcDevInfo tc_dev_info() {
     return d;
 }
 
-// The gated form: one launch of the cluster kernel (its producer CTAs compute the Gram, the
-// triangular solve and W per chunk, so there is no prep kernel), or its segment passes.
-template <int DK, int DV, typename TO>
-cudaError_t launch_gated(const void *q, const void *k, const void *v, const void *beta, const void *gate,
-                         const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
-                         void *ws, cudaStream_t s, bool allow_seg) {
-    const int BH = B * H, NC = (L + C - 1) / C, total = BH * NC;
-    const TcDevInfo di = tc_dev_info<DK, DV, TO>();
-    if (di.err != cudaSuccess) return di.err;
-    CUtensorMap mq, mk, mv;
-    if (!make_map_3d(&mq, q, DK, L, BH, 64, C) || !make_map_3d(&mk, k, DK, L, BH, 64, C) ||
-        !make_map_3d(&mv, v, DV, L, BH, 64, C))
-        return cudaErrorInvalidValue;
-    const __nv_bfloat16 *bt = (const __nv_bfloat16 *)beta, *gt = (const __nv_bfloat16 *)gate;
-    constexpr int PSMEM = pair::PairLayout<DK, DV>::SMEM;
-    constexpr int PT = pair::PR_THREADS;
-    const int G = allow_seg ? seg_count_pair(BH, NC, DK, DV, di.nsm) : 1;
-    if (G < 3) {
-        pair::tc_pair_kernel<DK, DV, TO, false, false, true><<<2 * BH, PT, PSMEM, s>>>(
-            mq, mk, mv, bt, euler, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, nullptr, nullptr, gt);
-        count_launches(1);
-        return cudaGetLastError();
-    }
-    if constexpr (DK == DV) {  // segment states after where the Ta tiles of the ungated form go
-        const int seg_chunks = (NC + G - 1) / G;
-        float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
-        pair::tc_pair_kernel<DK, DV, TO, true, false, true><<<2 * BH * (2 * G - 3), PT, PSMEM, s>>>(
-            mq, mk, mv, bt, euler, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, nullptr, nullptr, gt);
-        seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
-        pair::tc_pair_kernel<DK, DV, TO, true, false, true><<<2 * BH * (G - 1), PT, PSMEM, s>>>(
-            mq, mk, mv, bt, euler, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, nullptr, nullptr, gt);
-        count_launches(3);
-    }
-    return cudaGetLastError();
-}
-
-template <int DK, int DV, typename TO, bool SAVE = false>
+// The prep kernel, then the state kernel: one CTA per head, or the segment passes.  GATED:
+// the gated form, with the decays in g.
+template <int DK, int DV, typename TO, bool SAVE, bool GATED>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void *beta,
                         const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
-                        void *ws, cudaStream_t s, float *u_out = nullptr, float *ck_out = nullptr,
-                        bool allow_seg = true) {
+                        void *ws, cudaStream_t s, float *u_out, float *ck_out, bool allow_seg,
+                        const void *g) {
     const int BH = B * H, NC = (L + C - 1) / C, total = BH * NC;
     const TcDevInfo di = tc_dev_info<DK, DV, TO>();
     if (di.err != cudaSuccess) return di.err;
@@ -2076,30 +1294,31 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         !make_map_3d(&mv, v, DV, L, BH, 64, C) ||
         !make_map_2d(&mt, ws, C, (uint64_t)total * C, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
+    const __nv_bfloat16 *gt = (const __nv_bfloat16 *)g;
     const int pgrid = total < di.prep_grid ? total : di.prep_grid;
-    tc_prep_kernel<DK><<<pgrid, THREADS, prep_smem_bytes<DK>(), s>>>(mk, (const __nv_bfloat16 *)beta,
-                                                                      (__half *)ws, L, NC, total, euler);
+    tc_prep_kernel<DK, GATED><<<pgrid, THREADS, prep_smem_bytes<DK>(), s>>>(
+        mk, (const __nv_bfloat16 *)beta, gt, (__half *)ws, L, NC, total, euler);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    constexpr int SSM = StateLayout<DK, DV>::SMEM;
+    constexpr int SSM = StateLayout<DK, DV, GATED>::SMEM;
     const int G = allow_seg ? seg_count(BH, NC, DK, DV, di.nsm) : 1;
     if (G < 3) {
         // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
-        tc_state_kernel<DK, DV, TO, false, SAVE><<<BH, ST_THREADS, SSM, s>>>(mq, mk, mv, mt, S0, (TO *)o, S_final,
-                                                                      L, NC, nullptr, 1, NC, 0, u_out, ck_out);
+        tc_state_kernel<DK, DV, TO, false, SAVE, GATED><<<BH, ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt);
         count_launches(2);
         return cudaGetLastError();
     }
     if constexpr (DK == DV) {
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
-        tc_state_kernel<DK, DV, TO, true, SAVE><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out);
+        tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt);
         seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
-        tc_state_kernel<DK, DV, TO, true, SAVE><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out);
+        tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
+            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt);
         count_launches(4);
     }
     return cudaGetLastError();
@@ -2111,13 +1330,14 @@ cudaError_t launch_tc_o(const void *q, const void *k, const void *v, const void 
                         bool euler, void *ws, cudaStream_t s, bool allow_seg, const void *g) {
     using bf = __nv_bfloat16;
     if (g)
-        return o_bf16 ? launch_gated<DK, DV, bf>(q, k, v, beta, g, S0, o, S_final, B, H, L, euler, ws, s, allow_seg)
-                      : launch_gated<DK, DV, float>(q, k, v, beta, g, S0, o, S_final, B, H, L, euler, ws, s,
-                                                   allow_seg);
-    return o_bf16 ? launch_tc_t<DK, DV, bf>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s, nullptr,
-                                           nullptr, allow_seg)
-                  : launch_tc_t<DK, DV, float>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s, nullptr,
-                                              nullptr, allow_seg);
+        return o_bf16 ? launch_tc_t<DK, DV, bf, false, true>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s,
+                                                             nullptr, nullptr, allow_seg, g)
+                      : launch_tc_t<DK, DV, float, false, true>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws,
+                                                                s, nullptr, nullptr, allow_seg, g);
+    return o_bf16 ? launch_tc_t<DK, DV, bf, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s,
+                                                          nullptr, nullptr, allow_seg, nullptr)
+                  : launch_tc_t<DK, DV, float, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, s,
+                                                             nullptr, nullptr, allow_seg, nullptr);
 }
 
 }  // namespace
@@ -2168,16 +1388,16 @@ cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, co
                                  const float *S0, int B, int H, int L, int dk, int dv, bool euler,
                                  void *ws, float *u_out, float *ck_out, cudaStream_t s) {
     if (dk == 128 && dv == 128)
-        return launch_tc_t<128, 128, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
-                                                  u_out, ck_out);
+        return launch_tc_t<128, 128, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws,
+                                                         s, u_out, ck_out, true, nullptr);
     if (dk == 128 && dv == 64)
-        return launch_tc_t<128, 64, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
-                                                 u_out, ck_out);
+        return launch_tc_t<128, 64, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws,
+                                                        s, u_out, ck_out, true, nullptr);
     if (dk == 64 && dv == 128)
-        return launch_tc_t<64, 128, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
-                                                 u_out, ck_out);
-    return launch_tc_t<64, 64, float, true>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s, u_out,
-                                            ck_out);
+        return launch_tc_t<64, 128, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws,
+                                                        s, u_out, ck_out, true, nullptr);
+    return launch_tc_t<64, 64, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
+                                                   u_out, ck_out, true, nullptr);
 }
 
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s) {

@@ -41,20 +41,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// As mbar_try_wait, but a thread whose phase is not complete yet may be suspended by the
-// hardware until it completes or about `ns` nanoseconds pass, instead of spinning (a waiting
-// warp then takes no issue slots from the warps that do the work).
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
 // Wait for the phase with the given parity to complete; false after `budget` cycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -119,52 +105,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, uint64_t
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// ---------------------------------------------------------------- clusters
-// Rank of this CTA in its cluster.
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Address in the shared window of CTA `rank` of this cluster that corresponds to
-// the local shared::cta address `a`.
-__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-// Whole-cluster barrier (every thread of every CTA of the cluster).
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-// 32-bit store into another CTA's shared memory (cluster address).
-__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster, announcing `bytes` of
-// transactions that will complete on it.
-__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar_cluster, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
-                     bar_cluster),
-                 "r"(bytes)
-                 : "memory");
-}
-// Arrive (release, cluster scope) on an mbarrier of another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
-}
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this
-// CTA's shared memory into another CTA's shared memory, completion reported as
-// transaction bytes on an mbarrier of the destination CTA.  No multicast.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src_cta), "r"(bytes), "r"(bar_cluster)
         : "memory");
 }
 
@@ -334,12 +274,6 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t u, float f) {
     const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xffff0000u);
     return pack_f16(lo * f, hi * f);
-}
-
-// Two packed fp16 scaled by f (|f| <= 1), rounded to fp16.
-__device__ __forceinline__ uint32_t f16x2_scale(uint32_t u, float f) {
-    const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(&u));
-    return pack_f16(x.x * f, x.y * f);
 }
 
 // 32 lanes x 32 bits store of 16 consecutive columns; waits for completion.

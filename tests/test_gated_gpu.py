@@ -96,3 +96,60 @@ def test_gated_decode_step_matches_oracle(oracle_mod, dtype, dk, dv):
     tol = TOL[dtype]
     assert rel_err(o.cpu().numpy(), o_ref) <= tol
     assert rel_err(Sd.cpu().numpy(), S_ref) <= tol
+
+
+def test_gated_segments_match_oracle(oracle_mod):
+    """Few heads and a long sequence: the gated form on the sequence-segment path (each
+    segment's affine map, S_out = P S_in + H, carries the decays too), stiff inputs."""
+    w = inputs.workload(5, B=1, H=2, L=8192 + 37)
+    assert efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, 64, torch.bfloat16) == "tcgen05-segments"
+    x = inputs.make_inputs(w, seed=41)
+    x["g"] = _gate(x["beta"].shape, x["beta"].dtype, 42)
+    d = _dev(x)
+    o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64, g=d["g"])
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    o_ref, S_ref = oracle_mod.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], g=x["g"])
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("lo,hi", [(0.005, 0.05), (0.3, 0.6), (0.999, 1.0)])
+def test_gated_strong_and_weak_decays(oracle_mod, lo, hi):
+    """Decays from near 0 (the chunk's cumulative decay underflows: every factor the kernels
+    apply must stay a decay of at most 1) to near 1, with a nonzero starting state and a
+    ragged tail, bf16 output too."""
+    w = inputs.workload(2, B=1, H=3, L=700, dk=128, dv=64, s0_std=0.3)
+    x = inputs.make_inputs(w, seed=43)
+    gen = torch.Generator().manual_seed(44)
+    x["g"] = (lo + (hi - lo) * torch.rand(x["beta"].shape, generator=gen)).to(x["beta"].dtype)
+    d = _dev(x)
+    o_ref, S_ref = oracle_mod.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], g=x["g"])
+    for odt in (torch.float32, torch.bfloat16):
+        o, S = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64, g=d["g"], o_dtype=odt)
+        torch.cuda.synchronize()
+        assert efla.last_device_error() == 0
+        assert np.isfinite(o.float().cpu().numpy()).all()
+        tol = TOL["bf16"] + (2.0 ** -8 * np.abs(o_ref).max() / np.sqrt((o_ref ** 2).mean())
+                             if odt == torch.bfloat16 else 0.0)
+        assert rel_err(o.float().cpu().numpy(), o_ref) <= tol
+        assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"]
+
+
+def test_gate_of_one_on_the_tensor_cores_matches_the_ungated_forward(oracle_mod):
+    """bf16 at the tensor-core sizes: with g = 1 every decay factor is exactly 1, so the gated
+    kernels compute the ungated forward; they take the intra-chunk output term at higher
+    precision (fp16 hi + lo factors), so against the oracle their error is at most the ungated
+    kernels' (plus rounding noise), and the two results agree within the bf16 bound."""
+    w = inputs.workload(4, B=1, H=4, L=1000)
+    x = inputs.make_inputs(w, seed=45)
+    d = _dev(x)
+    one = torch.ones_like(d["beta"])
+    o1, S1 = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64)
+    o2, S2 = efla.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], chunk=64, g=one)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_mod.fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"])
+    e1, e2 = rel_err(o1.cpu().numpy(), o_ref), rel_err(o2.cpu().numpy(), o_ref)
+    assert e2 <= e1 * 1.1 + 1e-4, (e1, e2)
+    assert rel_err(S2.cpu().numpy(), S_ref) <= TOL["bf16"]
+    assert rel_err(o2.cpu().numpy(), o1.cpu().numpy()) <= TOL["bf16"]
