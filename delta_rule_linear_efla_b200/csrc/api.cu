@@ -251,10 +251,11 @@ unsigned long long efla_kernel_launches(void) {
 }
 
 efla_status efla_last_device_error(void *stream) {
-    unsigned int word = 0;
-    if (efla::tc_read_and_clear_error(&word, (cudaStream_t)stream) != cudaSuccess)
+    unsigned int word = 0, bwd_word = 0;
+    if (efla::tc_read_and_clear_error(&word, (cudaStream_t)stream) != cudaSuccess ||
+        efla::bwd_tc_read_and_clear_error(&bwd_word) != cudaSuccess)
         return EFLA_ERR_CUDA;
-    return word ? EFLA_ERR_TIMEOUT : EFLA_OK;
+    return (word | bwd_word) ? EFLA_ERR_TIMEOUT : EFLA_OK;
 }
 
 }  // extern "C"

@@ -30,6 +30,7 @@
 #include <algorithm>
 #include <cstdint>
 
+#include "bwd_gate.cuh"
 #include "common.cuh"
 #include "launchers.h"
 
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
                     const float *__restrict__ dO, const float *__restrict__ dSL,
                     float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
                     float *__restrict__ ws, float *__restrict__ part, const float *__restrict__ u_saved,
-                    const float *__restrict__ ck_saved, const int *__restrict__ hs) {
+                    const float *__restrict__ ck_saved, const int *__restrict__ hs, bool tc_heads) {
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
@@ -229,13 +230,8 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // spread of a from small betas (0.006 at a max/min ratio of 800).  So the saved values are
     // used only for heads whose largest ||k||^2 is at most 16, whose a spans at most a factor of
     // 1024, and whose a are all positive; other heads walk the forward in fp32 themselves (saved_ok).
-    bool saved_ok = false;
-    if (u_saved != nullptr) {
-        const int *h = hs + 4 * bh;
-        const float lam_max = __int_as_float(h[1]), a_min = __int_as_float(0x7fffffff - h[2]);
-        const float a_max = __int_as_float(h[3]);
-        saved_ok = h[0] == 0 && lam_max <= 16.f && a_max <= 1024.f * a_min;
-    }
+    const bool saved_ok = u_saved != nullptr && head_takes_saved(hs, bh);
+    if (saved_ok && tc_heads) return;  // the tensor-core backward takes this head
     auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
         return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
     };
@@ -436,18 +432,20 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     }
 }
 
-// out[e] = sum over s = 0..NS-1 of part[s n + e], in that order (blockIdx.y picks dq, dk, dbeta).
+// out[e] = sum over s = 0..NS-1 of part[s n + e], in that order (blockIdx.y picks dq, dk, dbeta);
+// with tc_hs, elements of heads that the tensor-core backward takes are left alone.
 struct SumSeg {
     const float *part;
     float *out;
     size_t n;
-    int vec;  // 1: n % 4 == 0 and both arrays 16-byte aligned
+    size_t per_head;  // elements per head
+    int vec;          // 1: n and per_head multiples of 4, both arrays 16-byte aligned
 };
 struct SumSegs {
     SumSeg seg[3];
 };
 
-__global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS) {
+__global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS, const int *__restrict__ tc_hs) {
     const SumSeg g = blockIdx.y == 0 ? segs.seg[0] : (blockIdx.y == 1 ? segs.seg[1] : segs.seg[2]);
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -456,6 +454,7 @@ __global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS) {
         const float4 *p4 = reinterpret_cast<const float4 *>(g.part);
         float4 *o4 = reinterpret_cast<float4 *>(g.out);
         for (size_t e = i0; e < n4; e += stride) {
+            if (tc_hs && head_takes_saved(tc_hs, (long long)(4 * e / g.per_head))) continue;
             float4 a = p4[e];
             for (int s = 1; s < NS; ++s) {
                 const float4 b = p4[(size_t)s * n4 + e];
@@ -465,6 +464,7 @@ __global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS) {
         }
     } else {
         for (size_t e = i0; e < g.n; e += stride) {
+            if (tc_hs && head_takes_saved(tc_hs, (long long)(e / g.per_head))) continue;
             float a = g.part[e];
             for (int s = 1; s < NS; ++s) a += g.part[(size_t)s * g.n + e];
             g.out[e] = a;
@@ -486,7 +486,7 @@ static bool bwd_tc_saves(int B, int H, int L, int dk, int dv) {
 }
 
 struct BwdLayout {  // float offsets into the workspace
-    size_t coef, zero, state, part, tc, u, ck, total;
+    size_t coef, zero, state, part, tc, u, ck, tcb, total;
 };
 
 static BwdLayout bwd_layout(int B, int H, int L, int dk, int dv) {
@@ -499,11 +499,12 @@ static BwdLayout bwd_layout(int B, int H, int L, int dk, int dv) {
     a.state = a.zero + up(4 * BH);
     a.part = a.state + up(bwd_state_floats(BH, L, dk, dv));
     a.tc = a.part + up(NS * ntok * (2 * (size_t)dk + 1));
-    a.u = a.ck = a.total = a.tc;
+    a.u = a.ck = a.tcb = a.total = a.tc;
     if (bwd_tc_saves(B, H, L, dk, dv)) {
         a.u = a.tc + up((tc_workspace_bytes(B, H, L, dk, dv, BWD_BLOCK) + 3) / 4);
         a.ck = a.u + up(ntok * (size_t)dv);
-        a.total = a.ck + BH * NB * (size_t)dk * dv;
+        a.tcb = a.ck + up(BH * NB * (size_t)dk * dv);
+        a.total = a.tcb + (bwd_tc_workspace_bytes(B, H, L, dk, dv) + 3) / 4;
     }
     return a;
 }
@@ -531,7 +532,13 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     float *part = wsf + lay.part;
     float *u_saved = nullptr, *ck_saved = nullptr;
     cudaError_t e;
-    if (is_bf16 && bwd_tc_saves(B, H, L, dk, dv)) {
+    // the tensor-core forward (TMA) and backward load q, k, v, S0 and dO 16 bytes at a time;
+    // inputs that are only element-aligned take the CUDA-core path for every head
+    auto al16 = [](const void *p) { return ((uintptr_t)p & 15) == 0; };
+    const bool tc_fwd = is_bf16 && bwd_tc_saves(B, H, L, dk, dv) && al16(q) && al16(k) && al16(v) &&
+                        (S0 == nullptr || al16(S0));
+    const bool tc_bwd = tc_fwd && al16(dO);
+    if (tc_fwd) {
         // the tensor-core forward, saving u and the block states instead of writing outputs
         u_saved = wsf + lay.u;
         ck_saved = wsf + lay.ck;
@@ -552,36 +559,43 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
                                                        hs);
         count_launches(1);
     }
+    if (tc_bwd && L > 0) {
+        e = launch_bwd_tc(q, k, v, S0, dO, dSL, coef, hs, u_saved, ck_saved, wsf + lay.tc, dq, dkey, dval, dbeta,
+                          dS0, B, H, L, dk, dv, wsf + lay.tcb, s);
+        if (e != cudaSuccess) return e;
+    }
     const int grid = (int)(BH * NS);
     if (is_bf16)
         bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, dO,
-            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, hs);
+            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, hs, tc_bwd);
     else
         bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
                                                           (const float *)v, coef, S0, dO, dSL, dval,
                                                           dS0, L, dk, dv, NS, state, part, nullptr,
-                                                          nullptr, hs);
+                                                          nullptr, hs, false);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess || L == 0) return e;
     // add the column blocks' shares of dq, dk and dbeta
     const size_t nq = (size_t)BH * L * dk, nb = (size_t)BH * L;
-    auto seg = [&](const float *pp, float *out, size_t n) {
+    auto seg = [&](const float *pp, float *out, size_t n, size_t per_head) {
         SumSeg g;
         g.part = pp;
         g.out = out;
         g.n = n;
-        g.vec = (n % 4 == 0 && ((uintptr_t)pp % 16) == 0 && ((uintptr_t)out % 16) == 0) ? 1 : 0;
+        g.per_head = per_head;
+        g.vec = (n % 4 == 0 && per_head % 4 == 0 && ((uintptr_t)pp % 16) == 0 && ((uintptr_t)out % 16) == 0)
+                    ? 1 : 0;
         return g;
     };
     SumSegs segs;
-    segs.seg[0] = seg(part, dq, nq);
-    segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq);
-    segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb);
+    segs.seg[0] = seg(part, dq, nq, (size_t)L * dk);
+    segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq, (size_t)L * dk);
+    segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb, (size_t)L);
     const size_t want = (nq / 4 + 255) / 256;
     const int gx = (int)std::min<size_t>(std::max<size_t>(want, 1), (size_t)nsm * 8);
-    bwd_sum_kernel<<<dim3(gx, 3), 256, 0, s>>>(segs, NS);
+    bwd_sum_kernel<<<dim3(gx, 3), 256, 0, s>>>(segs, NS, tc_bwd ? hs : nullptr);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -1,0 +1,792 @@
+// bwd_tc.cu -- tensor-core backward of the EFLA chunkwise forward, sm_100a (bf16 inputs,
+// chunk 64, dk and dv in {64, 128}).
+//
+// "Exact Flow Linear Attention: Exact Solution from Continuous-Time Dynamics", technical
+// summary, Methodology 3: the forward per chunk of C = 64 tokens entering with state S is
+//
+//   A = strictly-lower(diag(a) K K^T),  T = (I + A)^{-1},  R = V - K S,  U' = T diag(a) R,
+//   O = Q S + P U'  (P = lower-incl(Q K^T)),  S' = S + K^T U'.
+//
+// Reverse mode through those lines, given dO and dS' (the gradient of the state after the
+// chunk), splits into a chain over the chunks and work that is independent per chunk:
+//
+//   chain (bwd_state_kernel, one CTA per head, chunks last to first):
+//     dU' = K dS' + P^T dO,           dS = dS' + Q^T dO - W^T dU'   (W = Ta K, Ta = T diag(a))
+//   per chunk (bwd_chunk_kernel, every chunk in parallel):
+//     dR = Ta^T dU',  B = -strictly-lower(dR U'^T),  G = K K^T,
+//     da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t,   dP = lower-incl(dO U'^T),
+//     dQ = dO S^T + dP K,
+//     dK = U' dS'^T + dP^T Q - dR S^T + B K + B^T K + 2 da (df/dlambda) K,
+//     dV = dR,  dbeta = da (df/dbeta).
+//
+// (dR = diag(a) T^T dU' and B = diag(a) dA with dA = strictly-lower(-T^T dT T^T), dT =
+// dU' (diag(a) R)^T, which is -(T^T dU') U'^T since T diag(a) R = U'.)  The chain carries
+// dS^T in TMEM the way the forward carries S^T; both kernels take fp16 operands with fp32
+// accumulation, the precision of the forward's products.  The per-head gate of the backward
+// (keys of squared norm at most 16, a spanning at most a factor of 1024, every a positive)
+// decides which heads take this path; the others walk the forward in fp32 on CUDA cores.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "bwd_gate.cuh"
+#include "common.cuh"
+#include "launchers.h"
+#include "tc_ptx.cuh"
+#include "tmap.h"
+
+namespace efla {
+
+namespace {
+
+constexpr int C = 64;
+constexpr long long WAIT_BUDGET = 2000000000LL;  // ~1 s of SM cycles
+__device__ unsigned int g_bwd_error = 0;
+
+// ------------------------------------------------------------------ the chain over chunks
+// Shared memory per stage (double buffered): Q, K (bf16 by TMA, fp16 after the converter),
+// dO (fp16), Ta (fp16), -W and P (fp16, written by the side group); 64-token tiles of 128-byte
+// rows, 128-byte swizzle, one 8 KB slab per 64 columns.
+template <int DK, int DV>
+struct RevLayout {
+    static constexpr int QB = (DK / 64) * 8192, KB = QB, OB = (DV / 64) * 8192;
+    static constexpr int TB = C * C * 2, WB = QB, PB = C * C * 2;
+    static constexpr int OFF_Q = 0, OFF_K = QB, OFF_O = OFF_K + KB, OFF_T = OFF_O + OB;
+    static constexpr int OFF_W = OFF_T + TB, OFF_P = OFF_W + WB;
+    static constexpr int STAGE = OFF_P + PB;
+    static constexpr int SMEM = 2 * STAGE + 1024;  // + alignment slack
+};
+
+// Single-arrival barriers first, then those a warpgroup arrives on once per warp.
+struct RevBars {
+    uint64_t full[2], freeS[2], wdone, pdone, d1done, d2done, drain;
+    uint64_t conv[2], w_ready, p_ready, up_ready, s_ready;
+};
+constexpr int REV_ONE = 9;
+constexpr int REV_WARPS = 14;  // converter, side, chain warpgroups; MMA issuer; TMA producer
+constexpr int REV_THREADS = REV_WARPS * 32;
+constexpr int RW_ISSUE = 12, RW_PROD = 13;
+constexpr uint32_t RT_W = 256, RT_P = 384, RT_S16 = 448;
+
+__device__ __forceinline__ void rev_arrive(uint64_t *bar, int lane) {
+    tc::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(bar);
+}
+
+__device__ __forceinline__ void store_row16x32(uint8_t *tile, int row, int ch0, const float (&v)[32]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = tc::pack_f16(v[8 * c + 0], v[8 * c + 1]); u.y = tc::pack_f16(v[8 * c + 2], v[8 * c + 3]);
+        u.z = tc::pack_f16(v[8 * c + 4], v[8 * c + 5]); u.w = tc::pack_f16(v[8 * c + 6], v[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + tc::sw128_off(row, ch0 + c)) = u;
+    }
+}
+
+__device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_takes_saved(hs, bh); }
+
+// One CTA per head, chunks from last to first.  TMEM (fp32 columns): dS^T [0, DK), dU'^T
+// [DK, DK + 64) (fp16 dU'^T packed over its first 32 after the epilogue), W [256, 256 + DK),
+// P [384, 448), dS^T fp16 [448, 448 + DK/2).  Per chunk, in tensor-pipe order:
+//   D1a  dU'^T  = dO^T P            (off the chain)
+//   D1b  dU'^T += dS16^T K^T        (A = the fp16 copy of dS^T in TMEM)
+//   D2a  dS^T  += dO^T Q            (off the chain)
+//   W, P of the next chunk
+//   D2b  dS^T  += dU'16^T (-W)      (A = fp16 dU'^T in TMEM)
+// Outputs: dU' of every token (fp16, [BH][L][dv]); the gradient of the state after every chunk
+// as fp16 dSp [BH][NC][dk][dv] (dSp[NC-1] is dS_final); dS0 (fp32).
+template <int DK, int DV>
+__global__ void __launch_bounds__(REV_THREADS, 1)
+    bwd_state_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_t,
+                     const float *__restrict__ dSL, __half *__restrict__ dU, __half *__restrict__ dSp,
+                     float *__restrict__ dS0, const int *__restrict__ hs, int L, int NC) {
+    using Lay = RevLayout<DK, DV>;
+    constexpr uint32_t TM_S = 0, TM_U = DK;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+    uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    __shared__ RevBars bars;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+
+    const int bh = blockIdx.x;
+    if (!head_ok(hs, bh)) return;  // this head walks on CUDA cores (uniform over the CTA)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = warp >> 2, gtid = tid & 127;
+    const size_t DD = (size_t)DK * DV;
+    if (tid == 0) {
+        uint64_t *b = reinterpret_cast<uint64_t *>(&bars);
+        for (int i = 0; i < (int)(sizeof(RevBars) / sizeof(uint64_t)); ++i)
+            tc::mbar_init(b + i, i < REV_ONE ? 1 : 4);
+        tc::fence_mbar_init();
+        abort_flag = 0;
+        tc::tma_prefetch_desc(&tmap_q);
+        tc::tma_prefetch_desc(&tmap_k);
+        tc::tma_prefetch_desc(&tmap_o);
+        tc::tma_prefetch_desc(&tmap_t);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t sb = tc::smem_u32(base);
+    // state column v of this thread's TMEM lane (M = DV accumulators), or -1
+    const int vrow = DV == 128 ? 32 * (warp & 3) + lane : (lane < 16 ? 16 * (warp & 3) + lane : -1);
+
+    // ---- the initial state gradient dS_final (chain warpgroup): fp32 and fp16 copies in TMEM
+    if (wg == 2) {
+#pragma unroll
+        for (int cb = 0; cb < DK / 32; ++cb) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                v[j] = (dSL && vrow >= 0) ? dSL[(size_t)bh * DD + (size_t)(cb * 32 + j) * DV + vrow] : 0.f;
+            float lo[16], hi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { lo[j] = v[j]; hi[j] = v[16 + j]; }
+            tc::tmem_st16(tmem + lane_base + TM_S + cb * 32, lo);
+            tc::tmem_st16(tmem + lane_base + TM_S + cb * 32 + 16, hi);
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+            tc::tmem_st16u(tmem + lane_base + RT_S16 + cb * 16, w);
+            if (vrow >= 0) {  // dSp[NC - 1]: the gradient of the last chunk's final state
+                __half *dst = dSp + ((size_t)bh * NC + (NC - 1)) * DD + vrow;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * DV] = __float2half_rn(v[j]);
+            }
+        }
+        tc::tc_fence_before();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+
+    const long long budget = WAIT_BUDGET;
+    if (warp == RW_PROD) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int last[2] = {-1, -1};
+            for (int i = 0; i < NC; ++i) {
+                const int n = NC - 1 - i, st = i & 1;
+                uint8_t *stg = base + st * Lay::STAGE;
+                if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeS[st], ((i - 2) >> 1) & 1, &abort_flag, budget))
+                    break;
+                tc::mbar_expect_tx(&bars.full[st], Lay::QB + Lay::KB + Lay::OB + Lay::TB);
+#pragma unroll
+                for (int j = 0; j < DK / 64; ++j) {
+                    tc::tma_load_3d(stg + Lay::OFF_Q + j * 8192, &tmap_q, &bars.full[st], j * 64, n * C, bh);
+                    tc::tma_load_3d(stg + Lay::OFF_K + j * 8192, &tmap_k, &bars.full[st], j * 64, n * C, bh);
+                }
+#pragma unroll
+                for (int j = 0; j < DV / 64; ++j)
+                    tc::tma_load_3d(stg + Lay::OFF_O + j * 8192, &tmap_o, &bars.full[st], j * 64, n * C, bh);
+                tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.full[st], 0, (bh * NC + n) * C);
+                last[st] = i;
+            }
+            if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
+                for (int st = 0; st < 2; ++st)
+                    if (last[st] >= 0) tc::mbar_wait(&bars.full[st], (last[st] >> 1) & 1, budget / 8);
+            }
+        }
+    } else if (warp == RW_ISSUE) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_w = tc::idesc_f16(64, DK, false, true);   // W = Ta K
+            constexpr uint32_t id_p = tc::idesc_f16(64, 64, false, false);  // P = Q K^T
+            constexpr uint32_t id_1a = tc::idesc_f16(DV, 64, true, true);   // dO^T P
+            constexpr uint32_t id_1b = tc::idesc_f16(DV, 64, false, false); // dS16^T K^T
+            constexpr uint32_t id_2a = tc::idesc_f16(DV, DK, true, true);   // dO^T Q
+            constexpr uint32_t id_2b = tc::idesc_f16(DV, DK, false, true);  // dU'16^T (-W)
+            auto stage_addr = [&](int i) { return sb + (i & 1) * Lay::STAGE; };
+            auto issue_wp = [&](int i) {  // W and P of local chunk i (into their TMEM columns)
+                const uint32_t stg = stage_addr(i);
+                const uint32_t q = stg + Lay::OFF_Q, k = stg + Lay::OFF_K, t = stg + Lay::OFF_T;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + RT_W, tc::sdesc(t + kk * 32, 16, 1024), tc::sdesc(k + kk * 2048, 8192, 1024),
+                                 id_w, kk > 0);
+                tc::mma_commit(&bars.wdone);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    tc::mma_bf16(tmem + RT_P, tc::sdesc(q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(k + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_p, kk > 0);
+                tc::mma_commit(&bars.pdone);
+            };
+            auto wait = [&](uint64_t *bar, uint32_t par) {
+                return tc::mbar_wait_or_abort(bar, par, &abort_flag, budget);
+            };
+            bool issued_any = false;
+            bool ok = wait(&bars.conv[0], 0);
+            if (ok) {
+                tc::tc_fence_after();
+                issued_any = true;
+                issue_wp(0);
+            }
+            for (int i = 0; ok && i < NC; ++i) {
+                const int st = i & 1;
+                const uint32_t stg = stage_addr(i);
+                const uint32_t q = stg + Lay::OFF_Q, k = stg + Lay::OFF_K, o = stg + Lay::OFF_O;
+                const uint32_t w = stg + Lay::OFF_W, p = stg + Lay::OFF_P;
+                // D1a: dU'^T = dO^T P  (P read out of TMEM and stored masked by the side group)
+                if (!wait(&bars.p_ready, i & 1)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_U, tc::sdesc(o + kk * 2048, 8192, 1024), tc::sdesc(p + kk * 2048, 8192, 1024),
+                                 id_1a, kk > 0);
+                // D1b: dU'^T += dS16^T K^T  (the fp16 copy of the state gradient)
+                if (i > 0 && !wait(&bars.s_ready, (i - 1) & 1)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    tc::mma_tmem_a(tmem + TM_U, tmem + RT_S16 + kk * 8,
+                                   tc::sdesc(k + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_1b, 1u);
+                tc::mma_commit(&bars.d1done);
+                // D2a: dS^T += dO^T Q  (the chain has read dS^T for this chunk: s_ready above)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_S, tc::sdesc(o + kk * 2048, 8192, 1024), tc::sdesc(q + kk * 2048, 8192, 1024),
+                                 id_2a, 1u);
+                // W and P of the next chunk, once the side group has read this chunk's out of TMEM
+                // (-W of this chunk is then in shared memory too; its P was read before D1a)
+                if (!wait(&bars.w_ready, i & 1)) break;
+                if (i + 1 < NC) {
+                    if (!wait(&bars.conv[(i + 1) & 1], ((i + 1) >> 1) & 1)) break;
+                    tc::tc_fence_after();
+                    issue_wp(i + 1);
+                }
+                // D2b: dS^T += dU'16^T (-W)
+                if (!wait(&bars.up_ready, i & 1)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8, tc::sdesc(w + kk * 2048, 8192, 1024), id_2b, 1u);
+                tc::mma_commit(&bars.d2done);
+                tc::mma_commit(&bars.freeS[st]);
+            }
+            if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
+                tc::mma_commit(&bars.drain);
+                tc::mbar_wait(&bars.drain, 0, budget / 4);
+            }
+        }
+    } else if (wg == 0) {
+        // ---------------------------------------------------------- converter: q, k bf16 -> fp16
+        auto cvt = [](uint4 *t) {
+            uint4 u = *t;
+            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+            *t = u;
+        };
+        for (int i = 0; i < NC; ++i) {
+            const int st = i & 1;
+            uint8_t *stg = base + st * Lay::STAGE;
+            if (!tc::mbar_wait_or_abort(&bars.full[st], (i >> 1) & 1, &abort_flag, budget)) break;
+            uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_Q);  // Q then K: contiguous
+#pragma unroll 4
+            for (int e = gtid; e < (Lay::QB + Lay::KB) / 16; e += 128) cvt(tq + e);
+            tc::fence_async_smem();
+            rev_arrive(&bars.conv[st], lane);
+        }
+    } else if (wg == 1) {
+        // ---------------------------------------------------------- side: -W and the masked P
+        const int crow = lane < 16 ? 16 * (warp & 3) + lane : -1;  // token row of M = 64 accumulators
+        for (int i = 0; i < NC; ++i) {
+            const int st = i & 1;
+            uint8_t *stg = base + st * Lay::STAGE;
+            if (!tc::mbar_wait_or_abort(&bars.wdone, i & 1, &abort_flag, budget)) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < DK / 32; ++cb) {  // -W, rows s
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + RT_W + cb * 32, v);
+                if (crow >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = -v[j];
+                    store_row16x32(stg + Lay::OFF_W + (cb >> 1) * 8192, crow, (cb & 1) * 4, v);
+                }
+            }
+            tc::fence_async_smem();
+            rev_arrive(&bars.w_ready, lane);
+            if (!tc::mbar_wait_or_abort(&bars.pdone, i & 1, &abort_flag, budget)) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {  // P, row t, column s <= t
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + RT_P + cb * 32, v);
+                if (crow >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (cb * 32 + j > crow) v[j] = 0.f;
+                    store_row16x32(stg + Lay::OFF_P, crow, cb * 4, v);
+                }
+            }
+            tc::fence_async_smem();
+            rev_arrive(&bars.p_ready, lane);
+        }
+    } else if (wg == 2) {
+        // ---------------------------------------------------------- chain epilogue
+        bool done_all = true;
+        for (int i = 0; i < NC; ++i) {
+            const int n = NC - 1 - i;
+            if (!tc::mbar_wait_or_abort(&bars.d1done, i & 1, &abort_flag, budget)) { done_all = false; break; }
+            tc::tc_fence_after();
+            uint32_t wu[2][16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // dU'^T to fp16 in place, 32 tokens at a time
+                float u[32];
+                tc::tmem_ld32(tmem + lane_base + TM_U + h * 32, u);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) wu[h][j] = tc::pack_f16(u[2 * j], u[2 * j + 1]);
+                tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, wu[h]);  // over columns already read
+            }
+            rev_arrive(&bars.up_ready, lane);
+            if (vrow >= 0) {  // dU' of the chunk's tokens, fp16 [L][dv]
+                __half *dst = dU + ((size_t)bh * L + (size_t)n * C) * DV + vrow;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = 32 * h + 2 * j;
+                        const __half2 pr = *reinterpret_cast<const __half2 *>(&wu[h][j]);
+                        if (n * C + t < L) dst[(size_t)t * DV] = __low2half(pr);
+                        if (n * C + t + 1 < L) dst[(size_t)(t + 1) * DV] = __high2half(pr);
+                    }
+            }
+            if (!tc::mbar_wait_or_abort(&bars.d2done, i & 1, &abort_flag, budget)) { done_all = false; break; }
+            tc::tc_fence_after();
+            if (i + 1 < NC) {
+                // the state gradient after chunk n - 1: its fp16 copy for D1b, and to dSp
+                __half *dst = dSp + ((size_t)bh * NC + (n - 1)) * DD + (vrow >= 0 ? vrow : 0);
+#pragma unroll
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    float v[32];
+                    tc::tmem_ld32(tmem + lane_base + TM_S + cb * 32, v);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+                    tc::tmem_st16u(tmem + lane_base + RT_S16 + cb * 16, w);
+                    if (vrow >= 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const __half2 pr = *reinterpret_cast<const __half2 *>(&w[j]);
+                            dst[(size_t)(cb * 32 + 2 * j) * DV] = __low2half(pr);
+                            dst[(size_t)(cb * 32 + 2 * j + 1) * DV] = __high2half(pr);
+                        }
+                    }
+                }
+                rev_arrive(&bars.s_ready, lane);
+            }
+        }
+        if (done_all && dS0) {  // the gradient of the initial state
+#pragma unroll
+            for (int cb = 0; cb < DK / 16; ++cb) {
+                float v[16];
+                tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
+                if (vrow >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dS0[(size_t)bh * DD + (size_t)(cb * 16 + j) * DV + vrow] = v[j];
+                }
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && abort_flag) atomicOr(&g_bwd_error, 2u);
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ per chunk, in parallel
+// One CTA (8 warps) per chunk; every product on mma.sync (fp16 operands, fp32 accumulation)
+// out of 128-byte-swizzled fp16 tiles (64-column slabs of 128-byte rows, as the TMA lays them
+// out, so that ldmatrix reads are free of bank conflicts).
+namespace cw {
+constexpr int THREADS = 256;
+
+// Byte offset of element (r, c) (c a multiple of 8) in a tile of `rows` rows.
+__device__ __forceinline__ uint32_t off(int rows, int r, int c) {
+    return (uint32_t)((c >> 6) * rows * 128) + tc::sw128_off(r, (c & 63) >> 3);
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&d)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&d)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr));
+}
+__device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// An operand tile in shared memory: `rows` rows of 16-bit elements, row index first.
+struct Tile {
+    uint32_t base;  // shared address, 1024-aligned
+    int rows;
+};
+
+// acc[mt][nt] += A[m0 + 16 mt .., k] B[k, n0 + 8 nt ..] over k in [0, K), for one warp.
+// A_T = false: A's tile is [M][K] (row m); true: its tile is [K][M].  B_T = false: B's tile
+// is [N][K] (row n); true: [K][N].
+template <bool A_T, bool B_T, int MT, int NT>
+__device__ __forceinline__ void gemm(float (&acc)[MT][NT][4], Tile A, Tile B, int m0, int n0, int K, int lane) {
+    const int i = lane >> 3, r8 = lane & 7;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t a[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int mm = m0 + 16 * mt;
+            if (!A_T) ldsm4(a[mt], A.base + off(A.rows, mm + r8 + 8 * (i & 1), k0 + 8 * (i >> 1)));
+            else ldsm4t(a[mt], A.base + off(A.rows, k0 + 8 * (i >> 1) + r8, mm + 8 * (i & 1)));
+        }
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+            const int nn = n0 + 16 * np;
+            uint32_t b[4];  // {b0, b1} of n-tile 2 np, then of n-tile 2 np + 1
+            if (!B_T) ldsm4(b, B.base + off(B.rows, nn + 8 * (i >> 1) + r8, k0 + 8 * (i & 1)));
+            else ldsm4t(b, B.base + off(B.rows, k0 + 8 * (i & 1) + r8, nn + 8 * (i >> 1)));
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma(acc[mt][2 * np], a[mt], b[0], b[1]);
+                mma(acc[mt][2 * np + 1], a[mt], b[2], b[3]);
+            }
+        }
+    }
+}
+template <int MT, int NT>
+__device__ __forceinline__ void zero(float (&acc)[MT][NT][4]) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+}
+// Row and column of accumulator element e of tile (mt, nt) for this lane.
+__device__ __forceinline__ int acc_r(int m0, int mt, int e, int lane) { return m0 + 16 * mt + (lane >> 2) + 8 * (e >> 1); }
+__device__ __forceinline__ int acc_c(int n0, int nt, int e, int lane) { return n0 + 8 * nt + 2 * (lane & 3) + (e & 1); }
+
+// Store a warp's accumulators as fp16 into a tile ([rows][cols], row = accumulator row).
+template <int MT, int NT>
+__device__ __forceinline__ void store16(uint8_t *tile, int rows, const float (&acc)[MT][NT][4], int m0, int n0,
+                                        int lane) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = acc_r(m0, mt, 2 * h, lane), c = acc_c(n0, nt, 0, lane);
+                *reinterpret_cast<uint32_t *>(tile + off(rows, r, c & ~7) + 2 * (c & 7)) =
+                    tc::pack_f16(acc[mt][nt][2 * h], acc[mt][nt][2 * h + 1]);
+            }
+}
+
+// Fill a [rows][cols] fp16 tile from global memory (row stride ld elements), rows at or past
+// `valid` read as zero.  8 elements per thread and step.
+template <typename T>
+__device__ __forceinline__ void fill(uint8_t *tile, int rows, int cols, const T *src, size_t ld, int valid) {
+    const int per_row = cols / 8;
+    for (int e = threadIdx.x; e < rows * per_row; e += THREADS) {
+        const int r = e / per_row, c = (e - r * per_row) * 8;
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (r < valid) {
+            const T *p = src + (size_t)r * ld + c;
+            if constexpr (std::is_same<T, __half>::value) {
+                u = *reinterpret_cast<const uint4 *>(p);
+            } else if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(p);
+                u = make_uint4(tc::bf16x2_to_f16x2(x.x), tc::bf16x2_to_f16x2(x.y), tc::bf16x2_to_f16x2(x.z),
+                               tc::bf16x2_to_f16x2(x.w));
+            } else {
+                const float4 x0 = *reinterpret_cast<const float4 *>(p);
+                const float4 x1 = *reinterpret_cast<const float4 *>(p + 4);
+                u = make_uint4(tc::pack_f16(x0.x, x0.y), tc::pack_f16(x0.z, x0.w), tc::pack_f16(x1.x, x1.y),
+                               tc::pack_f16(x1.z, x1.w));
+            }
+        }
+        *reinterpret_cast<uint4 *>(tile + off(rows, r, c)) = u;
+    }
+}
+}  // namespace cw
+
+// Shared memory of the per-chunk kernel: fp16 tiles Q, K, dO, U', dU', -dR [64][d]; S, dS'
+// [dk][dv]; Ta, B, dP [64][64]; per-token a, df/dbeta, df/dlambda and the partial sums of da.
+template <int DK, int DV>
+struct ChunkLayout {
+    static constexpr int TQ = 0, TK = TQ + 128 * DK, TO = TK + 128 * DK, TU = TO + 128 * DV,
+                         TDU = TU + 128 * DV, TNR = TDU + 128 * DV, TS = TNR + 128 * DV,
+                         TDS = TS + 2 * DK * DV, TT = TDS + 2 * DK * DV, TB = TT + 8192, TP = TB + 8192,
+                         TEND = TP + 8192;
+    static constexpr int SMEM = TEND + 1024;  // + alignment slack
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(cw::THREADS, 1)
+    bwd_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                     const __nv_bfloat16 *__restrict__ v, const float4 *__restrict__ coef,
+                     const __half *__restrict__ dO16, const float *__restrict__ u_saved,
+                     const __half *__restrict__ dU, const float *__restrict__ ck_saved,
+                     const float *__restrict__ S0, const __half *__restrict__ dSp, const __half *__restrict__ ta,
+                     const int *__restrict__ hs, float *__restrict__ dq, float *__restrict__ dkey,
+                     float *__restrict__ dval, float *__restrict__ dbeta, int L, int NC) {
+    using Lay = ChunkLayout<DK, DV>;
+    using namespace cw;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+    uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    const uint32_t sb = tc::smem_u32(base);
+    __shared__ float sa[C], sfb[C], sfl[C], sda[2][4][C];  // sda: partials of da (2 kinds x 4 column groups)
+
+    const int chunk = blockIdx.x, bh = chunk / NC, n = chunk - bh * NC;
+    if (!head_ok(hs, bh)) return;  // this head walks on CUDA cores (uniform over the CTA)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = n * C, valid = min(C, L - t0);
+    const size_t DD = (size_t)DK * DV, tokq = (size_t)bh * L + t0;
+
+    // ---- operands into shared memory (fp16)
+    fill(base + Lay::TQ, C, DK, q + tokq * DK, DK, valid);
+    fill(base + Lay::TK, C, DK, k + tokq * DK, DK, valid);
+    fill(base + Lay::TO, C, DV, dO16 + tokq * DV, DV, valid);
+    fill(base + Lay::TU, C, DV, u_saved + tokq * DV, DV, valid);
+    fill(base + Lay::TDU, C, DV, dU + tokq * DV, DV, valid);
+    if (n > 0) fill(base + Lay::TS, DK, DV, ck_saved + ((size_t)bh * NC + n - 1) * DD, DV, DK);
+    else if (S0) fill(base + Lay::TS, DK, DV, S0 + (size_t)bh * DD, DV, DK);
+    else fill(base + Lay::TS, DK, DV, (const __half *)nullptr, DV, 0);
+    fill(base + Lay::TDS, DK, DV, dSp + ((size_t)bh * NC + n) * DD, DV, DK);
+    fill(base + Lay::TT, C, C, ta + (size_t)chunk * C * C, C, C);
+    if (tid < C) {
+        const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
+        sa[tid] = c.y;
+        sfb[tid] = c.z;
+        sfl[tid] = c.w;
+    }
+    __syncthreads();
+
+    const Tile tQ{sb + Lay::TQ, C}, tK{sb + Lay::TK, C}, tO{sb + Lay::TO, C}, tU{sb + Lay::TU, C};
+    const Tile tDU{sb + Lay::TDU, C}, tNR{sb + Lay::TNR, C}, tS{sb + Lay::TS, DK}, tDS{sb + Lay::TDS, DK};
+    const Tile tT{sb + Lay::TT, C}, tB{sb + Lay::TB, C}, tP{sb + Lay::TP, C};
+    // warp tile: rows m0 .. m0 + 31; columns n0 .. of a 64 x N output (N / 4 columns per warp)
+    const int m0 = 32 * (warp & 1), wc = warp >> 1;
+    constexpr int NV = DV / 32, NKK = DK / 32;  // n-tiles of 8 per warp for N = dv, N = dk
+
+    // ---- R = V - K S and dR = Ta^T dU' ([64][dv]); da's first part dR_t . R_t; dV = dR
+    {
+        float accR[2][NV][4], accD[2][NV][4];
+        zero(accR);
+        zero(accD);
+        const int n0 = wc * (DV / 4);
+        gemm<false, true>(accR, tK, tS, m0, n0, DK, lane);
+        gemm<true, true>(accD, tT, tDU, m0, n0, C, lane);
+        float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [mt][row half]
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NV; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
+                    const float vv = r < valid ? __bfloat162float(v[(tokq + r) * DV + c]) : 0.f;
+                    part[mt][e >> 1] += accD[mt][nt][e] * (vv - accR[mt][nt][e]);
+                    if (r < valid) dval[(tokq + r) * DV + c] = accD[mt][nt][e];
+                    accD[mt][nt][e] = -accD[mt][nt][e];
+                }
+        store16(base + Lay::TNR, C, accD, m0, n0, lane);  // -dR
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float x = part[mt][h];
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                if ((lane & 3) == 0) sda[0][wc][acc_r(m0, mt, 2 * h, lane)] = x;
+            }
+    }
+    __syncthreads();
+    // ---- G = K K^T, B = strictly-lower(-dR U'^T), dP = lower-incl(dO U'^T) ([64][64]);
+    // da's second part sum_s B_ts G_ts
+    {
+        float accG[2][2][4], accB[2][2][4];
+        zero(accG);
+        zero(accB);
+        const int n0 = wc * 16;
+        gemm<false, false>(accG, tK, tK, m0, n0, DK, lane);
+        gemm<false, false>(accB, tNR, tU, m0, n0, DV, lane);
+        float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
+                    if (c >= r) accB[mt][nt][e] = 0.f;
+                    part[mt][e >> 1] += accB[mt][nt][e] * accG[mt][nt][e];
+                }
+        store16(base + Lay::TB, C, accB, m0, n0, lane);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float x = part[mt][h];
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                if ((lane & 3) == 0) sda[1][wc][acc_r(m0, mt, 2 * h, lane)] = x;
+            }
+        float accP[2][2][4];
+        zero(accP);
+        gemm<false, false>(accP, tO, tU, m0, n0, DV, lane);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (acc_c(n0, nt, e, lane) > acc_r(m0, mt, e, lane)) accP[mt][nt][e] = 0.f;
+        store16(base + Lay::TP, C, accP, m0, n0, lane);
+    }
+    __syncthreads();
+    // ---- da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t;  dbeta = da df/dbeta
+    if (tid < C) {
+        const float s1 = sda[0][0][tid] + sda[0][1][tid] + sda[0][2][tid] + sda[0][3][tid];
+        const float s2 = sda[1][0][tid] + sda[1][1][tid] + sda[1][2][tid] + sda[1][3][tid];
+        const float da = tid < valid ? (s1 + s2) / sa[tid] : 0.f;
+        sa[tid] = da;  // from here on: da
+        if (tid < valid) dbeta[tokq + tid] = da * sfb[tid];
+    }
+    __syncthreads();
+    // ---- dQ = dO S^T + dP K ([64][dk])
+    const int n0k = wc * (DK / 4);
+    {
+        float acc[2][NKK][4];
+        zero(acc);
+        gemm<false, false>(acc, tO, tS, m0, n0k, DV, lane);
+        gemm<false, true>(acc, tP, tK, m0, n0k, C, lane);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NKK; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0k, nt, e, lane);
+                    if (r < valid) dq[(tokq + r) * DK + c] = acc[mt][nt][e];
+                }
+    }
+    // ---- dK = U' dS'^T + dP^T Q - dR S^T + B K + B^T K + 2 da (df/dlambda) K ([64][dk])
+    {
+        float acc[2][NKK][4];
+        zero(acc);
+        gemm<false, false>(acc, tU, tDS, m0, n0k, DV, lane);
+        gemm<true, true>(acc, tP, tQ, m0, n0k, C, lane);
+        gemm<false, false>(acc, tNR, tS, m0, n0k, DV, lane);
+        gemm<false, true>(acc, tB, tK, m0, n0k, C, lane);
+        gemm<true, true>(acc, tB, tK, m0, n0k, C, lane);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NKK; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0k, nt, e, lane);
+                    if (r < valid) {
+                        const float kk = __bfloat162float(k[(tokq + r) * DK + c]);
+                        dkey[(tokq + r) * DK + c] = acc[mt][nt][e] + 2.f * sa[r] * sfl[r] * kk;
+                    }
+                }
+    }
+}
+
+// dO (fp32) to fp16 for the products; and which heads take the tensor-core path.
+__global__ void __launch_bounds__(256) bwd_prepare_kernel(const float *__restrict__ dO, __half *__restrict__ dO16,
+                                                         size_t n4) {
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (size_t)gridDim.x * blockDim.x) {
+        const float4 x = reinterpret_cast<const float4 *>(dO)[e];
+        reinterpret_cast<uint2 *>(dO16)[e] = make_uint2(tc::pack_f16(x.x, x.y), tc::pack_f16(x.z, x.w));
+    }
+}
+
+template <int DK, int DV>
+cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const float *S0, const float *dO,
+                            const float *dSL, const float4 *coef, const int *hs, const float *u_saved,
+                            const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                            float *dbeta, float *dS0, int B, int H, int L, void *ws, cudaStream_t s) {
+    const int BH = B * H, NC = (L + C - 1) / C;
+    const size_t ntok = (size_t)BH * L;
+    __half *dO16 = (__half *)ws;
+    __half *dU = dO16 + ntok * DV;
+    __half *dSp = dU + ntok * DV;
+    static bool attr_done[64] = {};
+    int dev = 0, nsm = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        e = cudaFuncSetAttribute(bwd_state_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 RevLayout<DK, DV>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_chunk_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     ChunkLayout<DK, DV>::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    CUtensorMap mq, mk, mo, mt;
+    if (!tmap::make_3d(&mq, q, DK, L, BH, 64, C) || !tmap::make_3d(&mk, k, DK, L, BH, 64, C) ||
+        !tmap::make_3d(&mo, dO16, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !tmap::make_2d(&mt, ta, C, (uint64_t)BH * NC * C, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
+    const size_t n4 = ntok * DV / 4;
+    const int g = (int)std::min<size_t>((n4 + 255) / 256, (size_t)nsm * 16);
+    bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
+    bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, dSL, dU, dSp, dS0,
+                                                                              hs, L, NC);
+    bwd_chunk_kernel<DK, DV><<<BH * NC, cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, dO16, u_saved, dU,
+        ck_saved, S0, dSp, (const __half *)ta, hs, dq, dkey, dval, dbeta, L, NC);
+    count_launches(3);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_tc_workspace_bytes(int B, int H, int L, int dk, int dv) {
+    const size_t BH = (size_t)B * H, NC = (size_t)(L + C - 1) / C;
+    return (2 * BH * (size_t)L * dv + BH * NC * (size_t)dk * dv) * sizeof(__half);
+}
+
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *S0, const float *dO,
+                          const float *dSL, const void *coef, const int *hs, const float *u_saved,
+                          const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                          float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
+                          cudaStream_t s) {
+    const float4 *cf = (const float4 *)coef;
+    if (dk == 128 && dv == 128)
+        return launch_bwd_tc_t<128, 128>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
+                                         dS0, B, H, L, ws, s);
+    if (dk == 128 && dv == 64)
+        return launch_bwd_tc_t<128, 64>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
+                                        dS0, B, H, L, ws, s);
+    if (dk == 64 && dv == 128)
+        return launch_bwd_tc_t<64, 128>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
+                                        dS0, B, H, L, ws, s);
+    return launch_bwd_tc_t<64, 64>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
+                                   dS0, B, H, L, ws, s);
+}
+
+cudaError_t bwd_tc_read_and_clear_error(unsigned int *out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_bwd_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_bwd_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace efla

@@ -69,6 +69,19 @@ int chunk_fwd_entry(const void *q, const void *k, const void *v, const void *bet
 cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
                                  const float *S0, int B, int H, int L, int dk, int dv, bool euler,
                                  void *ws, float *u_out, float *ck_out, cudaStream_t s);
+// The backward on tensor cores for the heads the saved-forward gate lets through (bf16, chunk
+// 64, dk and dv in {64, 128}, q, k, dO and S0 16-byte aligned): dO to fp16, the reverse chain
+// over the chunks (dU' of every token and the state gradient after every chunk), then every
+// chunk's dq, dk, dv and dbeta in parallel; dS0 from the chain.  coef: the coefficient
+// kernel's per-token float4 pairs; hs: its per-head gate statistics; u_saved, ck_saved, ta: the
+// saving forward's outputs and Ta tiles.  Workspace: bwd_tc_workspace_bytes.
+size_t bwd_tc_workspace_bytes(int B, int H, int L, int dk, int dv);
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *S0, const float *dO,
+                          const float *dSL, const void *coef, const int *hs, const float *u_saved,
+                          const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                          float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
+                          cudaStream_t s);
+cudaError_t bwd_tc_read_and_clear_error(unsigned int *out);
 // A kernel whose one bounded wait runs out (nothing arrives): records a timeout, then returns.
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits): read and clear.

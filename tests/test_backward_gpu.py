@@ -2,9 +2,10 @@
 element on the same seeded inputs, for both rules, fp32 and bf16 inputs, ragged lengths and
 nonzero initial states; and the autograd wrapper end to end.
 
-Bounds: max|g_gpu - g_oracle| / RMS(g_oracle) <= 1e-3 for fp32 inputs (the kernel recomputes
-the forward in fp32 and walks each 64-token block back from its stored state) and <= 2e-2 for
-bf16 inputs; the oracle sees the dtype-rounded inputs.
+Bounds: max|g_gpu - g_oracle| / RMS(g_oracle) <= 1e-4 for fp32 inputs (the kernel recomputes
+the forward in fp32 and walks each 64-token block back from its stored state; measured up to
+2.2e-5, on the long stiff distribution) and <= 2e-2 for bf16 inputs, the forward's bounds; the
+oracle sees the dtype-rounded inputs.
 """
 import numpy as np
 import pytest
@@ -15,7 +16,7 @@ from delta_rule_linear_efla_b200 import efla, inputs
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"fp32": 1e-3, "bf16": 2e-2}
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
 
 
 def _case(wid, rule, seed=5, **kw):
@@ -173,4 +174,45 @@ def test_backward_at_the_edge_of_the_saved_forward_gate(oracle_mod):
     ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], dO, x["S0"], None)
     for name, gg, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
         e = rel_err(gg.cpu().numpy(), r)
+        assert e <= TOL["bf16"], (name, e)
+
+
+@pytest.mark.parametrize("rule", ["exact", "euler"])
+@pytest.mark.parametrize("kw", [dict(B=2, H=2, L=260, dk=64, dv=64), dict(B=1, H=3, L=129, dk=64, dv=128),
+                                dict(B=1, H=2, L=64, dk=128, dv=128), dict(B=1, H=1, L=1, dk=128, dv=64)])
+def test_backward_tensor_core_path(oracle_mod, rule, kw):
+    """bf16 heads the saved-forward gate lets through take the tensor-core backward: the reverse
+    chain over the chunks (dU' of every token, the state gradient after every chunk) and the
+    per-chunk gradients; ragged tails, a single token, nonzero S0 and dS_final, every head size
+    the tensor cores take."""
+    x = _case(4, rule, **kw)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    got = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"], rule=rule)
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], x["dO"], x["S0"], x["dS"], rule=rule)
+    for name, g, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+        e = rel_err(g.cpu().numpy(), r)
+        assert e <= TOL["bf16"], (name, e)
+
+
+def test_backward_element_aligned_inputs_walk_on_cuda_cores(oracle_mod):
+    """bf16 inputs that are only 2-byte aligned (views one element into a buffer) cannot be read
+    16 bytes at a time: every head takes the CUDA-core path, with the same results' bound."""
+    x = _case(4, "exact", B=1, H=2, L=100)
+    d = {}
+    for n, t in x.items():
+        if isinstance(t, torch.Tensor) and n in ("q", "k", "v"):
+            buf = torch.empty(t.numel() + 1, dtype=t.dtype, device="cuda")
+            buf[1:].copy_(t.reshape(-1).cuda())
+            d[n] = buf[1:].view(t.shape)
+            assert d[n].data_ptr() % 16 != 0
+        else:
+            d[n] = t.cuda() if isinstance(t, torch.Tensor) else t
+    got = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], x["dO"], x["S0"], x["dS"])
+    for name, g, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+        e = rel_err(g.cpu().numpy(), r)
         assert e <= TOL["bf16"], (name, e)
