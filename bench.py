@@ -1,13 +1,15 @@
 """Benchmark of the EFLA forward hot path on B200.
 
 One step = one pass of the whole hot path over one batch of the 1.3B-LM-shaped
-workload: the chunkwise forward (B=4, H=16, L=4096, dk=dv=128, chunk=64, bf16)
-followed by the recurrent decode step of its decode batch (B=64, H=16, one
-token each, fp32 carried state).  Throughput is token-heads per second
+workload: the chunkwise forward (B=4, H=16, L=4096, dk=dv=128, chunk=64, bf16,
+o written at the input dtype unless --o-dtype fp32) followed by the recurrent
+decode step of its decode batch (B=64, H=16, one token each, fp32 carried
+state).  Throughput is token-heads per second
 (B*H*L + B_dec*H_dec per step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload 3|4|5] [--no-e2e] [--no-cpu-baseline]
+                    [--o-dtype input|fp32] [--gated] [--rule exact|euler] [--pass fwd|bwd]
 
 Under torchrun (WORLD_SIZE > 1) every rank runs its own replica of the workload
 on disjoint heads (seeded per rank): heads are independent, so there is no
@@ -103,9 +105,12 @@ def run_bwd(args) -> None:
         "metric": "EFLA bwd tokens/s per GPU (B*H*L/time) and % of binding roofline", "value":
         w.token_heads / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic", "config": _config(w),
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": _config(w),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm"], "traffic": None, "kernel": "efla_bwd (SIMT: coefficients, column-block sweeps, share sum)",
+                     "frac": achieved / peaks["hbm"], "traffic": None,
+                     "kernel": "efla_bwd (bf16 heads the saved-forward gate admits: the saving tensor-core "
+                               "forward, the reverse chain over chunks on tcgen05, per-chunk gradients on "
+                               "mma.sync; other heads: the fp32 column-block walk on CUDA cores)",
                      "alg_bytes_per_launch": alg, "avg_launch_ms": ms},
         "gpu_launches": int(launches), "clocks": clocks}))
 
@@ -173,7 +178,7 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-FWD_SOURCES = ("chunk_tc.cu", "common.cuh", "tc_ptx.cuh")
+FWD_SOURCES = ("chunk_tc.cu", "common.cuh", "tc_ptx.cuh", "tmap.h")
 
 
 def kernel_source_hash() -> str:
@@ -188,9 +193,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(w) -> int | None:
+def profiled_traffic(w, o_dtype) -> int | None:
     """DRAM bytes of one efla_chunk_fwd call from the committed ncu capture, if it was taken on
-    this workload and on the current kernel sources; None otherwise."""
+    this workload, with this output dtype and on the current kernel sources; None otherwise."""
     if w.id != 4:
         return None
     p = os.path.join(ROOT, "profiles", "dram_traffic_lm1p3b.txt")
@@ -202,7 +207,7 @@ def profiled_traffic(w) -> int | None:
         if "=" in line:
             k, v = (x.strip() for x in line.split("=", 1))
             kv[k] = v
-    if kv.get("source_hash") != kernel_source_hash():
+    if kv.get("source_hash") != kernel_source_hash() or kv.get("o_dtype", "fp32") != _o_name(o_dtype):
         return None
     return int(kv["chunk_fwd_bytes"])
 
@@ -283,6 +288,7 @@ def run_reference(args) -> None:
 
 RULE = "exact"  # set from --rule: "exact" (the method) or "euler" (the delta rule, for comparison)
 GATED = False  # set from --gated: the gated form, a per-token decay g_t ~ sigmoid(N(2, 1))
+O_DT = "input"  # set from --o-dtype: o at the input dtype (default) or fp32
 
 
 def _with_gate(x: dict, seed: int) -> dict:
@@ -292,12 +298,22 @@ def _with_gate(x: dict, seed: int) -> dict:
     return x
 
 
+def _o_dtype(w):
+    """The output dtype of the timed calls: the input dtype by default (o at the input dtype, as
+    the algorithmic byte count has it), fp32 with --o-dtype fp32."""
+    return torch.float32 if (O_DT == "fp32" or w.dtype != "bf16") else torch.bfloat16
+
+
+def _o_name(dt) -> str:
+    return "fp32" if dt == torch.float32 else "bf16"
+
+
 def _config(w) -> dict:
     c = {"workload": "%s (B=%d H=%d L=%d dk=%d dv=%d chunk=%d %s)" % (
         w.name, w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.dtype),
         "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
         "l2": "inputs > L2 (126 MB): two rotating input sets per rank",
-        "o_dtype": "fp32", "rule": RULE}
+        "o_dtype": _o_name(_o_dtype(w)), "rule": RULE}
     if GATED:
         c["gate"] = "g_t ~ sigmoid(N(2, 1)) per token: S_t = g_t (I - a k k^T) S + a k v^T"
     if w.decode:
@@ -384,12 +400,12 @@ def run_ours(args) -> None:
         x = _with_gate(inputs.make_inputs(w, seed=edist.replica_seed(1000 + w.id, rank, r)),
                        edist.replica_seed(600, rank, r))
         sets.append({k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()})
-    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
+    odt = _o_dtype(w)
+    o_buf = [torch.empty((w.B, w.H, w.L, w.dv), dtype=odt, device=dev) for _ in range(2)]
     Sf_buf = [torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
-    ws_bytes = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(),
-                                   torch.float32)
+    ws_bytes = efla.workspace_size(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(), odt)
     wsp = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    path = efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype())
+    path = efla.chunk_fwd_path(w.B, w.H, w.L, w.dk, w.dv, w.chunk, w.torch_dtype(), odt)
 
     dec = None
     if w.decode:
@@ -404,7 +420,7 @@ def run_ours(args) -> None:
             dd["g"] = inputs.make_gate((w.decode["B"], w.decode["H"]), w.torch_dtype(), 700 + rank).to(dev)
         dd["S_init"] = S_carry
         dd["S"] = [S_carry.clone(), S_carry.clone()]
-        dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=torch.float32, device=dev)
+        dd["o"] = torch.empty((w.decode["B"], w.decode["H"], w.dv), dtype=odt, device=dev)
         dec = dd
     tok_dec = (w.decode["B"] * w.decode["H"]) if w.decode else 0
     tok_step = w.token_heads + tok_dec
@@ -452,8 +468,8 @@ def run_ours(args) -> None:
         raise RuntimeError("device error word set: %s" % efla.status_str(err))
 
     value = edist.aggregate_rate(tok_step, args.steps, ws, ms)
-    roofline = _roofline(w, chunk_ms, peaks, path)
-    roofline["traffic"] = profiled_traffic(w)
+    roofline = _roofline(w, chunk_ms, peaks, path, odt)
+    roofline["traffic"] = profiled_traffic(w, odt)
     roofline["source_hash"] = kernel_source_hash()
 
     # ---- end to end through the public API with host buffers ----
@@ -461,7 +477,7 @@ def run_ours(args) -> None:
     if not args.no_e2e:
         xh = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v)
               for k, v in _with_gate(inputs.make_inputs(w, seed=4242 + rank), 4343 + rank).items()}
-        o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32).pin_memory()
+        o_host = torch.empty((w.B, w.H, w.L, w.dv), dtype=odt).pin_memory()
         S_host = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
         names = ("q", "k", "v", "beta") + (("g",) if GATED else ())
         h2d = sum(xh[k].numel() * xh[k].element_size() for k in names)
@@ -541,11 +557,13 @@ def run_ours(args) -> None:
         per_workload = {}
         for wid in (3, 4, 5):
             if wid != w.id:
-                per_workload[str(wid)] = time_chunk_fwd(inputs.WORKLOADS[wid], dev, peaks, args.steps)
-        # the headline workload with o rounded to the input dtype (bf16), the output the
-        # algorithmic byte count assumes
-        per_workload["%d_o_bf16" % w.id] = time_chunk_fwd(w, dev, peaks, args.steps,
-                                                         o_dtype=torch.bfloat16)
+                ow = inputs.WORKLOADS[wid]
+                per_workload[str(wid)] = time_chunk_fwd(ow, dev, peaks, args.steps, o_dtype=_o_dtype(ow))
+        # the headline workload with the other output dtype
+        other = torch.float32 if odt == torch.bfloat16 else torch.bfloat16
+        if w.dtype == "bf16":
+            per_workload["%d_o_%s" % (w.id, _o_name(other))] = time_chunk_fwd(
+                w, dev, peaks, args.steps, o_dtype=other)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -582,6 +600,9 @@ def main():
                     help="the gated form: a per-token decay g_t ~ sigmoid(N(2, 1)) on the carried state")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip timing the other workloads' chunk forward after the timed region")
+    ap.add_argument("--o-dtype", choices=["input", "fp32"], default="input",
+                    help="output dtype of the timed chunk forward and decode: the input dtype "
+                         "(default; the algorithmic byte count's o) or fp32")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd (default): the forward step; bwd: the backward pass alone")
     ap.add_argument("--rule", choices=["exact", "euler"], default="exact",
@@ -589,9 +610,10 @@ def main():
                          "for the throughput comparison (the workload's keys are not normalised, "
                          "so under euler only the time is meaningful)")
     args = ap.parse_args()
-    global RULE, GATED
+    global RULE, GATED, O_DT
     RULE = args.rule
     GATED = args.gated
+    O_DT = args.o_dtype
     if args.warmup < 3:
         args.warmup = 3
     if args.gated and args.pass_ == "bwd":
