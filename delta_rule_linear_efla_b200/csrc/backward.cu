@@ -23,10 +23,10 @@
 // The per-token coefficients and the two dot products that link a pair's tokens come from a
 // prologue kernel.
 //
-// With bf16 inputs at the tensor-core sizes, the tensor-core forward runs first and saves every
-// token's u = a r and the state after every 64-token chunk; heads that pass an accuracy gate
-// (moderate key norms, see saved_ok in bwd_cols_kernel) then skip the forward sweep and take
-// r = u / a and the block states from it.
+// With bf16 inputs at the tensor-core sizes (16-byte aligned), the heads that pass an accuracy
+// gate (bwd_gate.cuh: moderate key norms) take the tensor-core backward instead (bwd_tc.cu: the
+// tensor-core forward saves every token's u and the state after every 64-token chunk, then a
+// reverse chain over the chunks and per-chunk products); this walk takes the other heads.
 #include <algorithm>
 #include <cstdint>
 
@@ -137,72 +137,197 @@ __device__ __forceinline__ void store_row16(float *p, const float *x) {
 // Per token t, two float4: (lambda = |k_t|^2, a_t, df/dbeta, df/dlambda) and
 // (q_t . k_t, k_t . k_{t-1}, 0, 0) (k_{-1} = 0); one warp per token.  Every column block of a
 // head reads them, so they are computed once, ahead of the sweeps.  It also gathers, per head,
-// what decides whether the reverse sweep may take r = u / a from the tensor-core forward's u (see
-// saved_ok below): hs[head] = {a token has a <= 0 (or NaN); max lambda (float bits); INT_MAX - min a
-// (float bits); max a (float bits)}, every field zero-initialised (a >= 0, lambda >= 0, so the
-// bit patterns order as the values do).
+// what decides whether the head takes the tensor-core forward's saved values (bwd_gate.cuh):
+// hs[head] = {a token has a <= 0 (or NaN); max lambda (float bits); INT_MAX - min a (float bits);
+// max a (float bits)}, every field zero-initialised (a >= 0, lambda >= 0, so the bit patterns
+// order as the values do).
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                        const T *__restrict__ beta, size_t ntok, int L,
                                                        int dk, bool euler, float4 *__restrict__ coef,
                                                        int *__restrict__ hs) {
+    // Work units of up to 64 tokens within one head, one warp each.  The warp computes the dot
+    // products of 32 tokens at a time (8 tokens' rows loaded at once, lane i holding elements
+    // i, i + 32, ... of a row) and hands token j's sums to lane j, so the coefficients of the
+    // 32 tokens are computed by the 32 lanes side by side; the head's gate statistics are
+    // reduced over the warp and added to hs once per unit.
+    constexpr int UNIT = 64, RJ = 4;  // dk <= 128
     const int lane = threadIdx.x & 31;
-    for (size_t tok = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); tok < ntok; tok += (size_t)gridDim.x * 8) {
-        const bool first = tok % (size_t)L == 0;
-        float lam = 0.f, qk = 0.f, kk = 0.f;
-        for (int i = lane; i < dk; i += 32) {
-            const float x = to_f32(k[tok * dk + i]);
-            lam = fmaf(x, x, lam);
-            qk = fmaf(to_f32(q[tok * dk + i]), x, qk);
-            if (!first) kk = fmaf(to_f32(k[(tok - 1) * dk + i]), x, kk);
+    const long long BH = (long long)(ntok / (size_t)L), upH = (L + UNIT - 1) / UNIT;
+    const long long nw = (long long)gridDim.x * 8, w0 = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    for (long long u = w0; u < BH * upH; u += nw) {
+        const long long head = u / upH;
+        const int r0 = (int)(u % upH) * UNIT, r1 = min(L, r0 + UNIT);
+        const size_t hb = (size_t)head * L;
+        int bad = 0, m_lam = 0, m_ia = 0, m_a = 0;
+        float kprev[RJ];  // k of the token before the current one (0 before the head's first)
+#pragma unroll
+        for (int e = 0; e < RJ; ++e) {
+            const int i = lane + 32 * e;
+            kprev[e] = (r0 > 0 && i < dk) ? to_f32(k[(hb + r0 - 1) * dk + i]) : 0.f;
         }
-        lam = warp_sum(lam);
-        qk = warp_sum(qk);
-        kk = warp_sum(kk);
+        for (int g0 = r0; g0 < r1; g0 += 32) {
+            float mylam = 0.f, myqk = 0.f, mykk = 0.f;
+            for (int b0 = 0; b0 < 32 && g0 + b0 < r1; b0 += 8) {
+                float kx[8][RJ], qx[8][RJ];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                    for (int e = 0; e < RJ; ++e) {
+                        const int t = g0 + b0 + j, i = lane + 32 * e;
+                        const bool in = t < r1 && i < dk;
+                        kx[j][e] = in ? to_f32(k[(hb + t) * dk + i]) : 0.f;
+                        qx[j][e] = in ? to_f32(q[(hb + t) * dk + i]) : 0.f;
+                    }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float lam = 0.f, qk = 0.f, kk = 0.f;
+#pragma unroll
+                    for (int e = 0; e < RJ; ++e) {
+                        const float kp = j == 0 ? kprev[e] : kx[j - 1][e];
+                        lam = fmaf(kx[j][e], kx[j][e], lam);
+                        qk = fmaf(qx[j][e], kx[j][e], qk);
+                        kk = fmaf(kp, kx[j][e], kk);
+                    }
+                    lam = warp_sum(lam);
+                    qk = warp_sum(qk);
+                    kk = warp_sum(kk);
+                    if (lane == b0 + j) {
+                        mylam = lam;
+                        myqk = qk;
+                        mykk = g0 + b0 + j == 0 ? 0.f : kk;  // k_{-1} = 0
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < RJ; ++e) kprev[e] = kx[7][e];
+            }
+            const int t = g0 + lane;
+            if (t < r1) {
+                const size_t tok = hb + t;
+                const float bt = to_f32(beta[tok]);
+                const float a = alpha_rule(mylam, bt, euler);
+                float dfdb, dfdl;
+                coeff_grads(mylam, bt, euler, a, dfdb, dfdl);
+                coef[2 * tok] = make_float4(mylam, a, dfdb, dfdl);
+                coef[2 * tok + 1] = make_float4(myqk, mykk, 0.f, 0.f);
+                // a zero a (u / a cannot give r), a negative one (from a negative beta) or NaN
+                // would also escape the min/max statistics, whose integer order holds for
+                // positive floats only: all of them send the head to the fp32 walk
+                if (!(a > 0.f)) bad = 1;
+                m_lam = max(m_lam, __float_as_int(mylam));
+                m_ia = max(m_ia, 0x7fffffff - __float_as_int(a));
+                m_a = max(m_a, __float_as_int(a));
+            }
+        }
+        bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            m_lam = max(m_lam, __shfl_xor_sync(0xffffffffu, m_lam, o));
+            m_ia = max(m_ia, __shfl_xor_sync(0xffffffffu, m_ia, o));
+            m_a = max(m_a, __shfl_xor_sync(0xffffffffu, m_a, o));
+        }
         if (lane == 0) {
-            const float bt = to_f32(beta[tok]);
-            const float a = alpha_rule(lam, bt, euler);
-            float dfdb, dfdl;
-            coeff_grads(lam, bt, euler, a, dfdb, dfdl);
-            coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
-            coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
-            int *h = hs + 4 * (tok / (size_t)L);
-            // u / a cannot give this head's r when a is zero; a negative a (from a negative beta)
-            // or NaN would also escape the min/max statistics below, whose integer order holds for
-            // positive floats only: all of them send the head to the fp32 walk
-            if (!(a > 0.f)) atomicOr(h, 1);
-            atomicMax(h + 1, __float_as_int(lam));
-            atomicMax(h + 2, 0x7fffffff - __float_as_int(a));
-            atomicMax(h + 3, __float_as_int(a));
+            int *h = hs + 4 * head;
+            if (bad) atomicOr(h, 1);
+            atomicMax(h + 1, m_lam);
+            atomicMax(h + 2, m_ia);
+            atomicMax(h + 3, m_a);
         }
     }
 }
 
-// Tokens go through both sweeps in pairs, with one CTA-wide sum per pair.  Forward, for the
-// pair (t, t+1) from S = S_{t-1}: the sum gives y0 = S^T k_t and y1 = S^T k_{t+1}; then
-//   r_t = v_t - y0,  r_{t+1} = v_{t+1} - (y1 + a_t (k_t . k_{t+1}) r_t),
-//   S += a_t k_t r_t^T + a_{t+1} k_{t+1} r_{t+1}^T.
-// Reverse, for the pair (t, t-1) from S = S_t and G = dL/dS_t without token t's own q do^T:
-// G1 = G + q_t do_t^T; the sum gives du_t = G1^T k_t and z = G1^T k_{t-1}; token t's step
-// (above) makes G2 = G1 - a_t k_t du_t^T, and then
-//   du_{t-1} = (G2 + q_{t-1} do_{t-1}^T)^T k_{t-1}
-//            = z - a_t (k_t . k_{t-1}) du_t + (q_{t-1} . k_{t-1}) do_{t-1}.
-// Pairs are aligned to even token offsets in each 64-token block; a block with an odd count
-// (the last one) pairs its last token with an absent one, whose k, q, v, dO, r and
-// coefficients are all zero, so that it changes nothing.
-//
-// Workspace: the coefficients [B*H][L][2] (float4); per (head, column block) r of every token
-// [L][16], then the block's state at every 64-token boundary and at the end [NB + 1][dk][16];
-// after all of those the column blocks' shares of dq and dk ([NS][B*H][L][dk] each) and of
-// dbeta ([NS][B*H][L]).
+// The same for bf16 rows of 64 or 128 elements, 16-byte aligned: eight lanes per token (16-byte
+// loads, a row's dot products summed over the eight), four tokens per warp at a time, and the
+// coefficients of a token computed by the first lane of its eight.
+template <int DKV>
+__global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                           const __nv_bfloat16 *__restrict__ k,
+                                                           const __nv_bfloat16 *__restrict__ beta, size_t ntok,
+                                                           int L, bool euler, float4 *__restrict__ coef,
+                                                           int *__restrict__ hs) {
+    constexpr int UNIT = 64, EPL = DKV / 8, NV = EPL / 8;  // elements and 16-byte words per lane
+    const int lane = threadIdx.x & 31, g = lane >> 3, sl = lane & 7;
+    const long long BH = (long long)(ntok / (size_t)L), upH = (L + UNIT - 1) / UNIT;
+    const long long nw = (long long)gridDim.x * 8, w0 = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    auto dot = [](const uint4 &a, const uint4 &b) {
+        const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 u = __bfloat1622float2(x[e]), v = __bfloat1622float2(y[e]);
+            s = fmaf(u.x, v.x, fmaf(u.y, v.y, s));
+        }
+        return s;
+    };
+    for (long long u = w0; u < BH * upH; u += nw) {
+        const long long head = u / upH;
+        const int r0 = (int)(u % upH) * UNIT, r1 = min(L, r0 + UNIT);
+        const size_t hb = (size_t)head * L;
+        int bad = 0, m_lam = 0, m_ia = 0, m_a = 0;
+        for (int t = r0 + g; t - g < r1; t += 4) {
+            const bool in = t < r1;
+            const size_t tok = hb + (in ? t : r0);
+            uint4 kx[NV], qx[NV], kp[NV];
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                const size_t o = tok * DKV + (size_t)sl * EPL + 8 * w;
+                kx[w] = *reinterpret_cast<const uint4 *>(k + o);
+                qx[w] = *reinterpret_cast<const uint4 *>(q + o);
+                kp[w] = (in && t > 0) ? *reinterpret_cast<const uint4 *>(k + o - DKV) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float lam = 0.f, qk = 0.f, kk = 0.f;
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                lam += dot(kx[w], kx[w]);
+                qk += dot(qx[w], kx[w]);
+                kk += dot(kp[w], kx[w]);
+            }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                lam += __shfl_xor_sync(0xffffffffu, lam, o);
+                qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            }
+            if (in && sl == 0) {
+                const float bt = __bfloat162float(beta[tok]);
+                const float a = alpha_rule(lam, bt, euler);
+                float dfdb, dfdl;
+                coeff_grads(lam, bt, euler, a, dfdb, dfdl);
+                coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
+                coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
+                // see bwd_coeff_kernel: any a that is not positive fails the gate
+                if (!(a > 0.f)) bad = 1;
+                m_lam = max(m_lam, __float_as_int(lam));
+                m_ia = max(m_ia, 0x7fffffff - __float_as_int(a));
+                m_a = max(m_a, __float_as_int(a));
+            }
+        }
+        bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            m_lam = max(m_lam, __shfl_xor_sync(0xffffffffu, m_lam, o));
+            m_ia = max(m_ia, __shfl_xor_sync(0xffffffffu, m_ia, o));
+            m_a = max(m_a, __shfl_xor_sync(0xffffffffu, m_a, o));
+        }
+        if (lane == 0) {
+            int *h = hs + 4 * head;
+            if (bad) atomicOr(h, 1);
+            atomicMax(h + 1, m_lam);
+            atomicMax(h + 2, m_ia);
+            atomicMax(h + 3, m_a);
+        }
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(BW_THREADS, 4)
     bwd_cols_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float4 *__restrict__ coef, const float *__restrict__ S0,
                     const float *__restrict__ dO, const float *__restrict__ dSL,
                     float *__restrict__ dval, float *__restrict__ dS0, int L, int dk, int dv, int NS,
-                    float *__restrict__ ws, float *__restrict__ part, const float *__restrict__ u_saved,
-                    const float *__restrict__ ck_saved, const int *__restrict__ hs, bool tc_heads) {
+                    float *__restrict__ ws, float *__restrict__ part, const int *__restrict__ hs,
+                    bool tc_heads) {
     __shared__ __align__(16) BwdRed red;
     __shared__ __align__(16) float xb[BWD_BLOCK][BW_CB];  // v (forward sweep) or dO (reverse)
     __shared__ __align__(16) float rb[BWD_BLOCK][BW_CB];  // r (reverse sweep)
@@ -220,18 +345,9 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     float *pdq = part + (size_t)s * nq + tk;
     float *pdk = part + (size_t)NS * nq + (size_t)s * nq + tk;
     float *pdb = part + 2 * (size_t)NS * nq + (size_t)s * BH * L + tb;
-    // The tensor-core forward may have saved every token's u = a r and the state after every
-    // 64-token block: then this sweep's forward half is not needed.  u carries the fp16 operand
-    // rounding of the chunk products, an absolute error at the scale of the chunk's largest u;
-    // r = u / a divides it by a, so a token whose a is small next to its neighbours' gets a
-    // large relative error in r (and in dbeta).  Emulating those roundings, the error grows with
-    // the keys' squared norm (dbeta's max error over its RMS: 0.007 with ||k||^2 up to 16,
-    // 0.013 up to 32, 0.032 for the stiff inputs with ||k||^2 up to 100) far more than with the
-    // spread of a from small betas (0.006 at a max/min ratio of 800).  So the saved values are
-    // used only for heads whose largest ||k||^2 is at most 16, whose a spans at most a factor of
-    // 1024, and whose a are all positive; other heads walk the forward in fp32 themselves (saved_ok).
-    const bool saved_ok = u_saved != nullptr && head_takes_saved(hs, bh);
-    if (saved_ok && tc_heads) return;  // the tensor-core backward takes this head
+    // With tc_heads, the heads the gate admits (bwd_gate.cuh) take the tensor-core backward; this
+    // kernel walks the others (uniform over the CTA: one head per CTA).
+    if (tc_heads && head_takes_saved(hs, bh)) return;
     auto ld = [&](const T *x, int t) {  // row `row` of token t's q or k (0 off the sequence)
         return (act && t >= 0 && t < L) ? to_f32(x[tk + (size_t)t * dk + row]) : 0.f;
     };
@@ -244,10 +360,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             const size_t g = tv + (size_t)(t0 + tt) * dv + c0 + j;
             if (reverse) {
                 xb[tt][j] = in ? dO[g] : 0.f;
-                if (saved_ok)
-                    rb[tt][j] = in ? u_saved[g] / coef[2 * (tb + t0 + tt)].y : 0.f;
-                else
-                    rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
+                rb[tt][j] = tt < cnt ? R[(size_t)(t0 + tt) * BW_CB + j] : 0.f;
             } else {
                 xb[tt][j] = in ? to_f32(v[g]) : 0.f;
             }
@@ -264,7 +377,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     // ---- forward sweep: r of every token and the block-boundary states
     int par = 0;
     float kn0 = ld(k, 0), kn1 = ld(k, 1);  // k rows of the next pair
-    for (int b = 0; b < (saved_ok ? 0 : NB); ++b) {
+    for (int b = 0; b < NB; ++b) {
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb and cb are done
         stage(t0, cnt, false);
@@ -307,7 +420,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
             par ^= 1;
         }
     }
-    if (act && !saved_ok) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
+    if (act) store_row16(CK + ((size_t)NB * dk + row) * BW_CB, S);
 
     // ---- reverse sweep
 #pragma unroll
@@ -322,12 +435,7 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
         const int t0 = b * BWD_BLOCK, cnt = min(BWD_BLOCK, L - t0);
         __syncthreads();  // the previous block's reads of xb, rb and cb are done
         stage(t0, cnt, true);
-        if (act) {  // S' after the block
-            if (saved_ok)
-                load_row16(ck_saved + (((size_t)bh * NB + b) * dk + row) * dv + c0, S);
-            else
-                load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);
-        }
+        if (act) load_row16(CK + ((size_t)(b + 1) * dk + row) * BW_CB, S);  // S' after the block
         __syncthreads();
         for (int tt = cnt - 1 + (cnt & 1); tt > 0; tt -= 2) {  // pair (t, t-1), t = t0 + tt
             const int t = t0 + tt;
@@ -432,8 +540,8 @@ __global__ void __launch_bounds__(BW_THREADS, 4)
     }
 }
 
-// out[e] = sum over s = 0..NS-1 of part[s n + e], in that order (blockIdx.y picks dq, dk, dbeta);
-// with tc_hs, elements of heads that the tensor-core backward takes are left alone.
+// out[e] = sum over s = 0..NS-1 of part[s n + e], in that order; with tc_hs, the heads that the
+// tensor-core backward takes are left alone.
 struct SumSeg {
     const float *part;
     float *out;
@@ -445,16 +553,18 @@ struct SumSegs {
     SumSeg seg[3];
 };
 
-__global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS, const int *__restrict__ tc_hs) {
+// Grid: (BH x SL, 3): block x takes head x / SL and, within it, every SL-th piece of 256
+// elements (float4 groups when vec); blockIdx.y picks dq, dk or dbeta.
+__global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS, int SL, const int *__restrict__ tc_hs) {
     const SumSeg g = blockIdx.y == 0 ? segs.seg[0] : (blockIdx.y == 1 ? segs.seg[1] : segs.seg[2]);
-    const size_t stride = (size_t)gridDim.x * blockDim.x;
-    const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long head = blockIdx.x / SL;
+    const int sl = blockIdx.x % SL;
+    if (tc_hs && head_takes_saved(tc_hs, head)) return;
     if (g.vec) {
-        const size_t n4 = g.n / 4;
+        const size_t n4 = g.n / 4, ph4 = g.per_head / 4, h0 = (size_t)head * ph4;
         const float4 *p4 = reinterpret_cast<const float4 *>(g.part);
         float4 *o4 = reinterpret_cast<float4 *>(g.out);
-        for (size_t e = i0; e < n4; e += stride) {
-            if (tc_hs && head_takes_saved(tc_hs, (long long)(4 * e / g.per_head))) continue;
+        for (size_t e = h0 + (size_t)sl * blockDim.x + threadIdx.x; e < h0 + ph4; e += (size_t)SL * blockDim.x) {
             float4 a = p4[e];
             for (int s = 1; s < NS; ++s) {
                 const float4 b = p4[(size_t)s * n4 + e];
@@ -463,8 +573,8 @@ __global__ void __launch_bounds__(256) bwd_sum_kernel(SumSegs segs, int NS, cons
             o4[e] = a;
         }
     } else {
-        for (size_t e = i0; e < g.n; e += stride) {
-            if (tc_hs && head_takes_saved(tc_hs, (long long)(e / g.per_head))) continue;
+        const size_t h0 = (size_t)head * g.per_head;
+        for (size_t e = h0 + (size_t)sl * blockDim.x + threadIdx.x; e < h0 + g.per_head; e += (size_t)SL * blockDim.x) {
             float a = g.part[e];
             for (int s = 1; s < NS; ++s) a += g.part[(size_t)s * g.n + e];
             g.out[e] = a;
@@ -502,8 +612,8 @@ static BwdLayout bwd_layout(int B, int H, int L, int dk, int dv) {
     a.u = a.ck = a.tcb = a.total = a.tc;
     if (bwd_tc_saves(B, H, L, dk, dv)) {
         a.u = a.tc + up((tc_workspace_bytes(B, H, L, dk, dv, BWD_BLOCK) + 3) / 4);
-        a.ck = a.u + up(ntok * (size_t)dv);
-        a.tcb = a.ck + up(BH * NB * (size_t)dk * dv);
+        a.ck = a.u + up((ntok * (size_t)dv + 1) / 2);  // fp16
+        a.tcb = a.ck + up((BH * NB * (size_t)dk * dv + 1) / 2);
         a.total = a.tcb + (bwd_tc_workspace_bytes(B, H, L, dk, dv) + 3) / 4;
     }
     return a;
@@ -530,26 +640,35 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     int *hs = (int *)(wsf + lay.zero);  // per-head statistics for the saved-forward gate
     float *state = wsf + lay.state;
     float *part = wsf + lay.part;
-    float *u_saved = nullptr, *ck_saved = nullptr;
+    __half *u_saved = nullptr, *ck_saved = nullptr;
     cudaError_t e;
     // the tensor-core forward (TMA) and backward load q, k, v, S0 and dO 16 bytes at a time;
     // inputs that are only element-aligned take the CUDA-core path for every head
     auto al16 = [](const void *p) { return ((uintptr_t)p & 15) == 0; };
-    const bool tc_fwd = is_bf16 && bwd_tc_saves(B, H, L, dk, dv) && al16(q) && al16(k) && al16(v) &&
-                        (S0 == nullptr || al16(S0));
-    const bool tc_bwd = tc_fwd && al16(dO);
-    if (tc_fwd) {
-        // the tensor-core forward, saving u and the block states instead of writing outputs
-        u_saved = wsf + lay.u;
-        ck_saved = wsf + lay.ck;
+    const bool tc_bwd = is_bf16 && bwd_tc_saves(B, H, L, dk, dv) && al16(q) && al16(k) && al16(v) &&
+                        al16(dO) && (S0 == nullptr || al16(S0));
+    if (tc_bwd) {
+        // the tensor-core forward, saving u and the block states (fp16) instead of writing outputs
+        u_saved = (__half *)(wsf + lay.u);
+        ck_saved = (__half *)(wsf + lay.ck);
         e = launch_chunk_tc_save(q, k, v, beta, S0, B, H, L, dk, dv, euler, wsf + lay.tc, u_saved, ck_saved, s);
         if (e != cudaSuccess) return e;
     }
     if (ntok > 0) {
         e = cudaMemsetAsync(hs, 0, 4 * (size_t)BH * sizeof(int), s);
         if (e != cudaSuccess) return e;
-        const int gc = (int)std::min<size_t>((ntok + 7) / 8, (size_t)nsm * 64);
-        if (is_bf16)
+        // one warp per unit of up to 64 tokens within a head
+        const long long units = (long long)BH * ((L + 63) / 64);
+        const int gc = (int)std::max<long long>(1, std::min<long long>((units + 7) / 8, (long long)nsm * 64));
+        const bool vec_rows = is_bf16 && (dk == 64 || dk == 128) && ((uintptr_t)q & 15) == 0 &&
+                              ((uintptr_t)k & 15) == 0;
+        if (vec_rows && dk == 128)
+            bwd_coeff_vec_kernel<128><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                                         (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs);
+        else if (vec_rows)
+            bwd_coeff_vec_kernel<64><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                                        (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs);
+        else if (is_bf16)
             bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>(
                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, ntok, L,
                 dk, euler, coef, hs);
@@ -568,12 +687,11 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     if (is_bf16)
         bwd_cols_kernel<__nv_bfloat16><<<grid, BW_THREADS, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, dO,
-            dSL, dval, dS0, L, dk, dv, NS, state, part, u_saved, ck_saved, hs, tc_bwd);
+            dSL, dval, dS0, L, dk, dv, NS, state, part, hs, tc_bwd);
     else
         bwd_cols_kernel<float><<<grid, BW_THREADS, 0, s>>>((const float *)q, (const float *)k,
                                                           (const float *)v, coef, S0, dO, dSL, dval,
-                                                          dS0, L, dk, dv, NS, state, part, nullptr,
-                                                          nullptr, hs, false);
+                                                          dS0, L, dk, dv, NS, state, part, hs, false);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess || L == 0) return e;
@@ -593,9 +711,10 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     segs.seg[0] = seg(part, dq, nq, (size_t)L * dk);
     segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq, (size_t)L * dk);
     segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb, (size_t)L);
-    const size_t want = (nq / 4 + 255) / 256;
-    const int gx = (int)std::min<size_t>(std::max<size_t>(want, 1), (size_t)nsm * 8);
-    bwd_sum_kernel<<<dim3(gx, 3), 256, 0, s>>>(segs, NS, tc_bwd ? hs : nullptr);
+    const int SL = (int)std::max<long long>(1, std::min<long long>(((long long)nsm * 8 + BH - 1) / BH,
+                                                                      ((long long)L * dk / 4 + 255) / 256));
+    if (BH * SL > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    bwd_sum_kernel<<<dim3((unsigned)(BH * SL), 3), 256, 0, s>>>(segs, NS, SL, tc_bwd ? hs : nullptr);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -95,8 +95,9 @@ __device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_tak
 //   D2a  dS^T  += dO^T Q            (off the chain)
 //   W, P of the next chunk
 //   D2b  dS^T  += dU'16^T (-W)      (A = fp16 dU'^T in TMEM)
-// Outputs: dU' of every token (fp16, [BH][L][dv]); the gradient of the state after every chunk
-// as fp16 dSp [BH][NC][dk][dv] (dSp[NC-1] is dS_final); dS0 (fp32).
+// Outputs (fp16; a warp's lanes write consecutive columns): dU' of every token [BH][L][dv] and
+// the gradient of the state after every chunk, dSp [BH][NC][dk][dv] (dSp[NC-1] is dS_final);
+// dS0 (fp32).
 template <int DK, int DV>
 __global__ void __launch_bounds__(REV_THREADS, 1)
     bwd_state_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -492,32 +493,46 @@ __device__ __forceinline__ void store16(uint8_t *tile, int rows, const float (&a
             }
 }
 
-// Fill a [rows][cols] fp16 tile from global memory (row stride ld elements), rows at or past
-// `valid` read as zero.  8 elements per thread and step.
-template <typename T>
-__device__ __forceinline__ void fill(uint8_t *tile, int rows, int cols, const T *src, size_t ld, int valid) {
-    const int per_row = cols / 8;
-    for (int e = threadIdx.x; e < rows * per_row; e += THREADS) {
-        const int r = e / per_row, c = (e - r * per_row) * 8;
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (r < valid) {
-            const T *p = src + (size_t)r * ld + c;
-            if constexpr (std::is_same<T, __half>::value) {
-                u = *reinterpret_cast<const uint4 *>(p);
-            } else if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(p);
-                u = make_uint4(tc::bf16x2_to_f16x2(x.x), tc::bf16x2_to_f16x2(x.y), tc::bf16x2_to_f16x2(x.z),
-                               tc::bf16x2_to_f16x2(x.w));
-            } else {
-                const float4 x0 = *reinterpret_cast<const float4 *>(p);
-                const float4 x1 = *reinterpret_cast<const float4 *>(p + 4);
-                u = make_uint4(tc::pack_f16(x0.x, x0.y), tc::pack_f16(x0.z, x0.w), tc::pack_f16(x1.x, x1.y),
-                               tc::pack_f16(x1.z, x1.w));
-            }
+// Tiles of fp16 in shared memory filled from global memory 16 bytes (8 elements) per thread
+// and step: every step's loads of a tile are issued before any of its stores (global memory
+// latency is paid once per tile, not once per step).  [rows][cols] with row stride ld
+// elements in global memory; rows at or past `valid` read as zero.
+template <typename T, int ROWS, int COLS>
+struct TileIn {
+    static constexpr int PER = ROWS * COLS / 8 / THREADS;  // steps per thread
+    static constexpr int W = sizeof(T) == 4 ? 2 : 1;       // 16-byte words per 8 elements
+    uint4 x[PER][W];
+    __device__ __forceinline__ void load(const T *src, size_t ld, int valid) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int e = threadIdx.x + j * THREADS, r = e / (COLS / 8), c = (e % (COLS / 8)) * 8;
+#pragma unroll
+            for (int w = 0; w < W; ++w)
+                x[j][w] = r < valid ? *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + c + 4 * w)
+                                    : make_uint4(0u, 0u, 0u, 0u);
         }
-        *reinterpret_cast<uint4 *>(tile + off(rows, r, c)) = u;
     }
-}
+    __device__ __forceinline__ void store(uint8_t *tile) const {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int e = threadIdx.x + j * THREADS, r = e / (COLS / 8), c = (e % (COLS / 8)) * 8;
+            uint4 u;
+            if constexpr (std::is_same<T, __half>::value) {
+                u = x[j][0];
+            } else if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                u = make_uint4(tc::bf16x2_to_f16x2(x[j][0].x), tc::bf16x2_to_f16x2(x[j][0].y),
+                               tc::bf16x2_to_f16x2(x[j][0].z), tc::bf16x2_to_f16x2(x[j][0].w));
+            } else {
+                const uint4 a = x[j][0], b = x[j][W - 1];
+                u = make_uint4(tc::pack_f16(__uint_as_float(a.x), __uint_as_float(a.y)),
+                               tc::pack_f16(__uint_as_float(a.z), __uint_as_float(a.w)),
+                               tc::pack_f16(__uint_as_float(b.x), __uint_as_float(b.y)),
+                               tc::pack_f16(__uint_as_float(b.z), __uint_as_float(b.w)));
+            }
+            *reinterpret_cast<uint4 *>(tile + off(ROWS, r, c)) = u;
+        }
+    }
+};
 }  // namespace cw
 
 // Shared memory of the per-chunk kernel: fp16 tiles Q, K, dO, U', dU', -dR [64][d]; S, dS'
@@ -533,13 +548,14 @@ struct ChunkLayout {
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(cw::THREADS, 1)
-    bwd_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                     const __nv_bfloat16 *__restrict__ v, const float4 *__restrict__ coef,
-                     const __half *__restrict__ dO16, const float *__restrict__ u_saved,
-                     const __half *__restrict__ dU, const float *__restrict__ ck_saved,
-                     const float *__restrict__ S0, const __half *__restrict__ dSp, const __half *__restrict__ ta,
-                     const int *__restrict__ hs, float *__restrict__ dq, float *__restrict__ dkey,
-                     float *__restrict__ dval, float *__restrict__ dbeta, int L, int NC) {
+    bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_u,
+                     const __grid_constant__ CUtensorMap tmap_du, const __grid_constant__ CUtensorMap tmap_s,
+                     const __grid_constant__ CUtensorMap tmap_ds, const __grid_constant__ CUtensorMap tmap_t,
+                     const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                     const float4 *__restrict__ coef, const float *__restrict__ S0, const int *__restrict__ hs,
+                     float *__restrict__ dq, float *__restrict__ dkey, float *__restrict__ dval,
+                     float *__restrict__ dbeta, int L, int NC) {
     using Lay = ChunkLayout<DK, DV>;
     using namespace cw;
     extern __shared__ uint8_t smem_raw[];
@@ -547,6 +563,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
     const uint32_t sb = tc::smem_u32(base);
     __shared__ float sa[C], sfb[C], sfl[C], sda[2][4][C];  // sda: partials of da (2 kinds x 4 column groups)
+    __shared__ uint64_t full[2];  // the operand tiles, in two groups (TMA)
 
     const int chunk = blockIdx.x, bh = chunk / NC, n = chunk - bh * NC;
     if (!head_ok(hs, bh)) return;  // this head walks on CUDA cores (uniform over the CTA)
@@ -554,17 +571,46 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     const int t0 = n * C, valid = min(C, L - t0);
     const size_t DD = (size_t)DK * DV, tokq = (size_t)bh * L + t0;
 
-    // ---- operands into shared memory (fp16)
-    fill(base + Lay::TQ, C, DK, q + tokq * DK, DK, valid);
-    fill(base + Lay::TK, C, DK, k + tokq * DK, DK, valid);
-    fill(base + Lay::TO, C, DV, dO16 + tokq * DV, DV, valid);
-    fill(base + Lay::TU, C, DV, u_saved + tokq * DV, DV, valid);
-    fill(base + Lay::TDU, C, DV, dU + tokq * DV, DV, valid);
-    if (n > 0) fill(base + Lay::TS, DK, DV, ck_saved + ((size_t)bh * NC + n - 1) * DD, DV, DK);
-    else if (S0) fill(base + Lay::TS, DK, DV, S0 + (size_t)bh * DD, DV, DK);
-    else fill(base + Lay::TS, DK, DV, (const __half *)nullptr, DV, 0);
-    fill(base + Lay::TDS, DK, DV, dSp + ((size_t)bh * NC + n) * DD, DV, DK);
-    fill(base + Lay::TT, C, C, ta + (size_t)chunk * C * C, C, C);
+    // ---- operand tiles by TMA (128-byte swizzle, as `off` lays them out), all in flight at
+    // once: group 0 (K, S, Ta, dU') for the first products, group 1 (Q, dO, U', dS') for the
+    // rest.  S of the first chunk is the initial state (fp32), rounded here.
+    const int ck = chunk * DK;  // row of this chunk's [dk][dv] tiles
+    if (tid == 0) {
+        tc::mbar_init(&full[0], 1);
+        tc::mbar_init(&full[1], 1);
+        tc::fence_mbar_init();
+        tc::mbar_expect_tx(&full[0], 128 * DK + (n > 0 ? 2 * DK * DV : 0) + C * C * 2 + 128 * DV);
+        for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TK + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
+        for (int j = 0; j < DV / 64; ++j) {
+            if (n > 0) tc::tma_load_2d(base + Lay::TS + j * 128 * DK, &tmap_s, &full[0], j * 64, ck - DK);
+            tc::tma_load_3d(base + Lay::TDU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
+        }
+        tc::tma_load_2d(base + Lay::TT, &tmap_t, &full[0], 0, chunk * C);
+        tc::mbar_expect_tx(&full[1], 128 * DK + 128 * DV + 128 * DV + 2 * DK * DV);
+        for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TQ + j * 8192, &tmap_q, &full[1], j * 64, t0, bh);
+        for (int j = 0; j < DV / 64; ++j) {
+            tc::tma_load_3d(base + Lay::TO + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
+            tc::tma_load_3d(base + Lay::TU + j * 8192, &tmap_u, &full[1], j * 64, t0, bh);
+            tc::tma_load_2d(base + Lay::TDS + j * 128 * DK, &tmap_ds, &full[1], j * 64, ck);
+        }
+    }
+    if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero
+        for (int e = tid; e < DK * DV; e += THREADS) {
+            const int kr = e / DV, vc = e - kr * DV;
+            const float x = S0 ? S0[(size_t)bh * DD + e] : 0.f;
+            *reinterpret_cast<__half *>(base + Lay::TS + off(DK, kr, vc & ~7) + 2 * (vc & 7)) = __float2half_rn(x);
+        }
+    }
+    __syncthreads();  // the barriers' initialisation, the initial state
+    bool ok = tc::mbar_wait(&full[0], 0, WAIT_BUDGET);
+    // K to fp16 in place (bf16 values are exact in fp16 from 2^-14 up)
+    for (int e = tid; e < 128 * DK / 16; e += THREADS) {
+        uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TK) + e;
+        uint4 u = *p;
+        u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+        u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+        *p = u;
+    }
     if (tid < C) {
         const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
         sa[tid] = c.y;
@@ -612,6 +658,15 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
                 if ((lane & 3) == 0) sda[0][wc][acc_r(m0, mt, 2 * h, lane)] = x;
             }
     }
+    ok = tc::mbar_wait(&full[1], 0, WAIT_BUDGET) && ok;
+    for (int e = tid; e < 128 * DK / 16; e += THREADS) {  // Q to fp16 in place
+        uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TQ) + e;
+        uint4 u = *p;
+        u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+        u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+        *p = u;
+    }
+    if (!ok && tid == 0) atomicOr(&g_bwd_error, 4u);  // a copy did not land in time
     __syncthreads();
     // ---- G = K K^T, B = strictly-lower(-dR U'^T), dP = lower-incl(dO U'^T) ([64][64]);
     // da's second part sum_s B_ts G_ts
@@ -704,6 +759,10 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
                     }
                 }
     }
+    if (!ok && tid == 0) {  // let this CTA's copies land before it exits (bounded)
+        tc::mbar_wait(&full[0], 0, WAIT_BUDGET / 4);
+        tc::mbar_wait(&full[1], 0, WAIT_BUDGET / 4);
+    }
 }
 
 // dO (fp32) to fp16 for the products; and which heads take the tensor-core path.
@@ -717,13 +776,13 @@ __global__ void __launch_bounds__(256) bwd_prepare_kernel(const float *__restric
 
 template <int DK, int DV>
 cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const float *S0, const float *dO,
-                            const float *dSL, const float4 *coef, const int *hs, const float *u_saved,
-                            const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                            const float *dSL, const float4 *coef, const int *hs, const __half *u_saved,
+                            const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
                             float *dbeta, float *dS0, int B, int H, int L, void *ws, cudaStream_t s) {
     const int BH = B * H, NC = (L + C - 1) / C;
     const size_t ntok = (size_t)BH * L;
     __half *dO16 = (__half *)ws;
-    __half *dU = dO16 + ntok * DV;
+    __half *dU = dO16 + ntok * DV;  // 16-byte aligned: dv is 64 or 128
     __half *dSp = dU + ntok * DV;
     static bool attr_done[64] = {};
     int dev = 0, nsm = 148;
@@ -749,9 +808,16 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
     bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
     bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, dSL, dU, dSp, dS0,
                                                                               hs, L, NC);
+    CUtensorMap mu, mdu, ms, mds;
+    const uint64_t rows = (uint64_t)BH * NC * DK;  // [BH][NC][dk] rows of dv columns
+    if (!tmap::make_3d(&mu, u_saved, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !tmap::make_3d(&mdu, dU, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !tmap::make_2d(&ms, ck_saved, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
     bwd_chunk_kernel<DK, DV><<<BH * NC, cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, dO16, u_saved, dU,
-        ck_saved, S0, dSp, (const __half *)ta, hs, dq, dkey, dval, dbeta, L, NC);
+        mq, mk, mo, mu, mdu, ms, mds, mt, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, hs, dq,
+        dkey, dval, dbeta, L, NC);
     count_launches(3);
     return cudaGetLastError();
 }
@@ -760,12 +826,13 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
 
 size_t bwd_tc_workspace_bytes(int B, int H, int L, int dk, int dv) {
     const size_t BH = (size_t)B * H, NC = (size_t)(L + C - 1) / C;
+    // fp16 dO and dU' [BH][L][dv], dSp [BH][NC][dk][dv]
     return (2 * BH * (size_t)L * dv + BH * NC * (size_t)dk * dv) * sizeof(__half);
 }
 
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *S0, const float *dO,
-                          const float *dSL, const void *coef, const int *hs, const float *u_saved,
-                          const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                          const float *dSL, const void *coef, const int *hs, const __half *u_saved,
+                          const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
                           float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
                           cudaStream_t s) {
     const float4 *cf = (const float4 *)coef;

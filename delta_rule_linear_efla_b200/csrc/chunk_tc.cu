@@ -294,10 +294,12 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = (cb * 16 + j < r) ? ar * v[j] : 0.f;
                     if constexpr (GATED) {  // Gam o G below the diagonal: e^{l_r - l_c} <= 1
+                        // (the fast exponential: CUDA bounds its error by 2 + 1.17 |x| ulp, under
+                        // 5e-5 relative for arguments down to -300, far below A's fp16 rounding)
                         const float lr = lg[r];
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            if (cb * 16 + j < r) v[j] *= expf(fminf(lr - lg[cb * 16 + j], 0.f));
+                            if (cb * 16 + j < r) v[j] *= __expf(fminf(lr - lg[cb * 16 + j], 0.f));
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(A16 + r * LD16 + cb * 16);
                     dst[0] = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
@@ -454,6 +456,7 @@ struct StateLayout {
     static constexpr int OFF_PH = 2 * STAGE, OFF_PL = OFF_PH + 8192;  // gated: P^T hi and lo
     static constexpr int BYTES = 2 * STAGE + (GATED ? 2 * 8192 : 0);
     static constexpr int SMEM = BYTES + 1024;             // alignment slack
+    static_assert(!GATED || OFF_PL + 8192 == BYTES, "gated shared-memory layout");
 };
 
 // Row of an M-row accumulator held by this thread, or -1: M = 128 puts row r in
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
                     float *__restrict__ segbuf, int G, int seg_chunks, int pass,
-                    float *__restrict__ u_out, float *__restrict__ ck_out,
+                    __half *__restrict__ u_out, __half *__restrict__ ck_out,
                     const __nv_bfloat16 *__restrict__ gate) {
     static_assert(!(SAVE && GATED), "the saving forward is for the ungated form");
     using Lay = StateLayout<DK, DV, GATED>;
@@ -936,7 +939,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                         const float *lt = gf(st, 0);
                         const float lin = lt[crow];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] *= expf(fminf(lt[cb * 32 + j] - lin, 0.f));
+                        for (int j = 0; j < 32; ++j) v[j] *= __expf(fminf(lt[cb * 32 + j] - lin, 0.f));  // as in prep
                         store_row_f16x32(base + Lay::OFF_PH, crow, cb * 4, v);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] -= __half2float(__float2half_rn(v[j]));
@@ -995,12 +998,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     }
                 }
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
-                if (SAVE && u_out && mode == 0 && vrow >= 0) {  // u_t = a_t r_t of every token, for the backward
+                if (SAVE && u_out && mode == 0 && vrow >= 0) {
+                    // u_t = a_t r_t of every token, for the backward: fp16 [B*H][L][dv] (a warp's
+                    // lanes write a token's consecutive columns)
                     const int t0 = (n0 + n) * C + h * 32;
-                    float *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
+                    __half *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (t0 + j < L) dst[(size_t)j * DV] = u[j];
+                        if (t0 + j < L) dst[(size_t)j * DV] = __float2half_rn(u[j]);
                 }
             }
 
@@ -1055,14 +1060,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
                 // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
                 // warp-collective: every lane takes it, the lanes that hold a state column store.
-                float *dst = ck_out + ((size_t)bh * NC + n0 + n) * DD + (vrow >= 0 ? vrow : 0);
+                // fp16 [B*H][NC][dk][dv] (a warp's lanes write a row's consecutive columns)
+                __half *dst = ck_out + ((size_t)bh * NC + n0 + n) * DD + (vrow >= 0 ? vrow : 0);
 #pragma unroll 1
                 for (int cb = 0; cb < DK / 16; ++cb) {
                     float v[16];
                     tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
                     if (vrow >= 0) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) dst[(size_t)(cb * 16 + j) * DV] = v[j];
+                        for (int j = 0; j < 16; ++j) dst[(size_t)(cb * 16 + j) * DV] = __float2half_rn(v[j]);
                     }
                 }
             }
@@ -1284,7 +1290,7 @@ TcDevInfo tc_dev_info() {
 template <int DK, int DV, typename TO, bool SAVE, bool GATED>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void *beta,
                         const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
-                        void *ws, cudaStream_t s, float *u_out, float *ck_out, bool allow_seg,
+                        void *ws, cudaStream_t s, __half *u_out, __half *ck_out, bool allow_seg,
                         const void *g) {
     const int BH = B * H, NC = (L + C - 1) / C, total = BH * NC;
     const TcDevInfo di = tc_dev_info<DK, DV, TO>();
@@ -1386,7 +1392,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
 
 cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
                                  const float *S0, int B, int H, int L, int dk, int dv, bool euler,
-                                 void *ws, float *u_out, float *ck_out, cudaStream_t s) {
+                                 void *ws, __half *u_out, __half *ck_out, cudaStream_t s) {
     if (dk == 128 && dv == 128)
         return launch_tc_t<128, 128, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws,
                                                          s, u_out, ck_out, true, nullptr);

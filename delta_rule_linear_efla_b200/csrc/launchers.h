@@ -3,6 +3,7 @@
 // cudaError_t from cudaGetLastError() after its launches.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -64,11 +65,11 @@ int chunk_fwd_entry(const void *q, const void *k, const void *v, const void *bet
                     bool allow_segments, const void *g);
 // The tensor-core forward without outputs, saving what the backward needs instead: every
 // token's u_t = a_t (v_t - S_{t-1}^T k_t) into u_out [B*H][L][dv] and the state after every
-// 64-token chunk into ck_out [B*H][ceil(L/64)][dk][dv] (fp32).  Same sizes as launch_chunk_tc,
-// chunk 64, and the same workspace.
+// 64-token chunk into ck_out [B*H][ceil(L/64)][dk][dv], rounded to fp16 (the backward's products
+// take them as fp16 operands).  Same sizes as launch_chunk_tc, chunk 64, and the same workspace.
 cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
                                  const float *S0, int B, int H, int L, int dk, int dv, bool euler,
-                                 void *ws, float *u_out, float *ck_out, cudaStream_t s);
+                                 void *ws, __half *u_out, __half *ck_out, cudaStream_t s);
 // The backward on tensor cores for the heads the saved-forward gate lets through (bf16, chunk
 // 64, dk and dv in {64, 128}, q, k, dO and S0 16-byte aligned): dO to fp16, the reverse chain
 // over the chunks (dU' of every token and the state gradient after every chunk), then every
@@ -77,8 +78,8 @@ cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, co
 // saving forward's outputs and Ta tiles.  Workspace: bwd_tc_workspace_bytes.
 size_t bwd_tc_workspace_bytes(int B, int H, int L, int dk, int dv);
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *S0, const float *dO,
-                          const float *dSL, const void *coef, const int *hs, const float *u_saved,
-                          const float *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
+                          const float *dSL, const void *coef, const int *hs, const __half *u_saved,
+                          const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
                           float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
                           cudaStream_t s);
 cudaError_t bwd_tc_read_and_clear_error(unsigned int *out);

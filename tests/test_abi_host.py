@@ -148,8 +148,8 @@ def test_bwd_workspace_size_and_alignment(lib):
     """The backward's workspace, every region rounded up to 256 bytes: eight fp32 coefficients per
     token; four ints of statistics per head; per (head, 16-column block) r of every token and the
     block's state every 64 tokens and at the end; the column blocks' shares of dq, dk and dbeta;
-    and, where the tensor-core forward can run (bf16 inputs), its workspace, every token's u, the
-    state after every 64-token block, and for the tensor-core backward the fp16 dO, every token's
+    and, where the tensor-core forward can run (bf16 inputs), its workspace, every token's u and the
+    state after every 64-token block (fp16), and for the tensor-core backward the fp16 dO, every token's
     dU' and the state gradient after every block.  A workspace that is not 16-byte aligned is
     refused before any CUDA call."""
     up = lambda f: (f + 63) // 64 * 64
@@ -159,7 +159,7 @@ def test_bwd_workspace_size_and_alignment(lib):
         up(NS * BH * L * (2 * dk + 1))
     tc = lib.efla_chunk_fwd_workspace_size(B, H, L, dk, dv, 64, BF16, F32)
     tcb = 2 * (2 * BH * L * dv + BH * NB * dk * dv)  # fp16 dO, dU' and the chunks' state gradients
-    saved = up(tc // 4) + up(BH * L * dv) + up(BH * NB * dk * dv) + (tcb + 3) // 4
+    saved = up(tc // 4) + up(BH * L * dv // 2) + up(BH * NB * dk * dv // 2) + (tcb + 3) // 4  # fp16 u, states
     assert lib.efla_bwd_workspace_size(B, H, L, dk, dv) == 4 * (base + saved)
     # ragged, no tensor-core forward (d_k = 8): dv = 20 takes two column blocks, L = 65 two blocks
     assert lib.efla_bwd_workspace_size(1, 1, 65, 8, 20) == \
