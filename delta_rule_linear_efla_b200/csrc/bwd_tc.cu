@@ -364,25 +364,26 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
             tc::tc_fence_after();
             if (i + 1 < NC) {
                 // the state gradient after chunk n - 1: its fp16 copy for D1b, and to dSp
-                __half *dst = dSp + ((size_t)bh * NC + (n - 1)) * DD + (vrow >= 0 ? vrow : 0);
+                // the fp16 copy first (D1b of the next chunk waits for it), the global copy after
+                uint32_t w[DK / 2];
 #pragma unroll
                 for (int cb = 0; cb < DK / 32; ++cb) {
                     float v[32];
                     tc::tmem_ld32(tmem + lane_base + TM_S + cb * 32, v);
-                    uint32_t w[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) w[j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
-                    tc::tmem_st16u(tmem + lane_base + RT_S16 + cb * 16, w);
-                    if (vrow >= 0) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const __half2 pr = *reinterpret_cast<const __half2 *>(&w[j]);
-                            dst[(size_t)(cb * 32 + 2 * j) * DV] = __low2half(pr);
-                            dst[(size_t)(cb * 32 + 2 * j + 1) * DV] = __high2half(pr);
-                        }
-                    }
+                    for (int j = 0; j < 16; ++j) w[cb * 16 + j] = tc::pack_f16(v[2 * j], v[2 * j + 1]);
+                    tc::tmem_st16u(tmem + lane_base + RT_S16 + cb * 16, *reinterpret_cast<uint32_t(*)[16]>(w + cb * 16));
                 }
                 rev_arrive(&bars.s_ready, lane);
+                if (vrow >= 0) {
+                    __half *dst = dSp + ((size_t)bh * NC + (n - 1)) * DD + vrow;
+#pragma unroll
+                    for (int j = 0; j < DK / 2; ++j) {
+                        const __half2 pr = *reinterpret_cast<const __half2 *>(&w[j]);
+                        dst[(size_t)(2 * j) * DV] = __low2half(pr);
+                        dst[(size_t)(2 * j + 1) * DV] = __high2half(pr);
+                    }
+                }
             }
         }
         if (done_all && dS0) {  // the gradient of the initial state
@@ -536,13 +537,14 @@ struct TileIn {
 }  // namespace cw
 
 // Shared memory of the per-chunk kernel: fp16 tiles Q, K, dO, U', dU', -dR [64][d]; S, dS'
-// [dk][dv]; Ta, B, dP [64][64]; per-token a, df/dbeta, df/dlambda and the partial sums of da.
+// [dk][dv]; Ta, B, dP [64][64]; V [64][dv] (bf16, for R = V - K S); per-token a, df/dbeta,
+// df/dlambda and the partial sums of da.
 template <int DK, int DV>
 struct ChunkLayout {
     static constexpr int TQ = 0, TK = TQ + 128 * DK, TO = TK + 128 * DK, TU = TO + 128 * DV,
                          TDU = TU + 128 * DV, TNR = TDU + 128 * DV, TS = TNR + 128 * DV,
                          TDS = TS + 2 * DK * DV, TT = TDS + 2 * DK * DV, TB = TT + 8192, TP = TB + 8192,
-                         TEND = TP + 8192;
+                         TV = TP + 8192, TEND = TV + 128 * DV;
     static constexpr int SMEM = TEND + 1024;  // + alignment slack
 };
 
@@ -552,7 +554,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
                      const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_u,
                      const __grid_constant__ CUtensorMap tmap_du, const __grid_constant__ CUtensorMap tmap_s,
                      const __grid_constant__ CUtensorMap tmap_ds, const __grid_constant__ CUtensorMap tmap_t,
-                     const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                     const __grid_constant__ CUtensorMap tmap_v,
                      const float4 *__restrict__ coef, const float *__restrict__ S0, const int *__restrict__ hs,
                      float *__restrict__ dq, float *__restrict__ dkey, float *__restrict__ dval,
                      float *__restrict__ dbeta, int L, int NC) {
@@ -579,11 +581,12 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         tc::mbar_init(&full[0], 1);
         tc::mbar_init(&full[1], 1);
         tc::fence_mbar_init();
-        tc::mbar_expect_tx(&full[0], 128 * DK + (n > 0 ? 2 * DK * DV : 0) + C * C * 2 + 128 * DV);
+        tc::mbar_expect_tx(&full[0], 128 * DK + (n > 0 ? 2 * DK * DV : 0) + C * C * 2 + 2 * 128 * DV);
         for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TK + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
         for (int j = 0; j < DV / 64; ++j) {
             if (n > 0) tc::tma_load_2d(base + Lay::TS + j * 128 * DK, &tmap_s, &full[0], j * 64, ck - DK);
             tc::tma_load_3d(base + Lay::TDU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
+            tc::tma_load_3d(base + Lay::TV + j * 8192, &tmap_v, &full[0], j * 64, t0, bh);
         }
         tc::tma_load_2d(base + Lay::TT, &tmap_t, &full[0], 0, chunk * C);
         tc::mbar_expect_tx(&full[1], 128 * DK + 128 * DV + 128 * DV + 2 * DK * DV);
@@ -642,7 +645,8 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
-                    const float vv = r < valid ? __bfloat162float(v[(tokq + r) * DV + c]) : 0.f;
+                    const float vv = __bfloat162float(  // zero past the sequence (TMA fill)
+                        *reinterpret_cast<const __nv_bfloat16 *>(base + Lay::TV + off(C, r, c & ~7) + 2 * (c & 7)));
                     part[mt][e >> 1] += accD[mt][nt][e] * (vv - accR[mt][nt][e]);
                     if (r < valid) dval[(tokq + r) * DV + c] = accD[mt][nt][e];
                     accD[mt][nt][e] = -accD[mt][nt][e];
@@ -753,8 +757,9 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = acc_r(m0, mt, e, lane), c = acc_c(n0k, nt, e, lane);
-                    if (r < valid) {
-                        const float kk = __bfloat162float(k[(tokq + r) * DK + c]);
+                    if (r < valid) {  // K's fp16 tile holds the bf16 values exactly
+                        const float kk = __half2float(
+                            *reinterpret_cast<const __half *>(base + Lay::TK + off(C, r, c & ~7) + 2 * (c & 7)));
                         dkey[(tokq + r) * DK + c] = acc[mt][nt][e] + 2.f * sa[r] * sfl[r] * kk;
                     }
                 }
@@ -808,16 +813,16 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
     bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
     bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, dSL, dU, dSp, dS0,
                                                                               hs, L, NC);
-    CUtensorMap mu, mdu, ms, mds;
+    CUtensorMap mu, mdu, ms, mds, mv;
     const uint64_t rows = (uint64_t)BH * NC * DK;  // [BH][NC][dk] rows of dv columns
     if (!tmap::make_3d(&mu, u_saved, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !tmap::make_3d(&mdu, dU, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !tmap::make_2d(&ms, ck_saved, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-        !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
     bwd_chunk_kernel<DK, DV><<<BH * NC, cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
-        mq, mk, mo, mu, mdu, ms, mds, mt, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, coef, S0, hs, dq,
-        dkey, dval, dbeta, L, NC);
+        mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC);
     count_launches(3);
     return cudaGetLastError();
 }

@@ -297,16 +297,23 @@ efla_status efla_state_affine(const float *P, const float *S_in, const float *H,
  *   workspace : efla_bwd_workspace_size(B,H,L,dk,dv) bytes, caller-owned scratch,
  *               16-byte aligned
  * Sizes: B,H >= 1, L >= 0, 1 <= dk,dv <= 128.  Other pointers aligned to their
- * element.  The state's columns evolve independently, so one CTA takes one head
- * and 16 of its state columns and walks the sequence twice (forward, then
- * reverse); dq, dkey and dbeta are sums over the columns, and a second kernel adds
- * the column blocks' shares in a fixed order (the result does not depend on
- * scheduling).  With bf16 inputs at the sizes efla_chunk_fwd runs on tensor cores
- * (chunk 64), that forward runs first and saves every token's alpha r and the
- * state after every 64 tokens; heads whose largest ||k||^2 is at most 16 and
- * whose alpha spans at most a factor of 1024 (all positive) take their reverse
- * sweep from it and skip the forward walk, the others walk it in fp32.  The
- * workspace size covers that forward whenever the sizes allow it.
+ * element.  Two paths, chosen per head on the device:
+ *   - tensor cores: with bf16 inputs at the sizes efla_chunk_fwd runs on tensor
+ *     cores (chunk 64; dk, dv in {64, 128}) and q, k, v, dO and S0 16-byte
+ *     aligned, heads whose largest ||k||^2 is at most 16 and whose alpha are all
+ *     positive and span at most a factor of 1024.  The tensor-core forward runs
+ *     first and saves every token's alpha r and the state after every 64 tokens
+ *     (fp16); a reverse chain over the chunks then gives every token's dU' and the
+ *     state gradient after every chunk, and every chunk's dq, dkey, dval and dbeta
+ *     follow in parallel, with fp16 operands and fp32 accumulation (the products'
+ *     precision of the forward; dO is rounded to fp16 for them, so |dO| must stay
+ *     below 65504).
+ *   - CUDA cores (every other head, and fp32 inputs): fp32 throughout; one CTA
+ *     takes one head and 16 of its state columns and walks the sequence twice
+ *     (forward, then reverse); dq, dkey and dbeta are sums over the columns, and
+ *     a second kernel adds the column blocks' shares in a fixed order.
+ * Both give results that do not depend on scheduling.  The workspace size covers
+ * the tensor-core path whenever the sizes allow it.
  * EFLA_ERR_ALIGN: a misaligned pointer.  EFLA_ERR_WORKSPACE: the workspace is
  * missing or too small.
  */
