@@ -666,10 +666,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
                 tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C);
                 if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeQ[st], par, &abort_flag, budget)) break;
-                tc::mbar_expect_tx(&bars.fullQ[st], DK * 128);
+                tc::mbar_expect_tx(&bars.fullQ[st], SAVE ? 0 : DK * 128);  // the saving forward reads no q
+                if constexpr (!SAVE) {
 #pragma unroll
-                for (int j = 0; j < DK / 64; ++j)
-                    tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
+                    for (int j = 0; j < DK / 64; ++j)
+                        tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
+                }
                 if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeK[st], par, &abort_flag, budget)) break;
                 tc::mbar_expect_tx(&bars.fullK[st], DK * 128);
 #pragma unroll
@@ -697,6 +699,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             constexpr uint32_t id_d2 = tc::idesc_f16(DV, DK + 64, false, true);
             constexpr uint32_t id_d2s = tc::idesc_f16(DV, DK, false, true);  // gated: S^T += U''^T K
             constexpr uint32_t id_d2o = tc::idesc_f16(DV, 64, false, true);  // gated: O^T += U'^T P^T
+            constexpr uint32_t id_d1s = tc::idesc_f16(DV, 64, false, false);  // saving: U'^T += S^T (-W)^T
             auto stage_addr = [&](int n) { return sb + (n & 1) * Lay::STAGE; };
             // U'^T := V^T Ta^T (prefill of the U' accumulator)
             auto issue_u = [&](int n) {
@@ -739,7 +742,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 tc::tc_fence_after();
                 issued_any = true;
                 issue_w(0);
-                issue_p(0);
+                if constexpr (!SAVE) issue_p(0);  // the saving forward computes no output
                 issue_u(0);
             }
             for (int n = 0; ok && n < cnt; ++n) {  // n: local chunk index
@@ -749,7 +752,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 // D1: [O^T | U'^T] += S^T [Q | -W]^T   (A = fp16 S^T in TMEM)
                 // the first 64 rows of S^T are packed before the rest: start on them
                 if (!tc::mbar_wait_or_abort(&bars.w_ready, n & 1, &abort_flag, budget)) break;
-                if (n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
+                if (!SAVE && n > 0 && !tc::mbar_wait_or_abort(&bars.o_free, (n - 1) & 1, &abort_flag, budget)) break;
                 if (n > 0 && !tc::mbar_wait_or_abort(&bars.s_ready_a, (n - 1) & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
                 bool ok2 = true;
@@ -760,9 +763,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                         if (!ok2) break;
                         tc::tc_fence_after();
                     }
-                    tc::mma_tmem_a(tmem + TM_O, tmem + TM_S16 + kk * 8,
-                                   tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
-                                   id_d1, 1u);
+                    if constexpr (SAVE)  // U'^T only: the -W rows of the QW slabs
+                        tc::mma_tmem_a(tmem + TM_U, tmem + TM_S16 + kk * 8,
+                                       tc::sdesc(qw + 8192 + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
+                                       id_d1s, 1u);
+                    else
+                        tc::mma_tmem_a(tmem + TM_O, tmem + TM_S16 + kk * 8,
+                                       tc::sdesc(qw + (kk >> 2) * Lay::QW_SLAB + (kk & 3) * 32, 16, 1024),
+                                       id_d1, 1u);
                 }
                 if (!ok2) break;
                 tc::mma_commit(&bars.d1done);
@@ -775,7 +783,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
                 // D2: [S^T | O^T] += U'^T [K | P^T]   (A = fp16 U'^T in TMEM)
                 // U' is packed in two halves of 32 tokens: start on the first
-                if (!tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
+                if (!SAVE && !tc::mbar_wait_or_abort(&bars.p_ready, n & 1, &abort_flag, budget)) break;
                 if (!tc::mbar_wait_or_abort(&bars.up_ready_a, n & 1, &abort_flag, budget)) break;
                 tc::tc_fence_after();
                 if constexpr (!GATED) {
@@ -786,8 +794,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                             if (!ok2) break;
                             tc::tc_fence_after();
                         }
-                        tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8,
-                                       tc::sdesc(kp + kk * 2048, 8192, 1024), id_d2, 1u);
+                        // the saving forward: the state update alone (N = dk), no output
+                        tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8, tc::sdesc(kp + kk * 2048, 8192, 1024),
+                                       SAVE ? id_d2s : id_d2, 1u);
                     }
                 } else {
                     // gated: O^T += U'^T P^T with both factors as fp16 hi + lo (the lo x lo term
@@ -823,7 +832,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeK[st]);
                 if (n + 1 < cnt) {  // P^T and the U' prefill of the next chunk
-                    issue_p(n + 1);
+                    if constexpr (!SAVE) issue_p(n + 1);
                     issue_u(n + 1);
                 }
             }
@@ -864,7 +873,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             }
             if (!tc::mbar_wait_or_abort(&bars.fullQ[st], par, &abort_flag, budget)) break;
 #pragma unroll
-            for (int j = 0; j < DK / 64; ++j) {  // Q: the first 8 KB of each QW slab
+            for (int j = 0; j < (SAVE ? 0 : DK / 64); ++j) {  // Q: the first 8 KB of each QW slab
                 uint4 *tq = reinterpret_cast<uint4 *>(stg + Lay::OFF_QW + j * Lay::QW_SLAB);
                 if constexpr (GATED) {
                     uint4 *tqp = reinterpret_cast<uint4 *>(stg + Lay::OFF_QP + j * 8192);
@@ -923,6 +932,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             tc::fence_async_smem();
             warp_arrive(&bars.w_ready, lane);
 
+            if constexpr (SAVE) continue;  // the saving forward computes no output: no P^T
             if (!tc::mbar_wait_or_abort(&bars.pdone, n & 1, &abort_flag, budget)) break;
             // gated: the chunk's l_t (the converter wrote them with the stage's tiles)
             if (GATED && !tc::mbar_wait_or_abort(&bars.conv[st], (n >> 1) & 1, &abort_flag, budget)) break;
@@ -1090,7 +1100,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         float z[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) z[j] = 0.f;
-        for (int n = 0; n < cnt; ++n) {  // n: local chunk index
+        for (int n = 0; n < (SAVE ? 0 : cnt); ++n) {  // n: local chunk index (the saving forward writes no o)
             const int c0 = (n0 + n) * C;
             if (!tc::mbar_wait_or_abort(&bars.d2done, n & 1, &abort_flag, budget)) break;
             tc::tc_fence_after();
