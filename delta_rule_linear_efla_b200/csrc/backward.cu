@@ -642,11 +642,13 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     float *part = wsf + lay.part;
     __half *u_saved = nullptr, *ck_saved = nullptr;
     cudaError_t e;
-    // the tensor-core forward (TMA) and backward load q, k, v, S0 and dO 16 bytes at a time;
-    // inputs that are only element-aligned take the CUDA-core path for every head
+    // the tensor-core forward (TMA) and backward load q, k, v, S0 and dO 16 bytes at a time and
+    // store dq, dk, dv 8 bytes at a time; arrays that are only element-aligned send every head to
+    // the CUDA-core path
     auto al16 = [](const void *p) { return ((uintptr_t)p & 15) == 0; };
+    auto al8 = [](const void *p) { return ((uintptr_t)p & 7) == 0; };
     const bool tc_bwd = is_bf16 && bwd_tc_saves(B, H, L, dk, dv) && al16(q) && al16(k) && al16(v) &&
-                        al16(dO) && (S0 == nullptr || al16(S0));
+                        al16(dO) && (S0 == nullptr || al16(S0)) && al8(dq) && al8(dkey) && al8(dval);
     if (tc_bwd) {
         // the tensor-core forward, saving u and the block states (fp16) instead of writing outputs
         u_saved = (__half *)(wsf + lay.u);

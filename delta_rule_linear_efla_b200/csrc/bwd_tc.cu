@@ -415,16 +415,19 @@ constexpr int THREADS = 256;
 __device__ __forceinline__ uint32_t off(int rows, int r, int c) {
     return (uint32_t)((c >> 6) * rows * 128) + tc::sw128_off(r, (c & 63) >> 3);
 }
+// Not volatile, so that the compiler may schedule the fragment loads of an unrolled k-loop ahead
+// of the MMAs that consume them; the loads keep a memory clobber, which orders them after the
+// shared-memory writes and barriers that precede each block of products.
 __device__ __forceinline__ void ldsm4(uint32_t (&d)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr));
+    asm("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr) : "memory");
 }
 __device__ __forceinline__ void ldsm4t(uint32_t (&d)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr));
+    asm("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr) : "memory");
 }
 __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -443,6 +446,7 @@ struct Tile {
 template <bool A_T, bool B_T, int MT, int NT>
 __device__ __forceinline__ void gemm(float (&acc)[MT][NT][4], Tile A, Tile B, int m0, int n0, int K, int lane) {
     const int i = lane >> 3, r8 = lane & 7;
+#pragma unroll
     for (int k0 = 0; k0 < K; k0 += 16) {
         uint32_t a[MT][4];
 #pragma unroll
@@ -548,6 +552,14 @@ struct ChunkLayout {
     static constexpr int SMEM = TEND + 1024;  // + alignment slack
 };
 
+// One CTA per SM walks the chunks blockIdx.x, blockIdx.x + gridDim.x, ... (skipping heads that
+// walk on CUDA cores) and loads its next chunk's tiles by TMA into the buffers the current
+// chunk is done with, in three groups:
+//   group 0 (Ta, dU', V), read only by R and dR: refilled after them;
+//   group 1 (K, S, dO), last read by dQ and by the K- and S-terms of dK: refilled after those;
+//   group 2 (Q, U', dS'), last read by the rest of dK: refilled at the end of the chunk;
+// so the next chunk's first products find their operands in place.  S of a head's first chunk
+// is its initial state (fp32), rounded here.
 template <int DK, int DV>
 __global__ void __launch_bounds__(cw::THREADS, 1)
     bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -557,7 +569,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
                      const __grid_constant__ CUtensorMap tmap_v,
                      const float4 *__restrict__ coef, const float *__restrict__ S0, const int *__restrict__ hs,
                      float *__restrict__ dq, float *__restrict__ dkey, float *__restrict__ dval,
-                     float *__restrict__ dbeta, int L, int NC) {
+                     float *__restrict__ dbeta, int L, int NC, int NCH) {
     using Lay = ChunkLayout<DK, DV>;
     using namespace cw;
     extern __shared__ uint8_t smem_raw[];
@@ -565,62 +577,55 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
     const uint32_t sb = tc::smem_u32(base);
     __shared__ float sa[C], sfb[C], sfl[C], sda[2][4][C];  // sda: partials of da (2 kinds x 4 column groups)
-    __shared__ uint64_t full[2];  // the operand tiles, in two groups (TMA)
+    __shared__ uint64_t full[3];  // the three tile groups (TMA)
 
-    const int chunk = blockIdx.x, bh = chunk / NC, n = chunk - bh * NC;
-    if (!head_ok(hs, bh)) return;  // this head walks on CUDA cores (uniform over the CTA)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = n * C, valid = min(C, L - t0);
-    const size_t DD = (size_t)DK * DV, tokq = (size_t)bh * L + t0;
+    const size_t DD = (size_t)DK * DV;
+    auto next_chunk = [&](int ch) {  // this CTA's next chunk whose head takes this path
+        for (ch += gridDim.x; ch < NCH; ch += gridDim.x)
+            if (head_ok(hs, ch / NC)) break;
+        return ch;
+    };
+    int ch = blockIdx.x;
+    if (ch < NCH && !head_ok(hs, ch / NC)) ch = next_chunk(ch);
+    if (ch >= NCH) return;  // uniform over the CTA
 
-    // ---- operand tiles by TMA (128-byte swizzle, as `off` lays them out), all in flight at
-    // once: group 0 (K, S, Ta, dU') for the first products, group 1 (Q, dO, U', dS') for the
-    // rest.  S of the first chunk is the initial state (fp32), rounded here.
-    const int ck = chunk * DK;  // row of this chunk's [dk][dv] tiles
+    // thread 0's bookkeeping of the copies in flight: group g is pending with parity pph[g]
+    bool pend[3] = {false, false, false};
+    uint32_t pph[3] = {0u, 0u, 0u};
+    auto issue = [&](int g, int c, uint32_t parity) {
+        const int bh = c / NC, n = c - bh * NC, t0 = n * C;
+        if (g == 0) {
+            tc::mbar_expect_tx(&full[0], C * C * 2 + 2 * 128 * DV);
+            for (int j = 0; j < DV / 64; ++j) {
+                tc::tma_load_3d(base + Lay::TDU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
+                tc::tma_load_3d(base + Lay::TV + j * 8192, &tmap_v, &full[0], j * 64, t0, bh);
+            }
+            tc::tma_load_2d(base + Lay::TT, &tmap_t, &full[0], 0, c * C);
+        } else if (g == 1) {
+            tc::mbar_expect_tx(&full[1], 128 * DK + (n > 0 ? 2 * DK * DV : 0) + 128 * DV);
+            for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TK + j * 8192, &tmap_k, &full[1], j * 64, t0, bh);
+            for (int j = 0; j < DV / 64; ++j) {
+                if (n > 0) tc::tma_load_2d(base + Lay::TS + j * 128 * DK, &tmap_s, &full[1], j * 64, (c - 1) * DK);
+                tc::tma_load_3d(base + Lay::TO + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
+            }
+        } else {
+            tc::mbar_expect_tx(&full[2], 128 * DK + 128 * DV + 2 * DK * DV);
+            for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TQ + j * 8192, &tmap_q, &full[2], j * 64, t0, bh);
+            for (int j = 0; j < DV / 64; ++j) {
+                tc::tma_load_3d(base + Lay::TU + j * 8192, &tmap_u, &full[2], j * 64, t0, bh);
+                tc::tma_load_2d(base + Lay::TDS + j * 128 * DK, &tmap_ds, &full[2], j * 64, c * DK);
+            }
+        }
+        pend[g] = true;
+        pph[g] = parity;
+    };
     if (tid == 0) {
-        tc::mbar_init(&full[0], 1);
-        tc::mbar_init(&full[1], 1);
+        for (int g = 0; g < 3; ++g) tc::mbar_init(&full[g], 1);
         tc::fence_mbar_init();
-        tc::mbar_expect_tx(&full[0], 128 * DK + (n > 0 ? 2 * DK * DV : 0) + C * C * 2 + 2 * 128 * DV);
-        for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TK + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
-        for (int j = 0; j < DV / 64; ++j) {
-            if (n > 0) tc::tma_load_2d(base + Lay::TS + j * 128 * DK, &tmap_s, &full[0], j * 64, ck - DK);
-            tc::tma_load_3d(base + Lay::TDU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
-            tc::tma_load_3d(base + Lay::TV + j * 8192, &tmap_v, &full[0], j * 64, t0, bh);
-        }
-        tc::tma_load_2d(base + Lay::TT, &tmap_t, &full[0], 0, chunk * C);
-        tc::mbar_expect_tx(&full[1], 128 * DK + 128 * DV + 128 * DV + 2 * DK * DV);
-        for (int j = 0; j < DK / 64; ++j) tc::tma_load_3d(base + Lay::TQ + j * 8192, &tmap_q, &full[1], j * 64, t0, bh);
-        for (int j = 0; j < DV / 64; ++j) {
-            tc::tma_load_3d(base + Lay::TO + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
-            tc::tma_load_3d(base + Lay::TU + j * 8192, &tmap_u, &full[1], j * 64, t0, bh);
-            tc::tma_load_2d(base + Lay::TDS + j * 128 * DK, &tmap_ds, &full[1], j * 64, ck);
-        }
+        for (int g = 0; g < 3; ++g) issue(g, ch, 0u);
     }
-    if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero
-        for (int e = tid; e < DK * DV; e += THREADS) {
-            const int kr = e / DV, vc = e - kr * DV;
-            const float x = S0 ? S0[(size_t)bh * DD + e] : 0.f;
-            *reinterpret_cast<__half *>(base + Lay::TS + off(DK, kr, vc & ~7) + 2 * (vc & 7)) = __float2half_rn(x);
-        }
-    }
-    __syncthreads();  // the barriers' initialisation, the initial state
-    bool ok = tc::mbar_wait(&full[0], 0, WAIT_BUDGET);
-    // K to fp16 in place (bf16 values are exact in fp16 from 2^-14 up)
-    for (int e = tid; e < 128 * DK / 16; e += THREADS) {
-        uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TK) + e;
-        uint4 u = *p;
-        u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
-        u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-        *p = u;
-    }
-    if (tid < C) {
-        const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
-        sa[tid] = c.y;
-        sfb[tid] = c.z;
-        sfl[tid] = c.w;
-    }
-    __syncthreads();
+    __syncthreads();  // the barriers' initialisation
 
     const Tile tQ{sb + Lay::TQ, C}, tK{sb + Lay::TK, C}, tO{sb + Lay::TO, C}, tU{sb + Lay::TU, C};
     const Tile tDU{sb + Lay::TDU, C}, tNR{sb + Lay::TNR, C}, tS{sb + Lay::TS, DK}, tDS{sb + Lay::TDS, DK};
@@ -628,125 +633,174 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     // warp tile: rows m0 .. m0 + 31; columns n0 .. of a 64 x N output (N / 4 columns per warp)
     const int m0 = 32 * (warp & 1), wc = warp >> 1;
     constexpr int NV = DV / 32, NKK = DK / 32;  // n-tiles of 8 per warp for N = dv, N = dk
-
-    // ---- R = V - K S and dR = Ta^T dU' ([64][dv]); da's first part dR_t . R_t; dV = dR
-    {
-        float accR[2][NV][4], accD[2][NV][4];
-        zero(accR);
-        zero(accD);
-        const int n0 = wc * (DV / 4);
-        gemm<false, true>(accR, tK, tS, m0, n0, DK, lane);
-        gemm<true, true>(accD, tT, tDU, m0, n0, C, lane);
-        float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [mt][row half]
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < NV; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
-                    const float vv = __bfloat162float(  // zero past the sequence (TMA fill)
-                        *reinterpret_cast<const __nv_bfloat16 *>(base + Lay::TV + off(C, r, c & ~7) + 2 * (c & 7)));
-                    part[mt][e >> 1] += accD[mt][nt][e] * (vv - accR[mt][nt][e]);
-                    if (r < valid) dval[(tokq + r) * DV + c] = accD[mt][nt][e];
-                    accD[mt][nt][e] = -accD[mt][nt][e];
-                }
-        store16(base + Lay::TNR, C, accD, m0, n0, lane);  // -dR
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float x = part[mt][h];
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                if ((lane & 3) == 0) sda[0][wc][acc_r(m0, mt, 2 * h, lane)] = x;
-            }
-    }
-    ok = tc::mbar_wait(&full[1], 0, WAIT_BUDGET) && ok;
-    for (int e = tid; e < 128 * DK / 16; e += THREADS) {  // Q to fp16 in place
-        uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TQ) + e;
-        uint4 u = *p;
-        u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
-        u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
-        *p = u;
-    }
-    if (!ok && tid == 0) atomicOr(&g_bwd_error, 4u);  // a copy did not land in time
-    __syncthreads();
-    // ---- G = K K^T, B = strictly-lower(-dR U'^T), dP = lower-incl(dO U'^T) ([64][64]);
-    // da's second part sum_s B_ts G_ts
-    {
-        float accG[2][2][4], accB[2][2][4];
-        zero(accG);
-        zero(accB);
-        const int n0 = wc * 16;
-        gemm<false, false>(accG, tK, tK, m0, n0, DK, lane);
-        gemm<false, false>(accB, tNR, tU, m0, n0, DV, lane);
-        float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
-                    if (c >= r) accB[mt][nt][e] = 0.f;
-                    part[mt][e >> 1] += accB[mt][nt][e] * accG[mt][nt][e];
-                }
-        store16(base + Lay::TB, C, accB, m0, n0, lane);
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float x = part[mt][h];
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                if ((lane & 3) == 0) sda[1][wc][acc_r(m0, mt, 2 * h, lane)] = x;
-            }
-        float accP[2][2][4];
-        zero(accP);
-        gemm<false, false>(accP, tO, tU, m0, n0, DV, lane);
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (acc_c(n0, nt, e, lane) > acc_r(m0, mt, e, lane)) accP[mt][nt][e] = 0.f;
-        store16(base + Lay::TP, C, accP, m0, n0, lane);
-    }
-    __syncthreads();
-    // ---- da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t;  dbeta = da df/dbeta
-    if (tid < C) {
-        const float s1 = sda[0][0][tid] + sda[0][1][tid] + sda[0][2][tid] + sda[0][3][tid];
-        const float s2 = sda[1][0][tid] + sda[1][1][tid] + sda[1][2][tid] + sda[1][3][tid];
-        const float da = tid < valid ? (s1 + s2) / sa[tid] : 0.f;
-        sa[tid] = da;  // from here on: da
-        if (tid < valid) dbeta[tokq + tid] = da * sfb[tid];
-    }
-    __syncthreads();
-    // ---- dQ = dO S^T + dP K ([64][dk])
     const int n0k = wc * (DK / 4);
-    {
-        float acc[2][NKK][4];
-        zero(acc);
-        gemm<false, false>(acc, tO, tS, m0, n0k, DV, lane);
-        gemm<false, true>(acc, tP, tK, m0, n0k, C, lane);
+    uint32_t ph = 0;
+    bool ok = true, aborted = false;
+    auto wait_group = [&](int g) {
+        const bool w = tc::mbar_wait(&full[g], ph, WAIT_BUDGET);
+        if (w && tid == 0) pend[g] = false;
+        ok = ok && w;
+    };
+    // the end of a step: every thread's accesses to the buffers about to be refilled are ordered
+    // before the copies (proxy fence, then the barrier); false if some copy did not land in time
+    auto step_end = [&]() {
+        tc::fence_async_smem();
+        aborted = __syncthreads_or(!ok);  // uniform over the CTA
+        return !aborted;
+    };
+
+    while (true) {
+        const int bh = ch / NC, n = ch - bh * NC;
+        const int t0 = n * C, valid = min(C, L - t0);
+        const size_t tokq = (size_t)bh * L + t0;
+        const int nx = next_chunk(ch);
+        if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero; S's buffer is free since the last dQ
+            for (int e = tid; e < DK * DV; e += THREADS) {
+                const int kr = e / DV, vc = e - kr * DV;
+                const float x = S0 ? S0[(size_t)bh * DD + e] : 0.f;
+                *reinterpret_cast<__half *>(base + Lay::TS + off(DK, kr, vc & ~7) + 2 * (vc & 7)) = __float2half_rn(x);
+            }
+        }
+        if (tid < C) {
+            const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
+            sa[tid] = c.y;
+            sfb[tid] = c.z;
+            sfl[tid] = c.w;
+        }
+        wait_group(1);
+        // K to fp16 in place (bf16 values are exact in fp16 from 2^-14 up)
+        for (int e = tid; e < 128 * DK / 16; e += THREADS) {
+            uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TK) + e;
+            uint4 u = *p;
+            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+            *p = u;
+        }
+        wait_group(0);
+        __syncthreads();
+
+        // ---- R = V - K S and dR = Ta^T dU' ([64][dv]); da's first part dR_t . R_t; dV = dR
+        {
+            float accR[2][NV][4], accD[2][NV][4];
+            zero(accR);
+            zero(accD);
+            const int n0 = wc * (DV / 4);
+            gemm<false, true>(accR, tK, tS, m0, n0, DK, lane);
+            gemm<true, true>(accD, tT, tDU, m0, n0, C, lane);
+            float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [mt][row half]
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < NKK; ++nt)
+                for (int nt = 0; nt < NV; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0k, nt, e, lane);
-                    if (r < valid) dq[(tokq + r) * DK + c] = acc[mt][nt][e];
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = acc_r(m0, mt, 2 * h, lane), c = acc_c(n0, nt, 0, lane);
+                        const __nv_bfloat162 vv = *reinterpret_cast<const __nv_bfloat162 *>(  // 0 past the end
+                            base + Lay::TV + off(C, r, c & ~7) + 2 * (c & 7));
+                        float *a = &accD[mt][nt][2 * h];
+                        part[mt][h] += a[0] * (__low2float(vv) - accR[mt][nt][2 * h]) +
+                                       a[1] * (__high2float(vv) - accR[mt][nt][2 * h + 1]);
+                        if (r < valid) *reinterpret_cast<float2 *>(dval + (tokq + r) * DV + c) = make_float2(a[0], a[1]);
+                        a[0] = -a[0];
+                        a[1] = -a[1];
+                    }
+            store16(base + Lay::TNR, C, accD, m0, n0, lane);  // -dR
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float x = part[mt][h];
+                    x += __shfl_xor_sync(0xffffffffu, x, 1);
+                    x += __shfl_xor_sync(0xffffffffu, x, 2);
+                    if ((lane & 3) == 0) sda[0][wc][acc_r(m0, mt, 2 * h, lane)] = x;
                 }
-    }
-    // ---- dK = U' dS'^T + dP^T Q - dR S^T + B K + B^T K + 2 da (df/dlambda) K ([64][dk])
-    {
+        }
+        if (!step_end()) break;
+        if (tid == 0 && nx < NCH) issue(0, nx, ph ^ 1u);  // Ta, dU', V are done with
+        wait_group(2);
+        for (int e = tid; e < 128 * DK / 16; e += THREADS) {  // Q to fp16 in place
+            uint4 *p = reinterpret_cast<uint4 *>(base + Lay::TQ) + e;
+            uint4 u = *p;
+            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+            *p = u;
+        }
+        if ((aborted = __syncthreads_or(!ok))) break;
+        // ---- G = K K^T, B = strictly-lower(-dR U'^T), dP = lower-incl(dO U'^T) ([64][64]);
+        // da's second part sum_s B_ts G_ts
+        {
+            float accG[2][2][4], accB[2][2][4];
+            zero(accG);
+            zero(accB);
+            const int n0 = wc * 16;
+            gemm<false, false>(accG, tK, tK, m0, n0, DK, lane);
+            gemm<false, false>(accB, tNR, tU, m0, n0, DV, lane);
+            float part[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = acc_r(m0, mt, e, lane), c = acc_c(n0, nt, e, lane);
+                        if (c >= r) accB[mt][nt][e] = 0.f;
+                        part[mt][e >> 1] += accB[mt][nt][e] * accG[mt][nt][e];
+                    }
+            store16(base + Lay::TB, C, accB, m0, n0, lane);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float x = part[mt][h];
+                    x += __shfl_xor_sync(0xffffffffu, x, 1);
+                    x += __shfl_xor_sync(0xffffffffu, x, 2);
+                    if ((lane & 3) == 0) sda[1][wc][acc_r(m0, mt, 2 * h, lane)] = x;
+                }
+            float accP[2][2][4];
+            zero(accP);
+            gemm<false, false>(accP, tO, tU, m0, n0, DV, lane);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (acc_c(n0, nt, e, lane) > acc_r(m0, mt, e, lane)) accP[mt][nt][e] = 0.f;
+            store16(base + Lay::TP, C, accP, m0, n0, lane);
+        }
+        __syncthreads();
+        // ---- da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t;  dbeta = da df/dbeta
+        if (tid < C) {
+            const float s1 = sda[0][0][tid] + sda[0][1][tid] + sda[0][2][tid] + sda[0][3][tid];
+            const float s2 = sda[1][0][tid] + sda[1][1][tid] + sda[1][2][tid] + sda[1][3][tid];
+            const float da = tid < valid ? (s1 + s2) / sa[tid] : 0.f;
+            sa[tid] = da;  // from here on: da
+            if (tid < valid) dbeta[tokq + tid] = da * sfb[tid];
+        }
+        __syncthreads();
+        // ---- dQ = dO S^T + dP K ([64][dk])
+        {
+            float acc[2][NKK][4];
+            zero(acc);
+            gemm<false, false>(acc, tO, tS, m0, n0k, DV, lane);
+            gemm<false, true>(acc, tP, tK, m0, n0k, C, lane);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NKK; ++nt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = acc_r(m0, mt, 2 * h, lane), c = acc_c(n0k, nt, 0, lane);
+                        if (r < valid)
+                            *reinterpret_cast<float2 *>(dq + (tokq + r) * DK + c) =
+                                make_float2(acc[mt][nt][2 * h], acc[mt][nt][2 * h + 1]);
+                    }
+        }
+        // ---- dK = U' dS'^T + dP^T Q - dR S^T + B K + B^T K + 2 da (df/dlambda) K ([64][dk]):
+        // the terms in S and K first, so that K, S and dO can be refilled while the rest runs
         float acc[2][NKK][4];
+        __half2 kreg[2][NKK][2];  // K at this thread's accumulator positions (exact bf16 values)
         zero(acc);
-        gemm<false, false>(acc, tU, tDS, m0, n0k, DV, lane);
-        gemm<true, true>(acc, tP, tQ, m0, n0k, C, lane);
         gemm<false, false>(acc, tNR, tS, m0, n0k, DV, lane);
         gemm<false, true>(acc, tB, tK, m0, n0k, C, lane);
         gemm<true, true>(acc, tB, tK, m0, n0k, C, lane);
@@ -755,18 +809,38 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
 #pragma unroll
             for (int nt = 0; nt < NKK; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = acc_r(m0, mt, e, lane), c = acc_c(n0k, nt, e, lane);
-                    if (r < valid) {  // K's fp16 tile holds the bf16 values exactly
-                        const float kk = __half2float(
-                            *reinterpret_cast<const __half *>(base + Lay::TK + off(C, r, c & ~7) + 2 * (c & 7)));
-                        dkey[(tokq + r) * DK + c] = acc[mt][nt][e] + 2.f * sa[r] * sfl[r] * kk;
+                for (int h = 0; h < 2; ++h) {
+                    const int r = acc_r(m0, mt, 2 * h, lane), c = acc_c(n0k, nt, 0, lane);
+                    kreg[mt][nt][h] = *reinterpret_cast<const __half2 *>(base + Lay::TK + off(C, r, c & ~7) + 2 * (c & 7));
+                }
+        if (!step_end()) break;
+        if (tid == 0 && nx < NCH) issue(1, nx, ph ^ 1u);  // K, S, dO are done with
+        gemm<false, false>(acc, tU, tDS, m0, n0k, DV, lane);
+        gemm<true, true>(acc, tP, tQ, m0, n0k, C, lane);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NKK; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = acc_r(m0, mt, 2 * h, lane), c = acc_c(n0k, nt, 0, lane);
+                    if (r < valid) {
+                        const float2 kk = __half22float2(kreg[mt][nt][h]);
+                        const float f = 2.f * sa[r] * sfl[r];
+                        *reinterpret_cast<float2 *>(dkey + (tokq + r) * DK + c) =
+                            make_float2(acc[mt][nt][2 * h] + f * kk.x, acc[mt][nt][2 * h + 1] + f * kk.y);
                     }
                 }
+        if (!step_end()) break;
+        if (tid == 0 && nx < NCH) issue(2, nx, ph ^ 1u);  // Q, U', dS' are done with
+        if (nx >= NCH) break;
+        ch = nx;
+        ph ^= 1u;
     }
-    if (!ok && tid == 0) {  // let this CTA's copies land before it exits (bounded)
-        tc::mbar_wait(&full[0], 0, WAIT_BUDGET / 4);
-        tc::mbar_wait(&full[1], 0, WAIT_BUDGET / 4);
+    if (aborted && tid == 0) {  // a copy did not land in time: let this CTA's copies land (bounded)
+        atomicOr(&g_bwd_error, 4u);
+        for (int g = 0; g < 3; ++g)
+            if (pend[g]) tc::mbar_wait(&full[g], pph[g], WAIT_BUDGET / 4);
     }
 }
 
@@ -821,8 +895,13 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
-    bwd_chunk_kernel<DK, DV><<<BH * NC, cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
-        mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC);
+    const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_chunk_kernel<DK, DV>, cw::THREADS,
+                                                      ChunkLayout<DK, DV>::SMEM) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    bwd_chunk_kernel<DK, DV><<<std::min(nch, nsm * per_sm), cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
+        mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
     count_launches(3);
     return cudaGetLastError();
 }

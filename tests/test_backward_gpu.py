@@ -196,6 +196,28 @@ def test_backward_tensor_core_path(oracle_mod, rule, kw):
         assert e <= TOL["bf16"], (name, e)
 
 
+def test_backward_chunk_walk_across_heads(oracle_mod):
+    """More chunks than SMs (6 heads of 65 chunks, the last ragged): every CTA of the per-chunk
+    kernel walks several chunks and crosses into the next head, where the state it reads is the
+    head's initial state; one head has a key of squared norm 30, fails the saved-forward gate and
+    walks on CUDA cores, so its chunks are skipped in the walk.  Every head against the oracle."""
+    x = _case(4, "exact", B=1, H=6, L=4133)
+    g = torch.Generator().manual_seed(12)
+    x["S0"] = torch.randn(1, 6, 128, 128, generator=g) * 0.1
+    k = x["k"].double()
+    k[0, 2, 100] *= (30.0 / k[0, 2, 100].pow(2).sum()).sqrt()
+    x["k"] = k.to(torch.bfloat16)
+    d = {kk: (v.cuda() if isinstance(v, torch.Tensor) else v) for kk, v in x.items()}
+    got = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    ref = oracle_mod.bwd(x["q"], x["k"], x["v"], x["beta"], x["dO"], x["S0"], x["dS"])
+    for name, gg, r in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+        for h in range(6):
+            e = rel_err(gg[0, h].cpu().numpy(), r[0, h])
+            assert e <= TOL["bf16"], (name, h, e)
+
+
 def test_backward_element_aligned_inputs_walk_on_cuda_cores(oracle_mod):
     """bf16 inputs that are only 2-byte aligned (views one element into a buffer) cannot be read
     16 bytes at a time: every head takes the CUDA-core path, with the same results' bound."""
