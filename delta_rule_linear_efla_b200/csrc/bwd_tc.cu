@@ -844,6 +844,329 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------ per-chunk products on tcgen05 (d = 128)
+// The same products transposed so that d_k or d_v (128) is the MMA M dimension and the chunk's
+// 64 tokens are N, with fp32 accumulators in tensor memory:
+//   (K S)^T = S^T K^T,  dR^T = dU'^T Ta,  G = K K^T,  dP = dO U'^T,  B = (-dR) U'^T   (the last
+//   three 64 x 64, M = 64, both operands K-major),  dQ^T = S dO^T + K^T dP^T,
+//   dK^T = dS' U'^T + Q^T dP + S (-dR)^T + K^T B^T + K^T B.
+// One CTA of 8 warps per SM walks the chunks as the mma.sync kernel does; thread 0 issues the
+// MMAs in four groups, [A] (KS)^T, dR^T, G and S dO^T; [B] dP and dS' U'^T; [C] B and S (-dR)^T,
+// after the -dR tile ([64][128], written from dR^T column by column); [D] the dP and B terms, after their tiles; and the TMA copies of the next
+// chunk.  Each warp reads one TMEM lane quarter and half of the 64 token columns.
+struct TcChunkLayout {
+    // 1024-aligned byte offsets: K twice (the next chunk's is loaded while this one's is read),
+    // Q, dO, U', dU', V, -dR [64][128]; S, dS' [128][128]; Ta, B, dP [64][64]
+    static constexpr int K0 = 0, Q = 32768, O = 49152, U = 65536, DU = 81920, V = 98304, S = 114688,
+                         DS = 147456, T = 180224, NR = 188416, BM = 204800, DP = 212992, END = 221184;
+    static constexpr int SMEM = END + 1024;  // + alignment slack
+};
+// TMEM columns of the accumulators (fp32, 64 columns each)
+constexpr uint32_t TM_R = 0, TM_DR = 64, TM_G = 128, TM_DP = 192, TM_B = 256, TM_DQ = 320, TM_DK = 384;
+
+__global__ void __launch_bounds__(cw::THREADS, 1)
+    bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_u,
+                        const __grid_constant__ CUtensorMap tmap_du, const __grid_constant__ CUtensorMap tmap_s,
+                        const __grid_constant__ CUtensorMap tmap_ds, const __grid_constant__ CUtensorMap tmap_t,
+                        const __grid_constant__ CUtensorMap tmap_v,
+                        const float4 *__restrict__ coef, const float *__restrict__ S0, const int *__restrict__ hs,
+                        float *__restrict__ dq, float *__restrict__ dkey, float *__restrict__ dval,
+                        float *__restrict__ dbeta, int L, int NC, int NCH) {
+    using Lay = TcChunkLayout;
+    using cw::off;
+    constexpr int DK = 128, DV = 128, THREADS = cw::THREADS;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+    uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    const uint32_t sb = tc::smem_u32(base);
+    __shared__ float sa[C], sfb[C], sfl[C], sda[2][4][C];  // sda[0][quarter][t], sda[1][half][t]
+    __shared__ uint64_t full[3], mbar[4];  // TMA groups; MMA groups A, C, D and the final drain
+    __shared__ uint32_t tmem_base;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qw = warp & 3, hh = warp >> 2;  // TMEM lane quarter, token-column half
+    const size_t DD = (size_t)DK * DV;
+    auto next_chunk = [&](int ch) {  // this CTA's next chunk whose head takes this path
+        for (ch += gridDim.x; ch < NCH; ch += gridDim.x)
+            if (head_ok(hs, ch / NC)) break;
+        return ch;
+    };
+    int ch = blockIdx.x;
+    if (ch < NCH && !head_ok(hs, ch / NC)) ch = next_chunk(ch);
+    if (ch >= NCH) return;  // uniform over the CTA
+
+    // thread 0's bookkeeping of the copies in flight: group g is pending with parity pph[g]
+    bool pend[3] = {false, false, false};
+    uint32_t pph[3] = {0u, 0u, 0u};
+    // group 0: Ta, dU', V and K (into buffer kbuf); group 1: S (past a head's first chunk), dO;
+    // group 2: Q, U', dS'
+    auto issue = [&](int g, int c, uint32_t parity, int kbuf) {
+        const int bh = c / NC, n = c - bh * NC, t0 = n * C;
+        if (g == 0) {
+            tc::mbar_expect_tx(&full[0], C * C * 2 + 3 * 128 * DV);
+            for (int j = 0; j < 2; ++j) {
+                tc::tma_load_3d(base + Lay::DU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
+                tc::tma_load_3d(base + Lay::V + j * 8192, &tmap_v, &full[0], j * 64, t0, bh);
+                tc::tma_load_3d(base + Lay::K0 + kbuf * 16384 + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
+            }
+            tc::tma_load_2d(base + Lay::T, &tmap_t, &full[0], 0, c * C);
+        } else if (g == 1) {
+            tc::mbar_expect_tx(&full[1], (n > 0 ? 2 * DK * DV : 0) + 128 * DV);
+            for (int j = 0; j < 2; ++j) {
+                if (n > 0) tc::tma_load_2d(base + Lay::S + j * 128 * DK, &tmap_s, &full[1], j * 64, (c - 1) * DK);
+                tc::tma_load_3d(base + Lay::O + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
+            }
+        } else {
+            tc::mbar_expect_tx(&full[2], 128 * DK + 128 * DV + 2 * DK * DV);
+            for (int j = 0; j < 2; ++j) {
+                tc::tma_load_3d(base + Lay::Q + j * 8192, &tmap_q, &full[2], j * 64, t0, bh);
+                tc::tma_load_3d(base + Lay::U + j * 8192, &tmap_u, &full[2], j * 64, t0, bh);
+                tc::tma_load_2d(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[2], j * 64, c * DK);
+            }
+        }
+        pend[g] = true;
+        pph[g] = parity;
+    };
+    if (tid == 0) {
+        for (int g = 0; g < 3; ++g) tc::mbar_init(&full[g], 1);
+        for (int g = 0; g < 4; ++g) tc::mbar_init(&mbar[g], 1);
+        tc::fence_mbar_init();
+        for (int g = 0; g < 3; ++g) issue(g, ch, 0u, 0);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tq = tmem + ((uint32_t)(32 * qw) << 16);  // this warp's lane quarter
+
+    // instruction descriptors (fp16 operands, fp32 accumulators): M, N, A MN-major, B MN-major
+    constexpr uint32_t ID_R = tc::idesc_f16(128, 64, true, false);     // S^T K^T
+    constexpr uint32_t ID_DR = tc::idesc_f16(128, 64, true, true);     // dU'^T Ta
+    constexpr uint32_t ID_G = tc::idesc_f16(64, 64, false, false);     // K K^T, dO U'^T, (-dR) U'^T
+    constexpr uint32_t ID_KM = tc::idesc_f16(128, 64, false, false);   // S dO^T, dS' U'^T, S (-dR)^T
+    constexpr uint32_t ID_KT = tc::idesc_f16(128, 64, true, false);    // K^T dP^T, K^T B^T
+    constexpr uint32_t ID_KTM = tc::idesc_f16(128, 64, true, true);    // Q^T dP, K^T B
+    // shared-memory descriptors: K-major [rows][64-column slabs] tiles step 32 bytes per 16
+    // columns and `slab` bytes per 64; MN-major tiles step 2048 bytes per 16 rows, their
+    // 64-element blocks `slab` bytes apart
+    auto kmaj = [&](int off0, int slab, int kk) {
+        return tc::sdesc(sb + off0 + (kk >> 2) * slab + (kk & 3) * 32, 16, 1024);
+    };
+    auto mnmaj = [&](int off0, int slab, int kk) { return tc::sdesc(sb + off0 + kk * 2048, slab, 1024); };
+
+    uint32_t ph = 0;
+    int kb = 0;  // K buffer of the current chunk
+    bool ok = true, aborted = false;
+    auto wait_group = [&](int g) {
+        const bool w = tc::mbar_wait(&full[g], ph, WAIT_BUDGET);
+        if (w && tid == 0) pend[g] = false;
+        ok = ok && w;
+    };
+    auto wait_mma = [&](int i) {
+        ok = tc::mbar_wait(&mbar[i], ph, WAIT_BUDGET) && ok;
+        tc::tc_fence_after();
+    };
+    // the end of a step: shared-memory writes and reads and TMEM reads of every thread are
+    // ordered before the MMAs and copies issued next; false if some wait ran out
+    auto step_end = [&]() {
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        aborted = __syncthreads_or(!ok);
+        tc::tc_fence_after();
+        return !aborted;
+    };
+    auto to_f16_in_place = [&](int off0) {  // a [64][128] bf16 tile to fp16
+        for (int e = tid; e < 1024; e += THREADS) {
+            uint4 *p = reinterpret_cast<uint4 *>(base + off0) + e;
+            uint4 u = *p;
+            u.x = tc::bf16x2_to_f16x2(u.x); u.y = tc::bf16x2_to_f16x2(u.y);
+            u.z = tc::bf16x2_to_f16x2(u.z); u.w = tc::bf16x2_to_f16x2(u.w);
+            *p = u;
+        }
+    };
+
+    while (true) {
+        const int bh = ch / NC, n = ch - bh * NC;
+        const int t0 = n * C, valid = min(C, L - t0);
+        const size_t tokq = (size_t)bh * L + t0;
+        const int nx = next_chunk(ch);
+        const int KB = Lay::K0 + kb * 16384;
+        if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero; S's buffer is free since [C]
+            for (int e = tid; e < DK * DV; e += THREADS) {
+                const int kr = e / DV, vc = e - kr * DV;
+                const float x = S0 ? S0[(size_t)bh * DD + e] : 0.f;
+                *reinterpret_cast<__half *>(base + Lay::S + off(DK, kr, vc & ~7) + 2 * (vc & 7)) = __float2half_rn(x);
+            }
+        }
+        if (tid < C) {
+            const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
+            sa[tid] = c.y;
+            sfb[tid] = c.z;
+            sfl[tid] = c.w;
+        }
+        wait_group(0);
+        wait_group(1);
+        to_f16_in_place(KB);  // bf16 values are exact in fp16 from 2^-14 up
+        if (!step_end()) break;
+        if (tid == 0) {
+            // [A] (K S)^T = S^T K^T and dR^T = dU'^T Ta; G = K K^T and S dO^T
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_R, mnmaj(Lay::S, 16384, kk), kmaj(KB, 8192, kk), ID_R, kk > 0);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DR, mnmaj(Lay::DU, 8192, kk), mnmaj(Lay::T, 8192, kk), ID_DR, kk > 0);
+            tc::mma_commit(&mbar[0]);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_G, kmaj(KB, 8192, kk), kmaj(KB, 8192, kk), ID_G, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DQ, kmaj(Lay::S, 16384, kk), kmaj(Lay::O, 8192, kk), ID_KM, kk > 0);
+            // [B] dP = dO U'^T and dK^T = dS' U'^T, once U' and dS' have landed
+            wait_group(2);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DP, kmaj(Lay::O, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::DS, 16384, kk), kmaj(Lay::U, 8192, kk), ID_KM, kk > 0);
+        }
+        __syncwarp();
+        // ---- E1: R = V - K S and dR (lane = value column v, 32 token columns per warp): dV = dR;
+        // -dR as an fp16 tile; da's first part sum_v dR_tv R_tv
+        wait_mma(0);
+        {
+            const int v = 32 * qw + lane;
+            float R[32], D[32];
+            tc::tmem_ld32(tq + TM_R + 32 * hh, R);
+            tc::tmem_ld32(tq + TM_DR + 32 * hh, D);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = 32 * hh + j;
+                const uint32_t o = off(C, t, v & ~7) + 2 * (v & 7);
+                const float vv = __bfloat162float(  // 0 past the sequence end (TMA fill)
+                    *reinterpret_cast<const __nv_bfloat16 *>(base + Lay::V + o));
+                if (t < valid) dval[(tokq + t) * DV + v] = D[j];
+                *reinterpret_cast<__half *>(base + Lay::NR + o) = __float2half_rn(-D[j]);
+                R[j] = D[j] * (vv - R[j]);
+            }
+            // sum over the warp's 32 values of v for each of its 32 tokens (lane j ends with token j)
+#pragma unroll
+            for (int s = 16; s >= 1; s >>= 1) {
+                const bool up = (lane & s) != 0;
+#pragma unroll
+                for (int j = 0; j < s; ++j) {
+                    const float keep = up ? R[j + s] : R[j], send = up ? R[j] : R[j + s];
+                    R[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+                }
+            }
+            sda[0][qw][32 * hh + lane] = R[0];
+        }
+        wait_group(2);
+        to_f16_in_place(Lay::Q);
+        if (!step_end()) break;  // -dR and Q visible to the MMAs; Ta, dU', V are done with
+        if (tid == 0) {
+            // [C] B = (-dR) U'^T and dK^T += S (-dR)^T
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_B, kmaj(Lay::NR, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::S, 16384, kk), kmaj(Lay::NR, 8192, kk), ID_KM, 1u);
+            tc::mma_commit(&mbar[1]);
+            if (nx < NCH) issue(0, nx, ph ^ 1u, kb ^ 1);
+        }
+        __syncwarp();
+        // ---- E2: G, dP, B (M = 64: row t = 16 quarter + lane at lanes 0-15 of the quarter;
+        // 32 columns s per warp): dP masked to s <= t and B to s < t as fp16 tiles; da's
+        // second part sum_s B_ts G_ts
+        wait_mma(1);
+        {
+            float G[32], P[32], Bv[32];
+            tc::tmem_ld32(tq + TM_G + 32 * hh, G);
+            tc::tmem_ld32(tq + TM_DP + 32 * hh, P);
+            tc::tmem_ld32(tq + TM_B + 32 * hh, Bv);
+            if (lane < 16) {
+                const int t = 16 * qw + lane;
+                float part = 0.f;
+                uint32_t pp[16], pb[16];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int s = 32 * hh + j;
+                    const float b = s < t ? Bv[j] : 0.f;
+                    part += b * G[j];
+                    Bv[j] = b;
+                    P[j] = s <= t ? P[j] : 0.f;
+                    if (j & 1) {
+                        pp[j >> 1] = tc::pack_f16(P[j - 1], P[j]);
+                        pb[j >> 1] = tc::pack_f16(Bv[j - 1], Bv[j]);
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int o = t * 128 + (((4 * hh + m) ^ (t & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(base + Lay::DP + o) = make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
+                    *reinterpret_cast<uint4 *>(base + Lay::BM + o) = make_uint4(pb[4 * m], pb[4 * m + 1], pb[4 * m + 2], pb[4 * m + 3]);
+                }
+                sda[1][hh][t] = part;
+            }
+        }
+        if (!step_end()) break;  // dP and B tiles visible to the MMAs; S and dO are done with
+        if (tid == 0) {
+            // [D] dQ^T += K^T dP^T; dK^T += Q^T dP + K^T B^T + K^T B
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DQ, mnmaj(KB, 8192, kk), kmaj(Lay::DP, 8192, kk), ID_KT, 1u);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(Lay::Q, 8192, kk), mnmaj(Lay::DP, 8192, kk), ID_KTM, 1u);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(KB, 8192, kk), kmaj(Lay::BM, 8192, kk), ID_KT, 1u);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(KB, 8192, kk), mnmaj(Lay::BM, 8192, kk), ID_KTM, 1u);
+            tc::mma_commit(&mbar[2]);
+            if (nx < NCH) issue(1, nx, ph ^ 1u, 0);
+        }
+        __syncwarp();
+        // ---- da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t;  dbeta = da df/dbeta
+        if (tid < C) {
+            const float s1 = sda[0][0][tid] + sda[0][1][tid] + sda[0][2][tid] + sda[0][3][tid];
+            const float da = tid < valid ? (s1 + sda[1][0][tid] + sda[1][1][tid]) / sa[tid] : 0.f;
+            sa[tid] = da;  // from here on: da
+            if (tid < valid) dbeta[tokq + tid] = da * sfb[tid];
+        }
+        __syncthreads();
+        // ---- E3: dQ^T and dK^T (lane = key column c, 32 token columns per warp);
+        // dK gets 2 da (df/dlambda) k
+        wait_mma(2);
+        {
+            const int c = 32 * qw + lane;
+            float A[32];
+            tc::tmem_ld32(tq + TM_DQ + 32 * hh, A);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = 32 * hh + j;
+                if (t < valid) dq[(tokq + t) * DK + c] = A[j];
+            }
+            tc::tmem_ld32(tq + TM_DK + 32 * hh, A);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = 32 * hh + j;
+                if (t < valid) {  // K's fp16 tile holds the bf16 values exactly
+                    const float kk = __half2float(
+                        *reinterpret_cast<const __half *>(base + KB + off(C, t, c & ~7) + 2 * (c & 7)));
+                    dkey[(tokq + t) * DK + c] = A[j] + 2.f * sa[t] * sfl[t] * kk;
+                }
+            }
+        }
+        if (!step_end()) break;  // Q, U', dS' and this K are done with
+        if (tid == 0 && nx < NCH) issue(2, nx, ph ^ 1u, 0);
+        if (nx >= NCH) break;
+        ch = nx;
+        ph ^= 1u;
+        kb ^= 1;
+    }
+    if (tid == 0) {
+        if (aborted) {  // a wait ran out: let this CTA's copies land (bounded)
+            atomicOr(&g_bwd_error, 4u);
+            for (int g = 0; g < 3; ++g)
+                if (pend[g]) tc::mbar_wait(&full[g], pph[g], WAIT_BUDGET / 4);
+        }
+        tc::mma_commit(&mbar[3]);  // arrives once every MMA issued so far has completed
+        if (!tc::mbar_wait(&mbar[3], 0, WAIT_BUDGET)) atomicOr(&g_bwd_error, 4u);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
 // dO (fp32) to fp16 for the products; and which heads take the tensor-core path.
 __global__ void __launch_bounds__(256) bwd_prepare_kernel(const float *__restrict__ dO, __half *__restrict__ dO16,
                                                          size_t n4) {
@@ -873,6 +1196,9 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(bwd_chunk_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      ChunkLayout<DK, DV>::SMEM);
+        if (e == cudaSuccess && DK == 128 && DV == 128)
+            e = cudaFuncSetAttribute(bwd_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     TcChunkLayout::SMEM);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
@@ -896,6 +1222,12 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
     const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
+    if (DK == 128 && DV == 128) {  // the products on tcgen05, one CTA per SM
+        bwd_chunk_tc_kernel<<<std::min(nch, nsm), cw::THREADS, TcChunkLayout::SMEM, s>>>(
+            mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
+        count_launches(3);
+        return cudaGetLastError();
+    }
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_chunk_kernel<DK, DV>, cw::THREADS,
                                                       ChunkLayout<DK, DV>::SMEM) != cudaSuccess || per_sm < 1)
