@@ -851,9 +851,10 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
 //   three 64 x 64, M = 64, both operands K-major),  dQ^T = S dO^T + K^T dP^T,
 //   dK^T = dS' U'^T + Q^T dP + S (-dR)^T + K^T B^T + K^T B.
 // One CTA of 8 warps per SM walks the chunks as the mma.sync kernel does; thread 0 issues the
-// MMAs in four groups, [A] (KS)^T, dR^T, G and S dO^T; [B] dP and dS' U'^T; [C] B and S (-dR)^T,
-// after the -dR tile ([64][128], written from dR^T column by column); [D] the dP and B terms, after their tiles; and the TMA copies of the next
-// chunk.  Each warp reads one TMEM lane quarter and half of the 64 token columns.
+// MMAs in five groups, each started as soon as the tiles it reads are written (the -dR tile is
+// [64][128], written from dR^T column by column), so that every epilogue but the first runs
+// beside the next group; and the TMA copies of the next chunk, in four groups, each as soon as
+// the buffers it refills are done with.  Each warp reads one TMEM lane quarter and half of the 64 token columns.
 struct TcChunkLayout {
     // 1024-aligned byte offsets: K twice (the next chunk's is loaded while this one's is read),
     // Q, dO, U', dU', V, -dR [64][128]; S, dS' [128][128]; Ta, B, dP [64][64]
@@ -881,7 +882,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     uint8_t *base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
     const uint32_t sb = tc::smem_u32(base);
     __shared__ float sa[C], sfb[C], sfl[C], sda[2][4][C];  // sda[0][quarter][t], sda[1][half][t]
-    __shared__ uint64_t full[3], mbar[4];  // TMA groups; MMA groups A, C, D and the final drain
+    __shared__ uint64_t full[4], mbar[6];  // TMA groups; MMA groups (see below) and the final drain
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -897,10 +898,10 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     if (ch >= NCH) return;  // uniform over the CTA
 
     // thread 0's bookkeeping of the copies in flight: group g is pending with parity pph[g]
-    bool pend[3] = {false, false, false};
-    uint32_t pph[3] = {0u, 0u, 0u};
-    // group 0: Ta, dU', V and K (into buffer kbuf); group 1: S (past a head's first chunk), dO;
-    // group 2: Q, U', dS'
+    bool pend[4] = {false, false, false, false};
+    uint32_t pph[4] = {0u, 0u, 0u, 0u};
+    // group 0: Ta, dU', V and K (into buffer kbuf); group 1: dO, dS'; group 2: S (past a head's
+    // first chunk), U'; group 3: Q
     auto issue = [&](int g, int c, uint32_t parity, int kbuf) {
         const int bh = c / NC, n = c - bh * NC, t0 = n * C;
         if (g == 0) {
@@ -912,27 +913,29 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             }
             tc::tma_load_2d(base + Lay::T, &tmap_t, &full[0], 0, c * C);
         } else if (g == 1) {
-            tc::mbar_expect_tx(&full[1], (n > 0 ? 2 * DK * DV : 0) + 128 * DV);
+            tc::mbar_expect_tx(&full[1], 128 * DV + 2 * DK * DV);
             for (int j = 0; j < 2; ++j) {
-                if (n > 0) tc::tma_load_2d(base + Lay::S + j * 128 * DK, &tmap_s, &full[1], j * 64, (c - 1) * DK);
                 tc::tma_load_3d(base + Lay::O + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
+                tc::tma_load_2d(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[1], j * 64, c * DK);
+            }
+        } else if (g == 2) {
+            tc::mbar_expect_tx(&full[2], (n > 0 ? 2 * DK * DV : 0) + 128 * DV);
+            for (int j = 0; j < 2; ++j) {
+                if (n > 0) tc::tma_load_2d(base + Lay::S + j * 128 * DK, &tmap_s, &full[2], j * 64, (c - 1) * DK);
+                tc::tma_load_3d(base + Lay::U + j * 8192, &tmap_u, &full[2], j * 64, t0, bh);
             }
         } else {
-            tc::mbar_expect_tx(&full[2], 128 * DK + 128 * DV + 2 * DK * DV);
-            for (int j = 0; j < 2; ++j) {
-                tc::tma_load_3d(base + Lay::Q + j * 8192, &tmap_q, &full[2], j * 64, t0, bh);
-                tc::tma_load_3d(base + Lay::U + j * 8192, &tmap_u, &full[2], j * 64, t0, bh);
-                tc::tma_load_2d(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[2], j * 64, c * DK);
-            }
+            tc::mbar_expect_tx(&full[3], 128 * DK);
+            for (int j = 0; j < 2; ++j) tc::tma_load_3d(base + Lay::Q + j * 8192, &tmap_q, &full[3], j * 64, t0, bh);
         }
         pend[g] = true;
         pph[g] = parity;
     };
     if (tid == 0) {
-        for (int g = 0; g < 3; ++g) tc::mbar_init(&full[g], 1);
-        for (int g = 0; g < 4; ++g) tc::mbar_init(&mbar[g], 1);
+        for (int g = 0; g < 4; ++g) tc::mbar_init(&full[g], 1);
+        for (int g = 0; g < 6; ++g) tc::mbar_init(&mbar[g], 1);
         tc::fence_mbar_init();
-        for (int g = 0; g < 3; ++g) issue(g, ch, 0u, 0);
+        for (int g = 0; g < 4; ++g) issue(g, ch, 0u, 0);
     }
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base, 512);
@@ -990,13 +993,19 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         }
     };
 
+    // MMA groups and their commit barriers (thread 0 issues them in this order):
+    //   mbar[0]: (K S)^T, dR^T                      -> E1
+    //   mbar[1]: G, S dO^T, dP, dS' U'^T            -> E2a (dP tile)
+    //   mbar[2]: B, S (-dR)^T (after E1's tile)     -> E2b (B tile, da)
+    //   mbar[3]: K^T dP^T, Q^T dP (after E2a)       -> E3a (dq)
+    //   mbar[4]: K^T B^T, K^T B (after E2b)         -> E3b (dk)
     while (true) {
         const int bh = ch / NC, n = ch - bh * NC;
         const int t0 = n * C, valid = min(C, L - t0);
         const size_t tokq = (size_t)bh * L + t0;
         const int nx = next_chunk(ch);
         const int KB = Lay::K0 + kb * 16384;
-        if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero; S's buffer is free since [C]
+        if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero; S's buffer is free since mbar[2]
             for (int e = tid; e < DK * DV; e += THREADS) {
                 const int kr = e / DV, vc = e - kr * DV;
                 const float x = S0 ? S0[(size_t)bh * DD + e] : 0.f;
@@ -1011,19 +1020,18 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         }
         wait_group(0);
         wait_group(1);
+        wait_group(2);
         to_f16_in_place(KB);  // bf16 values are exact in fp16 from 2^-14 up
         if (!step_end()) break;
         if (tid == 0) {
-            // [A] (K S)^T = S^T K^T and dR^T = dU'^T Ta; G = K K^T and S dO^T
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_R, mnmaj(Lay::S, 16384, kk), kmaj(KB, 8192, kk), ID_R, kk > 0);
             for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DR, mnmaj(Lay::DU, 8192, kk), mnmaj(Lay::T, 8192, kk), ID_DR, kk > 0);
             tc::mma_commit(&mbar[0]);
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_G, kmaj(KB, 8192, kk), kmaj(KB, 8192, kk), ID_G, kk > 0);
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DQ, kmaj(Lay::S, 16384, kk), kmaj(Lay::O, 8192, kk), ID_KM, kk > 0);
-            // [B] dP = dO U'^T and dK^T = dS' U'^T, once U' and dS' have landed
-            wait_group(2);
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DP, kmaj(Lay::O, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::DS, 16384, kk), kmaj(Lay::U, 8192, kk), ID_KM, kk > 0);
+            tc::mma_commit(&mbar[1]);
         }
         __syncwarp();
         // ---- E1: R = V - K S and dR (lane = value column v, 32 token columns per warp): dV = dR;
@@ -1056,60 +1064,70 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             }
             sda[0][qw][32 * hh + lane] = R[0];
         }
-        wait_group(2);
-        to_f16_in_place(Lay::Q);
-        if (!step_end()) break;  // -dR and Q visible to the MMAs; Ta, dU', V are done with
-        if (tid == 0) {
-            // [C] B = (-dR) U'^T and dK^T += S (-dR)^T
-            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_B, kmaj(Lay::NR, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
-            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::S, 16384, kk), kmaj(Lay::NR, 8192, kk), ID_KM, 1u);
-            tc::mma_commit(&mbar[1]);
-            if (nx < NCH) issue(0, nx, ph ^ 1u, kb ^ 1);
-        }
-        __syncwarp();
-        // ---- E2: G, dP, B (M = 64: row t = 16 quarter + lane at lanes 0-15 of the quarter;
-        // 32 columns s per warp): dP masked to s <= t and B to s < t as fp16 tiles; da's
-        // second part sum_s B_ts G_ts
+        // ---- E2a: dP (M = 64: row t = 16 quarter + lane at lanes 0-15 of the quarter; 32
+        // columns s per warp), masked to s <= t, as an fp16 tile; Q to fp16
         wait_mma(1);
         {
-            float G[32], P[32], Bv[32];
-            tc::tmem_ld32(tq + TM_G + 32 * hh, G);
+            float P[32];
             tc::tmem_ld32(tq + TM_DP + 32 * hh, P);
+            if (lane < 16) {
+                const int t = 16 * qw + lane;
+                uint32_t pp[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                    pp[j >> 1] = tc::pack_f16(32 * hh + j <= t ? P[j] : 0.f, 32 * hh + j + 1 <= t ? P[j + 1] : 0.f);
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(base + Lay::DP + t * 128 + (((4 * hh + m) ^ (t & 7)) << 4)) =
+                        make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
+            }
+        }
+        wait_group(3);
+        to_f16_in_place(Lay::Q);
+        if (!step_end()) break;  // -dR, dP and Q visible to the MMAs; Ta, dU', V, dO, dS' are done with
+        if (tid == 0) {
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_B, kmaj(Lay::NR, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::S, 16384, kk), kmaj(Lay::NR, 8192, kk), ID_KM, 1u);
+            tc::mma_commit(&mbar[2]);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DQ, mnmaj(KB, 8192, kk), kmaj(Lay::DP, 8192, kk), ID_KT, 1u);
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(Lay::Q, 8192, kk), mnmaj(Lay::DP, 8192, kk), ID_KTM, 1u);
+            tc::mma_commit(&mbar[3]);
+            if (nx < NCH) {
+                issue(0, nx, ph ^ 1u, kb ^ 1);
+                issue(1, nx, ph ^ 1u, 0);
+            }
+        }
+        __syncwarp();
+        // ---- E2b: G and B (M = 64 as dP): B masked to s < t as an fp16 tile; da's second part
+        // sum_s B_ts G_ts
+        wait_mma(2);
+        {
+            float G[32], Bv[32];
+            tc::tmem_ld32(tq + TM_G + 32 * hh, G);
             tc::tmem_ld32(tq + TM_B + 32 * hh, Bv);
             if (lane < 16) {
                 const int t = 16 * qw + lane;
                 float part = 0.f;
-                uint32_t pp[16], pb[16];
+                uint32_t pb[16];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const int s = 32 * hh + j;
-                    const float b = s < t ? Bv[j] : 0.f;
-                    part += b * G[j];
-                    Bv[j] = b;
-                    P[j] = s <= t ? P[j] : 0.f;
-                    if (j & 1) {
-                        pp[j >> 1] = tc::pack_f16(P[j - 1], P[j]);
-                        pb[j >> 1] = tc::pack_f16(Bv[j - 1], Bv[j]);
-                    }
+                    Bv[j] = 32 * hh + j < t ? Bv[j] : 0.f;
+                    part += Bv[j] * G[j];
+                    if (j & 1) pb[j >> 1] = tc::pack_f16(Bv[j - 1], Bv[j]);
                 }
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int o = t * 128 + (((4 * hh + m) ^ (t & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(base + Lay::DP + o) = make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
-                    *reinterpret_cast<uint4 *>(base + Lay::BM + o) = make_uint4(pb[4 * m], pb[4 * m + 1], pb[4 * m + 2], pb[4 * m + 3]);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(base + Lay::BM + t * 128 + (((4 * hh + m) ^ (t & 7)) << 4)) =
+                        make_uint4(pb[4 * m], pb[4 * m + 1], pb[4 * m + 2], pb[4 * m + 3]);
                 sda[1][hh][t] = part;
             }
         }
-        if (!step_end()) break;  // dP and B tiles visible to the MMAs; S and dO are done with
+        if (!step_end()) break;  // the B tile visible to the MMAs; S and U' are done with
         if (tid == 0) {
-            // [D] dQ^T += K^T dP^T; dK^T += Q^T dP + K^T B^T + K^T B
-            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DQ, mnmaj(KB, 8192, kk), kmaj(Lay::DP, 8192, kk), ID_KT, 1u);
-            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(Lay::Q, 8192, kk), mnmaj(Lay::DP, 8192, kk), ID_KTM, 1u);
             for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(KB, 8192, kk), kmaj(Lay::BM, 8192, kk), ID_KT, 1u);
             for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(KB, 8192, kk), mnmaj(Lay::BM, 8192, kk), ID_KTM, 1u);
-            tc::mma_commit(&mbar[2]);
-            if (nx < NCH) issue(1, nx, ph ^ 1u, 0);
+            tc::mma_commit(&mbar[4]);
+            if (nx < NCH) issue(2, nx, ph ^ 1u, 0);
         }
         __syncwarp();
         // ---- da_t = (dR_t . R_t + sum_s B_ts G_ts) / a_t;  dbeta = da df/dbeta
@@ -1119,32 +1137,31 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             sa[tid] = da;  // from here on: da
             if (tid < valid) dbeta[tokq + tid] = da * sfb[tid];
         }
-        __syncthreads();
-        // ---- E3: dQ^T and dK^T (lane = key column c, 32 token columns per warp);
-        // dK gets 2 da (df/dlambda) k
-        wait_mma(2);
-        {
-            const int c = 32 * qw + lane;
-            float A[32];
-            tc::tmem_ld32(tq + TM_DQ + 32 * hh, A);
+        // ---- E3a: dQ^T (lane = key column c, 32 token columns per warp)
+        const int c = 32 * qw + lane;
+        float A[32];
+        wait_mma(3);
+        tc::tmem_ld32(tq + TM_DQ + 32 * hh, A);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int t = 32 * hh + j;
-                if (t < valid) dq[(tokq + t) * DK + c] = A[j];
-            }
-            tc::tmem_ld32(tq + TM_DK + 32 * hh, A);
+        for (int j = 0; j < 32; ++j) {
+            const int t = 32 * hh + j;
+            if (t < valid) dq[(tokq + t) * DK + c] = A[j];
+        }
+        __syncthreads();  // da
+        // ---- E3b: dK^T, plus 2 da (df/dlambda) k
+        wait_mma(4);
+        tc::tmem_ld32(tq + TM_DK + 32 * hh, A);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int t = 32 * hh + j;
-                if (t < valid) {  // K's fp16 tile holds the bf16 values exactly
-                    const float kk = __half2float(
-                        *reinterpret_cast<const __half *>(base + KB + off(C, t, c & ~7) + 2 * (c & 7)));
-                    dkey[(tokq + t) * DK + c] = A[j] + 2.f * sa[t] * sfl[t] * kk;
-                }
+        for (int j = 0; j < 32; ++j) {
+            const int t = 32 * hh + j;
+            if (t < valid) {  // K's fp16 tile holds the bf16 values exactly
+                const float kk = __half2float(
+                    *reinterpret_cast<const __half *>(base + KB + off(C, t, c & ~7) + 2 * (c & 7)));
+                dkey[(tokq + t) * DK + c] = A[j] + 2.f * sa[t] * sfl[t] * kk;
             }
         }
-        if (!step_end()) break;  // Q, U', dS' and this K are done with
-        if (tid == 0 && nx < NCH) issue(2, nx, ph ^ 1u, 0);
+        if (!step_end()) break;  // Q and this K are done with
+        if (tid == 0 && nx < NCH) issue(3, nx, ph ^ 1u, 0);
         if (nx >= NCH) break;
         ch = nx;
         ph ^= 1u;
@@ -1153,11 +1170,11 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     if (tid == 0) {
         if (aborted) {  // a wait ran out: let this CTA's copies land (bounded)
             atomicOr(&g_bwd_error, 4u);
-            for (int g = 0; g < 3; ++g)
+            for (int g = 0; g < 4; ++g)
                 if (pend[g]) tc::mbar_wait(&full[g], pph[g], WAIT_BUDGET / 4);
         }
-        tc::mma_commit(&mbar[3]);  // arrives once every MMA issued so far has completed
-        if (!tc::mbar_wait(&mbar[3], 0, WAIT_BUDGET)) atomicOr(&g_bwd_error, 4u);
+        tc::mma_commit(&mbar[5]);  // arrives once every MMA issued so far has completed
+        if (!tc::mbar_wait(&mbar[5], 0, WAIT_BUDGET)) atomicOr(&g_bwd_error, 4u);
     }
     tc::tc_fence_before();
     __syncthreads();
