@@ -900,22 +900,22 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     // thread 0's bookkeeping of the copies in flight: group g is pending with parity pph[g]
     bool pend[4] = {false, false, false, false};
     uint32_t pph[4] = {0u, 0u, 0u, 0u};
-    // group 0: Ta, dU', V and K (into buffer kbuf); group 1: dO, dS'; group 2: S (past a head's
+    // group 0: Ta, dU' and K (into buffer kbuf); group 1: dO, dS', V; group 2: S (past a head's
     // first chunk), U'; group 3: Q
     auto issue = [&](int g, int c, uint32_t parity, int kbuf) {
         const int bh = c / NC, n = c - bh * NC, t0 = n * C;
         if (g == 0) {
-            tc::mbar_expect_tx(&full[0], C * C * 2 + 3 * 128 * DV);
+            tc::mbar_expect_tx(&full[0], C * C * 2 + 2 * 128 * DV);
             for (int j = 0; j < 2; ++j) {
                 tc::tma_load_3d(base + Lay::DU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
-                tc::tma_load_3d(base + Lay::V + j * 8192, &tmap_v, &full[0], j * 64, t0, bh);
                 tc::tma_load_3d(base + Lay::K0 + kbuf * 16384 + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
             }
             tc::tma_load_2d(base + Lay::T, &tmap_t, &full[0], 0, c * C);
         } else if (g == 1) {
-            tc::mbar_expect_tx(&full[1], 128 * DV + 2 * DK * DV);
+            tc::mbar_expect_tx(&full[1], 2 * 128 * DV + 2 * DK * DV);
             for (int j = 0; j < 2; ++j) {
                 tc::tma_load_3d(base + Lay::O + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
+                tc::tma_load_3d(base + Lay::V + j * 8192, &tmap_v, &full[1], j * 64, t0, bh);
                 tc::tma_load_2d(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[1], j * 64, c * DK);
             }
         } else if (g == 2) {
@@ -965,6 +965,14 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     uint32_t ph = 0;
     int kb = 0;  // K buffer of the current chunk
     bool ok = true, aborted = false;
+    // token tid's coefficients {lambda, a, df/dbeta, df/dlambda} of chunk c (tid < 64), loaded a
+    // chunk ahead so that the global-load latency is off the chunk's path
+    auto load_coef = [&](int c) {
+        if (tid >= C || c >= NCH) return make_float4(0.f, 1.f, 0.f, 0.f);
+        const int b2 = c / NC, t2 = (c - b2 * NC) * C + tid;
+        return t2 < L ? coef[2 * ((size_t)b2 * L + t2)] : make_float4(0.f, 1.f, 0.f, 0.f);
+    };
+    float4 coef_next = load_coef(ch);
     auto wait_group = [&](int g) {
         const bool w = tc::mbar_wait(&full[g], ph, WAIT_BUDGET);
         if (w && tid == 0) pend[g] = false;
@@ -1013,11 +1021,11 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             }
         }
         if (tid < C) {
-            const float4 c = tid < valid ? coef[2 * (tokq + tid)] : make_float4(0.f, 1.f, 0.f, 0.f);
-            sa[tid] = c.y;
-            sfb[tid] = c.z;
-            sfl[tid] = c.w;
+            sa[tid] = coef_next.y;
+            sfb[tid] = coef_next.z;
+            sfl[tid] = coef_next.w;
         }
+        coef_next = load_coef(nx);
         wait_group(0);
         wait_group(1);
         wait_group(2);
@@ -1037,6 +1045,8 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         // ---- E1: R = V - K S and dR (lane = value column v, 32 token columns per warp): dV = dR;
         // -dR as an fp16 tile; da's first part sum_v dR_tv R_tv
         wait_mma(0);
+        if (tid == 0 && nx < NCH) issue(0, nx, ph ^ 1u, kb ^ 1);  // Ta and dU' are done with
+        __syncwarp();
         {
             const int v = 32 * qw + lane;
             float R[32], D[32];
@@ -1084,7 +1094,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         }
         wait_group(3);
         to_f16_in_place(Lay::Q);
-        if (!step_end()) break;  // -dR, dP and Q visible to the MMAs; Ta, dU', V, dO, dS' are done with
+        if (!step_end()) break;  // -dR, dP and Q visible to the MMAs; V, dO, dS' are done with
         if (tid == 0) {
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_B, kmaj(Lay::NR, 8192, kk), kmaj(Lay::U, 8192, kk), ID_G, kk > 0);
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_DK, kmaj(Lay::S, 16384, kk), kmaj(Lay::NR, 8192, kk), ID_KM, 1u);
@@ -1092,10 +1102,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DQ, mnmaj(KB, 8192, kk), kmaj(Lay::DP, 8192, kk), ID_KT, 1u);
             for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tmem + TM_DK, mnmaj(Lay::Q, 8192, kk), mnmaj(Lay::DP, 8192, kk), ID_KTM, 1u);
             tc::mma_commit(&mbar[3]);
-            if (nx < NCH) {
-                issue(0, nx, ph ^ 1u, kb ^ 1);
-                issue(1, nx, ph ^ 1u, 0);
-            }
+            if (nx < NCH) issue(1, nx, ph ^ 1u, 0);
         }
         __syncwarp();
         // ---- E2b: G and B (M = 64 as dP): B masked to s < t as an fp16 tile; da's second part
