@@ -1210,6 +1210,8 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
     __half *dO16 = (__half *)ws;
     __half *dU = dO16 + ntok * DV;  // 16-byte aligned: dv is 64 or 128
     __half *dSp = dU + ntok * DV;
+    // the per-chunk products on tcgen05 at d = 128 (transposed, d the MMA M), on mma.sync otherwise
+    constexpr bool TC_CHUNK = DK == 128 && DV == 128;
     static bool attr_done[64] = {};
     int dev = 0, nsm = 148;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1217,12 +1219,14 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
         e = cudaFuncSetAttribute(bwd_state_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  RevLayout<DK, DV>::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_chunk_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     ChunkLayout<DK, DV>::SMEM);
-        if (e == cudaSuccess && DK == 128 && DV == 128)
-            e = cudaFuncSetAttribute(bwd_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     TcChunkLayout::SMEM);
+        if (e == cudaSuccess) {
+            if constexpr (TC_CHUNK)
+                e = cudaFuncSetAttribute(bwd_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcChunkLayout::SMEM);
+            else
+                e = cudaFuncSetAttribute(bwd_chunk_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         ChunkLayout<DK, DV>::SMEM);
+        }
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
@@ -1246,18 +1250,18 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
     const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
-    if (DK == 128 && DV == 128) {  // the products on tcgen05, one CTA per SM
+    if constexpr (TC_CHUNK) {  // one CTA per SM
         bwd_chunk_tc_kernel<<<std::min(nch, nsm), cw::THREADS, TcChunkLayout::SMEM, s>>>(
             mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
-        count_launches(3);
-        return cudaGetLastError();
+    } else {
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_chunk_kernel<DK, DV>, cw::THREADS,
+                                                          ChunkLayout<DK, DV>::SMEM) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        bwd_chunk_kernel<DK, DV><<<std::min(nch, nsm * per_sm), cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
+            mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
     }
-    int per_sm = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_chunk_kernel<DK, DV>, cw::THREADS,
-                                                      ChunkLayout<DK, DV>::SMEM) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    bwd_chunk_kernel<DK, DV><<<std::min(nch, nsm * per_sm), cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
-        mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
     count_launches(3);
     return cudaGetLastError();
 }
