@@ -55,15 +55,17 @@ struct RevLayout {
     static constexpr int OFF_Q = 0, OFF_K = QB, OFF_O = OFF_K + KB, OFF_T = OFF_O + OB;
     static constexpr int OFF_W = OFF_T + TB, OFF_P = OFF_W + WB;
     static constexpr int STAGE = OFF_P + PB;
-    static constexpr int SMEM = 2 * STAGE + 1024;  // + alignment slack
+    // the chain group's outputs on their way to global memory by TMA: dU' [64][DV], dS [DK][DV]
+    static constexpr int OFF_SU = 2 * STAGE, OFF_SS = OFF_SU + 128 * DV;
+    static constexpr int SMEM = OFF_SS + 2 * DK * DV + 1024;  // + alignment slack
 };
 
 // Single-arrival barriers first, then those a warpgroup arrives on once per warp.
 struct RevBars {
-    uint64_t full[2], freeS[2], wdone, pdone, d1done, d2done, drain;
-    uint64_t conv[2], w_ready, p_ready, up_ready, s_ready;
+    uint64_t full[2], freeS[2], wdone, pdone, d1done, d2done, drain, su_free, ss_free;
+    uint64_t conv[2], w_ready, p_ready, up_ready, s_ready, su_full, ss_full;
 };
-constexpr int REV_ONE = 9;
+constexpr int REV_ONE = 11;
 constexpr int REV_WARPS = 14;  // converter, side, chain warpgroups; MMA issuer; TMA producer
 constexpr int REV_THREADS = REV_WARPS * 32;
 constexpr int RW_ISSUE = 12, RW_PROD = 13;
@@ -87,6 +89,22 @@ __device__ __forceinline__ void store_row16x32(uint8_t *tile, int row, int ch0, 
 
 __device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_takes_saved(hs, bh); }
 
+// TMA stores from shared memory (bulk groups of the issuing thread)
+__device__ __forceinline__ void tma_store_2d(const void *map, const void *src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(src)), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const void *map, const void *src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one of this thread's bulk groups still reading shared memory
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every bulk group of this thread complete (its writes done)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // One CTA per head, chunks from last to first.  TMEM (fp32 columns): dS^T [0, DK), dU'^T
 // [DK, DK + 64) (fp16 dU'^T packed over its first 32 after the epilogue), W [256, 256 + DK),
 // P [384, 448), dS^T fp16 [448, 448 + DK/2).  Per chunk, in tensor-pipe order:
@@ -95,14 +113,15 @@ __device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_tak
 //   D2a  dS^T  += dO^T Q            (off the chain)
 //   W, P of the next chunk
 //   D2b  dS^T  += dU'16^T (-W)      (A = fp16 dU'^T in TMEM)
-// Outputs (fp16; a warp's lanes write consecutive columns): dU' of every token [BH][L][dv] and
-// the gradient of the state after every chunk, dSp [BH][NC][dk][dv] (dSp[NC-1] is dS_final);
-// dS0 (fp32).
+// Outputs (fp16): dU' of every token [BH][L][dv] and the gradient of the state after every
+// chunk, dSp [BH][NC][dk][dv] (dSp[NC-1] is dS_final), each written column by column into a
+// shared-memory tile (a warp's lanes write consecutive columns) and stored by TMA; dS0 (fp32).
 template <int DK, int DV>
 __global__ void __launch_bounds__(REV_THREADS, 1)
     bwd_state_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_t,
-                     const float *__restrict__ dSL, __half *__restrict__ dU, __half *__restrict__ dSp,
+                     const __grid_constant__ CUtensorMap tmap_du, const __grid_constant__ CUtensorMap tmap_ds,
+                     const float *__restrict__ dSL, __half *__restrict__ dSp,
                      float *__restrict__ dS0, const int *__restrict__ hs, int L, int NC) {
     using Lay = RevLayout<DK, DV>;
     constexpr uint32_t TM_S = 0, TM_U = DK;
@@ -348,17 +367,32 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                 tc::tmem_st16u(tmem + lane_base + TM_U + h * 16, wu[h]);  // over columns already read
             }
             rev_arrive(&bars.up_ready, lane);
-            if (vrow >= 0) {  // dU' of the chunk's tokens, fp16 [L][dv]
-                __half *dst = dU + ((size_t)bh * L + (size_t)n * C) * DV + vrow;
+            // dU' of the chunk's tokens to its staging tile ([64][dv], rows past L are not
+            // stored), once the tile's previous store has read it
+            if (gtid == 0 && i > 0) {
+                bulk_wait_read1();
+                tc::mbar_arrive(&bars.su_free);
+            }
+            if (i > 0 && !tc::mbar_wait_or_abort(&bars.su_free, (i - 1) & 1, &abort_flag, budget)) { done_all = false; break; }
+            if (vrow >= 0) {
+                uint8_t *tile = base + Lay::OFF_SU + (vrow >> 6) * 8192 + 2 * (vrow & 7);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = 32 * h + 2 * j;
                         const __half2 pr = *reinterpret_cast<const __half2 *>(&wu[h][j]);
-                        if (n * C + t < L) dst[(size_t)t * DV] = __low2half(pr);
-                        if (n * C + t + 1 < L) dst[(size_t)(t + 1) * DV] = __high2half(pr);
+                        *reinterpret_cast<__half *>(tile + tc::sw128_off(t, (vrow & 63) >> 3)) = __low2half(pr);
+                        *reinterpret_cast<__half *>(tile + tc::sw128_off(t + 1, (vrow & 63) >> 3)) = __high2half(pr);
                     }
+            }
+            tc::fence_async_smem();
+            rev_arrive(&bars.su_full, lane);
+            if (gtid == 0) {
+                if (!tc::mbar_wait_or_abort(&bars.su_full, i & 1, &abort_flag, budget)) { done_all = false; break; }
+                for (int j = 0; j < DV / 64; ++j)
+                    tma_store_3d(&tmap_du, base + Lay::OFF_SU + j * 8192, j * 64, n * C, bh);
+                bulk_commit();
             }
             if (!tc::mbar_wait_or_abort(&bars.d2done, i & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
@@ -375,17 +409,31 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                     tc::tmem_st16u(tmem + lane_base + RT_S16 + cb * 16, *reinterpret_cast<uint32_t(*)[16]>(w + cb * 16));
                 }
                 rev_arrive(&bars.s_ready, lane);
+                if (gtid == 0 && i > 0) {
+                    bulk_wait_read1();
+                    tc::mbar_arrive(&bars.ss_free);
+                }
+                if (i > 0 && !tc::mbar_wait_or_abort(&bars.ss_free, (i - 1) & 1, &abort_flag, budget)) { done_all = false; break; }
                 if (vrow >= 0) {
-                    __half *dst = dSp + ((size_t)bh * NC + (n - 1)) * DD + vrow;
+                    uint8_t *tile = base + Lay::OFF_SS + (vrow >> 6) * (DK * 128) + 2 * (vrow & 7);
 #pragma unroll
                     for (int j = 0; j < DK / 2; ++j) {
                         const __half2 pr = *reinterpret_cast<const __half2 *>(&w[j]);
-                        dst[(size_t)(2 * j) * DV] = __low2half(pr);
-                        dst[(size_t)(2 * j + 1) * DV] = __high2half(pr);
+                        *reinterpret_cast<__half *>(tile + tc::sw128_off(2 * j, (vrow & 63) >> 3)) = __low2half(pr);
+                        *reinterpret_cast<__half *>(tile + tc::sw128_off(2 * j + 1, (vrow & 63) >> 3)) = __high2half(pr);
                     }
+                }
+                tc::fence_async_smem();
+                rev_arrive(&bars.ss_full, lane);
+                if (gtid == 0) {
+                    if (!tc::mbar_wait_or_abort(&bars.ss_full, i & 1, &abort_flag, budget)) { done_all = false; break; }
+                    for (int j = 0; j < DV / 64; ++j)
+                        tma_store_2d(&tmap_ds, base + Lay::OFF_SS + j * (DK * 128), j * 64, ((int)bh * NC + n - 1) * DK);
+                    bulk_commit();
                 }
             }
         }
+        if (gtid == 0) bulk_wait_all();  // the stores have read their tiles and written dU', dSp
         if (done_all && dS0) {  // the gradient of the initial state
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {
@@ -1238,9 +1286,6 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         return cudaErrorInvalidValue;
     const size_t n4 = ntok * DV / 4;
     const int g = (int)std::min<size_t>((n4 + 255) / 256, (size_t)nsm * 16);
-    bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
-    bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, dSL, dU, dSp, dS0,
-                                                                              hs, L, NC);
     CUtensorMap mu, mdu, ms, mds, mv;
     const uint64_t rows = (uint64_t)BH * NC * DK;  // [BH][NC][dk] rows of dv columns
     if (!tmap::make_3d(&mu, u_saved, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -1249,6 +1294,9 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
+    bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
+    bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, mdu, mds, dSL, dSp,
+                                                                              dS0, hs, L, NC);
     const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
     if constexpr (TC_CHUNK) {  // one CTA per SM
         bwd_chunk_tc_kernel<<<std::min(nch, nsm), cw::THREADS, TcChunkLayout::SMEM, s>>>(
