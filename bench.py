@@ -98,6 +98,33 @@ def run_bwd(args) -> None:
     launches = efla.kernel_launches() - l0
     clocks = clk.stop()
     ms = a.elapsed_time(b) / args.steps
+    # a training step, forward then backward: chunk_fwd + bwd against the pair that keeps the
+    # forward's values for the backward (chunk_fwd_keep + bwd(kept=...)), o at the input dtype
+    train = None
+    if efla.keeps_for_bwd(x["q"], x["v"], rule=RULE):
+        o_dt = _o_dtype(w)
+
+        def plain_step():
+            efla.chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], o_dtype=o_dt, rule=RULE)
+            call()
+
+        def keep_step():
+            _, _, kept = efla.chunk_fwd_keep(x["q"], x["k"], x["v"], x["beta"], x["S0"], o_dtype=o_dt, rule=RULE)
+            efla.bwd(x["q"], x["k"], x["v"], x["beta"], dO, x["S0"], None, want_dS0=False, rule=RULE,
+                     workspace=ws, kept=kept)
+
+        train = {}
+        for name, f in (("ms_fwd_then_bwd", plain_step), ("ms_fwd_keep_then_bwd_kept", keep_step)):
+            for _ in range(3):
+                f()
+            torch.cuda.synchronize(dev)
+            a.record()
+            for _ in range(args.steps):
+                f()
+            b.record()
+            torch.cuda.synchronize(dev)
+            train[name] = a.elapsed_time(b) / args.steps
+        train["token_heads_per_s"] = w.token_heads / (train["ms_fwd_keep_then_bwd_kept"] / 1e3)
     alg = alg_bytes_bwd(w)
     peaks = _peaks()
     achieved = alg / (ms / 1e3) / 1e9
@@ -110,9 +137,10 @@ def run_bwd(args) -> None:
                      "frac": achieved / peaks["hbm"], "traffic": None,
                      "kernel": "efla_bwd (bf16 heads the saved-forward gate admits: the saving tensor-core "
                                "forward, the reverse chain over chunks on tcgen05, per-chunk gradients on "
-                               "mma.sync; other heads: the fp32 column-block walk on CUDA cores)",
+                               "tcgen05 at d = 128 and mma.sync at d = 64; other heads: the fp32 "
+                               "column-block walk on CUDA cores)",
                      "alg_bytes_per_launch": alg, "avg_launch_ms": ms},
-        "gpu_launches": int(launches), "clocks": clocks}))
+        "train_step": train, "gpu_launches": int(launches), "clocks": clocks}))
 
 
 def alg_bytes_decode(Bd, Hd, dk, dv, es=2) -> int:

@@ -215,11 +215,11 @@ size_t efla_bwd_workspace_size(int B, int H, int L, int dk, int dv) {
     return efla::bwd_workspace_bytes(B, H, L, dk, dv);
 }
 
-efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,
-                     const float *S0, const float *dO, const float *dS_final, float *dq,
-                     float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
-                     int dk, int dv, efla_dtype dt, efla_rule rule, void *workspace,
-                     size_t workspace_bytes, void *stream) {
+static efla_status bwd_entry(const void *q, const void *k, const void *v, const void *beta,
+                             const float *S0, const float *dO, const float *dS_final, float *dq,
+                             float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                             int dk, int dv, efla_dtype dt, efla_rule rule, void *workspace,
+                             size_t workspace_bytes, void *stream, const void *kept) {
     if (!rule_ok(rule)) return EFLA_ERR_RULE;
     if (!dtype_ok(dt)) return EFLA_ERR_DTYPE;
     if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
@@ -238,7 +238,57 @@ efla_status efla_bwd(const void *q, const void *k, const void *v, const void *be
     if (need > 0 && (!workspace || workspace_bytes < need)) return EFLA_ERR_WORKSPACE;
     return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_final, dq, dkey, dval, dbeta, dS0,
                                       B, H, L, dk, dv, dt == EFLA_BF16, rule == EFLA_RULE_EULER,
-                                      workspace, (cudaStream_t)stream));
+                                      workspace, (cudaStream_t)stream, kept));
+}
+
+efla_status efla_bwd(const void *q, const void *k, const void *v, const void *beta,
+                     const float *S0, const float *dO, const float *dS_final, float *dq,
+                     float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                     int dk, int dv, efla_dtype dt, efla_rule rule, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+    return bwd_entry(q, k, v, beta, S0, dO, dS_final, dq, dkey, dval, dbeta, dS0, B, H, L, dk, dv, dt, rule,
+                     workspace, workspace_bytes, stream, nullptr);
+}
+
+size_t efla_bwd_kept_size(int B, int H, int L, int dk, int dv) {
+    if (B < 1 || H < 1 || L < 1 || dk < 1 || dv < 1 || dk > 128 || dv > 128) return 0;
+    return efla::bwd_kept_bytes(B, H, L, dk, dv);
+}
+
+efla_status efla_bwd_kept(const void *q, const void *k, const void *v, const void *beta,
+                          const float *S0, const float *dO, const float *dS_final, float *dq,
+                          float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                          int dk, int dv, efla_dtype dt, efla_rule rule, const void *kept,
+                          size_t kept_bytes, void *workspace, size_t workspace_bytes, void *stream) {
+    const size_t need = efla_bwd_kept_size(B, H, L, dk, dv);
+    if (dt != EFLA_BF16 || need == 0) return EFLA_ERR_UNSUPPORTED;
+    if (!kept || kept_bytes < need) return EFLA_ERR_WORKSPACE;
+    if (!aligned16(kept)) return EFLA_ERR_ALIGN;
+    return bwd_entry(q, k, v, beta, S0, dO, dS_final, dq, dkey, dval, dbeta, dS0, B, H, L, dk, dv, dt, rule,
+                     workspace, workspace_bytes, stream, kept);
+}
+
+efla_status efla_chunk_fwd_keep(const void *q, const void *k, const void *v, const void *beta,
+                                const float *S0, void *o, float *S_final, int B, int H, int L,
+                                int dk, int dv, efla_dtype dt, efla_dtype o_dt, efla_rule rule,
+                                void *kept, size_t kept_bytes, void *stream) {
+    if (!rule_ok(rule)) return EFLA_ERR_RULE;
+    if (!dtype_ok(dt) || !dtype_ok(o_dt)) return EFLA_ERR_DTYPE;
+    if (B < 1 || H < 1 || L < 0 || dk < 1 || dv < 1) return EFLA_ERR_SHAPE;
+    if ((long long)B * H > 0x7fffffffLL || (long long)B * H * L > (1LL << 40)) return EFLA_ERR_SHAPE;
+    void *tc_ws = nullptr;
+    __half *u = nullptr, *ck = nullptr;
+    if (L < 1 || !efla::bwd_kept_regions(B, H, L, dk, dv, dt == EFLA_BF16, kept, &tc_ws, &u, &ck))
+        return EFLA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !beta || !o) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_elem(beta, dt) || !aligned16(S0) ||
+        !aligned16(o) || !aligned16(S_final))
+        return EFLA_ERR_ALIGN;
+    const size_t need = efla::bwd_kept_bytes(B, H, L, dk, dv);
+    if (!kept || kept_bytes < need) return EFLA_ERR_WORKSPACE;
+    if (!aligned16(kept)) return EFLA_ERR_ALIGN;
+    return from_cuda(efla::launch_chunk_tc_keep(q, k, v, beta, S0, o, S_final, B, H, L, dk, dv, o_dt == EFLA_BF16,
+                                                rule == EFLA_RULE_EULER, tc_ws, u, ck, (cudaStream_t)stream));
 }
 
 efla_status efla_selftest_bounded_wait(long long budget_cycles, void *stream) {

@@ -623,10 +623,29 @@ size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv) {
     return bwd_layout(B, H, L, dk, dv).total * sizeof(float);
 }
 
+// The kept buffer: the forward's workspace (Ta tiles, segment states), every token's u and the
+// state after every chunk, in the order and with the sizes of the workspace's own regions.
+size_t bwd_kept_bytes(int B, int H, int L, int dk, int dv) {
+    if (!bwd_tc_saves(B, H, L, dk, dv)) return 0;
+    const BwdLayout lay = bwd_layout(B, H, L, dk, dv);
+    return (lay.tcb - lay.tc) * sizeof(float);
+}
+
+bool bwd_kept_regions(int B, int H, int L, int dk, int dv, bool is_bf16, void *kept, void **tc_ws, __half **u,
+                      __half **ck) {
+    if (!is_bf16 || !bwd_tc_saves(B, H, L, dk, dv)) return false;
+    const BwdLayout lay = bwd_layout(B, H, L, dk, dv);
+    float *kf = (float *)kept;
+    *tc_ws = kf;
+    *u = (__half *)(kf + (lay.u - lay.tc));
+    *ck = (__half *)(kf + (lay.ck - lay.tc));
+    return true;
+}
+
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
                        const float *S0, const float *dO, const float *dSL, float *dq, float *dkey,
                        float *dval, float *dbeta, float *dS0, int B, int H, int L, int dk, int dv,
-                       bool is_bf16, bool euler, void *ws, cudaStream_t s) {
+                       bool is_bf16, bool euler, void *ws, cudaStream_t s, const void *kept) {
     const long long BH = (long long)B * H;
     const int NS = (dv + BW_CB - 1) / BW_CB;
     if (BH * NS > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -641,6 +660,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     float *state = wsf + lay.state;
     float *part = wsf + lay.part;
     __half *u_saved = nullptr, *ck_saved = nullptr;
+    void *ta_ws = wsf + lay.tc;  // the tensor-core forward's workspace (its Ta tiles)
     cudaError_t e;
     // the tensor-core forward (TMA) and backward load q, k, v, S0 and dO 16 bytes at a time and
     // store dq, dk, dv 8 bytes at a time; arrays that are only element-aligned send every head to
@@ -651,10 +671,14 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
                         al16(dO) && (S0 == nullptr || al16(S0)) && al8(dq) && al8(dkey) && al8(dval);
     if (tc_bwd) {
         // the tensor-core forward, saving u and the block states (fp16) instead of writing outputs
-        u_saved = (__half *)(wsf + lay.u);
-        ck_saved = (__half *)(wsf + lay.ck);
-        e = launch_chunk_tc_save(q, k, v, beta, S0, B, H, L, dk, dv, euler, wsf + lay.tc, u_saved, ck_saved, s);
-        if (e != cudaSuccess) return e;
+        if (kept) {  // the forward of this step kept them
+            bwd_kept_regions(B, H, L, dk, dv, true, const_cast<void *>(kept), &ta_ws, &u_saved, &ck_saved);
+        } else {
+            u_saved = (__half *)(wsf + lay.u);
+            ck_saved = (__half *)(wsf + lay.ck);
+            e = launch_chunk_tc_save(q, k, v, beta, S0, B, H, L, dk, dv, euler, ta_ws, u_saved, ck_saved, s);
+            if (e != cudaSuccess) return e;
+        }
     }
     if (ntok > 0) {
         e = cudaMemsetAsync(hs, 0, 4 * (size_t)BH * sizeof(int), s);
@@ -681,7 +705,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
         count_launches(1);
     }
     if (tc_bwd && L > 0) {
-        e = launch_bwd_tc(q, k, v, S0, dO, dSL, coef, hs, u_saved, ck_saved, wsf + lay.tc, dq, dkey, dval, dbeta,
+        e = launch_bwd_tc(q, k, v, S0, dO, dSL, coef, hs, u_saved, ck_saved, ta_ws, dq, dkey, dval, dbeta,
                           dS0, B, H, L, dk, dv, wsf + lay.tcb, s);
         if (e != cudaSuccess) return e;
     }

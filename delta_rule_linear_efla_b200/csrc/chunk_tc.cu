@@ -1008,9 +1008,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     }
                 }
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
-                if (SAVE && u_out && mode == 0 && vrow >= 0) {
+                if ((SAVE || !GATED) && u_out && mode == 0 && vrow >= 0) {
                     // u_t = a_t r_t of every token, for the backward: fp16 [B*H][L][dv] (a warp's
-                    // lanes write a token's consecutive columns)
+                    // lanes write a token's consecutive columns); also by the ungated forward that
+                    // writes o, when asked to keep it
                     const int t0 = (n0 + n) * C + h * 32;
                     __half *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
 #pragma unroll
@@ -1066,7 +1067,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
             warp_arrive(&bars.s_ready, lane);
-            if (SAVE && ck_out && mode == 0) {
+            if ((SAVE || !GATED) && ck_out && mode == 0) {
                 // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
                 // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
                 // warp-collective: every lane takes it, the lanes that hold a state column store.
@@ -1414,6 +1415,23 @@ cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, co
                                                         s, u_out, ck_out, true, nullptr);
     return launch_tc_t<64, 64, float, true, false>(q, k, v, beta, S0, nullptr, nullptr, B, H, L, euler, ws, s,
                                                    u_out, ck_out, true, nullptr);
+}
+
+cudaError_t launch_chunk_tc_keep(const void *q, const void *k, const void *v, const void *beta,
+                                 const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
+                                 int dv, bool o_bf16, bool euler, void *ws, __half *u_out, __half *ck_out,
+                                 cudaStream_t s) {
+    using bf = __nv_bfloat16;
+#define EFLA_KEEP(DK_, DV_)                                                                                \
+    return o_bf16 ? launch_tc_t<DK_, DV_, bf, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, \
+                                                            s, u_out, ck_out, true, nullptr)                  \
+                  : launch_tc_t<DK_, DV_, float, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler,  \
+                                                               ws, s, u_out, ck_out, true, nullptr)
+    if (dk == 128 && dv == 128) EFLA_KEEP(128, 128);
+    if (dk == 128 && dv == 64) EFLA_KEEP(128, 64);
+    if (dk == 64 && dv == 128) EFLA_KEEP(64, 128);
+    EFLA_KEEP(64, 64);
+#undef EFLA_KEEP
 }
 
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s) {

@@ -42,7 +42,15 @@ size_t bwd_workspace_bytes(int B, int H, int L, int dk, int dv);
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *beta,
                        const float *S0, const float *dO, const float *dSL, float *dq, float *dkey,
                        float *dval, float *dbeta, float *dS0, int B, int H, int L, int dk, int dv,
-                       bool is_bf16, bool euler, void *ws, cudaStream_t s);
+                       bool is_bf16, bool euler, void *ws, cudaStream_t s, const void *kept = nullptr);
+// A kept buffer (bwd_kept_bytes, 0 where the tensor-core backward does not run) holds the
+// tensor-core forward's workspace (its Ta tiles), every token's u and the state after every
+// chunk; bwd_kept_regions gives the three (false for sizes and dtypes the tensor-core backward
+// does not take).  launch_bwd with `kept` reads them from there instead of running that forward
+// again: launch_chunk_tc_keep must have filled them for the same inputs.
+size_t bwd_kept_bytes(int B, int H, int L, int dk, int dv);
+bool bwd_kept_regions(int B, int H, int L, int dk, int dv, bool is_bf16, void *kept, void **tc_ws, __half **u,
+                      __half **ck);
 
 // Tensor-core (tcgen05) chunkwise forward, bf16 only.
 bool tc_supported(int B, int H, int L, int dk, int dv, int chunk, bool is_bf16);
@@ -70,6 +78,12 @@ int chunk_fwd_entry(const void *q, const void *k, const void *v, const void *bet
 cudaError_t launch_chunk_tc_save(const void *q, const void *k, const void *v, const void *beta,
                                  const float *S0, int B, int H, int L, int dk, int dv, bool euler,
                                  void *ws, __half *u_out, __half *ck_out, cudaStream_t s);
+// The tensor-core forward writing o and S_final as launch_chunk_tc (chunk 64, ungated) and also
+// keeping u_out and ck_out as launch_chunk_tc_save does (ws: the workspace of that call).
+cudaError_t launch_chunk_tc_keep(const void *q, const void *k, const void *v, const void *beta,
+                                 const float *S0, void *o, float *S_final, int B, int H, int L, int dk,
+                                 int dv, bool o_bf16, bool euler, void *ws, __half *u_out, __half *ck_out,
+                                 cudaStream_t s);
 // The backward on tensor cores for the heads the saved-forward gate lets through (bf16, chunk
 // 64, dk and dv in {64, 128}, q, k, dO and S0 16-byte aligned): dO to fp16, the reverse chain
 // over the chunks (dU' of every token and the state gradient after every chunk), then every

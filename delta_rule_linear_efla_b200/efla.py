@@ -27,6 +27,7 @@ ABI_SYMBOLS = (
     "efla_kernel_launches", "efla_chunk_fwd_noalloc", "efla_alpha_rule", "efla_chunk_fwd_rule",
     "efla_recurrent_step_rule", "efla_state_affine", "efla_bwd_workspace_size", "efla_bwd",
     "efla_selftest_bounded_wait", "efla_chunk_fwd_gated", "efla_recurrent_step_gated",
+    "efla_bwd_kept_size", "efla_chunk_fwd_keep", "efla_bwd_kept",
 )
 
 _lib = None
@@ -87,6 +88,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     L.efla_chunk_fwd_gated.argtypes = [vp] * 8 + [i] * 9 + [vp, sz, vp]
     L.efla_recurrent_step_gated.restype = i
     L.efla_recurrent_step_gated.argtypes = [vp] * 7 + [i] * 7 + [vp]
+    L.efla_chunk_fwd_keep.restype = i
+    L.efla_chunk_fwd_keep.argtypes = [vp] * 7 + [i] * 8 + [vp, sz, vp]
+    L.efla_bwd_kept.restype = i
+    L.efla_bwd_kept.argtypes = [vp] * 12 + [i] * 7 + [vp, sz, vp, sz, vp]
+    L.efla_bwd_kept_size.restype = sz
+    L.efla_bwd_kept_size.argtypes = [i, i, i, i, i]
     if path is None:
         _lib = L
     return L
@@ -283,9 +290,10 @@ def state_affine(P, S_in=None, H=None, out=None, stream=None):
 
 
 def bwd(q, k, v, beta, dO, S0=None, dS_final=None, want_dS0: bool = True, rule: str = "exact",
-        workspace=None, stream=None):
+        workspace=None, stream=None, kept=None):
     """Gradients of chunk_fwd: returns (dq, dk, dv, dbeta, dS0 or None), all float32, given
-    dO = dL/do (float32 [B,H,L,dv]) and dS_final = dL/dS_final (float32 or None = 0)."""
+    dO = dL/do (float32 [B,H,L,dv]) and dS_final = dL/dS_final (float32 or None = 0).
+    kept: the buffer chunk_fwd_keep filled for the same inputs (efla_bwd_kept), or None."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L) or \
@@ -304,15 +312,49 @@ def bwd(q, k, v, beta, dO, S0=None, dS_final=None, want_dS0: bool = True, rule: 
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if need else None
-    st = load_library().efla_bwd(
+    kargs = ()
+    if kept is not None:
+        kargs = (_dev(kept, "kept"), kept.numel() * kept.element_size())
+    entry = load_library().efla_bwd_kept if kept is not None else load_library().efla_bwd
+    st = entry(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
         _dev(S0, "S0", torch.float32) if S0 is not None else None, _dev(dO, "dO", torch.float32),
         _dev(dS_final, "dS_final", torch.float32) if dS_final is not None else None,
         _dev(dq, "dq"), _dev(dkey, "dk"), _dev(dval, "dv"), _dev(dbeta, "dbeta"),
         _dev(dS0, "dS0") if dS0 is not None else None, B, H, L, dk, dv, code, _rule(rule),
-        ws_ptr, need if ws_ptr else 0, _stream_handle(stream))
-    _check(st, "efla_bwd")
+        *kargs, ws_ptr, need if ws_ptr else 0, _stream_handle(stream))
+    _check(st, "efla_bwd_kept" if kept is not None else "efla_bwd")
     return dq, dkey, dval, dbeta, dS0
+
+
+def keeps_for_bwd(q, v, chunk: int = 64, rule: str = "exact") -> bool:
+    """Whether chunk_fwd_keep takes these inputs: bf16 at the tensor-core backward's sizes."""
+    B, H, L, dk = q.shape
+    return (q.dtype == torch.bfloat16 and chunk == 64 and L > 0 and dk in (64, 128) and
+            v.shape[-1] in (64, 128) and rule in RULES)
+
+
+def chunk_fwd_keep(q, k, v, beta, S0=None, o_dtype=torch.float32, rule: str = "exact", stream=None):
+    """The forward of a training step (efla_chunk_fwd_keep): (o, S_final, kept), where o and
+    S_final are chunk_fwd's bit for bit and kept (efla_bwd_kept_size bytes) holds what
+    bwd(..., kept=kept) reads instead of running the forward again.  bf16 inputs at the
+    tensor-core sizes only (keeps_for_bwd)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or beta.shape != (B, H, L):
+        raise ValueError("shape mismatch: q,k [B,H,L,dk], v [B,H,L,dv], beta [B,H,L]")
+    code = _dtype_code(q)
+    o = torch.empty((B, H, L, dv), dtype=o_dtype, device=q.device)
+    S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(load_library().efla_bwd_kept_size(B, H, L, dk, dv))
+    kept = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load_library().efla_chunk_fwd_keep(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(beta, "beta"),
+        _dev(S0, "S0", torch.float32) if S0 is not None else None, _dev(o, "o", o_dtype),
+        _dev(S_final, "S_final", torch.float32), B, H, L, dk, dv, code, _code(o_dtype), _rule(rule),
+        _dev(kept, "kept"), need, _stream_handle(stream))
+    _check(st, "efla_chunk_fwd_keep")
+    return o, S_final, kept
 
 
 class EflaFunction(torch.autograd.Function):
@@ -321,9 +363,13 @@ class EflaFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, beta, S0, rule="exact", chunk=64):
-        o, S = chunk_fwd(q, k, v, beta, S0, chunk=chunk, rule=rule)
+        kept = None
+        if keeps_for_bwd(q, v, chunk, rule):  # the backward will read what this forward keeps
+            o, S, kept = chunk_fwd_keep(q, k, v, beta, S0, rule=rule)
+        else:
+            o, S = chunk_fwd(q, k, v, beta, S0, chunk=chunk, rule=rule)
         ctx.save_for_backward(q, k, v, beta, S0 if S0 is not None else torch.empty(0))
-        ctx.has_S0, ctx.rule = S0 is not None, rule
+        ctx.has_S0, ctx.rule, ctx.kept = S0 is not None, rule, kept
         return o, S
 
     @staticmethod
@@ -333,7 +379,8 @@ class EflaFunction(torch.autograd.Function):
             q.shape[:3] + v.shape[-1:], dtype=torch.float32, device=q.device)
         dS = dS.float().contiguous() if dS is not None else None
         dq, dk, dv, db, dS0 = bwd(q, k, v, beta, dO, S0 if ctx.has_S0 else None, dS,
-                                  want_dS0=ctx.has_S0, rule=ctx.rule)
+                                  want_dS0=ctx.has_S0, rule=ctx.rule, kept=ctx.kept)
+        ctx.kept = None
         return (dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), db.to(beta.dtype),
                 dS0 if ctx.has_S0 else None, None, None)
 

@@ -325,6 +325,39 @@ efla_status efla_bwd(const void *q, const void *k, const void *v, const void *be
                      size_t workspace_bytes, void *stream);
 
 /*
+ * A training step without the backward's second forward (the forward's own values,
+ * kept from the step's forward to its backward):
+ *
+ * efla_bwd_kept_size -- bytes of the kept buffer for these sizes: the tensor-core
+ * forward's T diag(alpha) tiles (with the sequence segments' states where it cuts the
+ * sequence), every token's alpha r and the state after every 64 tokens (fp16); 0 where
+ * the backward does not run on tensor cores (dk or dv not in {64, 128}, L = 0).
+ *
+ * efla_chunk_fwd_keep -- efla_chunk_fwd_rule at chunk 64 (same arguments; o and
+ * S_final bit for bit the same) that also fills `kept` (efla_bwd_kept_size bytes,
+ * 16-byte aligned, caller-owned until the matching efla_bwd_kept).  bf16 inputs only,
+ * q, k, v, o, S0 and S_final 16-byte aligned; EFLA_ERR_UNSUPPORTED for sizes or dtypes
+ * without a kept buffer (use efla_chunk_fwd_rule and efla_bwd); EFLA_ERR_WORKSPACE for
+ * a missing or short `kept`.
+ *
+ * efla_bwd_kept -- efla_bwd (same arguments and results, its own workspace as
+ * efla_bwd's) for a `kept` buffer that efla_chunk_fwd_keep filled for the same q, k,
+ * v, beta, S0, sizes and rule, unchanged since: the tensor-core heads read it instead
+ * of running the forward again (heads that walk on CUDA cores ignore it).  A buffer not
+ * filled that way gives wrong gradients; the library cannot tell.
+ */
+size_t efla_bwd_kept_size(int B, int H, int L, int dk, int dv);
+efla_status efla_chunk_fwd_keep(const void *q, const void *k, const void *v, const void *beta,
+                                const float *S0, void *o, float *S_final, int B, int H, int L,
+                                int dk, int dv, efla_dtype dt, efla_dtype o_dt, efla_rule rule,
+                                void *kept, size_t kept_bytes, void *stream);
+efla_status efla_bwd_kept(const void *q, const void *k, const void *v, const void *beta,
+                          const float *S0, const float *dO, const float *dS_final, float *dq,
+                          float *dkey, float *dval, float *dbeta, float *dS0, int B, int H, int L,
+                          int dk, int dv, efla_dtype dt, efla_rule rule, const void *kept,
+                          size_t kept_bytes, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Reads and clears the library's device error word after synchronising
  * `stream`.  Kernels that wait on barriers do so with bounded spins; when a
  * wait gives up the kernel records it here and exits, leaving the context

@@ -171,3 +171,29 @@ def test_bwd_workspace_size_and_alignment(lib):
     need = lib.efla_bwd_workspace_size(1, 1, 16, 16, 16)
     assert lib.efla_bwd(*args, ctypes.c_void_p(64 + 4), need, None) == EFLA_ERR_ALIGN
     assert lib.efla_bwd(*args, P, need - 4, None) == EFLA_ERR_WORKSPACE
+
+
+def test_kept_buffer_size_and_host_errors(lib):
+    """The training-step pair's kept buffer is the backward workspace's tensor-core forward
+    region, u and chunk states (every region rounded up to 256 bytes); sizes without a
+    tensor-core backward have none, and the entry points refuse them before any CUDA call."""
+    up = lambda f: (f + 63) // 64 * 64
+    B, H, L, dk, dv = 4, 16, 4096, 128, 128
+    BH, NB = B * H, 64
+    tc = lib.efla_chunk_fwd_workspace_size(B, H, L, dk, dv, 64, BF16, F32)
+    assert lib.efla_bwd_kept_size(B, H, L, dk, dv) == \
+        4 * (up(tc // 4) + up(BH * L * dv // 2) + up(BH * NB * dk * dv // 2))
+    assert lib.efla_bwd_kept_size(1, 1, 65, 8, 20) == 0
+    assert lib.efla_bwd_kept_size(1, 1, 0, 64, 64) == 0
+    P = ctypes.c_void_p(64)
+    UNSUPPORTED, WORKSPACE, ALIGN = 4, 7, 8
+    need = lib.efla_bwd_kept_size(1, 1, 64, 64, 64)
+    fwd = [P, P, P, P, None, P, P, 1, 1, 64, 64, 64]
+    assert lib.efla_chunk_fwd_keep(*fwd, F32, F32, 0, P, need, None) == UNSUPPORTED
+    assert lib.efla_chunk_fwd_keep(*fwd, BF16, F32, 0, None, 0, None) == WORKSPACE
+    assert lib.efla_chunk_fwd_keep(*fwd, BF16, F32, 0, P, need - 16, None) == WORKSPACE
+    assert lib.efla_chunk_fwd_keep(*fwd, BF16, F32, 0, ctypes.c_void_p(72), need, None) == ALIGN
+    bwd = [P, P, P, P, None, P, None, P, P, P, P, None, 1, 1, 64, 64, 64]
+    ws = lib.efla_bwd_workspace_size(1, 1, 64, 64, 64)
+    assert lib.efla_bwd_kept(*bwd, F32, 0, P, need, P, ws, None) == UNSUPPORTED
+    assert lib.efla_bwd_kept(*bwd, BF16, 0, None, 0, P, ws, None) == WORKSPACE
