@@ -89,21 +89,6 @@ __device__ __forceinline__ void store_row16x32(uint8_t *tile, int row, int ch0, 
 
 __device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_takes_saved(hs, bh); }
 
-// TMA stores from shared memory (bulk groups of the issuing thread)
-__device__ __forceinline__ void tma_store_2d(const void *map, const void *src, int c0, int c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(src)), "r"(c0), "r"(c1) : "memory");
-}
-__device__ __forceinline__ void tma_store_3d(const void *map, const void *src, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one of this thread's bulk groups still reading shared memory
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-// every bulk group of this thread complete (its writes done)
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One CTA per head, chunks from last to first.  TMEM (fp32 columns): dS^T [0, DK), dU'^T
 // [DK, DK + 64) (fp16 dU'^T packed over its first 32 after the epilogue), W [256, 256 + DK),
@@ -370,7 +355,7 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
             // dU' of the chunk's tokens to its staging tile ([64][dv], rows past L are not
             // stored), once the tile's previous store has read it
             if (gtid == 0 && i > 0) {
-                bulk_wait_read1();
+                tc::bulk_wait_read1();
                 tc::mbar_arrive(&bars.su_free);
             }
             if (i > 0 && !tc::mbar_wait_or_abort(&bars.su_free, (i - 1) & 1, &abort_flag, budget)) { done_all = false; break; }
@@ -391,8 +376,8 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
             if (gtid == 0) {
                 if (!tc::mbar_wait_or_abort(&bars.su_full, i & 1, &abort_flag, budget)) { done_all = false; break; }
                 for (int j = 0; j < DV / 64; ++j)
-                    tma_store_3d(&tmap_du, base + Lay::OFF_SU + j * 8192, j * 64, n * C, bh);
-                bulk_commit();
+                    tc::tma_store_3d(&tmap_du, base + Lay::OFF_SU + j * 8192, j * 64, n * C, bh);
+                tc::bulk_commit();
             }
             if (!tc::mbar_wait_or_abort(&bars.d2done, i & 1, &abort_flag, budget)) { done_all = false; break; }
             tc::tc_fence_after();
@@ -410,7 +395,7 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                 }
                 rev_arrive(&bars.s_ready, lane);
                 if (gtid == 0 && i > 0) {
-                    bulk_wait_read1();
+                    tc::bulk_wait_read1();
                     tc::mbar_arrive(&bars.ss_free);
                 }
                 if (i > 0 && !tc::mbar_wait_or_abort(&bars.ss_free, (i - 1) & 1, &abort_flag, budget)) { done_all = false; break; }
@@ -428,12 +413,12 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                 if (gtid == 0) {
                     if (!tc::mbar_wait_or_abort(&bars.ss_full, i & 1, &abort_flag, budget)) { done_all = false; break; }
                     for (int j = 0; j < DV / 64; ++j)
-                        tma_store_2d(&tmap_ds, base + Lay::OFF_SS + j * (DK * 128), j * 64, ((int)bh * NC + n - 1) * DK);
-                    bulk_commit();
+                        tc::tma_store_2d(&tmap_ds, base + Lay::OFF_SS + j * (DK * 128), j * 64, ((int)bh * NC + n - 1) * DK);
+                    tc::bulk_commit();
                 }
             }
         }
-        if (gtid == 0) bulk_wait_all();  // the stores have read their tiles and written dU', dSp
+        if (gtid == 0) tc::bulk_wait_all();  // the stores have read their tiles and written dU', dSp
         if (done_all && dS0) {  // the gradient of the initial state
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {

@@ -48,6 +48,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstring>
 #include <mutex>
 
 #include <type_traits>
@@ -455,7 +456,9 @@ struct StateLayout {
     static constexpr int STAGE = OFF_KH + XB;
     static constexpr int OFF_PH = 2 * STAGE, OFF_PL = OFF_PH + 8192;  // gated: P^T hi and lo
     static constexpr int BYTES = 2 * STAGE + (GATED ? 2 * 8192 : 0);
-    static constexpr int SMEM = BYTES + 1024;             // alignment slack
+    // ungated: the kept u [64][DV] and chunk state [DK][DV] (fp16) on their way out by TMA
+    static constexpr int OFF_KU = BYTES, OFF_KS = OFF_KU + (GATED ? 0 : 128 * DV);
+    static constexpr int SMEM = OFF_KS + (GATED ? 0 : 2 * DK * DV) + 1024;  // + alignment slack
     static_assert(!GATED || OFF_PL + 8192 == BYTES, "gated shared-memory layout");
 };
 
@@ -508,11 +511,11 @@ __device__ __forceinline__ void pack32_f16(const float (&v)[32], uint32_t (&w)[1
 struct StateBars {
     uint64_t fullV[2], fullQ[2], fullK[2];
     uint64_t freeV[2], freeQ[2], freeK[2];
-    uint64_t wdone, pdone, d1done, d2done, drain;
+    uint64_t wdone, pdone, d1done, d2done, drain, ku_free, ks_free;
     // per-warp arrivals (4 each) from here on
-    uint64_t conv[2], w_ready, p_ready, up_ready_a, up_ready, s_ready_a, s_ready, o_free;
+    uint64_t conv[2], w_ready, p_ready, up_ready_a, up_ready, s_ready_a, s_ready, o_free, ku_full, ks_full;
 };
-constexpr int BARS_ONE = 17;  // barriers before `conv` take a single arrival
+constexpr int BARS_ONE = 19;  // barriers before `conv` take a single arrival
 
 // Signal `bar` once this warp's TMEM and shared-memory writes are done (a shared-memory
 // writer issues fence.proxy.async first, so the tensor core sees its stores).
@@ -530,7 +533,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
-                    const __grid_constant__ CUtensorMap tmap_t, const float *__restrict__ S0,
+                    const __grid_constant__ CUtensorMap tmap_t, const __grid_constant__ CUtensorMap tmap_ku,
+                    const __grid_constant__ CUtensorMap tmap_ks, const float *__restrict__ S0,
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
                     float *__restrict__ segbuf, int G, int seg_chunks, int pass,
                     __half *__restrict__ u_out, __half *__restrict__ ck_out,
@@ -1008,15 +1012,45 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     }
                 }
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
-                if ((SAVE || !GATED) && u_out && mode == 0 && vrow >= 0) {
-                    // u_t = a_t r_t of every token, for the backward: fp16 [B*H][L][dv] (a warp's
-                    // lanes write a token's consecutive columns); also by the ungated forward that
-                    // writes o, when asked to keep it
-                    const int t0 = (n0 + n) * C + h * 32;
-                    __half *dst = u_out + ((size_t)bh * L + t0) * DV + vrow;
+                if constexpr (!GATED) {
+                    if (u_out && mode == 0) {
+                        // u_t = a_t r_t of every token, for the backward (also by the forward that
+                        // writes o, when asked to keep it): fp16 into the [64][dv] tile, column
+                        // vrow, once the tile's previous store has read it; stored by TMA
+                        if (h == 0 && n > 0) {
+                            if (gtid == 0) {
+                                tc::bulk_wait_read1();
+                                tc::mbar_arrive(&bars.ku_free);
+                            }
+                            if (!tc::mbar_wait_or_abort(&bars.ku_free, (n - 1) & 1, &abort_flag, budget)) {
+                                done_all = false;
+                                break;
+                            }
+                        }
+                        if (vrow >= 0) {
+                            uint8_t *tile = base + Lay::OFF_KU + (vrow >> 6) * 8192 + 2 * (vrow & 7);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (t0 + j < L) dst[(size_t)j * DV] = __float2half_rn(u[j]);
+                            for (int j = 0; j < 32; ++j)
+                                *reinterpret_cast<__half *>(tile + tc::sw128_off(h * 32 + j, (vrow & 63) >> 3)) =
+                                    __float2half_rn(u[j]);
+                        }
+                    }
+                }
+            }
+            if constexpr (!GATED) {
+                if (!done_all) break;
+                if (u_out && mode == 0) {  // rows past L are not stored
+                    tc::fence_async_smem();
+                    warp_arrive(&bars.ku_full, lane);
+                    if (gtid == 0) {
+                        if (!tc::mbar_wait_or_abort(&bars.ku_full, n & 1, &abort_flag, budget)) {
+                            done_all = false;
+                            break;
+                        }
+                        for (int j = 0; j < DV / 64; ++j)
+                            tc::tma_store_3d(&tmap_ku, base + Lay::OFF_KU + j * 8192, j * 64, (n0 + n) * C, bh);
+                        tc::bulk_commit();
+                    }
                 }
             }
 
@@ -1067,23 +1101,49 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
             warp_arrive(&bars.s_ready, lane);
-            if ((SAVE || !GATED) && ck_out && mode == 0) {
+            if (!GATED && ck_out && mode == 0) {
                 // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
                 // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
-                // warp-collective: every lane takes it, the lanes that hold a state column store.
-                // fp16 [B*H][NC][dk][dv] (a warp's lanes write a row's consecutive columns)
-                __half *dst = ck_out + ((size_t)bh * NC + n0 + n) * DD + (vrow >= 0 ? vrow : 0);
+                // warp-collective: every lane takes it, the lanes that hold a state column write
+                // it, fp16, into the [dk][dv] tile (column vrow) once the tile's previous store has
+                // read it; stored by TMA into [B*H][NC][dk][dv]
+                if (n > 0) {
+                    if (gtid == 0) {
+                        tc::bulk_wait_read1();
+                        tc::mbar_arrive(&bars.ks_free);
+                    }
+                    if (!tc::mbar_wait_or_abort(&bars.ks_free, (n - 1) & 1, &abort_flag, budget)) {
+                        done_all = false;
+                        break;
+                    }
+                }
+                uint8_t *tile = base + Lay::OFF_KS + (vrow >= 0 ? (vrow >> 6) * (DK * 128) + 2 * (vrow & 7) : 0);
 #pragma unroll 1
                 for (int cb = 0; cb < DK / 16; ++cb) {
                     float v[16];
                     tc::tmem_ld16(tmem + lane_base + TM_S + cb * 16, v);
                     if (vrow >= 0) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) dst[(size_t)(cb * 16 + j) * DV] = __float2half_rn(v[j]);
+                        for (int j = 0; j < 16; ++j)
+                            *reinterpret_cast<__half *>(tile + tc::sw128_off(cb * 16 + j, (vrow & 63) >> 3)) =
+                                __float2half_rn(v[j]);
                     }
+                }
+                tc::fence_async_smem();
+                warp_arrive(&bars.ks_full, lane);
+                if (gtid == 0) {
+                    if (!tc::mbar_wait_or_abort(&bars.ks_full, n & 1, &abort_flag, budget)) {
+                        done_all = false;
+                        break;
+                    }
+                    for (int j = 0; j < DV / 64; ++j)
+                        tc::tma_store_2d(&tmap_ks, base + Lay::OFF_KS + j * (DK * 128), j * 64,
+                                         ((int)bh * NC + n0 + n) * DK);
+                    tc::bulk_commit();
                 }
             }
         }
+        if (gtid == 0) tc::bulk_wait_all();  // the kept tiles' stores are done
         if (done_all && sfp) {
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {
@@ -1312,6 +1372,14 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         !make_map_2d(&mt, ws, C, (uint64_t)total * C, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     const __nv_bfloat16 *gt = (const __nv_bfloat16 *)g;
+    // the kept u and chunk states go out by TMA stores from shared-memory tiles
+    CUtensorMap mku, mks;
+    memset(&mku, 0, sizeof(mku));
+    memset(&mks, 0, sizeof(mks));
+    if (u_out && !tmap::make_3d(&mku, u_out, DV, L, BH, 64, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
+    if (ck_out && !make_map_2d(&mks, ck_out, DV, (uint64_t)total * DK, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
     const int pgrid = total < di.prep_grid ? total : di.prep_grid;
     tc_prep_kernel<DK, GATED><<<pgrid, THREADS, prep_smem_bytes<DK>(), s>>>(
         mk, (const __nv_bfloat16 *)beta, gt, (__half *)ws, L, NC, total, euler);
@@ -1324,7 +1392,7 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
         tc_state_kernel<DK, DV, TO, false, SAVE, GATED><<<BH, ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt);
         count_launches(2);
         return cudaGetLastError();
     }
@@ -1332,10 +1400,10 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
         tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt);
         seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
         tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt);
         count_launches(4);
     }
     return cudaGetLastError();
