@@ -456,11 +456,16 @@ struct StateLayout {
     static constexpr int STAGE = OFF_KH + XB;
     static constexpr int OFF_PH = 2 * STAGE, OFF_PL = OFF_PH + 8192;  // gated: P^T hi and lo
     static constexpr int BYTES = 2 * STAGE + (GATED ? 2 * 8192 : 0);
-    // ungated: the kept u [64][DV] and chunk state [DK][DV] (fp16) on their way out by TMA
-    static constexpr int OFF_KU = BYTES, OFF_KS = OFF_KU + (GATED ? 0 : 128 * DV);
-    static constexpr int SMEM = OFF_KS + (GATED ? 0 : 2 * DK * DV) + 1024;  // + alignment slack
+    static constexpr int SMEM = BYTES + 1024;             // alignment slack
+    // the forward that keeps u and the chunk states (ungated): u [64][DV] and the state
+    // [DK][DV] (fp16) on their way out by TMA, after the stages
+    static constexpr int OFF_KU = BYTES, OFF_KS = OFF_KU + 128 * DV;
     static_assert(!GATED || OFF_PL + 8192 == BYTES, "gated shared-memory layout");
 };
+
+// Shared memory the keeping and saving forwards add after the stages (StateLayout::OFF_KU, OFF_KS).
+template <int DK, int DV>
+constexpr int keep_stage_bytes() { return 128 * DV + 2 * DK * DV; }
 
 // Row of an M-row accumulator held by this thread, or -1: M = 128 puts row r in
 // lane r; M = 64 puts row r in lane (r % 16) + 32 (r / 16).
@@ -528,7 +533,7 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
 // SEG = false compiles the one-pass form only (pass 0); SEG = true also takes the segment runs.
 // SAVE: the forward of the backward pass (every token's u and the state after every chunk
 // instead of o).  GATED: the gated form, with the decays in `gate` ([B,H,L]).
-template <int DK, int DV, typename TO, bool SEG, bool SAVE = false, bool GATED = false>
+template <int DK, int DV, typename TO, bool SEG, bool SAVE = false, bool GATED = false, bool KEEP = false>
 __global__ void __launch_bounds__(ST_THREADS, 1)
     tc_state_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -539,7 +544,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     float *__restrict__ segbuf, int G, int seg_chunks, int pass,
                     __half *__restrict__ u_out, __half *__restrict__ ck_out,
                     const __nv_bfloat16 *__restrict__ gate) {
-    static_assert(!(SAVE && GATED), "the saving forward is for the ungated form");
+    static_assert(!((SAVE || KEEP) && GATED), "the saving and keeping forwards are for the ungated form");
     using Lay = StateLayout<DK, DV, GATED>;
     constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
     extern __shared__ uint8_t smem_raw[];
@@ -1012,7 +1017,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     }
                 }
                 warp_arrive(h == 0 ? &bars.up_ready_a : &bars.up_ready, lane);
-                if constexpr (!GATED) {
+                if constexpr (SAVE || KEEP) {
                     if (u_out && mode == 0) {
                         // u_t = a_t r_t of every token, for the backward (also by the forward that
                         // writes o, when asked to keep it): fp16 into the [64][dv] tile, column
@@ -1037,7 +1042,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     }
                 }
             }
-            if constexpr (!GATED) {
+            if constexpr (SAVE || KEEP) {
                 if (!done_all) break;
                 if (u_out && mode == 0) {  // rows past L are not stored
                     tc::fence_async_smem();
@@ -1101,7 +1106,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
             warp_arrive(&bars.s_ready, lane);
-            if (!GATED && ck_out && mode == 0) {
+            if ((SAVE || KEEP) && ck_out && mode == 0) {
                 // the state after this chunk, for the backward: S^T stays in TMEM until D2 of the
                 // next chunk, which waits for this warpgroup's next U' hand-over.  The TMEM load is
                 // warp-collective: every lane takes it, the lanes that hold a state column write
@@ -1143,7 +1148,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 }
             }
         }
-        if (gtid == 0) tc::bulk_wait_all();  // the kept tiles' stores are done
+        if constexpr (SAVE || KEEP)
+            if (gtid == 0) tc::bulk_wait_all();  // the kept tiles' stores are done
         if (done_all && sfp) {
 #pragma unroll
             for (int cb = 0; cb < DK / 16; ++cb) {
@@ -1327,14 +1333,22 @@ TcDevInfo tc_dev_info() {
     if (d.err == cudaSuccess && DK == DV)
         d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+    constexpr int KSMEM = StateLayout<DK, DV>::SMEM + keep_stage_bytes<DK, DV>();
     if constexpr (std::is_same<TO, float>::value) {  // the saving forward of the backward
         if (d.err == cudaSuccess)
             d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, KSMEM);
         if (d.err == cudaSuccess && DK == DV)
             d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, DV>::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, KSMEM);
     }
+    // the forward that writes o and keeps u and the chunk states
+    if (d.err == cudaSuccess)
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, false, false, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, KSMEM);
+    if (d.err == cudaSuccess && DK == DV)
+        d.err = cudaFuncSetAttribute(tc_state_kernel<DK, DV, TO, true, false, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, KSMEM);
     constexpr int GSMEM = StateLayout<DK, DV, true>::SMEM;  // the gated form
     if (d.err == cudaSuccess)
         d.err = cudaFuncSetAttribute(tc_prep_kernel<DK, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
@@ -1358,7 +1372,7 @@ TcDevInfo tc_dev_info() {
 
 // The prep kernel, then the state kernel: one CTA per head, or the segment passes.  GATED:
 // the gated form, with the decays in g.
-template <int DK, int DV, typename TO, bool SAVE, bool GATED>
+template <int DK, int DV, typename TO, bool SAVE, bool GATED, bool KEEP = false>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void *beta,
                         const float *S0, void *o, float *S_final, int B, int H, int L, bool euler,
                         void *ws, cudaStream_t s, __half *u_out, __half *ck_out, bool allow_seg,
@@ -1385,13 +1399,13 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         mk, (const __nv_bfloat16 *)beta, gt, (__half *)ws, L, NC, total, euler);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    constexpr int SSM = StateLayout<DK, DV, GATED>::SMEM;
+    constexpr int SSM = StateLayout<DK, DV, GATED>::SMEM + ((SAVE || KEEP) ? keep_stage_bytes<DK, DV>() : 0);
     const int G = allow_seg ? seg_count(BH, NC, DK, DV, di.nsm) : 1;
     if (G < 3) {
         // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
-        tc_state_kernel<DK, DV, TO, false, SAVE, GATED><<<BH, ST_THREADS, SSM, s>>>(
+        tc_state_kernel<DK, DV, TO, false, SAVE, GATED, KEEP><<<BH, ST_THREADS, SSM, s>>>(
             mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt);
         count_launches(2);
         return cudaGetLastError();
@@ -1399,10 +1413,10 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
     if constexpr (DK == DV) {
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
-        tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
+        tc_state_kernel<DK, DV, TO, true, SAVE, GATED, KEEP><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
             mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt);
         seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
-        tc_state_kernel<DK, DV, TO, true, SAVE, GATED><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
+        tc_state_kernel<DK, DV, TO, true, SAVE, GATED, KEEP><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
             mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt);
         count_launches(4);
     }
@@ -1491,10 +1505,10 @@ cudaError_t launch_chunk_tc_keep(const void *q, const void *k, const void *v, co
                                  cudaStream_t s) {
     using bf = __nv_bfloat16;
 #define EFLA_KEEP(DK_, DV_)                                                                                \
-    return o_bf16 ? launch_tc_t<DK_, DV_, bf, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler, ws, \
-                                                            s, u_out, ck_out, true, nullptr)                  \
-                  : launch_tc_t<DK_, DV_, float, false, false>(q, k, v, beta, S0, o, S_final, B, H, L, euler,  \
-                                                               ws, s, u_out, ck_out, true, nullptr)
+    return o_bf16 ? launch_tc_t<DK_, DV_, bf, false, false, true>(q, k, v, beta, S0, o, S_final, B, H, L, euler, \
+                                                                  ws, s, u_out, ck_out, true, nullptr)            \
+                  : launch_tc_t<DK_, DV_, float, false, false, true>(q, k, v, beta, S0, o, S_final, B, H, L,     \
+                                                                     euler, ws, s, u_out, ck_out, true, nullptr)
     if (dk == 128 && dv == 128) EFLA_KEEP(128, 128);
     if (dk == 128 && dv == 64) EFLA_KEEP(128, 64);
     if (dk == 64 && dv == 128) EFLA_KEEP(64, 128);
