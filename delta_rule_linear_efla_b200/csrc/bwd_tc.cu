@@ -28,6 +28,8 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cstdint>
+#include <cstring>
 #include <type_traits>
 
 #include "bwd_gate.cuh"
@@ -88,6 +90,8 @@ __device__ __forceinline__ void store_row16x32(uint8_t *tile, int row, int ch0, 
 }
 
 __device__ __forceinline__ bool head_ok(const int *hs, int bh) { return head_takes_saved(hs, bh); }
+// every bulk store group of this thread has read its shared-memory source
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 
 // One CTA per head, chunks from last to first.  TMEM (fp32 columns): dS^T [0, DK), dU'^T
@@ -903,10 +907,10 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
                         const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_u,
                         const __grid_constant__ CUtensorMap tmap_du, const __grid_constant__ CUtensorMap tmap_s,
                         const __grid_constant__ CUtensorMap tmap_ds, const __grid_constant__ CUtensorMap tmap_t,
-                        const __grid_constant__ CUtensorMap tmap_v,
-                        const float4 *__restrict__ coef, const float *__restrict__ S0, const int *__restrict__ hs,
-                        float *__restrict__ dq, float *__restrict__ dkey, float *__restrict__ dval,
-                        float *__restrict__ dbeta, int L, int NC, int NCH) {
+                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_dk,
+                        int dk_tma, const float4 *__restrict__ coef, const float *__restrict__ S0,
+                        const int *__restrict__ hs, float *__restrict__ dq, float *__restrict__ dkey,
+                        float *__restrict__ dval, float *__restrict__ dbeta, int L, int NC, int NCH) {
     using Lay = TcChunkLayout;
     using cw::off;
     constexpr int DK = 128, DV = 128, THREADS = cw::THREADS;
@@ -1063,6 +1067,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         wait_group(1);
         wait_group(2);
         to_f16_in_place(KB);  // bf16 values are exact in fp16 from 2^-14 up
+        if (tid == 0 && dk_tma) bulk_wait_read0();  // the last dk store has read -dR, B and dP's tiles
         if (!step_end()) break;
         if (tid == 0) {
             for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + TM_R, mnmaj(Lay::S, 16384, kk), kmaj(KB, 8192, kk), ID_R, kk > 0);
@@ -1188,19 +1193,27 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             if (t < valid) dq[(tokq + t) * DK + c] = A[j];
         }
         __syncthreads();  // da
-        // ---- E3b: dK^T, plus 2 da (df/dlambda) k
+        // ---- E3b: dK^T, plus 2 da (df/dlambda) k; into the [64][128] fp32 tile over -dR, B and
+        // dP (their products are done), stored by TMA (rows past L are not stored), or straight
+        // to global memory where dk is not 16-byte aligned
         wait_mma(4);
         tc::tmem_ld32(tq + TM_DK + 32 * hh, A);
+        float *dk_tile = reinterpret_cast<float *>(base + Lay::NR);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int t = 32 * hh + j;
-            if (t < valid) {  // K's fp16 tile holds the bf16 values exactly
-                const float kk = __half2float(
-                    *reinterpret_cast<const __half *>(base + KB + off(C, t, c & ~7) + 2 * (c & 7)));
-                dkey[(tokq + t) * DK + c] = A[j] + 2.f * sa[t] * sfl[t] * kk;
-            }
+            // K's fp16 tile holds the bf16 values exactly (zero past the sequence end)
+            const float kk = __half2float(
+                *reinterpret_cast<const __half *>(base + KB + off(C, t, c & ~7) + 2 * (c & 7)));
+            const float x = A[j] + 2.f * sa[t] * sfl[t] * kk;
+            if (dk_tma) dk_tile[t * DK + c] = x;
+            else if (t < valid) dkey[(tokq + t) * DK + c] = x;
         }
-        if (!step_end()) break;  // Q and this K are done with
+        if (!step_end()) break;  // Q and this K are done with; the dk tile written
+        if (tid == 0 && dk_tma) {
+            tc::tma_store_3d(&tmap_dk, dk_tile, 0, t0, bh);
+            tc::bulk_commit();
+        }
         if (tid == 0 && nx < NCH) issue(3, nx, ph ^ 1u, 0);
         if (nx >= NCH) break;
         ch = nx;
@@ -1213,6 +1226,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
             for (int g = 0; g < 4; ++g)
                 if (pend[g]) tc::mbar_wait(&full[g], pph[g], WAIT_BUDGET / 4);
         }
+        tc::bulk_wait_all();       // the dk stores are done
         tc::mma_commit(&mbar[5]);  // arrives once every MMA issued so far has completed
         if (!tc::mbar_wait(&mbar[5], 0, WAIT_BUDGET)) atomicOr(&g_bwd_error, 4u);
     }
@@ -1284,8 +1298,21 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
                                                                               dS0, hs, L, NC);
     const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
     if constexpr (TC_CHUNK) {  // one CTA per SM
+        // dk by TMA stores of [64][dk] fp32 row-major tiles where dk is 16-byte aligned
+        CUtensorMap mdk;
+        memset(&mdk, 0, sizeof(mdk));
+        int dk_tma = 0;
+        if (((uintptr_t)dkey & 15) == 0) {
+            auto fn = tmap::encode_fn();
+            const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)L, (cuuint64_t)BH};
+            const cuuint64_t strides[2] = {(cuuint64_t)DK * 4, (cuuint64_t)L * DK * 4};
+            const cuuint32_t box[3] = {(cuuint32_t)DK, (cuuint32_t)C, 1}, es[3] = {1, 1, 1};
+            dk_tma = fn && fn(&mdk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dkey, dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        }
         bwd_chunk_tc_kernel<<<std::min(nch, nsm), cw::THREADS, TcChunkLayout::SMEM, s>>>(
-            mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
+            mq, mk, mo, mu, mdu, ms, mds, mt, mv, mdk, dk_tma, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
     } else {
         int per_sm = 1;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_chunk_kernel<DK, DV>, cw::THREADS,

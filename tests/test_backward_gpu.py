@@ -243,6 +243,37 @@ def test_backward_captured_in_a_cuda_graph_matches_eager():
         assert torch.equal(a, b) and torch.equal(c, b)
 
 
+def test_backward_dk_only_8_byte_aligned_matches():
+    """The tensor-core backward stores dk by TMA from a shared-memory tile where dk is 16-byte
+    aligned, and with its own stores where it is only 8-byte aligned: the same gradients, bit for
+    bit (a call through the C ABI with dk one pair of floats into a buffer)."""
+    import ctypes
+
+    x = _case(4, "exact", B=1, H=2, L=200)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    B, H, L, dv = x["v"].shape
+    dk = x["k"].shape[-1]
+    ref = efla.bwd(d["q"], d["k"], d["v"], d["beta"], d["dO"], d["S0"], d["dS"])
+    lib = efla.load_library()
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dq, dvv, db = torch.empty(B, H, L, dk, **f32), torch.empty(B, H, L, dv, **f32), torch.empty(B, H, L, **f32)
+    dS0 = torch.empty(B, H, dk, dv, **f32)
+    buf = torch.empty(B * H * L * dk + 2, **f32)
+    dkey = buf[2:].view(B, H, L, dk)
+    assert dkey.data_ptr() % 16 == 8
+    need = int(lib.efla_bwd_workspace_size(B, H, L, dk, dv))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    st = lib.efla_bwd(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["beta"].data_ptr(),
+                      d["S0"].data_ptr() if d["S0"] is not None else None, d["dO"].data_ptr(),
+                      d["dS"].data_ptr(), dq.data_ptr(),
+                      dkey.data_ptr(), dvv.data_ptr(), db.data_ptr(), dS0.data_ptr(), B, H, L, dk, dv,
+                      efla.EFLA_BF16, 0, ws.data_ptr(), need, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == 0 and efla.last_device_error() == 0
+    for a, b in zip((dq, dkey, dvv, db, dS0), ref):
+        assert torch.equal(a, b)
+
+
 def test_backward_element_aligned_inputs_walk_on_cuda_cores(oracle_mod):
     """bf16 inputs that are only 2-byte aligned (views one element into a buffer) cannot be read
     16 bytes at a time: every head takes the CUDA-core path, with the same results' bound."""
