@@ -214,14 +214,18 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
             constexpr uint32_t id_2a = tc::idesc_f16(DV, DK, true, true);   // dO^T Q
             constexpr uint32_t id_2b = tc::idesc_f16(DV, DK, false, true);  // dU'16^T (-W)
             auto stage_addr = [&](int i) { return sb + (i & 1) * Lay::STAGE; };
-            auto issue_wp = [&](int i) {  // W and P of local chunk i (into their TMEM columns)
+            auto issue_w = [&](int i) {  // W of local chunk i (into its TMEM columns)
                 const uint32_t stg = stage_addr(i);
-                const uint32_t q = stg + Lay::OFF_Q, k = stg + Lay::OFF_K, t = stg + Lay::OFF_T;
+                const uint32_t k = stg + Lay::OFF_K, t = stg + Lay::OFF_T;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + RT_W, tc::sdesc(t + kk * 32, 16, 1024), tc::sdesc(k + kk * 2048, 8192, 1024),
                                  id_w, kk > 0);
                 tc::mma_commit(&bars.wdone);
+            };
+            auto issue_p = [&](int i) {  // P of local chunk i (into its TMEM columns)
+                const uint32_t stg = stage_addr(i);
+                const uint32_t q = stg + Lay::OFF_Q, k = stg + Lay::OFF_K;
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
                     tc::mma_bf16(tmem + RT_P, tc::sdesc(q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
@@ -236,7 +240,8 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
             if (ok) {
                 tc::tc_fence_after();
                 issued_any = true;
-                issue_wp(0);
+                issue_w(0);
+                issue_p(0);
             }
             for (int i = 0; ok && i < NC; ++i) {
                 const int st = i & 1;
@@ -263,13 +268,13 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_S, tc::sdesc(o + kk * 2048, 8192, 1024), tc::sdesc(q + kk * 2048, 8192, 1024),
                                  id_2a, 1u);
-                // W and P of the next chunk, once the side group has read this chunk's out of TMEM
-                // (-W of this chunk is then in shared memory too; its P was read before D1a)
+                // W of the next chunk, once the side group has read this chunk's out of TMEM (-W of
+                // this chunk is then in shared memory too)
                 if (!wait(&bars.w_ready, i & 1)) break;
                 if (i + 1 < NC) {
                     if (!wait(&bars.conv[(i + 1) & 1], ((i + 1) >> 1) & 1)) break;
                     tc::tc_fence_after();
-                    issue_wp(i + 1);
+                    issue_w(i + 1);
                 }
                 // D2b: dS^T += dU'16^T (-W)
                 if (!wait(&bars.up_ready, i & 1)) break;
@@ -279,6 +284,9 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                     tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8, tc::sdesc(w + kk * 2048, 8192, 1024), id_2b, 1u);
                 tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeS[st]);
+                // P of the next chunk after D2b, off the chain's path between D1b and D2b (this
+                // chunk's P was read out of TMEM before D1a)
+                if (i + 1 < NC) issue_p(i + 1);
             }
             if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
                 tc::mma_commit(&bars.drain);
