@@ -268,15 +268,8 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_S, tc::sdesc(o + kk * 2048, 8192, 1024), tc::sdesc(q + kk * 2048, 8192, 1024),
                                  id_2a, 1u);
-                // W of the next chunk, once the side group has read this chunk's out of TMEM (-W of
-                // this chunk is then in shared memory too)
+                // D2b: dS^T += dU'16^T (-W)  (-W of this chunk is in shared memory: w_ready)
                 if (!wait(&bars.w_ready, i & 1)) break;
-                if (i + 1 < NC) {
-                    if (!wait(&bars.conv[(i + 1) & 1], ((i + 1) >> 1) & 1)) break;
-                    tc::tc_fence_after();
-                    issue_w(i + 1);
-                }
-                // D2b: dS^T += dU'16^T (-W)
                 if (!wait(&bars.up_ready, i & 1)) break;
                 tc::tc_fence_after();
 #pragma unroll
@@ -284,9 +277,14 @@ __global__ void __launch_bounds__(REV_THREADS, 1)
                     tc::mma_tmem_a(tmem + TM_S, tmem + TM_U + kk * 8, tc::sdesc(w + kk * 2048, 8192, 1024), id_2b, 1u);
                 tc::mma_commit(&bars.d2done);
                 tc::mma_commit(&bars.freeS[st]);
-                // P of the next chunk after D2b, off the chain's path between D1b and D2b (this
-                // chunk's P was read out of TMEM before D1a)
-                if (i + 1 < NC) issue_p(i + 1);
+                // W and P of the next chunk after D2b, off the chain's path between D1b and D2b
+                // (this chunk's W and P were read out of TMEM before: w_ready, and before D1a)
+                if (i + 1 < NC) {
+                    if (!wait(&bars.conv[(i + 1) & 1], ((i + 1) >> 1) & 1)) break;
+                    tc::tc_fence_after();
+                    issue_w(i + 1);
+                    issue_p(i + 1);
+                }
             }
             if (abort_flag && issued_any) {  // wait (bounded) for every issued MMA to finish
                 tc::mma_commit(&bars.drain);
