@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                     TO *__restrict__ o, float *__restrict__ S_final, int L, int NC,
                     float *__restrict__ segbuf, int G, int seg_chunks, int pass,
                     __half *__restrict__ u_out, __half *__restrict__ ck_out,
-                    const __nv_bfloat16 *__restrict__ gate) {
+                    const __nv_bfloat16 *__restrict__ gate, uint8_t *ta_drop) {
     static_assert(!((SAVE || KEEP) && GATED), "the saving and keeping forwards are for the ungated form");
     using Lay = StateLayout<DK, DV, GATED>;
     constexpr uint32_t TM_S = 0, TM_O = DK, TM_U = DK + 64;
@@ -661,6 +661,27 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     if (warp == W_PROD) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
+            // The plain forward reads its tiles once, so they come in under evict-first: the
+            // k and Ta tiles that the prep kernel has just read or written then stay in L2 for
+            // this kernel.  The saving and keeping forwards load normally (the backward that
+            // follows them reads the same tiles again).
+            constexpr bool ONCE = !SAVE && !KEEP;
+            const uint64_t pol = ONCE ? tc::l2_evict_first_policy() : 0ull;
+            auto load3 = [&](void *dst, const CUtensorMap *m, uint64_t *b, int c0, int c1, int c2) {
+                if constexpr (ONCE) tc::tma_load_3d_hint(dst, m, b, c0, c1, c2, pol);
+                else tc::tma_load_3d(dst, m, b, c0, c1, c2);
+            };
+            // A run over the whole sequence that only outputs is the last reader of its Ta tiles:
+            // with ta_drop set (the tiles' base, 128-byte aligned), each tile's lines leave L2
+            // unwritten once its stage is released, which saves their write-back to HBM.
+            auto drop_ta = [&](int n) {
+                if constexpr (ONCE && !SEG) {
+                    if (ta_drop) {
+                        const uint8_t *t = ta_drop + (size_t)(bh * NC + n) * (C * C * 2);
+                        for (int l = 0; l < C * C * 2 / 128; ++l) tc::l2_discard_line(t + 128 * l);
+                    }
+                }
+            };
             int last[2] = {-1, -1};
             for (int i = 0; i < cnt; ++i) {
                 const int n = n0 + i, st = i & 1;
@@ -671,22 +692,31 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 if (mode != 2) {
 #pragma unroll
                     for (int j = 0; j < DV / 64; ++j)
-                        tc::tma_load_3d(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
+                        load3(stg + Lay::OFF_V + j * 8192, &tmap_v, &bars.fullV[st], j * 64, n * C, bh);
                 }
-                tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C);
+                if constexpr (ONCE) tc::tma_load_2d_hint(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C, pol);
+                else tc::tma_load_2d(stg + Lay::OFF_T, &tmap_t, &bars.fullV[st], 0, (bh * NC + n) * C);
                 if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeQ[st], par, &abort_flag, budget)) break;
                 tc::mbar_expect_tx(&bars.fullQ[st], SAVE ? 0 : DK * 128);  // the saving forward reads no q
                 if constexpr (!SAVE) {
 #pragma unroll
                     for (int j = 0; j < DK / 64; ++j)
-                        tc::tma_load_3d(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
+                        load3(stg + Lay::OFF_QW + j * Lay::QW_SLAB, &tmap_q, &bars.fullQ[st], j * 64, n * C, bh);
                 }
                 if (i >= 2 && !tc::mbar_wait_or_abort(&bars.freeK[st], par, &abort_flag, budget)) break;
                 tc::mbar_expect_tx(&bars.fullK[st], DK * 128);
 #pragma unroll
                 for (int j = 0; j < DK / 64; ++j)
-                    tc::tma_load_3d(stg + Lay::OFF_KP + j * 8192, &tmap_k, &bars.fullK[st], j * 64, n * C, bh);
+                    load3(stg + Lay::OFF_KP + j * 8192, &tmap_k, &bars.fullK[st], j * 64, n * C, bh);
                 last[st] = i;
+                if (i >= 2) drop_ta(n - 2);  // its stage was released above
+            }
+            if (!abort_flag) {  // the last two chunks' tiles, once their stages are released
+                for (int j = cnt < 2 ? 0 : cnt - 2; j < cnt; ++j) {
+                    if (!(ONCE && !SEG) || !ta_drop) break;
+                    if (!tc::mbar_wait_or_abort(&bars.freeV[j & 1], (j >> 1) & 1, &abort_flag, budget)) break;
+                    drop_ta(n0 + j);
+                }
             }
             if (abort_flag) {  // let this CTA's own copies land before it exits (bounded)
                 for (int st = 0; st < 2; ++st) {
@@ -1405,8 +1435,10 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         // One CTA per head.  A grid of at most half the SM count lands one CTA per TPC;
         // two heads' chunk loops on the two SMs of one TPC each run 15-25% slower
         // (measured), so nothing else is scheduled beside this kernel.
+        // the plain forward drops its Ta tiles from L2 as it goes (nothing reads them again)
+        uint8_t *drop = (!SAVE && !KEEP && ((uintptr_t)ws & 127u) == 0) ? (uint8_t *)ws : nullptr;
         tc_state_kernel<DK, DV, TO, false, SAVE, GATED, KEEP><<<BH, ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, nullptr, 1, NC, 0, u_out, ck_out, gt, drop);
         count_launches(2);
         return cudaGetLastError();
     }
@@ -1414,10 +1446,10 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const void 
         const int seg_chunks = (NC + G - 1) / G;
         float *segbuf = (float *)((uint8_t *)ws + ta_bytes(total));
         tc_state_kernel<DK, DV, TO, true, SAVE, GATED, KEEP><<<BH * (2 * G - 3), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 1, u_out, ck_out, gt, nullptr);
         seg_combine_kernel<DK><<<BH * (DV / 16), DK, 0, s>>>(segbuf, G);
         tc_state_kernel<DK, DV, TO, true, SAVE, GATED, KEEP><<<BH * (G - 1), ST_THREADS, SSM, s>>>(
-            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt);
+            mq, mk, mv, mt, mku, mks, S0, (TO *)o, S_final, L, NC, segbuf, G, seg_chunks, 2, u_out, ck_out, gt, nullptr);
         count_launches(4);
     }
     return cudaGetLastError();

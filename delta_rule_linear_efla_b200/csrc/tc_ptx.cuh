@@ -108,6 +108,36 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, uint64_t
         : "memory");
 }
 
+// An L2 policy under which the lines a load brings in are the first candidates for eviction:
+// for tiles read once, so that they do not push out lines that a later read still wants.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// Drops one 128-byte line of global memory from L2 without writing it back; the line's contents
+// become unspecified.  For scratch that nothing reads again.  a must be 128-byte aligned.
+__device__ __forceinline__ void l2_discard_line(const void *a) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(a)) : "memory");
+}
+// The 2D/3D loads above with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *map, uint64_t *bar, int c0,
+                                                 int c1, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_hint(void *dst, const void *map, uint64_t *bar, int c0,
+                                                 int c1, int c2, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
+        : "memory");
+}
+
 // TMA stores from shared memory (bulk groups of the issuing thread)
 __device__ __forceinline__ void tma_store_2d(const void *map, const void *src, int c0, int c1) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
