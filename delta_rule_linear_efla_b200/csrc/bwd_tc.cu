@@ -931,45 +931,55 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qw = warp & 3, hh = warp >> 2;  // TMEM lane quarter, token-column half
     const size_t DD = (size_t)DK * DV;
-    auto next_chunk = [&](int ch) {  // this CTA's next chunk whose head takes this path
-        for (ch += gridDim.x; ch < NCH; ch += gridDim.x)
-            if (head_ok(hs, ch / NC)) break;
-        return ch;
+    // The walk takes the chunks in the order chunk 0 of every head, then chunk 1, ...: the reverse
+    // chain has just written the low chunks' dU' and dS' last, so the first chunks walked find
+    // them (and the chain's q, k, dO and Ta tiles) still in L2.  Walk index w is chunk n = w / BH
+    // of head w % BH; NCH (as returned) means past the end.
+    const int BH = NCH / NC;
+    auto chunk_at = [&](int w) { return w < NCH ? (w % BH) * NC + w / BH : NCH; };
+    auto next_walk = [&](int w) {  // this CTA's next walk index whose head takes this path
+        for (w += gridDim.x; w < NCH; w += gridDim.x)
+            if (head_ok(hs, w % BH)) break;
+        return w;
     };
-    int ch = blockIdx.x;
-    if (ch < NCH && !head_ok(hs, ch / NC)) ch = next_chunk(ch);
-    if (ch >= NCH) return;  // uniform over the CTA
+    int wk = blockIdx.x;
+    if (wk < NCH && !head_ok(hs, wk % BH)) wk = next_walk(wk);
+    if (wk >= NCH) return;  // uniform over the CTA
+    int ch = chunk_at(wk);
 
     // thread 0's bookkeeping of the copies in flight: group g is pending with parity pph[g]
     bool pend[4] = {false, false, false, false};
     uint32_t pph[4] = {0u, 0u, 0u, 0u};
     // group 0: Ta, dU' and K (into buffer kbuf); group 1: dO, dS', V; group 2: S (past a head's
     // first chunk), U'; group 3: Q
+    // every tile is read once here (the last reader of each), so it comes in under evict-first:
+    // the lines the reverse chain left in L2 outlive this kernel's own reads
+    const uint64_t pol = tc::l2_evict_first_policy();
     auto issue = [&](int g, int c, uint32_t parity, int kbuf) {
         const int bh = c / NC, n = c - bh * NC, t0 = n * C;
         if (g == 0) {
             tc::mbar_expect_tx(&full[0], C * C * 2 + 2 * 128 * DV);
             for (int j = 0; j < 2; ++j) {
-                tc::tma_load_3d(base + Lay::DU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh);
-                tc::tma_load_3d(base + Lay::K0 + kbuf * 16384 + j * 8192, &tmap_k, &full[0], j * 64, t0, bh);
+                tc::tma_load_3d_hint(base + Lay::DU + j * 8192, &tmap_du, &full[0], j * 64, t0, bh, pol);
+                tc::tma_load_3d_hint(base + Lay::K0 + kbuf * 16384 + j * 8192, &tmap_k, &full[0], j * 64, t0, bh, pol);
             }
-            tc::tma_load_2d(base + Lay::T, &tmap_t, &full[0], 0, c * C);
+            tc::tma_load_2d_hint(base + Lay::T, &tmap_t, &full[0], 0, c * C, pol);
         } else if (g == 1) {
             tc::mbar_expect_tx(&full[1], 2 * 128 * DV + 2 * DK * DV);
             for (int j = 0; j < 2; ++j) {
-                tc::tma_load_3d(base + Lay::O + j * 8192, &tmap_o, &full[1], j * 64, t0, bh);
-                tc::tma_load_3d(base + Lay::V + j * 8192, &tmap_v, &full[1], j * 64, t0, bh);
-                tc::tma_load_2d(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[1], j * 64, c * DK);
+                tc::tma_load_3d_hint(base + Lay::O + j * 8192, &tmap_o, &full[1], j * 64, t0, bh, pol);
+                tc::tma_load_3d_hint(base + Lay::V + j * 8192, &tmap_v, &full[1], j * 64, t0, bh, pol);
+                tc::tma_load_2d_hint(base + Lay::DS + j * 128 * DK, &tmap_ds, &full[1], j * 64, c * DK, pol);
             }
         } else if (g == 2) {
             tc::mbar_expect_tx(&full[2], (n > 0 ? 2 * DK * DV : 0) + 128 * DV);
             for (int j = 0; j < 2; ++j) {
-                if (n > 0) tc::tma_load_2d(base + Lay::S + j * 128 * DK, &tmap_s, &full[2], j * 64, (c - 1) * DK);
-                tc::tma_load_3d(base + Lay::U + j * 8192, &tmap_u, &full[2], j * 64, t0, bh);
+                if (n > 0) tc::tma_load_2d_hint(base + Lay::S + j * 128 * DK, &tmap_s, &full[2], j * 64, (c - 1) * DK, pol);
+                tc::tma_load_3d_hint(base + Lay::U + j * 8192, &tmap_u, &full[2], j * 64, t0, bh, pol);
             }
         } else {
             tc::mbar_expect_tx(&full[3], 128 * DK);
-            for (int j = 0; j < 2; ++j) tc::tma_load_3d(base + Lay::Q + j * 8192, &tmap_q, &full[3], j * 64, t0, bh);
+            for (int j = 0; j < 2; ++j) tc::tma_load_3d_hint(base + Lay::Q + j * 8192, &tmap_q, &full[3], j * 64, t0, bh, pol);
         }
         pend[g] = true;
         pph[g] = parity;
@@ -1054,7 +1064,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         const int bh = ch / NC, n = ch - bh * NC;
         const int t0 = n * C, valid = min(C, L - t0);
         const size_t tokq = (size_t)bh * L + t0;
-        const int nx = next_chunk(ch);
+        const int nwk = next_walk(wk), nx = chunk_at(nwk);
         const int KB = Lay::K0 + kb * 16384;
         if (n == 0) {  // the initial state (fp32 [dk][dv]), or zero; S's buffer is free since mbar[2]
             for (int e = tid; e < DK * DV; e += THREADS) {
@@ -1223,6 +1233,7 @@ __global__ void __launch_bounds__(cw::THREADS, 1)
         if (tid == 0 && nx < NCH) issue(3, nx, ph ^ 1u, 0);
         if (nx >= NCH) break;
         ch = nx;
+        wk = nwk;
         ph ^= 1u;
         kb ^= 1;
     }
