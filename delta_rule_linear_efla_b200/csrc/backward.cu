@@ -238,8 +238,11 @@ __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q,
 
 // The same for bf16 rows of 64 or 128 elements, 16-byte aligned: eight lanes per token (16-byte
 // loads, a row's dot products summed over the eight), four tokens per warp at a time, and the
-// coefficients of a token computed by the first lane of its eight.
-template <int DKV>
+// coefficients of a token computed by the first lane of its eight.  Without PAIRS it writes only
+// the first record (lambda, a and the two derivatives) and reads no q: the second record
+// (q_t . k_t, k_{t-1} . k_t) is for the heads that walk on CUDA cores, which bwd_pairs_vec_kernel
+// fills once the gate has been decided.
+template <int DKV, bool PAIRS = true>
 __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 *__restrict__ q,
                                                            const __nv_bfloat16 *__restrict__ k,
                                                            const __nv_bfloat16 *__restrict__ beta, size_t ntok,
@@ -273,21 +276,27 @@ __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 
             for (int w = 0; w < NV; ++w) {
                 const size_t o = tok * DKV + (size_t)sl * EPL + 8 * w;
                 kx[w] = *reinterpret_cast<const uint4 *>(k + o);
-                qx[w] = *reinterpret_cast<const uint4 *>(q + o);
-                kp[w] = (in && t > 0) ? *reinterpret_cast<const uint4 *>(k + o - DKV) : make_uint4(0u, 0u, 0u, 0u);
+                if constexpr (PAIRS) {
+                    qx[w] = *reinterpret_cast<const uint4 *>(q + o);
+                    kp[w] = (in && t > 0) ? *reinterpret_cast<const uint4 *>(k + o - DKV) : make_uint4(0u, 0u, 0u, 0u);
+                }
             }
             float lam = 0.f, qk = 0.f, kk = 0.f;
 #pragma unroll
             for (int w = 0; w < NV; ++w) {
                 lam += dot(kx[w], kx[w]);
-                qk += dot(qx[w], kx[w]);
-                kk += dot(kp[w], kx[w]);
+                if constexpr (PAIRS) {
+                    qk += dot(qx[w], kx[w]);
+                    kk += dot(kp[w], kx[w]);
+                }
             }
 #pragma unroll
             for (int o = 4; o > 0; o >>= 1) {
                 lam += __shfl_xor_sync(0xffffffffu, lam, o);
-                qk += __shfl_xor_sync(0xffffffffu, qk, o);
-                kk += __shfl_xor_sync(0xffffffffu, kk, o);
+                if constexpr (PAIRS) {
+                    qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                    kk += __shfl_xor_sync(0xffffffffu, kk, o);
+                }
             }
             if (in && sl == 0) {
                 const float bt = __bfloat162float(beta[tok]);
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 
                 float dfdb, dfdl;
                 coeff_grads(lam, bt, euler, a, dfdb, dfdl);
                 coef[2 * tok] = make_float4(lam, a, dfdb, dfdl);
-                coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
+                if constexpr (PAIRS) coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
                 // see bwd_coeff_kernel: any a that is not positive fails the gate
                 if (!(a > 0.f)) bad = 1;
                 m_lam = max(m_lam, __float_as_int(lam));
@@ -316,6 +325,61 @@ __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 
             atomicMax(h + 1, m_lam);
             atomicMax(h + 2, m_ia);
             atomicMax(h + 3, m_a);
+        }
+    }
+}
+
+// The second coefficient record (q_t . k_t, k_{t-1} . k_t) of the heads that the gate sends to the
+// CUDA-core walk, after bwd_coeff_vec_kernel<DKV, false> has decided it; the same lanes and dot
+// products as that kernel's PAIRS form.  Warps whose unit belongs to a tensor-core head skip it.
+template <int DKV>
+__global__ void __launch_bounds__(256) bwd_pairs_vec_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                           const __nv_bfloat16 *__restrict__ k, size_t ntok,
+                                                           int L, float4 *__restrict__ coef,
+                                                           const int *__restrict__ hs) {
+    constexpr int UNIT = 64, EPL = DKV / 8, NV = EPL / 8;
+    const int lane = threadIdx.x & 31, g = lane >> 3, sl = lane & 7;
+    const long long BH = (long long)(ntok / (size_t)L), upH = (L + UNIT - 1) / UNIT;
+    const long long nw = (long long)gridDim.x * 8, w0 = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    auto dot = [](const uint4 &a, const uint4 &b) {
+        const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 u = __bfloat1622float2(x[e]), v = __bfloat1622float2(y[e]);
+            s = fmaf(u.x, v.x, fmaf(u.y, v.y, s));
+        }
+        return s;
+    };
+    for (long long u = w0; u < BH * upH; u += nw) {
+        const long long head = u / upH;
+        if (head_takes_saved(hs, head)) continue;  // uniform over the warp
+        const int r0 = (int)(u % upH) * UNIT, r1 = min(L, r0 + UNIT);
+        const size_t hb = (size_t)head * L;
+        for (int t = r0 + g; t - g < r1; t += 4) {
+            const bool in = t < r1;
+            const size_t tok = hb + (in ? t : r0);
+            uint4 kx[NV], qx[NV], kp[NV];
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                const size_t o = tok * DKV + (size_t)sl * EPL + 8 * w;
+                kx[w] = *reinterpret_cast<const uint4 *>(k + o);
+                qx[w] = *reinterpret_cast<const uint4 *>(q + o);
+                kp[w] = (in && t > 0) ? *reinterpret_cast<const uint4 *>(k + o - DKV) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float qk = 0.f, kk = 0.f;
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                qk += dot(qx[w], kx[w]);
+                kk += dot(kp[w], kx[w]);
+            }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            }
+            if (in && sl == 0) coef[2 * tok + 1] = make_float4(qk, kk, 0.f, 0.f);
         }
     }
 }
@@ -688,7 +752,20 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
         const int gc = (int)std::max<long long>(1, std::min<long long>((units + 7) / 8, (long long)nsm * 64));
         const bool vec_rows = is_bf16 && (dk == 64 || dk == 128) && ((uintptr_t)q & 15) == 0 &&
                               ((uintptr_t)k & 15) == 0;
-        if (vec_rows && dk == 128)
+        const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
+        if (vec_rows && tc_bwd) {
+            // the first records and the gate; then the second records of the heads the gate
+            // sends to the CUDA-core walk only (the tensor-core heads never read them)
+            const __nv_bfloat16 *bb = (const __nv_bfloat16 *)beta;
+            if (dk == 128) {
+                bwd_coeff_vec_kernel<128, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs);
+                bwd_pairs_vec_kernel<128><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
+            } else {
+                bwd_coeff_vec_kernel<64, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs);
+                bwd_pairs_vec_kernel<64><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
+            }
+            count_launches(1);
+        } else if (vec_rows && dk == 128)
             bwd_coeff_vec_kernel<128><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
                                                          (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs);
         else if (vec_rows)
