@@ -303,3 +303,28 @@ def test_bf16_inputs_near_the_fp16_range(oracle_mod):
     o, S = _run_gpu(x)
     o_ref, S_ref = _oracle(oracle_mod, x)
     _check(x, o, S, o_ref, S_ref)
+
+
+def test_workspace_alignment_does_not_change_results(oracle_mod):
+    """The tensor-core forward drops its Ta tiles from L2 unwritten once the state kernel has read
+    them, but only when the workspace is 128-byte aligned. A workspace that is only 16-byte
+    aligned keeps them. Both give the same outputs bit for bit. A call that follows a dropping
+    call on the same workspace is not affected by the dropped lines, and the result meets the
+    oracle's bf16 bound."""
+    x = inputs.make_inputs(inputs.workload(4, B=1, H=3, L=300))
+    d = _to_dev(x)
+    args = (d["q"], d["k"], d["v"], d["beta"], d["S0"])
+    B, H, L, dk = x["q"].shape
+    need = efla.workspace_size(B, H, L, dk, x["v"].shape[-1], 64, torch.bfloat16, torch.bfloat16)
+    buf = torch.empty(need + 256, dtype=torch.uint8, device="cuda")
+    assert buf.data_ptr() % 128 == 0 and (buf.data_ptr() + 16) % 128 != 0
+    runs = [efla.chunk_fwd(*args, chunk=64, o_dtype=torch.bfloat16, workspace=w)
+            for w in (buf[:need], buf[16:16 + need], buf[:need], buf[:need])]
+    torch.cuda.synchronize()
+    assert efla.last_device_error() == 0
+    for o, S in runs[1:]:
+        assert torch.equal(o, runs[0][0]) and torch.equal(S, runs[0][1])
+    o_ref, S_ref = _oracle(oracle_mod, x)
+    rms = float(np.sqrt(np.mean(o_ref ** 2)))
+    assert rel_err(runs[1][0].float().cpu().numpy(), o_ref) <= 2e-2 + 2.0 ** -8 * float(np.abs(o_ref).max()) / rms
+    assert rel_err(runs[1][1].cpu().numpy(), S_ref) <= 2e-2
