@@ -238,16 +238,19 @@ __global__ void __launch_bounds__(256) bwd_coeff_kernel(const T *__restrict__ q,
 
 // The same for bf16 rows of 64 or 128 elements, 16-byte aligned: eight lanes per token (16-byte
 // loads, a row's dot products summed over the eight), four tokens per warp at a time, and the
-// coefficients of a token computed by the first lane of its eight.  Without PAIRS it writes only
-// the first record (lambda, a and the two derivatives) and reads no q: the second record
-// (q_t . k_t, k_{t-1} . k_t) is for the heads that walk on CUDA cores, which bwd_pairs_vec_kernel
-// fills once the gate has been decided.
+// coefficients of a token computed by the first lane of its eight.  Without PAIRS (the form that
+// runs before the tensor-core backward) it writes only the first record (lambda, a and the two
+// derivatives) and reads no q: the second record (q_t . k_t, k_{t-1} . k_t) is for the heads that
+// walk on CUDA cores, which bwd_pairs_vec_kernel fills once the gate has been decided.  That form
+// also rounds its unit's rows of dO (fp32, dv per token) to the fp16 copy dO16 that the
+// tensor-core products read.
 template <int DKV, bool PAIRS = true>
 __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 *__restrict__ q,
                                                            const __nv_bfloat16 *__restrict__ k,
                                                            const __nv_bfloat16 *__restrict__ beta, size_t ntok,
                                                            int L, bool euler, float4 *__restrict__ coef,
-                                                           int *__restrict__ hs) {
+                                                           int *__restrict__ hs, const float *__restrict__ dO,
+                                                           __half *__restrict__ dO16, int dv) {
     constexpr int UNIT = 64, EPL = DKV / 8, NV = EPL / 8;  // elements and 16-byte words per lane
     const int lane = threadIdx.x & 31, g = lane >> 3, sl = lane & 7;
     const long long BH = (long long)(ntok / (size_t)L), upH = (L + UNIT - 1) / UNIT;
@@ -310,6 +313,17 @@ __global__ void __launch_bounds__(256) bwd_coeff_vec_kernel(const __nv_bfloat16 
                 m_lam = max(m_lam, __float_as_int(lam));
                 m_ia = max(m_ia, 0x7fffffff - __float_as_int(a));
                 m_a = max(m_a, __float_as_int(a));
+            }
+        }
+        if constexpr (!PAIRS) {  // the unit's rows of dO, 16 bytes in and 8 out per lane at a time
+            const size_t e0 = (hb + r0) * (size_t)dv / 4, n4 = (size_t)(r1 - r0) * dv / 4;
+            const float4 *src = reinterpret_cast<const float4 *>(dO) + e0;
+            uint2 *dst = reinterpret_cast<uint2 *>(dO16) + e0;
+#pragma unroll 4
+            for (size_t e = lane; e < n4; e += 32) {
+                const float4 x = src[e];
+                const __half2 lo = __floats2half2_rn(x.x, x.y), hi = __floats2half2_rn(x.z, x.w);
+                dst[e] = make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
             }
         }
         bad = __any_sync(0xffffffffu, bad);
@@ -744,6 +758,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
             if (e != cudaSuccess) return e;
         }
     }
+    bool dO16_done = false;  // the coefficient pass has written dO's fp16 copy
     if (ntok > 0) {
         e = cudaMemsetAsync(hs, 0, 4 * (size_t)BH * sizeof(int), s);
         if (e != cudaSuccess) return e;
@@ -757,20 +772,27 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
             // the first records and the gate; then the second records of the heads the gate
             // sends to the CUDA-core walk only (the tensor-core heads never read them)
             const __nv_bfloat16 *bb = (const __nv_bfloat16 *)beta;
+            // and dO's fp16 copy for the tensor-core products, at the head of their workspace
+            __half *dO16 = (__half *)(wsf + lay.tcb);
             if (dk == 128) {
-                bwd_coeff_vec_kernel<128, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs);
+                bwd_coeff_vec_kernel<128, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs, dO,
+                                                                    dO16, dv);
                 bwd_pairs_vec_kernel<128><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
             } else {
-                bwd_coeff_vec_kernel<64, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs);
+                bwd_coeff_vec_kernel<64, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs, dO,
+                                                                   dO16, dv);
                 bwd_pairs_vec_kernel<64><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
             }
+            dO16_done = true;
             count_launches(1);
         } else if (vec_rows && dk == 128)
             bwd_coeff_vec_kernel<128><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
-                                                         (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs);
+                                                         (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs,
+                                                         nullptr, nullptr, 0);
         else if (vec_rows)
             bwd_coeff_vec_kernel<64><<<gc, 256, 0, s>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
-                                                        (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs);
+                                                        (const __nv_bfloat16 *)beta, ntok, L, euler, coef, hs,
+                                                        nullptr, nullptr, 0);
         else if (is_bf16)
             bwd_coeff_kernel<__nv_bfloat16><<<gc, 256, 0, s>>>(
                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)beta, ntok, L,
@@ -783,7 +805,7 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     }
     if (tc_bwd && L > 0) {
         e = launch_bwd_tc(q, k, v, S0, dO, dSL, coef, hs, u_saved, ck_saved, ta_ws, dq, dkey, dval, dbeta,
-                          dS0, B, H, L, dk, dv, wsf + lay.tcb, s);
+                          dS0, B, H, L, dk, dv, wsf + lay.tcb, s, dO16_done);
         if (e != cudaSuccess) return e;
     }
     const int grid = (int)(BH * NS);

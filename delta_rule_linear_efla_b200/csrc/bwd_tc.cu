@@ -1268,7 +1268,8 @@ template <int DK, int DV>
 cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const float *S0, const float *dO,
                             const float *dSL, const float4 *coef, const int *hs, const __half *u_saved,
                             const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
-                            float *dbeta, float *dS0, int B, int H, int L, void *ws, cudaStream_t s) {
+                            float *dbeta, float *dS0, int B, int H, int L, void *ws, cudaStream_t s,
+                            bool dO16_ready) {
     const int BH = B * H, NC = (L + C - 1) / C;
     const size_t ntok = (size_t)BH * L;
     __half *dO16 = (__half *)ws;
@@ -1310,7 +1311,7 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         !tmap::make_2d(&mds, dSp, DV, rows, 64, DK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !tmap::make_3d(&mv, v, DV, L, BH, 64, C))
         return cudaErrorInvalidValue;
-    bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
+    if (!dO16_ready) bwd_prepare_kernel<<<g, 256, 0, s>>>(dO, dO16, n4);
     bwd_state_kernel<DK, DV><<<BH, REV_THREADS, RevLayout<DK, DV>::SMEM, s>>>(mq, mk, mo, mt, mdu, mds, dSL, dSp,
                                                                               dS0, hs, L, NC);
     const int nch = BH * NC;  // as many CTAs as fit on the SMs at once, each walking every grid-th chunk
@@ -1339,7 +1340,7 @@ cudaError_t launch_bwd_tc_t(const void *q, const void *k, const void *v, const f
         bwd_chunk_kernel<DK, DV><<<std::min(nch, nsm * per_sm), cw::THREADS, ChunkLayout<DK, DV>::SMEM, s>>>(
             mq, mk, mo, mu, mdu, ms, mds, mt, mv, coef, S0, hs, dq, dkey, dval, dbeta, L, NC, nch);
     }
-    count_launches(3);
+    count_launches(dO16_ready ? 2 : 3);
     return cudaGetLastError();
 }
 
@@ -1355,19 +1356,19 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
                           const float *dSL, const void *coef, const int *hs, const __half *u_saved,
                           const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
                           float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool dO16_ready) {
     const float4 *cf = (const float4 *)coef;
     if (dk == 128 && dv == 128)
         return launch_bwd_tc_t<128, 128>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
-                                         dS0, B, H, L, ws, s);
+                                         dS0, B, H, L, ws, s, dO16_ready);
     if (dk == 128 && dv == 64)
         return launch_bwd_tc_t<128, 64>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
-                                        dS0, B, H, L, ws, s);
+                                        dS0, B, H, L, ws, s, dO16_ready);
     if (dk == 64 && dv == 128)
         return launch_bwd_tc_t<64, 128>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
-                                        dS0, B, H, L, ws, s);
+                                        dS0, B, H, L, ws, s, dO16_ready);
     return launch_bwd_tc_t<64, 64>(q, k, v, S0, dO, dSL, cf, hs, u_saved, ck_saved, ta, dq, dkey, dval, dbeta,
-                                   dS0, B, H, L, ws, s);
+                                   dS0, B, H, L, ws, s, dO16_ready);
 }
 
 cudaError_t bwd_tc_read_and_clear_error(unsigned int *out) {

@@ -89,13 +89,14 @@ cudaError_t launch_chunk_tc_keep(const void *q, const void *k, const void *v, co
 // over the chunks (dU' of every token and the state gradient after every chunk), then every
 // chunk's dq, dk, dv and dbeta in parallel; dS0 from the chain.  coef: the coefficient
 // kernel's per-token float4 pairs; hs: its per-head gate statistics; u_saved, ck_saved, ta: the
-// saving forward's outputs and Ta tiles.  Workspace: bwd_tc_workspace_bytes.
+// saving forward's outputs and Ta tiles.  Workspace: bwd_tc_workspace_bytes; dO16_ready: its
+// head already holds dO rounded to fp16 ([BH][L][dv]), so the conversion kernel is skipped.
 size_t bwd_tc_workspace_bytes(int B, int H, int L, int dk, int dv);
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *S0, const float *dO,
                           const float *dSL, const void *coef, const int *hs, const __half *u_saved,
                           const __half *ck_saved, const void *ta, float *dq, float *dkey, float *dval,
                           float *dbeta, float *dS0, int B, int H, int L, int dk, int dv, void *ws,
-                          cudaStream_t s);
+                          cudaStream_t s, bool dO16_ready);
 cudaError_t bwd_tc_read_and_clear_error(unsigned int *out);
 // A kernel whose one bounded wait runs out (nothing arrives): records a timeout, then returns.
 cudaError_t launch_selftest_wait(long long budget_cycles, cudaStream_t s);
