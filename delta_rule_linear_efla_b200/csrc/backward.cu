@@ -774,14 +774,15 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
             const __nv_bfloat16 *bb = (const __nv_bfloat16 *)beta;
             // and dO's fp16 copy for the tensor-core products, at the head of their workspace
             __half *dO16 = (__half *)(wsf + lay.tcb);
+            const int gp = std::min(gc, nsm);  // its warps mostly only check the gate
             if (dk == 128) {
                 bwd_coeff_vec_kernel<128, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs, dO,
                                                                     dO16, dv);
-                bwd_pairs_vec_kernel<128><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
+                bwd_pairs_vec_kernel<128><<<gp, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
             } else {
                 bwd_coeff_vec_kernel<64, false><<<gc, 256, 0, s>>>(qb, kb, bb, ntok, L, euler, coef, hs, dO,
                                                                    dO16, dv);
-                bwd_pairs_vec_kernel<64><<<gc, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
+                bwd_pairs_vec_kernel<64><<<gp, 256, 0, s>>>(qb, kb, ntok, L, coef, hs);
             }
             dO16_done = true;
             count_launches(1);
@@ -836,8 +837,10 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *
     segs.seg[0] = seg(part, dq, nq, (size_t)L * dk);
     segs.seg[1] = seg(part + (size_t)NS * nq, dkey, nq, (size_t)L * dk);
     segs.seg[2] = seg(part + 2 * (size_t)NS * nq, dbeta, nb, (size_t)L);
-    const int SL = (int)std::max<long long>(1, std::min<long long>(((long long)nsm * 8 + BH - 1) / BH,
-                                                                      ((long long)L * dk / 4 + 255) / 256));
+    // slices per head: enough blocks to fill the GPU when every head walks; with the tensor-core
+    // heads returning at once, about one block per SM (most blocks would only check the gate)
+    const long long fill = tc_bwd ? std::max<long long>(1, nsm / BH) : ((long long)nsm * 8 + BH - 1) / BH;
+    const int SL = (int)std::max<long long>(1, std::min<long long>(fill, ((long long)L * dk / 4 + 255) / 256));
     if (BH * SL > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     bwd_sum_kernel<<<dim3((unsigned)(BH * SL), 3), 256, 0, s>>>(segs, NS, SL, tc_bwd ? hs : nullptr);
     count_launches(1);
