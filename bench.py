@@ -134,12 +134,14 @@ def run_bwd(args) -> None:
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": _config(w),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm"], "traffic": None,
+                     "frac": achieved / peaks["hbm"],
+                     "traffic": profiled_bwd_traffic(w) if RULE == "exact" else None,
                      "kernel": "efla_bwd (bf16 heads the saved-forward gate admits: the saving tensor-core "
                                "forward, the reverse chain over chunks on tcgen05, per-chunk gradients on "
                                "tcgen05 at d = 128 and mma.sync at d = 64; other heads: the fp32 "
                                "column-block walk on CUDA cores)",
-                     "alg_bytes_per_launch": alg, "avg_launch_ms": ms},
+                     "alg_bytes_per_launch": alg, "avg_launch_ms": ms,
+                     "source_hash": kernel_source_hash(BWD_SOURCES)},
         "train_step": train, "gpu_launches": int(launches), "clocks": clocks}))
 
 
@@ -207,18 +209,44 @@ class ClockSampler:
 
 
 FWD_SOURCES = ("chunk_tc.cu", "common.cuh", "tc_ptx.cuh", "tmap.h")
+# the backward's kernels: its own sources and the saving forward's
+BWD_SOURCES = FWD_SOURCES + ("backward.cu", "bwd_tc.cu", "bwd_gate.cuh")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources the chunk forward's kernels are built from (the tcgen05 pair and
-    segment kernels and the helpers they include): ties profiled counters to them."""
+def kernel_source_hash(files=FWD_SOURCES) -> str:
+    """Hash of the CUDA sources a pass's kernels are built from (for the chunk forward: the
+    tcgen05 pair and segment kernels and the helpers they include): ties profiled counters to
+    them."""
     import hashlib
 
     h = hashlib.sha256()
-    for f in FWD_SOURCES:
+    for f in files:
         h.update(f.encode())
         h.update(open(os.path.join(ROOT, "delta_rule_linear_efla_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
+
+
+def _profile_keys(name: str) -> dict:
+    p = os.path.join(ROOT, "profiles", name)
+    kv = {}
+    if os.path.exists(p):
+        for line in open(p):
+            line = line.split("#")[0].strip()
+            if "=" in line:
+                k, v = (x.strip() for x in line.split("=", 1))
+                kv[k] = v
+    return kv
+
+
+def profiled_bwd_traffic(w) -> int | None:
+    """DRAM bytes of one efla_bwd call from the committed ncu capture, if it was taken on this
+    workload and on the current backward sources; None otherwise."""
+    if w.id != 4:
+        return None
+    kv = _profile_keys("dram_traffic_bwd_lm1p3b.txt")
+    if kv.get("source_hash") != kernel_source_hash(BWD_SOURCES) or "bwd_bytes" not in kv:
+        return None
+    return int(kv["bwd_bytes"])
 
 
 def profiled_traffic(w, o_dtype) -> int | None:
